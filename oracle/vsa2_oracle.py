@@ -1,0 +1,202 @@
+"""Plain fp64 CPU oracle for the VSA2 hot path. TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, the smoke check of the package entry module and the benchmark's CPU
+baseline leg may import this module. The product path (the CUDA library and its Python
+binding) never calls it and shares no code with it.
+
+Source: "Improving Video Sparse Attention with Fine-grained Router and Sparse Rebasing"
+(arXiv 2609.32882), §2.1 Background and §2.2 VSA2, Eq. 5-9 and Eq. 12.
+
+Layout: every per-(b, h) tensor is (L, D) in cube-major token order (§2.2 "Permutation"):
+tile i is rows [i*Bt, (i+1)*Bt); inside it, router sub-cube a is rows [a*R, (a+1)*R), so tile i
+owns sub-cubes G*i .. G*i+G-1 with G = Bt / R.
+
+Readings of the pages that this oracle commits to (each is listed in the design notes):
+  * Eq. 7 "MeanPool_{GxG}" is emitted scaled by G (mean over the G query sub-cubes, sum over the
+    G key sub-cubes), so each score row sums to 1. G is a power of two, so the scaling is exact
+    and leaves the TopK result unchanged.
+  * Eq. 8-9 TopK: scores are ranked in fp32 (the kernel's precision), descending; equal scores
+    go to the lower flat index i*N + j. The budget N*K is per (batch, head).
+  * Eq. 12 for a query tile with no selected KV tile: output 0, LSE = -inf, zero gradients.
+  * Softmax scale 1/sqrt(D) (§2.1).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "mean_pool",
+    "router_scores",
+    "router_scores_dense_attention",
+    "topk_select",
+    "sparse_attn_fwd",
+    "sparse_attn_bwd",
+]
+
+
+def mean_pool(x: np.ndarray, group: int) -> np.ndarray:
+    """MeanPool over consecutive groups of `group` tokens of a cube-major (L, D) tensor (Eq. 5)."""
+    x = np.asarray(x, dtype=np.float64)
+    L, D = x.shape
+    return x.reshape(L // group, group, D).mean(axis=1)
+
+
+def router_scores(q: np.ndarray, k: np.ndarray, tile_tokens: int = 64, pool_tokens: int = 16,
+                  row_chunk: int = 2048) -> np.ndarray:
+    """Tile-level router scores Pr (N, N) for one (b, h), Eq. 5-7.
+
+    Qr, Kr = MeanPool_R(Q, K)                        (Eq. 5)
+    P_hat  = row-softmax(Qr Kr^T / sqrt(D))          (Eq. 6), over all L/R pooled keys
+    Pr[i,j] = (1/G) sum_{a in i} sum_{b in j} P_hat[a,b]   (Eq. 7, scaled by G; rows sum to 1)
+
+    P_hat is formed exactly (max-subtracted fp64), a block of pooled query rows at a time; each
+    block holds complete rows, so the softmax is the textbook one.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    L, D = q.shape
+    G = tile_tokens // pool_tokens
+    N = L // tile_tokens
+    qr = mean_pool(q, pool_tokens)
+    kr = mean_pool(k, pool_tokens)
+    Lr = qr.shape[0]
+    scale = 1.0 / np.sqrt(D)
+    out = np.empty((N, N), dtype=np.float64)
+    rows_per = max(G, (row_chunk // G) * G)
+    for a0 in range(0, Lr, rows_per):
+        a1 = min(Lr, a0 + rows_per)
+        s = (qr[a0:a1] @ kr.T) * scale
+        s -= s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        p /= p.sum(axis=1, keepdims=True)
+        # pool: G query sub-rows of each tile (mean) x G key sub-cubes of each tile (sum)
+        blk = p.reshape((a1 - a0) // G, G, N, G).sum(axis=(1, 3)) / G
+        out[a0 // G:a1 // G] = blk
+    return out
+
+
+def router_scores_dense_attention(q: np.ndarray, k: np.ndarray, tile_tokens: int = 64) -> np.ndarray:
+    """The compute-unbounded router of Eq. 10-11: token-level softmax, then tile pooling
+    (scaled like `router_scores` so rows sum to 1). Diagnostic only (router recall)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    L, D = q.shape
+    N = L // tile_tokens
+    s = (q @ k.T) / np.sqrt(D)
+    s -= s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    p /= p.sum(axis=1, keepdims=True)
+    return p.reshape(N, tile_tokens, N, tile_tokens).sum(axis=(1, 3)) / tile_tokens
+
+
+def topk_select(scores: np.ndarray, topk: int) -> dict:
+    """Per-sequence TopK over the flattened N x N tile scores (Eq. 8-9).
+
+    `scores` must be float32 (the precision in which both sides rank). Entries are ordered by
+    (score descending, flat index ascending) and the first N*topk are kept. Returns the boolean
+    mask and its CSR (per query tile, ascending KV tile) and CSC (per KV tile, ascending query
+    tile) index lists as int32 arrays.
+    """
+    s = np.asarray(scores)
+    if s.dtype != np.float32:
+        raise TypeError("rank in fp32: pass float32 scores")
+    N = s.shape[0]
+    if s.shape != (N, N):
+        raise ValueError("scores must be square")
+    if not (1 <= topk <= N):
+        raise ValueError("need 1 <= topk <= N")
+    flat = s.reshape(-1)
+    budget = N * topk
+    order = np.lexsort((np.arange(N * N), -flat.astype(np.float64)))
+    mask = np.zeros(N * N, dtype=bool)
+    mask[order[:budget]] = True
+    mask = mask.reshape(N, N)
+    counts = mask.sum(axis=1)
+    kv_off = np.zeros(N + 1, dtype=np.int32)
+    kv_off[1:] = np.cumsum(counts)
+    kv_idx = np.nonzero(mask)[1].astype(np.int32)  # row-major scan: ascending j within row i
+    ccounts = mask.sum(axis=0)
+    q_off = np.zeros(N + 1, dtype=np.int32)
+    q_off[1:] = np.cumsum(ccounts)
+    q_idx = np.nonzero(mask.T)[1].astype(np.int32)
+    return {"mask": mask, "kv_off": kv_off, "kv_idx": kv_idx, "q_off": q_off, "q_idx": q_idx}
+
+
+def _tiles(x: np.ndarray, tile_tokens: int) -> np.ndarray:
+    L, D = x.shape
+    return x.reshape(L // tile_tokens, tile_tokens, D)
+
+
+def sparse_attn_fwd(q, k, v, kv_off, kv_idx, tile_tokens: int = 64, query_tiles=None):
+    """Block-sparse attention forward for one (b, h), Eq. 12 with the §2.1 definition:
+    for each query token t of tile i, o_t = sum_u softmax_u(q_t . k_u / sqrt(D)) v_u over the
+    tokens u of the KV tiles selected for tile i; lse_t = log sum_u exp(q_t . k_u / sqrt(D)).
+
+    Returns (o (L, D) fp64, lse (L,) fp64). With `query_tiles` given, only those tiles are
+    computed (rows of other tiles are left as NaN) - used to time a bounded sample.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    L, D = q.shape
+    N = L // tile_tokens
+    scale = 1.0 / np.sqrt(D)
+    qt, kt, vt = _tiles(q, tile_tokens), _tiles(k, tile_tokens), _tiles(v, tile_tokens)
+    o = np.full((N, tile_tokens, D), np.nan)
+    lse = np.full((N, tile_tokens), np.nan)
+    for i in (range(N) if query_tiles is None else query_tiles):
+        sel = np.asarray(kv_idx[kv_off[i]:kv_off[i + 1]])
+        if sel.size == 0:
+            o[i] = 0.0
+            lse[i] = -np.inf
+            continue
+        ks = kt[sel].reshape(-1, D)
+        vs = vt[sel].reshape(-1, D)
+        s = (qt[i] @ ks.T) * scale
+        m = s.max(axis=1, keepdims=True)
+        p = np.exp(s - m)
+        l = p.sum(axis=1, keepdims=True)
+        o[i] = (p @ vs) / l
+        lse[i] = (m + np.log(l))[:, 0]
+    return o.reshape(L, D), lse.reshape(L)
+
+
+def sparse_attn_bwd(q, k, v, do, kv_off, kv_idx, tile_tokens: int = 64):
+    """Gradients (dQ, dK, dV) of the Eq. 12 output for one (b, h) given upstream dO.
+
+    Textbook softmax-attention backward restricted to the selected tile pairs (the router
+    receives no gradient, §2.1): with P the softmax of S = Q K_S^T / sqrt(D) per query row,
+    dV_S = P^T dO, dP = dO V_S^T, dS = P * (dP - rowsum(dO * O)), dQ = dS K_S / sqrt(D),
+    dK_S = dS^T Q / sqrt(D). The softmax is recomputed here in fp64 from Q, K, V.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    L, D = q.shape
+    N = L // tile_tokens
+    scale = 1.0 / np.sqrt(D)
+    qt, kt, vt, dot = (_tiles(x, tile_tokens) for x in (q, k, v, do))
+    dq = np.zeros_like(qt)
+    dk = np.zeros_like(kt)
+    dv = np.zeros_like(vt)
+    for i in range(N):
+        sel = np.asarray(kv_idx[kv_off[i]:kv_off[i + 1]])
+        if sel.size == 0:
+            continue
+        ks = kt[sel].reshape(-1, D)
+        vs = vt[sel].reshape(-1, D)
+        s = (qt[i] @ ks.T) * scale
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        o = p @ vs
+        delta = np.sum(dot[i] * o, axis=1, keepdims=True)
+        dvs = p.T @ dot[i]
+        dp = dot[i] @ vs.T
+        ds = p * (dp - delta)
+        dq[i] = (ds @ ks) * scale
+        dks = (ds.T @ qt[i]) * scale
+        n = sel.size
+        np.add.at(dk, sel, dks.reshape(n, tile_tokens, D))
+        np.add.at(dv, sel, dvs.reshape(n, tile_tokens, D))
+    return dq.reshape(L, D), dk.reshape(L, D), dv.reshape(L, D)

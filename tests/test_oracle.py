@@ -1,0 +1,368 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix (CPU only).
+
+Each test checks the oracle against something other than itself: a brute-force restatement of
+the definition on the raster token grid, a closed form, a special case that reduces to a library
+routine, an invariant, or a value printed on the pages (tests/golden/).
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import synthetic as S
+from oracle import vsa2_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+TILE, POOL = (4, 4, 4), (2, 2, 4)
+
+
+def _raster_inputs(grid, d, seed, smooth=True):
+    rng = np.random.default_rng(seed)
+    if smooth:
+        return S.smoothed_field(rng, grid, d).astype(np.float64)
+    return rng.standard_normal((*grid, d))
+
+
+# --------------------------------------------------------------------------------------------
+# synthetic inputs (layout contract shared by both sides)
+# --------------------------------------------------------------------------------------------
+
+def test_cube_major_roundtrip_and_tile_membership():
+    grid = (8, 8, 12)
+    x = np.arange(np.prod(grid) * 2, dtype=np.float64).reshape(*grid, 2)
+    y = S.raster_to_cube_major(x, TILE, POOL)
+    assert np.array_equal(S.cube_major_to_raster(y, grid, TILE, POOL), x)
+    # every cube-major tile i holds exactly the tokens of one 4x4x4 cube, tiles in raster order
+    nt, nh, nw = grid[0] // 4, grid[1] // 4, grid[2] // 4
+    for i in range(nt * nh * nw):
+        a, b, c = i // (nh * nw), (i // nw) % nh, i % nw
+        cube = x[4 * a:4 * a + 4, 4 * b:4 * b + 4, 4 * c:4 * c + 4, 0].ravel()
+        assert set(y[64 * i:64 * i + 64, 0]) == set(cube)
+        # ... and each 16-row group is one 2x2x4 sub-cube
+        for g in range(4):
+            st, sh = g // 2, g % 2
+            sub = x[4 * a + 2 * st:4 * a + 2 * st + 2, 4 * b + 2 * sh:4 * b + 2 * sh + 2, 4 * c:4 * c + 4, 0]
+            assert set(y[64 * i + 16 * g:64 * i + 16 * g + 16, 0]) == set(sub.ravel())
+
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal(100000) * 10.0 ** rng.integers(-6, 6, 100000)).astype(np.float32)
+    ours = S.round_to_dtype(x, "bf16")
+    ref = torch.from_numpy(x).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(ours, ref)
+
+
+def test_field_statistics():
+    wl = S.WORKLOADS["tiny"]
+    x = S.make_slice(wl, "q", 0, 0)
+    assert x.shape == (wl.tokens, wl.head_dim)
+    assert abs(x.var() - 1.25) < 0.1
+    # smooth: neighbouring tokens along w (adjacent rows inside a sub-cube) correlate strongly
+    xr = S.cube_major_to_raster(x, wl.grid, wl.tile, wl.pool)
+    c = np.corrcoef(xr[:, :, :-1].ravel(), xr[:, :, 1:].ravel())[0, 1]
+    assert c > 0.5
+
+
+# --------------------------------------------------------------------------------------------
+# router, Eq. 5-7
+# --------------------------------------------------------------------------------------------
+
+def _router_bruteforce(xq, xk, grid):
+    """Eq. 5-7 restated on the raster grid with explicit loops: pooled means over each
+    2x2x4 sub-cube, softmax over all pooled keys, then sum over key sub-cubes and mean over
+    query sub-cubes of each 4x4x4 tile."""
+    T, H, W, D = xq.shape
+    subs = []  # (tile index, pooled q, pooled k)
+    nt, nh, nw = T // 4, H // 4, W // 4
+    for a, b, c in itertools.product(range(nt), range(nh), range(nw)):
+        tile = (a * nh + b) * nw + c
+        for st, sh in itertools.product(range(2), range(2)):
+            t0, h0, w0 = 4 * a + 2 * st, 4 * b + 2 * sh, 4 * c
+            qs = np.zeros(D)
+            ks = np.zeros(D)
+            for dt, dh, dw in itertools.product(range(2), range(2), range(4)):
+                qs += xq[t0 + dt, h0 + dh, w0 + dw]
+                ks += xk[t0 + dt, h0 + dh, w0 + dw]
+            subs.append((tile, qs / 16.0, ks / 16.0))
+    N = nt * nh * nw
+    out = np.zeros((N, N))
+    for ti, qa, _ in subs:
+        logits = [float(qa @ kb) / math.sqrt(D) for _, _, kb in subs]
+        m = max(logits)
+        ex = [math.exp(z - m) for z in logits]
+        z = sum(ex)
+        for (tj, _, _), e in zip(subs, ex):
+            out[ti, tj] += e / z / 4.0
+    return out
+
+
+@pytest.mark.parametrize("grid,d", [((4, 8, 8), 8), ((8, 8, 8), 16)])
+def test_router_matches_bruteforce_on_raster_grid(grid, d):
+    xq = _raster_inputs(grid, d, 1)
+    xk = _raster_inputs(grid, d, 2)
+    want = _router_bruteforce(xq, xk, grid)
+    got = O.router_scores(S.raster_to_cube_major(xq, TILE, POOL), S.raster_to_cube_major(xk, TILE, POOL))
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-15)
+
+
+def test_router_tile_constant_case_equals_coarse_attention():
+    """If Q and K are constant inside every 4x4x4 tile, the router scores equal the coarse
+    branch's block attention P_c = softmax(Qc Kc^T / sqrt(D)) of Eq. 1-2."""
+    N, D = 12, 32
+    rng = np.random.default_rng(5)
+    qc = rng.standard_normal((N, D)) * 2
+    kc = rng.standard_normal((N, D)) * 2
+    q = np.repeat(qc, 64, axis=0)
+    k = np.repeat(kc, 64, axis=0)
+    pc = torch.softmax(torch.from_numpy(qc) @ torch.from_numpy(kc).T / math.sqrt(D), dim=-1).numpy()
+    np.testing.assert_allclose(O.router_scores(q, k), pc, rtol=1e-12, atol=1e-15)
+
+
+def test_router_rows_sum_to_one_and_are_probabilities():
+    wl = S.WORKLOADS["tiny"]
+    q = S.make_slice(wl, "q", 0, 1)
+    k = S.make_slice(wl, "k", 0, 1)
+    p = O.router_scores(q, k, row_chunk=64)  # several row blocks
+    assert p.shape == (wl.num_tiles, wl.num_tiles)
+    assert np.all(p >= 0) and np.all(p <= 1)
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(p, O.router_scores(q, k, row_chunk=1 << 20), rtol=1e-13, atol=0)
+
+
+def test_router_with_unit_pool_is_the_dense_oracle_router():
+    """With R = 1 the pool-softmax-pool router is the token-level router of Eq. 10-11."""
+    rng = np.random.default_rng(9)
+    q = rng.standard_normal((256, 16))
+    k = rng.standard_normal((256, 16))
+    np.testing.assert_allclose(O.router_scores(q, k, 64, 1), O.router_scores_dense_attention(q, k, 64),
+                               rtol=1e-12, atol=1e-16)
+
+
+def test_router_uniform_keys_give_uniform_scores():
+    rng = np.random.default_rng(2)
+    q = rng.standard_normal((512, 16))
+    k = np.ones((512, 16))
+    np.testing.assert_allclose(O.router_scores(q, k), 1.0 / 8, rtol=1e-13)
+
+
+# --------------------------------------------------------------------------------------------
+# per-sequence TopK, Eq. 8-9
+# --------------------------------------------------------------------------------------------
+
+def _check_topk_structure(sel, scores, topk):
+    N = scores.shape[0]
+    kv_off, kv_idx, q_off, q_idx, mask = sel["kv_off"], sel["kv_idx"], sel["q_off"], sel["q_idx"], sel["mask"]
+    assert kv_off[0] == 0 and kv_off[-1] == N * topk == mask.sum()
+    assert np.all(np.diff(kv_off) >= 0)
+    assert kv_idx.min() >= 0 and kv_idx.max() < N
+    for i in range(N):
+        row = kv_idx[kv_off[i]:kv_off[i + 1]]
+        assert np.all(np.diff(row) > 0)
+        assert set(row) == set(np.nonzero(mask[i])[0])
+    for j in range(N):
+        col = q_idx[q_off[j]:q_off[j + 1]]
+        assert np.all(np.diff(col) > 0)
+        assert set(col) == set(np.nonzero(mask[:, j])[0])
+
+
+def test_topk_bruteforce_sort_with_ties():
+    rng = np.random.default_rng(11)
+    N, K = 9, 3
+    s = rng.integers(0, 6, (N, N)).astype(np.float32) / 8  # many exact ties
+    sel = O.topk_select(s, K)
+    ranked = sorted(((-float(s[i, j]), i * N + j) for i in range(N) for j in range(N)))
+    want = np.zeros(N * N, bool)
+    for _, f in ranked[:N * K]:
+        want[f] = True
+    assert np.array_equal(sel["mask"].ravel(), want)
+    _check_topk_structure(sel, s, K)
+
+
+def test_topk_invariants_on_router_scores():
+    wl = S.WORKLOADS["tiny"]
+    q, k = S.make_slice(wl, "q", 0, 0), S.make_slice(wl, "k", 0, 0)
+    s = O.router_scores(q, k).astype(np.float32)
+    sel = O.topk_select(s, wl.topk)
+    _check_topk_structure(sel, s, wl.topk)
+    m = sel["mask"]
+    assert s[m].min() >= s[~m].max()
+    thr = s[m].min()
+    tied_in = np.flatnonzero(m.ravel() & (s.ravel() == thr))
+    tied_out = np.flatnonzero(~m.ravel() & (s.ravel() == thr))
+    if tied_out.size:
+        assert tied_in.max() < tied_out.min()
+
+
+def test_topk_full_budget_selects_everything():
+    rng = np.random.default_rng(1)
+    s = rng.random((7, 7)).astype(np.float32)
+    sel = O.topk_select(s, 7)
+    assert sel["mask"].all()
+
+
+def test_topk_golden_uniform_scores():
+    """All scores equal: the tie rule keeps the N*K lowest flat indices, i.e. rows 0..K-1."""
+    path = os.path.join(GOLDEN, "topk_uniform_n8_k3.txt")
+    lines = [l for l in open(path) if not l.startswith("#") and l.strip()]
+    spec = dict(l.split("=", 1) for l in lines)
+    N, K = int(spec["N"]), int(spec["K"])
+    sel = O.topk_select(np.full((N, N), 1.0 / N, np.float32), K)
+    assert list(sel["kv_off"]) == [int(v) for v in spec["kv_off"].split()]
+    assert list(sel["kv_idx"]) == [int(v) for v in spec["kv_idx"].split()]
+    assert list(sel["q_off"]) == [int(v) for v in spec["q_off"].split()]
+    assert list(sel["q_idx"]) == [int(v) for v in spec["q_idx"].split()]
+
+
+def test_sparsity_estimate_matches_printed_values():
+    """App. B Eq. 15-16 with the budget the TopK actually spends, against the sparsities the
+    deep-read blog derives for Table 2 (B=128, R=8)."""
+    path = os.path.join(GOLDEN, "table2_sparsity.txt")
+    rows = [l.split() for l in open(path) if l.strip() and not l.startswith("#")]
+    rng = np.random.default_rng(0)
+    for L, B, R, K, printed in rows:
+        L, B, R, K, printed = int(L), int(B), int(R), int(K), float(printed)
+        N = L // B
+        sel = O.topk_select(rng.random((N, N)).astype(np.float32), K)
+        pairs = int(sel["kv_off"][-1])
+        sparsity = 1.0 - (1.0 / R ** 2 + pairs * B * B / float(N * B) ** 2)
+        assert abs(sparsity - printed) <= 0.0006, (L, K, sparsity, printed)
+
+
+# --------------------------------------------------------------------------------------------
+# block-sparse attention forward, Eq. 12
+# --------------------------------------------------------------------------------------------
+
+def _masked_attention_bruteforce(q, k, v, mask, bt=64):
+    """softmax(Q K^T / sqrt(D) + M) V with M = -inf outside the selected tile pairs (§2.1),
+    expanded to tokens; a row with no selected tile gives 0 and lse = -inf."""
+    L, D = q.shape
+    tok = np.repeat(np.repeat(mask, bt, axis=0), bt, axis=1)
+    s = q @ k.T / math.sqrt(D)
+    s = np.where(tok, s, -np.inf)
+    o = np.zeros_like(q)
+    lse = np.full(L, -np.inf)
+    for t in range(L):
+        if not tok[t].any():
+            continue
+        m = s[t][tok[t]].max()
+        e = np.where(tok[t], np.exp(s[t] - m), 0.0)
+        o[t] = e @ v / e.sum()
+        lse[t] = m + math.log(e.sum())
+    return o, lse
+
+
+def _csr(mask):
+    N = mask.shape[0]
+    off = np.zeros(N + 1, np.int32)
+    off[1:] = np.cumsum(mask.sum(1))
+    return off, np.nonzero(mask)[1].astype(np.int32)
+
+
+def test_fwd_matches_bruteforce_masked_attention():
+    rng = np.random.default_rng(4)
+    L, D = 6 * 64, 16
+    q, k, v = (rng.standard_normal((L, D)) * 1.5 for _ in range(3))
+    mask = rng.random((6, 6)) < 0.4
+    mask[2] = False  # a query tile with no KV tile
+    off, idx = _csr(mask)
+    o, lse = O.sparse_attn_fwd(q, k, v, off, idx)
+    o2, lse2 = _masked_attention_bruteforce(q, k, v, mask)
+    np.testing.assert_allclose(o, o2, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, lse2, rtol=1e-12, atol=1e-13)
+    assert np.all(o[128:192] == 0) and np.all(np.isneginf(lse[128:192]))
+
+
+def test_fwd_full_budget_equals_dense_attention():
+    rng = np.random.default_rng(6)
+    L, D = 4 * 64, 32
+    q, k, v = (rng.standard_normal((L, D)) for _ in range(3))
+    sel = O.topk_select(rng.random((4, 4)).astype(np.float32), 4)
+    o, lse = O.sparse_attn_fwd(q, k, v, sel["kv_off"], sel["kv_idx"])
+    tq, tk, tv = (torch.from_numpy(x)[None, None] for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv)[0, 0].numpy()
+    ref_lse = torch.logsumexp(torch.from_numpy(q @ k.T) / math.sqrt(D), dim=-1).numpy()
+    np.testing.assert_allclose(o, ref, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=1e-12, atol=1e-12)
+
+
+def test_fwd_constant_keys_closed_form():
+    """Equal keys give equal weights: o_t is the mean of the selected value rows and
+    lse_t = q_t.k/sqrt(D) + log(#selected tokens)."""
+    rng = np.random.default_rng(8)
+    L, D = 5 * 64, 8
+    q, v = rng.standard_normal((L, D)), rng.standard_normal((L, D))
+    kvec = rng.standard_normal(D)
+    k = np.tile(kvec, (L, 1))
+    mask = rng.random((5, 5)) < 0.5
+    mask[:, 0] = True
+    off, idx = _csr(mask)
+    o, lse = O.sparse_attn_fwd(q, k, v, off, idx)
+    vt = v.reshape(5, 64, D)
+    for i in range(5):
+        sel = np.nonzero(mask[i])[0]
+        np.testing.assert_allclose(o[64 * i:64 * i + 64], np.broadcast_to(vt[sel].reshape(-1, D).mean(0), (64, D)),
+                                   rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(lse[64 * i:64 * i + 64], q[64 * i:64 * i + 64] @ kvec / math.sqrt(D) + math.log(64 * sel.size),
+                                   rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------------------------
+# backward
+# --------------------------------------------------------------------------------------------
+
+def _loss(q, k, v, do, off, idx):
+    o, _ = O.sparse_attn_fwd(q, k, v, off, idx)
+    return float(np.sum(o * do))
+
+
+def test_bwd_central_finite_differences():
+    rng = np.random.default_rng(12)
+    L, D = 3 * 64, 8
+    q, k, v, do = (rng.standard_normal((L, D)) for _ in range(4))
+    mask = np.array([[1, 0, 1], [0, 0, 0], [1, 1, 0]], bool)
+    off, idx = _csr(mask)
+    dq, dk, dv = O.sparse_attn_bwd(q, k, v, do, off, idx)
+    eps = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        dirn = rng.standard_normal(x.shape)
+        args = {"q": q, "k": k, "v": v}
+        plus = dict(args, **{name: x + eps * dirn})
+        minus = dict(args, **{name: x - eps * dirn})
+        fd = (_loss(plus["q"], plus["k"], plus["v"], do, off, idx) - _loss(minus["q"], minus["k"], minus["v"], do, off, idx)) / (2 * eps)
+        an = float(np.sum(g * dirn))
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+    assert np.all(dq[64:128] == 0)
+
+
+def test_bwd_full_budget_equals_dense_autograd():
+    rng = np.random.default_rng(13)
+    L, D = 3 * 64, 16
+    q, k, v, do = (rng.standard_normal((L, D)) for _ in range(4))
+    off, idx = _csr(np.ones((3, 3), bool))
+    dq, dk, dv = O.sparse_attn_bwd(q, k, v, do, off, idx)
+    tq, tk, tv = (torch.from_numpy(x).requires_grad_() for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(tq[None, None], tk[None, None], tv[None, None])[0, 0]
+    o.backward(torch.from_numpy(do))
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_bwd_invariants():
+    """Each softmax row's dS sums to zero, so the key gradients sum to zero; the probabilities
+    of a non-empty row sum to one, so the value gradients sum to the sum of dO over
+    non-empty query rows."""
+    rng = np.random.default_rng(14)
+    L, D = 5 * 64, 16
+    q, k, v, do = (rng.standard_normal((L, D)) for _ in range(4))
+    mask = rng.random((5, 5)) < 0.5
+    mask[3] = False
+    off, idx = _csr(mask)
+    dq, dk, dv = O.sparse_attn_bwd(q, k, v, do, off, idx)
+    np.testing.assert_allclose(dk.sum(0), 0, atol=1e-11)
+    live = np.repeat(mask.any(1), 64)
+    np.testing.assert_allclose(dv.sum(0), do[live].sum(0), rtol=1e-12, atol=1e-11)
