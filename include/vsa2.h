@@ -1,0 +1,161 @@
+/*
+ * vsa2.h - C ABI of the VSA2 hot path on NVIDIA B200 (sm_100a): fine-grained router,
+ * per-sequence TopK and block-sparse attention forward / backward.
+ *
+ * Method: "Improving Video Sparse Attention with Fine-grained Router and Sparse Rebasing"
+ * (arXiv 2609.32882), §2.2 VSA2: Eq. 5-7 (router), Eq. 8-9 (per-sequence TopK), Eq. 12
+ * (block-sparse fine branch); §2.1 Background gives the attention definition with the -inf
+ * block mask; Fig. 5 gives the two-pass (LSE, then softmax + on-chip pooling) router.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor arguments are DEVICE pointers owned by the caller. The library never
+ *    allocates or frees device memory and never synchronises, except vsa2_get_device_error.
+ *    Every compute call only enqueues kernels on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and returns.
+ *  - Token layout: Q, K, V, O, dO, dQ, dK, dV are [batch, heads, L, head_dim] row-major
+ *    (head_dim innermost), L = grid_t*grid_h*grid_w in CUBE-MAJOR order (§2.2 "Permutation"):
+ *    tiles of tile_t x tile_h x tile_w tokens in raster order over the tile grid; inside a
+ *    tile, the router sub-cubes of pool_t x pool_h x pool_w tokens in raster order; inside a
+ *    sub-cube, tokens in raster order. So tile i is rows [i*Bt, (i+1)*Bt) and its G = Bt/R
+ *    sub-cubes are consecutive groups of R rows.
+ *  - Sizes: Bt = tile_t*tile_h*tile_w must be 64; R = pool_t*pool_h*pool_w must be 16
+ *    (G = 4); the grid must be divisible by the tile and the tile by the pool; head_dim is
+ *    64 or 128; N = L/64 tiles; 1 <= topk <= N. Other shapes return VSA2_ERR_UNSUPPORTED.
+ *  - dtype covers Q, K, V, O and dO. Router scores, LSE and gradients are fp32; index lists
+ *    are int32. Pointers must be 16-byte aligned.
+ *  - Softmax scale is 1/sqrt(head_dim) everywhere (§2.1).
+ *  - Errors: argument errors are reported synchronously by the return value and nothing is
+ *    enqueued. A failed launch returns VSA2_ERR_CUDA. Faults found on the device (a bounded
+ *    wait that expired, an index out of range when VSA2_FLAG_VALIDATE is set) are written to
+ *    an error word at the start of the workspace and read back by vsa2_get_device_error.
+ *  - Workspace: `ws` is caller-owned device memory of at least vsa2_workspace_size() bytes,
+ *    256-byte aligned, zeroed once by vsa2_workspace_init before first use. One workspace
+ *    must not be used by two calls that may run concurrently.
+ */
+#ifndef VSA2_H_
+#define VSA2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VSA2_OK = 0,
+  VSA2_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer, small workspace */
+  VSA2_ERR_UNSUPPORTED = 2, /* shape or dtype outside the supported set */
+  VSA2_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  VSA2_ERR_TIMEOUT = 4,     /* a bounded device-side wait expired (kernel returned early) */
+  VSA2_ERR_BAD_INDEX = 5    /* validate mode: an offset or index was out of range */
+} vsa2_status;
+
+typedef enum { VSA2_BF16 = 0, VSA2_FP32 = 1 } vsa2_dtype;
+
+enum {
+  VSA2_FLAG_VALIDATE = 1u << 0 /* kernels bounds-check every offset and index they read */
+};
+
+typedef struct vsa2_problem {
+  int64_t batch, heads, head_dim;   /* Bsz, H, D */
+  int64_t grid_t, grid_h, grid_w;   /* latent token grid T x H x W */
+  int32_t tile_t, tile_h, tile_w;   /* block (tile) cube, 4 x 4 x 4 -> Bt = 64 */
+  int32_t pool_t, pool_h, pool_w;   /* router pooling sub-cube, 2 x 2 x 4 -> R = 16 */
+  int32_t dtype;                    /* vsa2_dtype */
+  uint32_t flags;                   /* VSA2_FLAG_* */
+  uint32_t wait_timeout_ms;         /* bound on any single device-side wait; 0 = 2000 ms */
+  uint32_t reserved;
+} vsa2_problem;
+
+/* Bytes of workspace that every call below needs for this problem and budget. */
+size_t vsa2_workspace_size(const vsa2_problem* p, int32_t topk);
+
+/* Zero the workspace header (the device error word); enqueued on `stream`. Call once after
+ * allocating a workspace. Returns VSA2_ERR_INVALID_ARG for a null or too-small workspace. */
+vsa2_status vsa2_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Router scores, Eq. 5-7 with the two-pass fused kernel of Fig. 5.
+ *   q, k    : [batch, heads, L, D] of dtype, cube-major (read only)
+ *   scores  : [batch, heads, N, N] fp32 (written). scores[b,h,i,j] =
+ *             (1/G) * sum_{a in tile i} sum_{c in tile j} softmax_c(qr_a . kr_c / sqrt(D)),
+ *             qr, kr the means of Q, K over each R-token sub-cube (Eq. 5), the softmax over all
+ *             L/R pooled keys of (b, h) (Eq. 6), pooled G x G (Eq. 7) and scaled by G so each
+ *             row sums to 1 (the pages' MeanPool_{GxG} divided by G; TopK is unaffected).
+ * The pooled Qr, Kr and per-row LSE live in the workspace; the L/R x L/R matrix is never
+ * written to memory.
+ */
+vsa2_status vsa2_router_scores(const vsa2_problem* p, const void* q, const void* k, float* scores,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Per-sequence TopK, Eq. 8-9: for each (b, h) keep the N*topk largest of the N*N scores;
+ * equal scores are ranked by flat index i*N + j, lower first (the pages fix no tie order).
+ *   scores  : [batch, heads, N, N] fp32, every entry >= 0 and finite (read only)
+ *   kv_off  : [batch, heads, N+1] int32 (written) CSR row offsets, kv_off[.,.,0] = 0,
+ *             kv_off[.,.,N] = N*topk
+ *   kv_idx  : [batch, heads, N*topk] int32 (written) selected KV tiles of query tile i in
+ *             kv_idx[kv_off[i] .. kv_off[i+1]), ascending
+ *   q_off, q_idx : optional (both NULL or both non-NULL) CSC of the same selection: query
+ *             tiles that selected KV tile j, ascending; needed by the backward pass
+ * A query tile may receive zero KV tiles; the total per (b, h) is always N*topk.
+ */
+vsa2_status vsa2_topk_select(const vsa2_problem* p, const float* scores, int32_t topk,
+                             int32_t* kv_off, int32_t* kv_idx, int32_t* q_off, int32_t* q_idx,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Block-sparse attention forward, Eq. 12 with the §2.1 definition. For every query token t
+ * of tile i: o_t = sum_u softmax_u(q_t . k_u / sqrt(D)) v_u over the tokens u of the KV tiles
+ * listed for tile i; lse_t = ln sum_u exp(q_t . k_u / sqrt(D)). A tile with an empty list
+ * gets o = 0 and lse = -inf.
+ *   q, k, v        : [batch, heads, L, D] of dtype (read only)
+ *   topk           : the budget the CSR was built with; kv_idx holds N*topk entries per (b, h)
+ *   kv_off, kv_idx : CSR from vsa2_topk_select, or any CSR of distinct tiles per row with
+ *                    offsets local to each (b, h) and kv_off[., ., N] <= N*topk (read only)
+ *   o              : [batch, heads, L, D] of dtype (written)
+ *   lse            : [batch, heads, L] fp32, natural log (written)
+ */
+vsa2_status vsa2_sparse_attn_fwd(const vsa2_problem* p, const void* q, const void* k, const void* v,
+                                 int32_t topk, const int32_t* kv_off, const int32_t* kv_idx,
+                                 void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Block-sparse attention backward (gradients of Eq. 12; the router receives none, §2.1).
+ *   q, k, v, o, dout : [batch, heads, L, D] of dtype (read only); o and lse from the forward
+ *   lse              : [batch, heads, L] fp32 (read only)
+ *   topk             : budget of the selection (index lists hold N*topk entries per (b, h))
+ *   kv_off, kv_idx   : CSR of the selection; q_off, q_idx : its CSC (read only)
+ *   dq, dk, dv       : [batch, heads, L, D] fp32 (written; fully overwritten)
+ * With P = exp(S - lse), dV = P^T dO, dS = P * (dO V^T - rowsum(dO * O)),
+ * dQ = dS K / sqrt(D), dK = dS^T Q / sqrt(D), each restricted to the selected tile pairs.
+ */
+vsa2_status vsa2_sparse_attn_bwd(const vsa2_problem* p, const void* q, const void* k, const void* v,
+                                 const void* o, const float* lse, const void* dout, int32_t topk,
+                                 const int32_t* kv_off, const int32_t* kv_idx,
+                                 const int32_t* q_off, const int32_t* q_idx,
+                                 float* dq, float* dk, float* dv,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, read and clear the device error word of `ws`. Returns VSA2_OK,
+ * VSA2_ERR_TIMEOUT, VSA2_ERR_BAD_INDEX, or VSA2_ERR_CUDA if the synchronisation failed. */
+vsa2_status vsa2_get_device_error(void* ws, void* stream);
+
+/* Diagnostic: enqueue one kernel that waits, with the problem's bounded wait, on a barrier
+ * that nothing completes. It returns after `timeout_ms` and records VSA2_ERR_TIMEOUT in the
+ * workspace error word; no GPU state other than that word is touched. */
+vsa2_status vsa2_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t timeout_ms, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* vsa2_status_string(vsa2_status s);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t vsa2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA2_H_ */

@@ -1,0 +1,81 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments synchronously (nothing is enqueued)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import synthetic as S
+from trainable_block_sparse_fine_b200 import _capi as C
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "vsa2.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vsa2_[a-z_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = C.lib()
+    declared = _declared_symbols()
+    assert len(declared) >= 10
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) == set(C.EXPORTS)
+
+
+def test_problem_struct_layout():
+    assert ctypes.sizeof(C.Problem) == 88
+    assert C.Problem.dtype.offset == 72
+
+
+def test_status_strings_and_version():
+    for code, name in C.STATUS_NAMES.items():
+        assert C.vsa2_status_string(code) == name
+    assert C.vsa2_version() >= 100
+
+
+@pytest.mark.parametrize("name", list(S.WORKLOADS))
+def test_workspace_size_for_every_workload(name):
+    wl = S.WORKLOADS[name]
+    p = C.make_problem(wl.batch, wl.heads, wl.head_dim, wl.grid, wl.dtype)
+    n = C.vsa2_workspace_size(p, wl.topk)
+    assert n > 0 and n % 256 == 0
+    # pooled Q and K dominate; the workspace stays far below device memory
+    assert n < 1 << 30
+
+
+def test_unsupported_shapes_give_zero_workspace():
+    assert C.vsa2_workspace_size(C.make_problem(1, 2, 96, (8, 16, 16)), 8) == 0  # head_dim
+    assert C.vsa2_workspace_size(C.make_problem(1, 2, 64, (6, 16, 16)), 8) == 0  # grid % tile
+    assert C.vsa2_workspace_size(C.make_problem(1, 2, 64, (8, 16, 16), pool=(2, 2, 2)), 8) == 0  # R != 16
+
+
+def test_argument_errors_are_synchronous():
+    lib = C.lib()
+    p = C.make_problem(1, 2, 64, (8, 16, 16), "fp32")
+    bp = ctypes.byref(p)
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails before any launch
+    ws = ctypes.c_void_p(1 << 24)
+    n = C.vsa2_workspace_size(p, 8)
+    # null pointers
+    assert lib.vsa2_router_scores(bp, None, fake, fake, ws, n, None) == 1
+    # misaligned pointer
+    assert lib.vsa2_router_scores(bp, ctypes.c_void_p((1 << 20) + 4), fake, fake, ws, n, None) == 1
+    # workspace too small
+    assert lib.vsa2_router_scores(bp, fake, fake, fake, ws, n - 256, None) == 1
+    # topk out of range
+    assert lib.vsa2_topk_select(bp, fake, 0, fake, fake, None, None, ws, n, None) == 2
+    assert lib.vsa2_topk_select(bp, fake, 33, fake, fake, None, None, ws, n, None) == 2
+    # CSC pointers must come as a pair
+    assert lib.vsa2_topk_select(bp, fake, 8, fake, fake, fake, None, ws, n, None) == 1
+    assert lib.vsa2_sparse_attn_fwd(bp, fake, fake, fake, 8, fake, None, fake, fake, ws, n, None) == 1
+    assert lib.vsa2_sparse_attn_bwd(bp, fake, fake, fake, fake, fake, fake, 8, fake, fake, None, fake, fake, fake,
+                                    fake, ws, n, None) == 1
+    bad = C.make_problem(1, 2, 64, (8, 16, 16), "fp32")
+    bad.dtype = 7
+    assert lib.vsa2_router_scores(ctypes.byref(bad), fake, fake, fake, ws, n, None) == 2
+    assert lib.vsa2_selftest_wait_timeout(ws, n, 0, None) == 1

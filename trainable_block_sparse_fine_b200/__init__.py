@@ -1,0 +1,108 @@
+"""VSA2 hot path on B200: fine-grained router -> per-sequence TopK -> block-sparse attention.
+
+Every step runs in the CUDA kernels of libvsa2.so (see include/vsa2.h); this module only
+allocates device memory with PyTorch and marshals arguments. Method: "Improving Video Sparse
+Attention with Fine-grained Router and Sparse Rebasing" (arXiv 2609.32882), §2.2.
+
+Inputs are [batch, heads, L, D] tensors in cube-major token order (tiles of 4x4x4 tokens,
+router sub-cubes of 2x2x4 tokens inside each tile).
+"""
+from __future__ import annotations
+
+import torch
+
+from ._capi import (VSA2_FLAG_VALIDATE, Problem, Vsa2Error, lib, make_problem, vsa2_get_device_error,
+                    vsa2_router_scores, vsa2_selftest_wait_timeout, vsa2_sparse_attn_bwd, vsa2_sparse_attn_fwd,
+                    vsa2_status_string, vsa2_topk_select, vsa2_version, vsa2_workspace_init, vsa2_workspace_size)
+
+__all__ = ["VSA2", "Vsa2Error", "Problem", "make_problem", "block_sparse_attention", "lib", "VSA2_FLAG_VALIDATE",
+           "vsa2_router_scores", "vsa2_topk_select", "vsa2_sparse_attn_fwd", "vsa2_sparse_attn_bwd",
+           "vsa2_workspace_size", "vsa2_workspace_init", "vsa2_get_device_error", "vsa2_selftest_wait_timeout",
+           "vsa2_status_string", "vsa2_version"]
+
+
+class VSA2:
+    """One problem shape with its workspace; methods enqueue on the current CUDA stream."""
+
+    def __init__(self, batch, heads, head_dim, grid, dtype="bf16", topk=64, device="cuda", flags=0,
+                 wait_timeout_ms=0):
+        if not torch.cuda.is_available():
+            raise RuntimeError("VSA2 needs a CUDA device")
+        lib()  # fail loudly if the native library is missing
+        self.p = make_problem(batch, heads, head_dim, grid, dtype, flags=flags, wait_timeout_ms=wait_timeout_ms)
+        self.batch, self.heads, self.head_dim, self.grid, self.topk = batch, heads, head_dim, tuple(grid), topk
+        self.L = grid[0] * grid[1] * grid[2]
+        self.N = self.L // 64
+        self.dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+        self.device = torch.device(device)
+        n = vsa2_workspace_size(self.p, topk)
+        if n == 0:
+            raise Vsa2Error(2, "vsa2_workspace_size")
+        self.ws = torch.empty((n + 255) // 256 * 256, dtype=torch.uint8, device=self.device)
+        vsa2_workspace_init(self.ws)
+
+    # -- the four calls of the hot path -----------------------------------------------------
+    def router_scores(self, q, k, out=None):
+        out = out if out is not None else torch.empty(self.batch, self.heads, self.N, self.N, dtype=torch.float32,
+                                                      device=self.device)
+        vsa2_router_scores(self.p, q, k, out, self.ws)
+        return out
+
+    def topk_select(self, scores, topk=None, csc=True):
+        topk = self.topk if topk is None else topk
+        bh = (self.batch, self.heads)
+        i32 = dict(dtype=torch.int32, device=self.device)
+        kv_off = torch.empty(*bh, self.N + 1, **i32)
+        kv_idx = torch.empty(*bh, self.N * topk, **i32)
+        q_off = torch.empty(*bh, self.N + 1, **i32) if csc else None
+        q_idx = torch.empty(*bh, self.N * topk, **i32) if csc else None
+        vsa2_topk_select(self.p, scores, topk, kv_off, kv_idx, q_off, q_idx, self.ws)
+        return kv_off, kv_idx, q_off, q_idx
+
+    def attn_fwd(self, q, k, v, kv_off, kv_idx, topk=None, o=None, lse=None):
+        topk = self.topk if topk is None else topk
+        o = o if o is not None else torch.empty_like(q)
+        lse = lse if lse is not None else torch.empty(self.batch, self.heads, self.L, dtype=torch.float32,
+                                                      device=self.device)
+        vsa2_sparse_attn_fwd(self.p, q, k, v, topk, kv_off, kv_idx, o, lse, self.ws)
+        return o, lse
+
+    def attn_bwd(self, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, topk=None):
+        topk = self.topk if topk is None else topk
+        f32 = dict(dtype=torch.float32, device=self.device)
+        dq, dk, dv = (torch.empty(q.shape, **f32) for _ in range(3))
+        vsa2_sparse_attn_bwd(self.p, q, k, v, o, lse, dout, topk, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, self.ws)
+        return dq, dk, dv
+
+    def forward(self, q, k, v, topk=None, csc=False):
+        """Router -> TopK -> block-sparse attention forward. Returns (o, lse, selection)."""
+        scores = self.router_scores(q, k)
+        sel = self.topk_select(scores, topk, csc=csc)
+        o, lse = self.attn_fwd(q, k, v, sel[0], sel[1], topk)
+        return o, lse, sel
+
+    def device_error(self) -> int:
+        return vsa2_get_device_error(self.ws)
+
+
+class _BlockSparseAttention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, engine: VSA2, topk):
+        with torch.no_grad():  # the router receives no gradient (§2.1)
+            scores = engine.router_scores(q, k)
+            kv_off, kv_idx, q_off, q_idx = engine.topk_select(scores, topk, csc=True)
+        o, lse = engine.attn_fwd(q, k, v, kv_off, kv_idx, topk)
+        ctx.save_for_backward(q, k, v, o, lse, kv_off, kv_idx, q_off, q_idx)
+        ctx.engine, ctx.topk = engine, topk
+        return o
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, o, lse, kv_off, kv_idx, q_off, q_idx = ctx.saved_tensors
+        dq, dk, dv = ctx.engine.attn_bwd(q, k, v, o, lse, dout.contiguous(), kv_off, kv_idx, q_off, q_idx, ctx.topk)
+        return dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), None, None
+
+
+def block_sparse_attention(q, k, v, engine: VSA2, topk=None):
+    """VSA2 fine branch with its router: o = BlockSparseAttn(q, k, v; TopK_{NK}(router(q, k)))."""
+    return _BlockSparseAttention.apply(q, k, v, engine, engine.topk if topk is None else topk)

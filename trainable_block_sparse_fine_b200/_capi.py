@@ -1,0 +1,147 @@
+"""ctypes binding of libvsa2.so: the C entry points under the same names, with torch tensors
+marshalled to device pointers. No arithmetic of the method happens here."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libvsa2.so")
+
+VSA2_OK = 0
+STATUS_NAMES = {0: "VSA2_OK", 1: "VSA2_ERR_INVALID_ARG", 2: "VSA2_ERR_UNSUPPORTED", 3: "VSA2_ERR_CUDA",
+                4: "VSA2_ERR_TIMEOUT", 5: "VSA2_ERR_BAD_INDEX"}
+VSA2_BF16, VSA2_FP32 = 0, 1
+VSA2_FLAG_VALIDATE = 1
+
+# every symbol the header declares
+EXPORTS = ("vsa2_workspace_size", "vsa2_workspace_init", "vsa2_router_scores", "vsa2_topk_select",
+           "vsa2_sparse_attn_fwd", "vsa2_sparse_attn_bwd", "vsa2_get_device_error",
+           "vsa2_selftest_wait_timeout", "vsa2_status_string", "vsa2_version")
+
+
+class Vsa2Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("heads", ctypes.c_int64), ("head_dim", ctypes.c_int64),
+                ("grid_t", ctypes.c_int64), ("grid_h", ctypes.c_int64), ("grid_w", ctypes.c_int64),
+                ("tile_t", ctypes.c_int32), ("tile_h", ctypes.c_int32), ("tile_w", ctypes.c_int32),
+                ("pool_t", ctypes.c_int32), ("pool_h", ctypes.c_int32), ("pool_w", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("flags", ctypes.c_uint32), ("wait_timeout_ms", ctypes.c_uint32),
+                ("reserved", ctypes.c_uint32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libvsa2.so (built in-tree). Fails loudly when it is missing: there is no fallback."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing; build it with trainable_block_sparse_fine_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER(Problem)
+        vp, sz, i32, u32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_uint32
+        L.vsa2_workspace_size.argtypes = [P, i32]
+        L.vsa2_workspace_size.restype = sz
+        L.vsa2_workspace_init.argtypes = [vp, sz, vp]
+        L.vsa2_router_scores.argtypes = [P, vp, vp, vp, vp, sz, vp]
+        L.vsa2_topk_select.argtypes = [P, vp, i32, vp, vp, vp, vp, vp, sz, vp]
+        L.vsa2_sparse_attn_fwd.argtypes = [P, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]
+        L.vsa2_sparse_attn_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.vsa2_get_device_error.argtypes = [vp, vp]
+        L.vsa2_selftest_wait_timeout.argtypes = [vp, sz, u32, vp]
+        L.vsa2_status_string.argtypes = [ctypes.c_int]
+        L.vsa2_status_string.restype = ctypes.c_char_p
+        L.vsa2_version.restype = i32
+        for name in ("vsa2_workspace_init", "vsa2_router_scores", "vsa2_topk_select", "vsa2_sparse_attn_fwd",
+                     "vsa2_sparse_attn_bwd", "vsa2_get_device_error", "vsa2_selftest_wait_timeout"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+        return t.data_ptr()
+    return int(t)
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(status: int, where: str) -> None:
+    if status != VSA2_OK:
+        raise Vsa2Error(status, where)
+
+
+def make_problem(batch, heads, head_dim, grid, dtype="bf16", tile=(4, 4, 4), pool=(2, 2, 4), flags=0,
+                 wait_timeout_ms=0) -> Problem:
+    return Problem(batch, heads, head_dim, *grid, *tile, *pool, VSA2_BF16 if dtype == "bf16" else VSA2_FP32,
+                   flags, wait_timeout_ms, 0)
+
+
+def vsa2_workspace_size(p: Problem, topk: int) -> int:
+    return lib().vsa2_workspace_size(ctypes.byref(p), topk)
+
+
+def vsa2_workspace_init(ws: torch.Tensor, stream=None) -> None:
+    _check(lib().vsa2_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "vsa2_workspace_init")
+
+
+def vsa2_router_scores(p: Problem, q, k, scores, ws, stream=None) -> None:
+    _check(lib().vsa2_router_scores(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(scores), _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream(stream)), "vsa2_router_scores")
+
+
+def vsa2_topk_select(p: Problem, scores, topk, kv_off, kv_idx, q_off, q_idx, ws, stream=None) -> None:
+    _check(lib().vsa2_topk_select(ctypes.byref(p), _ptr(scores), topk, _ptr(kv_off), _ptr(kv_idx), _ptr(q_off),
+                                  _ptr(q_idx), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "vsa2_topk_select")
+
+
+def vsa2_sparse_attn_fwd(p: Problem, q, k, v, topk, kv_off, kv_idx, o, lse, ws, stream=None) -> None:
+    _check(lib().vsa2_sparse_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), topk, _ptr(kv_off), _ptr(kv_idx),
+                                      _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "vsa2_sparse_attn_fwd")
+
+
+def vsa2_sparse_attn_bwd(p: Problem, q, k, v, o, lse, dout, topk, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, ws,
+                         stream=None) -> None:
+    _check(lib().vsa2_sparse_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                      topk, _ptr(kv_off), _ptr(kv_idx), _ptr(q_off), _ptr(q_idx), _ptr(dq), _ptr(dk),
+                                      _ptr(dv), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "vsa2_sparse_attn_bwd")
+
+
+def vsa2_get_device_error(ws, stream=None) -> int:
+    return lib().vsa2_get_device_error(_ptr(ws), _stream(stream))
+
+
+def vsa2_selftest_wait_timeout(ws, timeout_ms: int, stream=None) -> None:
+    _check(lib().vsa2_selftest_wait_timeout(_ptr(ws), ws.numel() * ws.element_size(), timeout_ms, _stream(stream)),
+           "vsa2_selftest_wait_timeout")
+
+
+def vsa2_status_string(status: int) -> str:
+    return lib().vsa2_status_string(status).decode()
+
+
+def vsa2_version() -> int:
+    return lib().vsa2_version()

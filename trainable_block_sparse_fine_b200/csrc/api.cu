@@ -1,0 +1,211 @@
+// C ABI of libvsa2: argument validation, workspace layout and dispatch to the kernels.
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace vsa2 {
+
+vsa2_status make_dims(const vsa2_problem* p, Dims* d) {
+  if (!p || !d) return VSA2_ERR_INVALID_ARG;
+  if (p->batch <= 0 || p->heads <= 0 || p->head_dim <= 0 || p->grid_t <= 0 || p->grid_h <= 0 || p->grid_w <= 0)
+    return VSA2_ERR_INVALID_ARG;
+  if (p->tile_t <= 0 || p->tile_h <= 0 || p->tile_w <= 0 || p->pool_t <= 0 || p->pool_h <= 0 || p->pool_w <= 0)
+    return VSA2_ERR_INVALID_ARG;
+  if (p->dtype != VSA2_BF16 && p->dtype != VSA2_FP32) return VSA2_ERR_UNSUPPORTED;
+  if (p->head_dim != 64 && p->head_dim != 128) return VSA2_ERR_UNSUPPORTED;
+  if (p->tile_t * p->tile_h * p->tile_w != kTile) return VSA2_ERR_UNSUPPORTED;
+  if (p->pool_t * p->pool_h * p->pool_w != kPool) return VSA2_ERR_UNSUPPORTED;
+  if (p->grid_t % p->tile_t || p->grid_h % p->tile_h || p->grid_w % p->tile_w) return VSA2_ERR_UNSUPPORTED;
+  if (p->tile_t % p->pool_t || p->tile_h % p->pool_h || p->tile_w % p->pool_w) return VSA2_ERR_UNSUPPORTED;
+  const int64_t L = p->grid_t * p->grid_h * p->grid_w;
+  const int64_t N = L / kTile;
+  const int64_t BH = p->batch * p->heads;
+  // index arithmetic below uses 32-bit tile and row counts
+  if (N > 32768 || BH > 65535 || BH * L > (int64_t(1) << 31)) return VSA2_ERR_UNSUPPORTED;
+  d->B = (int)p->batch;
+  d->H = (int)p->heads;
+  d->D = (int)p->head_dim;
+  d->BH = (int)BH;
+  d->L = L;
+  d->N = (int)N;
+  d->Lr = (int)(L / kPool);
+  d->dtype = p->dtype;
+  d->esize = p->dtype == VSA2_BF16 ? 2 : 4;
+  d->flags = p->flags;
+  d->timeout_ns = (uint64_t)(p->wait_timeout_ms ? p->wait_timeout_ms : 2000u) * 1000000ull;
+  return VSA2_OK;
+}
+
+WsLayout ws_layout(const Dims& d) {
+  WsLayout w{};
+  size_t off = kWsHeader;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off += align256(bytes);
+    return at;
+  };
+  w.qr = take((size_t)d.BH * d.Lr * d.D * d.esize);
+  w.kr = take((size_t)d.BH * d.Lr * d.D * d.esize);
+  w.lse_r = take((size_t)d.BH * d.Lr * 4);
+  w.hist = take((size_t)d.BH * 3 * 2048 * 4);
+  w.state = take((size_t)d.BH * 8 * 4);
+  w.row_gt = take((size_t)d.BH * d.N * 4);
+  w.row_eq = take((size_t)d.BH * d.N * 4);
+  w.row_take = take((size_t)d.BH * d.N * 4);
+  w.col_cnt = take((size_t)d.BH * d.N * 4);
+  w.words = (d.N + 31) / 32;
+  w.col_bits = take((size_t)d.BH * d.N * w.words * 4);
+  w.delta = take((size_t)d.BH * d.L * 4);
+  w.total = off;
+  return w;
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t outer,
+                       uint32_t box_cols, uint32_t box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cols, rows, outer};
+  cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
+  cuuint32_t box[3] = {box_cols, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static vsa2_status check_ws(const Dims& d, void* ws, size_t ws_bytes) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return VSA2_ERR_INVALID_ARG;
+  if (ws_bytes < ws_layout(d).total) return VSA2_ERR_INVALID_ARG;
+  return VSA2_OK;
+}
+
+}  // namespace vsa2
+
+using namespace vsa2;
+
+extern "C" {
+
+size_t vsa2_workspace_size(const vsa2_problem* p, int32_t topk) {
+  (void)topk;
+  Dims d;
+  if (make_dims(p, &d) != VSA2_OK) return 0;
+  return ws_layout(d).total;
+}
+
+vsa2_status vsa2_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < kWsHeader || (reinterpret_cast<uintptr_t>(ws) & 255u)) return VSA2_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(ws, 0, kWsHeader, (cudaStream_t)stream) != cudaSuccess) return VSA2_ERR_CUDA;
+  return VSA2_OK;
+}
+
+vsa2_status vsa2_router_scores(const vsa2_problem* p, const void* q, const void* k, float* scores, void* ws,
+                               size_t ws_bytes, void* stream) {
+  Dims d;
+  vsa2_status st = make_dims(p, &d);
+  if (st != VSA2_OK) return st;
+  if (!q || !k || !scores) return VSA2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(scores)) return VSA2_ERR_INVALID_ARG;
+  if ((st = check_ws(d, ws, ws_bytes)) != VSA2_OK) return st;
+  return launch_router(d, q, k, scores, (char*)ws, (cudaStream_t)stream);
+}
+
+vsa2_status vsa2_topk_select(const vsa2_problem* p, const float* scores, int32_t topk, int32_t* kv_off,
+                             int32_t* kv_idx, int32_t* q_off, int32_t* q_idx, void* ws, size_t ws_bytes,
+                             void* stream) {
+  Dims d;
+  vsa2_status st = make_dims(p, &d);
+  if (st != VSA2_OK) return st;
+  if (!scores || !kv_off || !kv_idx) return VSA2_ERR_INVALID_ARG;
+  if ((q_off == nullptr) != (q_idx == nullptr)) return VSA2_ERR_INVALID_ARG;
+  if (topk < 1 || topk > d.N) return VSA2_ERR_UNSUPPORTED;
+  if (!aligned16(scores)) return VSA2_ERR_INVALID_ARG;
+  if ((st = check_ws(d, ws, ws_bytes)) != VSA2_OK) return st;
+  return launch_topk(d, scores, topk, kv_off, kv_idx, q_off, q_idx, (char*)ws, (cudaStream_t)stream);
+}
+
+vsa2_status vsa2_sparse_attn_fwd(const vsa2_problem* p, const void* q, const void* k, const void* v, int32_t topk,
+                                 const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  Dims d;
+  vsa2_status st = make_dims(p, &d);
+  if (st != VSA2_OK) return st;
+  if (!q || !k || !v || !kv_off || !kv_idx || !o || !lse) return VSA2_ERR_INVALID_ARG;
+  if (topk < 1 || topk > d.N) return VSA2_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return VSA2_ERR_INVALID_ARG;
+  if ((st = check_ws(d, ws, ws_bytes)) != VSA2_OK) return st;
+  return launch_attn_fwd(d, q, k, v, topk, kv_off, kv_idx, o, lse, (char*)ws, (cudaStream_t)stream);
+}
+
+vsa2_status vsa2_sparse_attn_bwd(const vsa2_problem* p, const void* q, const void* k, const void* v, const void* o,
+                                 const float* lse, const void* dout, int32_t topk, const int32_t* kv_off,
+                                 const int32_t* kv_idx,
+                                 const int32_t* q_off, const int32_t* q_idx, float* dq, float* dk, float* dv,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  vsa2_status st = make_dims(p, &d);
+  if (st != VSA2_OK) return st;
+  if (!q || !k || !v || !o || !lse || !dout || !kv_off || !kv_idx || !q_off || !q_idx || !dq || !dk || !dv)
+    return VSA2_ERR_INVALID_ARG;
+  if (topk < 1 || topk > d.N) return VSA2_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || !aligned16(lse))
+    return VSA2_ERR_INVALID_ARG;
+  if ((st = check_ws(d, ws, ws_bytes)) != VSA2_OK) return st;
+  return launch_attn_bwd(d, q, k, v, o, lse, dout, topk, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, (char*)ws,
+                         (cudaStream_t)stream);
+}
+
+vsa2_status vsa2_get_device_error(void* ws, void* stream) {
+  if (!ws) return VSA2_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return VSA2_ERR_CUDA;
+  int code = 0;
+  if (cudaMemcpy(&code, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return VSA2_ERR_CUDA;
+  if (code != 0) {
+    int zero = 0;
+    if (cudaMemcpy(ws, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return VSA2_ERR_CUDA;
+  }
+  return (vsa2_status)code;
+}
+
+vsa2_status vsa2_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t timeout_ms, void* stream) {
+  if (!ws || ws_bytes < kWsHeader || (reinterpret_cast<uintptr_t>(ws) & 255u)) return VSA2_ERR_INVALID_ARG;
+  if (timeout_ms == 0 || timeout_ms > 10000) return VSA2_ERR_INVALID_ARG;
+  return launch_wait_timeout_probe((int*)ws, (uint64_t)timeout_ms * 1000000ull, (cudaStream_t)stream);
+}
+
+const char* vsa2_status_string(vsa2_status s) {
+  switch (s) {
+    case VSA2_OK: return "VSA2_OK";
+    case VSA2_ERR_INVALID_ARG: return "VSA2_ERR_INVALID_ARG";
+    case VSA2_ERR_UNSUPPORTED: return "VSA2_ERR_UNSUPPORTED";
+    case VSA2_ERR_CUDA: return "VSA2_ERR_CUDA";
+    case VSA2_ERR_TIMEOUT: return "VSA2_ERR_TIMEOUT";
+    case VSA2_ERR_BAD_INDEX: return "VSA2_ERR_BAD_INDEX";
+  }
+  return "VSA2_UNKNOWN_STATUS";
+}
+
+int32_t vsa2_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,326 @@
+// CUDA-core block-sparse attention (Eq. 12 of "Improving Video Sparse Attention with
+// Fine-grained Router and Sparse Rebasing"; §2.1 definition) for the shapes the tensor-core
+// kernels do not take: fp32 inputs and head_dim 64, plus the backward pass.
+// Arithmetic is fp32 throughout.
+#include "common.cuh"
+#include "internal.h"
+
+namespace vsa2 {
+
+template <typename T>
+__device__ __forceinline__ float ldf(const T* p) {
+  if constexpr (sizeof(T) == 2)
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
+  else
+    return *p;
+}
+template <typename T>
+__device__ __forceinline__ void stf(T* p, float v) {
+  if constexpr (sizeof(T) == 2)
+    *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(v);
+  else
+    *p = v;
+}
+
+// Checks one CSR/CSC row in validate mode; returns false (and records the error) if broken.
+__device__ __forceinline__ bool row_ok(int beg, int end, int cap, const DevCtx& ctx) {
+  if (!(ctx.flags & VSA2_FLAG_VALIDATE)) return true;
+  if (beg < 0 || end < beg || end > cap) {
+    set_error(ctx.err, VSA2_ERR_BAD_INDEX);
+    return false;
+  }
+  return true;
+}
+__device__ __forceinline__ bool idx_ok(int j, int N, const DevCtx& ctx) {
+  if (!(ctx.flags & VSA2_FLAG_VALIDATE)) return true;
+  if (j < 0 || j >= N) {
+    set_error(ctx.err, VSA2_ERR_BAD_INDEX);
+    return false;
+  }
+  return true;
+}
+
+namespace {
+
+// Forward: CTA = one query tile of one (b, h), thread t = query row t.
+template <typename T, int D>
+__global__ void __launch_bounds__(64) attn_fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                           const T* __restrict__ v, const int32_t* __restrict__ kv_off,
+                                                           const int32_t* __restrict__ kv_idx, T* __restrict__ o,
+                                                           float* __restrict__ lse, int N, int64_t L, int topk,
+                                                           DevCtx ctx) {
+  extern __shared__ float sm[];
+  float* qT = sm;              // [D][64]
+  float* ks = qT + D * 64;     // [64][D]
+  float* vs = ks + 64 * D;     // [64][D]
+  float* oT = vs + 64 * D;     // [D][64]
+  const int i = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+  const size_t tok0 = (size_t)bh * L + (size_t)i * kTile;
+  for (int e = t; e < 64 * D; e += 64) {
+    const int r = e / D, c = e % D;
+    qT[c * 64 + r] = ldf(q + (tok0 + r) * D + c);
+    oT[c * 64 + r] = 0.f;
+  }
+  const int beg = kv_off[(size_t)bh * (N + 1) + i], end = kv_off[(size_t)bh * (N + 1) + i + 1];
+  const bool ok = row_ok(beg, end, N * topk, ctx);
+  const int32_t* idx = kv_idx + (size_t)bh * N * topk;
+  const float scale = rsqrtf((float)D);
+  float m = -INFINITY, l = 0.f;
+  __syncthreads();
+  for (int p = beg; ok && p < end; ++p) {
+    const int j = idx[p];
+    if (!idx_ok(j, N, ctx)) break;
+    const size_t kt0 = (size_t)bh * L + (size_t)j * kTile;
+    __syncthreads();
+    for (int e = t; e < 64 * D; e += 64) {
+      ks[e] = ldf(k + kt0 * D + e);
+      vs[e] = ldf(v + kt0 * D + e);
+    }
+    __syncthreads();
+    float s[64];
+    float mx = -INFINITY;
+#pragma unroll 4
+    for (int u = 0; u < 64; ++u) {
+      float acc = 0.f;
+      for (int d = 0; d < D; ++d) acc += qT[d * 64 + t] * ks[u * D + d];
+      s[u] = acc * scale;
+      mx = fmaxf(mx, s[u]);
+    }
+    const float mn = fmaxf(m, mx);
+    const float alpha = __expf(m - mn);
+    float sum = 0.f;
+#pragma unroll
+    for (int u = 0; u < 64; ++u) {
+      s[u] = __expf(s[u] - mn);
+      sum += s[u];
+    }
+    l = l * alpha + sum;
+    m = mn;
+    for (int d = 0; d < D; ++d) {
+      float acc = oT[d * 64 + t] * alpha;
+#pragma unroll
+      for (int u = 0; u < 64; ++u) acc += s[u] * vs[u * D + d];
+      oT[d * 64 + t] = acc;
+    }
+  }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  for (int d = 0; d < D; ++d) stf(o + (tok0 + t) * D + d, oT[d * 64 + t] * inv);
+  lse[tok0 + t] = l > 0.f ? m + __logf(l) : -INFINITY;
+}
+
+// delta = rowsum(dO * O), warp per row.
+template <typename T>
+__global__ void __launch_bounds__(256) attn_bwd_delta_kernel(const T* __restrict__ o, const T* __restrict__ dout,
+                                                             float* __restrict__ delta, int64_t rows, int D) {
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float acc = 0.f;
+  for (int d = lane; d < D; d += 32) acc += ldf(o + row * D + d) * ldf(dout + row * D + d);
+#pragma unroll
+  for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) delta[row] = acc;
+}
+
+// dQ: CTA = one query tile, 128 threads = (query row t, half h). Over the tile's CSR list.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) attn_bwd_dq_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                               const T* __restrict__ v, const T* __restrict__ dout,
+                                                               const float* __restrict__ lse,
+                                                               const float* __restrict__ delta,
+                                                               const int32_t* __restrict__ kv_off,
+                                                               const int32_t* __restrict__ kv_idx,
+                                                               float* __restrict__ dq, int N, int64_t L, int topk,
+                                                               DevCtx ctx) {
+  extern __shared__ float sm[];
+  float* qT = sm;             // [D][64]
+  float* doT = qT + D * 64;   // [D][64]
+  float* ks = doT + D * 64;   // [64][D]
+  float* vs = ks + 64 * D;    // [64][D]
+  float* dsT = vs + 64 * D;   // [64 (u)][64 (t)]
+  const int i = blockIdx.x, bh = blockIdx.y;
+  const int t = threadIdx.x & 63, h = threadIdx.x >> 6;
+  const size_t tok0 = (size_t)bh * L + (size_t)i * kTile;
+  for (int e = threadIdx.x; e < 64 * D; e += 128) {
+    const int r = e / D, c = e % D;
+    qT[c * 64 + r] = ldf(q + (tok0 + r) * D + c);
+    doT[c * 64 + r] = ldf(dout + (tok0 + r) * D + c);
+  }
+  const float my_lse = lse[tok0 + t], my_delta = delta[tok0 + t];
+  const float scale = rsqrtf((float)D);
+  float acc[D / 2];
+#pragma unroll
+  for (int d = 0; d < D / 2; ++d) acc[d] = 0.f;
+  const int beg = kv_off[(size_t)bh * (N + 1) + i], end = kv_off[(size_t)bh * (N + 1) + i + 1];
+  const bool ok = row_ok(beg, end, N * topk, ctx);
+  const int32_t* idx = kv_idx + (size_t)bh * N * topk;
+  for (int p = beg; ok && p < end; ++p) {
+    const int j = idx[p];
+    if (!idx_ok(j, N, ctx)) break;
+    const size_t kt0 = (size_t)bh * L + (size_t)j * kTile;
+    __syncthreads();
+    for (int e = threadIdx.x; e < 64 * D; e += 128) {
+      ks[e] = ldf(k + kt0 * D + e);
+      vs[e] = ldf(v + kt0 * D + e);
+    }
+    __syncthreads();
+    for (int u = 32 * h; u < 32 * h + 32; ++u) {
+      float s = 0.f, dp = 0.f;
+      for (int d = 0; d < D; ++d) {
+        s += qT[d * 64 + t] * ks[u * D + d];
+        dp += doT[d * 64 + t] * vs[u * D + d];
+      }
+      const float pr = my_lse == -INFINITY ? 0.f : __expf(s * scale - my_lse);
+      dsT[u * 64 + t] = pr * (dp - my_delta);
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int u = 0; u < 64; ++u) {
+      const float ds = dsT[u * 64 + t];
+#pragma unroll
+      for (int d = 0; d < D / 2; ++d) acc[d] += ds * ks[u * D + h * (D / 2) + d];
+    }
+  }
+#pragma unroll
+  for (int d = 0; d < D / 2; ++d) dq[(tok0 + t) * D + h * (D / 2) + d] = acc[d] * scale;
+}
+
+// dK, dV: CTA = one KV tile, 128 threads = (key row u, half h). Over the tile's CSC list.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) attn_bwd_dkdv_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                                 const T* __restrict__ v, const T* __restrict__ dout,
+                                                                 const float* __restrict__ lse,
+                                                                 const float* __restrict__ delta,
+                                                                 const int32_t* __restrict__ q_off,
+                                                                 const int32_t* __restrict__ q_idx,
+                                                                 float* __restrict__ dk, float* __restrict__ dv, int N,
+                                                                 int64_t L, int topk, DevCtx ctx) {
+  extern __shared__ float sm[];
+  float* kT = sm;             // [D][64]
+  float* vT = kT + D * 64;    // [D][64]
+  float* qs = vT + D * 64;    // [64][D]
+  float* dos = qs + 64 * D;   // [64][D]
+  float* ps = dos + 64 * D;   // [64 (t)][64 (u)]
+  float* dss = ps + 64 * 64;  // [64 (t)][64 (u)]
+  __shared__ float lse_s[64], delta_s[64];
+  const int j = blockIdx.x, bh = blockIdx.y;
+  const int u = threadIdx.x & 63, h = threadIdx.x >> 6;
+  const size_t kt0 = (size_t)bh * L + (size_t)j * kTile;
+  for (int e = threadIdx.x; e < 64 * D; e += 128) {
+    const int r = e / D, c = e % D;
+    kT[c * 64 + r] = ldf(k + (kt0 + r) * D + c);
+    vT[c * 64 + r] = ldf(v + (kt0 + r) * D + c);
+  }
+  const float scale = rsqrtf((float)D);
+  float adk[D / 2], adv[D / 2];
+#pragma unroll
+  for (int d = 0; d < D / 2; ++d) adk[d] = 0.f, adv[d] = 0.f;
+  const int beg = q_off[(size_t)bh * (N + 1) + j], end = q_off[(size_t)bh * (N + 1) + j + 1];
+  const bool ok = row_ok(beg, end, N * topk, ctx);
+  const int32_t* idx = q_idx + (size_t)bh * N * topk;
+  for (int p = beg; ok && p < end; ++p) {
+    const int i = idx[p];
+    if (!idx_ok(i, N, ctx)) break;
+    const size_t tok0 = (size_t)bh * L + (size_t)i * kTile;
+    __syncthreads();
+    for (int e = threadIdx.x; e < 64 * D; e += 128) {
+      qs[e] = ldf(q + tok0 * D + e);
+      dos[e] = ldf(dout + tok0 * D + e);
+    }
+    if (threadIdx.x < 64) {
+      lse_s[threadIdx.x] = lse[tok0 + threadIdx.x];
+      delta_s[threadIdx.x] = delta[tok0 + threadIdx.x];
+    }
+    __syncthreads();
+    for (int t = 32 * h; t < 32 * h + 32; ++t) {
+      float s = 0.f, dp = 0.f;
+      for (int d = 0; d < D; ++d) {
+        s += qs[t * D + d] * kT[d * 64 + u];
+        dp += dos[t * D + d] * vT[d * 64 + u];
+      }
+      const float pr = lse_s[t] == -INFINITY ? 0.f : __expf(s * scale - lse_s[t]);
+      ps[t * 64 + u] = pr;
+      dss[t * 64 + u] = pr * (dp - delta_s[t]);
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int t = 0; t < 64; ++t) {
+      const float pr = ps[t * 64 + u], ds = dss[t * 64 + u];
+#pragma unroll
+      for (int d = 0; d < D / 2; ++d) {
+        adv[d] += pr * dos[t * D + h * (D / 2) + d];
+        adk[d] += ds * qs[t * D + h * (D / 2) + d];
+      }
+    }
+  }
+#pragma unroll
+  for (int d = 0; d < D / 2; ++d) {
+    dk[(kt0 + u) * D + h * (D / 2) + d] = adk[d] * scale;
+    dv[(kt0 + u) * D + h * (D / 2) + d] = adv[d];
+  }
+}
+
+template <typename T, int D>
+vsa2_status fwd_simt(const Dims& d, const void* q, const void* k, const void* v, const int32_t* kv_off,
+                     const int32_t* kv_idx, void* o, float* lse, const DevCtx& ctx, int topk, cudaStream_t s) {
+  const size_t smem = (size_t)4 * 64 * D * sizeof(float);
+  auto kern = attn_fwd_simt_kernel<T, D>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  kern<<<dim3(d.N, d.BH), 64, smem, s>>>((const T*)q, (const T*)k, (const T*)v, kv_off, kv_idx, (T*)o, lse, d.N,
+                                         d.L, topk, ctx);
+  return cudaGetLastError() == cudaSuccess ? VSA2_OK : VSA2_ERR_CUDA;
+}
+
+template <typename T, int D>
+vsa2_status bwd_simt(const Dims& d, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                     const void* dout, const int32_t* kv_off, const int32_t* kv_idx, const int32_t* q_off,
+                     const int32_t* q_idx, float* dq, float* dk, float* dv, float* delta, int topk,
+                     const DevCtx& ctx, cudaStream_t s) {
+  const int64_t rows = (int64_t)d.BH * d.L;
+  attn_bwd_delta_kernel<T><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>((const T*)o, (const T*)dout, delta, rows, d.D);
+  const size_t smem_dq = ((size_t)4 * 64 * D + 64 * 64) * sizeof(float);
+  auto kq = attn_bwd_dq_simt_kernel<T, D>;
+  cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dq);
+  kq<<<dim3(d.N, d.BH), 128, smem_dq, s>>>((const T*)q, (const T*)k, (const T*)v, (const T*)dout, lse, delta,
+                                           kv_off, kv_idx, dq, d.N, d.L, topk, ctx);
+  const size_t smem_kv = ((size_t)4 * 64 * D + 2 * 64 * 64) * sizeof(float);
+  auto kk = attn_bwd_dkdv_simt_kernel<T, D>;
+  cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_kv);
+  kk<<<dim3(d.N, d.BH), 128, smem_kv, s>>>((const T*)q, (const T*)k, (const T*)v, (const T*)dout, lse, delta, q_off,
+                                           q_idx, dk, dv, d.N, d.L, topk, ctx);
+  return cudaGetLastError() == cudaSuccess ? VSA2_OK : VSA2_ERR_CUDA;
+}
+
+}  // namespace
+
+vsa2_status attn_fwd_simt(const Dims& d, const void* q, const void* k, const void* v, int topk,
+                          const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
+                          cudaStream_t s) {
+  DevCtx ctx{reinterpret_cast<int*>(ws), d.timeout_ns, d.flags};
+  if (d.dtype == VSA2_BF16) {
+    if (d.D == 128) return fwd_simt<__nv_bfloat16, 128>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, s);
+    return fwd_simt<__nv_bfloat16, 64>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, s);
+  }
+  if (d.D == 128) return fwd_simt<float, 128>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, s);
+  return fwd_simt<float, 64>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, s);
+}
+
+vsa2_status attn_bwd_simt(const Dims& d, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                          const void* dout, const int32_t* kv_off, const int32_t* kv_idx, const int32_t* q_off,
+                          const int32_t* q_idx, float* dq, float* dk, float* dv, int topk, char* ws, cudaStream_t s) {
+  DevCtx ctx{reinterpret_cast<int*>(ws), d.timeout_ns, d.flags};
+  float* delta = reinterpret_cast<float*>(ws + ws_layout(d).delta);
+  if (d.dtype == VSA2_BF16) {
+    if (d.D == 128)
+      return bwd_simt<__nv_bfloat16, 128>(d, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, delta,
+                                          topk, ctx, s);
+    return bwd_simt<__nv_bfloat16, 64>(d, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, delta,
+                                       topk, ctx, s);
+  }
+  if (d.D == 128)
+    return bwd_simt<float, 128>(d, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, delta, topk, ctx,
+                                s);
+  return bwd_simt<float, 64>(d, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, delta, topk, ctx, s);
+}
+
+}  // namespace vsa2

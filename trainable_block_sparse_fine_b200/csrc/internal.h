@@ -1,0 +1,78 @@
+// Host-side internals of libvsa2: validated problem sizes, workspace layout, launchers.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "vsa2.h"
+
+namespace vsa2 {
+
+constexpr int kTile = 64;  // tokens per tile (4 x 4 x 4 cube)
+constexpr int kPool = 16;  // tokens per router sub-cube (2 x 2 x 4)
+constexpr int kG = kTile / kPool;
+
+struct Dims {
+  int B, H, D, BH;
+  int64_t L;   // tokens per (b, h)
+  int N;       // tiles per (b, h)
+  int Lr;      // pooled rows per (b, h)
+  int dtype;   // vsa2_dtype
+  int esize;   // bytes per element of Q/K/V/O/dO
+  uint32_t flags;
+  uint64_t timeout_ns;
+};
+
+// Validate a problem description; fills `d` on success.
+vsa2_status make_dims(const vsa2_problem* p, Dims* d);
+
+// Workspace regions (byte offsets from the workspace base, all 256-byte aligned).
+struct WsLayout {
+  size_t qr, kr;         // pooled Q, K: [BH, Lr, D] in the input dtype
+  size_t lse_r;          // router per-pooled-row LSE (log2 domain), [BH, Lr] fp32
+  size_t hist;           // TopK radix histograms [BH, 3, 2048] u32
+  size_t state;          // TopK per-(b,h) state [BH, 8] u32
+  size_t row_gt, row_eq, row_take;  // [BH, N] i32
+  size_t col_cnt;        // [BH, N] i32
+  size_t col_bits;       // [BH, N, words] u32
+  int words;             // ceil(N / 32)
+  size_t delta;          // backward rowsum(dO * O), [BH, L] fp32
+  size_t total;
+};
+WsLayout ws_layout(const Dims& d);
+
+// Tensor map for a row-major [outer, rows, cols] bf16 tensor, box (box_cols x box_rows x 1),
+// 128-byte swizzle. Returns false if the driver entry point is unavailable or encoding failed.
+bool make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t outer,
+                       uint32_t box_cols, uint32_t box_rows);
+
+// Launchers (enqueue only). Each returns VSA2_OK or VSA2_ERR_CUDA.
+vsa2_status launch_router(const Dims& d, const void* q, const void* k, float* scores, char* ws, cudaStream_t s);
+vsa2_status launch_topk(const Dims& d, const float* scores, int topk, int32_t* kv_off, int32_t* kv_idx,
+                        int32_t* q_off, int32_t* q_idx, char* ws, cudaStream_t s);
+vsa2_status launch_attn_fwd(const Dims& d, const void* q, const void* k, const void* v, int topk,
+                            const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
+                            cudaStream_t s);
+vsa2_status launch_attn_bwd(const Dims& d, const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dout, int topk, const int32_t* kv_off,
+                            const int32_t* kv_idx, const int32_t* q_off, const int32_t* q_idx, float* dq, float* dk,
+                            float* dv, char* ws, cudaStream_t s);
+// CUDA-core paths (fp32 inputs, head_dim 64, and the backward pass)
+vsa2_status attn_fwd_simt(const Dims& d, const void* q, const void* k, const void* v, int topk,
+                          const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
+                          cudaStream_t s);
+vsa2_status attn_bwd_simt(const Dims& d, const void* q, const void* k, const void* v, const void* o,
+                          const float* lse, const void* dout, const int32_t* kv_off, const int32_t* kv_idx,
+                          const int32_t* q_off, const int32_t* q_idx, float* dq, float* dk, float* dv, int topk,
+                          char* ws, cudaStream_t s);
+// tensor-core forward (bf16, head_dim 128)
+vsa2_status attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v, int topk,
+                        const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
+                        cudaStream_t s);
+vsa2_status launch_wait_timeout_probe(int* err, uint64_t timeout_ns, cudaStream_t s);
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace vsa2

@@ -1,0 +1,405 @@
+// Fine-grained router of VSA2 ("Improving Video Sparse Attention with Fine-grained Router and
+// Sparse Rebasing", §2.2 Eq. 5-7 and Fig. 5): MeanPool_R of Q and K, then a fused two-pass
+// kernel - pass 1 accumulates the log-sum-exp of every pooled query row over all pooled keys,
+// pass 2 recomputes the logits, applies the softmax and pools G x G on chip, writing only the
+// N x N tile scores.
+#include "common.cuh"
+#include "internal.h"
+
+namespace vsa2 {
+namespace {
+
+// ------------------------------------------------------------------------------------------
+// MeanPool_R (Eq. 5): each pooled row is the mean of R = 16 consecutive cube-major rows.
+// One thread per (pooled row, 16-byte column chunk); 16 independent 16-byte loads per thread.
+// ------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) router_pool_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                          T* __restrict__ qr, T* __restrict__ kr,
+                                                          int64_t pooled_rows, int chunks_per_row) {
+  constexpr int EPC = 16 / sizeof(T);  // elements per 16-byte chunk
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t per_tensor = pooled_rows * chunks_per_row;
+  if (tid >= 2 * per_tensor) return;
+  const bool is_k = tid >= per_tensor;
+  const int64_t t = is_k ? tid - per_tensor : tid;
+  const int64_t prow = t / chunks_per_row;
+  const int chunk = (int)(t % chunks_per_row);
+  const T* src = (is_k ? k : q) + (prow * kPool) * (int64_t)chunks_per_row * EPC + chunk * EPC;
+  const int64_t stride = (int64_t)chunks_per_row * EPC;
+  float acc[EPC];
+#pragma unroll
+  for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+  uint4 buf[kPool];
+#pragma unroll
+  for (int r = 0; r < kPool; ++r) buf[r] = __ldg(reinterpret_cast<const uint4*>(src + r * stride));
+#pragma unroll
+  for (int r = 0; r < kPool; ++r) {
+    if constexpr (sizeof(T) == 2) {
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&buf[r]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float2 f = __bfloat1622float2(h[e]);
+        acc[2 * e] += f.x;
+        acc[2 * e + 1] += f.y;
+      }
+    } else {
+      const float* f = reinterpret_cast<const float*>(&buf[r]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] += f[e];
+    }
+  }
+  T* dst = (is_k ? kr : qr) + prow * stride + chunk * EPC;
+  uint4 out;
+  if constexpr (sizeof(T) == 2) {
+    uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] = pack_bf16(acc[2 * e] * (1.f / kPool), acc[2 * e + 1] * (1.f / kPool));
+  } else {
+    float* o = reinterpret_cast<float*>(&out);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] = acc[e] * (1.f / kPool);
+  }
+  *reinterpret_cast<uint4*>(dst) = out;
+}
+
+// ------------------------------------------------------------------------------------------
+// Fused two-pass router scores on tcgen05 (bf16 Qr/Kr, fp32 accumulate in TMEM).
+// CTA = 128 pooled query rows (32 query tiles) of one (b, h). Key chunks of 256 pooled keys
+// (64 key tiles) stream through a 2-stage TMA ring; S = Qr Kr^T lands in one of two TMEM
+// buffers (256 fp32 columns each).
+// Warp roles: 0 = TMA producer, 1 = MMA issuer (+ TMEM owner), 2..9 = softmax/pool epilogue
+// (warp w reads TMEM lanes 32*(w%4).., columns half (w-2)/4 of the chunk).
+// ------------------------------------------------------------------------------------------
+constexpr int RS_M = 128;
+constexpr int RS_N = 256;
+constexpr int RS_THREADS = 320;
+
+template <int ND>  // ND = head_dim / 64
+struct RouterSmem {
+  static constexpr uint32_t kQBytes = 16384u * ND;   // 128 rows x 128 B per 64-column half
+  static constexpr uint32_t kKBytes = 32768u * ND;   // 256 rows x 128 B per half
+  static constexpr uint32_t kQOff = 0;
+  static constexpr uint32_t kKOff = kQBytes;
+  static constexpr uint32_t kTotal = kQBytes + 2 * kKBytes;
+  // slack to align the base to 1024 B; at least 117 KB so that one CTA (and its 512 TMEM
+  // columns) owns the SM
+  static constexpr uint32_t kDyn = (kTotal + 1024 > 119808u) ? kTotal + 1024 : 119808u;
+};
+
+template <int ND>
+__global__ void __launch_bounds__(RS_THREADS, 1)
+    router_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                            float* __restrict__ scores, int Lr, int N, float c2, DevCtx ctx) {
+  using SL = RouterSmem<ND>;
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bar_q, bar_kfull[2], bar_kempty[2], bar_sfull[2], bar_sfree[2], bar_done;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  __shared__ float m_half[2][RS_M], l_half[2][RS_M], lse_sh[RS_M];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const int m0 = blockIdx.x * RS_M;
+  const int nchunk = (Lr + RS_N - 1) / RS_N;
+
+  if (threadIdx.x == 0) {
+    abort_sh = 0;
+    mbar_init(&bar_q, 1);
+    mbar_init(&bar_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_kfull[i], 1);
+      mbar_init(&bar_kempty[i], 1);
+      mbar_init(&bar_sfull[i], 1);
+      mbar_init(&bar_sfree[i], 8);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int* abort = &abort_sh;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      mbar_arrive_expect_tx(&bar_q, SL::kQBytes);
+      for (int h = 0; h < ND; ++h) tma_load_3d(dsm + SL::kQOff + h * 16384, &tm_q, h * 64, m0, bh, &bar_q);
+      int issued[2] = {-1, -1};
+      for (int it = 0; it < 2 * nchunk; ++it) {
+        const int st = it & 1, c = it % nchunk;
+        if (!mbar_wait(&bar_kempty[st], ((it >> 1) & 1) ^ 1, abort, ctx)) break;
+        mbar_arrive_expect_tx(&bar_kfull[st], SL::kKBytes);
+        for (int h = 0; h < ND; ++h)
+          tma_load_3d(dsm + SL::kKOff + st * SL::kKBytes + h * 32768, &tm_k, h * 64, c * RS_N, bh, &bar_kfull[st]);
+        issued[st] = it;
+      }
+      if (*abort) {  // drain the copies still in flight before the CTA exits
+        mbar_wait_drain(&bar_q, 0, ctx.timeout_ns);
+        for (int st = 0; st < 2; ++st)
+          if (issued[st] >= 0) mbar_wait_drain(&bar_kfull[st], (issued[st] >> 1) & 1, ctx.timeout_ns);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(RS_M, RS_N, false, false);
+      const uint32_t qa = smem_u32(dsm + SL::kQOff);
+      bool ok = mbar_wait(&bar_q, 0, abort, ctx);
+      for (int it = 0; ok && it < 2 * nchunk; ++it) {
+        const int st = it & 1;
+        if (!mbar_wait(&bar_kfull[st], (it >> 1) & 1, abort, ctx)) break;
+        if (!mbar_wait(&bar_sfree[st], ((it >> 1) & 1) ^ 1, abort, ctx)) break;
+        tc_fence_after();
+        const uint32_t ka = smem_u32(dsm + SL::kKOff + st * SL::kKBytes);
+#pragma unroll
+        for (int kk = 0; kk < 4 * ND; ++kk) {
+          const uint32_t h = kk >> 2, sub = (kk & 3) * 32;
+          mma_bf16_ss(tmem + st * RS_N, sdesc_sw128(qa + h * 16384 + sub, 16, 1024),
+                      sdesc_sw128(ka + h * 32768 + sub, 16, 1024), idesc, kk > 0);
+        }
+        mma_commit(&bar_kempty[st]);
+        mma_commit(&bar_sfull[st]);
+      }
+      // every MMA issued above has finished once this barrier completes (also on abort)
+      mma_commit(&bar_done);
+      mbar_wait_drain(&bar_done, 0, ctx.timeout_ns);
+    }
+  } else {
+    // epilogue warps
+    const int ew = warp - 2;
+    const int quarter = warp & 3;
+    const int half = ew >> 2;
+    const int row = 32 * quarter + lane;
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    float m = -INFINITY, l = 0.f;
+    for (int it = 0; it < nchunk; ++it) {
+      const int st = it & 1;
+      if (!mbar_wait(&bar_sfull[st], (it >> 1) & 1, abort, ctx)) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int piece = 0; piece < 4; ++piece) {
+        const int col0 = half * 128 + piece * 32;
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + st * RS_N + col0, r);
+        tmem_ld_wait();
+        const int key0 = it * RS_N + col0;
+        float x[32];
+        float pm = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          x[j] = (key0 + j < Lr) ? __uint_as_float(r[j]) * c2 : -INFINITY;
+          pm = fmaxf(pm, x[j]);
+        }
+        const float mn = fmaxf(m, pm);
+        if (mn == -INFINITY) continue;
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) s += ex2(x[j] - mn);
+        l = l * ex2(m - mn) + s;
+        m = mn;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_sfree[st]);
+    }
+    m_half[half][row] = m;
+    l_half[half][row] = l;
+    named_bar_sync(1, 256);
+    if (half == 0) {
+      const float m1 = m_half[0][row], m2 = m_half[1][row];
+      const float mm = fmaxf(m1, m2);
+      const float ll = l_half[0][row] * ex2(m1 - mm) + l_half[1][row] * ex2(m2 - mm);
+      lse_sh[row] = mm + __log2f(ll);
+    }
+    named_bar_sync(1, 256);
+    const float lse2 = lse_sh[row];
+    const int qtile = (m0 + row) >> 2;  // G = 4 pooled rows per tile
+    const bool row_ok = qtile < N;
+    float* out_row = scores + ((size_t)bh * N + (row_ok ? qtile : 0)) * N;
+    for (int it = nchunk; it < 2 * nchunk; ++it) {
+      const int st = it & 1, c = it - nchunk;
+      if (!mbar_wait(&bar_sfull[st], (it >> 1) & 1, abort, ctx)) break;
+      tc_fence_after();
+      float t[32];
+#pragma unroll
+      for (int piece = 0; piece < 4; ++piece) {
+        const int col0 = half * 128 + piece * 32;
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + st * RS_N + col0, r);
+        tmem_ld_wait();
+        const int key0 = c * RS_N + col0;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          float acc = 0.f;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 4 * jj + e;
+            acc += (key0 + j < Lr) ? ex2(__uint_as_float(r[j]) * c2 - lse2) : 0.f;
+          }
+          t[piece * 8 + jj] = acc;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_sfree[st]);
+      // sum over the G = 4 query sub-rows (lanes 4g..4g+3), reduce-scatter: lane keeps 8 tiles
+      float u[16];
+      const bool hi2 = lane & 2;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float send = hi2 ? t[j] : t[16 + j];
+        const float keep = hi2 ? t[16 + j] : t[j];
+        u[j] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+      }
+      float w[8];
+      const bool hi1 = lane & 1;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float send = hi1 ? u[j] : u[8 + j];
+        const float keep = hi1 ? u[8 + j] : u[j];
+        w[j] = (keep + __shfl_xor_sync(0xffffffffu, send, 1)) * (1.f / kG);
+      }
+      const int j0 = (c * RS_N + half * 128) / 4 + (hi2 ? 16 : 0) + (hi1 ? 8 : 0);
+      if (row_ok) {
+        if (j0 + 8 <= N) {
+          float4* dst = reinterpret_cast<float4*>(out_row + j0);
+          if ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+            dst[0] = make_float4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_float4(w[4], w[5], w[6], w[7]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) out_row[j0 + j] = w[j];
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (j0 + j < N) out_row[j0 + j] = w[j];
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// CUDA-core router scores for fp32 inputs (and head_dim 64): CTA = one query tile of one
+// (b, h). Step 1: LSE of its G pooled query rows over all pooled keys. Step 2: one thread per
+// key tile sums exp(s - lse) over the G x G pooled pairs.
+// ------------------------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(128) router_scores_simt_kernel(const T* __restrict__ qr, const T* __restrict__ kr,
+                                                                 float* __restrict__ scores, int Lr, int N) {
+  __shared__ float qs[kG][D];
+  __shared__ float red_m[kG][128], red_l[kG][128];
+  __shared__ float lse_s[kG];
+  const int i = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+  const T* qb = qr + ((size_t)bh * Lr + (size_t)i * kG) * D;
+  const T* kb = kr + (size_t)bh * Lr * D;
+  for (int e = t; e < kG * D; e += 128) qs[e / D][e % D] = (float)qb[e];
+  __syncthreads();
+  const float scale = rsqrtf((float)D);
+  float m[kG], l[kG];
+#pragma unroll
+  for (int a = 0; a < kG; ++a) m[a] = -INFINITY, l[a] = 0.f;
+  for (int b = t; b < Lr; b += 128) {
+    float s[kG] = {};
+    for (int d = 0; d < D; ++d) {
+      const float kv = (float)kb[(size_t)b * D + d];
+#pragma unroll
+      for (int a = 0; a < kG; ++a) s[a] += qs[a][d] * kv;
+    }
+#pragma unroll
+    for (int a = 0; a < kG; ++a) {
+      const float x = s[a] * scale;
+      const float mn = fmaxf(m[a], x);
+      l[a] = l[a] * __expf(m[a] - mn) + __expf(x - mn);
+      m[a] = mn;
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < kG; ++a) red_m[a][t] = m[a], red_l[a][t] = l[a];
+  __syncthreads();
+  if (t < kG) {
+    float mm = -INFINITY;
+    for (int u = 0; u < 128; ++u) mm = fmaxf(mm, red_m[t][u]);
+    float ll = 0.f;
+    for (int u = 0; u < 128; ++u)
+      if (red_m[t][u] != -INFINITY) ll += red_l[t][u] * __expf(red_m[t][u] - mm);
+    lse_s[t] = mm + __logf(ll);
+  }
+  __syncthreads();
+  for (int j = t; j < N; j += 128) {
+    float acc = 0.f;
+    for (int b = kG * j; b < kG * j + kG; ++b) {
+      float s[kG] = {};
+      for (int d = 0; d < D; ++d) {
+        const float kv = (float)kb[(size_t)b * D + d];
+#pragma unroll
+        for (int a = 0; a < kG; ++a) s[a] += qs[a][d] * kv;
+      }
+#pragma unroll
+      for (int a = 0; a < kG; ++a) acc += __expf(s[a] * scale - lse_s[a]);
+    }
+    scores[((size_t)bh * N + i) * N + j] = acc * (1.f / kG);
+  }
+}
+
+}  // namespace
+
+vsa2_status launch_router(const Dims& d, const void* q, const void* k, float* scores, char* ws, cudaStream_t s) {
+  const WsLayout w = ws_layout(d);
+  void* qr = ws + w.qr;
+  void* kr = ws + w.kr;
+  DevCtx ctx{reinterpret_cast<int*>(ws), d.timeout_ns, d.flags};
+  const int64_t pooled = (int64_t)d.BH * d.Lr;
+  const int cpr = d.D * d.esize / 16;
+  const int64_t threads = 2 * pooled * cpr;
+  const unsigned blocks = (unsigned)((threads + 255) / 256);
+  if (d.dtype == VSA2_BF16) {
+    router_pool_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                                                             (__nv_bfloat16*)qr, (__nv_bfloat16*)kr, pooled, cpr);
+  } else {
+    router_pool_kernel<float><<<blocks, 256, 0, s>>>((const float*)q, (const float*)k, (float*)qr, (float*)kr,
+                                                     pooled, cpr);
+  }
+  if (cudaGetLastError() != cudaSuccess) return VSA2_ERR_CUDA;
+
+  if (d.dtype == VSA2_BF16) {
+    CUtensorMap tq, tk;
+    if (!make_tmap_3d_bf16(&tq, qr, d.D, d.Lr, d.BH, 64, RS_M)) return VSA2_ERR_CUDA;
+    if (!make_tmap_3d_bf16(&tk, kr, d.D, d.Lr, d.BH, 64, RS_N)) return VSA2_ERR_CUDA;
+    const float c2 = 1.4426950408889634f / sqrtf((float)d.D);
+    dim3 grid((d.Lr + RS_M - 1) / RS_M, d.BH);
+    if (d.D == 128) {
+      auto kern = router_scores_tc_kernel<2>;
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, RouterSmem<2>::kDyn);
+      kern<<<grid, RS_THREADS, RouterSmem<2>::kDyn, s>>>(tq, tk, scores, d.Lr, d.N, c2, ctx);
+    } else {
+      auto kern = router_scores_tc_kernel<1>;
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, RouterSmem<1>::kDyn);
+      kern<<<grid, RS_THREADS, RouterSmem<1>::kDyn, s>>>(tq, tk, scores, d.Lr, d.N, c2, ctx);
+    }
+  } else {
+    dim3 grid(d.N, d.BH);
+    if (d.D == 128)
+      router_scores_simt_kernel<float, 128><<<grid, 128, 0, s>>>((const float*)qr, (const float*)kr, scores, d.Lr, d.N);
+    else
+      router_scores_simt_kernel<float, 64><<<grid, 128, 0, s>>>((const float*)qr, (const float*)kr, scores, d.Lr, d.N);
+  }
+  if (cudaGetLastError() != cudaSuccess) return VSA2_ERR_CUDA;
+  return VSA2_OK;
+}
+
+}  // namespace vsa2
