@@ -1,0 +1,336 @@
+"""Benchmark of the VSA2 hot path on B200: router -> per-sequence TopK -> block-sparse attention.
+
+One step = one pass of the whole path over one batch of synthetic input of the 720p workload
+(B=1, H=20, D=128, grid 56x48x80 = 215,040 tokens, 3360 tiles, top64, bf16): router pooling,
+router scores, TopK, attention forward. With --workload 480p_train_top64 the step also runs the
+backward pass (training step of the fine branch; the router gets no gradient).
+
+Prints one JSON line (rank 0). `value` is the effective TFLOPS of the whole step: FLOPs of the
+selected tile pairs only (4*64*64*D per pair forward, 2.5x that backward) over the step time,
+summed over ranks, divided by the max step time over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic as S  # noqa: E402
+
+METRIC = "VSA2 attn fwd ms & effective TFLOPS, 215K tok H20 D128 top64"
+DEFAULT_WORKLOAD = "720p_top64"
+# kernels of ours launched per call (memsets are not counted)
+LAUNCHES = {"router": 2, "topk": 9, "topk_csc": 11, "fwd": 1, "bwd": 3}
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained", p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def pair_flops(wl, pairs, backward):
+    f = 4.0 * 64 * 64 * wl.head_dim * pairs
+    return f * (3.5 if backward else 1.0)
+
+
+class Clocks:
+    """nvidia-smi sampler running during the timed region."""
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.device_index = device_index
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.device_index),
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+                self.lines = [l for l in out.splitlines() if l.strip()]
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            try:
+                sm.append(float(f[0]))
+                mx = max(mx, float(f[1]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------------------------
+# reference arm and CPU baseline: the fp64 oracle on a bounded sample
+# ----------------------------------------------------------------------------------------------
+def oracle_sample(wl, budget_s=20.0, tiles=None):
+    """Time the oracle's hot path on head 0 of batch 0: router + TopK on the whole head, the
+    forward (and backward) on a sample of query tiles; extrapolate to all tiles and heads."""
+    from oracle import vsa2_oracle as O
+
+    q, k, v = (S.make_slice(wl, n, 0, 0) for n in ("q", "k", "v"))
+    t0 = time.perf_counter()
+    sc = O.router_scores(q, k).astype(np.float32)
+    t1 = time.perf_counter()
+    sel = O.topk_select(sc, wl.topk)
+    t2 = time.perf_counter()
+    N = wl.num_tiles
+    rng = np.random.default_rng(0)
+    order = rng.permutation(N)
+    done, t_att = 0, 0.0
+    for i in order:
+        ts = time.perf_counter()
+        O.sparse_attn_fwd(q, k, v, sel["kv_off"], sel["kv_idx"], query_tiles=[int(i)])
+        t_att += time.perf_counter() - ts
+        done += 1
+        if tiles is not None and done >= tiles:
+            break
+        if tiles is None and (t2 - t0) + t_att > budget_s:
+            break
+    per_head = (t1 - t0) + (t2 - t1) + t_att * N / done
+    if wl.backward:
+        per_head += 2.5 * t_att * N / done  # backward restated as 2.5x the forward GEMM work
+    total_s = per_head * wl.heads * wl.batch
+    pairs = wl.batch * wl.heads * N * wl.topk
+    flops = pair_flops(wl, pairs, wl.backward)
+    return {"seconds_per_step": total_s, "tflops": flops / total_s / 1e12, "router_s": t1 - t0, "topk_s": t2 - t1,
+            "fwd_tiles_sampled": done, "tiles": N,
+            "sample": f"head 0 of {wl.heads}: router+TopK whole head, forward on {done}/{N} query tiles; "
+                      f"extrapolated to {wl.heads} heads"}
+
+
+def cores():
+    return len(os.sched_getaffinity(0))
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    steps = []
+    for _ in range(args.warmup):
+        oracle_sample(wl, tiles=2)
+    for _ in range(args.steps):
+        steps.append(oracle_sample(wl, tiles=8))
+    sec = statistics.mean(s["seconds_per_step"] for s in steps)
+    pairs = wl.batch * wl.heads * wl.num_tiles * wl.topk
+    val = pair_flops(wl, pairs, wl.backward) / sec / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOPS", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "heads": wl.heads, "head_dim": wl.head_dim,
+                       "grid": list(wl.grid), "tokens": wl.tokens, "topk": wl.topk},
+            "cpu_baseline": {"value": val, "unit": "TFLOPS", "cores": cores(), "kind": "oracle",
+                             "sample": steps[-1]["sample"]},
+            "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------------------------
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    import trainable_block_sparse_fine_b200 as V
+
+    dev = torch.device("cuda", local)
+    # weak scaling: every rank runs the full workload on its own batch element (seed offset)
+    wl_r = wl.with_(seed=wl.seed + rank)
+    names = ("q", "k", "v", "do") if wl.backward else ("q", "k", "v")
+    host = {n: S.make_tensor(wl_r, n) for n in names}
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    pinned = {n: torch.from_numpy(host[n]).to(dt).pin_memory() for n in names}
+    x = {n: pinned[n].to(dev) for n in names}
+    e = V.VSA2(wl.batch, wl.heads, wl.head_dim, wl.grid, wl.dtype, wl.topk)
+    stream = torch.cuda.current_stream()
+    l2_flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    scores = torch.empty(wl.batch, wl.heads, wl.num_tiles, wl.num_tiles, dtype=torch.float32, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def step(timers=None):
+        t = timers or {}
+        if t: t["r0"].record(stream)
+        e.router_scores(x["q"], x["k"], out=scores)
+        if t: t["r1"].record(stream)
+        sel = e.topk_select(scores, wl.topk, csc=wl.backward)
+        if t: t["t1"].record(stream)
+        o, lse = e.attn_fwd(x["q"], x["k"], x["v"], sel[0], sel[1])
+        if t: t["f1"].record(stream)
+        if wl.backward:
+            grads = e.attn_bwd(x["q"], x["k"], x["v"], o, lse, x["do"], *sel)
+            if t: t["b1"].record(stream)
+            return o, grads
+        return o, None
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    err = e.device_error()
+    if err != 0:
+        raise RuntimeError(f"device error {V.vsa2_status_string(err)} during warm-up")
+
+    keys = ["r0", "r1", "t1", "f1"] + (["b1"] if wl.backward else [])
+    per = {k: [] for k in ("router", "topk", "fwd", "bwd", "step")}
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with Clocks(local) as clk:
+        for _ in range(args.steps):
+            l2_flush.zero_()  # L2 flush between timed steps (outside the timed events)
+            timers = {k: ev() for k in keys}
+            step(timers)
+            torch.cuda.synchronize()
+            per["router"].append(timers["r0"].elapsed_time(timers["r1"]))
+            per["topk"].append(timers["r1"].elapsed_time(timers["t1"]))
+            per["fwd"].append(timers["t1"].elapsed_time(timers["f1"]))
+            if wl.backward:
+                per["bwd"].append(timers["f1"].elapsed_time(timers["b1"]))
+            per["step"].append(timers["r0"].elapsed_time(timers[keys[-1]]))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_local = statistics.mean(per["step"])
+    ms = ms_local
+    if world > 1:
+        t = torch.tensor([ms_local], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    err = e.device_error()
+    if err != 0:
+        raise RuntimeError(f"device error {V.vsa2_status_string(err)} in the timed region")
+
+    pairs = wl.batch * wl.heads * wl.num_tiles * wl.topk
+    flops_rank = pair_flops(wl, pairs, wl.backward)
+    value = flops_rank * world / (ms * 1e-3) / 1e12
+
+    # end to end through the public API: H2D of the step's inputs, the step, D2H of its output
+    h2d = sum(pinned[n].numel() * pinned[n].element_size() for n in names)
+    out_host = torch.empty(x["q"].shape, dtype=dt, pin_memory=True)
+    d2h = out_host.numel() * out_host.element_size()
+    e2e_ms = []
+    for it in range(args.warmup + args.steps):
+        l2_flush.zero_()
+        a, b = ev(), ev()
+        a.record(stream)
+        xs = {n: pinned[n].to(dev, non_blocking=True) for n in names}
+        o = e.forward(xs["q"], xs["k"], xs["v"], wl.topk, csc=wl.backward)
+        if wl.backward:
+            e.attn_bwd(xs["q"], xs["k"], xs["v"], o[0], o[1], xs["do"], *o[2])
+        out_host.copy_(o[0], non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e_local = statistics.mean(e2e_ms)
+    e2e = e2e_local
+    if world > 1:
+        t = torch.tensor([e2e_local], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e = float(t.item())
+
+    hbm, bf16_burst, bf16_sus, peak_kind = load_peaks()
+    fwd_ms = statistics.mean(per["fwd"])
+    fwd_tflops = pair_flops(wl, pairs, False) / (fwd_ms * 1e-3) / 1e12
+    router_ms = statistics.mean(per["router"])
+    router_bytes = 2 * wl.batch * wl.heads * wl.tokens * wl.head_dim * (2 if wl.dtype == "bf16" else 4) \
+        + wl.batch * wl.heads * wl.num_tiles ** 2 * 4
+    launches = LAUNCHES["router"] + (LAUNCHES["topk_csc"] if wl.backward else LAUNCHES["topk"]) + LAUNCHES["fwd"] \
+        + (LAUNCHES["bwd"] if wl.backward else 0)
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            c = oracle_sample(wl, budget_s=20.0)
+            cpu = {"value": c["tflops"], "unit": "TFLOPS", "cores": cores(), "kind": "oracle", "sample": c["sample"],
+                   "seconds_per_step": c["seconds_per_step"]}
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "fp32", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "heads": wl.heads, "head_dim": wl.head_dim,
+                       "grid": list(wl.grid), "tokens": wl.tokens, "tiles": wl.num_tiles, "topk": wl.topk,
+                       "selected_pairs_per_rank": pairs, "backward": wl.backward,
+                       "l2": "256 MB buffer written between timed steps; inputs also exceed L2"},
+            "stages_ms": {"router": router_ms, "topk": statistics.mean(per["topk"]), "fwd": fwd_ms,
+                          **({"bwd": statistics.mean(per["bwd"])} if wl.backward else {})},
+            "fwd_kernel": {"ms": fwd_ms, "effective_tflops": fwd_tflops},
+            "router": {"ms": router_ms, "algorithmic_bytes": router_bytes,
+                       "gbs": router_bytes / (router_ms * 1e-3) / 1e9, "hbm_frac": router_bytes / (router_ms * 1e-3) / 1e9 / hbm},
+            "roofline": {"bound": "tensor", "kernel": "attn_fwd_tc_kernel", "achieved": fwd_tflops,
+                         "peak": bf16_sus, "unit": "TFLOP/s", "frac": fwd_tflops / bf16_sus,
+                         "peak_kind": f"{peak_kind} sustained bf16", "traffic": None},
+            "cpu_baseline": cpu,
+            "e2e": {"value": flops_rank * world / (e2e * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches * args.steps,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(S.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = S.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

@@ -151,6 +151,10 @@ vsa2_status vsa2_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t timeo
 /* Human-readable name of a status code (static storage). */
 const char* vsa2_status_string(vsa2_status s);
 
+/* Message of the last failed CUDA call or launch inside the library (static or per-thread
+ * storage; valid until the next failure on the same thread). */
+const char* vsa2_last_cuda_error(void);
+
 /* Library version, major*10000 + minor*100 + patch. */
 int32_t vsa2_version(void);
 

@@ -19,7 +19,7 @@ VSA2_FLAG_VALIDATE = 1
 # every symbol the header declares
 EXPORTS = ("vsa2_workspace_size", "vsa2_workspace_init", "vsa2_router_scores", "vsa2_topk_select",
            "vsa2_sparse_attn_fwd", "vsa2_sparse_attn_bwd", "vsa2_get_device_error",
-           "vsa2_selftest_wait_timeout", "vsa2_status_string", "vsa2_version")
+           "vsa2_selftest_wait_timeout", "vsa2_status_string", "vsa2_version", "vsa2_last_cuda_error")
 
 
 class Vsa2Error(RuntimeError):
@@ -61,6 +61,7 @@ def lib() -> ctypes.CDLL:
         L.vsa2_status_string.argtypes = [ctypes.c_int]
         L.vsa2_status_string.restype = ctypes.c_char_p
         L.vsa2_version.restype = i32
+        L.vsa2_last_cuda_error.restype = ctypes.c_char_p
         for name in ("vsa2_workspace_init", "vsa2_router_scores", "vsa2_topk_select", "vsa2_sparse_attn_fwd",
                      "vsa2_sparse_attn_bwd", "vsa2_get_device_error", "vsa2_selftest_wait_timeout"):
             getattr(L, name).restype = ctypes.c_int
@@ -88,6 +89,8 @@ def _stream(stream) -> int | None:
 
 def _check(status: int, where: str) -> None:
     if status != VSA2_OK:
+        if status == 3:
+            where = f"{where} ({lib().vsa2_last_cuda_error().decode()})"
         raise Vsa2Error(status, where)
 
 

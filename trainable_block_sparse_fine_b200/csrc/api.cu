@@ -1,6 +1,8 @@
 // C ABI of libvsa2: argument validation, workspace layout and dispatch to the kernels.
 #include <cudaTypedefs.h>
 
+#include <atomic>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -89,6 +91,36 @@ bool make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                       uint32_t box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static std::atomic<const char*> g_last_cuda_error{"no CUDA error recorded"};
+static thread_local char g_msg[256];
+
+vsa2_status cuda_fail(const char* what) {
+  g_last_cuda_error.store(what);
+  return VSA2_ERR_CUDA;
+}
+
+vsa2_status check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return VSA2_OK;
+  snprintf(g_msg, sizeof(g_msg), "%s: %s", what, cudaGetErrorString(e));
+  g_last_cuda_error.store(g_msg);
+  return VSA2_ERR_CUDA;
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -207,5 +239,7 @@ const char* vsa2_status_string(vsa2_status s) {
 }
 
 int32_t vsa2_version(void) { return 100; }
+
+const char* vsa2_last_cuda_error(void) { return g_last_cuda_error.load(); }
 
 }  // extern "C"

@@ -268,7 +268,7 @@ vsa2_status fwd_simt(const Dims& d, const void* q, const void* k, const void* v,
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   kern<<<dim3(d.N, d.BH), 64, smem, s>>>((const T*)q, (const T*)k, (const T*)v, kv_off, kv_idx, (T*)o, lse, d.N,
                                          d.L, topk, ctx);
-  return cudaGetLastError() == cudaSuccess ? VSA2_OK : VSA2_ERR_CUDA;
+  return check_launch(__func__);
 }
 
 template <typename T, int D>
@@ -288,7 +288,7 @@ vsa2_status bwd_simt(const Dims& d, const void* q, const void* k, const void* v,
   cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_kv);
   kk<<<dim3(d.N, d.BH), 128, smem_kv, s>>>((const T*)q, (const T*)k, (const T*)v, (const T*)dout, lse, delta, q_off,
                                            q_idx, dk, dv, d.N, d.L, topk, ctx);
-  return cudaGetLastError() == cudaSuccess ? VSA2_OK : VSA2_ERR_CUDA;
+  return check_launch(__func__);
 }
 
 }  // namespace

@@ -21,7 +21,7 @@ __global__ void wait_timeout_probe_kernel(int* err, uint64_t timeout_ns) {
 
 vsa2_status launch_wait_timeout_probe(int* err, uint64_t timeout_ns, cudaStream_t s) {
   wait_timeout_probe_kernel<<<1, 32, 0, s>>>(err, timeout_ns);
-  return cudaGetLastError() == cudaSuccess ? VSA2_OK : VSA2_ERR_CUDA;
+  return check_launch(__func__);
 }
 
 vsa2_status launch_attn_fwd(const Dims& d, const void* q, const void* k, const void* v, int topk,

@@ -75,4 +75,9 @@ vsa2_status launch_wait_timeout_probe(int* err, uint64_t timeout_ns, cudaStream_
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Records the message of a failed CUDA call (see vsa2_last_cuda_error) and returns VSA2_ERR_CUDA.
+vsa2_status cuda_fail(const char* what);
+// VSA2_OK if the last launch succeeded, else records the CUDA error and returns VSA2_ERR_CUDA.
+vsa2_status check_launch(const char* what);
+
 }  // namespace vsa2

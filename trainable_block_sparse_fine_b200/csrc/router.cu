@@ -374,12 +374,12 @@ vsa2_status launch_router(const Dims& d, const void* q, const void* k, float* sc
     router_pool_kernel<float><<<blocks, 256, 0, s>>>((const float*)q, (const float*)k, (float*)qr, (float*)kr,
                                                      pooled, cpr);
   }
-  if (cudaGetLastError() != cudaSuccess) return VSA2_ERR_CUDA;
+  if (check_launch(__func__) != VSA2_OK) return VSA2_ERR_CUDA;
 
   if (d.dtype == VSA2_BF16) {
     CUtensorMap tq, tk;
-    if (!make_tmap_3d_bf16(&tq, qr, d.D, d.Lr, d.BH, 64, RS_M)) return VSA2_ERR_CUDA;
-    if (!make_tmap_3d_bf16(&tk, kr, d.D, d.Lr, d.BH, 64, RS_N)) return VSA2_ERR_CUDA;
+    if (!make_tmap_3d_bf16(&tq, qr, d.D, d.Lr, d.BH, 64, RS_M)) return cuda_fail("tensor map encoding (Qr) failed");
+    if (!make_tmap_3d_bf16(&tk, kr, d.D, d.Lr, d.BH, 64, RS_N)) return cuda_fail("tensor map encoding (Kr) failed");
     const float c2 = 1.4426950408889634f / sqrtf((float)d.D);
     dim3 grid((d.Lr + RS_M - 1) / RS_M, d.BH);
     if (d.D == 128) {
@@ -398,7 +398,7 @@ vsa2_status launch_router(const Dims& d, const void* q, const void* k, float* sc
     else
       router_scores_simt_kernel<float, 64><<<grid, 128, 0, s>>>((const float*)qr, (const float*)kr, scores, d.Lr, d.N);
   }
-  if (cudaGetLastError() != cudaSuccess) return VSA2_ERR_CUDA;
+  if (check_launch(__func__) != VSA2_OK) return VSA2_ERR_CUDA;
   return VSA2_OK;
 }
 

@@ -306,7 +306,7 @@ vsa2_status launch_topk(const Dims& d, const float* scores, int topk, int32_t* k
     topk_csc_offsets_kernel<<<d.BH, 1024, 0, s>>>(d.N, col_cnt, q_off);
     topk_csc_emit_kernel<<<rgrid, 256, 0, s>>>(d.N, topk, col_bits, w.words, q_off, q_idx);
   }
-  if (cudaGetLastError() != cudaSuccess) return VSA2_ERR_CUDA;
+  if (check_launch(__func__) != VSA2_OK) return VSA2_ERR_CUDA;
   return VSA2_OK;
 }
 
