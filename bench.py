@@ -254,7 +254,7 @@ def run_ours(args, wl):
     out_host = torch.empty(x["q"].shape, dtype=dt, pin_memory=True)
     d2h = out_host.numel() * out_host.element_size()
     e2e_ms = []
-    for it in range(args.warmup + args.steps):
+    for it in range(0 if args.no_e2e else args.warmup + args.steps):
         l2_flush.zero_()
         a, b = ev(), ev()
         a.record(stream)
@@ -267,7 +267,7 @@ def run_ours(args, wl):
         torch.cuda.synchronize()
         if it >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
-    e2e_local = statistics.mean(e2e_ms)
+    e2e_local = statistics.mean(e2e_ms) if e2e_ms else float("nan")
     e2e = e2e_local
     if world > 1:
         t = torch.tensor([e2e_local], device=dev)
@@ -324,8 +324,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(S.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
+    ap.add_argument("--heads", type=int, default=None, help="override the head count (profiling runs)")
     args = ap.parse_args()
     wl = S.WORKLOADS[args.workload]
+    if args.heads:
+        wl = wl.with_(heads=args.heads)
     if args.impl == "reference":
         run_reference(args, wl)
     else:
