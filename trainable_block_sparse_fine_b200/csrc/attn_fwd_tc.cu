@@ -3,19 +3,20 @@
 // with the attention definition of its §2.1: per query tile, softmax over the tokens of the
 // KV tiles its router selected.
 //
-// Shape choice for sm_100a: a query tile has only 64 rows, and tcgen05 runs M=64 at half
-// rate, so both GEMMs are issued transposed with M=128:
-//   S^T[128 kv, 64 q]  = [K_j1; K_j2] . Q_i^T     (two selected KV tiles per block)
-//   O^T[128 d, 64 q]  += [V_j1; V_j2]^T . P^T      (V^T read MN-major straight from the TMA tile)
-// The softmax runs down the columns of S^T: each thread owns one KV row; the running max per
-// query column lives in shared memory and is only raised (with an O^T rescale) when a new score
-// exceeds it by more than 2^8, so the common block needs a single warpgroup barrier.
+// Design for sm_100a. Gathered K/V tiles reach shared memory through TMA and are read once by
+// the tensor core, so shared-memory bandwidth (128 B/clk/SM, shared by TMA writes and MMA
+// operand reads) is the binding resource. Both GEMMs therefore take their A operand from
+// tensor memory and only their B operand from shared memory:
+//   S  [64 q, 128 kv] = Q  . [K_j1; K_j2]^T   A = Q (TMEM, written once per tile), B = K (K-major)
+//   O  [64 q, 128 d] += P  . [V_j1; V_j2]     A = P (TMEM, written by the softmax), B = V (MN-major)
+// M=64 tiles occupy half of the TMEM lanes (lanes 0-15 of each 32-lane quarter), so two query
+// tiles ("slots") share the same TMEM columns: slot 0 at lane offset 0, slot 1 at offset 16.
 //
-// CTA (persistent, one query tile at a time): warps 0-3 and 4-7 are two softmax warpgroups that
-// split the 64 query columns (32 each); warp 8 loads Q and K, warp 10 loads V (two TMA issuing
-// threads keep more copies in flight than one), warp 9 issues the MMAs.
-// Double buffers: Q (per tile), S^T and P^T (per block), O^T (per tile, so the epilogue of one
-// tile overlaps the first MMAs of the next). K and V rings of two blocks each.
+// CTA (persistent): warps 0-3 run the softmax of slot 0, warps 4-7 of slot 1. A warp owns 16
+// rows of its slot; the 16x64b TMEM access gives each row to a pair of threads (even / odd
+// columns), so row max and row sum need one shuffle and no block-level barrier. Warp 8 loads K,
+// warp 10 loads V, warp 9 issues the MMAs. The running max is raised (with an O rescale in
+// TMEM) only when a row's new maximum exceeds it by more than 2^8.
 #include <algorithm>
 
 #include "common.cuh"
@@ -26,40 +27,38 @@ namespace {
 
 constexpr int FT = 352;            // 11 warps
 constexpr uint32_t TILE_B = 8192;  // one 64x64 bf16 box (64 rows x 128 B)
-constexpr uint32_t Q_B = 16384;    // Q tile: 2 column halves of 64 rows
 constexpr uint32_t BLK_B = 32768;  // K or V block: [half0: tile A, tile B][half1: tile A, tile B]
-constexpr uint32_t PT_B = 16384;   // P^T: 128 kv rows x 64 q (bf16), MN-major 128B swizzle
-constexpr uint32_t ST_B = 8192;    // output staging per warpgroup: 32 rows x 128 bf16
+constexpr int KST = 4;             // K ring stages
+constexpr int VST = 3;             // V ring stages
 
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K = OFF_Q + 2 * Q_B;
-constexpr uint32_t OFF_V = OFF_K + 2 * BLK_B;
-constexpr uint32_t OFF_P = OFF_V + 2 * BLK_B;
-constexpr uint32_t OFF_ST = OFF_P + 2 * PT_B;
-constexpr uint32_t OFF_BAR = OFF_ST + 2 * ST_B;
-constexpr uint32_t OFF_M = OFF_BAR + 256;                 // [2 wg][32] running max (log2 units)
-constexpr uint32_t OFF_RED = OFF_M + 2 * 32 * 4;          // [2 wg][4 warps][32]
-constexpr uint32_t OFF_ALPHA = OFF_RED + 2 * 4 * 32 * 4;  // [2 wg][32]
-constexpr uint32_t OFF_FLAG = OFF_ALPHA + 2 * 32 * 4;
+constexpr uint32_t OFF_K = 0;
+constexpr uint32_t OFF_V = OFF_K + KST * BLK_B;
+constexpr uint32_t OFF_BAR = OFF_V + VST * BLK_B;
+constexpr uint32_t OFF_FLAG = OFF_BAR + 512;
 constexpr uint32_t SMEM_USED = OFF_FLAG + 64;
 constexpr uint32_t SMEM_DYN = SMEM_USED + 1024;
 static_assert(SMEM_DYN <= 232448, "shared memory budget");
 
-constexpr uint32_t TM_COLS = 256;  // S^T at columns 0 / 64, O^T at 128 / 192
-constexpr float kThresh = 8.0f;    // log2 headroom before the running max must move
+// TMEM columns (each region used by both slots through the lane halves)
+constexpr uint32_t TM_S = 0;      // two S buffers of 128 fp32 columns
+constexpr uint32_t TM_P = 256;    // P: 128 bf16 = 64 columns
+constexpr uint32_t TM_Q = 320;    // Q: 128 bf16 = 64 columns
+constexpr uint32_t TM_O = 384;    // O: 128 fp32 columns
+constexpr uint32_t TM_COLS = 512;
+constexpr float kThresh = 8.0f;   // log2 headroom before the running max must move
 
 struct Bars {
-  uint64_t kfull[2], kempty[2], vfull[2], vempty[2];
-  uint64_t qfull[2], qempty[2];
-  uint64_t sfull[2], sfree[2], pfull[2], odone[2], ofree[2];
+  uint64_t kfull[KST], kempty[KST], vfull[VST], vempty[VST];
+  uint64_t sfull[2][2], sfree[2][2];  // [slot][buffer]
+  uint64_t pfull[2], pvdone[2], qready[2];
   uint64_t done;
 };
-static_assert(sizeof(Bars) <= 256, "barrier area");
+static_assert(sizeof(Bars) <= 512, "barrier area");
 
-// Sanitised CSR row of query tile i of head bh; every role reads it the same way.
 struct Row {
   int beg, len;
 };
+// Sanitised CSR row of query tile i of head bh; every role reads it the same way.
 __device__ __forceinline__ Row load_row(const int32_t* kv_off, int bh, int i, int N, int cap, const DevCtx& ctx,
                                         bool report) {
   int b = kv_off[(size_t)bh * (N + 1) + i];
@@ -71,33 +70,58 @@ __device__ __forceinline__ Row load_row(const int32_t* kv_off, int bh, int i, in
   return Row{b, e - b};
 }
 
-__device__ __forceinline__ uint32_t u32(float f) { return __float_as_uint(f); }
-
-// 32-column reduce-scatter across a warp: afterwards lane l holds column l.
-template <bool MAX>
-__device__ __forceinline__ float warp_rs32(float (&v)[32], const int lane) {
-#pragma unroll
-  for (int step = 0; step < 5; ++step) {
-    const int half = 16 >> step;
-    const int mask = 16 >> step;
-    const bool hi = lane & mask;
-#pragma unroll
-    for (int j = 0; j < half; ++j) {
-      const float send = hi ? v[j] : v[half + j];
-      const float keep = hi ? v[half + j] : v[j];
-      const float recv = __shfl_xor_sync(0xffffffffu, send, mask);
-      v[j] = MAX ? fmaxf(keep, recv) : keep + recv;
-    }
+// Per-slot op stream of a CTA: items (b*h, query tile) in head-major order, slot s of CTA c takes
+// items r*2G + 2c + s. For a tile of n blocks the ops are S0, S1, O0, S2, O1, ..., O(n-1).
+// The MMA issuer and both producers walk the same merged stream (slot 0 op, slot 1 op, ...).
+struct SlotSeq {
+  int item, stride, items;
+  int bh, qt, nblk, len, beg;
+  int s_next, o_next;
+  int tile;  // non-empty tiles started so far
+  bool active;
+  __device__ void init(int first, int step, int total) {
+    item = first - step;
+    stride = step;
+    items = total;
+    nblk = 0;
+    s_next = o_next = 0;
+    tile = 0;
+    active = true;
   }
-  return v[0];
+};
+
+// 0 = none, 1 = S op, 2 = O op; *blk = block index within the tile
+__device__ __forceinline__ int next_op(SlotSeq& q, int* blk, const int32_t* kv_off, int N, int cap,
+                                       const DevCtx& ctx) {
+  while (q.active) {
+    if (q.s_next < q.nblk && q.s_next <= q.o_next + 1) {
+      *blk = q.s_next++;
+      return 1;
+    }
+    if (q.o_next < q.nblk) {
+      *blk = q.o_next++;
+      return 2;
+    }
+    q.item += q.stride;
+    if (q.item >= q.items) {
+      q.active = false;
+      return 0;
+    }
+    q.bh = q.item / N;
+    q.qt = q.item - q.bh * N;
+    const Row r = load_row(kv_off, q.bh, q.qt, N, cap, ctx, false);
+    q.len = r.len;
+    q.beg = r.beg;
+    q.nblk = (r.len + 1) >> 1;
+    q.s_next = q.o_next = 0;
+    if (q.nblk > 0) q.tile++;
+  }
+  return 0;
 }
 
-// Phase parity of the n-th completion of a barrier used by every other block (double buffers).
-__device__ __forceinline__ uint32_t par(int n) { return (uint32_t)((n >> 1) & 1); }
-
 __global__ void __launch_bounds__(FT, 1)
-    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ kv_off,
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                       const __nv_bfloat16* __restrict__ qg, const int32_t* __restrict__ kv_off,
                        const int32_t* __restrict__ kv_idx, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
                        int N, int L, int topk, int items, float c2, DevCtx ctx) {
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
@@ -108,16 +132,17 @@ __global__ void __launch_bounds__(FT, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cap = N * topk;
+  const int step = 2 * gridDim.x;
 
   if (threadIdx.x == 0) {
     flag_sh[0] = 0;
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&B.kfull[i], 1), mbar_init(&B.kempty[i], 1);
-      mbar_init(&B.vfull[i], 1), mbar_init(&B.vempty[i], 1);
-      mbar_init(&B.qfull[i], 1), mbar_init(&B.qempty[i], 1);
-      mbar_init(&B.sfull[i], 1), mbar_init(&B.sfree[i], 8);
-      mbar_init(&B.pfull[i], 8), mbar_init(&B.odone[i], 1);
-      mbar_init(&B.ofree[i], 8);
+    for (int i = 0; i < KST; ++i) mbar_init(&B.kfull[i], 1), mbar_init(&B.kempty[i], 1);
+    for (int i = 0; i < VST; ++i) mbar_init(&B.vfull[i], 1), mbar_init(&B.vempty[i], 1);
+    for (int s = 0; s < 2; ++s) {
+      for (int b = 0; b < 2; ++b) mbar_init(&B.sfull[s][b], 1), mbar_init(&B.sfree[s][b], 4);
+      mbar_init(&B.pfull[s], 4);
+      mbar_init(&B.pvdone[s], 1);
+      mbar_init(&B.qready[s], 4);
     }
     mbar_init(&B.done, 1);
     fence_mbar_init();
@@ -133,261 +158,230 @@ __global__ void __launch_bounds__(FT, 1)
 
   if (warp == 8 || warp == 10) {
     // ------------------------------------------------------------------ TMA producers
+    // warp 8 loads K for the S ops, warp 10 loads V for the O ops, both in the MMA issue order.
     const bool k_role = warp == 8;
-    if (lane == 0) {
-      tma_prefetch_desc(k_role ? &tm_k : &tm_v);
-      if (k_role) tma_prefetch_desc(&tm_q);
-      int t = 0, g = 0;
-      int last = -1, last_q = -1;
-      bool ok = true;
-      for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
-        const int bh = item / N, qt = item - bh * N;
-        const Row row = load_row(kv_off, bh, qt, N, cap, ctx, false);
-        const int nblk = (row.len + 1) >> 1;
-        if (nblk == 0) continue;
-        const int row0 = bh * L;
-        if (k_role) {
-          const int qb = t & 1;
-          if (!(ok = mbar_wait(&B.qempty[qb], par(t) ^ 1, abort, ctx))) break;
-          mbar_arrive_expect_tx(&B.qfull[qb], Q_B);
-          for (int h = 0; h < 2; ++h)
-            tma_load_2d(dsm + OFF_Q + qb * Q_B + h * TILE_B, &tm_q, h * 64, row0 + qt * 64, &B.qfull[qb]);
-          last_q = t;
-        }
-        const int32_t* idx = kv_idx + (size_t)bh * cap + row.beg;
-        for (int n = 0; n < nblk; ++n, ++g) {
-          const int st = g & 1;
-          const int ntile = min(2, row.len - 2 * n);
-          uint64_t* empty = k_role ? &B.kempty[st] : &B.vempty[st];
-          uint64_t* full = k_role ? &B.kfull[st] : &B.vfull[st];
-          const CUtensorMap* map = k_role ? &tm_k : &tm_v;
-          uint8_t* dst = dsm + (k_role ? OFF_K : OFF_V) + st * BLK_B;
-          if (!(ok = mbar_wait(empty, par(g) ^ 1, abort, ctx))) break;
-          mbar_arrive_expect_tx(full, ntile * 2 * TILE_B);
+    const CUtensorMap* map = k_role ? &tm_k : &tm_v;
+    if (lane == 0) tma_prefetch_desc(map);
+    const int nst = k_role ? KST : VST;
+    SlotSeq sq[2];
+    sq[0].init(2 * blockIdx.x, step, items);
+    sq[1].init(2 * blockIdx.x + 1, step, items);
+    int c = 0, last = -1;
+    bool ok = true;
+    while (ok && (sq[0].active || sq[1].active)) {
 #pragma unroll
-          for (int tt = 0; tt < 2; ++tt) {
-            if (tt >= ntile) break;
-            int j = idx[2 * n + tt];
-            if (j < 0 || j >= N) {
-              if (ctx.flags & VSA2_FLAG_VALIDATE) set_error(ctx.err, VSA2_ERR_BAD_INDEX);
-              j = j < 0 ? 0 : N - 1;
-            }
-            tma_load_2d(dst + tt * TILE_B, map, 0, row0 + j * 64, full);
-            tma_load_2d(dst + 2 * TILE_B + tt * TILE_B, map, 64, row0 + j * 64, full);
+      for (int s = 0; s < 2; ++s) {
+        if (!ok) break;
+        int blk;
+        const int op = next_op(sq[s], &blk, kv_off, N, cap, ctx);
+        if (op == 0 || (op == 1) != k_role) continue;
+        const SlotSeq& q = sq[s];
+        const int ntile = min(2, q.len - 2 * blk);
+        int j = 0;
+        if (lane < 2 * ntile) {
+          j = kv_idx[(size_t)q.bh * cap + q.beg + 2 * blk + (lane >> 1)];
+          if (j < 0 || j >= N) {
+            if (ctx.flags & VSA2_FLAG_VALIDATE) set_error(ctx.err, VSA2_ERR_BAD_INDEX);
+            j = min(max(j, 0), N - 1);
           }
-          last = g;
         }
-        ++t;
+        const int st = c % nst;
+        uint64_t* empty = k_role ? &B.kempty[st] : &B.vempty[st];
+        uint64_t* full = k_role ? &B.kfull[st] : &B.vfull[st];
+        int w_ok = 1;
+        if (lane == 0) {
+          w_ok = mbar_wait(empty, ((c / nst) & 1) ^ 1, abort, ctx);
+          if (w_ok) mbar_arrive_expect_tx(full, ntile * 2 * TILE_B);
+        }
+        if (!(ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0)) break;
+        if (lane < 2 * ntile) {
+          const int tt = lane >> 1, h = lane & 1;
+          tma_load_2d(dsm + (k_role ? OFF_K : OFF_V) + st * BLK_B + h * 2 * TILE_B + tt * TILE_B, map, h * 64,
+                      q.bh * L + j * 64, full);
+        }
+        last = c++;
       }
-      if (*abort) {  // let copies still in flight land before the CTA exits
-        for (int gg = max(0, last - 1); gg <= last; ++gg)
-          mbar_wait_drain(k_role ? &B.kfull[gg & 1] : &B.vfull[gg & 1], par(gg), ctx.timeout_ns);
-        if (last_q >= 0) mbar_wait_drain(&B.qfull[last_q & 1], par(last_q), ctx.timeout_ns);
-      }
+    }
+    if (lane == 0 && *abort) {  // let copies still in flight land before the CTA exits
+      for (int cc = max(0, last - nst + 1); cc <= last; ++cc)
+        mbar_wait_drain(k_role ? &B.kfull[cc % nst] : &B.vfull[cc % nst], (cc / nst) & 1, ctx.timeout_ns);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t id_s = idesc_bf16_f32(128, 64, false, false);
-      constexpr uint32_t id_o = idesc_bf16_f32(128, 64, true, true);
-      int t = 0, g0 = 0;
+      constexpr uint32_t id_s = idesc_bf16_f32(64, 128, false, false);
+      constexpr uint32_t id_o = idesc_bf16_f32(64, 128, false, true);
+      SlotSeq sq[2];
+      sq[0].init(2 * blockIdx.x, step, items);
+      sq[1].init(2 * blockIdx.x + 1, step, items);
+      int kc = 0, vc = 0;
+      int g[2] = {0, 0};   // S blocks issued per slot
+      int go[2] = {0, 0};  // O blocks issued per slot
       bool ok = true;
-      for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
-        const int bh = item / N, qt = item - bh * N;
-        const Row row = load_row(kv_off, bh, qt, N, cap, ctx, false);
-        const int nblk = (row.len + 1) >> 1;
-        if (nblk == 0) continue;
-        const int qb = t & 1;
-        const uint32_t qa = smem_u32(dsm + OFF_Q + qb * Q_B);
-        const uint32_t o_acc = tmem + 128 + (t & 1) * 64;
-        if (!(ok = mbar_wait(&B.qfull[qb], par(t), abort, ctx))) break;
-        int s_next = 0, o_next = 0;
-        while (ok && o_next < nblk) {
-          if (s_next < nblk && s_next <= o_next + 1) {
-            const int g = g0 + s_next;
-            if (!(ok = mbar_wait(&B.kfull[g & 1], par(g), abort, ctx))) break;
-            if (!(ok = mbar_wait(&B.sfree[g & 1], par(g) ^ 1, abort, ctx))) break;
-            tc_fence_after();
-            const uint32_t ka = smem_u32(dsm + OFF_K + (g & 1) * BLK_B);
+      while (ok && (sq[0].active || sq[1].active)) {
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t h = kk >> 2, sub = (kk & 3) * 32;
-              mma_bf16_ss(tmem + (g & 1) * 64, sdesc_sw128(ka + h * 2 * TILE_B + sub, 16, 1024),
-                          sdesc_sw128(qa + h * TILE_B + sub, 16, 1024), id_s, kk > 0);
-            }
-            mma_commit(&B.kempty[g & 1]);
-            mma_commit(&B.sfull[g & 1]);
-            if (s_next == nblk - 1) mma_commit(&B.qempty[qb]);
-            ++s_next;
-          } else {
-            const int n = o_next, g = g0 + n;
-            if (n == 0 && !(ok = mbar_wait(&B.ofree[t & 1], par(t) ^ 1, abort, ctx))) break;
-            if (!(ok = mbar_wait(&B.vfull[g & 1], par(g), abort, ctx))) break;
-            if (!(ok = mbar_wait(&B.pfull[g & 1], par(g), abort, ctx))) break;
+        for (int s = 0; s < 2; ++s) {
+          if (!ok) break;
+          int blk;
+          const int op = next_op(sq[s], &blk, kv_off, N, cap, ctx);
+          if (op == 0) continue;
+          const uint32_t lanes = (uint32_t)(16 * s) << 16;
+          if (op == 1) {
+            if (blk == 0 && !(ok = mbar_wait(&B.qready[s], (sq[s].tile - 1) & 1, abort, ctx))) break;
+            const int st = kc % KST;
+            const int gb = g[s];
+            if (!(ok = mbar_wait(&B.kfull[st], (kc / KST) & 1, abort, ctx))) break;
+            if (!(ok = mbar_wait(&B.sfree[s][gb & 1], ((gb >> 1) & 1) ^ 1, abort, ctx))) break;
             tc_fence_after();
-            const uint32_t va = smem_u32(dsm + OFF_V + (g & 1) * BLK_B);
-            const uint32_t pa = smem_u32(dsm + OFF_P + (g & 1) * PT_B);
-            const int ksteps = (2 * n + 1 == row.len) ? 4 : 8;
+            const uint32_t ka = smem_u32(dsm + OFF_K + st * BLK_B);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_bf16_ts(tmem + lanes + TM_S + (gb & 1) * 128, tmem + lanes + TM_Q + 8 * kk,
+                          sdesc_sw128(ka + (kk >> 2) * 2 * TILE_B + (kk & 3) * 32, 16, 1024), id_s, kk > 0);
+            mma_commit(&B.kempty[st]);
+            mma_commit(&B.sfull[s][gb & 1]);
+            ++kc;
+            ++g[s];
+          } else {
+            const int st = vc % VST;
+            const int gb = go[s];
+            if (!(ok = mbar_wait(&B.vfull[st], (vc / VST) & 1, abort, ctx))) break;
+            if (!(ok = mbar_wait(&B.pfull[s], gb & 1, abort, ctx))) break;
+            tc_fence_after();
+            const uint32_t va = smem_u32(dsm + OFF_V + st * BLK_B);
+            const int ksteps = (2 * blk + 1 == sq[s].len) ? 4 : 8;
             for (int kk = 0; kk < ksteps; ++kk)
-              mma_bf16_ss(o_acc, sdesc_sw128(va + kk * 2048, 2 * TILE_B, 1024), sdesc_sw128(pa + kk * 2048, PT_B, 1024),
-                          id_o, (n > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(&B.vempty[g & 1]);
-            mma_commit(&B.odone[g & 1]);
-            ++o_next;
+              mma_bf16_ts(tmem + lanes + TM_O, tmem + lanes + TM_P + 8 * kk,
+                          sdesc_sw128(va + kk * 2048, 2 * TILE_B, 1024), id_o, (blk > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&B.vempty[st]);
+            mma_commit(&B.pvdone[s]);
+            ++vc;
+            ++go[s];
           }
         }
-        g0 += nblk;
-        ++t;
       }
       mma_commit(&B.done);
       mbar_wait_drain(&B.done, 0, ctx.timeout_ns);
     }
   } else if (warp < 8) {
-    // ------------------------------------------------------------------ softmax warpgroups
-    const int w = warp >> 2;   // warpgroup: query columns 32w .. 32w+31
-    const int wq = warp & 3;   // TMEM lane quarter
-    const int tid = threadIdx.x & 127;
-    const int bar_id = 1 + w;
-    float* m_s = reinterpret_cast<float*>(dsm + OFF_M) + w * 32;
-    float* red = reinterpret_cast<float*>(dsm + OFF_RED) + w * 128;
-    float* alpha = reinterpret_cast<float*>(dsm + OFF_ALPHA) + w * 32;
-    uint8_t* stage = dsm + OFF_ST + w * ST_B;
-    const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
-    int t = 0, g = 0;
-    for (int item = blockIdx.x; item < items; item += gridDim.x) {
+    // ------------------------------------------------------------------ softmax, one slot per warpgroup
+    const int s = warp >> 2;
+    const int w = warp & 3;                        // TMEM lane quarter
+    const int bar_id = 1 + s;
+    const int r16 = 8 * (lane & 1) + (lane >> 2);  // row within this warp's 16
+    const int par_c = (lane >> 1) & 1;             // even / odd columns
+    const int row = 16 * w + r16;                  // row within the query tile
+    const uint32_t tl = tmem + ((uint32_t)(32 * w + 16 * s) << 16);
+    int g = 0;  // blocks processed by this slot
+    for (int item = 2 * blockIdx.x + s; item < items; item += step) {
       const int bh = item / N, qt = item - bh * N;
-      const Row row = load_row(kv_off, bh, qt, N, cap, ctx, tid == 0 && w == 0);
-      const int nblk = (row.len + 1) >> 1;
-      const size_t tok0 = (size_t)bh * L + (size_t)qt * 64 + 32 * w;  // this warpgroup's 32 query rows
+      const Row rw = load_row(kv_off, bh, qt, N, cap, ctx, w == 0 && lane == 0);
+      const int nblk = (rw.len + 1) >> 1;
+      const size_t tok = (size_t)bh * L + (size_t)qt * 64 + row;
       if (nblk == 0) {
-        uint4* o4 = reinterpret_cast<uint4*>(out + tok0 * 128);
-        for (int e = tid; e < 32 * 128 / 8; e += 128) o4[e] = make_uint4(0, 0, 0, 0);
-        if (tid < 32) lse[tok0 + tid] = -INFINITY;
+        // empty selection: o = 0, lse = -inf (each thread of a pair writes half the row)
+        uint4* o4 = reinterpret_cast<uint4*>(out + tok * 128 + par_c * 64);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o4[e] = make_uint4(0, 0, 0, 0);
+        if (par_c == 0) lse[tok] = -INFINITY;
         continue;
       }
-      const uint32_t o_acc = tmem + lane_off + 128 + (t & 1) * 64 + 32 * w;
-      if (tid < 32) m_s[tid] = -INFINITY;
-      float lpart[32];
+      {
+        // Q row into TMEM (A operand of S): packed words j = 2i + par_c hold d = 2j, 2j+1
+        uint32_t qv[32];
+        const uint2* src = reinterpret_cast<const uint2*>(qg + tok * 128);
 #pragma unroll
-      for (int q = 0; q < 32; ++q) lpart[q] = 0.f;
-      named_bar_sync(bar_id, 128);
-      for (int n = 0; n < nblk; ++n, ++g) {
-        const bool valid_row = !(2 * n + 1 == row.len && tid >= 64);
-        const uint32_t s_addr = tmem + lane_off + (g & 1) * 64 + 32 * w;
-        mbar_wait(&B.sfull[g & 1], par(g), abort, ctx);
-        tc_fence_after();
-        uint32_t r[32];
-        tmem_ld32(s_addr, r);
-        tmem_ld_wait();
-        float tmax = -INFINITY;
-        if (valid_row) {
-#pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            const float4 mv = reinterpret_cast<const float4*>(m_s)[q4];
-            tmax = fmaxf(tmax, fmaf(__uint_as_float(r[4 * q4 + 0]), c2, -mv.x));
-            tmax = fmaxf(tmax, fmaf(__uint_as_float(r[4 * q4 + 1]), c2, -mv.y));
-            tmax = fmaxf(tmax, fmaf(__uint_as_float(r[4 * q4 + 2]), c2, -mv.z));
-            tmax = fmaxf(tmax, fmaf(__uint_as_float(r[4 * q4 + 3]), c2, -mv.w));
-          }
+        for (int i = 0; i < 32; ++i) {
+          const uint2 v = __ldg(src + i);
+          qv[i] = par_c ? v.y : v.x;
         }
-        if (named_bar_or(bar_id, 128, tmax > kThresh)) {
-          // raise the running max of these 32 columns to the block's column max
-          float v[32];
-#pragma unroll
-          for (int q = 0; q < 32; ++q) v[q] = valid_row ? __uint_as_float(r[q]) * c2 : -INFINITY;
-          red[wq * 32 + lane] = warp_rs32<true>(v, lane);
-          named_bar_sync(bar_id, 128);
-          if (tid < 32) {
-            const float cm = fmaxf(fmaxf(red[tid], red[32 + tid]), fmaxf(red[64 + tid], red[96 + tid]));
-            const float mo = m_s[tid];
-            const float mn = fmaxf(mo, cm);
-            alpha[tid] = mo == -INFINITY ? 0.f : ex2(mo - mn);
-            m_s[tid] = mn;
-          }
-          named_bar_sync(bar_id, 128);
-#pragma unroll
-          for (int q = 0; q < 32; ++q) lpart[q] *= alpha[q];
-          if (n > 0) {
-            // O^T holds blocks 0..n-1 of this tile: wait for the last, then scale our columns
-            mbar_wait(&B.odone[(g - 1) & 1], par(g - 1), abort, ctx);
-            tc_fence_after();
-            uint32_t o[32];
-            tmem_ld32(o_acc, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int q = 0; q < 32; ++q) o[q] = u32(__uint_as_float(o[q]) * alpha[q]);
-            tmem_st32(o_acc, o);
-            tmem_st_wait();
-          }
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 mv = reinterpret_cast<const float4*>(m_s)[q4];
-          float p0 = ex2(fmaf(__uint_as_float(r[4 * q4 + 0]), c2, -mv.x));
-          float p1 = ex2(fmaf(__uint_as_float(r[4 * q4 + 1]), c2, -mv.y));
-          float p2 = ex2(fmaf(__uint_as_float(r[4 * q4 + 2]), c2, -mv.z));
-          float p3 = ex2(fmaf(__uint_as_float(r[4 * q4 + 3]), c2, -mv.w));
-          if (!valid_row) p0 = p1 = p2 = p3 = 0.f;
-          lpart[4 * q4 + 0] += p0;
-          lpart[4 * q4 + 1] += p1;
-          lpart[4 * q4 + 2] += p2;
-          lpart[4 * q4 + 3] += p3;
-          pk[2 * q4] = pack_bf16(p0, p1);
-          pk[2 * q4 + 1] = pack_bf16(p2, p3);
-        }
-        // P^T buffer g&1 was last read by the O MMA of block g-2
-        mbar_wait(&B.odone[g & 1], par(g) ^ 1, abort, ctx);
-        if (valid_row) {
-          const uint32_t rowaddr = smem_u32(dsm + OFF_P + (g & 1) * PT_B) + tid * 128;
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            st_shared_v4(rowaddr + (((4 * w + c) ^ (tid & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
-                         pk[4 * c + 3]);
-        }
-        fence_proxy_async_smem();
+        tmem_st16x64b_x32(tl + TM_Q, qv);
+        tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&B.sfree[g & 1]);
-          mbar_arrive(&B.pfull[g & 1]);
-        }
+        if (lane == 0) mbar_arrive(&B.qready[s]);
       }
-      // ---- epilogue: wait for the last O block, finish the row sums, normalise, store
-      mbar_wait(&B.odone[(g - 1) & 1], par(g - 1), abort, ctx);
-      tc_fence_after();
-      red[wq * 32 + lane] = warp_rs32<false>(lpart, lane);
-      named_bar_sync(bar_id, 128);
-      if (tid < 32) {
-        const float l = (red[tid] + red[32 + tid]) + (red[64 + tid] + red[96 + tid]);
-        alpha[tid] = 1.f / l;
-        lse[tok0 + tid] = (m_s[tid] + __log2f(l)) * 0.6931471805599453f;
-      }
-      named_bar_sync(bar_id, 128);
-      {
-        // thread tid owns O^T row d = tid; O[q][d] for this warpgroup's 32 query rows
-        uint32_t o[32];
-        tmem_ld32(o_acc, o);
+      float m = -INFINITY, l = 0.f;
+      for (int n = 0; n < nblk; ++n, ++g) {
+        const bool half = (2 * n + 1 == rw.len);
+        mbar_wait(&B.sfull[s][g & 1], (g >> 1) & 1, abort, ctx);
+        tc_fence_after();
+        uint32_t x[64];
+        tmem_ld16x64b_x64(tl + TM_S + (g & 1) * 128, x);
         tmem_ld_wait();
-        __nv_bfloat16* st = reinterpret_cast<__nv_bfloat16*>(stage);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.sfree[s][g & 1]);
+        // columns 2i + par_c; in a half block only the first 64 columns are real
+        float mx = -INFINITY;
 #pragma unroll
-        for (int q = 0; q < 32; ++q) st[q * 128 + tid] = __float2bfloat16_rn(__uint_as_float(o[q]) * alpha[q]);
+        for (int i = 0; i < 64; ++i)
+          if (!(half && i >= 32)) mx = fmaxf(mx, __uint_as_float(x[i]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2)) * c2;
+        float alpha = 1.f;
+        const bool raise = mx > m + kThresh;
+        if (raise) {
+          alpha = (m == -INFINITY) ? 0.f : ex2(m - mx);
+          m = mx;
+          l *= alpha;
+        }
+        if (__any_sync(0xffffffffu, raise && n > 0)) {
+          // O holds blocks 0..n-1 of this tile: scale the raised rows once the last O MMA is done
+          mbar_wait(&B.pvdone[s], (g - 1) & 1, abort, ctx);
+          tc_fence_after();
+          uint32_t o[64];
+          tmem_ld16x64b_x64(tl + TM_O, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 64; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st16x64b_x64(tl + TM_O, o);
+          tmem_st_wait();
+        }
+        // probabilities (<= 2^8), partial row sum, pack bf16 pairs of adjacent columns:
+        // the pair partner holds the neighbouring column, so swap half of the values
+        uint32_t pk[32];
+        float ls = 0.f;
+#pragma unroll
+        for (int i2 = 0; i2 < 32; ++i2) {
+          float pa = ex2(fmaf(__uint_as_float(x[2 * i2]), c2, -m));
+          float pb = ex2(fmaf(__uint_as_float(x[2 * i2 + 1]), c2, -m));
+          if (half && i2 >= 16) pa = pb = 0.f;
+          ls += pa + pb;
+          const float send = par_c ? pa : pb;
+          const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
+          // even thread: word 2*i2 = (col 4*i2, 4*i2+1); odd thread: word 2*i2+1 = (4*i2+2, 4*i2+3)
+          pk[i2] = par_c ? pack_bf16(recv, pb) : pack_bf16(pa, recv);
+        }
+        l += ls;
+        // P region is free once the O MMA of the previous block has finished
+        if (n > 0) mbar_wait(&B.pvdone[s], (g - 1) & 1, abort, ctx);
+        tmem_st16x64b_x32(tl + TM_P, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.pfull[s]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&B.ofree[t & 1]);
-      fence_proxy_async_smem();
-      named_bar_sync(bar_id, 128);
-      if (tid == 0) {
-        bulk_store(out + tok0 * 128, stage, ST_B);
-        bulk_commit();
-        bulk_wait_read0();
+      // ---- epilogue: last O block done -> normalise and store
+      mbar_wait(&B.pvdone[s], (g - 1) & 1, abort, ctx);
+      tc_fence_after();
+      l += __shfl_xor_sync(0xffffffffu, l, 2);
+      const float inv = 1.f / l;
+      if (par_c == 0) lse[tok] = (m + __log2f(l)) * 0.6931471805599453f;
+      uint32_t o[64];
+      tmem_ld16x64b_x64(tl + TM_O, o);
+      tmem_ld_wait();
+      // o[i] = O[row][2i + par_c]; swap so each thread holds adjacent pairs, then 4-byte stores
+      uint32_t* dst = reinterpret_cast<uint32_t*>(out + tok * 128);
+#pragma unroll
+      for (int i2 = 0; i2 < 32; ++i2) {
+        const float a = __uint_as_float(o[2 * i2]) * inv, b = __uint_as_float(o[2 * i2 + 1]) * inv;
+        const float send = par_c ? a : b;
+        const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
+        dst[2 * i2 + par_c] = par_c ? pack_bf16(recv, b) : pack_bf16(a, recv);
       }
-      ++t;
       // leave together if any wait of this CTA has expired
       if (named_bar_or(bar_id, 128, *abort != 0)) break;
     }
-    if (tid == 0) bulk_wait0();
   }
   tc_fence_before();
   __syncthreads();
@@ -404,21 +398,20 @@ bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64
 
 vsa2_status attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v, int topk, const int32_t* kv_off,
                         const int32_t* kv_idx, void* o, float* lse, char* ws, cudaStream_t s) {
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tk, tv;
   const uint64_t rows = (uint64_t)d.BH * d.L;
-  if (!make_tmap_2d_bf16(&tq, q, 128, rows, 64, 64) || !make_tmap_2d_bf16(&tk, k, 128, rows, 64, 64) ||
-      !make_tmap_2d_bf16(&tv, v, 128, rows, 64, 64))
+  if (!make_tmap_2d_bf16(&tk, k, 128, rows, 64, 64) || !make_tmap_2d_bf16(&tv, v, 128, rows, 64, 64))
     return cuda_fail("tensor map encoding for the attention operands failed");
   DevCtx ctx{reinterpret_cast<int*>(ws), d.timeout_ns, d.flags};
   const int items = d.BH * d.N;
   int sms = 148;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = std::min(sms, items);
+  const int grid = std::max(1, std::min(sms, (items + 1) / 2));
   const float c2 = 1.4426950408889634f / sqrtf(128.f);
   cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
-  attn_fwd_tc_kernel<<<grid, FT, SMEM_DYN, s>>>(tq, tk, tv, kv_off, kv_idx, (__nv_bfloat16*)o, lse, d.N, (int)d.L,
-                                                topk, items, c2, ctx);
+  attn_fwd_tc_kernel<<<grid, FT, SMEM_DYN, s>>>(tk, tv, (const __nv_bfloat16*)q, kv_off, kv_idx, (__nv_bfloat16*)o,
+                                                lse, d.N, (int)d.L, topk, items, c2, ctx);
   return check_launch(__func__);
 }
 
