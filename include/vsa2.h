@@ -139,6 +139,26 @@ vsa2_status vsa2_sparse_attn_bwd(const vsa2_problem* p, const void* q, const voi
                                  float* dq, float* dk, float* dv,
                                  void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * Per-sequence TopK like vsa2_topk_select (same ranking, same CSR output, no CSC), for callers
+ * that cannot allocate device memory when they call in: for example a host program whose device
+ * memory is entirely owned by another allocator or pool, or a call site where the implicit
+ * synchronisation of cudaMalloc is not acceptable. It takes no workspace and allocates nothing
+ * (no cudaMalloc, cudaFree or allocating library routine). This entry point has no counterpart
+ * in the paper.
+ *   scores, topk, kv_off, kv_idx : as for vsa2_topk_select
+ * Scratch: a fixed 8 MiB array in the library's device image, held by every GPU that loads
+ * the library until the process exits. One call needs
+ *   256 + 256*ceil(batch*heads*24576/256) + 256*ceil(batch*heads*32/256) + 3*256*ceil(batch*heads*N*4/256)
+ * bytes of it (about batch*heads*(24.6 KiB + 12*N)); larger problems return VSA2_ERR_UNSUPPORTED
+ * before anything is enqueued. The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and should come before any stream capture. Every call shares the one
+ * array, which keeps the previous call's contents (the call clears what must start at zero):
+ * calls that may overlap on the GPU, on any streams, race. VSA2_FLAG_VALIDATE is ignored.
+ */
+vsa2_status vsa2_topk_select_noalloc(const vsa2_problem* p, const float* scores, int32_t topk,
+                                     int32_t* kv_off, int32_t* kv_idx, void* stream);
+
 /* Synchronise `stream`, read and clear the device error word of `ws`. Returns VSA2_OK,
  * VSA2_ERR_TIMEOUT, VSA2_ERR_BAD_INDEX, or VSA2_ERR_CUDA if the synchronisation failed. */
 vsa2_status vsa2_get_device_error(void* ws, void* stream);

@@ -19,7 +19,8 @@ VSA2_FLAG_VALIDATE = 1
 # every symbol the header declares
 EXPORTS = ("vsa2_workspace_size", "vsa2_workspace_init", "vsa2_router_scores", "vsa2_topk_select",
            "vsa2_sparse_attn_fwd", "vsa2_sparse_attn_bwd", "vsa2_get_device_error",
-           "vsa2_selftest_wait_timeout", "vsa2_status_string", "vsa2_version", "vsa2_last_cuda_error")
+           "vsa2_selftest_wait_timeout", "vsa2_status_string", "vsa2_version", "vsa2_last_cuda_error",
+           "vsa2_topk_select_noalloc")
 
 
 class Vsa2Error(RuntimeError):
@@ -56,13 +57,15 @@ def lib() -> ctypes.CDLL:
         L.vsa2_topk_select.argtypes = [P, vp, i32, vp, vp, vp, vp, vp, sz, vp]
         L.vsa2_sparse_attn_fwd.argtypes = [P, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]
         L.vsa2_sparse_attn_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.vsa2_topk_select_noalloc.argtypes = [P, vp, i32, vp, vp, vp]
         L.vsa2_get_device_error.argtypes = [vp, vp]
         L.vsa2_selftest_wait_timeout.argtypes = [vp, sz, u32, vp]
         L.vsa2_status_string.argtypes = [ctypes.c_int]
         L.vsa2_status_string.restype = ctypes.c_char_p
         L.vsa2_version.restype = i32
         L.vsa2_last_cuda_error.restype = ctypes.c_char_p
-        for name in ("vsa2_workspace_init", "vsa2_router_scores", "vsa2_topk_select", "vsa2_sparse_attn_fwd",
+        for name in ("vsa2_workspace_init", "vsa2_router_scores", "vsa2_topk_select", "vsa2_topk_select_noalloc",
+                     "vsa2_sparse_attn_fwd",
                      "vsa2_sparse_attn_bwd", "vsa2_get_device_error", "vsa2_selftest_wait_timeout"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -117,6 +120,12 @@ def vsa2_topk_select(p: Problem, scores, topk, kv_off, kv_idx, q_off, q_idx, ws,
     _check(lib().vsa2_topk_select(ctypes.byref(p), _ptr(scores), topk, _ptr(kv_off), _ptr(kv_idx), _ptr(q_off),
                                   _ptr(q_idx), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "vsa2_topk_select")
+
+
+def vsa2_topk_select_noalloc(p: Problem, scores, topk, kv_off, kv_idx, stream=None) -> None:
+    """TopK (CSR only) that allocates nothing: its scratch is a fixed device array in the library."""
+    _check(lib().vsa2_topk_select_noalloc(ctypes.byref(p), _ptr(scores), topk, _ptr(kv_off), _ptr(kv_idx),
+                                          _stream(stream)), "vsa2_topk_select_noalloc")
 
 
 def vsa2_sparse_attn_fwd(p: Problem, q, k, v, topk, kv_off, kv_idx, o, lse, ws, stream=None) -> None:

@@ -208,6 +208,18 @@ vsa2_status vsa2_sparse_attn_bwd(const vsa2_problem* p, const void* q, const voi
                          (cudaStream_t)stream);
 }
 
+vsa2_status vsa2_topk_select_noalloc(const vsa2_problem* p, const float* scores, int32_t topk, int32_t* kv_off,
+                                     int32_t* kv_idx, void* stream) {
+  Dims d;
+  vsa2_status st = make_dims(p, &d);
+  if (st != VSA2_OK) return st;
+  if (!scores || !kv_off || !kv_idx) return VSA2_ERR_INVALID_ARG;
+  if (topk < 1 || topk > d.N) return VSA2_ERR_UNSUPPORTED;
+  if (!aligned16(scores)) return VSA2_ERR_INVALID_ARG;
+  if (topk_noalloc_bytes(d) > topk_noalloc_capacity()) return VSA2_ERR_UNSUPPORTED;
+  return launch_topk_noalloc(d, scores, topk, kv_off, kv_idx, (cudaStream_t)stream);
+}
+
 vsa2_status vsa2_get_device_error(void* ws, void* stream) {
   if (!ws) return VSA2_ERR_INVALID_ARG;
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return VSA2_ERR_CUDA;

@@ -72,6 +72,11 @@ vsa2_status attn_fwd_tc(const Dims& d, const void* q, const void* k, const void*
                         const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
                         cudaStream_t s);
 vsa2_status launch_wait_timeout_probe(int* err, uint64_t timeout_ns, cudaStream_t s);
+// allocation-free TopK (scratch in a fixed device array of the library)
+size_t topk_noalloc_bytes(const Dims& d);
+size_t topk_noalloc_capacity();
+vsa2_status launch_topk_noalloc(const Dims& d, const float* scores, int topk, int32_t* kv_off, int32_t* kv_idx,
+                                cudaStream_t s);
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 

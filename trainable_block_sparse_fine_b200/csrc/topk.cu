@@ -7,6 +7,8 @@
 // a per-row scan assigns the tie quota row by row, then each row is compacted in ascending j
 // (CSR). The CSC used by the backward pass is built from a per-column bitmap, so both lists
 // are deterministic.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -308,6 +310,95 @@ vsa2_status launch_topk(const Dims& d, const float* scores, int topk, int32_t* k
   }
   if (check_launch(__func__) != VSA2_OK) return VSA2_ERR_CUDA;
   return VSA2_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// Allocation-free variant (CSR only). Its scratch is a fixed array in the library's device
+// image instead of a caller workspace; see vsa2_topk_select_noalloc in vsa2.h.
+// ------------------------------------------------------------------------------------------
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per device
+__device__ __align__(256) unsigned char g_topk_scratch[kNoAllocScratchBytes];
+
+struct NoAllocLayout {
+  size_t err, hist, state, row_gt, row_eq, row_take, total;
+};
+NoAllocLayout noalloc_layout(const Dims& d) {
+  NoAllocLayout l{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += align256(bytes);
+    return at;
+  };
+  l.err = take(sizeof(int));
+  l.hist = take((size_t)d.BH * 3 * 2048 * 4);
+  l.state = take((size_t)d.BH * 8 * 4);
+  l.row_gt = take((size_t)d.BH * d.N * 4);
+  l.row_eq = take((size_t)d.BH * d.N * 4);
+  l.row_take = take((size_t)d.BH * d.N * 4);
+  l.total = off;
+  return l;
+}
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[64] = {};  // device address of g_topk_scratch, per device ordinal
+
+// Device address of the scratch array for the current device, looked up once per device
+// (cudaGetSymbolAddress with that device current; the host-side symbol is not a device address).
+vsa2_status noalloc_scratch(char** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice failed");
+  if (dev < 0 || dev >= 64) return cuda_fail("device ordinal out of range for the TopK scratch table");
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_topk_scratch) != cudaSuccess || !ptr)
+      return cuda_fail("cudaGetSymbolAddress of the TopK scratch array failed");
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = static_cast<char*>(g_scratch_ptr[dev]);
+  return VSA2_OK;
+}
+}  // namespace
+
+size_t topk_noalloc_bytes(const Dims& d) { return noalloc_layout(d).total; }
+size_t topk_noalloc_capacity() { return kNoAllocScratchBytes; }
+
+vsa2_status launch_topk_noalloc(const Dims& d, const float* scores, int topk, int32_t* kv_off, int32_t* kv_idx,
+                                cudaStream_t s) {
+  const NoAllocLayout w = noalloc_layout(d);
+  if (w.total > kNoAllocScratchBytes) return VSA2_ERR_UNSUPPORTED;
+  char* base = nullptr;
+  vsa2_status st = noalloc_scratch(&base);
+  if (st != VSA2_OK) return st;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(base + w.hist);
+  uint32_t* state = reinterpret_cast<uint32_t*>(base + w.state);
+  int32_t* row_gt = reinterpret_cast<int32_t*>(base + w.row_gt);
+  int32_t* row_eq = reinterpret_cast<int32_t*>(base + w.row_eq);
+  int32_t* row_take = reinterpret_cast<int32_t*>(base + w.row_take);
+  // validate-mode reports have nowhere to go without a workspace: the flag is ignored here
+  DevCtx ctx{reinterpret_cast<int*>(base + w.err), d.timeout_ns, 0};
+  const int64_t nn = (int64_t)d.N * d.N;
+  const uint32_t budget = (uint32_t)d.N * (uint32_t)topk;
+  // the array keeps the previous call's contents: the histograms must start at zero
+  if (cudaMemsetAsync(base, 0, w.state, s) != cudaSuccess) return cuda_fail("cudaMemsetAsync of the TopK scratch failed");
+  int per_head = (int)((nn + 16383) / 16384);
+  const int cap = (148 * 8 + d.BH - 1) / d.BH;
+  if (per_head > cap) per_head = cap;
+  if (per_head < 1) per_head = 1;
+  dim3 hgrid(per_head, d.BH);
+  topk_hist_kernel<0><<<hgrid, 512, 0, s>>>(scores, nn, state, hist);
+  topk_select_digit_kernel<0><<<d.BH, 1024, 0, s>>>(hist, state, budget);
+  topk_hist_kernel<1><<<hgrid, 512, 0, s>>>(scores, nn, state, hist);
+  topk_select_digit_kernel<1><<<d.BH, 1024, 0, s>>>(hist, state, budget);
+  topk_hist_kernel<2><<<hgrid, 512, 0, s>>>(scores, nn, state, hist);
+  topk_select_digit_kernel<2><<<d.BH, 1024, 0, s>>>(hist, state, budget);
+  dim3 rgrid((d.N + 7) / 8, d.BH);
+  topk_row_count_kernel<<<rgrid, 256, 0, s>>>(scores, d.N, state, row_gt, row_eq);
+  topk_offsets_kernel<<<d.BH, 1024, 0, s>>>(d.N, state, row_gt, row_eq, row_take, kv_off);
+  topk_emit_kernel<<<rgrid, 256, 0, s>>>(scores, d.N, topk, state, row_take, kv_off, kv_idx, nullptr, nullptr, 0, ctx);
+  return check_launch(__func__);
 }
 
 }  // namespace vsa2
