@@ -14,8 +14,10 @@ summed over ranks, divided by the max step time over ranks.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -41,6 +43,23 @@ def load_peaks():
         return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained", p["bf16_tflops"]), "measured"
     except Exception:
         return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def profiled_traffic(wl, pairs):
+    """DRAM bytes of one forward launch from the committed ncu summary, scaled by selected pairs;
+    None when the kernel source changed since the counters were taken or for other workloads."""
+    if wl.grid != (56, 48, 80) or wl.head_dim != 128 or wl.topk != 64:
+        return None
+    try:
+        txt = open(os.path.join(ROOT, "profiles", "attn_fwd_tc_720p_8heads.md")).read()
+        src = open(os.path.join(ROOT, "trainable_block_sparse_fine_b200", "csrc", "attn_fwd_tc.cu"), "rb").read()
+    except OSError:
+        return None
+    per = re.search(r"dram_bytes_per_pair:\s*(\d+)", txt)
+    sha = re.search(r"source_sha1:\s*([0-9a-f]{40})", txt)
+    if not (per and sha) or hashlib.sha1(src).hexdigest() != sha.group(1):
+        return None
+    return int(per.group(1)) * pairs
 
 
 def pair_flops(wl, pairs, backward):
@@ -177,6 +196,7 @@ def run_ours(args, wl):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     import trainable_block_sparse_fine_b200 as V
+    from trainable_block_sparse_fine_b200.sharding import max_over_ranks
 
     dev = torch.device("cuda", local)
     # weak scaling: every rank runs the full workload on its own batch element (seed offset)
@@ -235,12 +255,7 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms_local = statistics.mean(per["step"])
-    ms = ms_local
-    if world > 1:
-        t = torch.tensor([ms_local], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(statistics.mean(per["step"]), dev)
     err = e.device_error()
     if err != 0:
         raise RuntimeError(f"device error {V.vsa2_status_string(err)} in the timed region")
@@ -267,12 +282,7 @@ def run_ours(args, wl):
         torch.cuda.synchronize()
         if it >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
-    e2e_local = statistics.mean(e2e_ms) if e2e_ms else float("nan")
-    e2e = e2e_local
-    if world > 1:
-        t = torch.tensor([e2e_local], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e = float(t.item())
+    e2e = max_over_ranks(statistics.mean(e2e_ms) if e2e_ms else float("nan"), dev)
 
     hbm, bf16_burst, bf16_sus, peak_kind = load_peaks()
     fwd_ms = statistics.mean(per["fwd"])
@@ -303,7 +313,7 @@ def run_ours(args, wl):
                        "gbs": router_bytes / (router_ms * 1e-3) / 1e9, "hbm_frac": router_bytes / (router_ms * 1e-3) / 1e9 / hbm},
             "roofline": {"bound": "tensor", "kernel": "attn_fwd_tc_kernel", "achieved": fwd_tflops,
                          "peak": bf16_sus, "unit": "TFLOP/s", "frac": fwd_tflops / bf16_sus,
-                         "peak_kind": f"{peak_kind} sustained bf16", "traffic": None},
+                         "peak_kind": f"{peak_kind} sustained bf16", "traffic": profiled_traffic(wl, pairs)},
             "cpu_baseline": cpu,
             "e2e": {"value": flops_rank * world / (e2e * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
