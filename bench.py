@@ -20,6 +20,7 @@ import os
 import re
 import statistics
 import subprocess
+import threading
 import sys
 import time
 
@@ -33,7 +34,7 @@ import synthetic as S  # noqa: E402
 METRIC = "VSA2 attn fwd ms & effective TFLOPS, 215K tok H20 D128 top64"
 DEFAULT_WORKLOAD = "720p_top64"
 # kernels of ours launched per call (memsets are not counted)
-LAUNCHES = {"router": 2, "topk": 9, "topk_csc": 11, "fwd": 1, "bwd": 3}
+LAUNCHES = {"router": 2, "topk": 9, "topk_csc": 11, "fwd": 1, "bwd": 2}
 
 
 def load_peaks():
@@ -68,13 +69,49 @@ def pair_flops(wl, pairs, backward):
 
 
 class Clocks:
-    """nvidia-smi sampler running during the timed region."""
+    """Samples the SM clock and the clock-event (throttle) reasons every 20 ms through NVML, in
+    a thread, while the timed region runs (read-only queries; no setting is changed). Falls back
+    to an `nvidia-smi -lms` subprocess when NVML cannot be opened."""
+
+    PERIOD_S = 0.02
 
     def __init__(self, device_index):
-        self.proc = None
         self.device_index = device_index
+        self.samples = []  # (sm_mhz, max_mhz, reasons bitmask)
+        self.proc = None
+        self.lines = []
+        self._stop = threading.Event()
+        self._thread = None
+
+    def _nvml_loop(self, nv, h):
+        while True:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                self.samples.append((float(sm), float(mx), int(get(h))))
+            except Exception:
+                pass
+            if self._stop.wait(self.PERIOD_S):
+                return
 
     def __enter__(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            try:
+                import torch
+                idx = torch.cuda._get_nvml_device_index(self.device_index)
+            except Exception:
+                idx = self.device_index
+            h = nv.nvmlDeviceGetHandleByIndex(idx)
+            self._nv = nv
+            self._thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+            self._thread.start()
+            return self
+        except Exception:
+            self._thread = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.device_index),
@@ -88,7 +125,9 @@ class Clocks:
         return self
 
     def __exit__(self, *a):
-        self.lines = []
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -98,21 +137,35 @@ class Clocks:
                 self.proc.kill()
 
     def summary(self):
-        sm, mx, reasons = [], 0.0, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
-            f = [x.strip() for x in l.split(",")]
-            try:
-                sm.append(float(f[0]))
-                mx = max(mx, float(f[1]))
-            except (ValueError, IndexError):
-                continue
-            for n, v in zip(names, f[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
+        sm, mx, reasons = [], 0.0, set()
+        if self.samples:
+            nv = self._nv
+            bits = {"hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+                    "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+                    "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+                    "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4)}
+            for f_sm, f_mx, r in self.samples:
+                sm.append(f_sm)
+                mx = max(mx, f_mx)
+                reasons.update(n for n in names if r & bits[n])
+            src = "nvml"
+        else:
+            for l in self.lines:
+                f = [x.strip() for x in l.split(",")]
+                try:
+                    sm.append(float(f[0]))
+                    mx = max(mx, float(f[1]))
+                except (ValueError, IndexError):
+                    continue
+                for n, v in zip(names, f[4:8]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+            src = "nvidia-smi"
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm),
+                "source": src}
 
 
 # ----------------------------------------------------------------------------------------------

@@ -161,13 +161,20 @@ def sparse_attn_fwd(q, k, v, kv_off, kv_idx, tile_tokens: int = 64, query_tiles=
     return o.reshape(L, D), lse.reshape(L)
 
 
-def sparse_attn_bwd(q, k, v, do, kv_off, kv_idx, tile_tokens: int = 64):
+def sparse_attn_bwd(q, k, v, do, kv_off, kv_idx, tile_tokens: int = 64, query_tiles=None, o=None):
     """Gradients (dQ, dK, dV) of the Eq. 12 output for one (b, h) given upstream dO.
 
     Textbook softmax-attention backward restricted to the selected tile pairs (the router
     receives no gradient, §2.1): with P the softmax of S = Q K_S^T / sqrt(D) per query row,
     dV_S = P^T dO, dP = dO V_S^T, dS = P * (dP - rowsum(dO * O)), dQ = dS K_S / sqrt(D),
     dK_S = dS^T Q / sqrt(D). The softmax is recomputed here in fp64 from Q, K, V.
+
+    With `query_tiles` given, only those query tiles contribute: dQ is then exact on them, and
+    dK, dV are exact on every KV tile all of whose selecting query tiles are in the subset.
+
+    `o` is the forward output the rowsum(dO * O) term is formed from, as in a backward pass
+    that receives the stored output of the forward (for instance rounded to the storage
+    dtype); by default the exact O recomputed here.
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -177,10 +184,11 @@ def sparse_attn_bwd(q, k, v, do, kv_off, kv_idx, tile_tokens: int = 64):
     N = L // tile_tokens
     scale = 1.0 / np.sqrt(D)
     qt, kt, vt, dot = (_tiles(x, tile_tokens) for x in (q, k, v, do))
+    ot = None if o is None else _tiles(np.asarray(o, dtype=np.float64), tile_tokens)
     dq = np.zeros_like(qt)
     dk = np.zeros_like(kt)
     dv = np.zeros_like(vt)
-    for i in range(N):
+    for i in (range(N) if query_tiles is None else query_tiles):
         sel = np.asarray(kv_idx[kv_off[i]:kv_off[i + 1]])
         if sel.size == 0:
             continue
@@ -189,8 +197,8 @@ def sparse_attn_bwd(q, k, v, do, kv_off, kv_idx, tile_tokens: int = 64):
         s = (qt[i] @ ks.T) * scale
         p = np.exp(s - s.max(axis=1, keepdims=True))
         p /= p.sum(axis=1, keepdims=True)
-        o = p @ vs
-        delta = np.sum(dot[i] * o, axis=1, keepdims=True)
+        oi = p @ vs if ot is None else ot[i]
+        delta = np.sum(dot[i] * oi, axis=1, keepdims=True)
         dvs = p.T @ dot[i]
         dp = dot[i] @ vs.T
         ds = p * (dp - delta)

@@ -79,6 +79,75 @@ def oracle_scores(wl, x, heads=None):
     return out
 
 
+def lists_from_masks(masks, topk):
+    """Boolean tile masks [B, H, N, N] -> padded CSR (kv_off, kv_idx) and CSC (q_off, q_idx)."""
+    B, H, N, _ = masks.shape
+    kv_off = np.zeros((B, H, N + 1), np.int32)
+    kv_idx = np.zeros((B, H, N * topk), np.int32)
+    q_off = np.zeros((B, H, N + 1), np.int32)
+    q_idx = np.zeros((B, H, N * topk), np.int32)
+    for b in range(B):
+        for h in range(H):
+            m = masks[b, h]
+            assert m.sum() <= N * topk
+            kv_off[b, h, 1:] = np.cumsum(m.sum(1))
+            r = np.nonzero(m)[1]
+            kv_idx[b, h, :r.size] = r
+            q_off[b, h, 1:] = np.cumsum(m.sum(0))
+            c = np.nonzero(m.T)[1]
+            q_idx[b, h, :c.size] = c
+    return kv_off, kv_idx, q_off, q_idx
+
+
+def edge_masks(pattern, wl, seed=3):
+    """Selections the method can produce or that stress the kernels' edges: rows with no tile,
+    every tile, one tile per row, and odd list lengths (a half block at the end of a row)."""
+    N = wl.num_tiles
+    rng = np.random.default_rng(seed)
+    masks = np.zeros((wl.batch, wl.heads, N, N), bool)
+    for b in range(wl.batch):
+        for h in range(wl.heads):
+            if pattern == "empty_rows":
+                m = rng.random((N, N)) < wl.topk / N
+                m[::3] = False
+            elif pattern == "dense":
+                m = np.ones((N, N), bool)
+            elif pattern == "single":
+                m = np.zeros((N, N), bool)
+                m[np.arange(N), rng.integers(0, N, N)] = True
+            else:
+                m = np.zeros((N, N), bool)
+                for i in range(N):
+                    m[i, rng.choice(N, size=2 * (i % 5) + 1, replace=False)] = True
+            masks[b, h] = m
+    topk = max(int(np.ceil(masks[b, h].sum() / N)) for b in range(wl.batch) for h in range(wl.heads))
+    return masks, topk
+
+
+_sel480 = {}
+
+
+def c480_lists(heads):
+    """480p selection: the oracle's router + TopK on the heads in `heads`, and on every other
+    head a fixed band pattern (row i takes tiles i + 7t mod N, t < topk), so that the kernels
+    run at full size while the oracle only needs the sampled heads."""
+    wl = C480
+    key = tuple(heads)
+    if key not in _sel480:
+        x = inputs(wl)
+        N = wl.num_tiles
+        masks = np.zeros((1, wl.heads, N, N), bool)
+        for h in range(wl.heads):
+            if h in heads:
+                sc = O.router_scores(x["q"][0, h], x["k"][0, h]).astype(np.float32)
+                masks[0, h] = O.topk_select(sc, wl.topk)["mask"]
+            else:
+                rows = np.repeat(np.arange(N), wl.topk)
+                masks[0, h, rows, (rows + 7 * np.tile(np.arange(wl.topk), N)) % N] = True
+        _sel480[key] = masks
+    return _sel480[key]
+
+
 # ------------------------------------------------------------------------------------------
 # router
 # ------------------------------------------------------------------------------------------
@@ -187,66 +256,91 @@ def test_fwd_on_oracle_selection(wl):
 
 @pytest.mark.parametrize("pattern", ["empty_rows", "dense", "single", "odd_lengths"])
 def test_fwd_edge_selections(pattern):
-    wl = SMALL
-    x = inputs(wl)
-    N = wl.num_tiles
-    rng = np.random.default_rng(3)
-    masks = []
-    for h in range(wl.heads):
-        if pattern == "empty_rows":
-            m = rng.random((N, N)) < wl.topk / N
-            m[::3] = False
-        elif pattern == "dense":
-            m = np.ones((N, N), bool)
-        elif pattern == "single":
-            m = np.zeros((N, N), bool)
-            m[np.arange(N), rng.integers(0, N, N)] = True
-        else:
-            m = np.zeros((N, N), bool)
-            for i in range(N):
-                m[i, rng.choice(N, size=2 * (i % 5) + 1, replace=False)] = True
-        masks.append(m)
-    topk = max(int(np.ceil(m.sum() / N)) for m in masks)
-    wl = wl.with_(topk=topk)
-    kv_off = np.zeros((1, wl.heads, N + 1), np.int32)
-    kv_idx = np.zeros((1, wl.heads, N * topk), np.int32)
-    for h, m in enumerate(masks):
-        kv_off[0, h, 1:] = np.cumsum(m.sum(1))
-        idx = np.nonzero(m)[1]
-        kv_idx[0, h, :idx.size] = idx
-    _fwd_case(wl, x, kv_off, kv_idx)
+    masks, topk = edge_masks(pattern, SMALL)
+    wl = SMALL.with_(topk=topk)
+    kv_off, kv_idx, _, _ = lists_from_masks(masks, topk)
+    _fwd_case(wl, inputs(wl), kv_off, kv_idx)
 
 
 def test_fwd_480p_sampled_heads():
     wl = C480
-    x = inputs(wl)
-    e = engine(wl)
-    q, k = dev(x["q"], "bf16"), dev(x["k"], "bf16")
-    kv_off, kv_idx, _, _ = e.topk_select(e.router_scores(q, k), wl.topk, csc=False)
-    _fwd_case(wl, x, kv_off.cpu().numpy(), kv_idx.cpu().numpy(), heads=[0, 19], tiles=[0, 1, 100, 363, 364, 727])
+    heads = [0, 19]
+    kv_off, kv_idx, _, _ = lists_from_masks(c480_lists(heads), wl.topk)
+    _fwd_case(wl, inputs(wl), kv_off, kv_idx, heads=heads, tiles=[0, 1, 100, 363, 364, 727])
 
 
 # ------------------------------------------------------------------------------------------
 # backward
 # ------------------------------------------------------------------------------------------
+def _bwd_case(wl, x, lists, heads=None, q_tiles=None, kv_tiles=None):
+    """Backward through the C ABI against the oracle. Both sides get the oracle's forward
+    output (rounded to the storage dtype) and LSE, so the rowsum(dO * O) term is formed from
+    the same O. With q_tiles / kv_tiles only the query tiles those gradients depend on are
+    computed by the oracle (dQ of q_tiles, dK / dV of kv_tiles); the forward rows the compared
+    gradients do not depend on are filled from the GPU forward."""
+    kv_off, kv_idx, q_off, q_idx = lists
+    e = engine(wl)
+    q, k, v, do = (dev(x[n], wl.dtype) for n in ("q", "k", "v", "do"))
+    t = lambda a: torch.from_numpy(a).cuda()
+    o_gpu, lse_gpu = e.attn_fwd(q, k, v, t(kv_off), t(kv_idx))
+    o_in = o_gpu.float().cpu().numpy()
+    lse_in = lse_gpu.cpu().numpy()
+    todo = {}
+    for b in range(wl.batch):
+        for h in (range(wl.heads) if heads is None else heads):
+            if q_tiles is None:
+                need = list(range(wl.num_tiles))
+            else:
+                need = set(q_tiles)
+                for j in kv_tiles:
+                    need.update(q_idx[b, h, q_off[b, h, j]:q_off[b, h, j + 1]].tolist())
+                need = sorted(need)
+            wo, wlse = O.sparse_attn_fwd(x["q"][b, h], x["k"][b, h], x["v"][b, h], kv_off[b, h], kv_idx[b, h],
+                                         query_tiles=need)
+            rows = np.concatenate([np.arange(64 * i, 64 * i + 64) for i in need])
+            o_in[b, h][rows] = S.round_to_dtype(wo[rows], wl.dtype)
+            lse_in[b, h][rows] = wlse[rows]
+            todo[(b, h)] = need
+    dq, dk, dv = e.attn_bwd(q, k, v, dev(o_in, wl.dtype), torch.from_numpy(lse_in).cuda(), do, t(kv_off), t(kv_idx),
+                            t(q_off), t(q_idx))
+    assert e.device_error() == 0
+    dq, dk, dv = (g.cpu().numpy() for g in (dq, dk, dv))
+    for (b, h), need in todo.items():
+        want = O.sparse_attn_bwd(x["q"][b, h], x["k"][b, h], x["v"][b, h], x["do"][b, h], kv_off[b, h],
+                                 kv_idx[b, h], query_tiles=None if q_tiles is None else need, o=o_in[b, h])
+        if q_tiles is None:
+            for name, g, w in zip(("dq", "dk", "dv"), (dq, dk, dv), want):
+                assert_attn_close(g[b, h], w, f"{name}[{b},{h}]")
+            continue
+        qr = np.concatenate([np.arange(64 * i, 64 * i + 64) for i in q_tiles])
+        kr = np.concatenate([np.arange(64 * j, 64 * j + 64) for j in kv_tiles])
+        assert_attn_close(dq[b, h][qr], want[0][qr], f"dq[{b},{h}]")
+        assert_attn_close(dk[b, h][kr], want[1][kr], f"dk[{b},{h}]")
+        assert_attn_close(dv[b, h][kr], want[2][kr], f"dv[{b},{h}]")
+
+
 @pytest.mark.parametrize("wl", [TINY, SMALL, SMALL64], ids=["tiny_fp32", "small_bf16", "small_bf16_d64"])
 def test_bwd_on_oracle_selection(wl):
     x = inputs(wl, ("q", "k", "v", "do"))
     sc = oracle_scores(wl, x)
     s32 = np.stack([np.stack([sc[(b, h)] for h in range(wl.heads)]) for b in range(wl.batch)]).astype(np.float32)
-    kv_off, kv_idx, q_off, q_idx = oracle_csr(wl, s32)
-    e = engine(wl)
-    q, k, v, do = (dev(x[n], wl.dtype) for n in ("q", "k", "v", "do"))
-    t = lambda a: torch.from_numpy(a).cuda()
-    o, lse = e.attn_fwd(q, k, v, t(kv_off), t(kv_idx))
-    dq, dk, dv = e.attn_bwd(q, k, v, o, lse, do, t(kv_off), t(kv_idx), t(q_off), t(q_idx))
-    assert e.device_error() == 0
-    for b in range(wl.batch):
-        for h in range(wl.heads):
-            want = O.sparse_attn_bwd(x["q"][b, h], x["k"][b, h], x["v"][b, h], x["do"][b, h], kv_off[b, h],
-                                     kv_idx[b, h])
-            for name, g, w in zip(("dq", "dk", "dv"), (dq, dk, dv), want):
-                assert_attn_close(g[b, h].cpu().numpy(), w, f"{name}[{b},{h}]")
+    _bwd_case(wl, x, oracle_csr(wl, s32))
+
+
+@pytest.mark.parametrize("pattern", ["empty_rows", "dense", "single", "odd_lengths"])
+def test_bwd_edge_selections(pattern):
+    masks, topk = edge_masks(pattern, SMALL)
+    wl = SMALL.with_(topk=topk)
+    lists = lists_from_masks(masks, topk)
+    _bwd_case(wl, inputs(wl, ("q", "k", "v", "do")), lists)
+
+
+def test_bwd_480p_sampled():
+    wl = C480
+    heads = [0, 19]
+    lists = lists_from_masks(c480_lists(heads), wl.topk)
+    _bwd_case(wl, inputs(wl, ("q", "k", "v", "do")), lists, heads=heads, q_tiles=[0, 363, 727],
+              kv_tiles=[0, 364, 727])
 
 
 def test_autograd_function_matches_explicit_calls():

@@ -366,3 +366,55 @@ def test_bwd_invariants():
     np.testing.assert_allclose(dk.sum(0), 0, atol=1e-11)
     live = np.repeat(mask.any(1), 64)
     np.testing.assert_allclose(dv.sum(0), do[live].sum(0), rtol=1e-12, atol=1e-11)
+
+
+def test_bwd_query_tile_subset_is_exact_where_complete():
+    """Restricting the backward to a subset of query tiles leaves dQ on those tiles, and dK, dV
+    on every KV tile selected only by tiles of the subset, equal to the full computation."""
+    rng = np.random.default_rng(15)
+    L, D = 6 * 64, 16
+    q, k, v, do = (rng.standard_normal((L, D)) for _ in range(4))
+    mask = rng.random((6, 6)) < 0.45
+    mask[:, 4] = False
+    mask[[0, 5], 4] = True  # KV tile 4 is selected by query tiles 0 and 5 only
+    off, idx = _csr(mask)
+    full = O.sparse_attn_bwd(q, k, v, do, off, idx)
+    sub = O.sparse_attn_bwd(q, k, v, do, off, idx, query_tiles=[0, 5])
+    for i in (0, 5):
+        np.testing.assert_array_equal(sub[0][64 * i:64 * i + 64], full[0][64 * i:64 * i + 64])
+    for g_sub, g_full in zip(sub[1:], full[1:]):
+        np.testing.assert_allclose(g_sub[256:320], g_full[256:320], rtol=1e-12, atol=1e-13)
+    assert np.all(sub[0][64:256] == 0)
+
+
+def test_bwd_given_output_enters_only_through_rowsum():
+    """Passing the exact forward output reproduces the default; the output only enters through
+    rowsum(dO * O): a change orthogonal to each dO row changes nothing, and dV never depends
+    on it. A change along dO shifts dQ by the closed form -P (dO . u) K / sqrt(D) per row."""
+    rng = np.random.default_rng(16)
+    L, D = 4 * 64, 16
+    q, k, v, do = (rng.standard_normal((L, D)) for _ in range(4))
+    mask = rng.random((4, 4)) < 0.6
+    mask[:, 1] = True
+    off, idx = _csr(mask)
+    o, _ = O.sparse_attn_fwd(q, k, v, off, idx)
+    base = O.sparse_attn_bwd(q, k, v, do, off, idx)
+    same = O.sparse_attn_bwd(q, k, v, do, off, idx, o=o)
+    for a, b in zip(base, same):
+        np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+    u = rng.standard_normal((L, D))
+    u -= (np.sum(u * do, 1) / np.sum(do * do, 1))[:, None] * do  # orthogonal to dO, row by row
+    orth = O.sparse_attn_bwd(q, k, v, do, off, idx, o=o + 3.0 * u)
+    for a, b in zip(base, orth):
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-11)
+    shift = O.sparse_attn_bwd(q, k, v, do, off, idx, o=o + 0.5 * do)
+    np.testing.assert_array_equal(shift[2], base[2])
+    # row t of tile i: Delta grows by 0.5 |dO_t|^2, so dS_t drops by 0.5 |dO_t|^2 P_t
+    i = 0
+    sel = idx[off[i]:off[i + 1]]
+    ks = k.reshape(4, 64, D)[sel].reshape(-1, D)
+    s = q[:64] @ ks.T / math.sqrt(D)
+    p = np.exp(s - s.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    want = base[0][:64] - (0.5 * np.sum(do[:64] ** 2, 1))[:, None] * (p @ ks) / math.sqrt(D)
+    np.testing.assert_allclose(shift[0][:64], want, rtol=1e-10, atol=1e-11)

@@ -79,10 +79,21 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
+static thread_local int g_encode_result = 0;
+
+// The encoder is a driver call: make the current device's primary context current on this
+// thread first (a thread that has issued no runtime call yet, such as an autograd worker whose
+// tensors all came from a caching allocator, may have none).
+static bool bind_context() {
+  int dev = 0;
+  return cudaGetDevice(&dev) == cudaSuccess && cudaSetDevice(dev) == cudaSuccess;
+}
+
 bool make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t outer,
                        uint32_t box_cols, uint32_t box_rows) {
   auto enc = get_encode();
-  if (!enc) return false;
+  g_encode_result = -1;
+  if (!enc || !bind_context()) return false;
   cuuint64_t dims[3] = {cols, rows, outer};
   cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
   cuuint32_t box[3] = {box_cols, box_rows, 1};
@@ -90,13 +101,15 @@ bool make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  g_encode_result = (int)r;
   return r == CUDA_SUCCESS;
 }
 
 bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
                        uint32_t box_rows) {
   auto enc = get_encode();
-  if (!enc) return false;
+  g_encode_result = -1;
+  if (!enc || !bind_context()) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
   cuuint32_t box[2] = {box_cols, box_rows};
@@ -104,6 +117,7 @@ bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  g_encode_result = (int)r;
   return r == CUDA_SUCCESS;
 }
 
@@ -112,6 +126,13 @@ static thread_local char g_msg[256];
 
 vsa2_status cuda_fail(const char* what) {
   g_last_cuda_error.store(what);
+  return VSA2_ERR_CUDA;
+}
+
+vsa2_status tmap_fail(const char* what) {
+  snprintf(g_msg, sizeof(g_msg), "%s (cuTensorMapEncodeTiled result %d, -1 = no encoder or no context)", what,
+           g_encode_result);
+  g_last_cuda_error.store(g_msg);
   return VSA2_ERR_CUDA;
 }
 

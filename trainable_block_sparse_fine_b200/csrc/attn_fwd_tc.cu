@@ -401,7 +401,7 @@ vsa2_status attn_fwd_tc(const Dims& d, const void* q, const void* k, const void*
   CUtensorMap tk, tv;
   const uint64_t rows = (uint64_t)d.BH * d.L;
   if (!make_tmap_2d_bf16(&tk, k, 128, rows, 64, 64) || !make_tmap_2d_bf16(&tv, v, 128, rows, 64, 64))
-    return cuda_fail("tensor map encoding for the attention operands failed");
+    return tmap_fail("tensor map encoding for the attention operands failed");
   DevCtx ctx{reinterpret_cast<int*>(ws), d.timeout_ns, d.flags};
   const int items = d.BH * d.N;
   int sms = 148;

@@ -35,6 +35,8 @@ vsa2_status launch_attn_bwd(const Dims& d, const void* q, const void* k, const v
                             const float* lse, const void* dout, int topk, const int32_t* kv_off,
                             const int32_t* kv_idx, const int32_t* q_off, const int32_t* q_idx, float* dq, float* dk,
                             float* dv, char* ws, cudaStream_t s) {
+  if (d.dtype == VSA2_BF16 && d.D == 128)
+    return attn_bwd_tc(d, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, topk, ws, s);
   return attn_bwd_simt(d, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, topk, ws, s);
 }
 

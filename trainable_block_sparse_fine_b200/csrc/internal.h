@@ -71,6 +71,10 @@ vsa2_status attn_bwd_simt(const Dims& d, const void* q, const void* k, const voi
 vsa2_status attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v, int topk,
                         const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
                         cudaStream_t s);
+// tensor-core backward (bf16, head_dim 128): dQ kernel (also writes Delta), then dK/dV kernel
+vsa2_status attn_bwd_tc(const Dims& d, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, const int32_t* kv_off, const int32_t* kv_idx, const int32_t* q_off,
+                        const int32_t* q_idx, float* dq, float* dk, float* dv, int topk, char* ws, cudaStream_t s);
 vsa2_status launch_wait_timeout_probe(int* err, uint64_t timeout_ns, cudaStream_t s);
 // allocation-free TopK (scratch in a fixed device array of the library)
 size_t topk_noalloc_bytes(const Dims& d);
@@ -82,6 +86,8 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Records the message of a failed CUDA call (see vsa2_last_cuda_error) and returns VSA2_ERR_CUDA.
 vsa2_status cuda_fail(const char* what);
+// Records a failed tensor-map encoding (with the driver's result code) and returns VSA2_ERR_CUDA.
+vsa2_status tmap_fail(const char* what);
 // VSA2_OK if the last launch succeeded, else records the CUDA error and returns VSA2_ERR_CUDA.
 vsa2_status check_launch(const char* what);
 

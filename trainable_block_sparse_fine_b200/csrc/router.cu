@@ -378,8 +378,8 @@ vsa2_status launch_router(const Dims& d, const void* q, const void* k, float* sc
 
   if (d.dtype == VSA2_BF16) {
     CUtensorMap tq, tk;
-    if (!make_tmap_3d_bf16(&tq, qr, d.D, d.Lr, d.BH, 64, RS_M)) return cuda_fail("tensor map encoding (Qr) failed");
-    if (!make_tmap_3d_bf16(&tk, kr, d.D, d.Lr, d.BH, 64, RS_N)) return cuda_fail("tensor map encoding (Kr) failed");
+    if (!make_tmap_3d_bf16(&tq, qr, d.D, d.Lr, d.BH, 64, RS_M)) return tmap_fail("tensor map encoding (Qr) failed");
+    if (!make_tmap_3d_bf16(&tk, kr, d.D, d.Lr, d.BH, 64, RS_N)) return tmap_fail("tensor map encoding (Kr) failed");
     const float c2 = 1.4426950408889634f / sqrtf((float)d.D);
     dim3 grid((d.Lr + RS_M - 1) / RS_M, d.BH);
     if (d.D == 128) {
