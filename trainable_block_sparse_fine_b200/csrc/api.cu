@@ -62,6 +62,7 @@ WsLayout ws_layout(const Dims& d) {
   w.words = (d.N + 31) / 32;
   w.col_bits = take((size_t)d.BH * d.N * w.words * 4);
   w.delta = take((size_t)d.BH * d.L * 4);
+  w.nlse2 = take((size_t)d.BH * d.L * 4);
   w.total = off;
   return w;
 }

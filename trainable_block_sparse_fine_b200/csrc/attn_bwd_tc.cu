@@ -24,7 +24,8 @@
 namespace vsa2 {
 namespace {
 
-constexpr int BT = 352;            // 11 warps: 0-7 two softmax warpgroups, 8/10 producers, 9 MMA
+constexpr int BT = 352;            // dQ kernel: 11 warps (0-7 softmax, 8/10 producers, 9 MMA)
+constexpr int BT_KV = 384;         // dK/dV kernel: 12 warps (0-7 softmax, 8/10 producers, 9/11 MMA)
 constexpr uint32_t TILE_B = 8192;  // one 64 x 64 bf16 box (64 rows x 128 B, 128-byte swizzle)
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -138,17 +139,19 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 512, "barrier area");
 
-// dS for 64 columns (32 per thread, columns 2j + par_c of the half), packed to 16 bf16 words
-__device__ __forceinline__ void ds_half(const uint32_t (&sv)[32], const uint32_t (&dp)[32], float c2, float lse2,
-                                        float dlt, int par_c, uint32_t* pk) {
+// dS for 64 columns (32 per thread, columns 2j + par_c of the half), packed to 16 bf16 words.
+// nl2 = -lse * log2(e), nd = -Delta; the two columns of a step go through packed fp32 math.
+__device__ __forceinline__ void ds_half(const uint32_t (&sv)[32], const uint32_t (&dp)[32], float c2, float nl2,
+                                        float nd, int par_c, uint32_t* pk) {
+  const float2 cc = make_float2(c2, c2), ll = make_float2(nl2, nl2), dd = make_float2(nd, nd);
 #pragma unroll
   for (int i2 = 0; i2 < 16; ++i2) {
-    const float pa = ex2(fmaf(__uint_as_float(sv[2 * i2]), c2, -lse2));
-    const float pb = ex2(fmaf(__uint_as_float(sv[2 * i2 + 1]), c2, -lse2));
-    const float da = pa * (__uint_as_float(dp[2 * i2]) - dlt);
-    const float db = pb * (__uint_as_float(dp[2 * i2 + 1]) - dlt);
-    const float recv = __shfl_xor_sync(0xffffffffu, par_c ? da : db, 2);
-    pk[i2] = par_c ? pack_bf16(recv, db) : pack_bf16(da, recv);
+    const float2 arg = __ffma2_rn(make_float2(__uint_as_float(sv[2 * i2]), __uint_as_float(sv[2 * i2 + 1])), cc, ll);
+    const float2 p = make_float2(ex2(arg.x), ex2(arg.y));
+    const float2 ds =
+        __fmul2_rn(p, __fadd2_rn(make_float2(__uint_as_float(dp[2 * i2]), __uint_as_float(dp[2 * i2 + 1])), dd));
+    const float recv = __shfl_xor_sync(0xffffffffu, par_c ? ds.x : ds.y, 2);
+    pk[i2] = par_c ? pack_bf16(recv, ds.y) : pack_bf16(ds.x, recv);
   }
 }
 }  // namespace dqk
@@ -157,7 +160,7 @@ __global__ void __launch_bounds__(BT, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const __nv_bfloat16* __restrict__ qg, const __nv_bfloat16* __restrict__ og,
                           const __nv_bfloat16* __restrict__ dog, const float* __restrict__ lse,
-                          float* __restrict__ delta, const int32_t* __restrict__ kv_off,
+                          float* __restrict__ ndelta, float* __restrict__ nlse2, const int32_t* __restrict__ kv_off,
                           const int32_t* __restrict__ kv_idx, float* __restrict__ dq_out, int N, int L, int topk,
                           int items, float c2, float scale, DevCtx ctx) {
   using namespace dqk;
@@ -340,8 +343,13 @@ __global__ void __launch_bounds__(BT, 1)
         tmem_st16x64b_x32(tl + TM_DO, v);
         dlt = part + __shfl_xor_sync(0xffffffffu, part, 2);
       }
-      if (par_c == 0) delta[tok] = dlt;
-      const float lse2 = lse[tok] * kLog2e;
+      const float nl2 = -lse[tok] * kLog2e;
+      if (par_c == 0) {
+        // for the dK/dV kernel: each tile's 64 values ordered even rows, then odd rows
+        const size_t perm = (size_t)bh * L + (size_t)qt * 64 + (row & 1) * 32 + (row >> 1);
+        ndelta[perm] = -dlt;
+        nlse2[perm] = nl2;
+      }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -356,14 +364,14 @@ __global__ void __launch_bounds__(BT, 1)
           tmem_ld16x64b_x32(tl + TM_S, sv);
           tmem_ld16x64b_x32(tl + TM_DP, dp);
           tmem_ld_wait();
-          ds_half(sv, dp, c2, lse2, dlt, par_c, pk);
+          ds_half(sv, dp, c2, nl2, -dlt, par_c, pk);
         }
         if (!half) {
           uint32_t sv[32], dp[32];
           tmem_ld16x64b_x32(tl + TM_S + 64, sv);
           tmem_ld16x64b_x32(tl + TM_DP + 64, dp);
           tmem_ld_wait();
-          ds_half(sv, dp, c2, lse2, dlt, par_c, pk + 16);
+          ds_half(sv, dp, c2, nl2, -dlt, par_c, pk + 16);
         } else {
 #pragma unroll
           for (int i = 16; i < 32; ++i) pk[i] = 0u;
@@ -408,18 +416,20 @@ constexpr uint32_t TM_K = 0, TM_V = 64, TM_S = 128, TM_DP = 192, TM_DV = 256, TM
 struct Bars {
   uint64_t full[2 * RST], empty[2 * RST];
   uint64_t sfull[2], pfull[2], bdone[2], kvready[2];
-  uint64_t done;
+  uint64_t done[2];
 };
 static_assert(sizeof(Bars) <= 512, "barrier area");
 }  // namespace dkv
 
-__global__ void __launch_bounds__(BT, 1)
+// The two slots are independent pipelines that share only the tensor pipe: slot s has its own
+// producer warp (8 + 2s) and its own MMA-issuing warp (9 + 2s), so neither waits on the other.
+__global__ void __launch_bounds__(BT_KV, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                             const __nv_bfloat16* __restrict__ kg, const __nv_bfloat16* __restrict__ vg,
-                            const float* __restrict__ lse, const float* __restrict__ delta,
+                            const float* __restrict__ nlse2, const float* __restrict__ ndelta,
                             const int32_t* __restrict__ q_off, const int32_t* __restrict__ q_idx,
                             float* __restrict__ dk_out, float* __restrict__ dv_out, int N, int L, int topk, int items,
-                            float c1, float scale, DevCtx ctx) {
+                            float c2, float scale, DevCtx ctx) {
   using namespace dkv;
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
   uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
@@ -432,14 +442,14 @@ __global__ void __launch_bounds__(BT, 1)
 
   if (threadIdx.x == 0) {
     flag_sh[0] = 0;
-    for (int i = 0; i < 2 * RST; ++i) mbar_init(&B.full[i], 2), mbar_init(&B.empty[i], 1);
+    for (int i = 0; i < 2 * RST; ++i) mbar_init(&B.full[i], 1), mbar_init(&B.empty[i], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&B.sfull[s], 1);
       mbar_init(&B.pfull[s], 4);
       mbar_init(&B.bdone[s], 1);
       mbar_init(&B.kvready[s], 4);
+      mbar_init(&B.done[s], 1);
     }
-    mbar_init(&B.done, 1);
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -452,106 +462,95 @@ __global__ void __launch_bounds__(BT, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(flag_sh + 4);
 
   if (warp == 8 || warp == 10) {
-    // ------------------------------------------------------------------ producers (lane 0)
-    // warp 8: Q tile + lse, warp 10: dO tile + Delta, of each selected query tile, into the
-    // slot's own ring (stage = the slot's tile count mod RST)
+    // ------------------------------------------------------------------ producer of slot (warp - 8) / 2
+    // per selected query tile: its Q and dO tiles (two boxes each) and its 64 -lse*log2(e) and
+    // -Delta values (written by the dQ kernel), into the slot's ring (stage = the slot's tile count mod RST)
     if (lane == 0) {
-      const bool q_role = warp == 8;
-      const CUtensorMap* map = q_role ? &tm_q : &tm_do;
-      const float* rowvec = q_role ? lse : delta;
-      const uint32_t off_t = q_role ? 0u : 2 * TILE_B;
-      const uint32_t off_v = 4 * TILE_B + (q_role ? 0u : 256u);
-      tma_prefetch_desc(map);
-      Seq sq[2];
-      sq[0].init(2 * blockIdx.x, step, items);
-      sq[1].init(2 * blockIdx.x + 1, step, items);
-      int cnt[2] = {0, 0};
+      const int s = (warp - 8) >> 1;
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_do);
+      Seq sq;
+      sq.init(2 * blockIdx.x + s, step, items);
+      int cnt = 0;
       bool ok = true;
-      while (ok && (sq[0].active || sq[1].active)) {
-#pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          if (!ok) break;
-          int blk;
-          if (next_op(sq[s], &blk, q_off, N, cap, 1, ctx) != 1) continue;
-          const Seq& q = sq[s];
-          int i = q_idx[(size_t)q.bh * cap + q.beg + blk];
-          if (i < 0 || i >= N) {
-            if (ctx.flags & VSA2_FLAG_VALIDATE) set_error(ctx.err, VSA2_ERR_BAD_INDEX);
-            i = min(max(i, 0), N - 1);
-          }
-          const int r = s * RST + cnt[s] % RST;
-          if (!(ok = mbar_wait(&B.empty[r], ((cnt[s] / RST) & 1) ^ 1, abort, ctx))) break;
-          uint8_t* stage = dsm + r * STAGE_B;
-          const int row0 = q.bh * L + i * 64;
-          mbar_arrive_expect_tx(&B.full[r], 2 * TILE_B + 256);
-          tma_load_2d(stage + off_t, map, 0, row0, &B.full[r]);
-          tma_load_2d(stage + off_t + TILE_B, map, 64, row0, &B.full[r]);
-          bulk_load(stage + off_v, rowvec + row0, 256, &B.full[r]);
-          ++cnt[s];
+      while (ok && sq.active) {
+        int blk;
+        if (next_op(sq, &blk, q_off, N, cap, 1, ctx) != 1) continue;
+        int i = q_idx[(size_t)sq.bh * cap + sq.beg + blk];
+        if (i < 0 || i >= N) {
+          if (ctx.flags & VSA2_FLAG_VALIDATE) set_error(ctx.err, VSA2_ERR_BAD_INDEX);
+          i = min(max(i, 0), N - 1);
         }
+        const int r = s * RST + cnt % RST;
+        if (!(ok = mbar_wait(&B.empty[r], ((cnt / RST) & 1) ^ 1, abort, ctx))) break;
+        uint8_t* stage = dsm + r * STAGE_B;
+        const int row0 = sq.bh * L + i * 64;
+        mbar_arrive_expect_tx(&B.full[r], 4 * TILE_B + 512);
+        tma_load_2d(stage, &tm_q, 0, row0, &B.full[r]);
+        tma_load_2d(stage + TILE_B, &tm_q, 64, row0, &B.full[r]);
+        tma_load_2d(stage + 2 * TILE_B, &tm_do, 0, row0, &B.full[r]);
+        tma_load_2d(stage + 3 * TILE_B, &tm_do, 64, row0, &B.full[r]);
+        bulk_load(stage + 4 * TILE_B, nlse2 + row0, 256, &B.full[r]);
+        bulk_load(stage + 4 * TILE_B + 256, ndelta + row0, 256, &B.full[r]);
+        ++cnt;
       }
-      if (*abort) {  // let copies still in flight land before the CTA exits
-        for (int s = 0; s < 2; ++s)
-          for (int cc = max(0, cnt[s] - RST); cc < cnt[s]; ++cc)
-            mbar_wait_drain(&B.full[s * RST + cc % RST], (cc / RST) & 1, ctx.timeout_ns);
-      }
+      if (*abort)  // let copies still in flight land before the CTA exits
+        for (int cc = max(0, cnt - RST); cc < cnt; ++cc)
+          mbar_wait_drain(&B.full[s * RST + cc % RST], (cc / RST) & 1, ctx.timeout_ns);
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == 9 || warp == 11) {
+    // ------------------------------------------------------------------ MMA issuer of slot (warp - 9) / 2
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16_f32(64, 64, false, false);  // S^T, dP^T: N = 64 queries
       constexpr uint32_t id_g = idesc_bf16_f32(64, 128, false, true);  // dV, dK: N = 128 (d)
-      Seq sq[2];
-      sq[0].init(2 * blockIdx.x, step, items);
-      sq[1].init(2 * blockIdx.x + 1, step, items);
-      int ga[2] = {0, 0}, gb[2] = {0, 0};
+      const int s = (warp - 9) >> 1;
+      const uint32_t lanes = (uint32_t)(16 * s) << 16;
+      Seq sq;
+      sq.init(2 * blockIdx.x + s, step, items);
+      int ga = 0, gb = 0;
       bool ok = true;
-      while (ok && (sq[0].active || sq[1].active)) {
+      while (ok && sq.active) {
+        int blk;
+        const int op = next_op(sq, &blk, q_off, N, cap, 1, ctx);
+        if (op == 1) {
+          if (blk == 0 && !(ok = mbar_wait(&B.kvready[s], (sq.tile - 1) & 1, abort, ctx))) break;
+          // S^T / dP^T are free once the previous dV / dK MMAs (which read P^T / dS^T) are done
+          if (ga > 0 && !(ok = mbar_wait(&B.bdone[s], (ga - 1) & 1, abort, ctx))) break;
+          const int r = s * RST + ga % RST;
+          if (!(ok = mbar_wait(&B.full[r], (ga / RST) & 1, abort, ctx))) break;
+          tc_fence_after();
+          const uint32_t qa = smem_u32(dsm + r * STAGE_B), da = qa + 2 * TILE_B;
 #pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          if (!ok) break;
-          int blk;
-          const int op = next_op(sq[s], &blk, q_off, N, cap, 1, ctx);
-          if (op == 0) continue;
-          const uint32_t lanes = (uint32_t)(16 * s) << 16;
-          if (op == 1) {
-            if (blk == 0 && !(ok = mbar_wait(&B.kvready[s], (sq[s].tile - 1) & 1, abort, ctx))) break;
-            if (ga[s] > 0 && !(ok = mbar_wait(&B.bdone[s], (ga[s] - 1) & 1, abort, ctx))) break;
-            const int r = s * RST + ga[s] % RST;
-            if (!(ok = mbar_wait(&B.full[r], (ga[s] / RST) & 1, abort, ctx))) break;
-            tc_fence_after();
-            const uint32_t qa = smem_u32(dsm + r * STAGE_B), da = qa + 2 * TILE_B;
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ts(tmem + lanes + TM_S, tmem + lanes + TM_K + 8 * kk,
+                        sdesc_sw128(qa + (kk >> 2) * TILE_B + (kk & 3) * 32, 16, 1024), id_s, kk > 0);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_bf16_ts(tmem + lanes + TM_S, tmem + lanes + TM_K + 8 * kk,
-                          sdesc_sw128(qa + (kk >> 2) * TILE_B + (kk & 3) * 32, 16, 1024), id_s, kk > 0);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ts(tmem + lanes + TM_DP, tmem + lanes + TM_V + 8 * kk,
+                        sdesc_sw128(da + (kk >> 2) * TILE_B + (kk & 3) * 32, 16, 1024), id_s, kk > 0);
+          mma_commit(&B.sfull[s]);
+          ++ga;
+        } else if (op == 2) {
+          // dV += P^T dO, dK += dS^T Q; P^T / dS^T in TMEM (bf16), dO / Q read MN-major
+          if (!(ok = mbar_wait(&B.pfull[s], gb & 1, abort, ctx))) break;
+          tc_fence_after();
+          const int r = s * RST + gb % RST;
+          const uint32_t qa = smem_u32(dsm + r * STAGE_B), da = qa + 2 * TILE_B;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_bf16_ts(tmem + lanes + TM_DP, tmem + lanes + TM_V + 8 * kk,
-                          sdesc_sw128(da + (kk >> 2) * TILE_B + (kk & 3) * 32, 16, 1024), id_s, kk > 0);
-            mma_commit(&B.sfull[s]);
-            ++ga[s];
-          } else {
-            if (!(ok = mbar_wait(&B.pfull[s], gb[s] & 1, abort, ctx))) break;
-            tc_fence_after();
-            const int r = s * RST + gb[s] % RST;
-            const uint32_t qa = smem_u32(dsm + r * STAGE_B), da = qa + 2 * TILE_B;
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ts(tmem + lanes + TM_DV, tmem + lanes + TM_S + 8 * kk, sdesc_sw128(da + kk * 2048, TILE_B, 1024),
+                        id_g, (blk > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ts(tmem + lanes + TM_DV, tmem + lanes + TM_S + 8 * kk, sdesc_sw128(da + kk * 2048, TILE_B, 1024),
-                          id_g, (blk > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ts(tmem + lanes + TM_DK, tmem + lanes + TM_DP + 8 * kk, sdesc_sw128(qa + kk * 2048, TILE_B, 1024),
-                          id_g, (blk > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(&B.empty[r]);
-            mma_commit(&B.bdone[s]);
-            ++gb[s];
-          }
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ts(tmem + lanes + TM_DK, tmem + lanes + TM_DP + 8 * kk, sdesc_sw128(qa + kk * 2048, TILE_B, 1024),
+                        id_g, (blk > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&B.empty[r]);
+          mma_commit(&B.bdone[s]);
+          ++gb;
         }
       }
-      mma_commit(&B.done);
-      mbar_wait_drain(&B.done, 0, ctx.timeout_ns);
+      mma_commit(&B.done[s]);
+      mbar_wait_drain(&B.done[s], 0, ctx.timeout_ns);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax, one slot per warpgroup
@@ -587,27 +586,27 @@ __global__ void __launch_bounds__(BT, 1)
         // the stage's lse / Delta were written by the bulk copy: observe its barrier too
         mbar_wait(&B.full[r], (g / RST) & 1, abort, ctx);
         tc_fence_after();
-        const float4* lse4 = reinterpret_cast<const float4*>(dsm + r * STAGE_B + 4 * TILE_B);
-        const float4* dlt4 = lse4 + 16;
+        // this thread's query columns are 4*i2 + par_c and 4*i2 + 2 + par_c: in the even/odd
+        // order of the stage they are one aligned float2
+        const float2* nl2 = reinterpret_cast<const float2*>(dsm + r * STAGE_B + 4 * TILE_B) + par_c * 16;
+        const float2* nd2 = nl2 + 32;
         uint32_t sv[32], dp[32];
         tmem_ld16x64b_x32(tl + TM_S, sv);
         tmem_ld16x64b_x32(tl + TM_DP, dp);
         tmem_ld_wait();
+        const float2 cc = make_float2(c2, c2);
         uint32_t pk[16], dk[16];
 #pragma unroll
         for (int i2 = 0; i2 < 16; ++i2) {
-          // values 2*i2, 2*i2+1 are queries 4*i2 + par_c and 4*i2 + 2 + par_c
-          const float4 l4 = lse4[i2], d4 = dlt4[i2];
-          const float la = par_c ? l4.y : l4.x, lb = par_c ? l4.w : l4.z;
-          const float ea = par_c ? d4.y : d4.x, eb = par_c ? d4.w : d4.z;
-          const float pa = ex2(fmaf(__uint_as_float(sv[2 * i2]), c1, -la) * kLog2e);
-          const float pb = ex2(fmaf(__uint_as_float(sv[2 * i2 + 1]), c1, -lb) * kLog2e);
-          const float da = pa * (__uint_as_float(dp[2 * i2]) - ea);
-          const float db = pb * (__uint_as_float(dp[2 * i2 + 1]) - eb);
-          const float rp = __shfl_xor_sync(0xffffffffu, par_c ? pa : pb, 2);
-          const float rd = __shfl_xor_sync(0xffffffffu, par_c ? da : db, 2);
-          pk[i2] = par_c ? pack_bf16(rp, pb) : pack_bf16(pa, rp);
-          dk[i2] = par_c ? pack_bf16(rd, db) : pack_bf16(da, rd);
+          const float2 arg =
+              __ffma2_rn(make_float2(__uint_as_float(sv[2 * i2]), __uint_as_float(sv[2 * i2 + 1])), cc, nl2[i2]);
+          const float2 p = make_float2(ex2(arg.x), ex2(arg.y));
+          const float2 ds = __fmul2_rn(
+              p, __fadd2_rn(make_float2(__uint_as_float(dp[2 * i2]), __uint_as_float(dp[2 * i2 + 1])), nd2[i2]));
+          const float rp = __shfl_xor_sync(0xffffffffu, par_c ? p.x : p.y, 2);
+          const float rd = __shfl_xor_sync(0xffffffffu, par_c ? ds.x : ds.y, 2);
+          pk[i2] = par_c ? pack_bf16(rp, p.y) : pack_bf16(p.x, rp);
+          dk[i2] = par_c ? pack_bf16(rd, ds.y) : pack_bf16(ds.x, rd);
         }
         tmem_st16x64b_x16(tl + TM_S, pk);
         tmem_st16x64b_x16(tl + TM_DP, dk);
@@ -650,7 +649,8 @@ vsa2_status attn_bwd_tc(const Dims& d, const void* q, const void* k, const void*
       !make_tmap_2d_bf16(&tq, q, 128, rows, 64, 64) || !make_tmap_2d_bf16(&tdo, dout, 128, rows, 64, 64))
     return tmap_fail("tensor map encoding for the backward operands failed");
   DevCtx ctx{reinterpret_cast<int*>(ws), d.timeout_ns, d.flags};
-  float* delta = reinterpret_cast<float*>(ws + ws_layout(d).delta);
+  float* ndelta = reinterpret_cast<float*>(ws + ws_layout(d).delta);
+  float* nlse2 = reinterpret_cast<float*>(ws + ws_layout(d).nlse2);
   const int items = d.BH * d.N;
   int sms = 148;
   int dev = 0;
@@ -660,13 +660,13 @@ vsa2_status attn_bwd_tc(const Dims& d, const void* q, const void* k, const void*
   const float c2 = kLog2e * c1;
   cudaFuncSetAttribute(attn_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dqk::SMEM_DYN);
   attn_bwd_dq_tc_kernel<<<grid, BT, dqk::SMEM_DYN, s>>>(
-      tk, tv, (const __nv_bfloat16*)q, (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, lse, delta, kv_off, kv_idx,
-      dq, d.N, (int)d.L, topk, items, c2, c1, ctx);
+      tk, tv, (const __nv_bfloat16*)q, (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, lse, ndelta, nlse2, kv_off,
+      kv_idx, dq, d.N, (int)d.L, topk, items, c2, c1, ctx);
   if (check_launch("attn_bwd_dq_tc_kernel") != VSA2_OK) return VSA2_ERR_CUDA;
   cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dkv::SMEM_DYN);
-  attn_bwd_dkdv_tc_kernel<<<grid, BT, dkv::SMEM_DYN, s>>>(tq, tdo, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-                                                          lse, delta, q_off, q_idx, dk, dv, d.N, (int)d.L, topk, items,
-                                                          c1, c1, ctx);
+  attn_bwd_dkdv_tc_kernel<<<grid, BT_KV, dkv::SMEM_DYN, s>>>(tq, tdo, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+                                                          nlse2, ndelta, q_off, q_idx, dk, dv, d.N, (int)d.L, topk,
+                                                          items, c2, c1, ctx);
   return check_launch("attn_bwd_dkdv_tc_kernel");
 }
 

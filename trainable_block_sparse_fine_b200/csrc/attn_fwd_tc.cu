@@ -339,20 +339,23 @@ __global__ void __launch_bounds__(FT, 1)
         }
         // probabilities (<= 2^8), partial row sum, pack bf16 pairs of adjacent columns:
         // the pair partner holds the neighbouring column, so swap half of the values
+        // the two columns of a step go through packed fp32 math (one FFMA2, one FADD2)
         uint32_t pk[32];
-        float ls = 0.f;
+        const float2 cc = make_float2(c2, c2), nm = make_float2(-m, -m);
+        float2 ls = make_float2(0.f, 0.f);
 #pragma unroll
         for (int i2 = 0; i2 < 32; ++i2) {
-          float pa = ex2(fmaf(__uint_as_float(x[2 * i2]), c2, -m));
-          float pb = ex2(fmaf(__uint_as_float(x[2 * i2 + 1]), c2, -m));
+          const float2 arg =
+              __ffma2_rn(make_float2(__uint_as_float(x[2 * i2]), __uint_as_float(x[2 * i2 + 1])), cc, nm);
+          float pa = ex2(arg.x), pb = ex2(arg.y);
           if (half && i2 >= 16) pa = pb = 0.f;
-          ls += pa + pb;
+          ls = __fadd2_rn(ls, make_float2(pa, pb));
           const float send = par_c ? pa : pb;
           const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
           // even thread: word 2*i2 = (col 4*i2, 4*i2+1); odd thread: word 2*i2+1 = (4*i2+2, 4*i2+3)
           pk[i2] = par_c ? pack_bf16(recv, pb) : pack_bf16(pa, recv);
         }
-        l += ls;
+        l += ls.x + ls.y;
         // P region is free once the O MMA of the previous block has finished
         if (n > 0) mbar_wait(&B.pvdone[s], (g - 1) & 1, abort, ctx);
         tmem_st16x64b_x32(tl + TM_P, pk);
