@@ -24,8 +24,7 @@
 namespace vsa2 {
 namespace {
 
-constexpr int BT = 352;            // dQ kernel: 11 warps (0-7 softmax, 8/10 producers, 9 MMA)
-constexpr int BT_KV = 384;         // dK/dV kernel: 12 warps (0-7 softmax, 8/10 producers, 9/11 MMA)
+constexpr int BT = 384;            // 12 warps: 0-7 softmax (two slots), 8/10 producers, 9/11 MMA issuers
 constexpr uint32_t TILE_B = 8192;  // one 64 x 64 bf16 box (64 rows x 128 B, 128-byte swizzle)
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -135,7 +134,7 @@ constexpr uint32_t TM_S = 0, TM_DP = 128, TM_Q = 256, TM_DO = 320, TM_DQ = 384;
 struct Bars {
   uint64_t kfull[KST], kempty[KST], vfull[VST], vempty[VST];
   uint64_t sfull[2], dsfull[2], bdone[2], qready[2];
-  uint64_t done;
+  uint64_t done[2];
 };
 static_assert(sizeof(Bars) <= 512, "barrier area");
 
@@ -182,8 +181,8 @@ __global__ void __launch_bounds__(BT, 1)
       mbar_init(&B.dsfull[s], 4);
       mbar_init(&B.bdone[s], 1);
       mbar_init(&B.qready[s], 4);
+      mbar_init(&B.done[s], 1);
     }
-    mbar_init(&B.done, 1);
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -244,9 +243,11 @@ __global__ void __launch_bounds__(BT, 1)
       for (int cc = max(0, last - nst + 1); cc <= last; ++cc)
         mbar_wait_drain(k_role ? &B.kfull[cc % nst] : &B.vfull[cc % nst], (cc / nst) & 1, ctx.timeout_ns);
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == 9 || warp == 11) {
+    // ------------------------------------------------------------------ MMA issuer of slot (warp - 9) / 2
+    // walks the merged op stream of both slots (the K/V ring order) and issues its own slot's ops
     if (lane == 0) {
+      const int me = (warp - 9) >> 1;
       constexpr uint32_t id_kmaj = idesc_bf16_f32(64, 128, false, false);  // S, dP: N = 128 keys
       constexpr uint32_t id_mn = idesc_bf16_f32(64, 128, false, true);     // dQ: N = 128 (d)
       Seq sq[2];
@@ -263,6 +264,10 @@ __global__ void __launch_bounds__(BT, 1)
           int blk;
           const int op = next_op(sq[s], &blk, kv_off, N, cap, 2, ctx);
           if (op == 0) continue;
+          if (s != me) {  // the other slot's op: only its ring positions
+            if (op == 1) ++kc, ++vc;
+            continue;
+          }
           const uint32_t lanes = (uint32_t)(16 * s) << 16;
           if (op == 1) {
             if (blk == 0 && !(ok = mbar_wait(&B.qready[s], (sq[s].tile - 1) & 1, abort, ctx))) break;
@@ -302,8 +307,8 @@ __global__ void __launch_bounds__(BT, 1)
           }
         }
       }
-      mma_commit(&B.done);
-      mbar_wait_drain(&B.done, 0, ctx.timeout_ns);
+      mma_commit(&B.done[me]);
+      mbar_wait_drain(&B.done[me], 0, ctx.timeout_ns);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax, one slot per warpgroup
@@ -423,7 +428,7 @@ static_assert(sizeof(Bars) <= 512, "barrier area");
 
 // The two slots are independent pipelines that share only the tensor pipe: slot s has its own
 // producer warp (8 + 2s) and its own MMA-issuing warp (9 + 2s), so neither waits on the other.
-__global__ void __launch_bounds__(BT_KV, 1)
+__global__ void __launch_bounds__(BT, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                             const __nv_bfloat16* __restrict__ kg, const __nv_bfloat16* __restrict__ vg,
                             const float* __restrict__ nlse2, const float* __restrict__ ndelta,
@@ -664,7 +669,7 @@ vsa2_status attn_bwd_tc(const Dims& d, const void* q, const void* k, const void*
       kv_idx, dq, d.N, (int)d.L, topk, items, c2, c1, ctx);
   if (check_launch("attn_bwd_dq_tc_kernel") != VSA2_OK) return VSA2_ERR_CUDA;
   cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dkv::SMEM_DYN);
-  attn_bwd_dkdv_tc_kernel<<<grid, BT_KV, dkv::SMEM_DYN, s>>>(tq, tdo, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+  attn_bwd_dkdv_tc_kernel<<<grid, BT, dkv::SMEM_DYN, s>>>(tq, tdo, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
                                                           nlse2, ndelta, q_off, q_idx, dk, dv, d.N, (int)d.L, topk,
                                                           items, c2, c1, ctx);
   return check_launch("attn_bwd_dkdv_tc_kernel");

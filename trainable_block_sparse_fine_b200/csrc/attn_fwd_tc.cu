@@ -15,7 +15,8 @@
 // CTA (persistent): warps 0-3 run the softmax of slot 0, warps 4-7 of slot 1. A warp owns 16
 // rows of its slot; the 16x64b TMEM access gives each row to a pair of threads (even / odd
 // columns), so row max and row sum need one shuffle and no block-level barrier. Warp 8 loads K,
-// warp 10 loads V, warp 9 issues the MMAs. The running max is raised (with an O rescale in
+// warp 10 loads V; warps 9 and 11 issue the MMAs of slot 0 and slot 1, so one slot's MMAs never
+// wait behind the other slot's dependencies. The running max is raised (with an O rescale in
 // TMEM) only when a row's new maximum exceeds it by more than 2^8.
 #include <algorithm>
 
@@ -25,7 +26,7 @@
 namespace vsa2 {
 namespace {
 
-constexpr int FT = 352;            // 11 warps
+constexpr int FT = 384;            // 12 warps
 constexpr uint32_t TILE_B = 8192;  // one 64x64 bf16 box (64 rows x 128 B)
 constexpr uint32_t BLK_B = 32768;  // K or V block: [half0: tile A, tile B][half1: tile A, tile B]
 constexpr int KST = 4;             // K ring stages
@@ -51,7 +52,7 @@ struct Bars {
   uint64_t kfull[KST], kempty[KST], vfull[VST], vempty[VST];
   uint64_t sfull[2][2], sfree[2][2];  // [slot][buffer]
   uint64_t pfull[2], pvdone[2], qready[2];
-  uint64_t done;
+  uint64_t done[2];
 };
 static_assert(sizeof(Bars) <= 512, "barrier area");
 
@@ -144,7 +145,8 @@ __global__ void __launch_bounds__(FT, 1)
       mbar_init(&B.pvdone[s], 1);
       mbar_init(&B.qready[s], 4);
     }
-    mbar_init(&B.done, 1);
+    mbar_init(&B.done[0], 1);
+    mbar_init(&B.done[1], 1);
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -206,9 +208,11 @@ __global__ void __launch_bounds__(FT, 1)
       for (int cc = max(0, last - nst + 1); cc <= last; ++cc)
         mbar_wait_drain(k_role ? &B.kfull[cc % nst] : &B.vfull[cc % nst], (cc / nst) & 1, ctx.timeout_ns);
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == 9 || warp == 11) {
+    // ------------------------------------------------------------------ MMA issuer of slot (warp - 9) / 2
+    // walks the merged op stream of both slots (the K/V ring order) and issues its own slot's ops
     if (lane == 0) {
+      const int me = (warp - 9) >> 1;
       constexpr uint32_t id_s = idesc_bf16_f32(64, 128, false, false);
       constexpr uint32_t id_o = idesc_bf16_f32(64, 128, false, true);
       SlotSeq sq[2];
@@ -225,6 +229,13 @@ __global__ void __launch_bounds__(FT, 1)
           int blk;
           const int op = next_op(sq[s], &blk, kv_off, N, cap, ctx);
           if (op == 0) continue;
+          if (s != me) {  // the other slot's op: only its ring position
+            if (op == 1)
+              ++kc;
+            else
+              ++vc;
+            continue;
+          }
           const uint32_t lanes = (uint32_t)(16 * s) << 16;
           if (op == 1) {
             if (blk == 0 && !(ok = mbar_wait(&B.qready[s], (sq[s].tile - 1) & 1, abort, ctx))) break;
@@ -260,8 +271,8 @@ __global__ void __launch_bounds__(FT, 1)
           }
         }
       }
-      mma_commit(&B.done);
-      mbar_wait_drain(&B.done, 0, ctx.timeout_ns);
+      mma_commit(&B.done[me]);
+      mbar_wait_drain(&B.done[me], 0, ctx.timeout_ns);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax, one slot per warpgroup
