@@ -190,6 +190,23 @@ __global__ void __launch_bounds__(RS_THREADS, 1)
         tmem_ld32(tmem + lane_off + st * RS_N + col0, r);
         tmem_ld_wait();
         const int key0 = it * RS_N + col0;
+        if (key0 + 32 <= Lr) {
+          // full piece: max on the raw scores (c2 > 0), then one packed FMA per column pair
+          float pm = __uint_as_float(r[0]);
+#pragma unroll
+          for (int j = 1; j < 32; ++j) pm = fmaxf(pm, __uint_as_float(r[j]));
+          const float mn = fmaxf(m, pm * c2);
+          const float2 cc = make_float2(c2, c2), nm = make_float2(-mn, -mn);
+          float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float2 a = __ffma2_rn(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])), cc, nm);
+            s2 = __fadd2_rn(s2, make_float2(ex2(a.x), ex2(a.y)));
+          }
+          l = l * ex2(m - mn) + (s2.x + s2.y);
+          m = mn;
+          continue;
+        }
         float x[32];
         float pm = -INFINITY;
 #pragma unroll
@@ -235,6 +252,20 @@ __global__ void __launch_bounds__(RS_THREADS, 1)
         tmem_ld32(tmem + lane_off + st * RS_N + col0, r);
         tmem_ld_wait();
         const int key0 = c * RS_N + col0;
+        if (key0 + 32 <= Lr) {
+          // full piece: packed FMA for the exponent arguments and packed sums per key sub-cube
+          const float2 cc = make_float2(c2, c2), nl = make_float2(-lse2, -lse2);
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const float2 a0 =
+                __ffma2_rn(make_float2(__uint_as_float(r[4 * jj]), __uint_as_float(r[4 * jj + 1])), cc, nl);
+            const float2 a1 =
+                __ffma2_rn(make_float2(__uint_as_float(r[4 * jj + 2]), __uint_as_float(r[4 * jj + 3])), cc, nl);
+            const float2 sum = __fadd2_rn(make_float2(ex2(a0.x), ex2(a0.y)), make_float2(ex2(a1.x), ex2(a1.y)));
+            t[piece * 8 + jj] = sum.x + sum.y;
+          }
+          continue;
+        }
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
           float acc = 0.f;
