@@ -46,14 +46,23 @@ def load_peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def profiled_traffic(wl, pairs):
-    """DRAM bytes of one forward launch from the committed ncu summary, scaled by selected pairs;
-    None when the kernel source changed since the counters were taken or for other workloads."""
-    if wl.grid != (56, 48, 80) or wl.head_dim != 128 or wl.topk != 64:
+# Committed ncu summaries that carry DRAM bytes per selected pair for one kernel source and
+# workload shape: (summary file, kernel source, token grid).
+TRAFFIC_PROFILES = {
+    "fwd": ("attn_fwd_tc_720p_8heads.md", "attn_fwd_tc.cu", (56, 48, 80)),
+    "bwd": ("attn_bwd_tc_480p_4heads.md", "attn_bwd_tc.cu", (28, 32, 52)),
+}
+
+
+def profiled_traffic(kind, wl, pairs):
+    """DRAM bytes of one launch from the committed ncu summary, scaled by selected pairs; None
+    when the kernel source changed since the counters were taken or for other workloads."""
+    name, kernel_src, grid = TRAFFIC_PROFILES[kind]
+    if wl.grid != grid or wl.head_dim != 128 or wl.topk != 64:
         return None
     try:
-        txt = open(os.path.join(ROOT, "profiles", "attn_fwd_tc_720p_8heads.md")).read()
-        src = open(os.path.join(ROOT, "trainable_block_sparse_fine_b200", "csrc", "attn_fwd_tc.cu"), "rb").read()
+        txt = open(os.path.join(ROOT, "profiles", name)).read()
+        src = open(os.path.join(ROOT, "trainable_block_sparse_fine_b200", "csrc", kernel_src), "rb").read()
     except OSError:
         return None
     per = re.search(r"dram_bytes_per_pair:\s*(\d+)", txt)
@@ -340,6 +349,14 @@ def run_ours(args, wl):
     hbm, bf16_burst, bf16_sus, peak_kind = load_peaks()
     fwd_ms = statistics.mean(per["fwd"])
     fwd_tflops = pair_flops(wl, pairs, False) / (fwd_ms * 1e-3) / 1e12
+    if wl.backward:  # the backward pass (dQ kernel + dK/dV kernel) dominates a training step
+        bwd_ms = statistics.mean(per["bwd"])
+        bwd_tflops = 2.5 * pair_flops(wl, pairs, False) / (bwd_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": "attn_bwd_dq_tc_kernel + attn_bwd_dkdv_tc_kernel (one call)",
+                "achieved": bwd_tflops, "traffic": profiled_traffic("bwd", wl, pairs)}
+    else:
+        roof = {"bound": "tensor", "kernel": "attn_fwd_tc_kernel", "achieved": fwd_tflops,
+                "traffic": profiled_traffic("fwd", wl, pairs)}
     router_ms = statistics.mean(per["router"])
     router_bytes = 2 * wl.batch * wl.heads * wl.tokens * wl.head_dim * (2 if wl.dtype == "bf16" else 4) \
         + wl.batch * wl.heads * wl.num_tiles ** 2 * 4
@@ -364,9 +381,10 @@ def run_ours(args, wl):
             "fwd_kernel": {"ms": fwd_ms, "effective_tflops": fwd_tflops},
             "router": {"ms": router_ms, "algorithmic_bytes": router_bytes,
                        "gbs": router_bytes / (router_ms * 1e-3) / 1e9, "hbm_frac": router_bytes / (router_ms * 1e-3) / 1e9 / hbm},
-            "roofline": {"bound": "tensor", "kernel": "attn_fwd_tc_kernel", "achieved": fwd_tflops,
-                         "peak": bf16_sus, "unit": "TFLOP/s", "frac": fwd_tflops / bf16_sus,
-                         "peak_kind": f"{peak_kind} sustained bf16", "traffic": profiled_traffic(wl, pairs)},
+            **({"bwd_pass": {"ms": bwd_ms, "effective_tflops": bwd_tflops}} if wl.backward else {}),
+            "roofline": {"bound": roof["bound"], "kernel": roof["kernel"], "achieved": roof["achieved"],
+                         "peak": bf16_sus, "unit": "TFLOP/s", "frac": roof["achieved"] / bf16_sus,
+                         "peak_kind": f"{peak_kind} sustained bf16", "traffic": roof["traffic"]},
             "cpu_baseline": cpu,
             "e2e": {"value": flops_rank * world / (e2e * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
