@@ -121,18 +121,20 @@ __device__ __forceinline__ void store_row_f32(float* dst, const uint32_t (&v)[64
 // dQ kernel
 // =========================================================================================
 namespace dqk {
-constexpr int KST = 4, VST = 3;
+constexpr int KST = 2, VST = 1;         // per slot: a K block is held until its dQ MMAs are done
 constexpr uint32_t BLK_B = 4 * TILE_B;  // two KV tiles: [d half 0: tile a, tile b][d half 1: tile a, tile b]
-constexpr uint32_t OFF_K = 0;
-constexpr uint32_t OFF_V = OFF_K + KST * BLK_B;
-constexpr uint32_t OFF_BAR = OFF_V + VST * BLK_B;
+// Each slot has its own K and V rings (one producer, one consumer each), so every barrier wait
+// is for the phase in progress or the one just completed.
+constexpr uint32_t OFF_K = 0;                          // [slot][KST] blocks
+constexpr uint32_t OFF_V = OFF_K + 2 * KST * BLK_B;    // [slot][VST] blocks
+constexpr uint32_t OFF_BAR = OFF_V + 2 * VST * BLK_B;
 constexpr uint32_t OFF_FLAG = OFF_BAR + 512;
 constexpr uint32_t SMEM_DYN = OFF_FLAG + 64 + 1024;
 static_assert(SMEM_DYN <= 232448, "shared memory budget");
 // TMEM columns (both slots, through the lane halves)
 constexpr uint32_t TM_S = 0, TM_DP = 128, TM_Q = 256, TM_DO = 320, TM_DQ = 384;
 struct Bars {
-  uint64_t kfull[KST], kempty[KST], vfull[VST], vempty[VST];
+  uint64_t kfull[2][KST], kempty[2][KST], vfull[2][VST], vempty[2][VST];  // [slot][stage]
   uint64_t sfull[2], dsfull[2], bdone[2], qready[2];
   uint64_t done[2];
 };
@@ -174,9 +176,9 @@ __global__ void __launch_bounds__(BT, 1)
 
   if (threadIdx.x == 0) {
     flag_sh[0] = 0;
-    for (int i = 0; i < KST; ++i) mbar_init(&B.kfull[i], 1), mbar_init(&B.kempty[i], 1);
-    for (int i = 0; i < VST; ++i) mbar_init(&B.vfull[i], 1), mbar_init(&B.vempty[i], 1);
     for (int s = 0; s < 2; ++s) {
+      for (int i = 0; i < KST; ++i) mbar_init(&B.kfull[s][i], 1), mbar_init(&B.kempty[s][i], 1);
+      for (int i = 0; i < VST; ++i) mbar_init(&B.vfull[s][i], 1), mbar_init(&B.vempty[s][i], 1);
       mbar_init(&B.sfull[s], 1);
       mbar_init(&B.dsfull[s], 4);
       mbar_init(&B.bdone[s], 1);
@@ -195,120 +197,106 @@ __global__ void __launch_bounds__(BT, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(flag_sh + 4);
 
   if (warp == 8 || warp == 10) {
-    // ------------------------------------------------------------------ TMA producers
-    // warp 8 loads K, warp 10 loads V, one block of two KV tiles per A op
-    const bool k_role = warp == 8;
-    const CUtensorMap* map = k_role ? &tm_k : &tm_v;
-    if (lane == 0) tma_prefetch_desc(map);
-    const int nst = k_role ? KST : VST;
-    Seq sq[2];
-    sq[0].init(2 * blockIdx.x, step, items);
-    sq[1].init(2 * blockIdx.x + 1, step, items);
-    int c = 0, last = -1;
-    bool ok = true;
-    while (ok && (sq[0].active || sq[1].active)) {
-#pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        if (!ok) break;
+    // ------------------------------------------------------------------ TMA producer of slot (warp - 8) / 2
+    // the K block and the V block (two KV tiles each) of every A op of the slot, one thread
+    if (lane == 0) {
+      const int s = (warp - 8) >> 1;
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      Seq sq;
+      sq.init(2 * blockIdx.x + s, step, items);
+      int c = 0;
+      bool ok = true;
+      while (ok && sq.active) {
         int blk;
-        if (next_op(sq[s], &blk, kv_off, N, cap, 2, ctx) != 1) continue;
-        const Seq& q = sq[s];
-        const int ntile = min(2, q.len - 2 * blk);
-        int j = 0;
-        if (lane < 2 * ntile) {
-          j = kv_idx[(size_t)q.bh * cap + q.beg + 2 * blk + (lane >> 1)];
-          if (j < 0 || j >= N) {
+        if (next_op(sq, &blk, kv_off, N, cap, 2, ctx) != 1) continue;
+        const int ntile = min(2, sq.len - 2 * blk);
+        int j[2] = {0, 0};
+        for (int tt = 0; tt < ntile; ++tt) {
+          int v = kv_idx[(size_t)sq.bh * cap + sq.beg + 2 * blk + tt];
+          if (v < 0 || v >= N) {
             if (ctx.flags & VSA2_FLAG_VALIDATE) set_error(ctx.err, VSA2_ERR_BAD_INDEX);
-            j = min(max(j, 0), N - 1);
+            v = min(max(v, 0), N - 1);
           }
+          j[tt] = v;
         }
-        const int st = c % nst;
-        uint64_t* empty = k_role ? &B.kempty[st] : &B.vempty[st];
-        uint64_t* full = k_role ? &B.kfull[st] : &B.vfull[st];
-        int w_ok = 1;
-        if (lane == 0) {
-          w_ok = mbar_wait(empty, ((c / nst) & 1) ^ 1, abort, ctx);
-          if (w_ok) mbar_arrive_expect_tx(full, ntile * 2 * TILE_B);
+        const int ks = c % KST, vs = c % VST;
+        if (!(ok = mbar_wait(&B.kempty[s][ks], ((c / KST) & 1) ^ 1, abort, ctx))) break;
+        mbar_arrive_expect_tx(&B.kfull[s][ks], ntile * 2 * TILE_B);
+        uint8_t* kd = dsm + OFF_K + (s * KST + ks) * BLK_B;
+        for (int tt = 0; tt < ntile; ++tt)
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d(kd + h * 2 * TILE_B + tt * TILE_B, &tm_k, h * 64, sq.bh * L + j[tt] * 64, &B.kfull[s][ks]);
+        if (!(ok = mbar_wait(&B.vempty[s][vs], ((c / VST) & 1) ^ 1, abort, ctx))) {
+          ++c;  // the K block of position c is in flight
+          break;
         }
-        if (!(ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0)) break;
-        if (lane < 2 * ntile) {
-          const int tt = lane >> 1, h = lane & 1;
-          tma_load_2d(dsm + (k_role ? OFF_K : OFF_V) + st * BLK_B + h * 2 * TILE_B + tt * TILE_B, map, h * 64,
-                      q.bh * L + j * 64, full);
-        }
-        last = c++;
+        mbar_arrive_expect_tx(&B.vfull[s][vs], ntile * 2 * TILE_B);
+        uint8_t* vd = dsm + OFF_V + (s * VST + vs) * BLK_B;
+        for (int tt = 0; tt < ntile; ++tt)
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d(vd + h * 2 * TILE_B + tt * TILE_B, &tm_v, h * 64, sq.bh * L + j[tt] * 64, &B.vfull[s][vs]);
+        ++c;
       }
-    }
-    if (lane == 0 && *abort) {  // let copies still in flight land before the CTA exits
-      for (int cc = max(0, last - nst + 1); cc <= last; ++cc)
-        mbar_wait_drain(k_role ? &B.kfull[cc % nst] : &B.vfull[cc % nst], (cc / nst) & 1, ctx.timeout_ns);
+      if (*abort) {  // let copies still in flight land before the CTA exits
+        for (int cc = max(0, c - KST); cc < c; ++cc)
+          mbar_wait_drain(&B.kfull[s][cc % KST], (cc / KST) & 1, ctx.timeout_ns);
+        for (int cc = max(0, c - VST); cc < c; ++cc)
+          mbar_wait_drain(&B.vfull[s][cc % VST], (cc / VST) & 1, ctx.timeout_ns);
+      }
     }
   } else if (warp == 9 || warp == 11) {
     // ------------------------------------------------------------------ MMA issuer of slot (warp - 9) / 2
-    // walks the merged op stream of both slots (the K/V ring order) and issues its own slot's ops
     if (lane == 0) {
-      const int me = (warp - 9) >> 1;
+      const int s = (warp - 9) >> 1;
       constexpr uint32_t id_kmaj = idesc_bf16_f32(64, 128, false, false);  // S, dP: N = 128 keys
       constexpr uint32_t id_mn = idesc_bf16_f32(64, 128, false, true);     // dQ: N = 128 (d)
-      Seq sq[2];
-      sq[0].init(2 * blockIdx.x, step, items);
-      sq[1].init(2 * blockIdx.x + 1, step, items);
-      int kc = 0, vc = 0;
-      int ga[2] = {0, 0}, gb[2] = {0, 0};
-      int kst_of[2] = {0, 0};  // K stage of the block between its A and B op, per slot
+      const uint32_t lanes = (uint32_t)(16 * s) << 16;
+      Seq sq;
+      sq.init(2 * blockIdx.x + s, step, items);
+      int ga = 0, gb = 0;  // A and B ops issued
       bool ok = true;
-      while (ok && (sq[0].active || sq[1].active)) {
+      while (ok && sq.active) {
+        int blk;
+        const int op = next_op(sq, &blk, kv_off, N, cap, 2, ctx);
+        if (op == 1) {
+          if (blk == 0 && !(ok = mbar_wait(&B.qready[s], (sq.tile - 1) & 1, abort, ctx))) break;
+          // S / dP of this slot are free once the previous dQ MMAs (which read dS) are done
+          if (ga > 0 && !(ok = mbar_wait(&B.bdone[s], (ga - 1) & 1, abort, ctx))) break;
+          const int ks = ga % KST, vs = ga % VST;
+          if (!(ok = mbar_wait(&B.kfull[s][ks], (ga / KST) & 1, abort, ctx))) break;
+          if (!(ok = mbar_wait(&B.vfull[s][vs], (ga / VST) & 1, abort, ctx))) break;
+          tc_fence_after();
+          const uint32_t ka = smem_u32(dsm + OFF_K + (s * KST + ks) * BLK_B);
+          const uint32_t va = smem_u32(dsm + OFF_V + (s * VST + vs) * BLK_B);
 #pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          if (!ok) break;
-          int blk;
-          const int op = next_op(sq[s], &blk, kv_off, N, cap, 2, ctx);
-          if (op == 0) continue;
-          if (s != me) {  // the other slot's op: only its ring positions
-            if (op == 1) ++kc, ++vc;
-            continue;
-          }
-          const uint32_t lanes = (uint32_t)(16 * s) << 16;
-          if (op == 1) {
-            if (blk == 0 && !(ok = mbar_wait(&B.qready[s], (sq[s].tile - 1) & 1, abort, ctx))) break;
-            // S / dP of this slot are free once the previous dQ MMAs (which read dS) are done
-            if (ga[s] > 0 && !(ok = mbar_wait(&B.bdone[s], (ga[s] - 1) & 1, abort, ctx))) break;
-            const int ks = kc % KST, vs = vc % VST;
-            if (!(ok = mbar_wait(&B.kfull[ks], (kc / KST) & 1, abort, ctx))) break;
-            if (!(ok = mbar_wait(&B.vfull[vs], (vc / VST) & 1, abort, ctx))) break;
-            tc_fence_after();
-            const uint32_t ka = smem_u32(dsm + OFF_K + ks * BLK_B), va = smem_u32(dsm + OFF_V + vs * BLK_B);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ts(tmem + lanes + TM_S, tmem + lanes + TM_Q + 8 * kk,
+                        sdesc_sw128(ka + (kk >> 2) * 2 * TILE_B + (kk & 3) * 32, 16, 1024), id_kmaj, kk > 0);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_bf16_ts(tmem + lanes + TM_S, tmem + lanes + TM_Q + 8 * kk,
-                          sdesc_sw128(ka + (kk >> 2) * 2 * TILE_B + (kk & 3) * 32, 16, 1024), id_kmaj, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_bf16_ts(tmem + lanes + TM_DP, tmem + lanes + TM_DO + 8 * kk,
-                          sdesc_sw128(va + (kk >> 2) * 2 * TILE_B + (kk & 3) * 32, 16, 1024), id_kmaj, kk > 0);
-            mma_commit(&B.vempty[vs]);
-            mma_commit(&B.sfull[s]);
-            kst_of[s] = ks;
-            ++kc;
-            ++vc;
-            ++ga[s];
-          } else {
-            if (!(ok = mbar_wait(&B.dsfull[s], gb[s] & 1, abort, ctx))) break;
-            tc_fence_after();
-            const int ks = kst_of[s];
-            const uint32_t ka = smem_u32(dsm + OFF_K + ks * BLK_B);
-            const int ksteps = (2 * blk + 1 == sq[s].len) ? 4 : 8;
-            for (int kk = 0; kk < ksteps; ++kk)
-              mma_bf16_ts(tmem + lanes + TM_DQ, tmem + lanes + TM_S + 8 * kk,
-                          sdesc_sw128(ka + kk * 2048, 2 * TILE_B, 1024), id_mn, (blk > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(&B.kempty[ks]);
-            mma_commit(&B.bdone[s]);
-            ++gb[s];
-          }
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ts(tmem + lanes + TM_DP, tmem + lanes + TM_DO + 8 * kk,
+                        sdesc_sw128(va + (kk >> 2) * 2 * TILE_B + (kk & 3) * 32, 16, 1024), id_kmaj, kk > 0);
+          mma_commit(&B.vempty[s][vs]);
+          mma_commit(&B.sfull[s]);
+          ++ga;
+        } else if (op == 2) {
+          // dQ += dS K, dS in the S region (bf16), K read MN-major from the A op's stage
+          if (!(ok = mbar_wait(&B.dsfull[s], gb & 1, abort, ctx))) break;
+          tc_fence_after();
+          const int ks = gb % KST;
+          const uint32_t ka = smem_u32(dsm + OFF_K + (s * KST + ks) * BLK_B);
+          const int ksteps = (2 * blk + 1 == sq.len) ? 4 : 8;
+          for (int kk = 0; kk < ksteps; ++kk)
+            mma_bf16_ts(tmem + lanes + TM_DQ, tmem + lanes + TM_S + 8 * kk,
+                        sdesc_sw128(ka + kk * 2048, 2 * TILE_B, 1024), id_mn, (blk > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&B.kempty[s][ks]);
+          mma_commit(&B.bdone[s]);
+          ++gb;
         }
       }
-      mma_commit(&B.done[me]);
-      mbar_wait_drain(&B.done[me], 0, ctx.timeout_ns);
+      mma_commit(&B.done[s]);
+      mbar_wait_drain(&B.done[s], 0, ctx.timeout_ns);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax, one slot per warpgroup

@@ -14,9 +14,9 @@
 //
 // CTA (persistent): warps 0-3 run the softmax of slot 0, warps 4-7 of slot 1. A warp owns 16
 // rows of its slot; the 16x64b TMEM access gives each row to a pair of threads (even / odd
-// columns), so row max and row sum need one shuffle and no block-level barrier. Warp 8 loads K,
-// warp 10 loads V; warps 9 and 11 issue the MMAs of slot 0 and slot 1, so one slot's MMAs never
-// wait behind the other slot's dependencies. The running max is raised (with an O rescale in
+// columns), so row max and row sum need one shuffle and no block-level barrier. The two slots
+// are independent pipelines sharing only the tensor pipe: warps 8 and 10 load the K and V
+// blocks of slot 0 and slot 1 into the slot's own rings, warps 9 and 11 issue its MMAs. The running max is raised (with an O rescale in
 // TMEM) only when a row's new maximum exceeds it by more than 2^8.
 #include <algorithm>
 
@@ -29,12 +29,14 @@ namespace {
 constexpr int FT = 384;            // 12 warps
 constexpr uint32_t TILE_B = 8192;  // one 64x64 bf16 box (64 rows x 128 B)
 constexpr uint32_t BLK_B = 32768;  // K or V block: [half0: tile A, tile B][half1: tile A, tile B]
-constexpr int KST = 4;             // K ring stages
-constexpr int VST = 3;             // V ring stages
+constexpr int KST = 2;             // K ring stages per slot
+constexpr int VST = 1;             // V ring stages per slot
 
-constexpr uint32_t OFF_K = 0;
-constexpr uint32_t OFF_V = OFF_K + KST * BLK_B;
-constexpr uint32_t OFF_BAR = OFF_V + VST * BLK_B;
+// Each slot has its own K and V rings (one producer, one consumer each), so every barrier wait
+// is for the phase in progress or the one just completed.
+constexpr uint32_t OFF_K = 0;                              // [slot][KST] blocks
+constexpr uint32_t OFF_V = OFF_K + 2 * KST * BLK_B;        // [slot][VST] blocks
+constexpr uint32_t OFF_BAR = OFF_V + 2 * VST * BLK_B;
 constexpr uint32_t OFF_FLAG = OFF_BAR + 512;
 constexpr uint32_t SMEM_USED = OFF_FLAG + 64;
 constexpr uint32_t SMEM_DYN = SMEM_USED + 1024;
@@ -49,8 +51,8 @@ constexpr uint32_t TM_COLS = 512;
 constexpr float kThresh = 8.0f;   // log2 headroom before the running max must move
 
 struct Bars {
-  uint64_t kfull[KST], kempty[KST], vfull[VST], vempty[VST];
-  uint64_t sfull[2][2], sfree[2][2];  // [slot][buffer]
+  uint64_t kfull[2][KST], kempty[2][KST], vfull[2][VST], vempty[2][VST];  // [slot][stage]
+  uint64_t sfull[2][2], sfree[2][2];                                       // [slot][buffer]
   uint64_t pfull[2], pvdone[2], qready[2];
   uint64_t done[2];
 };
@@ -137,9 +139,9 @@ __global__ void __launch_bounds__(FT, 1)
 
   if (threadIdx.x == 0) {
     flag_sh[0] = 0;
-    for (int i = 0; i < KST; ++i) mbar_init(&B.kfull[i], 1), mbar_init(&B.kempty[i], 1);
-    for (int i = 0; i < VST; ++i) mbar_init(&B.vfull[i], 1), mbar_init(&B.vempty[i], 1);
     for (int s = 0; s < 2; ++s) {
+      for (int i = 0; i < KST; ++i) mbar_init(&B.kfull[s][i], 1), mbar_init(&B.kempty[s][i], 1);
+      for (int i = 0; i < VST; ++i) mbar_init(&B.vfull[s][i], 1), mbar_init(&B.vempty[s][i], 1);
       for (int b = 0; b < 2; ++b) mbar_init(&B.sfull[s][b], 1), mbar_init(&B.sfree[s][b], 4);
       mbar_init(&B.pfull[s], 4);
       mbar_init(&B.pvdone[s], 1);
@@ -159,120 +161,98 @@ __global__ void __launch_bounds__(FT, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(flag_sh + 4);
 
   if (warp == 8 || warp == 10) {
-    // ------------------------------------------------------------------ TMA producers
-    // warp 8 loads K for the S ops, warp 10 loads V for the O ops, both in the MMA issue order.
-    const bool k_role = warp == 8;
-    const CUtensorMap* map = k_role ? &tm_k : &tm_v;
-    if (lane == 0) tma_prefetch_desc(map);
-    const int nst = k_role ? KST : VST;
-    SlotSeq sq[2];
-    sq[0].init(2 * blockIdx.x, step, items);
-    sq[1].init(2 * blockIdx.x + 1, step, items);
-    int c = 0, last = -1;
-    bool ok = true;
-    while (ok && (sq[0].active || sq[1].active)) {
-#pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        if (!ok) break;
+    // ------------------------------------------------------------------ TMA producer of slot (warp - 8) / 2
+    // K blocks for the slot's S ops and V blocks for its O ops, in the slot's op order, one thread
+    if (lane == 0) {
+      const int s = (warp - 8) >> 1;
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      SlotSeq sq;
+      sq.init(2 * blockIdx.x + s, step, items);
+      int kc = 0, vc = 0;
+      bool ok = true;
+      while (ok && sq.active) {
         int blk;
-        const int op = next_op(sq[s], &blk, kv_off, N, cap, ctx);
-        if (op == 0 || (op == 1) != k_role) continue;
-        const SlotSeq& q = sq[s];
-        const int ntile = min(2, q.len - 2 * blk);
-        int j = 0;
-        if (lane < 2 * ntile) {
-          j = kv_idx[(size_t)q.bh * cap + q.beg + 2 * blk + (lane >> 1)];
-          if (j < 0 || j >= N) {
+        const int op = next_op(sq, &blk, kv_off, N, cap, ctx);
+        if (op == 0) continue;
+        const bool k_op = op == 1;
+        const int ntile = min(2, sq.len - 2 * blk);
+        int j[2] = {0, 0};
+        for (int tt = 0; tt < ntile; ++tt) {
+          int v = kv_idx[(size_t)sq.bh * cap + sq.beg + 2 * blk + tt];
+          if (v < 0 || v >= N) {
             if (ctx.flags & VSA2_FLAG_VALIDATE) set_error(ctx.err, VSA2_ERR_BAD_INDEX);
-            j = min(max(j, 0), N - 1);
+            v = min(max(v, 0), N - 1);
           }
+          j[tt] = v;
         }
-        const int st = c % nst;
-        uint64_t* empty = k_role ? &B.kempty[st] : &B.vempty[st];
-        uint64_t* full = k_role ? &B.kfull[st] : &B.vfull[st];
-        int w_ok = 1;
-        if (lane == 0) {
-          w_ok = mbar_wait(empty, ((c / nst) & 1) ^ 1, abort, ctx);
-          if (w_ok) mbar_arrive_expect_tx(full, ntile * 2 * TILE_B);
-        }
-        if (!(ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0)) break;
-        if (lane < 2 * ntile) {
-          const int tt = lane >> 1, h = lane & 1;
-          tma_load_2d(dsm + (k_role ? OFF_K : OFF_V) + st * BLK_B + h * 2 * TILE_B + tt * TILE_B, map, h * 64,
-                      q.bh * L + j * 64, full);
-        }
-        last = c++;
+        const int c = k_op ? kc : vc, nst = k_op ? KST : VST, st = c % nst;
+        uint64_t* empty = k_op ? &B.kempty[s][st] : &B.vempty[s][st];
+        uint64_t* full = k_op ? &B.kfull[s][st] : &B.vfull[s][st];
+        uint8_t* dst = dsm + (k_op ? OFF_K + (s * KST + st) * BLK_B : OFF_V + (s * VST + st) * BLK_B);
+        if (!(ok = mbar_wait(empty, ((c / nst) & 1) ^ 1, abort, ctx))) break;
+        mbar_arrive_expect_tx(full, ntile * 2 * TILE_B);
+        for (int tt = 0; tt < ntile; ++tt)
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d(dst + h * 2 * TILE_B + tt * TILE_B, k_op ? &tm_k : &tm_v, h * 64, sq.bh * L + j[tt] * 64,
+                        full);
+        if (k_op)
+          ++kc;
+        else
+          ++vc;
       }
-    }
-    if (lane == 0 && *abort) {  // let copies still in flight land before the CTA exits
-      for (int cc = max(0, last - nst + 1); cc <= last; ++cc)
-        mbar_wait_drain(k_role ? &B.kfull[cc % nst] : &B.vfull[cc % nst], (cc / nst) & 1, ctx.timeout_ns);
+      if (*abort) {  // let copies still in flight land before the CTA exits
+        for (int cc = max(0, kc - KST); cc < kc; ++cc)
+          mbar_wait_drain(&B.kfull[s][cc % KST], (cc / KST) & 1, ctx.timeout_ns);
+        for (int cc = max(0, vc - VST); cc < vc; ++cc)
+          mbar_wait_drain(&B.vfull[s][cc % VST], (cc / VST) & 1, ctx.timeout_ns);
+      }
     }
   } else if (warp == 9 || warp == 11) {
     // ------------------------------------------------------------------ MMA issuer of slot (warp - 9) / 2
-    // walks the merged op stream of both slots (the K/V ring order) and issues its own slot's ops
     if (lane == 0) {
-      const int me = (warp - 9) >> 1;
+      const int s = (warp - 9) >> 1;
       constexpr uint32_t id_s = idesc_bf16_f32(64, 128, false, false);
       constexpr uint32_t id_o = idesc_bf16_f32(64, 128, false, true);
-      SlotSeq sq[2];
-      sq[0].init(2 * blockIdx.x, step, items);
-      sq[1].init(2 * blockIdx.x + 1, step, items);
-      int kc = 0, vc = 0;
-      int g[2] = {0, 0};   // S blocks issued per slot
-      int go[2] = {0, 0};  // O blocks issued per slot
+      const uint32_t lanes = (uint32_t)(16 * s) << 16;
+      SlotSeq sq;
+      sq.init(2 * blockIdx.x + s, step, items);
+      int kc = 0, vc = 0;  // S and O blocks issued
       bool ok = true;
-      while (ok && (sq[0].active || sq[1].active)) {
+      while (ok && sq.active) {
+        int blk;
+        const int op = next_op(sq, &blk, kv_off, N, cap, ctx);
+        if (op == 1) {
+          if (blk == 0 && !(ok = mbar_wait(&B.qready[s], (sq.tile - 1) & 1, abort, ctx))) break;
+          const int st = kc % KST;
+          if (!(ok = mbar_wait(&B.kfull[s][st], (kc / KST) & 1, abort, ctx))) break;
+          if (!(ok = mbar_wait(&B.sfree[s][kc & 1], ((kc >> 1) & 1) ^ 1, abort, ctx))) break;
+          tc_fence_after();
+          const uint32_t ka = smem_u32(dsm + OFF_K + (s * KST + st) * BLK_B);
 #pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          if (!ok) break;
-          int blk;
-          const int op = next_op(sq[s], &blk, kv_off, N, cap, ctx);
-          if (op == 0) continue;
-          if (s != me) {  // the other slot's op: only its ring position
-            if (op == 1)
-              ++kc;
-            else
-              ++vc;
-            continue;
-          }
-          const uint32_t lanes = (uint32_t)(16 * s) << 16;
-          if (op == 1) {
-            if (blk == 0 && !(ok = mbar_wait(&B.qready[s], (sq[s].tile - 1) & 1, abort, ctx))) break;
-            const int st = kc % KST;
-            const int gb = g[s];
-            if (!(ok = mbar_wait(&B.kfull[st], (kc / KST) & 1, abort, ctx))) break;
-            if (!(ok = mbar_wait(&B.sfree[s][gb & 1], ((gb >> 1) & 1) ^ 1, abort, ctx))) break;
-            tc_fence_after();
-            const uint32_t ka = smem_u32(dsm + OFF_K + st * BLK_B);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_bf16_ts(tmem + lanes + TM_S + (gb & 1) * 128, tmem + lanes + TM_Q + 8 * kk,
-                          sdesc_sw128(ka + (kk >> 2) * 2 * TILE_B + (kk & 3) * 32, 16, 1024), id_s, kk > 0);
-            mma_commit(&B.kempty[st]);
-            mma_commit(&B.sfull[s][gb & 1]);
-            ++kc;
-            ++g[s];
-          } else {
-            const int st = vc % VST;
-            const int gb = go[s];
-            if (!(ok = mbar_wait(&B.vfull[st], (vc / VST) & 1, abort, ctx))) break;
-            if (!(ok = mbar_wait(&B.pfull[s], gb & 1, abort, ctx))) break;
-            tc_fence_after();
-            const uint32_t va = smem_u32(dsm + OFF_V + st * BLK_B);
-            const int ksteps = (2 * blk + 1 == sq[s].len) ? 4 : 8;
-            for (int kk = 0; kk < ksteps; ++kk)
-              mma_bf16_ts(tmem + lanes + TM_O, tmem + lanes + TM_P + 8 * kk,
-                          sdesc_sw128(va + kk * 2048, 2 * TILE_B, 1024), id_o, (blk > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(&B.vempty[st]);
-            mma_commit(&B.pvdone[s]);
-            ++vc;
-            ++go[s];
-          }
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ts(tmem + lanes + TM_S + (kc & 1) * 128, tmem + lanes + TM_Q + 8 * kk,
+                        sdesc_sw128(ka + (kk >> 2) * 2 * TILE_B + (kk & 3) * 32, 16, 1024), id_s, kk > 0);
+          mma_commit(&B.kempty[s][st]);
+          mma_commit(&B.sfull[s][kc & 1]);
+          ++kc;
+        } else if (op == 2) {
+          const int st = vc % VST;
+          if (!(ok = mbar_wait(&B.vfull[s][st], (vc / VST) & 1, abort, ctx))) break;
+          if (!(ok = mbar_wait(&B.pfull[s], vc & 1, abort, ctx))) break;
+          tc_fence_after();
+          const uint32_t va = smem_u32(dsm + OFF_V + (s * VST + st) * BLK_B);
+          const int ksteps = (2 * blk + 1 == sq.len) ? 4 : 8;
+          for (int kk = 0; kk < ksteps; ++kk)
+            mma_bf16_ts(tmem + lanes + TM_O, tmem + lanes + TM_P + 8 * kk,
+                        sdesc_sw128(va + kk * 2048, 2 * TILE_B, 1024), id_o, (blk > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&B.vempty[s][st]);
+          mma_commit(&B.pvdone[s]);
+          ++vc;
         }
       }
-      mma_commit(&B.done[me]);
-      mbar_wait_drain(&B.done[me], 0, ctx.timeout_ns);
+      mma_commit(&B.done[s]);
+      mbar_wait_drain(&B.done[s], 0, ctx.timeout_ns);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax, one slot per warpgroup
