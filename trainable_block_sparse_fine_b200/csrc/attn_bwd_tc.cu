@@ -151,8 +151,7 @@ __device__ __forceinline__ void ds_half(const uint32_t (&sv)[32], const uint32_t
     const float2 p = make_float2(ex2(arg.x), ex2(arg.y));
     const float2 ds =
         __fmul2_rn(p, __fadd2_rn(make_float2(__uint_as_float(dp[2 * i2]), __uint_as_float(dp[2 * i2 + 1])), dd));
-    const float recv = __shfl_xor_sync(0xffffffffu, par_c ? ds.x : ds.y, 2);
-    pk[i2] = par_c ? pack_bf16(recv, ds.y) : pack_bf16(ds.x, recv);
+    pk[i2] = pair_pack_bf16(ds.x, ds.y, pair_perm(par_c));
   }
 }
 }  // namespace dqk
@@ -588,6 +587,7 @@ __global__ void __launch_bounds__(BT, 1)
         tmem_ld16x64b_x32(tl + TM_DP, dp);
         tmem_ld_wait();
         const float2 cc = make_float2(c2, c2);
+        const uint32_t perm = pair_perm(par_c);
         uint32_t pk[16], dk[16];
 #pragma unroll
         for (int i2 = 0; i2 < 16; ++i2) {
@@ -596,10 +596,8 @@ __global__ void __launch_bounds__(BT, 1)
           const float2 p = make_float2(ex2(arg.x), ex2(arg.y));
           const float2 ds = __fmul2_rn(
               p, __fadd2_rn(make_float2(__uint_as_float(dp[2 * i2]), __uint_as_float(dp[2 * i2 + 1])), nd2[i2]));
-          const float rp = __shfl_xor_sync(0xffffffffu, par_c ? p.x : p.y, 2);
-          const float rd = __shfl_xor_sync(0xffffffffu, par_c ? ds.x : ds.y, 2);
-          pk[i2] = par_c ? pack_bf16(rp, p.y) : pack_bf16(p.x, rp);
-          dk[i2] = par_c ? pack_bf16(rd, ds.y) : pack_bf16(ds.x, rd);
+          pk[i2] = pair_pack_bf16(p.x, p.y, perm);
+          dk[i2] = pair_pack_bf16(ds.x, ds.y, perm);
         }
         tmem_st16x64b_x16(tl + TM_S, pk);
         tmem_st16x64b_x16(tl + TM_DP, dk);

@@ -304,10 +304,16 @@ __global__ void __launch_bounds__(FT, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&B.sfree[s][g & 1]);
         // columns 2i + par_c; in a half block only the first 64 columns are real
-        float mx = -INFINITY;
+        float mx = __uint_as_float(x[0]);
+        if (!half) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (!(half && i >= 32)) mx = fmaxf(mx, __uint_as_float(x[i]));
+          for (int i = 1; i < 63; i += 2) mx = fmax3(mx, __uint_as_float(x[i]), __uint_as_float(x[i + 1]));
+          mx = fmaxf(mx, __uint_as_float(x[63]));
+        } else {
+#pragma unroll
+          for (int i = 1; i < 31; i += 2) mx = fmax3(mx, __uint_as_float(x[i]), __uint_as_float(x[i + 1]));
+          mx = fmaxf(mx, __uint_as_float(x[31]));
+        }
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2)) * c2;
         float alpha = 1.f;
         const bool raise = mx > m + kThresh;
@@ -332,6 +338,7 @@ __global__ void __launch_bounds__(FT, 1)
         // the pair partner holds the neighbouring column, so swap half of the values
         // the two columns of a step go through packed fp32 math (one FFMA2, one FADD2)
         uint32_t pk[32];
+        const uint32_t perm = pair_perm(par_c);
         const float2 cc = make_float2(c2, c2), nm = make_float2(-m, -m);
         float2 ls = make_float2(0.f, 0.f);
 #pragma unroll
@@ -341,10 +348,8 @@ __global__ void __launch_bounds__(FT, 1)
           float pa = ex2(arg.x), pb = ex2(arg.y);
           if (half && i2 >= 16) pa = pb = 0.f;
           ls = __fadd2_rn(ls, make_float2(pa, pb));
-          const float send = par_c ? pa : pb;
-          const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
           // even thread: word 2*i2 = (col 4*i2, 4*i2+1); odd thread: word 2*i2+1 = (4*i2+2, 4*i2+3)
-          pk[i2] = par_c ? pack_bf16(recv, pb) : pack_bf16(pa, recv);
+          pk[i2] = pair_pack_bf16(pa, pb, perm);
         }
         l += ls.x + ls.y;
         // P region is free once the O MMA of the previous block has finished

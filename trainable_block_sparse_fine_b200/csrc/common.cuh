@@ -272,6 +272,20 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+// max of three fp32 values in one instruction (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// A thread pair (lanes l and l^2) holds the columns 4i+p and 4i+2+p of a row (p = the lane's
+// column parity). Each thread packs its two values to bf16, the pair swaps the packed words, and
+// a byte permute leaves the even thread with columns (4i, 4i+1) and the odd one with (4i+2, 4i+3).
+__device__ __forceinline__ uint32_t pair_pack_bf16(float a, float b, uint32_t perm) {
+  const uint32_t w = pack_bf16(a, b);
+  return __byte_perm(w, __shfl_xor_sync(0xffffffffu, w, 2), perm);
+}
+__device__ __forceinline__ uint32_t pair_perm(int par_c) { return par_c ? 0x3276u : 0x5410u; }
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }

@@ -194,7 +194,8 @@ __global__ void __launch_bounds__(RS_THREADS, 1)
           // full piece: max on the raw scores (c2 > 0), then one packed FMA per column pair
           float pm = __uint_as_float(r[0]);
 #pragma unroll
-          for (int j = 1; j < 32; ++j) pm = fmaxf(pm, __uint_as_float(r[j]));
+          for (int j = 1; j < 31; j += 2) pm = fmax3(pm, __uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+          pm = fmaxf(pm, __uint_as_float(r[31]));
           const float mn = fmaxf(m, pm * c2);
           const float2 cc = make_float2(c2, c2), nm = make_float2(-mn, -mn);
           float2 s2 = make_float2(0.f, 0.f);
