@@ -27,6 +27,7 @@ SMALL = S.Workload("small_bf16", 1, 2, 128, (8, 16, 20), 6, "bf16")  # N=40, Lr=
 SMALL64 = S.Workload("small_bf16_d64", 2, 1, 64, (4, 16, 24), 5, "bf16")  # N=24, batch 2
 TINY = S.WORKLOADS["tiny"]
 C480 = S.WORKLOADS["480p_top64"]
+C720 = S.WORKLOADS["720p_top64"]
 
 
 def dev(x, dtype):
@@ -148,6 +149,31 @@ def c480_lists(heads):
     return _sel480[key]
 
 
+def c720_head0():
+    """720p (the headline size): head 0 of Q, K, V from the seeded generator, its oracle router
+    scores (fp64) and the oracle's TopK on them. Only head 0 is compared; the kernels still run
+    all 20 heads, as the benchmark does."""
+    if "720p_h0" not in _cache:
+        x0 = {n: S.make_slice(C720, n, 0, 0) for n in ("q", "k", "v")}
+        sc = O.router_scores(x0["q"], x0["k"])
+        sel = O.topk_select(sc.astype(np.float32), C720.topk)
+        _cache["720p_h0"] = (x0, sc, sel)
+    return _cache["720p_h0"]
+
+
+def c720_device(x0, names=("q", "k", "v")):
+    """[1, 20, L, D] bf16 device tensors: head 0 = the generator's slice, heads 1-19 seeded
+    normals (their outputs are not compared)."""
+    g = torch.Generator(device="cuda").manual_seed(720)
+    out = {}
+    for n in names:
+        t = torch.randn((1, C720.heads, C720.tokens, C720.head_dim), generator=g, device="cuda") * 1.1
+        t[0, 0] = torch.from_numpy(x0[n]).cuda()
+        out[n] = t.to(torch.bfloat16)
+        del t
+    return out
+
+
 # ------------------------------------------------------------------------------------------
 # router
 # ------------------------------------------------------------------------------------------
@@ -260,6 +286,57 @@ def test_fwd_edge_selections(pattern):
     wl = SMALL.with_(topk=topk)
     kv_off, kv_idx, _, _ = lists_from_masks(masks, topk)
     _fwd_case(wl, inputs(wl), kv_off, kv_idx)
+
+
+def test_router_720p_head0():
+    x0, want, _ = c720_head0()
+    x = c720_device(x0, ("q", "k"))
+    e = engine(C720)
+    got = e.router_scores(x["q"], x["k"])
+    assert e.device_error() == 0
+    g = got[0, 0].cpu().numpy().astype(np.float64)
+    rel = np.linalg.norm(g - want) / np.linalg.norm(want)
+    assert rel <= 5e-3, rel
+    assert np.abs(g - want).max() <= 1e-2 * want.max()
+    np.testing.assert_allclose(g.sum(1), 1.0, atol=5e-3)
+
+
+def test_topk_720p_head0_bit_exact_on_oracle_scores():
+    _, sc, sel = c720_head0()
+    N = C720.num_tiles
+    rng = np.random.default_rng(7)
+    s32 = rng.random((1, C720.heads, N, N), dtype=np.float32)
+    s32[0, 0] = sc.astype(np.float32)
+    e = engine(C720)
+    kv_off, kv_idx, q_off, q_idx = e.topk_select(torch.from_numpy(s32).cuda(), C720.topk, csc=True)
+    assert e.device_error() == 0
+    for name, got in zip(("kv_off", "kv_idx", "q_off", "q_idx"), (kv_off, kv_idx, q_off, q_idx)):
+        assert np.array_equal(got[0, 0].cpu().numpy(), sel[name]), name
+
+
+def test_fwd_720p_sampled_head0():
+    """The 720p top64 forward in the benchmark's launch configuration (20 heads); head 0 runs on
+    the oracle's selection and is compared on sampled query tiles (first, last, middle, ragged
+    rows of the selection)."""
+    x0, _, sel = c720_head0()
+    x = c720_device(x0)
+    N = C720.num_tiles
+    masks = np.zeros((1, C720.heads, N, N), bool)
+    masks[0, 0] = sel["mask"]
+    rows = np.repeat(np.arange(N), C720.topk)
+    for h in range(1, C720.heads):
+        masks[0, h, rows, (rows + 11 * h + 7 * np.tile(np.arange(C720.topk), N)) % N] = True
+    kv_off, kv_idx, _, _ = lists_from_masks(masks, C720.topk)
+    e = engine(C720)
+    o, lse = e.attn_fwd(x["q"], x["k"], x["v"], torch.from_numpy(kv_off).cuda(), torch.from_numpy(kv_idx).cuda())
+    assert e.device_error() == 0
+    lens = sel["kv_off"][1:] - sel["kv_off"][:-1]
+    tiles = sorted({0, 1, N // 2, N - 1, int(np.argmin(lens)), int(np.argmax(lens))})
+    wo, wlse = O.sparse_attn_fwd(x0["q"], x0["k"], x0["v"], sel["kv_off"], sel["kv_idx"], query_tiles=tiles)
+    r = np.concatenate([np.arange(64 * i, 64 * i + 64) for i in tiles])
+    assert_attn_close(o[0, 0].float().cpu().numpy()[r], wo[r], "o[0,0]")
+    lg = lse[0, 0].cpu().numpy()[r]
+    assert np.abs(lg - wlse[r]).max() <= 2e-3 * max(1.0, np.abs(wlse[r]).max())
 
 
 def test_fwd_480p_sampled_heads():
