@@ -64,11 +64,12 @@ struct Seq {
   }
 };
 
-// 0 = none (slot finished), 1 = A op, 2 = B op; *blk = block index within the item
+// 0 = none (slot finished), 1 = A op, 2 = B op; *blk = block index within the item. With
+// ahead = 1 the A op of block n+1 comes before the B op of block n.
 __device__ __forceinline__ int next_op(Seq& q, int* blk, const int32_t* off, int N, int cap, int per_blk,
-                                       const DevCtx& ctx) {
+                                       const DevCtx& ctx, int ahead = 0) {
   while (q.active) {
-    if (q.a_next < q.nblk && q.a_next == q.b_next) {
+    if (q.a_next < q.nblk && q.a_next <= q.b_next + ahead) {
       *blk = q.a_next++;
       return 1;
     }
@@ -336,11 +337,9 @@ __global__ void __launch_bounds__(BT, 1)
         dlt = part + __shfl_xor_sync(0xffffffffu, part, 2);
       }
       const float nl2 = -lse[tok] * kLog2e;
-      if (par_c == 0) {
-        // for the dK/dV kernel: each tile's 64 values ordered even rows, then odd rows
-        const size_t perm = (size_t)bh * L + (size_t)qt * 64 + (row & 1) * 32 + (row >> 1);
-        ndelta[perm] = -dlt;
-        nlse2[perm] = nl2;
+      if (par_c == 0) {  // for the dK/dV kernel
+        ndelta[tok] = -dlt;
+        nlse2[tok] = nl2;
       }
       tmem_st_wait();
       tc_fence_before();
@@ -395,27 +394,36 @@ __global__ void __launch_bounds__(BT, 1)
 // =========================================================================================
 // dK / dV kernel
 // =========================================================================================
+// One KV tile per CTA at a time, M=128 MMAs over all TMEM lanes. Lane 2j holds key j's K row and
+// lane 2j+1 its V row, so with B = [Q; dO] of one selected query tile (N = 128) a single MMA per
+// K-step gives S^T = K Q^T on the even lanes (columns 0-63) and dP^T = V dO^T on the odd lanes
+// (columns 64-127); the two other quadrants are not used. The softmax writes P^T (even lanes)
+// and dS^T (odd lanes) back as one bf16 A operand, and with B = [Q | dO] (N = 256) the second MMA
+// accumulates dV = P^T dO on the even lanes and dK = dS^T Q on the odd lanes. Per query tile the
+// tensor pipe does two M=128 K-loops instead of the four M=64, N=64 ones of a per-key-half split.
 namespace dkv {
-constexpr int RST = 3;                        // ring stages per slot
-constexpr uint32_t STAGE_B = 33792;           // Q tile 16 KB, dO tile 16 KB, lse 256 B, Delta 256 B (1 KB aligned)
-constexpr uint32_t OFF_BAR = 2 * RST * STAGE_B;
+constexpr int KT = 384;               // 12 warps: 0-7 softmax, 8/10 producers, 9 and 11 MMA issuers
+constexpr int RST = 6;                // ring stages; warp 8 fills the even ring positions, warp 10 the odd
+constexpr uint32_t STAGE_B = 33792;   // [d half 0: Q, dO][d half 1: Q, dO], then 64 -lse*log2e, 64 -Delta
+constexpr uint32_t OFF_BAR = RST * STAGE_B;
 constexpr uint32_t OFF_FLAG = OFF_BAR + 512;
 constexpr uint32_t SMEM_DYN = OFF_FLAG + 64 + 1024;
 static_assert(SMEM_DYN <= 232448, "shared memory budget");
-// TMEM columns: K and V (A operands, 64 each), S^T and dP^T (64 fp32 columns each; P^T and
-// dS^T are written back as bf16 over their first 32), dV and dK accumulators (128 each)
-constexpr uint32_t TM_K = 0, TM_V = 64, TM_S = 128, TM_DP = 192, TM_DV = 256, TM_DK = 384;
+static_assert(RST % 2 == 0, "each ring stage must have a single producer");
+// TMEM columns (all 128 lanes)
+constexpr uint32_t TM_KV = 0;     // A of the first MMA: K row (even lanes) / V row (odd lanes), 64 columns
+constexpr uint32_t TM_SP = 64;    // D of the first MMA: S^T (even lanes, 0-63), dP^T (odd lanes, 64-127)
+constexpr uint32_t TM_PDS = 192;  // A of the second MMA: P^T (even) / dS^T (odd) in bf16, 2 buffers x 32
+constexpr uint32_t TM_G = 256;    // D of the second MMA: dV (even lanes) / dK (odd lanes), 256 columns
 struct Bars {
-  uint64_t full[2 * RST], empty[2 * RST];
-  uint64_t sfull[2], pfull[2], bdone[2], kvready[2];
+  uint64_t full[RST], empty[RST];
+  uint64_t spfull, spfree, pdsfull[2], pdsfree[2], itemdone, kvready;
   uint64_t done[2];
 };
 static_assert(sizeof(Bars) <= 512, "barrier area");
 }  // namespace dkv
 
-// The two slots are independent pipelines that share only the tensor pipe: slot s has its own
-// producer warp (8 + 2s) and its own MMA-issuing warp (9 + 2s), so neither waits on the other.
-__global__ void __launch_bounds__(BT, 1)
+__global__ void __launch_bounds__(dkv::KT, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                             const __nv_bfloat16* __restrict__ kg, const __nv_bfloat16* __restrict__ vg,
                             const float* __restrict__ nlse2, const float* __restrict__ ndelta,
@@ -430,18 +438,18 @@ __global__ void __launch_bounds__(BT, 1)
   volatile int* abort = flag_sh;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cap = N * topk;
-  const int step = 2 * gridDim.x;
+  const int step = gridDim.x;
 
   if (threadIdx.x == 0) {
     flag_sh[0] = 0;
-    for (int i = 0; i < 2 * RST; ++i) mbar_init(&B.full[i], 1), mbar_init(&B.empty[i], 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&B.sfull[s], 1);
-      mbar_init(&B.pfull[s], 4);
-      mbar_init(&B.bdone[s], 1);
-      mbar_init(&B.kvready[s], 4);
-      mbar_init(&B.done[s], 1);
-    }
+    for (int i = 0; i < RST; ++i) mbar_init(&B.full[i], 1), mbar_init(&B.empty[i], 1);
+    mbar_init(&B.spfull, 1);
+    mbar_init(&B.spfree, 8);
+    for (int b = 0; b < 2; ++b) mbar_init(&B.pdsfull[b], 8), mbar_init(&B.pdsfree[b], 1);
+    mbar_init(&B.itemdone, 1);
+    mbar_init(&B.kvready, 8);
+    mbar_init(&B.done[0], 1);
+    mbar_init(&B.done[1], 1);
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -454,168 +462,193 @@ __global__ void __launch_bounds__(BT, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(flag_sh + 4);
 
   if (warp == 8 || warp == 10) {
-    // ------------------------------------------------------------------ producer of slot (warp - 8) / 2
-    // per selected query tile: its Q and dO tiles (two boxes each) and its 64 -lse*log2(e) and
-    // -Delta values (written by the dQ kernel), into the slot's ring (stage = the slot's tile count mod RST)
+    // ------------------------------------------------------------------ producers (lane 0)
+    // ring position c holds the c-th selecting query tile of this CTA: its Q and dO tiles (two
+    // boxes each) and its 64 -lse*log2(e) and -Delta values; warp 8 fills even positions and
+    // warp 10 odd ones, so every stage has one producer
     if (lane == 0) {
-      const int s = (warp - 8) >> 1;
+      const int par = (warp - 8) >> 1;
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
       Seq sq;
-      sq.init(2 * blockIdx.x + s, step, items);
-      int cnt = 0;
+      sq.init(blockIdx.x, step, items);
+      int c = 0, last = -1;
       bool ok = true;
       while (ok && sq.active) {
         int blk;
         if (next_op(sq, &blk, q_off, N, cap, 1, ctx) != 1) continue;
+        const int pos = c++;
+        if ((pos & 1) != par) continue;
         int i = q_idx[(size_t)sq.bh * cap + sq.beg + blk];
         if (i < 0 || i >= N) {
           if (ctx.flags & VSA2_FLAG_VALIDATE) set_error(ctx.err, VSA2_ERR_BAD_INDEX);
           i = min(max(i, 0), N - 1);
         }
-        const int r = s * RST + cnt % RST;
-        if (!(ok = mbar_wait(&B.empty[r], ((cnt / RST) & 1) ^ 1, abort, ctx))) break;
-        uint8_t* stage = dsm + r * STAGE_B;
+        const int st = pos % RST;
+        if (!(ok = mbar_wait(&B.empty[st], ((pos / RST) & 1) ^ 1, abort, ctx))) break;
+        uint8_t* stage = dsm + st * STAGE_B;
         const int row0 = sq.bh * L + i * 64;
-        mbar_arrive_expect_tx(&B.full[r], 4 * TILE_B + 512);
-        tma_load_2d(stage, &tm_q, 0, row0, &B.full[r]);
-        tma_load_2d(stage + TILE_B, &tm_q, 64, row0, &B.full[r]);
-        tma_load_2d(stage + 2 * TILE_B, &tm_do, 0, row0, &B.full[r]);
-        tma_load_2d(stage + 3 * TILE_B, &tm_do, 64, row0, &B.full[r]);
-        bulk_load(stage + 4 * TILE_B, nlse2 + row0, 256, &B.full[r]);
-        bulk_load(stage + 4 * TILE_B + 256, ndelta + row0, 256, &B.full[r]);
-        ++cnt;
+        mbar_arrive_expect_tx(&B.full[st], 4 * TILE_B + 512);
+        tma_load_2d(stage, &tm_q, 0, row0, &B.full[st]);
+        tma_load_2d(stage + TILE_B, &tm_do, 0, row0, &B.full[st]);
+        tma_load_2d(stage + 2 * TILE_B, &tm_q, 64, row0, &B.full[st]);
+        tma_load_2d(stage + 3 * TILE_B, &tm_do, 64, row0, &B.full[st]);
+        bulk_load(stage + 4 * TILE_B, nlse2 + row0, 256, &B.full[st]);
+        bulk_load(stage + 4 * TILE_B + 256, ndelta + row0, 256, &B.full[st]);
+        last = pos;
       }
       if (*abort)  // let copies still in flight land before the CTA exits
-        for (int cc = max(0, cnt - RST); cc < cnt; ++cc)
-          mbar_wait_drain(&B.full[s * RST + cc % RST], (cc / RST) & 1, ctx.timeout_ns);
+        for (int pos = last; pos >= 0 && pos > last - RST; pos -= 2)
+          mbar_wait_drain(&B.full[pos % RST], (pos / RST) & 1, ctx.timeout_ns);
     }
   } else if (warp == 9 || warp == 11) {
-    // ------------------------------------------------------------------ MMA issuer of slot (warp - 9) / 2
+    // ------------------------------------------------------------------ MMA issuers (lane 0)
+    // warp 9 issues the S^T / dP^T MMAs, warp 11 the dV / dK MMAs, so the next query tile's first
+    // MMAs are never held behind the previous tile's second ones in one issue order. The stage
+    // of tile n is released after its second MMAs, which start only after its first ones are
+    // done (through the softmax), and each commit covers the MMAs of its own thread.
     if (lane == 0) {
-      constexpr uint32_t id_s = idesc_bf16_f32(64, 64, false, false);  // S^T, dP^T: N = 64 queries
-      constexpr uint32_t id_g = idesc_bf16_f32(64, 128, false, true);  // dV, dK: N = 128 (d)
-      const int s = (warp - 9) >> 1;
-      const uint32_t lanes = (uint32_t)(16 * s) << 16;
+      const bool first = warp == 9;
+      constexpr uint32_t id_a = idesc_bf16_f32(128, 128, false, false);  // [K;V] x [Q;dO]^T
+      constexpr uint32_t id_b = idesc_bf16_f32(128, 256, false, true);   // [P;dS] x [Q | dO]
       Seq sq;
-      sq.init(2 * blockIdx.x + s, step, items);
-      int ga = 0, gb = 0;
+      sq.init(blockIdx.x, step, items);
+      int cnt = 0;  // MMAs groups issued by this thread
       bool ok = true;
       while (ok && sq.active) {
         int blk;
         const int op = next_op(sq, &blk, q_off, N, cap, 1, ctx);
-        if (op == 1) {
-          if (blk == 0 && !(ok = mbar_wait(&B.kvready[s], (sq.tile - 1) & 1, abort, ctx))) break;
-          // S^T / dP^T are free once the previous dV / dK MMAs (which read P^T / dS^T) are done
-          if (ga > 0 && !(ok = mbar_wait(&B.bdone[s], (ga - 1) & 1, abort, ctx))) break;
-          const int r = s * RST + ga % RST;
-          if (!(ok = mbar_wait(&B.full[r], (ga / RST) & 1, abort, ctx))) break;
+        if (op == 1 && first) {
+          if (blk == 0 && !(ok = mbar_wait(&B.kvready, (sq.tile - 1) & 1, abort, ctx))) break;
+          // S^T / dP^T of the previous query tile must have been read by the softmax
+          if (cnt > 0 && !(ok = mbar_wait(&B.spfree, (cnt - 1) & 1, abort, ctx))) break;
+          const int st = cnt % RST;
+          if (!(ok = mbar_wait(&B.full[st], (cnt / RST) & 1, abort, ctx))) break;
           tc_fence_after();
-          const uint32_t qa = smem_u32(dsm + r * STAGE_B), da = qa + 2 * TILE_B;
+          const uint32_t qa = smem_u32(dsm + st * STAGE_B);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ts(tmem + lanes + TM_S, tmem + lanes + TM_K + 8 * kk,
-                        sdesc_sw128(qa + (kk >> 2) * TILE_B + (kk & 3) * 32, 16, 1024), id_s, kk > 0);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ts(tmem + lanes + TM_DP, tmem + lanes + TM_V + 8 * kk,
-                        sdesc_sw128(da + (kk >> 2) * TILE_B + (kk & 3) * 32, 16, 1024), id_s, kk > 0);
-          mma_commit(&B.sfull[s]);
-          ++ga;
-        } else if (op == 2) {
-          // dV += P^T dO, dK += dS^T Q; P^T / dS^T in TMEM (bf16), dO / Q read MN-major
-          if (!(ok = mbar_wait(&B.pfull[s], gb & 1, abort, ctx))) break;
+            mma_bf16_ts(tmem + TM_SP, tmem + TM_KV + 8 * kk,
+                        sdesc_sw128(qa + (kk >> 2) * 2 * TILE_B + (kk & 3) * 32, 16, 1024), id_a, kk > 0);
+          mma_commit(&B.spfull);
+          ++cnt;
+        } else if (op == 2 && !first) {
+          const int b = cnt & 1;
+          if (!(ok = mbar_wait(&B.pdsfull[b], (cnt >> 1) & 1, abort, ctx))) break;
           tc_fence_after();
-          const int r = s * RST + gb % RST;
-          const uint32_t qa = smem_u32(dsm + r * STAGE_B), da = qa + 2 * TILE_B;
+          const uint32_t qa = smem_u32(dsm + (cnt % RST) * STAGE_B);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ts(tmem + lanes + TM_DV, tmem + lanes + TM_S + 8 * kk, sdesc_sw128(da + kk * 2048, TILE_B, 1024),
-                        id_g, (blk > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ts(tmem + lanes + TM_DK, tmem + lanes + TM_DP + 8 * kk, sdesc_sw128(qa + kk * 2048, TILE_B, 1024),
-                        id_g, (blk > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&B.empty[r]);
-          mma_commit(&B.bdone[s]);
-          ++gb;
+            mma_bf16_ts(tmem + TM_G, tmem + TM_PDS + 32 * b + 8 * kk, sdesc_sw128(qa + kk * 2048, TILE_B, 1024), id_b,
+                        (blk > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&B.empty[cnt % RST]);
+          mma_commit(&B.pdsfree[b]);
+          if (blk == sq.len - 1) mma_commit(&B.itemdone);
+          ++cnt;
         }
       }
-      mma_commit(&B.done[s]);
-      mbar_wait_drain(&B.done[s], 0, ctx.timeout_ns);
+      mma_commit(&B.done[first ? 0 : 1]);
+      mbar_wait_drain(&B.done[first ? 0 : 1], 0, ctx.timeout_ns);
     }
   } else if (warp < 8) {
-    // ------------------------------------------------------------------ softmax, one slot per warpgroup
-    // rows are keys of the KV tile, columns are queries of the selected query tile
-    const int s = warp >> 2, w = warp & 3;
-    const int bar_id = 1 + s;
-    const int par_c = (lane >> 1) & 1;
-    const int row = 16 * w + 8 * (lane & 1) + (lane >> 2);
-    const uint32_t tl = tmem + ((uint32_t)(32 * w + 16 * s) << 16);
-    int g = 0;  // query tiles processed by this slot
-    for (int item = 2 * blockIdx.x + s; item < items; item += step) {
+    // ------------------------------------------------------------------ softmax (8 warps)
+    // warp w reads TMEM lane quarter w % 4 and handles query half c = w / 4 of each tile
+    const int c = warp >> 2;
+    const int lrow = 32 * (warp & 3) + lane;
+    const int j = lrow >> 1, kind = lrow & 1;  // key row of the tile; 0: K side, 1: V side
+    const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    const float2 cc = make_float2(c2, c2);
+    int n = 0, it = 0;  // query tiles processed, non-empty items processed
+    for (int item = blockIdx.x; item < items; item += step) {
       const int bh = item / N, kt = item - bh * N;
-      const Row rw = load_list(q_off, bh, kt, N, cap, ctx, w == 0 && lane == 0);
-      const size_t tok = (size_t)bh * L + (size_t)kt * 64 + row;
-      float* dkd = dk_out + tok * 128;
-      float* dvd = dv_out + tok * 128;
+      const Row rw = load_list(q_off, bh, kt, N, cap, ctx, warp == 0 && lane == 0);
+      const size_t tok = (size_t)bh * L + (size_t)kt * 64 + j;
+      float* gout = (kind ? dk_out : dv_out) + tok * 128 + 64 * c;
       if (rw.len == 0) {
-        float4* a4 = reinterpret_cast<float4*>(dkd + par_c * 64);
-        float4* b4 = reinterpret_cast<float4*>(dvd + par_c * 64);
+        float4* z = reinterpret_cast<float4*>(gout);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) a4[e] = b4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int e = 0; e < 16; ++e) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
         continue;
       }
-      row_to_tmem(tl + TM_K, kg + tok * 128, par_c);
-      row_to_tmem(tl + TM_V, vg + tok * 128, par_c);
-      tmem_st_wait();
+      {
+        // this lane's K or V row into the first MMA's A operand (d in [64c, 64c + 64))
+        uint32_t v[32];
+        const uint32_t* src = reinterpret_cast<const uint32_t*>((kind ? vg : kg) + tok * 128) + 32 * c;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __ldg(src + i);
+        tmem_st32(tl + TM_KV + 32 * c, v);
+        tmem_st_wait();
+      }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&B.kvready[s]);
-      for (int n = 0; n < rw.len; ++n, ++g) {
-        const int r = s * RST + g % RST;
-        mbar_wait(&B.sfull[s], g & 1, abort, ctx);
-        // the stage's lse / Delta were written by the bulk copy: observe its barrier too
-        mbar_wait(&B.full[r], (g / RST) & 1, abort, ctx);
+      if (lane == 0) mbar_arrive(&B.kvready);
+      for (int t = 0; t < rw.len; ++t, ++n) {
+        const int st = n % RST, b = n & 1;
+        mbar_wait(&B.spfull, n & 1, abort, ctx);
+        mbar_wait(&B.full[st], (n / RST) & 1, abort, ctx);  // the stage's per-query vectors
         tc_fence_after();
-        // this thread's query columns are 4*i2 + par_c and 4*i2 + 2 + par_c: in the even/odd
-        // order of the stage they are one aligned float2
-        const float2* nl2 = reinterpret_cast<const float2*>(dsm + r * STAGE_B + 4 * TILE_B) + par_c * 16;
-        const float2* nd2 = nl2 + 32;
-        uint32_t sv[32], dp[32];
-        tmem_ld16x64b_x32(tl + TM_S, sv);
-        tmem_ld16x64b_x32(tl + TM_DP, dp);
+        uint32_t sa[32], da[32];
+        tmem_ld32(tl + TM_SP + 32 * c, sa);       // even lanes: S^T[j][32c + i]
+        tmem_ld32(tl + TM_SP + 64 + 32 * c, da);  // odd lanes: dP^T[j][32c + i]
         tmem_ld_wait();
-        const float2 cc = make_float2(c2, c2);
-        const uint32_t perm = pair_perm(par_c);
-        uint32_t pk[16], dk[16];
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.spfree);
+        // this thread takes queries 32c + 16*kind + i (i < 16): the lane pair swaps S and dP
+        float sv[16], dv[16];
 #pragma unroll
-        for (int i2 = 0; i2 < 16; ++i2) {
-          const float2 arg =
-              __ffma2_rn(make_float2(__uint_as_float(sv[2 * i2]), __uint_as_float(sv[2 * i2 + 1])), cc, nl2[i2]);
-          const float2 p = make_float2(ex2(arg.x), ex2(arg.y));
-          const float2 ds = __fmul2_rn(
-              p, __fadd2_rn(make_float2(__uint_as_float(dp[2 * i2]), __uint_as_float(dp[2 * i2 + 1])), nd2[i2]));
-          pk[i2] = pair_pack_bf16(p.x, p.y, perm);
-          dk[i2] = pair_pack_bf16(ds.x, ds.y, perm);
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t recv = __shfl_xor_sync(0xffffffffu, kind ? da[i] : sa[16 + i], 1);
+          sv[i] = __uint_as_float(kind ? recv : sa[i]);
+          dv[i] = __uint_as_float(kind ? da[16 + i] : recv);
         }
-        tmem_st16x64b_x16(tl + TM_S, pk);
-        tmem_st16x64b_x16(tl + TM_DP, dk);
+        const float2* nl = reinterpret_cast<const float2*>(dsm + st * STAGE_B + 4 * TILE_B) + 16 * c + 8 * kind;
+        const float2* nd = nl + 32;
+        uint32_t own[8], other[8];  // packed bf16 pairs: even lanes own P, odd lanes own dS
+#pragma unroll
+        for (int i2 = 0; i2 < 8; ++i2) {
+          const float2 arg = __ffma2_rn(make_float2(sv[2 * i2], sv[2 * i2 + 1]), cc, nl[i2]);
+          const float2 p = make_float2(ex2(arg.x), ex2(arg.y));
+          const float2 ds = __fmul2_rn(p, __fadd2_rn(make_float2(dv[2 * i2], dv[2 * i2 + 1]), nd[i2]));
+          const uint32_t wp = pack_bf16(p.x, p.y), wd = pack_bf16(ds.x, ds.y);
+          own[i2] = kind ? wd : wp;
+          other[i2] = kind ? wp : wd;
+        }
+        // even lanes' row is P^T, odd lanes' dS^T: swap the halves the other lane needs
+        uint32_t row16[16];
+#pragma unroll
+        for (int i2 = 0; i2 < 8; ++i2) {
+          const uint32_t r = __shfl_xor_sync(0xffffffffu, other[i2], 1);
+          row16[i2] = kind ? r : own[i2];
+          row16[8 + i2] = kind ? own[i2] : r;
+        }
+        if (n >= 2) mbar_wait(&B.pdsfree[b], ((n >> 1) - 1) & 1, abort, ctx);  // second MMA of n - 2
+        tmem_st32x16(tl + TM_PDS + 32 * b + 16 * c, row16);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&B.pfull[s]);
+        if (lane == 0) mbar_arrive(&B.pdsfull[b]);
       }
-      mbar_wait(&B.bdone[s], (g - 1) & 1, abort, ctx);
+      // epilogue: the item's MMAs are done; this lane's half row of dV (even) or dK (odd)
+      mbar_wait(&B.itemdone, it & 1, abort, ctx);
+      ++it;
       tc_fence_after();
-      uint32_t o[64];
-      tmem_ld16x64b_x64(tl + TM_DV, o);
-      tmem_ld_wait();
-      store_row_f32(dvd, o, 1.f, par_c);
-      tmem_ld16x64b_x64(tl + TM_DK, o);
-      tmem_ld_wait();
-      store_row_f32(dkd, o, scale, par_c);
-      if (named_bar_or(bar_id, 128, *abort != 0)) break;
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t gk[32], gv[32];
+        tmem_ld32(tl + TM_G + 128 * c + 32 * h2, gk);       // dK columns of d half c (odd lanes)
+        tmem_ld32(tl + TM_G + 128 * c + 64 + 32 * h2, gv);  // dV columns of d half c (even lanes)
+        tmem_ld_wait();
+        float4* dst = reinterpret_cast<float4*>(gout + 32 * h2);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint32_t* src = kind ? gk + 4 * e : gv + 4 * e;
+          const float f = kind ? scale : 1.f;
+          dst[e] = make_float4(__uint_as_float(src[0]) * f, __uint_as_float(src[1]) * f, __uint_as_float(src[2]) * f,
+                               __uint_as_float(src[3]) * f);
+        }
+      }
+      if (named_bar_or(1, 256, *abort != 0)) break;
     }
   }
   tc_fence_before();
@@ -655,7 +688,8 @@ vsa2_status attn_bwd_tc(const Dims& d, const void* q, const void* k, const void*
       kv_idx, dq, d.N, (int)d.L, topk, items, c2, c1, ctx);
   if (check_launch("attn_bwd_dq_tc_kernel") != VSA2_OK) return VSA2_ERR_CUDA;
   cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dkv::SMEM_DYN);
-  attn_bwd_dkdv_tc_kernel<<<grid, BT, dkv::SMEM_DYN, s>>>(tq, tdo, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+  const int grid_kv = std::max(1, std::min(sms, items));
+  attn_bwd_dkdv_tc_kernel<<<grid_kv, dkv::KT, dkv::SMEM_DYN, s>>>(tq, tdo, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
                                                           nlse2, ndelta, q_off, q_idx, dk, dv, d.N, (int)d.L, topk,
                                                           items, c2, c1, ctx);
   return check_launch("attn_bwd_dkdv_tc_kernel");

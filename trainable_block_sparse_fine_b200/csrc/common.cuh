@@ -221,6 +221,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+// 32 lanes x 32 bit, 16 consecutive columns: thread t of the warp writes lane (base + t).
+__device__ __forceinline__ void tmem_st32x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 // 16 lanes x 64 bit, 64 repetitions: thread t gets lane (8*(t&1) + t/4) of the 16-lane group at
 // `taddr` and the 32-bit columns 2i + ((t>>1)&1), i = 0..63.
 __device__ __forceinline__ void tmem_ld16x64b_x64(uint32_t taddr, uint32_t (&r)[64]) {
