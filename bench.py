@@ -264,9 +264,15 @@ def run_ours(args, wl):
     # weak scaling: every rank runs the full workload on its own batch element (seed offset)
     wl_r = wl.with_(seed=wl.seed + rank)
     names = ("q", "k", "v", "do") if wl.backward else ("q", "k", "v")
-    host = {n: S.make_tensor(wl_r, n) for n in names}
     dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
-    pinned = {n: torch.from_numpy(host[n]).to(dt).pin_memory() for n in names}
+    # inputs in pinned host memory (the end-to-end leg copies them every step); each fp32 array
+    # is dropped once converted, and the generator's worker pool is shared by the ranks of a node
+    workers = max(1, min(16, len(os.sched_getaffinity(0)) // max(1, int(os.environ.get("LOCAL_WORLD_SIZE", world)))))
+    pinned = {}
+    for n in names:
+        a32 = S.make_tensor(wl_r, n, workers=workers)
+        pinned[n] = torch.from_numpy(a32).to(dt).pin_memory()
+        del a32
     x = {n: pinned[n].to(dev) for n in names}
     e = V.VSA2(wl.batch, wl.heads, wl.head_dim, wl.grid, wl.dtype, wl.topk)
     stream = torch.cuda.current_stream()
