@@ -125,6 +125,12 @@ __global__ void __launch_bounds__(1024) topk_select_digit_kernel(const uint32_t*
 }
 
 // Warp per row: entries above the threshold and entries equal to it.
+// Every row of a scores block starts on a 16-byte boundary when the block itself does and N is
+// a multiple of 4; then rows are read as float4.
+__device__ __forceinline__ bool rows_vec4(const float* scores, int N) {
+  return (N & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0;
+}
+
 __global__ void __launch_bounds__(256) topk_row_count_kernel(const float* __restrict__ scores, int N,
                                                              const uint32_t* __restrict__ state,
                                                              int32_t* __restrict__ row_gt, int32_t* __restrict__ row_eq) {
@@ -134,10 +140,21 @@ __global__ void __launch_bounds__(256) topk_row_count_kernel(const float* __rest
   const uint32_t T = state[bh * 8 + ST_THRESH];
   const float* s = scores + ((size_t)bh * N + row) * N;
   int gt = 0, eq = 0;
-  for (int j = lane; j < N; j += 32) {
-    const uint32_t key = score_key(__ldg(s + j));
-    gt += key > T;
-    eq += key == T;
+  if (rows_vec4(scores, N)) {  // four columns per lane and load
+    const float4* s4 = reinterpret_cast<const float4*>(s);
+#pragma unroll 4
+    for (int q = lane; q < (N >> 2); q += 32) {
+      const float4 v = __ldg(s4 + q);
+      const uint32_t k0 = score_key(v.x), k1 = score_key(v.y), k2 = score_key(v.z), k3 = score_key(v.w);
+      gt += (k0 > T) + (k1 > T) + (k2 > T) + (k3 > T);
+      eq += (k0 == T) + (k1 == T) + (k2 == T) + (k3 == T);
+    }
+  } else {
+    for (int j = lane; j < N; j += 32) {
+      const uint32_t key = score_key(__ldg(s + j));
+      gt += key > T;
+      eq += key == T;
+    }
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) {
@@ -198,6 +215,57 @@ __global__ void __launch_bounds__(256) topk_emit_kernel(const float* __restrict_
   int32_t* out = kv_idx + (size_t)bh * N * topk;
   int written = 0, ties_seen = 0;
   const uint32_t lt_mask = (1u << lane) - 1u;
+  if (rows_vec4(scores, N)) {
+    // four consecutive columns per lane (lane-major order is column order): per element slot one
+    // ballot for ties and one for selections; positions add the lower lanes' counts to the
+    // lane's own prefix
+    const float4* s4 = reinterpret_cast<const float4*>(s);
+#pragma unroll 2
+    for (int j0 = 0; j0 < N; j0 += 128) {
+      const int jl = j0 + 4 * lane;
+      const bool valid = jl < N;
+      const float4 v = valid ? __ldg(s4 + (jl >> 2)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const uint32_t key[4] = {score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w)};
+      uint32_t eqm[4];
+      int ties_before = ties_seen;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        eqm[e] = __ballot_sync(0xffffffffu, valid && key[e] == T);
+        ties_before += __popc(eqm[e] & lt_mask);
+      }
+      bool sel[4];
+      int tr = ties_before;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool is_eq = valid && key[e] == T;
+        sel[e] = valid && (key[e] > T || (is_eq && tr < take));
+        tr += is_eq;
+      }
+      int pos = base + written, nsel = 0, nties = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t selm = __ballot_sync(0xffffffffu, sel[e]);
+        pos += __popc(selm & lt_mask);
+        nsel += __popc(selm);
+        nties += __popc(eqm[e]);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (!sel[e]) continue;
+        const int j = jl + e;
+        if (pos < next) out[pos] = j;
+        ++pos;
+        if (col_cnt) {
+          atomicAdd(&col_cnt[(size_t)bh * N + j], 1);
+          atomicOr(&col_bits[((size_t)bh * N + j) * words + (row >> 5)], 1u << (row & 31));
+        }
+      }
+      written += nsel;
+      ties_seen += nties;
+    }
+    if ((ctx.flags & VSA2_FLAG_VALIDATE) && lane == 0 && base + written != next) set_error(ctx.err, VSA2_ERR_BAD_INDEX);
+    return;
+  }
   for (int j0 = 0; j0 < N; j0 += 32) {
     const int j = j0 + lane;
     const uint32_t key = j < N ? score_key(__ldg(s + j)) : 0u;
