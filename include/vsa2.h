@@ -9,8 +9,9 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- *  - All tensor arguments are DEVICE pointers owned by the caller. The library never
- *    allocates or frees device memory and never synchronises, except vsa2_get_device_error.
+ *  - All tensor arguments are DEVICE pointers owned by the caller, except the host buffers of
+ *    vsa2_forward_host. The library never allocates or frees device memory and never
+ *    synchronises, except vsa2_get_device_error.
  *    Every compute call only enqueues kernels on `stream` (a cudaStream_t; NULL = the legacy
  *    default stream) and returns.
  *  - Token layout: Q, K, V, O, dO, dQ, dK, dV are [batch, heads, L, head_dim] row-major
@@ -138,6 +139,39 @@ vsa2_status vsa2_sparse_attn_bwd(const vsa2_problem* p, const void* q, const voi
                                  const int32_t* q_off, const int32_t* q_idx,
                                  float* dq, float* dk, float* dv,
                                  void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * End-to-end forward from HOST memory: router (Eq. 5-7), per-sequence TopK (Eq. 8-9) and
+ * block-sparse attention (Eq. 12) for inputs and outputs that live in host memory. It computes
+ * exactly what vsa2_router_scores + vsa2_topk_select + vsa2_sparse_attn_fwd compute on device
+ * copies of the same inputs (bit-identical O and LSE).
+ *   q, k, v  : HOST pointers, [batch, heads, L, D] of dtype (read only). Page-locked memory
+ *              (cudaHostAlloc / cudaHostRegister) lets the copies overlap the kernels; pageable
+ *              memory works but the host-to-device copies then block the calling thread.
+ *   topk     : per-tile budget as for vsa2_topk_select
+ *   heads_per_group : flat (b, h) indices processed per group, >= 0; 0 picks a group of at
+ *              least 65536 tokens (one head at 720p)
+ *   o        : HOST pointer, [batch, heads, L, D] of dtype (written)
+ *   lse      : HOST pointer, [batch, heads, L] fp32 (written), or NULL
+ *   ws       : DEVICE workspace of vsa2_forward_host_workspace_size() bytes, 256-byte aligned,
+ *              initialised by vsa2_workspace_init. It holds the kernels' workspace (its error
+ *              word is read by vsa2_get_device_error), one group's scores and CSR, and three
+ *              staging slots of one group's Q, K, V, O and LSE.
+ * The flat (b, h) range is cut into groups; group g's host-to-device copies, its kernels on
+ * `stream`, and its device-to-host copies run as three chains, so that the copies of
+ * neighbouring groups overlap group g's kernels. The copies run on two library-owned streams
+ * that wait for the work already queued on `stream` and that `stream` waits for before any
+ * later work: the outputs are in host memory once `stream` has been synchronised. The library
+ * creates those two streams and a few events on the first call on each device and keeps them
+ * for the process; concurrent calls from several host threads are serialised while they
+ * enqueue. Argument errors return before anything is enqueued; a failed copy or launch
+ * returns VSA2_ERR_CUDA after the streams have been joined.
+ */
+size_t vsa2_forward_host_workspace_size(const vsa2_problem* p, int32_t topk, int32_t heads_per_group);
+
+vsa2_status vsa2_forward_host(const vsa2_problem* p, const void* q, const void* k, const void* v, int32_t topk,
+                              int32_t heads_per_group, void* o, float* lse, void* ws, size_t ws_bytes,
+                              void* stream);
 
 /*
  * Per-sequence TopK like vsa2_topk_select (same ranking, same CSR output, no CSC), for callers

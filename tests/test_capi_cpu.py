@@ -79,3 +79,30 @@ def test_argument_errors_are_synchronous():
     bad.dtype = 7
     assert lib.vsa2_router_scores(ctypes.byref(bad), fake, fake, fake, ws, n, None) == 2
     assert lib.vsa2_selftest_wait_timeout(ws, n, 0, None) == 1
+
+
+def test_forward_host_workspace_and_argument_errors():
+    lib = C.lib()
+    p = C.make_problem(1, 5, 128, (8, 16, 20))  # N = 40, L = 2560
+    bp = ctypes.byref(p)
+    one = C.vsa2_forward_host_workspace_size(p, 6, 1)
+    two = C.vsa2_forward_host_workspace_size(p, 6, 2)
+    auto = C.vsa2_forward_host_workspace_size(p, 6, 0)
+    everything = C.vsa2_forward_host_workspace_size(p, 6, 5)
+    assert 0 < one < two < auto and one % 256 == 0
+    assert auto == everything  # 65536 tokens round up to all five heads here
+    assert C.vsa2_forward_host_workspace_size(p, 6, 9) == everything  # clamped to the head count
+    # three staging slots of Q, K, V, O (bf16) and LSE (fp32) for one head at least
+    assert one >= 3 * (4 * 2560 * 128 * 2 + 2560 * 4)
+    assert C.vsa2_forward_host_workspace_size(p, 0, 1) == 0
+    assert C.vsa2_forward_host_workspace_size(p, 41, 1) == 0
+    assert C.vsa2_forward_host_workspace_size(p, 6, -1) == 0
+    host = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails before any copy
+    ws = ctypes.c_void_p(1 << 24)
+    assert lib.vsa2_forward_host(bp, None, host, host, 6, 1, host, None, ws, one, None) == 1
+    assert lib.vsa2_forward_host(bp, host, host, host, 6, 1, None, None, ws, one, None) == 1
+    assert lib.vsa2_forward_host(bp, host, host, host, 6, 1, host, None, ws, one - 256, None) == 1
+    assert lib.vsa2_forward_host(bp, host, host, host, 6, 1, host, None, ctypes.c_void_p((1 << 24) + 16), one,
+                                 None) == 1
+    assert lib.vsa2_forward_host(bp, host, host, host, 6, -1, host, None, ws, one, None) == 1
+    assert lib.vsa2_forward_host(bp, host, host, host, 0, 1, host, None, ws, one, None) == 2

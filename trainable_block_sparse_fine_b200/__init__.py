@@ -11,14 +11,15 @@ from __future__ import annotations
 
 import torch
 
-from ._capi import (VSA2_FLAG_VALIDATE, Problem, Vsa2Error, lib, make_problem, vsa2_get_device_error,
-                    vsa2_router_scores, vsa2_selftest_wait_timeout, vsa2_sparse_attn_bwd, vsa2_sparse_attn_fwd,
-                    vsa2_status_string, vsa2_topk_select, vsa2_version, vsa2_workspace_init, vsa2_workspace_size)
+from ._capi import (VSA2_FLAG_VALIDATE, Problem, Vsa2Error, lib, make_problem, vsa2_forward_host,
+                    vsa2_forward_host_workspace_size, vsa2_get_device_error, vsa2_router_scores,
+                    vsa2_selftest_wait_timeout, vsa2_sparse_attn_bwd, vsa2_sparse_attn_fwd, vsa2_status_string,
+                    vsa2_topk_select, vsa2_version, vsa2_workspace_init, vsa2_workspace_size)
 
 __all__ = ["VSA2", "Vsa2Error", "Problem", "make_problem", "block_sparse_attention", "lib", "VSA2_FLAG_VALIDATE",
            "vsa2_router_scores", "vsa2_topk_select", "vsa2_sparse_attn_fwd", "vsa2_sparse_attn_bwd",
            "vsa2_workspace_size", "vsa2_workspace_init", "vsa2_get_device_error", "vsa2_selftest_wait_timeout",
-           "vsa2_status_string", "vsa2_version"]
+           "vsa2_status_string", "vsa2_version", "vsa2_forward_host", "vsa2_forward_host_workspace_size"]
 
 
 class VSA2:
@@ -41,7 +42,7 @@ class VSA2:
         self.ws = torch.empty((n + 255) // 256 * 256, dtype=torch.uint8, device=self.device)
         vsa2_workspace_init(self.ws)
 
-    # -- the four calls of the hot path -----------------------------------------------------
+    # -- the calls of the hot path -----------------------------------------------------------
     def router_scores(self, q, k, out=None):
         out = out if out is not None else torch.empty(self.batch, self.heads, self.N, self.N, dtype=torch.float32,
                                                       device=self.device)
@@ -81,8 +82,30 @@ class VSA2:
         o, lse = self.attn_fwd(q, k, v, sel[0], sel[1], topk)
         return o, lse, sel
 
+    def forward_host(self, q, k, v, topk=None, o=None, lse=None, heads_per_group=0, want_lse=False):
+        """Router -> TopK -> forward on HOST tensors, copies overlapped with the kernels per group of
+        heads (vsa2_forward_host). Returns (o, lse) in host memory once the current stream has been
+        synchronised; lse is None unless requested."""
+        topk = self.topk if topk is None else topk
+        n = vsa2_forward_host_workspace_size(self.p, topk, heads_per_group)
+        if n == 0:
+            raise Vsa2Error(2, "vsa2_forward_host_workspace_size")
+        key = (topk, heads_per_group)
+        if getattr(self, "_host_ws_key", None) != key:
+            self.ws_host = torch.empty((n + 255) // 256 * 256, dtype=torch.uint8, device=self.device)
+            vsa2_workspace_init(self.ws_host)
+            self._host_ws_key = key
+        o = o if o is not None else torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        if want_lse and lse is None:
+            lse = torch.empty(self.batch, self.heads, self.L, dtype=torch.float32, pin_memory=True)
+        vsa2_forward_host(self.p, q, k, v, topk, heads_per_group, o, lse, self.ws_host)
+        return o, lse
+
     def device_error(self) -> int:
-        return vsa2_get_device_error(self.ws)
+        err = vsa2_get_device_error(self.ws)
+        if err == 0 and getattr(self, "ws_host", None) is not None:
+            err = vsa2_get_device_error(self.ws_host)
+        return err
 
 
 class _BlockSparseAttention(torch.autograd.Function):

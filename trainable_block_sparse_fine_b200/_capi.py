@@ -20,7 +20,7 @@ VSA2_FLAG_VALIDATE = 1
 EXPORTS = ("vsa2_workspace_size", "vsa2_workspace_init", "vsa2_router_scores", "vsa2_topk_select",
            "vsa2_sparse_attn_fwd", "vsa2_sparse_attn_bwd", "vsa2_get_device_error",
            "vsa2_selftest_wait_timeout", "vsa2_status_string", "vsa2_version", "vsa2_last_cuda_error",
-           "vsa2_topk_select_noalloc")
+           "vsa2_topk_select_noalloc", "vsa2_forward_host", "vsa2_forward_host_workspace_size")
 
 
 class Vsa2Error(RuntimeError):
@@ -58,6 +58,9 @@ def lib() -> ctypes.CDLL:
         L.vsa2_sparse_attn_fwd.argtypes = [P, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]
         L.vsa2_sparse_attn_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.vsa2_topk_select_noalloc.argtypes = [P, vp, i32, vp, vp, vp]
+        L.vsa2_forward_host_workspace_size.argtypes = [P, i32, i32]
+        L.vsa2_forward_host_workspace_size.restype = sz
+        L.vsa2_forward_host.argtypes = [P, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
         L.vsa2_get_device_error.argtypes = [vp, vp]
         L.vsa2_selftest_wait_timeout.argtypes = [vp, sz, u32, vp]
         L.vsa2_status_string.argtypes = [ctypes.c_int]
@@ -65,7 +68,7 @@ def lib() -> ctypes.CDLL:
         L.vsa2_version.restype = i32
         L.vsa2_last_cuda_error.restype = ctypes.c_char_p
         for name in ("vsa2_workspace_init", "vsa2_router_scores", "vsa2_topk_select", "vsa2_topk_select_noalloc",
-                     "vsa2_sparse_attn_fwd",
+                     "vsa2_sparse_attn_fwd", "vsa2_forward_host",
                      "vsa2_sparse_attn_bwd", "vsa2_get_device_error", "vsa2_selftest_wait_timeout"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -140,6 +143,20 @@ def vsa2_sparse_attn_bwd(p: Problem, q, k, v, o, lse, dout, topk, kv_off, kv_idx
                                       topk, _ptr(kv_off), _ptr(kv_idx), _ptr(q_off), _ptr(q_idx), _ptr(dq), _ptr(dk),
                                       _ptr(dv), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "vsa2_sparse_attn_bwd")
+
+
+def vsa2_forward_host_workspace_size(p: Problem, topk: int, heads_per_group: int = 0) -> int:
+    return lib().vsa2_forward_host_workspace_size(ctypes.byref(p), topk, heads_per_group)
+
+
+def vsa2_forward_host(p: Problem, q, k, v, topk, heads_per_group, o, lse, ws, stream=None) -> None:
+    """q, k, v, o, lse are HOST tensors (page-locked for overlap); lse may be None."""
+    for t in (q, k, v, o, lse):
+        if isinstance(t, torch.Tensor) and t.is_cuda:
+            raise ValueError("vsa2_forward_host takes host tensors")
+    _check(lib().vsa2_forward_host(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), topk, heads_per_group, _ptr(o),
+                                   _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "vsa2_forward_host")
 
 
 def vsa2_get_device_error(ws, stream=None) -> int:

@@ -39,8 +39,8 @@ struct WsLayout {
   size_t col_bits;       // [BH, N, words] u32
   int words;             // ceil(N / 32)
   size_t delta;          // backward rowsum(dO * O), [BH, L] fp32 (the tcgen05 backward keeps
-                         // -Delta here, each 64-row tile ordered even rows then odd rows)
-  size_t nlse2;          // tcgen05 backward: -lse * log2(e), [BH, L] fp32, same tile order
+                         // -Delta here, in token order)
+  size_t nlse2;          // tcgen05 backward: -lse * log2(e), [BH, L] fp32, token order
   size_t total;
 };
 WsLayout ws_layout(const Dims& d);
