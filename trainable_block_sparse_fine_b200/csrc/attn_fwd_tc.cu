@@ -16,8 +16,11 @@
 // rows of its slot; the 16x64b TMEM access gives each row to a pair of threads (even / odd
 // columns), so row max and row sum need one shuffle and no block-level barrier. The two slots
 // are independent pipelines sharing only the tensor pipe: warps 8 and 10 load the K and V
-// blocks of slot 0 and slot 1 into the slot's own rings, warps 9 and 11 issue its MMAs. The running max is raised (with an O rescale in
-// TMEM) only when a row's new maximum exceeds it by more than 2^8.
+// blocks of slot 0 and slot 1 into the slot's own ring, warps 9 and 11 issue its MMAs. The ring
+// holds K and V blocks alike, in the slot's op order, so each block is requested three ops ahead
+// of its MMA: V(i) as soon as S(i) has read K(i), K(i+1) once O(i-2) has read V(i-2). The running
+// max is raised (with an O rescale in TMEM) only when a row's new maximum exceeds it by more
+// than 2^8.
 #include <algorithm>
 
 #include "common.cuh"
@@ -29,14 +32,12 @@ namespace {
 constexpr int FT = 384;            // 12 warps
 constexpr uint32_t TILE_B = 8192;  // one 64x64 bf16 box (64 rows x 128 B)
 constexpr uint32_t BLK_B = 32768;  // K or V block: [half0: tile A, tile B][half1: tile A, tile B]
-constexpr int KST = 2;             // K ring stages per slot
-constexpr int VST = 1;             // V ring stages per slot
+constexpr int RST = 3;             // ring stages per slot (K and V blocks in op order)
 
-// Each slot has its own K and V rings (one producer, one consumer each), so every barrier wait
-// is for the phase in progress or the one just completed.
-constexpr uint32_t OFF_K = 0;                              // [slot][KST] blocks
-constexpr uint32_t OFF_V = OFF_K + 2 * KST * BLK_B;        // [slot][VST] blocks
-constexpr uint32_t OFF_BAR = OFF_V + 2 * VST * BLK_B;
+// Each slot has its own ring (one producer, one consumer, both in the slot's op order), so
+// every barrier wait is for the phase in progress or the one just completed.
+constexpr uint32_t OFF_RING = 0;                           // [slot][RST] blocks
+constexpr uint32_t OFF_BAR = OFF_RING + 2 * RST * BLK_B;
 constexpr uint32_t OFF_FLAG = OFF_BAR + 512;
 constexpr uint32_t SMEM_USED = OFF_FLAG + 64;
 constexpr uint32_t SMEM_DYN = SMEM_USED + 1024;
@@ -51,7 +52,7 @@ constexpr uint32_t TM_COLS = 512;
 constexpr float kThresh = 8.0f;   // log2 headroom before the running max must move
 
 struct Bars {
-  uint64_t kfull[2][KST], kempty[2][KST], vfull[2][VST], vempty[2][VST];  // [slot][stage]
+  uint64_t full[2][RST], empty[2][RST];                                    // [slot][stage]
   uint64_t sfull[2][2], sfree[2][2];                                       // [slot][buffer]
   uint64_t pfull[2], pvdone[2], qready[2];
   uint64_t done[2];
@@ -140,8 +141,7 @@ __global__ void __launch_bounds__(FT, 1)
   if (threadIdx.x == 0) {
     flag_sh[0] = 0;
     for (int s = 0; s < 2; ++s) {
-      for (int i = 0; i < KST; ++i) mbar_init(&B.kfull[s][i], 1), mbar_init(&B.kempty[s][i], 1);
-      for (int i = 0; i < VST; ++i) mbar_init(&B.vfull[s][i], 1), mbar_init(&B.vempty[s][i], 1);
+      for (int i = 0; i < RST; ++i) mbar_init(&B.full[s][i], 1), mbar_init(&B.empty[s][i], 1);
       for (int b = 0; b < 2; ++b) mbar_init(&B.sfull[s][b], 1), mbar_init(&B.sfree[s][b], 4);
       mbar_init(&B.pfull[s], 4);
       mbar_init(&B.pvdone[s], 1);
@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(FT, 1)
       tma_prefetch_desc(&tm_v);
       SlotSeq sq;
       sq.init(2 * blockIdx.x + s, step, items);
-      int kc = 0, vc = 0;
+      int c = 0;  // ring position: blocks requested so far
       bool ok = true;
       while (ok && sq.active) {
         int blk;
@@ -186,26 +186,20 @@ __global__ void __launch_bounds__(FT, 1)
           }
           j[tt] = v;
         }
-        const int c = k_op ? kc : vc, nst = k_op ? KST : VST, st = c % nst;
-        uint64_t* empty = k_op ? &B.kempty[s][st] : &B.vempty[s][st];
-        uint64_t* full = k_op ? &B.kfull[s][st] : &B.vfull[s][st];
-        uint8_t* dst = dsm + (k_op ? OFF_K + (s * KST + st) * BLK_B : OFF_V + (s * VST + st) * BLK_B);
-        if (!(ok = mbar_wait(empty, ((c / nst) & 1) ^ 1, abort, ctx))) break;
+        const int st = c % RST;
+        uint64_t* full = &B.full[s][st];
+        uint8_t* dst = dsm + OFF_RING + (s * RST + st) * BLK_B;
+        if (!(ok = mbar_wait(&B.empty[s][st], ((c / RST) & 1) ^ 1, abort, ctx))) break;
         mbar_arrive_expect_tx(full, ntile * 2 * TILE_B);
         for (int tt = 0; tt < ntile; ++tt)
           for (int h = 0; h < 2; ++h)
             tma_load_2d(dst + h * 2 * TILE_B + tt * TILE_B, k_op ? &tm_k : &tm_v, h * 64, sq.bh * L + j[tt] * 64,
                         full);
-        if (k_op)
-          ++kc;
-        else
-          ++vc;
+        ++c;
       }
       if (*abort) {  // let copies still in flight land before the CTA exits
-        for (int cc = max(0, kc - KST); cc < kc; ++cc)
-          mbar_wait_drain(&B.kfull[s][cc % KST], (cc / KST) & 1, ctx.timeout_ns);
-        for (int cc = max(0, vc - VST); cc < vc; ++cc)
-          mbar_wait_drain(&B.vfull[s][cc % VST], (cc / VST) & 1, ctx.timeout_ns);
+        for (int cc = max(0, c - RST); cc < c; ++cc)
+          mbar_wait_drain(&B.full[s][cc % RST], (cc / RST) & 1, ctx.timeout_ns);
       }
     }
   } else if (warp == 9 || warp == 11) {
@@ -218,37 +212,40 @@ __global__ void __launch_bounds__(FT, 1)
       SlotSeq sq;
       sq.init(2 * blockIdx.x + s, step, items);
       int kc = 0, vc = 0;  // S and O blocks issued
+      int c = 0;           // ring position
       bool ok = true;
       while (ok && sq.active) {
         int blk;
         const int op = next_op(sq, &blk, kv_off, N, cap, ctx);
         if (op == 1) {
           if (blk == 0 && !(ok = mbar_wait(&B.qready[s], (sq.tile - 1) & 1, abort, ctx))) break;
-          const int st = kc % KST;
-          if (!(ok = mbar_wait(&B.kfull[s][st], (kc / KST) & 1, abort, ctx))) break;
+          const int st = c % RST;
+          if (!(ok = mbar_wait(&B.full[s][st], (c / RST) & 1, abort, ctx))) break;
           if (!(ok = mbar_wait(&B.sfree[s][kc & 1], ((kc >> 1) & 1) ^ 1, abort, ctx))) break;
           tc_fence_after();
-          const uint32_t ka = smem_u32(dsm + OFF_K + (s * KST + st) * BLK_B);
+          const uint32_t ka = smem_u32(dsm + OFF_RING + (s * RST + st) * BLK_B);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_bf16_ts(tmem + lanes + TM_S + (kc & 1) * 128, tmem + lanes + TM_Q + 8 * kk,
                         sdesc_sw128(ka + (kk >> 2) * 2 * TILE_B + (kk & 3) * 32, 16, 1024), id_s, kk > 0);
-          mma_commit(&B.kempty[s][st]);
+          mma_commit(&B.empty[s][st]);
           mma_commit(&B.sfull[s][kc & 1]);
           ++kc;
+          ++c;
         } else if (op == 2) {
-          const int st = vc % VST;
-          if (!(ok = mbar_wait(&B.vfull[s][st], (vc / VST) & 1, abort, ctx))) break;
+          const int st = c % RST;
+          if (!(ok = mbar_wait(&B.full[s][st], (c / RST) & 1, abort, ctx))) break;
           if (!(ok = mbar_wait(&B.pfull[s], vc & 1, abort, ctx))) break;
           tc_fence_after();
-          const uint32_t va = smem_u32(dsm + OFF_V + (s * VST + st) * BLK_B);
+          const uint32_t va = smem_u32(dsm + OFF_RING + (s * RST + st) * BLK_B);
           const int ksteps = (2 * blk + 1 == sq.len) ? 4 : 8;
           for (int kk = 0; kk < ksteps; ++kk)
             mma_bf16_ts(tmem + lanes + TM_O, tmem + lanes + TM_P + 8 * kk,
                         sdesc_sw128(va + kk * 2048, 2 * TILE_B, 1024), id_o, (blk > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&B.vempty[s][st]);
+          mma_commit(&B.empty[s][st]);
           mma_commit(&B.pvdone[s]);
           ++vc;
+          ++c;
         }
       }
       mma_commit(&B.done[s]);
