@@ -5,7 +5,8 @@ baseline leg may import this module. The product path (the CUDA library and its 
 binding) never calls it and shares no code with it.
 
 Source: "Improving Video Sparse Attention with Fine-grained Router and Sparse Rebasing"
-(arXiv 2609.32882), §2.1 Background and §2.2 VSA2, Eq. 5-9 and Eq. 12.
+(arXiv 2609.32882), §2.1 Background and §2.2 VSA2: Eq. 5-9 (router, TopK), Eq. 12 (fine
+branch), Eq. 1-4 (coarse branch) and Eq. 13-14 (gated merge).
 
 Layout: every per-(b, h) tensor is (L, D) in cube-major token order (§2.2 "Permutation"):
 tile i is rows [i*Bt, (i+1)*Bt); inside it, router sub-cube a is rows [a*R, (a+1)*R), so tile i
@@ -19,6 +20,8 @@ Readings of the pages that this oracle commits to (each is listed in the design 
     go to the lower flat index i*N + j. The budget N*K is per (batch, head).
   * Eq. 12 for a query tile with no selected KV tile: output 0, LSE = -inf, zero gradients.
   * Softmax scale 1/sqrt(D) (§2.1).
+  * Eq. 13's gate G = tanh(X W_g) takes the projection X W_g (one value per token and head) as
+    its input: the projection of the hidden states belongs with the layer's input projections.
 """
 from __future__ import annotations
 
@@ -31,6 +34,8 @@ __all__ = [
     "topk_select",
     "sparse_attn_fwd",
     "sparse_attn_bwd",
+    "coarse_attn",
+    "gated_merge",
 ]
 
 
@@ -208,3 +213,33 @@ def sparse_attn_bwd(q, k, v, do, kv_off, kv_idx, tile_tokens: int = 64, query_ti
         np.add.at(dk, sel, dks.reshape(n, tile_tokens, D))
         np.add.at(dv, sel, dvs.reshape(n, tile_tokens, D))
     return dq.reshape(L, D), dk.reshape(L, D), dv.reshape(L, D)
+
+
+def coarse_attn(q, k, v, tile_tokens: int = 64):
+    """Coarse branch for one (b, h), Eq. 1-3:
+    Qc, Kc, Vc = MeanPool_B(Q, K, V)            (Eq. 1), one row per tile, (N, D)
+    P_c        = row-softmax(Qc Kc^T / sqrt(D)) (Eq. 2), over all N tiles
+    O_c_hat    = P_c Vc                         (Eq. 3)
+    Returns (O_c_hat (N, D) fp64, lse_c (N,) fp64 = log of each row's softmax denominator).
+    """
+    qc = mean_pool(q, tile_tokens)
+    kc = mean_pool(k, tile_tokens)
+    vc = mean_pool(v, tile_tokens)
+    D = qc.shape[1]
+    s = (qc @ kc.T) / np.sqrt(D)
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    l = p.sum(axis=1, keepdims=True)
+    return (p @ vc) / l, (m + np.log(l))[:, 0]
+
+
+def gated_merge(o_f, o_c_hat, gate_logits, tile_tokens: int = 64):
+    """Output of one (b, h), Eq. 4 and Eq. 13-14:
+    O_c = Repeat_B(O_c_hat)       (Eq. 4), every token of tile i gets row i
+    G   = tanh(X W_g)             (Eq. 13), gate_logits = X W_g, one per token, shape (L,)
+    O   = G * O_c + O_f           (Eq. 14), G broadcast over the D channels
+    """
+    o_f = np.asarray(o_f, dtype=np.float64)
+    o_c = np.repeat(np.asarray(o_c_hat, dtype=np.float64), tile_tokens, axis=0)
+    g = np.tanh(np.asarray(gate_logits, dtype=np.float64))[:, None]
+    return g * o_c + o_f

@@ -418,3 +418,91 @@ def test_bwd_given_output_enters_only_through_rowsum():
     p /= p.sum(1, keepdims=True)
     want = base[0][:64] - (0.5 * np.sum(do[:64] ** 2, 1))[:, None] * (p @ ks) / math.sqrt(D)
     np.testing.assert_allclose(shift[0][:64], want, rtol=1e-10, atol=1e-11)
+
+
+# --------------------------------------------------------------------------------------------
+# coarse branch, Eq. 1-4, and gated merge, Eq. 13-14
+# --------------------------------------------------------------------------------------------
+
+def _coarse_bruteforce(xq, xk, xv):
+    """Eq. 1-3 restated on the raster grid with explicit loops: the mean of every 4x4x4 cube of
+    Q, K and V (cubes in raster order), then softmax attention from each cube to all cubes."""
+    T, H, W, D = xq.shape
+    nt, nh, nw = T // 4, H // 4, W // 4
+    means = {n: [] for n in "qkv"}
+    for a, b, c in itertools.product(range(nt), range(nh), range(nw)):
+        for n, x in zip("qkv", (xq, xk, xv)):
+            acc = np.zeros(D)
+            for dt, dh, dw in itertools.product(range(4), repeat=3):
+                acc += x[4 * a + dt, 4 * b + dh, 4 * c + dw]
+            means[n].append(acc / 64.0)
+    N = len(means["q"])
+    out, lse = np.zeros((N, D)), np.zeros(N)
+    for i in range(N):
+        logits = [float(means["q"][i] @ kj) / math.sqrt(D) for kj in means["k"]]
+        m = max(logits)
+        ex = [math.exp(z - m) for z in logits]
+        z = sum(ex)
+        out[i] = sum(e * vj for e, vj in zip(ex, means["v"])) / z
+        lse[i] = m + math.log(z)
+    return out, lse
+
+
+@pytest.mark.parametrize("grid,d", [((4, 8, 8), 8), ((8, 8, 12), 16)])
+def test_coarse_matches_bruteforce_on_raster_grid(grid, d):
+    xq, xk, xv = (_raster_inputs(grid, d, s) for s in (11, 12, 13))
+    want_o, want_lse = _coarse_bruteforce(xq, xk, xv)
+    o, lse = O.coarse_attn(*(S.raster_to_cube_major(x, TILE, POOL) for x in (xq, xk, xv)))
+    np.testing.assert_allclose(o, want_o, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(lse, want_lse, rtol=1e-12, atol=1e-14)
+
+
+def test_coarse_tile_constant_inputs_equal_dense_attention():
+    """With Q, K, V constant inside every tile, each token of tile i sees 64 copies of the key
+    and value of every tile j, so dense token-level attention (a library routine) equals
+    Repeat_B of the coarse output, and its log-sum-exp is the coarse one plus log 64."""
+    N, D = 7, 16
+    rng = np.random.default_rng(21)
+    qc, kc, vc = (rng.standard_normal((N, D)) * 1.5 for _ in range(3))
+    q, k, v = (np.repeat(x, 64, axis=0) for x in (qc, kc, vc))
+    o_c, lse_c = O.coarse_attn(q, k, v)
+    tq, tk, tv = (torch.from_numpy(x)[None, None] for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv)[0, 0].numpy()
+    ref_lse = torch.logsumexp(torch.from_numpy(q @ k.T) / math.sqrt(D), dim=-1).numpy()
+    np.testing.assert_allclose(np.repeat(o_c, 64, axis=0), ref, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(np.repeat(lse_c, 64) + math.log(64), ref_lse, rtol=1e-12, atol=1e-12)
+
+
+def test_coarse_single_tile_and_equal_keys_closed_forms():
+    rng = np.random.default_rng(22)
+    D = 8
+    # one tile: a softmax over one key is 1, so the output is the tile's mean value row
+    q, k, v = (rng.standard_normal((64, D)) for _ in range(3))
+    o, lse = O.coarse_attn(q, k, v)
+    np.testing.assert_allclose(o[0], v.mean(axis=0), rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(lse[0], q.mean(axis=0) @ k.mean(axis=0) / math.sqrt(D), rtol=1e-13)
+    # equal keys everywhere: uniform weights over the 5 tiles, so every row is the mean of V
+    # and lse = qc . k / sqrt(D) + log 5
+    q5, v5 = rng.standard_normal((5 * 64, D)), rng.standard_normal((5 * 64, D))
+    kvec = rng.standard_normal(D)
+    o, lse = O.coarse_attn(q5, np.tile(kvec, (5 * 64, 1)), v5)
+    np.testing.assert_allclose(o, np.tile(v5.mean(axis=0), (5, 1)), rtol=1e-12, atol=1e-14)
+    qc = q5.reshape(5, 64, D).mean(axis=1)
+    np.testing.assert_allclose(lse, qc @ kvec / math.sqrt(D) + math.log(5), rtol=1e-12, atol=1e-14)
+
+
+def test_gated_merge_closed_forms():
+    rng = np.random.default_rng(23)
+    L, D = 3 * 64, 4
+    o_f = rng.standard_normal((L, D))
+    o_c_hat = rng.standard_normal((3, D))
+    # G = tanh(0) = 0: the fine branch alone
+    np.testing.assert_array_equal(O.gated_merge(o_f, o_c_hat, np.zeros(L)), o_f)
+    # saturated gates: tanh(+-40) rounds to +-1 in fp64
+    sign = np.where(np.arange(L) % 2 == 0, 1.0, -1.0)
+    want = o_f + sign[:, None] * np.repeat(o_c_hat, 64, axis=0)
+    np.testing.assert_allclose(O.gated_merge(o_f, o_c_hat, 40.0 * sign), want, rtol=0, atol=1e-15)
+    # G = 1/2 at the logit atanh(1/2) = ln(3)/2; token 130 lies in tile 2
+    out = O.gated_merge(o_f, o_c_hat, np.full(L, math.log(3) / 2))
+    np.testing.assert_allclose(out[130], o_f[130] + 0.5 * o_c_hat[2], rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(out[63], o_f[63] + 0.5 * o_c_hat[0], rtol=1e-14, atol=1e-15)
