@@ -49,7 +49,7 @@ def load_peaks():
 # Committed ncu summaries that carry DRAM bytes per selected pair for one kernel source and
 # workload shape: (summary file, kernel source, token grid).
 TRAFFIC_PROFILES = {
-    "fwd": ("attn_fwd_tc_720p_8heads.md", "attn_fwd_tc.cu", (56, 48, 80)),
+    "fwd": ("attn_fwd_tc_720p_4heads.md", "attn_fwd_tc.cu", (56, 48, 80)),
     "bwd": ("attn_bwd_tc_480p_4heads.md", "attn_bwd_tc.cu", (28, 32, 52)),
 }
 
@@ -246,6 +246,53 @@ def run_reference(args, wl):
 # ----------------------------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------------------------
+def time_next_rows(e, x, wl, steps, stream, l2_flush, ev, hbm, tc_peak):
+    """The coarse branch (Eq. 1-3) and the gated merge (Eq. 4, 13-14), each timed on its own
+    after the step, with L2 flushed before every launch. They are not part of the fine-branch
+    step that the headline metric times."""
+    import torch
+
+    dev = x["q"].device
+    B, H, N, L, D = wl.batch, wl.heads, wl.num_tiles, wl.tokens, wl.head_dim
+    esize = 2 if wl.dtype == "bf16" else 4
+    logits = torch.randn(B, H, L, generator=torch.Generator(device=dev).manual_seed(1234), device=dev)
+    oc = torch.empty(B, H, N, D, dtype=x["q"].dtype, device=dev)
+    lse_c = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    out = torch.empty_like(x["q"])
+    for _ in range(3):
+        e.coarse_attn(x["q"], x["k"], x["v"], oc, lse_c)
+        e.gated_merge(x["v"], logits, oc, out)  # V stands in for the fine output (same shape and dtype)
+    tc, tm = [], []
+    for _ in range(steps):
+        t = [ev() for _ in range(4)]
+        l2_flush.zero_()
+        t[0].record(stream)
+        e.coarse_attn(x["q"], x["k"], x["v"], oc, lse_c)
+        t[1].record(stream)
+        l2_flush.zero_()
+        t[2].record(stream)
+        e.gated_merge(x["v"], logits, oc, out)
+        t[3].record(stream)
+        torch.cuda.synchronize()
+        tc.append(t[0].elapsed_time(t[1]))
+        tm.append(t[2].elapsed_time(t[3]))
+    err = e.device_error()
+    if err != 0:
+        raise RuntimeError(f"device error {err} in the coarse branch")
+    c_ms, m_ms = statistics.mean(tc), statistics.mean(tm)
+    c_flops = 4.0 * N * N * D * B * H
+    pool_bytes = 3 * B * H * L * D * esize
+    m_bytes = 2 * B * H * L * D * esize + B * H * L * 4 + B * H * N * D * esize
+    return {
+        "coarse_attn": {"ms": c_ms, "effective_tflops": c_flops / (c_ms * 1e-3) / 1e12,
+                        "frac_of_sustained_bf16": c_flops / (c_ms * 1e-3) / 1e12 / tc_peak,
+                        "pool_bytes": pool_bytes, "pool_floor_ms": pool_bytes / (hbm * 1e9) * 1e3,
+                        "kernels": "coarse_pool_kernel + coarse_csr_kernel + attn_fwd_tc_kernel<true>"},
+        "gated_merge": {"ms": m_ms, "algorithmic_bytes": m_bytes, "gbs": m_bytes / (m_ms * 1e-3) / 1e9,
+                        "hbm_frac": m_bytes / (m_ms * 1e-3) / 1e9 / hbm},
+    }
+
+
 def run_ours(args, wl):
     import torch
     import torch.distributed as dist
@@ -355,6 +402,9 @@ def run_ours(args, wl):
     e2e = max_over_ranks(statistics.mean(e2e_ms) if e2e_ms else float("nan"), dev)
 
     hbm, bf16_burst, bf16_sus, peak_kind = load_peaks()
+    next_rows = None
+    if not wl.backward and not args.no_next:
+        next_rows = time_next_rows(e, x, wl, args.steps, stream, l2_flush, ev, hbm, bf16_sus)
     fwd_ms = statistics.mean(per["fwd"])
     fwd_tflops = pair_flops(wl, pairs, False) / (fwd_ms * 1e-3) / 1e12
     if wl.backward:  # the backward pass (dQ kernel + dK/dV kernel) dominates a training step
@@ -399,6 +449,7 @@ def run_ours(args, wl):
                     "api": "VSA2.forward + attn_bwd after H2D copies" if wl.backward else "vsa2_forward_host"},
             "gpu_launches": launches * args.steps,
             "clocks": clk.summary(),
+            **({"next_rows": next_rows} if next_rows else {}),
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -416,6 +467,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--heads", type=int, default=None, help="override the head count (profiling runs)")
+    ap.add_argument("--no-next", action="store_true", help="skip timing the coarse branch and the gated merge")
     args = ap.parse_args()
     wl = S.WORKLOADS[args.workload]
     if args.heads:

@@ -1,11 +1,13 @@
 /*
  * vsa2.h - C ABI of the VSA2 hot path on NVIDIA B200 (sm_100a): fine-grained router,
- * per-sequence TopK and block-sparse attention forward / backward.
+ * per-sequence TopK, block-sparse attention forward / backward, and the coarse branch with
+ * its gated merge.
  *
  * Method: "Improving Video Sparse Attention with Fine-grained Router and Sparse Rebasing"
  * (arXiv 2609.32882), §2.2 VSA2: Eq. 5-7 (router), Eq. 8-9 (per-sequence TopK), Eq. 12
- * (block-sparse fine branch); §2.1 Background gives the attention definition with the -inf
- * block mask; Fig. 5 gives the two-pass (LSE, then softmax + on-chip pooling) router.
+ * (block-sparse fine branch), Eq. 1-4 (coarse branch), Eq. 13-14 (gated merge). §2.1
+ * Background gives the attention definition with the -inf block mask; Fig. 5 gives the
+ * two-pass (LSE, then softmax + on-chip pooling) router.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -139,6 +141,34 @@ vsa2_status vsa2_sparse_attn_bwd(const vsa2_problem* p, const void* q, const voi
                                  const int32_t* q_off, const int32_t* q_idx,
                                  float* dq, float* dk, float* dv,
                                  void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Coarse branch, Eq. 1-3 (§2.2 "Coarse Branch"): cube-level dense attention.
+ *   Qc, Kc, Vc = the mean of Q, K, V over each tile of 64 tokens (Eq. 1), one row per tile;
+ *   oc[b,h,i] = sum_j softmax_j(Qc_i . Kc_j / sqrt(D)) Vc_j over all N tiles (Eq. 2-3);
+ *   lse_c[b,h,i] = ln sum_j exp(Qc_i . Kc_j / sqrt(D)).
+ *   q, k, v : [batch, heads, L, D] of dtype (read only)
+ *   oc      : [batch, heads, N, D] of dtype (written): O_c_hat, before Repeat_B (Eq. 4)
+ *   lse_c   : [batch, heads, N] fp32 (written), or NULL
+ * The pooled rows are rounded to dtype before the attention (as the inputs of the fine branch
+ * are); the softmax and accumulation are fp32. Uses the workspace of vsa2_workspace_size().
+ */
+vsa2_status vsa2_coarse_attn(const vsa2_problem* p, const void* q, const void* k, const void* v, void* oc,
+                             float* lse_c, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Gated merge, Eq. 4 and Eq. 13-14 (§2.2 "Gated Merge"):
+ *   o[b,h,t,:] = tanh(gate_logits[b,h,t]) * oc[b,h,t/64,:] + o_f[b,h,t,:]
+ *   o_f         : [batch, heads, L, D] of dtype (read only): the fine branch output (Eq. 12)
+ *   gate_logits : [batch, heads, L] fp32 (read only): X W_g of Eq. 13, one value per token and
+ *                 head (the projection of the hidden states is the caller's, like Q, K, V)
+ *   oc          : [batch, heads, N, D] of dtype (read only): O_c_hat from vsa2_coarse_attn
+ *   o           : [batch, heads, L, D] of dtype (written); may be the same buffer as o_f
+ * The result is formed in fp32 (one fused multiply-add) and rounded once to dtype. Takes no
+ * workspace.
+ */
+vsa2_status vsa2_gated_merge(const vsa2_problem* p, const void* o_f, const float* gate_logits, const void* oc,
+                             void* o, void* stream);
 
 /*
  * End-to-end forward from HOST memory: router (Eq. 5-7), per-sequence TopK (Eq. 8-9) and

@@ -106,3 +106,19 @@ def test_forward_host_workspace_and_argument_errors():
                                  None) == 1
     assert lib.vsa2_forward_host(bp, host, host, host, 6, -1, host, None, ws, one, None) == 1
     assert lib.vsa2_forward_host(bp, host, host, host, 0, 1, host, None, ws, one, None) == 2
+
+
+def test_coarse_and_merge_argument_errors():
+    lib = C.lib()
+    p = C.make_problem(1, 2, 128, (8, 16, 20))
+    bp = ctypes.byref(p)
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails before any launch
+    ws = ctypes.c_void_p(1 << 24)
+    n = C.vsa2_workspace_size(p, 6)
+    assert lib.vsa2_coarse_attn(bp, fake, fake, None, fake, None, ws, n, None) == 1
+    assert lib.vsa2_coarse_attn(bp, fake, fake, fake, ctypes.c_void_p((1 << 20) + 8), None, ws, n, None) == 1
+    assert lib.vsa2_coarse_attn(bp, fake, fake, fake, fake, None, ws, n - 256, None) == 1
+    assert lib.vsa2_gated_merge(bp, fake, None, fake, fake, None) == 1
+    assert lib.vsa2_gated_merge(bp, fake, fake, fake, ctypes.c_void_p((1 << 20) + 2), None) == 1
+    bad = C.make_problem(1, 2, 96, (8, 16, 20))
+    assert lib.vsa2_gated_merge(ctypes.byref(bad), fake, fake, fake, fake, None) == 2

@@ -1,0 +1,146 @@
+"""GPU parity of the coarse branch (Eq. 1-3) and the gated merge (Eq. 4, 13-14) against the
+fp64 oracle, through the C ABI.
+
+Tolerances are the attention-output ones: max |err| <= 2e-2 and relative L2 <= 5e-3, and LSE
+within 2e-3 relative. The GPU rounds the pooled rows to the input dtype before the coarse
+attention (both branches take bf16 operands); the oracle pools in fp64.
+
+The cases cover the pooled sequence's shapes:
+  * shorter than one tile (one padded tile);
+  * several tiles with a ragged last tile, on one and on two batch elements;
+  * a whole number of tiles;
+  * 480p and 720p heads (12 and 53 tiles, with 24 and 32 rows in the last one);
+  * the tensor-core kernel (bf16, D = 128) and the CUDA-core kernel (fp32 or D = 64).
+"""
+import numpy as np
+import pytest
+import torch
+
+import synthetic as S
+from oracle import vsa2_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import trainable_block_sparse_fine_b200 as V
+
+CASES = {
+    "one_padded_tile": S.Workload("coarse_n40", 1, 2, 128, (8, 16, 20), 6, "bf16"),       # N = 40
+    "ragged_tail": S.Workload("coarse_n160", 2, 1, 128, (16, 16, 40), 6, "bf16"),        # N = 160 = 64+64+32
+    "whole_tiles": S.Workload("coarse_n256", 1, 1, 128, (16, 16, 64), 6, "bf16"),        # N = 256
+    "d64_bf16": S.Workload("coarse_d64", 1, 2, 64, (4, 16, 24), 5, "bf16"),              # N = 24, CUDA cores
+    "fp32_d64": S.WORKLOADS["tiny"],                                                     # N = 32, fp32
+    "fp32_d128_ragged": S.Workload("coarse_f32", 1, 1, 128, (16, 16, 24), 6, "fp32"),    # N = 96
+}
+
+
+def _dev(x, dtype):
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda()
+    return t.to(torch.bfloat16) if dtype == "bf16" else t
+
+
+def _engine(wl):
+    return V.VSA2(wl.batch, wl.heads, wl.head_dim, wl.grid, wl.dtype, wl.topk)
+
+
+def _close(got, want, what, lse_got=None, lse_want=None):
+    got, want = np.asarray(got, np.float64), np.asarray(want, np.float64)
+    err = np.abs(got - want)
+    rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+    assert err.max() <= 2e-2 and rel <= 5e-3, f"{what}: max abs {err.max():.3e}, rel L2 {rel:.3e}"
+    if lse_got is not None:
+        d = np.abs(np.asarray(lse_got, np.float64) - lse_want)
+        assert d.max() <= 2e-3 * max(1.0, np.abs(lse_want).max()), f"{what}: lse error {d.max():.3e}"
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_coarse_attn_matches_oracle(case):
+    wl = CASES[case]
+    x = {n: S.make_tensor(wl, n) for n in "qkv"}
+    e = _engine(wl)
+    oc, lse_c = e.coarse_attn(*(_dev(x[n], wl.dtype) for n in "qkv"))
+    assert e.device_error() == 0
+    assert oc.shape == (wl.batch, wl.heads, wl.num_tiles, wl.head_dim)
+    oc, lse_c = oc.float().cpu().numpy(), lse_c.cpu().numpy()
+    for b in range(wl.batch):
+        for h in range(wl.heads):
+            want, want_lse = O.coarse_attn(x["q"][b, h], x["k"][b, h], x["v"][b, h])
+            _close(oc[b, h], want, f"{case} oc[{b},{h}]", lse_c[b, h], want_lse)
+
+
+def test_coarse_attn_480p_two_heads():
+    """480p: 728 pooled rows per head, 12 tiles of which the last holds 24 rows."""
+    wl480 = S.WORKLOADS["480p_top64"]
+    heads = [0, 13]
+    x = {n: S.make_tensor(wl480, n, heads=heads) for n in "qkv"}
+    wl = wl480.with_(heads=len(heads))
+    e = _engine(wl)
+    oc, lse_c = e.coarse_attn(*(_dev(x[n], wl.dtype) for n in "qkv"))
+    assert e.device_error() == 0
+    oc, lse_c = oc.float().cpu().numpy(), lse_c.cpu().numpy()
+    for i, h in enumerate(heads):
+        want, want_lse = O.coarse_attn(x["q"][0, i], x["k"][0, i], x["v"][0, i])
+        _close(oc[0, i], want, f"480p head {h}", lse_c[0, i], want_lse)
+
+
+def test_coarse_attn_720p_all_heads_head0_compared():
+    """720p, in the configuration the benchmark times (20 heads in one call): 3360 pooled rows
+    per head, 53 tiles of which the last holds 32 rows. Head 0 comes from the seeded generator
+    and is compared; heads 1-19 are seeded normals."""
+    wl = S.WORKLOADS["720p_top64"]
+    x0 = {n: S.make_slice(wl, n, 0, 0) for n in "qkv"}
+    g = torch.Generator(device="cuda").manual_seed(7200)
+    dev = {}
+    for n in "qkv":
+        t = torch.randn((1, wl.heads, wl.tokens, wl.head_dim), generator=g, device="cuda")
+        t[0, 0] = torch.from_numpy(x0[n]).cuda()
+        dev[n] = t.to(torch.bfloat16)
+        del t
+    e = _engine(wl)
+    oc, lse_c = e.coarse_attn(dev["q"], dev["k"], dev["v"])
+    assert e.device_error() == 0
+    want, want_lse = O.coarse_attn(x0["q"], x0["k"], x0["v"])
+    _close(oc[0, 0].float().cpu().numpy(), want, "720p head 0", lse_c[0, 0].cpu().numpy(), want_lse)
+    assert torch.isfinite(oc.float()).all()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("in_place", [False, True], ids=["out_of_place", "in_place"])
+def test_gated_merge_matches_oracle(dtype, in_place):
+    wl = S.Workload("merge", 2, 3, 128, (8, 16, 20), 6, dtype)
+    rng = np.random.default_rng(31)
+    N, L, D = wl.num_tiles, wl.tokens, wl.head_dim
+    o_f = S.round_to_dtype(rng.standard_normal((wl.batch, wl.heads, L, D)).astype(np.float32), dtype)
+    oc = S.round_to_dtype(rng.standard_normal((wl.batch, wl.heads, N, D)).astype(np.float32), dtype)
+    logits = (rng.standard_normal((wl.batch, wl.heads, L)) * 2).astype(np.float32)
+    logits[0, 0, :64] = 0.0  # tanh(0) = 0: these rows are the fine output alone
+    e = _engine(wl)
+    o_f_d = _dev(o_f, dtype)
+    out = e.gated_merge(o_f_d, torch.from_numpy(logits).cuda(), _dev(oc, dtype), out=o_f_d if in_place else None)
+    got = out.float().cpu().numpy()
+    tol = 2e-2 if dtype == "bf16" else 1e-5
+    for b in range(wl.batch):
+        for h in range(wl.heads):
+            want = O.gated_merge(o_f[b, h], oc[b, h], logits[b, h])
+            err = np.abs(got[b, h] - want)
+            assert err.max() <= tol * max(1.0, np.abs(want).max()), f"[{b},{h}] max abs {err.max():.3e}"
+    np.testing.assert_array_equal(got[0, 0, :64], o_f[0, 0, :64])
+
+
+def test_attention_output_is_the_gated_sum_of_both_branches():
+    """VSA2.attention (Eq. 14) against the oracle's gated merge of its fine branch (on the
+    selection the GPU made) and its coarse branch."""
+    wl = CASES["ragged_tail"]
+    x = {n: S.make_tensor(wl, n) for n in "qkv"}
+    logits = np.random.default_rng(32).standard_normal((wl.batch, wl.heads, wl.tokens)).astype(np.float32)
+    e = _engine(wl)
+    xd = {n: _dev(x[n], wl.dtype) for n in "qkv"}
+    sel = e.topk_select(e.router_scores(xd["q"], xd["k"]), wl.topk, csc=False)
+    o = e.attention(xd["q"], xd["k"], xd["v"], torch.from_numpy(logits).cuda()).float().cpu().numpy()
+    assert e.device_error() == 0
+    kv_off, kv_idx = sel[0].cpu().numpy(), sel[1].cpu().numpy()
+    for b in range(wl.batch):
+        for h in range(wl.heads):
+            o_f, _ = O.sparse_attn_fwd(x["q"][b, h], x["k"][b, h], x["v"][b, h], kv_off[b, h], kv_idx[b, h])
+            oc, _ = O.coarse_attn(x["q"][b, h], x["k"][b, h], x["v"][b, h])
+            _close(o[b, h], O.gated_merge(o_f, oc, logits[b, h]), f"o[{b},{h}]")

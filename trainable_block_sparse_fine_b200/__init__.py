@@ -11,15 +11,16 @@ from __future__ import annotations
 
 import torch
 
-from ._capi import (VSA2_FLAG_VALIDATE, Problem, Vsa2Error, lib, make_problem, vsa2_forward_host,
-                    vsa2_forward_host_workspace_size, vsa2_get_device_error, vsa2_router_scores,
+from ._capi import (VSA2_FLAG_VALIDATE, Problem, Vsa2Error, lib, make_problem, vsa2_coarse_attn, vsa2_forward_host,
+                    vsa2_forward_host_workspace_size, vsa2_gated_merge, vsa2_get_device_error, vsa2_router_scores,
                     vsa2_selftest_wait_timeout, vsa2_sparse_attn_bwd, vsa2_sparse_attn_fwd, vsa2_status_string,
                     vsa2_topk_select, vsa2_version, vsa2_workspace_init, vsa2_workspace_size)
 
 __all__ = ["VSA2", "Vsa2Error", "Problem", "make_problem", "block_sparse_attention", "lib", "VSA2_FLAG_VALIDATE",
            "vsa2_router_scores", "vsa2_topk_select", "vsa2_sparse_attn_fwd", "vsa2_sparse_attn_bwd",
            "vsa2_workspace_size", "vsa2_workspace_init", "vsa2_get_device_error", "vsa2_selftest_wait_timeout",
-           "vsa2_status_string", "vsa2_version", "vsa2_forward_host", "vsa2_forward_host_workspace_size"]
+           "vsa2_status_string", "vsa2_version", "vsa2_forward_host", "vsa2_forward_host_workspace_size",
+           "vsa2_coarse_attn", "vsa2_gated_merge"]
 
 
 class VSA2:
@@ -81,6 +82,28 @@ class VSA2:
         sel = self.topk_select(scores, topk, csc=csc)
         o, lse = self.attn_fwd(q, k, v, sel[0], sel[1], topk)
         return o, lse, sel
+
+    def coarse_attn(self, q, k, v, oc=None, lse_c=None):
+        """Coarse branch, Eq. 1-3: O_c_hat [B, H, N, D] (input dtype) and its LSE [B, H, N]."""
+        oc = oc if oc is not None else torch.empty(self.batch, self.heads, self.N, self.head_dim, dtype=q.dtype,
+                                                   device=self.device)
+        lse_c = lse_c if lse_c is not None else torch.empty(self.batch, self.heads, self.N, dtype=torch.float32,
+                                                            device=self.device)
+        vsa2_coarse_attn(self.p, q, k, v, oc, lse_c, self.ws)
+        return oc, lse_c
+
+    def gated_merge(self, o_f, gate_logits, oc, out=None):
+        """Eq. 4, 13-14: tanh(gate_logits) * Repeat_B(oc) + o_f; out may be o_f (in place)."""
+        out = out if out is not None else torch.empty_like(o_f)
+        vsa2_gated_merge(self.p, o_f, gate_logits, oc, out)
+        return out
+
+    def attention(self, q, k, v, gate_logits, topk=None):
+        """The whole VSA2 attention output, Eq. 14: fine branch (router, TopK, Eq. 12) plus the
+        gated coarse branch. Returns o."""
+        o_f, _, _ = self.forward(q, k, v, topk)
+        oc, _ = self.coarse_attn(q, k, v)
+        return self.gated_merge(o_f, gate_logits, oc, out=o_f)
 
     def forward_host(self, q, k, v, topk=None, o=None, lse=None, heads_per_group=0, want_lse=False):
         """Router -> TopK -> forward on HOST tensors, copies overlapped with the kernels per group of

@@ -63,6 +63,15 @@ WsLayout ws_layout(const Dims& d) {
   w.col_bits = take((size_t)d.BH * d.N * w.words * 4);
   w.delta = take((size_t)d.BH * d.L * 4);
   w.nlse2 = take((size_t)d.BH * d.L * 4);
+  w.Nc_tiles = (d.N + kTile - 1) / kTile;
+  const size_t lc = (size_t)kTile * w.Nc_tiles;
+  w.qc = take((size_t)d.BH * lc * d.D * d.esize);
+  w.kc = take((size_t)d.BH * lc * d.D * d.esize);
+  w.vc = take((size_t)d.BH * lc * d.D * d.esize);
+  w.oc = take((size_t)d.BH * lc * d.D * d.esize);
+  w.lse_c = take((size_t)d.BH * lc * 4);
+  w.c_off = take((size_t)d.BH * (w.Nc_tiles + 1) * 4);
+  w.c_idx = take((size_t)d.BH * w.Nc_tiles * w.Nc_tiles * 4);
   w.total = off;
   return w;
 }
@@ -228,6 +237,28 @@ vsa2_status vsa2_sparse_attn_bwd(const vsa2_problem* p, const void* q, const voi
   if ((st = check_ws(d, ws, ws_bytes)) != VSA2_OK) return st;
   return launch_attn_bwd(d, q, k, v, o, lse, dout, topk, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, (char*)ws,
                          (cudaStream_t)stream);
+}
+
+vsa2_status vsa2_coarse_attn(const vsa2_problem* p, const void* q, const void* k, const void* v, void* oc,
+                             float* lse_c, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  vsa2_status st = make_dims(p, &d);
+  if (st != VSA2_OK) return st;
+  if (!q || !k || !v || !oc) return VSA2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(oc) || (lse_c && !aligned16(lse_c)))
+    return VSA2_ERR_INVALID_ARG;
+  if ((st = check_ws(d, ws, ws_bytes)) != VSA2_OK) return st;
+  return launch_coarse_attn(d, q, k, v, oc, lse_c, (char*)ws, (cudaStream_t)stream);
+}
+
+vsa2_status vsa2_gated_merge(const vsa2_problem* p, const void* o_f, const float* gate_logits, const void* oc,
+                             void* o, void* stream) {
+  Dims d;
+  vsa2_status st = make_dims(p, &d);
+  if (st != VSA2_OK) return st;
+  if (!o_f || !gate_logits || !oc || !o) return VSA2_ERR_INVALID_ARG;
+  if (!aligned16(o_f) || !aligned16(gate_logits) || !aligned16(oc) || !aligned16(o)) return VSA2_ERR_INVALID_ARG;
+  return launch_gated_merge(d, o_f, gate_logits, oc, o, (cudaStream_t)stream);
 }
 
 vsa2_status vsa2_topk_select_noalloc(const vsa2_problem* p, const float* scores, int32_t topk, int32_t* kv_off,

@@ -21,6 +21,10 @@
 // of its MMA: V(i) as soon as S(i) has read K(i), K(i+1) once O(i-2) has read V(i-2). The running
 // max is raised (with an O rescale in TMEM) only when a row's new maximum exceeds it by more
 // than 2^8.
+//
+// kPad = true masks keys at or beyond `kv_valid` tokens of a head (a sequence whose last tile is
+// partly padding, such as the coarse branch's N pooled rows, Eq. 1-3). Every listed tile must
+// hold at least one valid key. kPad = false is the fine branch (Eq. 12), with no key mask.
 #include <algorithm>
 
 #include "common.cuh"
@@ -123,11 +127,12 @@ __device__ __forceinline__ int next_op(SlotSeq& q, int* blk, const int32_t* kv_o
   return 0;
 }
 
+template <bool kPad>
 __global__ void __launch_bounds__(FT, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const __nv_bfloat16* __restrict__ qg, const int32_t* __restrict__ kv_off,
                        const int32_t* __restrict__ kv_idx, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
-                       int N, int L, int topk, int items, float c2, DevCtx ctx) {
+                       int N, int L, int topk, int items, float c2, int kv_valid, DevCtx ctx) {
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
   uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   Bars& B = *reinterpret_cast<Bars*>(dsm + OFF_BAR);
@@ -300,6 +305,17 @@ __global__ void __launch_bounds__(FT, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&B.sfree[s][g & 1]);
+        if constexpr (kPad) {
+          // keys of the block's two tiles at or beyond kv_valid get a score of -inf
+          const int32_t* ix = kv_idx + (size_t)bh * cap + rw.beg + 2 * n;
+          const int v1 = kv_valid - 64 * __ldg(ix);
+          const int v2 = half ? 64 : kv_valid - 64 * __ldg(ix + 1);
+          if (v1 < 64 || v2 < 64) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+              if (((2 * i + par_c) & 63) >= (i < 32 ? v1 : v2)) x[i] = __float_as_uint(-INFINITY);
+          }
+        }
         // columns 2i + par_c; in a half block only the first 64 columns are real
         float mx = __uint_as_float(x[0]);
         if (!half) {
@@ -392,8 +408,11 @@ __global__ void __launch_bounds__(FT, 1)
 bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
                        uint32_t box_rows);
 
-vsa2_status attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v, int topk, const int32_t* kv_off,
-                        const int32_t* kv_idx, void* o, float* lse, char* ws, cudaStream_t s) {
+namespace {
+template <bool kPad>
+vsa2_status launch_fwd_tc(const Dims& d, const void* q, const void* k, const void* v, int topk,
+                          const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws, int kv_valid,
+                          cudaStream_t s) {
   CUtensorMap tk, tv;
   const uint64_t rows = (uint64_t)d.BH * d.L;
   if (!make_tmap_2d_bf16(&tk, k, 128, rows, 64, 64) || !make_tmap_2d_bf16(&tv, v, 128, rows, 64, 64))
@@ -405,10 +424,23 @@ vsa2_status attn_fwd_tc(const Dims& d, const void* q, const void* k, const void*
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::max(1, std::min(sms, (items + 1) / 2));
   const float c2 = 1.4426950408889634f / sqrtf(128.f);
-  cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
-  attn_fwd_tc_kernel<<<grid, FT, SMEM_DYN, s>>>(tk, tv, (const __nv_bfloat16*)q, kv_off, kv_idx, (__nv_bfloat16*)o,
-                                                lse, d.N, (int)d.L, topk, items, c2, ctx);
-  return check_launch(__func__);
+  cudaFuncSetAttribute(attn_fwd_tc_kernel<kPad>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
+  attn_fwd_tc_kernel<kPad><<<grid, FT, SMEM_DYN, s>>>(tk, tv, (const __nv_bfloat16*)q, kv_off, kv_idx,
+                                                      (__nv_bfloat16*)o, lse, d.N, (int)d.L, topk, items, c2,
+                                                      kv_valid, ctx);
+  return check_launch("attn_fwd_tc");
+}
+}  // namespace
+
+vsa2_status attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v, int topk, const int32_t* kv_off,
+                        const int32_t* kv_idx, void* o, float* lse, char* ws, cudaStream_t s) {
+  return launch_fwd_tc<false>(d, q, k, v, topk, kv_off, kv_idx, o, lse, ws, (int)d.L, s);
+}
+
+vsa2_status attn_fwd_tc_masked(const Dims& d, const void* q, const void* k, const void* v, int topk,
+                               const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
+                               int kv_valid, cudaStream_t s) {
+  return launch_fwd_tc<true>(d, q, k, v, topk, kv_off, kv_idx, o, lse, ws, kv_valid, s);
 }
 
 }  // namespace vsa2

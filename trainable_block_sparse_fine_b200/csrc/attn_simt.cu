@@ -48,7 +48,7 @@ __global__ void __launch_bounds__(64) attn_fwd_simt_kernel(const T* __restrict__
                                                            const T* __restrict__ v, const int32_t* __restrict__ kv_off,
                                                            const int32_t* __restrict__ kv_idx, T* __restrict__ o,
                                                            float* __restrict__ lse, int N, int64_t L, int topk,
-                                                           DevCtx ctx) {
+                                                           int64_t kv_valid, DevCtx ctx) {
   extern __shared__ float sm[];
   float* qT = sm;              // [D][64]
   float* ks = qT + D * 64;     // [64][D]
@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(64) attn_fwd_simt_kernel(const T* __restrict__
     for (int u = 0; u < 64; ++u) {
       float acc = 0.f;
       for (int d = 0; d < D; ++d) acc += qT[d * 64 + t] * ks[u * D + d];
-      s[u] = acc * scale;
+      s[u] = (int64_t)j * kTile + u < kv_valid ? acc * scale : -INFINITY;  // keys past kv_valid are padding
       mx = fmaxf(mx, s[u]);
     }
     const float mn = fmaxf(m, mx);
@@ -262,12 +262,13 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_simt_kernel(const T* __rest
 
 template <typename T, int D>
 vsa2_status fwd_simt(const Dims& d, const void* q, const void* k, const void* v, const int32_t* kv_off,
-                     const int32_t* kv_idx, void* o, float* lse, const DevCtx& ctx, int topk, cudaStream_t s) {
+                     const int32_t* kv_idx, void* o, float* lse, const DevCtx& ctx, int topk, int64_t kv_valid,
+                     cudaStream_t s) {
   const size_t smem = (size_t)4 * 64 * D * sizeof(float);
   auto kern = attn_fwd_simt_kernel<T, D>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   kern<<<dim3(d.N, d.BH), 64, smem, s>>>((const T*)q, (const T*)k, (const T*)v, kv_off, kv_idx, (T*)o, lse, d.N,
-                                         d.L, topk, ctx);
+                                         d.L, topk, kv_valid, ctx);
   return check_launch(__func__);
 }
 
@@ -295,14 +296,14 @@ vsa2_status bwd_simt(const Dims& d, const void* q, const void* k, const void* v,
 
 vsa2_status attn_fwd_simt(const Dims& d, const void* q, const void* k, const void* v, int topk,
                           const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
-                          cudaStream_t s) {
+                          int64_t kv_valid, cudaStream_t s) {
   DevCtx ctx{reinterpret_cast<int*>(ws), d.timeout_ns, d.flags};
   if (d.dtype == VSA2_BF16) {
-    if (d.D == 128) return fwd_simt<__nv_bfloat16, 128>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, s);
-    return fwd_simt<__nv_bfloat16, 64>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, s);
+    if (d.D == 128) return fwd_simt<__nv_bfloat16, 128>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, s);
+    return fwd_simt<__nv_bfloat16, 64>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, s);
   }
-  if (d.D == 128) return fwd_simt<float, 128>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, s);
-  return fwd_simt<float, 64>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, s);
+  if (d.D == 128) return fwd_simt<float, 128>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, s);
+  return fwd_simt<float, 64>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, s);
 }
 
 vsa2_status attn_bwd_simt(const Dims& d, const void* q, const void* k, const void* v, const void* o, const float* lse,

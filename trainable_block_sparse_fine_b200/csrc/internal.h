@@ -41,6 +41,11 @@ struct WsLayout {
   size_t delta;          // backward rowsum(dO * O), [BH, L] fp32 (the tcgen05 backward keeps
                          // -Delta here, in token order)
   size_t nlse2;          // tcgen05 backward: -lse * log2(e), [BH, L] fp32, token order
+  int Nc_tiles;          // coarse branch: ceil(N / 64) tiles of pooled rows per (b, h)
+  size_t qc, kc, vc, oc; // coarse branch: pooled Q, K, V and output, [BH, 64 * Nc_tiles, D] dtype,
+                         // rows >= N zero (Q, K, V) or unused (output)
+  size_t lse_c;          // coarse branch LSE, [BH, 64 * Nc_tiles] fp32
+  size_t c_off, c_idx;   // coarse branch: CSR listing every tile, [BH, Nc_tiles + 1], [BH, Nc_tiles^2] i32
   size_t total;
 };
 WsLayout ws_layout(const Dims& d);
@@ -61,18 +66,28 @@ vsa2_status launch_attn_bwd(const Dims& d, const void* q, const void* k, const v
                             const float* lse, const void* dout, int topk, const int32_t* kv_off,
                             const int32_t* kv_idx, const int32_t* q_off, const int32_t* q_idx, float* dq, float* dk,
                             float* dv, char* ws, cudaStream_t s);
-// CUDA-core paths (fp32 inputs, head_dim 64, and the backward pass)
+// CUDA-core paths (fp32 inputs, head_dim 64, and the backward pass). The forward masks keys at
+// or beyond kv_valid tokens of each head (d.L for the fine branch: no mask).
 vsa2_status attn_fwd_simt(const Dims& d, const void* q, const void* k, const void* v, int topk,
                           const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
-                          cudaStream_t s);
+                          int64_t kv_valid, cudaStream_t s);
 vsa2_status attn_bwd_simt(const Dims& d, const void* q, const void* k, const void* v, const void* o,
                           const float* lse, const void* dout, const int32_t* kv_off, const int32_t* kv_idx,
                           const int32_t* q_off, const int32_t* q_idx, float* dq, float* dk, float* dv, int topk,
                           char* ws, cudaStream_t s);
-// tensor-core forward (bf16, head_dim 128)
+// tensor-core forward (bf16, head_dim 128); the masked variant treats keys at or beyond
+// kv_valid tokens of each head as padding (each listed tile must hold a valid key)
 vsa2_status attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v, int topk,
                         const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
                         cudaStream_t s);
+vsa2_status attn_fwd_tc_masked(const Dims& d, const void* q, const void* k, const void* v, int topk,
+                               const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
+                               int kv_valid, cudaStream_t s);
+// Coarse branch (Eq. 1-3) and gated merge (Eq. 4, 13-14)
+vsa2_status launch_coarse_attn(const Dims& d, const void* q, const void* k, const void* v, void* oc, float* lse_c,
+                               char* ws, cudaStream_t s);
+vsa2_status launch_gated_merge(const Dims& d, const void* o_f, const float* gate_logits, const void* oc, void* o,
+                               cudaStream_t s);
 // tensor-core backward (bf16, head_dim 128): dQ kernel (also writes Delta), then dK/dV kernel
 vsa2_status attn_bwd_tc(const Dims& d, const void* q, const void* k, const void* v, const void* o, const float* lse,
                         const void* dout, const int32_t* kv_off, const int32_t* kv_idx, const int32_t* q_off,
