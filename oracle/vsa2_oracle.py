@@ -36,6 +36,8 @@ __all__ = [
     "sparse_attn_bwd",
     "coarse_attn",
     "gated_merge",
+    "coarse_attn_bwd",
+    "gated_merge_bwd",
 ]
 
 
@@ -243,3 +245,44 @@ def gated_merge(o_f, o_c_hat, gate_logits, tile_tokens: int = 64):
     o_c = np.repeat(np.asarray(o_c_hat, dtype=np.float64), tile_tokens, axis=0)
     g = np.tanh(np.asarray(gate_logits, dtype=np.float64))[:, None]
     return g * o_c + o_f
+
+
+def coarse_attn_bwd(q, k, v, d_oc):
+    """Gradients of Eq. 1-3 for one (b, h): given d_oc = dLoss/dO_c_hat (N, D), returns
+    (dQ, dK, dV), each (L, D). With P_c, O_c_hat from the forward:
+    dP   = d_oc Vc^T,  Delta = rowsum(d_oc * O_c_hat),  dS = P_c * (dP - Delta)
+    dQc  = dS Kc / sqrt(D),  dKc = dS^T Qc / sqrt(D),  dVc = P_c^T d_oc
+    and MeanPool_B spreads each pooled gradient evenly: dQ[t] = dQc[tile(t)] / B, same for K, V.
+    """
+    qc = mean_pool(q, 64)
+    kc = mean_pool(k, 64)
+    vc = mean_pool(v, 64)
+    d_oc = np.asarray(d_oc, dtype=np.float64)
+    D = qc.shape[1]
+    s = (qc @ kc.T) / np.sqrt(D)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    o = p @ vc
+    dp = d_oc @ vc.T
+    delta = (d_oc * o).sum(axis=1, keepdims=True)
+    ds = p * (dp - delta)
+    dqc = ds @ kc / np.sqrt(D)
+    dkc = ds.T @ qc / np.sqrt(D)
+    dvc = p.T @ d_oc
+    return tuple(np.repeat(x, 64, axis=0) / 64.0 for x in (dqc, dkc, dvc))
+
+
+def gated_merge_bwd(dout, o_c_hat, gate_logits, tile_tokens: int = 64):
+    """Gradients of Eq. 4, 13-14 for one (b, h), given dout = dLoss/dO (L, D):
+    dO_f           = dout
+    dO_c_hat[i]    = sum over the tokens t of tile i of G[t] * dout[t]   (Repeat_B's adjoint)
+    d gate_logits  = (1 - G^2) * rowsum(dout * O_c)                     (tanh' = 1 - tanh^2)
+    Returns (dO_f (L, D), dO_c_hat (N, D), d_gate_logits (L,)).
+    """
+    dout = np.asarray(dout, dtype=np.float64)
+    g = np.tanh(np.asarray(gate_logits, dtype=np.float64))
+    o_c = np.repeat(np.asarray(o_c_hat, dtype=np.float64), tile_tokens, axis=0)
+    L, D = dout.shape
+    d_oc = (g[:, None] * dout).reshape(L // tile_tokens, tile_tokens, D).sum(axis=1)
+    d_logits = (1.0 - g * g) * (dout * o_c).sum(axis=1)
+    return dout.copy(), d_oc, d_logits

@@ -506,3 +506,63 @@ def test_gated_merge_closed_forms():
     out = O.gated_merge(o_f, o_c_hat, np.full(L, math.log(3) / 2))
     np.testing.assert_allclose(out[130], o_f[130] + 0.5 * o_c_hat[2], rtol=1e-14, atol=1e-15)
     np.testing.assert_allclose(out[63], o_f[63] + 0.5 * o_c_hat[0], rtol=1e-14, atol=1e-15)
+
+
+def _central_diff(f, x, h=1e-6):
+    g = np.zeros_like(x)
+    for idx in np.ndindex(x.shape):
+        old = x[idx]
+        x[idx] = old + h
+        up = f()
+        x[idx] = old - h
+        dn = f()
+        x[idx] = old
+        g[idx] = (up - dn) / (2 * h)
+    return g
+
+
+def test_coarse_bwd_central_finite_differences():
+    rng = np.random.default_rng(24)
+    L, D = 3 * 64, 4
+    q, k, v = (rng.standard_normal((L, D)) for _ in range(3))
+    w = rng.standard_normal((3, D))  # loss = sum(w * O_c_hat), so dLoss/dO_c_hat = w
+    dq, dk, dv = O.coarse_attn_bwd(q, k, v, w)
+    for x, got in ((q, dq), (k, dk), (v, dv)):
+        num = _central_diff(lambda: float((w * O.coarse_attn(q, k, v)[0]).sum()), x)
+        np.testing.assert_allclose(got, num, rtol=1e-6, atol=1e-9)
+
+
+def test_coarse_bwd_tile_constant_case_equals_dense_autograd():
+    """With Q, K, V and dO constant inside every tile, dense token attention and the coarse
+    branch give the same output, and by symmetry the same gradient at every token: each token's
+    dense-attention gradient is the pooled gradient divided by 64 (torch autograd, fp64)."""
+    N, D = 5, 8
+    rng = np.random.default_rng(25)
+    qc, kc, vc, gc = (rng.standard_normal((N, D)) for _ in range(4))
+    q, k, v, g = (np.repeat(x, 64, axis=0) for x in (qc, kc, vc, gc))
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    out = torch.nn.functional.scaled_dot_product_attention(tq[None, None], tk[None, None], tv[None, None])[0, 0]
+    (out * torch.from_numpy(g)).sum().backward()
+    # dLoss/dO_c_hat for the coarse branch: the 64 tokens of a tile share one output row
+    dq, dk, dv = O.coarse_attn_bwd(q, k, v, 64.0 * gc)
+    for got, t in ((dq, tq), (dk, tk), (dv, tv)):
+        np.testing.assert_allclose(got, t.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_gated_merge_bwd_finite_differences_and_zero_gate():
+    rng = np.random.default_rng(26)
+    L, D = 2 * 64, 3
+    o_f = rng.standard_normal((L, D))
+    oc = rng.standard_normal((2, D))
+    logits = rng.standard_normal(L)
+    dout = rng.standard_normal((L, D))
+    d_of, d_oc, d_logits = O.gated_merge_bwd(dout, oc, logits)
+    loss = lambda: float((dout * O.gated_merge(o_f, oc, logits)).sum())
+    np.testing.assert_array_equal(d_of, dout)
+    np.testing.assert_allclose(d_oc, _central_diff(loss, oc), rtol=1e-7, atol=1e-9)
+    np.testing.assert_allclose(d_logits, _central_diff(loss, logits), rtol=1e-7, atol=1e-9)
+    np.testing.assert_allclose(_central_diff(loss, o_f), dout, rtol=1e-7, atol=1e-9)
+    # closed forms at G = 0: no gradient reaches O_c_hat, and the logit gradient is dout . O_c
+    _, d_oc0, d_l0 = O.gated_merge_bwd(dout, oc, np.zeros(L))
+    assert np.all(d_oc0 == 0)
+    np.testing.assert_allclose(d_l0, (dout * np.repeat(oc, 64, axis=0)).sum(axis=1), rtol=1e-15)
