@@ -247,12 +247,15 @@ def gated_merge(o_f, o_c_hat, gate_logits, tile_tokens: int = 64):
     return g * o_c + o_f
 
 
-def coarse_attn_bwd(q, k, v, d_oc):
+def coarse_attn_bwd(q, k, v, d_oc, o_c_hat=None):
     """Gradients of Eq. 1-3 for one (b, h): given d_oc = dLoss/dO_c_hat (N, D), returns
     (dQ, dK, dV), each (L, D). With P_c, O_c_hat from the forward:
     dP   = d_oc Vc^T,  Delta = rowsum(d_oc * O_c_hat),  dS = P_c * (dP - Delta)
     dQc  = dS Kc / sqrt(D),  dKc = dS^T Qc / sqrt(D),  dVc = P_c^T d_oc
     and MeanPool_B spreads each pooled gradient evenly: dQ[t] = dQc[tile(t)] / B, same for K, V.
+
+    `o_c_hat`, when given, is the forward output Delta is formed from, as in a backward pass that
+    receives the stored output of the forward; by default the exact output is recomputed.
     """
     qc = mean_pool(q, 64)
     kc = mean_pool(k, 64)
@@ -262,7 +265,7 @@ def coarse_attn_bwd(q, k, v, d_oc):
     s = (qc @ kc.T) / np.sqrt(D)
     p = np.exp(s - s.max(axis=1, keepdims=True))
     p /= p.sum(axis=1, keepdims=True)
-    o = p @ vc
+    o = p @ vc if o_c_hat is None else np.asarray(o_c_hat, dtype=np.float64)
     dp = d_oc @ vc.T
     delta = (d_oc * o).sum(axis=1, keepdims=True)
     ds = p * (dp - delta)

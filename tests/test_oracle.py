@@ -566,3 +566,20 @@ def test_gated_merge_bwd_finite_differences_and_zero_gate():
     _, d_oc0, d_l0 = O.gated_merge_bwd(dout, oc, np.zeros(L))
     assert np.all(d_oc0 == 0)
     np.testing.assert_allclose(d_l0, (dout * np.repeat(oc, 64, axis=0)).sum(axis=1), rtol=1e-15)
+
+
+def test_coarse_bwd_given_output_enters_only_through_rowsum():
+    """Passing the exact forward output reproduces the default; a perturbed output changes
+    the gradients only through Delta = rowsum(d_oc * O): dV does not move."""
+    rng = np.random.default_rng(27)
+    L, D = 3 * 64, 4
+    q, k, v = (rng.standard_normal((L, D)) for _ in range(3))
+    w = rng.standard_normal((3, D))
+    o, _ = O.coarse_attn(q, k, v)
+    base = O.coarse_attn_bwd(q, k, v, w)
+    same = O.coarse_attn_bwd(q, k, v, w, o_c_hat=o)
+    for a, b in zip(base, same):
+        np.testing.assert_allclose(a, b, rtol=1e-13, atol=1e-15)
+    moved = O.coarse_attn_bwd(q, k, v, w, o_c_hat=o + 0.01)
+    np.testing.assert_array_equal(moved[2], base[2])
+    assert np.abs(moved[0] - base[0]).max() > 1e-6
