@@ -247,9 +247,9 @@ def run_reference(args, wl):
 # our arm
 # ----------------------------------------------------------------------------------------------
 def time_next_rows(e, x, wl, steps, stream, l2_flush, ev, hbm, tc_peak):
-    """The coarse branch (Eq. 1-3) and the gated merge (Eq. 4, 13-14), each timed on its own
-    after the step, with L2 flushed before every launch. They are not part of the fine-branch
-    step that the headline metric times."""
+    """The coarse branch (Eq. 1-3) and the gated merge (Eq. 4, 13-14), and for training
+    workloads their gradients, each timed on its own after the step, with L2 flushed before every
+    launch. They are not part of the fine-branch step that the headline metric times."""
     import torch
 
     dev = x["q"].device
@@ -276,6 +276,36 @@ def time_next_rows(e, x, wl, steps, stream, l2_flush, ev, hbm, tc_peak):
         torch.cuda.synchronize()
         tc.append(t[0].elapsed_time(t[1]))
         tm.append(t[2].elapsed_time(t[3]))
+    extra = {}
+    if wl.backward:  # gradients of the merge and of the coarse branch, after the fine backward
+        grads = [torch.zeros(B, H, L, D, dtype=torch.float32, device=dev) for _ in range(3)]
+        for _ in range(3):
+            _, d_oc = e.gated_merge_bwd(x["do"], logits, oc)
+            e.coarse_attn_bwd(x["q"], x["k"], x["v"], oc, lse_c, d_oc, *grads)
+        tmb, tcb = [], []
+        for _ in range(steps):
+            t = [ev() for _ in range(4)]
+            l2_flush.zero_()
+            t[0].record(stream)
+            e.gated_merge_bwd(x["do"], logits, oc)
+            t[1].record(stream)
+            l2_flush.zero_()
+            t[2].record(stream)
+            e.coarse_attn_bwd(x["q"], x["k"], x["v"], oc, lse_c, d_oc, *grads)
+            t[3].record(stream)
+            torch.cuda.synchronize()
+            tmb.append(t[0].elapsed_time(t[1]))
+            tcb.append(t[2].elapsed_time(t[3]))
+        mb_ms, cb_ms = statistics.mean(tmb), statistics.mean(tcb)
+        mb_bytes = B * H * L * D * esize + 8 * B * H * L + B * H * N * D * (esize + 4)
+        cb_flops = 2.5 * 4.0 * N * N * D * B * H
+        extra = {
+            "gated_merge_bwd": {"ms": mb_ms, "algorithmic_bytes": mb_bytes, "gbs": mb_bytes / (mb_ms * 1e-3) / 1e9,
+                                "hbm_frac": mb_bytes / (mb_ms * 1e-3) / 1e9 / hbm},
+            "coarse_attn_bwd": {"ms": cb_ms, "effective_tflops": cb_flops / (cb_ms * 1e-3) / 1e12,
+                                "kernels": "pool + pad + attn_bwd_dq_tc_kernel + attn_bwd_dkdv_tc_kernel + "
+                                           "coarse_pool_bwd_kernel"},
+        }
     err = e.device_error()
     if err != 0:
         raise RuntimeError(f"device error {err} in the coarse branch")
@@ -290,6 +320,7 @@ def time_next_rows(e, x, wl, steps, stream, l2_flush, ev, hbm, tc_peak):
                         "kernels": "coarse_pool_kernel + coarse_csr_kernel + attn_fwd_tc_kernel<true>"},
         "gated_merge": {"ms": m_ms, "algorithmic_bytes": m_bytes, "gbs": m_bytes / (m_ms * 1e-3) / 1e9,
                         "hbm_frac": m_bytes / (m_ms * 1e-3) / 1e9 / hbm},
+        **extra,
     }
 
 
@@ -403,7 +434,7 @@ def run_ours(args, wl):
 
     hbm, bf16_burst, bf16_sus, peak_kind = load_peaks()
     next_rows = None
-    if not wl.backward and not args.no_next:
+    if not args.no_next:
         next_rows = time_next_rows(e, x, wl, args.steps, stream, l2_flush, ev, hbm, bf16_sus)
     fwd_ms = statistics.mean(per["fwd"])
     fwd_tflops = pair_flops(wl, pairs, False) / (fwd_ms * 1e-3) / 1e12

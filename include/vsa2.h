@@ -171,6 +171,37 @@ vsa2_status vsa2_gated_merge(const vsa2_problem* p, const void* o_f, const float
                              void* o, void* stream);
 
 /*
+ * Gradients of the gated merge, Eq. 4 and Eq. 13-14. With G = tanh(gate_logits):
+ *   d_logits[b,h,t] = (1 - G[t]^2) * sum_d dout[b,h,t,d] * oc[b,h,t/64,d]
+ *   d_oc[b,h,i,:]   = sum over the 64 tokens t of tile i of G[t] * dout[b,h,t,:]
+ * The fine branch's output gradient is dout itself (pass dout to vsa2_sparse_attn_bwd).
+ *   dout        : [batch, heads, L, D] of dtype (read only), the gradient of o
+ *   gate_logits : [batch, heads, L] fp32 (read only); oc : [batch, heads, N, D] of dtype
+ *   d_logits    : [batch, heads, L] fp32 (written); d_oc : [batch, heads, N, D] fp32 (written)
+ * Takes no workspace.
+ */
+vsa2_status vsa2_gated_merge_bwd(const vsa2_problem* p, const void* dout, const float* gate_logits, const void* oc,
+                                 float* d_logits, float* d_oc, void* stream);
+
+/*
+ * Gradients of the coarse branch, Eq. 1-3, ADDED to dq, dk, dv. With P_c and O_c_hat = oc:
+ *   dS = P_c * (d_oc Vc^T - rowsum(d_oc * oc)),  dQc = dS Kc / sqrt(D),  dKc = dS^T Qc / sqrt(D),
+ *   dVc = P_c^T d_oc, and MeanPool_B's adjoint spreads them: dq[t] += dQc[t/64] / 64 (same for
+ *   dk, dv). Call it after vsa2_sparse_attn_bwd (which overwrites dq, dk, dv) to obtain the
+ *   gradients of the whole Eq. 14 output.
+ *   q, k, v : [batch, heads, L, D] of dtype (read only)
+ *   oc      : [batch, heads, N, D] of dtype and lse_c : [batch, heads, N] fp32, from
+ *             vsa2_coarse_attn (read only)
+ *   d_oc    : [batch, heads, N, D] fp32 (read only), e.g. from vsa2_gated_merge_bwd; rounded to
+ *             dtype for the tensor cores
+ *   dq, dk, dv : [batch, heads, L, D] fp32 (read and written: +=)
+ * Uses the workspace of vsa2_workspace_size().
+ */
+vsa2_status vsa2_coarse_attn_bwd(const vsa2_problem* p, const void* q, const void* k, const void* v, const void* oc,
+                                 const float* lse_c, const float* d_oc, float* dq, float* dk, float* dv, void* ws,
+                                 size_t ws_bytes, void* stream);
+
+/*
  * End-to-end forward from HOST memory: router (Eq. 5-7), per-sequence TopK (Eq. 8-9) and
  * block-sparse attention (Eq. 12) for inputs and outputs that live in host memory. It computes
  * exactly what vsa2_router_scores + vsa2_topk_select + vsa2_sparse_attn_fwd compute on device

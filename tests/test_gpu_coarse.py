@@ -1,5 +1,5 @@
-"""GPU parity of the coarse branch (Eq. 1-3) and the gated merge (Eq. 4, 13-14) against the
-fp64 oracle, through the C ABI.
+"""GPU parity of the coarse branch (Eq. 1-3) and the gated merge (Eq. 4, 13-14), forward and
+backward, against the fp64 oracle, through the C ABI.
 
 Tolerances are the attention-output ones: max |err| <= 2e-2 and relative L2 <= 5e-3, and LSE
 within 2e-3 relative. The GPU rounds the pooled rows to the input dtype before the coarse
@@ -11,6 +11,8 @@ The cases cover the pooled sequence's shapes:
   * a whole number of tiles;
   * 480p and 720p heads (12 and 53 tiles, with 24 and 32 rows in the last one);
   * the tensor-core kernel (bf16, D = 128) and the CUDA-core kernel (fp32 or D = 64).
+The gradient tests use tile-constant inputs with tile values exact in the dtype, so that both
+sides pool to the same operands, and give both sides the same stored forward output.
 """
 import numpy as np
 import pytest
@@ -144,3 +146,98 @@ def test_attention_output_is_the_gated_sum_of_both_branches():
             o_f, _ = O.sparse_attn_fwd(x["q"][b, h], x["k"][b, h], x["v"][b, h], kv_off[b, h], kv_idx[b, h])
             oc, _ = O.coarse_attn(x["q"][b, h], x["k"][b, h], x["v"][b, h])
             _close(o[b, h], O.gated_merge(o_f, oc, logits[b, h]), f"o[{b},{h}]")
+
+
+# ------------------------------------------------------------------------------------------
+# gradients
+# ------------------------------------------------------------------------------------------
+def _tile_constant(wl, rng):
+    """Q, K, V constant inside every tile, with tile values exactly representable in the dtype.
+    The coarse branch sees only tile means, so these inputs lose nothing for it, and both sides
+    then pool to the same values (the GPU rounds pooled rows to the dtype)."""
+    shape = (wl.batch, wl.heads, wl.num_tiles, wl.head_dim)
+    return {n: np.repeat(S.round_to_dtype(rng.standard_normal(shape).astype(np.float32), wl.dtype), 64, axis=2)
+            for n in "qkv"}
+
+
+@pytest.mark.parametrize("case", ["one_padded_tile", "ragged_tail", "whole_tiles", "d64_bf16", "fp32_d64"])
+def test_coarse_attn_bwd_matches_oracle(case):
+    wl = CASES[case]
+    rng = np.random.default_rng(41)
+    x = _tile_constant(wl, rng)
+    B, H, N, L, D = wl.batch, wl.heads, wl.num_tiles, wl.tokens, wl.head_dim
+    d_oc = S.round_to_dtype(rng.standard_normal((B, H, N, D)).astype(np.float32), wl.dtype)
+    # both sides take the same stored forward: the oracle's O_c_hat rounded to the dtype, its LSE
+    oc, lse = np.zeros((B, H, N, D), np.float32), np.zeros((B, H, N), np.float32)
+    for b in range(B):
+        for h in range(H):
+            o, l_ = O.coarse_attn(x["q"][b, h], x["k"][b, h], x["v"][b, h])
+            oc[b, h], lse[b, h] = S.round_to_dtype(o.astype(np.float32), wl.dtype), l_
+    e = _engine(wl)
+    g0 = {n: torch.randn(B, H, L, D, device="cuda") for n in "qkv"}  # the call adds to these
+    g = {n: t.clone() for n, t in g0.items()}
+    e.coarse_attn_bwd(*(_dev(x[n], wl.dtype) for n in "qkv"), _dev(oc, wl.dtype), torch.from_numpy(lse).cuda(),
+                      torch.from_numpy(d_oc).cuda(), g["q"], g["k"], g["v"])
+    assert e.device_error() == 0
+    got = {n: (g[n] - g0[n]).cpu().numpy() for n in "qkv"}
+    for b in range(B):
+        for h in range(H):
+            want = O.coarse_attn_bwd(x["q"][b, h], x["k"][b, h], x["v"][b, h], d_oc[b, h], o_c_hat=oc[b, h])
+            for n, w in zip("qkv", want):
+                _close(got[n][b, h], w, f"{case} d{n}[{b},{h}]")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_gated_merge_bwd_matches_oracle(dtype):
+    wl = S.Workload("merge_bwd", 2, 3, 128, (8, 16, 20), 6, dtype)
+    rng = np.random.default_rng(42)
+    B, H, N, L, D = wl.batch, wl.heads, wl.num_tiles, wl.tokens, wl.head_dim
+    dout = S.round_to_dtype(rng.standard_normal((B, H, L, D)).astype(np.float32), dtype)
+    oc = S.round_to_dtype(rng.standard_normal((B, H, N, D)).astype(np.float32), dtype)
+    logits = (rng.standard_normal((B, H, L)) * 2).astype(np.float32)
+    e = _engine(wl)
+    d_logits, d_oc = e.gated_merge_bwd(_dev(dout, dtype), torch.from_numpy(logits).cuda(), _dev(oc, dtype))
+    d_logits, d_oc = d_logits.cpu().numpy(), d_oc.cpu().numpy()
+    for b in range(B):
+        for h in range(H):
+            _, want_oc, want_l = O.gated_merge_bwd(dout[b, h], oc[b, h], logits[b, h])
+            for got, want, what in ((d_oc[b, h], want_oc, "d_oc"), (d_logits[b, h], want_l, "d_logits")):
+                err = np.abs(got - want).max()
+                assert err <= 1e-4 * max(1.0, np.abs(want).max()), f"{dtype} {what}[{b},{h}]: {err:.3e}"
+
+
+def test_vsa2_attention_autograd_matches_oracle():
+    """Gradients of the whole Eq. 14 output through the autograd function against the oracle:
+    the fine branch's backward on the GPU's selection, the merge's and the coarse branch's.
+    Tile-constant inputs keep the coarse operands exact on both sides. The tolerance is twice the
+    attention one in relative L2: the fine backward forms Delta from the bf16 output it stored
+    (reading 10), and the gradients are returned in bf16."""
+    wl = CASES["ragged_tail"]
+    rng = np.random.default_rng(43)
+    x = _tile_constant(wl, rng)
+    B, H, L, D = wl.batch, wl.heads, wl.tokens, wl.head_dim
+    logits = rng.standard_normal((B, H, L)).astype(np.float32)
+    w = S.round_to_dtype(rng.standard_normal((B, H, L, D)).astype(np.float32), "bf16")
+    e = _engine(wl)
+    xd = {n: _dev(x[n], "bf16").requires_grad_(True) for n in "qkv"}
+    ld = torch.from_numpy(logits).cuda().requires_grad_(True)
+    with torch.no_grad():
+        sel = e.topk_select(e.router_scores(xd["q"], xd["k"]), wl.topk, csc=False)
+    o = V.vsa2_attention(xd["q"], xd["k"], xd["v"], ld, e)
+    (o.float() * torch.from_numpy(w).cuda()).sum().backward()
+    assert e.device_error() == 0
+    kv_off, kv_idx = sel[0].cpu().numpy(), sel[1].cpu().numpy()
+    for b in range(B):
+        for h in range(H):
+            qh, kh, vh = x["q"][b, h], x["k"][b, h], x["v"][b, h]
+            fine = O.sparse_attn_bwd(qh, kh, vh, w[b, h], kv_off[b, h], kv_idx[b, h])
+            oc, _ = O.coarse_attn(qh, kh, vh)
+            _, d_oc, d_logits = O.gated_merge_bwd(w[b, h], oc, logits[b, h])
+            coarse = O.coarse_attn_bwd(qh, kh, vh, d_oc)
+            for n, f, c in zip("qkv", fine, coarse):
+                got = xd[n].grad[b, h].float().cpu().numpy()
+                want = f + c
+                rel = np.linalg.norm(got - want) / np.linalg.norm(want)
+                assert rel <= 1e-2, f"d{n}[{b},{h}]: rel L2 {rel:.3e}"
+            gl = ld.grad[b, h].cpu().numpy()
+            assert np.abs(gl - d_logits).max() <= 2e-2 * max(1.0, np.abs(d_logits).max()), f"d_logits[{b},{h}]"

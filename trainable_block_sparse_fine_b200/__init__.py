@@ -11,8 +11,9 @@ from __future__ import annotations
 
 import torch
 
-from ._capi import (VSA2_FLAG_VALIDATE, Problem, Vsa2Error, lib, make_problem, vsa2_coarse_attn, vsa2_forward_host,
-                    vsa2_forward_host_workspace_size, vsa2_gated_merge, vsa2_get_device_error, vsa2_router_scores,
+from ._capi import (VSA2_FLAG_VALIDATE, Problem, Vsa2Error, lib, make_problem, vsa2_coarse_attn,
+                    vsa2_coarse_attn_bwd, vsa2_forward_host, vsa2_forward_host_workspace_size, vsa2_gated_merge,
+                    vsa2_gated_merge_bwd, vsa2_get_device_error, vsa2_router_scores,
                     vsa2_selftest_wait_timeout, vsa2_sparse_attn_bwd, vsa2_sparse_attn_fwd, vsa2_status_string,
                     vsa2_topk_select, vsa2_version, vsa2_workspace_init, vsa2_workspace_size)
 
@@ -20,7 +21,7 @@ __all__ = ["VSA2", "Vsa2Error", "Problem", "make_problem", "block_sparse_attenti
            "vsa2_router_scores", "vsa2_topk_select", "vsa2_sparse_attn_fwd", "vsa2_sparse_attn_bwd",
            "vsa2_workspace_size", "vsa2_workspace_init", "vsa2_get_device_error", "vsa2_selftest_wait_timeout",
            "vsa2_status_string", "vsa2_version", "vsa2_forward_host", "vsa2_forward_host_workspace_size",
-           "vsa2_coarse_attn", "vsa2_gated_merge"]
+           "vsa2_coarse_attn", "vsa2_gated_merge", "vsa2_gated_merge_bwd", "vsa2_coarse_attn_bwd", "vsa2_attention"]
 
 
 class VSA2:
@@ -98,6 +99,18 @@ class VSA2:
         vsa2_gated_merge(self.p, o_f, gate_logits, oc, out)
         return out
 
+    def gated_merge_bwd(self, dout, gate_logits, oc):
+        """Gradients of Eq. 4, 13-14: (d_gate_logits [B, H, L], d_oc [B, H, N, D]), fp32."""
+        d_logits = torch.empty(gate_logits.shape, dtype=torch.float32, device=self.device)
+        d_oc = torch.empty(oc.shape, dtype=torch.float32, device=self.device)
+        vsa2_gated_merge_bwd(self.p, dout, gate_logits, oc, d_logits, d_oc)
+        return d_logits, d_oc
+
+    def coarse_attn_bwd(self, q, k, v, oc, lse_c, d_oc, dq, dk, dv):
+        """Adds the coarse branch's gradients (Eq. 1-3) to the fp32 tensors dq, dk, dv."""
+        vsa2_coarse_attn_bwd(self.p, q, k, v, oc, lse_c, d_oc, dq, dk, dv, self.ws)
+        return dq, dk, dv
+
     def attention(self, q, k, v, gate_logits, topk=None):
         """The whole VSA2 attention output, Eq. 14: fine branch (router, TopK, Eq. 12) plus the
         gated coarse branch. Returns o."""
@@ -147,6 +160,38 @@ class _BlockSparseAttention(torch.autograd.Function):
         q, k, v, o, lse, kv_off, kv_idx, q_off, q_idx = ctx.saved_tensors
         dq, dk, dv = ctx.engine.attn_bwd(q, k, v, o, lse, dout.contiguous(), kv_off, kv_idx, q_off, q_idx, ctx.topk)
         return dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), None, None
+
+
+class _Vsa2Attention(torch.autograd.Function):
+    """Eq. 14: o = tanh(gate_logits) * Repeat_B(coarse(q, k, v)) + fine(q, k, v; router TopK)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, gate_logits, engine: VSA2, topk):
+        with torch.no_grad():  # the router receives no gradient (§2.1)
+            scores = engine.router_scores(q, k)
+            kv_off, kv_idx, q_off, q_idx = engine.topk_select(scores, topk, csc=True)
+        o_f, lse = engine.attn_fwd(q, k, v, kv_off, kv_idx, topk)
+        oc, lse_c = engine.coarse_attn(q, k, v)
+        o = engine.gated_merge(o_f, gate_logits, oc)
+        ctx.save_for_backward(q, k, v, o_f, lse, kv_off, kv_idx, q_off, q_idx, oc, lse_c, gate_logits)
+        ctx.engine, ctx.topk = engine, topk
+        return o
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, o_f, lse, kv_off, kv_idx, q_off, q_idx, oc, lse_c, gate_logits = ctx.saved_tensors
+        e = ctx.engine
+        dout = dout.contiguous()
+        dq, dk, dv = e.attn_bwd(q, k, v, o_f, lse, dout, kv_off, kv_idx, q_off, q_idx, ctx.topk)
+        d_logits, d_oc = e.gated_merge_bwd(dout, gate_logits, oc)
+        e.coarse_attn_bwd(q, k, v, oc, lse_c, d_oc, dq, dk, dv)
+        return dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), d_logits.to(gate_logits.dtype), None, None
+
+
+def vsa2_attention(q, k, v, gate_logits, engine: VSA2, topk=None):
+    """The whole VSA2 attention (coarse branch, router, fine branch, gated merge; Eq. 1-14) as an
+    autograd function. gate_logits = X W_g (Eq. 13), fp32 [B, H, L]."""
+    return _Vsa2Attention.apply(q, k, v, gate_logits, engine, engine.topk if topk is None else topk)
 
 
 def block_sparse_attention(q, k, v, engine: VSA2, topk=None):

@@ -72,6 +72,10 @@ WsLayout ws_layout(const Dims& d) {
   w.lse_c = take((size_t)d.BH * lc * 4);
   w.c_off = take((size_t)d.BH * (w.Nc_tiles + 1) * 4);
   w.c_idx = take((size_t)d.BH * w.Nc_tiles * w.Nc_tiles * 4);
+  w.doc = take((size_t)d.BH * lc * d.D * d.esize);
+  w.dqc = take((size_t)d.BH * lc * d.D * 4);
+  w.dkc = take((size_t)d.BH * lc * d.D * 4);
+  w.dvc = take((size_t)d.BH * lc * d.D * 4);
   w.total = off;
   return w;
 }
@@ -259,6 +263,31 @@ vsa2_status vsa2_gated_merge(const vsa2_problem* p, const void* o_f, const float
   if (!o_f || !gate_logits || !oc || !o) return VSA2_ERR_INVALID_ARG;
   if (!aligned16(o_f) || !aligned16(gate_logits) || !aligned16(oc) || !aligned16(o)) return VSA2_ERR_INVALID_ARG;
   return launch_gated_merge(d, o_f, gate_logits, oc, o, (cudaStream_t)stream);
+}
+
+vsa2_status vsa2_gated_merge_bwd(const vsa2_problem* p, const void* dout, const float* gate_logits, const void* oc,
+                                 float* d_logits, float* d_oc, void* stream) {
+  Dims d;
+  vsa2_status st = make_dims(p, &d);
+  if (st != VSA2_OK) return st;
+  if (!dout || !gate_logits || !oc || !d_logits || !d_oc) return VSA2_ERR_INVALID_ARG;
+  if (!aligned16(dout) || !aligned16(gate_logits) || !aligned16(oc) || !aligned16(d_logits) || !aligned16(d_oc))
+    return VSA2_ERR_INVALID_ARG;
+  return launch_gated_merge_bwd(d, dout, gate_logits, oc, d_logits, d_oc, (cudaStream_t)stream);
+}
+
+vsa2_status vsa2_coarse_attn_bwd(const vsa2_problem* p, const void* q, const void* k, const void* v, const void* oc,
+                                 const float* lse_c, const float* d_oc, float* dq, float* dk, float* dv, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  Dims d;
+  vsa2_status st = make_dims(p, &d);
+  if (st != VSA2_OK) return st;
+  if (!q || !k || !v || !oc || !lse_c || !d_oc || !dq || !dk || !dv) return VSA2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(oc) || !aligned16(lse_c) || !aligned16(d_oc) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return VSA2_ERR_INVALID_ARG;
+  if ((st = check_ws(d, ws, ws_bytes)) != VSA2_OK) return st;
+  return launch_coarse_attn_bwd(d, q, k, v, oc, lse_c, d_oc, dq, dk, dv, (char*)ws, (cudaStream_t)stream);
 }
 
 vsa2_status vsa2_topk_select_noalloc(const vsa2_problem* p, const float* scores, int32_t topk, int32_t* kv_off,

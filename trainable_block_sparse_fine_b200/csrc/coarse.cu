@@ -3,6 +3,7 @@
 //   Qc, Kc, Vc = MeanPool_B(Q, K, V)                 Eq. 1 (one row per 64-token tile)
 //   O_c_hat    = softmax(Qc Kc^T / sqrt(D)) Vc       Eq. 2-3 (dense over the N pooled rows)
 //   O          = tanh(X W_g) * Repeat_B(O_c_hat) + O_f   Eq. 4, 13-14 (X W_g given per token)
+// and their gradients.
 //
 // The pooled rows of a head form a sequence of N "tokens", padded to Nc = ceil(N / 64) tiles.
 // Dense attention over it is the block-sparse forward with every tile listed and the padded
@@ -136,6 +137,104 @@ __global__ void __launch_bounds__(256) gated_merge_kernel(const T* o_f, const fl
   }
 }
 
+// Gradients of Eq. 4, 13-14, warp per tile i of head bh (64 tokens t):
+//   d_logits[t] = (1 - G[t]^2) * (dout[t] . oc[i]),   d_oc[i] = sum_t G[t] * dout[t],   G = tanh(logits)
+template <typename T, int D>
+__global__ void __launch_bounds__(256) gated_merge_bwd_kernel(const T* __restrict__ dout,
+                                                              const float* __restrict__ gate_logits,
+                                                              const T* __restrict__ oc, float* __restrict__ d_logits,
+                                                              float* __restrict__ d_oc, int N, int64_t L) {
+  constexpr int V = D / 32;
+  const int bh = blockIdx.y;
+  const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (i >= N) return;
+  const size_t row0 = (size_t)bh * L + (size_t)i * kTile;
+  float c[V], acc[V];
+  load_vec<T, V>(oc + ((size_t)bh * N + i) * D + lane * V, c);
+#pragma unroll
+  for (int e = 0; e < V; ++e) acc[e] = 0.f;
+  const float g0 = tanhf(__ldg(gate_logits + row0 + lane)), g1 = tanhf(__ldg(gate_logits + row0 + 32 + lane));
+  float r0 = 0.f, r1 = 0.f;
+#pragma unroll 4
+  for (int t = 0; t < kTile; ++t) {
+    float x[V];
+    load_vec<T, V>(dout + (row0 + t) * D + lane * V, x);
+    const float G = __shfl_sync(0xffffffffu, t < 32 ? g0 : g1, t & 31);
+    float dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < V; ++e) {
+      dot = fmaf(x[e], c[e], dot);
+      acc[e] = fmaf(G, x[e], acc[e]);
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    if (lane == (t & 31)) (t < 32 ? r0 : r1) = (1.f - G * G) * dot;
+  }
+  d_logits[row0 + lane] = r0;
+  d_logits[row0 + 32 + lane] = r1;
+  float* dst = d_oc + ((size_t)bh * N + i) * D + lane * V;
+#pragma unroll
+  for (int e = 0; e < V; ++e) dst[e] = acc[e];
+}
+
+// Inputs of the pooled sequence's backward, padded to Lc rows per head: O_c_hat and its
+// gradient in the input dtype with zero rows past N, and the LSE with 0 past N. With zero K, V,
+// O and dO rows there, the padded rows add nothing to the gradients of the real rows.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) coarse_pad_bwd_kernel(const T* __restrict__ oc, const float* __restrict__ lse_c,
+                                                             const float* __restrict__ d_oc, T* __restrict__ oc_pad,
+                                                             float* __restrict__ lse_pad, T* __restrict__ doc_pad,
+                                                             int N, int Lc) {
+  constexpr int V = D / 32;
+  const int bh = blockIdx.y;
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= Lc) return;
+  float o[V], g[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) o[e] = g[e] = 0.f;
+  if (r < N) {
+    load_vec<T, V>(oc + ((size_t)bh * N + r) * D + lane * V, o);
+#pragma unroll
+    for (int e = 0; e < V; ++e) g[e] = __ldg(d_oc + ((size_t)bh * N + r) * D + lane * V + e);
+  }
+  const size_t dst = ((size_t)bh * Lc + r) * D + lane * V;
+  store_vec<T, V>(oc_pad + dst, o);
+  store_vec<T, V>(doc_pad + dst, g);
+  if (lane == 0) lse_pad[(size_t)bh * Lc + r] = r < N ? __ldg(lse_c + (size_t)bh * N + r) : 0.f;
+}
+
+// MeanPool_B's adjoint, accumulated: dx[t] += dxc[tile(t)] / 64 for Q, K and V (fp32), four
+// channels per thread and iteration.
+__global__ void __launch_bounds__(256) coarse_pool_bwd_kernel(const float* __restrict__ dqc,
+                                                              const float* __restrict__ dkc,
+                                                              const float* __restrict__ dvc, float* __restrict__ dq,
+                                                              float* __restrict__ dk, float* __restrict__ dv,
+                                                              int64_t rows, int64_t L, int Lc, int D) {
+  const int cpr = D / 4;
+  const int64_t total = rows * cpr;
+  for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < total; c += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = c / cpr;
+    const int col = (int)(c - row * cpr) * 4;
+    const int64_t bh = row / L;
+    const int64_t src = ((size_t)bh * Lc + (row - bh * L) / kTile) * D + col;
+    const float* in[3] = {dqc, dkc, dvc};
+    float* out[3] = {dq, dk, dv};
+#pragma unroll
+    for (int x = 0; x < 3; ++x) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(in[x] + src));
+      float4* o = reinterpret_cast<float4*>(out[x] + row * D + col);
+      float4 b = *o;
+      b.x = fmaf(a.x, 1.f / kTile, b.x);
+      b.y = fmaf(a.y, 1.f / kTile, b.y);
+      b.z = fmaf(a.z, 1.f / kTile, b.z);
+      b.w = fmaf(a.w, 1.f / kTile, b.w);
+      *o = b;
+    }
+  }
+}
+
 template <typename T, int D>
 void launch_pool(const Dims& d, const void* q, const void* k, const void* v, char* ws, const WsLayout& w,
                  cudaStream_t s) {
@@ -191,6 +290,81 @@ vsa2_status launch_coarse_attn(const Dims& d, const void* q, const void* k, cons
                                  cudaMemcpyDeviceToDevice, s) != cudaSuccess)
     return cuda_fail("coarse branch: copy of the LSE rows");
   return VSA2_OK;
+}
+
+vsa2_status launch_gated_merge_bwd(const Dims& d, const void* dout, const float* gate_logits, const void* oc,
+                                   float* d_logits, float* d_oc, cudaStream_t s) {
+  const dim3 grid((d.N + 7) / 8, d.BH);
+  if (d.dtype == VSA2_BF16 && d.D == 128)
+    gated_merge_bwd_kernel<__nv_bfloat16, 128><<<grid, 256, 0, s>>>((const __nv_bfloat16*)dout, gate_logits,
+                                                                    (const __nv_bfloat16*)oc, d_logits, d_oc, d.N, d.L);
+  else if (d.dtype == VSA2_BF16)
+    gated_merge_bwd_kernel<__nv_bfloat16, 64><<<grid, 256, 0, s>>>((const __nv_bfloat16*)dout, gate_logits,
+                                                                   (const __nv_bfloat16*)oc, d_logits, d_oc, d.N, d.L);
+  else if (d.D == 128)
+    gated_merge_bwd_kernel<float, 128><<<grid, 256, 0, s>>>((const float*)dout, gate_logits, (const float*)oc,
+                                                            d_logits, d_oc, d.N, d.L);
+  else
+    gated_merge_bwd_kernel<float, 64><<<grid, 256, 0, s>>>((const float*)dout, gate_logits, (const float*)oc,
+                                                           d_logits, d_oc, d.N, d.L);
+  return check_launch("gated_merge_bwd_kernel");
+}
+
+namespace {
+template <typename T, int D>
+void launch_pad_bwd(const Dims& d, const void* oc, const float* lse_c, const float* d_oc, char* ws, const WsLayout& w,
+                    cudaStream_t s) {
+  const int Lc = kTile * w.Nc_tiles;
+  coarse_pad_bwd_kernel<T, D><<<dim3((Lc + 7) / 8, d.BH), 256, 0, s>>>(
+      (const T*)oc, lse_c, d_oc, (T*)(ws + w.oc), (float*)(ws + w.lse_c), (T*)(ws + w.doc), d.N, Lc);
+}
+}  // namespace
+
+vsa2_status launch_coarse_attn_bwd(const Dims& d, const void* q, const void* k, const void* v, const void* oc,
+                                   const float* lse_c, const float* d_oc, float* dq, float* dk, float* dv, char* ws,
+                                   cudaStream_t s) {
+  const WsLayout w = ws_layout(d);
+  const int Nc = w.Nc_tiles;
+  const int Lc = kTile * Nc;
+  Dims dc = d;
+  dc.L = Lc;
+  dc.N = Nc;
+  dc.Lr = Lc / kPool;
+  // the backward of the pooled sequence keeps its Delta and LSE where ws_layout(dc) puts them;
+  // every region of dc is at most the size of d's, so they end before the coarse regions
+  if (ws_layout(dc).nlse2 + align256((size_t)dc.BH * Lc * 4) > w.qc) return VSA2_ERR_UNSUPPORTED;
+  // pooled operands (Eq. 1) again, the padded O_c_hat, LSE and dO_c_hat, and the dense CSR / CSC
+  if (d.dtype == VSA2_BF16 && d.D == 128) {
+    launch_pool<__nv_bfloat16, 128>(d, q, k, v, ws, w, s);
+    launch_pad_bwd<__nv_bfloat16, 128>(d, oc, lse_c, d_oc, ws, w, s);
+  } else if (d.dtype == VSA2_BF16) {
+    launch_pool<__nv_bfloat16, 64>(d, q, k, v, ws, w, s);
+    launch_pad_bwd<__nv_bfloat16, 64>(d, oc, lse_c, d_oc, ws, w, s);
+  } else if (d.D == 128) {
+    launch_pool<float, 128>(d, q, k, v, ws, w, s);
+    launch_pad_bwd<float, 128>(d, oc, lse_c, d_oc, ws, w, s);
+  } else {
+    launch_pool<float, 64>(d, q, k, v, ws, w, s);
+    launch_pad_bwd<float, 64>(d, oc, lse_c, d_oc, ws, w, s);
+  }
+  int32_t* c_off = reinterpret_cast<int32_t*>(ws + w.c_off);
+  int32_t* c_idx = reinterpret_cast<int32_t*>(ws + w.c_idx);
+  coarse_csr_kernel<<<d.BH, 256, 0, s>>>(Nc, c_off, c_idx);
+  vsa2_status st = check_launch("coarse backward: pooling and padding");
+  if (st != VSA2_OK) return st;
+  // gradients of Eq. 2-3 over the pooled sequence; every tile lists every tile, so the CSC
+  // equals the CSR
+  float* dqc = reinterpret_cast<float*>(ws + w.dqc);
+  float* dkc = reinterpret_cast<float*>(ws + w.dkc);
+  float* dvc = reinterpret_cast<float*>(ws + w.dvc);
+  st = launch_attn_bwd(dc, ws + w.qc, ws + w.kc, ws + w.vc, ws + w.oc, reinterpret_cast<const float*>(ws + w.lse_c),
+                       ws + w.doc, Nc, c_off, c_idx, c_off, c_idx, dqc, dkc, dvc, ws, s);
+  if (st != VSA2_OK) return st;
+  // MeanPool_B's adjoint, added to the caller's gradients
+  const int64_t rows = (int64_t)d.BH * d.L;
+  coarse_pool_bwd_kernel<<<grid_for(rows * (d.D / 4), 256), 256, 0, s>>>(dqc, dkc, dvc, dq, dk, dv, rows, d.L, Lc,
+                                                                         d.D);
+  return check_launch("coarse_pool_bwd_kernel");
 }
 
 vsa2_status launch_gated_merge(const Dims& d, const void* o_f, const float* gate_logits, const void* oc, void* o,

@@ -46,6 +46,8 @@ struct WsLayout {
                          // rows >= N zero (Q, K, V) or unused (output)
   size_t lse_c;          // coarse branch LSE, [BH, 64 * Nc_tiles] fp32
   size_t c_off, c_idx;   // coarse branch: CSR listing every tile, [BH, Nc_tiles + 1], [BH, Nc_tiles^2] i32
+  size_t doc;            // coarse backward: padded gradient of O_c_hat, [BH, 64 * Nc_tiles, D] dtype
+  size_t dqc, dkc, dvc;  // coarse backward: gradients of the pooled rows, [BH, 64 * Nc_tiles, D] fp32
   size_t total;
 };
 WsLayout ws_layout(const Dims& d);
@@ -88,6 +90,11 @@ vsa2_status launch_coarse_attn(const Dims& d, const void* q, const void* k, cons
                                char* ws, cudaStream_t s);
 vsa2_status launch_gated_merge(const Dims& d, const void* o_f, const float* gate_logits, const void* oc, void* o,
                                cudaStream_t s);
+vsa2_status launch_gated_merge_bwd(const Dims& d, const void* dout, const float* gate_logits, const void* oc,
+                                   float* d_logits, float* d_oc, cudaStream_t s);
+vsa2_status launch_coarse_attn_bwd(const Dims& d, const void* q, const void* k, const void* v, const void* oc,
+                                   const float* lse_c, const float* d_oc, float* dq, float* dk, float* dv, char* ws,
+                                   cudaStream_t s);
 // tensor-core backward (bf16, head_dim 128): dQ kernel (also writes Delta), then dK/dV kernel
 vsa2_status attn_bwd_tc(const Dims& d, const void* q, const void* k, const void* v, const void* o, const float* lse,
                         const void* dout, const int32_t* kv_off, const int32_t* kv_idx, const int32_t* q_off,
