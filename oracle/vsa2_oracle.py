@@ -38,6 +38,8 @@ __all__ = [
     "gated_merge",
     "coarse_attn_bwd",
     "gated_merge_bwd",
+    "permute_to_cube_major",
+    "permute_to_raster",
 ]
 
 
@@ -289,3 +291,37 @@ def gated_merge_bwd(dout, o_c_hat, gate_logits, tile_tokens: int = 64):
     d_oc = (g[:, None] * dout).reshape(L // tile_tokens, tile_tokens, D).sum(axis=1)
     d_logits = (1.0 - g * g) * (dout * o_c).sum(axis=1)
     return dout.copy(), d_oc, d_logits
+
+
+def _cube_major_coords(grid, tile, pool):
+    """Raster coordinates (t, h, w) of the tokens in cube-major order (§2.2 "Permutation"):
+    tiles of `tile` tokens in raster order over the tile grid; inside a tile, its sub-cubes of
+    `pool` tokens in raster order; inside a sub-cube, its tokens in raster order."""
+    T, H, W = grid
+    bt, bh, bw = tile
+    rt, rh, rw = pool
+    for a in range(T // bt):
+        for b in range(H // bh):
+            for c in range(W // bw):
+                for st in range(bt // rt):
+                    for sh in range(bh // rh):
+                        for sw in range(bw // rw):
+                            for dt in range(rt):
+                                for dh in range(rh):
+                                    for dw in range(rw):
+                                        yield (a * bt + st * rt + dt, b * bh + sh * rh + dh, c * bw + sw * rw + dw)
+
+
+def permute_to_cube_major(x, tile=(4, 4, 4), pool=(2, 2, 4)):
+    """(T, H, W, D) tokens in raster order -> (T*H*W, D) in cube-major order."""
+    T, H, W, D = x.shape
+    return np.stack([x[t, h, w] for t, h, w in _cube_major_coords((T, H, W), tile, pool)])
+
+
+def permute_to_raster(y, grid, tile=(4, 4, 4), pool=(2, 2, 4)):
+    """Inverse of permute_to_cube_major: (T*H*W, D) cube-major -> (T, H, W, D) raster."""
+    T, H, W = grid
+    out = np.empty((T, H, W, y.shape[1]), dtype=y.dtype)
+    for l, (t, h, w) in enumerate(_cube_major_coords(grid, tile, pool)):
+        out[t, h, w] = y[l]
+    return out

@@ -583,3 +583,32 @@ def test_coarse_bwd_given_output_enters_only_through_rowsum():
     moved = O.coarse_attn_bwd(q, k, v, w, o_c_hat=o + 0.01)
     np.testing.assert_array_equal(moved[2], base[2])
     assert np.abs(moved[0] - base[0]).max() > 1e-6
+
+
+# --------------------------------------------------------------------------------------------
+# token permutation, §2.2 "Permutation"
+# --------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("grid,tile,pool", [((8, 16, 20), (4, 4, 4), (2, 2, 4)), ((4, 8, 16), (2, 4, 8), (1, 2, 8)),
+                                            ((12, 12, 8), (4, 4, 4), (2, 2, 4))])
+def test_permutation_matches_reshape_transpose_and_round_trips(grid, tile, pool):
+    """Against the input generator's reshape/transpose formulation (a different construction of
+    the same order), and the inverse restores the raster tensor exactly."""
+    x = np.random.default_rng(28).standard_normal((*grid, 3))
+    y = O.permute_to_cube_major(x, tile, pool)
+    np.testing.assert_array_equal(y, S.raster_to_cube_major(x, tile, pool))
+    np.testing.assert_array_equal(O.permute_to_raster(y, grid, tile, pool), x)
+
+
+def test_permutation_tile_and_subcube_membership():
+    """Row block i of 64 holds exactly the tokens of the i-th 4x4x4 cube in raster order of the
+    cube grid, and each block of 16 inside it one 2x2x4 sub-cube."""
+    grid = (8, 8, 8)
+    T, H, W = grid
+    idx = np.arange(T * H * W, dtype=np.float64).reshape(T, H, W, 1)  # value = raster index
+    y = O.permute_to_cube_major(idx)[:, 0].astype(int)
+    t, h, w = np.unravel_index(y, grid)
+    tiles = (t // 4) * (H // 4) * (W // 4) + (h // 4) * (W // 4) + (w // 4)
+    np.testing.assert_array_equal(tiles, np.repeat(np.arange(T * H * W // 64), 64))
+    sub = ((t % 4) // 2) * 2 + (h % 4) // 2
+    np.testing.assert_array_equal(sub, np.tile(np.repeat(np.arange(4), 16), T * H * W // 64))
