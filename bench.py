@@ -306,6 +306,21 @@ def time_next_rows(e, x, wl, steps, stream, l2_flush, ev, hbm, tc_peak):
                                 "kernels": "pool + pad + attn_bwd_dq_tc_kernel + attn_bwd_dkdv_tc_kernel + "
                                            "coarse_pool_bwd_kernel"},
         }
+    # the token permutation (§2.2): Q from raster to cube-major order, one read and one write
+    tp = []
+    for it in range(3 + steps):
+        t = [ev() for _ in range(2)]
+        l2_flush.zero_()
+        t[0].record(stream)
+        e.to_cube_major(x["q"], out=out)
+        t[1].record(stream)
+        torch.cuda.synchronize()
+        if it >= 3:
+            tp.append(t[0].elapsed_time(t[1]))
+    p_ms = statistics.mean(tp)
+    p_bytes = 2 * B * H * L * D * esize
+    extra["permute"] = {"ms": p_ms, "algorithmic_bytes": p_bytes, "gbs": p_bytes / (p_ms * 1e-3) / 1e9,
+                        "hbm_frac": p_bytes / (p_ms * 1e-3) / 1e9 / hbm, "kernel": "permute_kernel (Q)"}
     err = e.device_error()
     if err != 0:
         raise RuntimeError(f"device error {err} in the coarse branch")

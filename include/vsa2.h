@@ -202,6 +202,19 @@ vsa2_status vsa2_coarse_attn_bwd(const vsa2_problem* p, const void* q, const voi
                                  size_t ws_bytes, void* stream);
 
 /*
+ * Token permutation, §2.2 "Permutation": between raster order (t, h, w), t slowest, and the
+ * cube-major order every other call takes (tiles of tile_t x tile_h x tile_w tokens in raster
+ * order; inside a tile its pool_t x pool_h x pool_w sub-cubes in raster order; inside a
+ * sub-cube its tokens in raster order). The paper applies it once at the start of the
+ * transformer; it costs one read and one write of the tensor.
+ *   src, dst      : [batch, heads, L, D] of dtype, distinct buffers (dst written)
+ *   to_cube_major : nonzero: src is in raster order, dst in cube-major order; zero: the inverse
+ * Takes no workspace.
+ */
+vsa2_status vsa2_permute_tokens(const vsa2_problem* p, const void* src, void* dst, int32_t to_cube_major,
+                                void* stream);
+
+/*
  * End-to-end forward from HOST memory: router (Eq. 5-7), per-sequence TopK (Eq. 8-9) and
  * block-sparse attention (Eq. 12) for inputs and outputs that live in host memory. It computes
  * exactly what vsa2_router_scores + vsa2_topk_select + vsa2_sparse_attn_fwd compute on device

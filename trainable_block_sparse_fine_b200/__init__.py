@@ -13,7 +13,7 @@ import torch
 
 from ._capi import (VSA2_FLAG_VALIDATE, Problem, Vsa2Error, lib, make_problem, vsa2_coarse_attn,
                     vsa2_coarse_attn_bwd, vsa2_forward_host, vsa2_forward_host_workspace_size, vsa2_gated_merge,
-                    vsa2_gated_merge_bwd, vsa2_get_device_error, vsa2_router_scores,
+                    vsa2_gated_merge_bwd, vsa2_get_device_error, vsa2_permute_tokens, vsa2_router_scores,
                     vsa2_selftest_wait_timeout, vsa2_sparse_attn_bwd, vsa2_sparse_attn_fwd, vsa2_status_string,
                     vsa2_topk_select, vsa2_version, vsa2_workspace_init, vsa2_workspace_size)
 
@@ -21,7 +21,8 @@ __all__ = ["VSA2", "Vsa2Error", "Problem", "make_problem", "block_sparse_attenti
            "vsa2_router_scores", "vsa2_topk_select", "vsa2_sparse_attn_fwd", "vsa2_sparse_attn_bwd",
            "vsa2_workspace_size", "vsa2_workspace_init", "vsa2_get_device_error", "vsa2_selftest_wait_timeout",
            "vsa2_status_string", "vsa2_version", "vsa2_forward_host", "vsa2_forward_host_workspace_size",
-           "vsa2_coarse_attn", "vsa2_gated_merge", "vsa2_gated_merge_bwd", "vsa2_coarse_attn_bwd", "vsa2_attention"]
+           "vsa2_coarse_attn", "vsa2_gated_merge", "vsa2_gated_merge_bwd", "vsa2_coarse_attn_bwd", "vsa2_attention",
+           "vsa2_permute_tokens"]
 
 
 class VSA2:
@@ -83,6 +84,19 @@ class VSA2:
         sel = self.topk_select(scores, topk, csc=csc)
         o, lse = self.attn_fwd(q, k, v, sel[0], sel[1], topk)
         return o, lse, sel
+
+    def to_cube_major(self, x, out=None):
+        """[B, H, L, D] (or [B, H, T, H, W, D]) in raster token order -> [B, H, L, D] cube-major."""
+        out = out if out is not None else torch.empty(self.batch, self.heads, self.L, self.head_dim, dtype=x.dtype,
+                                                      device=self.device)
+        vsa2_permute_tokens(self.p, x, out, True)
+        return out
+
+    def to_raster(self, x, out=None):
+        """[B, H, L, D] cube-major -> [B, H, L, D] in raster token order (t, h, w)."""
+        out = out if out is not None else torch.empty_like(x)
+        vsa2_permute_tokens(self.p, x, out, False)
+        return out
 
     def coarse_attn(self, q, k, v, oc=None, lse_c=None):
         """Coarse branch, Eq. 1-3: O_c_hat [B, H, N, D] (input dtype) and its LSE [B, H, N]."""

@@ -21,7 +21,8 @@ EXPORTS = ("vsa2_workspace_size", "vsa2_workspace_init", "vsa2_router_scores", "
            "vsa2_sparse_attn_fwd", "vsa2_sparse_attn_bwd", "vsa2_get_device_error",
            "vsa2_selftest_wait_timeout", "vsa2_status_string", "vsa2_version", "vsa2_last_cuda_error",
            "vsa2_topk_select_noalloc", "vsa2_forward_host", "vsa2_forward_host_workspace_size",
-           "vsa2_coarse_attn", "vsa2_gated_merge", "vsa2_gated_merge_bwd", "vsa2_coarse_attn_bwd")
+           "vsa2_coarse_attn", "vsa2_gated_merge", "vsa2_gated_merge_bwd", "vsa2_coarse_attn_bwd",
+           "vsa2_permute_tokens")
 
 
 class Vsa2Error(RuntimeError):
@@ -65,6 +66,7 @@ def lib() -> ctypes.CDLL:
         L.vsa2_coarse_attn.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
         L.vsa2_gated_merge.argtypes = [P, vp, vp, vp, vp, vp]
         L.vsa2_gated_merge_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp]
+        L.vsa2_permute_tokens.argtypes = [P, vp, vp, i32, vp]
         L.vsa2_coarse_attn_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.vsa2_get_device_error.argtypes = [vp, vp]
         L.vsa2_selftest_wait_timeout.argtypes = [vp, sz, u32, vp]
@@ -74,7 +76,7 @@ def lib() -> ctypes.CDLL:
         L.vsa2_last_cuda_error.restype = ctypes.c_char_p
         for name in ("vsa2_workspace_init", "vsa2_router_scores", "vsa2_topk_select", "vsa2_topk_select_noalloc",
                      "vsa2_sparse_attn_fwd", "vsa2_forward_host", "vsa2_coarse_attn", "vsa2_gated_merge",
-                     "vsa2_gated_merge_bwd", "vsa2_coarse_attn_bwd",
+                     "vsa2_gated_merge_bwd", "vsa2_coarse_attn_bwd", "vsa2_permute_tokens",
                      "vsa2_sparse_attn_bwd", "vsa2_get_device_error", "vsa2_selftest_wait_timeout"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -170,6 +172,11 @@ def vsa2_coarse_attn_bwd(p: Problem, q, k, v, oc, lse_c, d_oc, dq, dk, dv, ws, s
     _check(lib().vsa2_coarse_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(oc), _ptr(lse_c), _ptr(d_oc),
                                       _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel() * ws.element_size(),
                                       _stream(stream)), "vsa2_coarse_attn_bwd")
+
+
+def vsa2_permute_tokens(p: Problem, src, dst, to_cube_major: bool, stream=None) -> None:
+    _check(lib().vsa2_permute_tokens(ctypes.byref(p), _ptr(src), _ptr(dst), 1 if to_cube_major else 0,
+                                     _stream(stream)), "vsa2_permute_tokens")
 
 
 def vsa2_forward_host_workspace_size(p: Problem, topk: int, heads_per_group: int = 0) -> int:

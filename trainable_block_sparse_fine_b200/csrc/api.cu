@@ -290,6 +290,16 @@ vsa2_status vsa2_coarse_attn_bwd(const vsa2_problem* p, const void* q, const voi
   return launch_coarse_attn_bwd(d, q, k, v, oc, lse_c, d_oc, dq, dk, dv, (char*)ws, (cudaStream_t)stream);
 }
 
+vsa2_status vsa2_permute_tokens(const vsa2_problem* p, const void* src, void* dst, int32_t to_cube_major,
+                                void* stream) {
+  Dims d;
+  vsa2_status st = make_dims(p, &d);
+  if (st != VSA2_OK) return st;
+  if (!src || !dst || src == dst) return VSA2_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(dst)) return VSA2_ERR_INVALID_ARG;
+  return launch_permute(d, p, src, dst, to_cube_major != 0, (cudaStream_t)stream);
+}
+
 vsa2_status vsa2_topk_select_noalloc(const vsa2_problem* p, const float* scores, int32_t topk, int32_t* kv_off,
                                      int32_t* kv_idx, void* stream) {
   Dims d;

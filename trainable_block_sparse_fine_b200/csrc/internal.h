@@ -99,6 +99,9 @@ vsa2_status launch_coarse_attn_bwd(const Dims& d, const void* q, const void* k, 
 vsa2_status attn_bwd_tc(const Dims& d, const void* q, const void* k, const void* v, const void* o, const float* lse,
                         const void* dout, const int32_t* kv_off, const int32_t* kv_idx, const int32_t* q_off,
                         const int32_t* q_idx, float* dq, float* dk, float* dv, int topk, char* ws, cudaStream_t s);
+// Token permutation raster <-> cube-major (to_cube != 0: raster -> cube-major)
+vsa2_status launch_permute(const Dims& d, const vsa2_problem* p, const void* src, void* dst, int to_cube,
+                           cudaStream_t s);
 vsa2_status launch_wait_timeout_probe(int* err, uint64_t timeout_ns, cudaStream_t s);
 // allocation-free TopK (scratch in a fixed device array of the library)
 size_t topk_noalloc_bytes(const Dims& d);
