@@ -342,7 +342,7 @@ const char* vsa2_status_string(vsa2_status s) {
   return "VSA2_UNKNOWN_STATUS";
 }
 
-int32_t vsa2_version(void) { return 100; }
+int32_t vsa2_version(void) { return 200; }  // 0.2.0: coarse branch, gated merge, permutation, host-buffer forward
 
 const char* vsa2_last_cuda_error(void) { return g_last_cuda_error.load(); }
 
