@@ -28,6 +28,7 @@ SMALL64 = S.Workload("small_bf16_d64", 2, 1, 64, (4, 16, 24), 5, "bf16")  # N=24
 TINY = S.WORKLOADS["tiny"]
 C480 = S.WORKLOADS["480p_top64"]
 C720 = S.WORKLOADS["720p_top64"]
+C480_128 = S.WORKLOADS["480p_top128"]  # same tensors as 480p_top64 (same grid and seeds), twice the budget
 
 
 def dev(x, dtype):
@@ -344,6 +345,19 @@ def test_fwd_480p_sampled_heads():
     heads = [0, 19]
     kv_off, kv_idx, _, _ = lists_from_masks(c480_lists(heads), wl.topk)
     _fwd_case(wl, inputs(wl), kv_off, kv_idx, heads=heads, tiles=[0, 1, 100, 363, 364, 727])
+
+
+def test_480p_top128_topk_bit_exact_and_forward_sampled():
+    """480p with top128 (93,184 selected pairs per head): TopK on the oracle's fp32 scores of all
+    20 heads is bit-exact, CSR and CSC, and the forward on that selection matches the oracle on
+    sampled query tiles (first, last, middle) of two heads."""
+    wl = C480_128
+    x = inputs(C480)
+    sc = oracle_scores(C480, x)
+    s32 = np.stack([np.stack([sc[(0, h)] for h in range(wl.heads)])]).astype(np.float32)
+    _topk_case(wl, s32)
+    kv_off, kv_idx, _, _ = oracle_csr(wl, s32)
+    _fwd_case(wl, x, kv_off, kv_idx, heads=[0, 19], tiles=[0, 1, 100, 363, 364, 727])
 
 
 # ------------------------------------------------------------------------------------------
