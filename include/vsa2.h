@@ -207,7 +207,8 @@ vsa2_status vsa2_coarse_attn_bwd(const vsa2_problem* p, const void* q, const voi
  * order; inside a tile its pool_t x pool_h x pool_w sub-cubes in raster order; inside a
  * sub-cube its tokens in raster order). The paper applies it once at the start of the
  * transformer; it costs one read and one write of the tensor.
- *   src, dst      : [batch, heads, L, D] of dtype, distinct buffers (dst written)
+ *   src, dst      : [batch, heads, L, D] of dtype, non-overlapping buffers (dst written);
+ *                   src == dst returns VSA2_ERR_INVALID_ARG
  *   to_cube_major : nonzero: src is in raster order, dst in cube-major order; zero: the inverse
  * Takes no workspace.
  */

@@ -122,3 +122,15 @@ def test_coarse_and_merge_argument_errors():
     assert lib.vsa2_gated_merge(bp, fake, fake, fake, ctypes.c_void_p((1 << 20) + 2), None) == 1
     bad = C.make_problem(1, 2, 96, (8, 16, 20))
     assert lib.vsa2_gated_merge(ctypes.byref(bad), fake, fake, fake, fake, None) == 2
+
+
+def test_permute_argument_errors():
+    lib = C.lib()
+    p = C.make_problem(1, 2, 128, (8, 16, 20))
+    bp = ctypes.byref(p)
+    a, b = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 24)  # never dereferenced
+    assert lib.vsa2_permute_tokens(bp, a, a, 1, None) == 1  # in place
+    assert lib.vsa2_permute_tokens(bp, None, b, 1, None) == 1
+    assert lib.vsa2_permute_tokens(bp, a, ctypes.c_void_p((1 << 24) + 4), 0, None) == 1
+    bad = C.make_problem(1, 2, 128, (8, 16, 20), tile=(4, 4, 2))  # tile of 32 tokens
+    assert lib.vsa2_permute_tokens(ctypes.byref(bad), a, b, 1, None) == 2
