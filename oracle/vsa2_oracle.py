@@ -40,6 +40,11 @@ __all__ = [
     "gated_merge_bwd",
     "permute_to_cube_major",
     "permute_to_raster",
+    "pad_to_tiles",
+    "router_scores_padded",
+    "sparse_attn_fwd_padded",
+    "coarse_attn_padded",
+    "vsa2_forward_padded",
 ]
 
 
@@ -325,3 +330,116 @@ def permute_to_raster(y, grid, tile=(4, 4, 4), pool=(2, 2, 4)):
     for l, (t, h, w) in enumerate(_cube_major_coords(grid, tile, pool)):
         out[t, h, w] = y[l]
     return out
+
+
+# ------------------------------------------------------------------------------------------
+# grids that the tile does not divide (§2.2 "Kernel Implementation": pad every dimension to a
+# multiple of the tile and mask the padding). Readings: pooled means run over real tokens only;
+# a sub-cube with no real token is masked as a key and has no query row; Eq. 7 averages the
+# real query sub-cubes of a tile; padding keys are masked in both attention branches; rows of
+# padding tokens are dropped when the output is cropped back to the grid.
+# ------------------------------------------------------------------------------------------
+
+def pad_to_tiles(x, tile=(4, 4, 4)):
+    """(T, H, W, D) raster -> ((T', H', W', D) zero-padded to multiples of the tile,
+    (T', H', W') bool mask of the real tokens)."""
+    T, H, W, D = x.shape
+    Tp, Hp, Wp = (-(-n // b) * b for n, b in zip((T, H, W), tile))
+    out = np.zeros((Tp, Hp, Wp, D), dtype=np.float64)
+    out[:T, :H, :W] = x
+    valid = np.zeros((Tp, Hp, Wp), dtype=bool)
+    valid[:T, :H, :W] = True
+    return out, valid
+
+
+def _masked_mean_pool(x, valid, group):
+    """Mean of the real rows of each group of `group` consecutive rows, and their counts."""
+    x = np.asarray(x, dtype=np.float64)
+    L, D = x.shape
+    w = np.asarray(valid, dtype=np.float64).reshape(L // group, group)
+    sums = (x.reshape(L // group, group, D) * w[:, :, None]).sum(axis=1)
+    counts = w.sum(axis=1)
+    means = np.where(counts[:, None] > 0, sums / np.maximum(counts, 1)[:, None], 0.0)
+    return means, counts
+
+
+def router_scores_padded(q, k, valid, tile_tokens: int = 64, pool_tokens: int = 16):
+    """Eq. 5-7 on a padded cube-major sequence; `valid` (L,) marks the real tokens.
+    Qr, Kr are means over real tokens; sub-cubes without one are masked keys and have no
+    query row; Pr[i, j] = (1 / g_i) sum over the g_i real query sub-cubes a of tile i of
+    sum over the real key sub-cubes b of tile j of P_hat[a, b]."""
+    qr, cq = _masked_mean_pool(q, valid, pool_tokens)
+    kr, ck = _masked_mean_pool(k, valid, pool_tokens)
+    G = tile_tokens // pool_tokens
+    Lr, D = qr.shape
+    N = Lr // G
+    s = (qr @ kr.T) / np.sqrt(D)
+    s[:, ck == 0] = -np.inf
+    s -= s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    p /= p.sum(axis=1, keepdims=True)
+    p[cq == 0] = 0.0
+    g = (cq > 0).reshape(N, G).sum(axis=1)
+    return p.reshape(N, G, N, G).sum(axis=(1, 3)) / g[:, None]
+
+
+def sparse_attn_fwd_padded(q, k, v, kv_off, kv_idx, valid, tile_tokens: int = 64):
+    """Eq. 12 with padding keys masked: for each query token t of tile i, the softmax runs over
+    the real tokens of the tiles selected for i. Padding query rows are returned as 0 (they
+    are dropped with the padding)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    L, D = q.shape
+    N = L // tile_tokens
+    o = np.zeros((L, D))
+    for i in range(N):
+        sel = np.asarray(kv_idx[kv_off[i]:kv_off[i + 1]])
+        if sel.size == 0:
+            continue
+        keys = np.concatenate([np.arange(j * tile_tokens, (j + 1) * tile_tokens) for j in sel])
+        keys = keys[np.asarray(valid)[keys]]
+        rows = np.arange(i * tile_tokens, (i + 1) * tile_tokens)
+        s = (q[rows] @ k[keys].T) / np.sqrt(D)
+        s -= s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        o[rows] = (p @ v[keys]) / p.sum(axis=1, keepdims=True)
+    o[~np.asarray(valid)] = 0.0
+    return o
+
+
+def coarse_attn_padded(q, k, v, valid, tile_tokens: int = 64):
+    """Eq. 1-3 on a padded sequence: Qc, Kc, Vc are means over the real tokens of each tile
+    (every tile of a padded grid holds one), then the dense softmax of Eq. 2 over all tiles."""
+    qc, _ = _masked_mean_pool(q, valid, tile_tokens)
+    kc, _ = _masked_mean_pool(k, valid, tile_tokens)
+    vc, _ = _masked_mean_pool(v, valid, tile_tokens)
+    D = qc.shape[1]
+    s = (qc @ kc.T) / np.sqrt(D)
+    s -= s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    return (p @ vc) / p.sum(axis=1, keepdims=True)
+
+
+def vsa2_forward_padded(q, k, v, gate_logits, topk, tile=(4, 4, 4), pool=(2, 2, 4)):
+    """Eq. 1-14 for one (b, h) on a raster grid (T, H, W) that the tile need not divide:
+    pad, permute to cube-major order, router with masked padding, per-sequence TopK over the
+    padded grid's tiles (budget N' * topk), fine and coarse branches with padding keys masked,
+    gated merge, then back to raster order, cropped to (T, H, W). Returns (O (T, H, W, D),
+    the TopK selection)."""
+    T, H, W, D = q.shape
+    qp, valid = pad_to_tiles(q, tile)
+    kp, _ = pad_to_tiles(k, tile)
+    vp, _ = pad_to_tiles(v, tile)
+    gp, _ = pad_to_tiles(np.asarray(gate_logits, dtype=np.float64)[..., None], tile)
+    grid_p = qp.shape[:3]
+    qc, kc, vc, gc = (permute_to_cube_major(x, tile, pool) for x in (qp, kp, vp, gp))
+    vm = permute_to_cube_major(valid[..., None].astype(np.float64), tile, pool)[:, 0] > 0
+    tile_tokens = int(np.prod(tile))
+    pool_tokens = int(np.prod(pool))
+    scores = router_scores_padded(qc, kc, vm, tile_tokens, pool_tokens)
+    sel = topk_select(scores.astype(np.float32), topk)
+    o_f = sparse_attn_fwd_padded(qc, kc, vc, sel["kv_off"], sel["kv_idx"], vm, tile_tokens)
+    o_c = coarse_attn_padded(qc, kc, vc, vm, tile_tokens)
+    o = gated_merge(o_f, o_c, gc[:, 0], tile_tokens)
+    return permute_to_raster(o, grid_p, tile, pool)[:T, :H, :W], sel

@@ -612,3 +612,135 @@ def test_permutation_tile_and_subcube_membership():
     np.testing.assert_array_equal(tiles, np.repeat(np.arange(T * H * W // 64), 64))
     sub = ((t % 4) // 2) * 2 + (h % 4) // 2
     np.testing.assert_array_equal(sub, np.tile(np.repeat(np.arange(4), 16), T * H * W // 64))
+
+
+# --------------------------------------------------------------------------------------------
+# grids the tile does not divide: padding and masks (§2.2 "Kernel Implementation")
+# --------------------------------------------------------------------------------------------
+
+def _padded_cube_major(x, tile=TILE, pool=POOL):
+    xp, valid = O.pad_to_tiles(x, tile)
+    vm = O.permute_to_cube_major(valid[..., None].astype(np.float64), tile, pool)[:, 0] > 0
+    return O.permute_to_cube_major(xp, tile, pool), vm, xp.shape[:3]
+
+
+def test_padded_functions_equal_the_unpadded_ones_on_divisible_grids():
+    grid, d, topk = (8, 8, 12), 8, 3
+    xq, xk, xv = (_raster_inputs(grid, d, s) for s in (61, 62, 63))
+    g = np.random.default_rng(64).standard_normal(grid)
+    q, k, v = (S.raster_to_cube_major(x, TILE, POOL) for x in (xq, xk, xv))
+    valid = np.ones(q.shape[0], bool)
+    sc = O.router_scores(q, k)
+    np.testing.assert_allclose(O.router_scores_padded(q, k, valid), sc, rtol=1e-12, atol=1e-15)
+    sel = O.topk_select(sc.astype(np.float32), topk)
+    o_f, _ = O.sparse_attn_fwd(q, k, v, sel["kv_off"], sel["kv_idx"])
+    np.testing.assert_allclose(O.sparse_attn_fwd_padded(q, k, v, sel["kv_off"], sel["kv_idx"], valid), o_f,
+                               rtol=1e-12, atol=1e-14)
+    o_c, _ = O.coarse_attn(q, k, v)
+    np.testing.assert_allclose(O.coarse_attn_padded(q, k, v, valid), o_c, rtol=1e-12, atol=1e-14)
+    o_all, _ = O.vsa2_forward_padded(xq, xk, xv, g, topk)
+    want = O.gated_merge(o_f, o_c, S.raster_to_cube_major(g[..., None], TILE, POOL)[:, 0])
+    np.testing.assert_allclose(o_all, S.cube_major_to_raster(want, grid, TILE, POOL), rtol=1e-12, atol=1e-14)
+
+
+def test_padding_values_change_no_real_output():
+    """Fill the padding with large values instead of zeros: every output on real tokens is
+    bit-identical, so the padding is masked everywhere (pooling, router softmax, both branches)."""
+    grid, d = (6, 7, 10), 8
+    rng = np.random.default_rng(65)
+    x = {n: _raster_inputs(grid, d, s) for n, s in zip("qkv", (66, 67, 68))}
+    cm = {n: _padded_cube_major(x[n]) for n in "qkv"}
+    q, vm, grid_p = cm["q"]
+    k, v = cm["k"][0], cm["v"][0]
+    noisy = {n: np.where(vm[:, None], a, 50.0 * rng.standard_normal(a.shape)) for n, a in (("q", q), ("k", k), ("v", v))}
+    sc = O.router_scores_padded(q, k, vm)
+    np.testing.assert_array_equal(O.router_scores_padded(noisy["q"], noisy["k"], vm), sc)
+    np.testing.assert_allclose(sc.sum(axis=1), 1.0, rtol=1e-12)
+    sel = O.topk_select(sc.astype(np.float32), 4)
+    o = O.sparse_attn_fwd_padded(q, k, v, sel["kv_off"], sel["kv_idx"], vm)
+    o2 = O.sparse_attn_fwd_padded(noisy["q"], noisy["k"], noisy["v"], sel["kv_off"], sel["kv_idx"], vm)
+    np.testing.assert_array_equal(o2[vm], o[vm])
+    np.testing.assert_array_equal(O.coarse_attn_padded(noisy["q"], noisy["k"], noisy["v"], vm),
+                                  O.coarse_attn_padded(q, k, v, vm))
+
+
+def test_padded_full_budget_fine_branch_is_dense_attention_over_real_tokens():
+    grid, d = (5, 6, 9), 8
+    x = {n: _raster_inputs(grid, d, s) for n, s in zip("qkv", (69, 70, 71))}
+    (q, vm, grid_p), (k, _, _), (v, _, _) = (_padded_cube_major(x[n]) for n in "qkv")
+    N = q.shape[0] // 64
+    sel = O.topk_select(np.ones((N, N), np.float32), N)  # every tile pair
+    o = O.sparse_attn_fwd_padded(q, k, v, sel["kv_off"], sel["kv_idx"], vm)
+    got = O.permute_to_raster(o, grid_p)[:grid[0], :grid[1], :grid[2]].reshape(-1, d)
+    tq, tk, tv = (torch.from_numpy(x[n].reshape(-1, d))[None, None] for n in "qkv")
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv)[0, 0].numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
+
+
+def _router_padded_bruteforce(xq, xk, grid):
+    """Eq. 5-7 with padding on the raster grid, explicit loops: pad to whole 4x4x4 tiles; each
+    2x2x4 sub-cube's pooled vectors average its real tokens; sub-cubes without one are skipped
+    as queries and keys; the score of tile pair (i, j) is the mean over i's real query
+    sub-cubes of the softmax mass on j's sub-cubes."""
+    T, H, W = grid
+    D = xq.shape[-1]
+    nt, nh, nw = -(-T // 4), -(-H // 4), -(-W // 4)
+    subs = []
+    for a, b, c in itertools.product(range(nt), range(nh), range(nw)):
+        tile = (a * nh + b) * nw + c
+        for st, sh in itertools.product(range(2), range(2)):
+            qs, ks, n = np.zeros(D), np.zeros(D), 0
+            for dt, dh, dw in itertools.product(range(2), range(2), range(4)):
+                t, h, w = 4 * a + 2 * st + dt, 4 * b + 2 * sh + dh, 4 * c + dw
+                if t < T and h < H and w < W:
+                    qs += xq[t, h, w]
+                    ks += xk[t, h, w]
+                    n += 1
+            if n:
+                subs.append((tile, qs / n, ks / n))
+    N = nt * nh * nw
+    out = np.zeros((N, N))
+    g = np.zeros(N)
+    for ti, qa, _ in subs:
+        g[ti] += 1
+        logits = [float(qa @ kb) / math.sqrt(D) for _, _, kb in subs]
+        m = max(logits)
+        ex = [math.exp(z - m) for z in logits]
+        z = sum(ex)
+        for (tj, _, _), e in zip(subs, ex):
+            out[ti, tj] += e / z
+    return out / g[:, None]
+
+
+def _coarse_padded_bruteforce(xq, xk, xv, grid):
+    T, H, W = grid
+    D = xq.shape[-1]
+    nt, nh, nw = -(-T // 4), -(-H // 4), -(-W // 4)
+    means = {n: [] for n in "qkv"}
+    for a, b, c in itertools.product(range(nt), range(nh), range(nw)):
+        for n, x in zip("qkv", (xq, xk, xv)):
+            acc, cnt = np.zeros(D), 0
+            for dt, dh, dw in itertools.product(range(4), repeat=3):
+                t, h, w = 4 * a + dt, 4 * b + dh, 4 * c + dw
+                if t < T and h < H and w < W:
+                    acc += x[t, h, w]
+                    cnt += 1
+            means[n].append(acc / cnt)
+    out = []
+    for qi in means["q"]:
+        logits = [float(qi @ kj) / math.sqrt(D) for kj in means["k"]]
+        m = max(logits)
+        ex = [math.exp(z - m) for z in logits]
+        out.append(sum(e * vj for e, vj in zip(ex, means["v"])) / sum(ex))
+    return np.array(out)
+
+
+@pytest.mark.parametrize("grid", [(6, 7, 10), (5, 8, 5)])
+def test_router_and_coarse_padded_match_bruteforce_on_raster_grid(grid):
+    d = 8
+    xq, xk, xv = (_raster_inputs(grid, d, s) for s in (72, 73, 74))
+    (q, vm, _), (k, _, _), (v, _, _) = (_padded_cube_major(x) for x in (xq, xk, xv))
+    np.testing.assert_allclose(O.router_scores_padded(q, k, vm), _router_padded_bruteforce(xq, xk, grid),
+                               rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(O.coarse_attn_padded(q, k, v, vm), _coarse_padded_bruteforce(xq, xk, xv, grid),
+                               rtol=1e-12, atol=1e-14)
