@@ -32,6 +32,7 @@ __all__ = [
     "router_scores",
     "router_scores_dense_attention",
     "topk_select",
+    "topk_select_per_row",
     "sparse_attn_fwd",
     "sparse_attn_bwd",
     "coarse_attn",
@@ -132,6 +133,28 @@ def topk_select(scores: np.ndarray, topk: int) -> dict:
     ccounts = mask.sum(axis=0)
     q_off = np.zeros(N + 1, dtype=np.int32)
     q_off[1:] = np.cumsum(ccounts)
+    q_idx = np.nonzero(mask.T)[1].astype(np.int32)
+    return {"mask": mask, "kv_off": kv_off, "kv_idx": kv_idx, "q_off": q_off, "q_idx": q_idx}
+
+
+def topk_select_per_row(scores: np.ndarray, topk: int) -> dict:
+    """The per-query-tile TopK of VSA, the variant §2.2 contrasts with Eq. 8-9: every query tile
+    keeps its own `topk` best KV tiles, so each row has exactly `topk` entries. Ranked in fp32,
+    descending; equal scores go to the lower KV tile. Same output format as `topk_select`."""
+    s = np.asarray(scores)
+    if s.dtype != np.float32:
+        raise TypeError("rank in fp32: pass float32 scores")
+    N = s.shape[0]
+    if s.shape != (N, N) or not (1 <= topk <= N):
+        raise ValueError("need square scores and 1 <= topk <= N")
+    mask = np.zeros((N, N), dtype=bool)
+    for i in range(N):
+        order = np.lexsort((np.arange(N), -s[i].astype(np.float64)))
+        mask[i, order[:topk]] = True
+    kv_off = np.arange(N + 1, dtype=np.int32) * topk
+    kv_idx = np.nonzero(mask)[1].astype(np.int32)
+    q_off = np.zeros(N + 1, dtype=np.int32)
+    q_off[1:] = np.cumsum(mask.sum(axis=0))
     q_idx = np.nonzero(mask.T)[1].astype(np.int32)
     return {"mask": mask, "kv_off": kv_off, "kv_idx": kv_idx, "q_off": q_off, "q_idx": q_idx}
 

@@ -744,3 +744,41 @@ def test_router_and_coarse_padded_match_bruteforce_on_raster_grid(grid):
                                rtol=1e-12, atol=1e-15)
     np.testing.assert_allclose(O.coarse_attn_padded(q, k, v, vm), _coarse_padded_bruteforce(xq, xk, xv, grid),
                                rtol=1e-12, atol=1e-14)
+
+
+# --------------------------------------------------------------------------------------------
+# per-query-tile TopK (VSA's selection, the variant of §2.2)
+# --------------------------------------------------------------------------------------------
+
+def test_topk_per_row_bruteforce_with_ties():
+    rng = np.random.default_rng(81)
+    N, K = 9, 4
+    s = (rng.integers(0, 4, (N, N)) / 4).astype(np.float32)  # heavy ties
+    sel = O.topk_select_per_row(s, K)
+    for i in range(N):
+        want = sorted(sorted(range(N), key=lambda j: (-float(s[i, j]), j))[:K])
+        assert list(sel["kv_idx"][sel["kv_off"][i]:sel["kv_off"][i + 1]]) == want
+    assert np.all(sel["mask"].sum(axis=1) == K)
+    # the CSC lists the same pairs, column by column
+    for j in range(N):
+        assert list(sel["q_idx"][sel["q_off"][j]:sel["q_off"][j + 1]]) == list(np.nonzero(sel["mask"][:, j])[0])
+
+
+def test_topk_per_row_separable_scores_closed_form():
+    """Scores f(i) + g(j): every row ranks the KV tiles by g alone, so all rows keep the K tiles
+    of largest g."""
+    rng = np.random.default_rng(82)
+    N, K = 12, 5
+    f, g = rng.standard_normal(N), rng.permutation(N).astype(np.float64)
+    s = (f[:, None] + g[None, :]).astype(np.float32)  # g's gaps of 1 survive fp32 rounding
+    sel = O.topk_select_per_row(s, K)
+    best = np.sort(np.argsort(-g)[:K])
+    for i in range(N):
+        np.testing.assert_array_equal(sel["kv_idx"][i * K:(i + 1) * K], best)
+
+
+def test_topk_per_row_full_budget_equals_per_sequence():
+    s = np.random.default_rng(83).random((7, 7)).astype(np.float32)
+    a, b = O.topk_select_per_row(s, 7), O.topk_select(s, 7)
+    for key in ("kv_off", "kv_idx", "q_off", "q_idx"):
+        np.testing.assert_array_equal(a[key], b[key])
