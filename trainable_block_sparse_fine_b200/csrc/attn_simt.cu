@@ -1,7 +1,8 @@
 // CUDA-core block-sparse attention (Eq. 12 of "Improving Video Sparse Attention with
 // Fine-grained Router and Sparse Rebasing"; §2.1 definition) for the shapes the tensor-core
 // kernels do not take: fp32 inputs and head_dim 64, plus the backward pass.
-// Arithmetic is fp32 throughout.
+// Arithmetic is fp32 throughout. The forward treats keys at or beyond `kv_valid` tokens of a
+// head as padding (the coarse branch's pooled sequence, Eq. 1-3, ends in a partial tile).
 #include "common.cuh"
 #include "internal.h"
 
