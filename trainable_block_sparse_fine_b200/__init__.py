@@ -17,7 +17,9 @@ from ._capi import (VSA2_FLAG_VALIDATE, Problem, Vsa2Error, lib, make_problem, v
                     vsa2_selftest_wait_timeout, vsa2_sparse_attn_bwd, vsa2_sparse_attn_fwd, vsa2_status_string,
                     vsa2_topk_select, vsa2_version, vsa2_workspace_init, vsa2_workspace_size)
 
-__all__ = ["VSA2", "Vsa2Error", "Problem", "make_problem", "block_sparse_attention", "lib", "VSA2_FLAG_VALIDATE",
+from .ulysses import heads_to_seq, seq_to_heads, ulysses_attention
+
+__all__ = ["VSA2", "ulysses_attention", "seq_to_heads", "heads_to_seq", "Vsa2Error", "Problem", "make_problem", "block_sparse_attention", "lib", "VSA2_FLAG_VALIDATE",
            "vsa2_router_scores", "vsa2_topk_select", "vsa2_sparse_attn_fwd", "vsa2_sparse_attn_bwd",
            "vsa2_workspace_size", "vsa2_workspace_init", "vsa2_get_device_error", "vsa2_selftest_wait_timeout",
            "vsa2_status_string", "vsa2_version", "vsa2_forward_host", "vsa2_forward_host_workspace_size",
