@@ -115,7 +115,7 @@ def test_gated_merge_matches_oracle(dtype, in_place):
     o_f = S.round_to_dtype(rng.standard_normal((wl.batch, wl.heads, L, D)).astype(np.float32), dtype)
     oc = S.round_to_dtype(rng.standard_normal((wl.batch, wl.heads, N, D)).astype(np.float32), dtype)
     logits = (rng.standard_normal((wl.batch, wl.heads, L)) * 2).astype(np.float32)
-    logits[0, 0, :64] = 0.0  # tanh(0) = 0: these rows are the fine output alone
+    logits[0, 0, :64] = 0.0  # tanh(0) = 0: the fine output alone, as with W_g = 0 at the start (§2.3)
     e = _engine(wl)
     o_f_d = _dev(o_f, dtype)
     out = e.gated_merge(o_f_d, torch.from_numpy(logits).cuda(), _dev(oc, dtype), out=o_f_d if in_place else None)

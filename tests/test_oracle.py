@@ -496,7 +496,8 @@ def test_gated_merge_closed_forms():
     L, D = 3 * 64, 4
     o_f = rng.standard_normal((L, D))
     o_c_hat = rng.standard_normal((3, D))
-    # G = tanh(0) = 0: the fine branch alone
+    # G = tanh(0) = 0: the fine branch alone. §2.3 (Sparse Rebasing) relies on this: W_g starts
+    # at zero, so a model switched to VSA2 outputs only O_f at first.
     np.testing.assert_array_equal(O.gated_merge(o_f, o_c_hat, np.zeros(L)), o_f)
     # saturated gates: tanh(+-40) rounds to +-1 in fp64
     sign = np.where(np.arange(L) % 2 == 0, 1.0, -1.0)
