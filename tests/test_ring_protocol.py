@@ -1,5 +1,5 @@
-"""A model of the forward kernel's per-slot pipeline and its mbarriers, run under random
-schedules on the CPU.
+"""Models of the forward kernel's per-slot pipeline and of the dK/dV kernel's pipeline, with
+their mbarriers, run under random schedules on the CPU.
 
 An mbarrier parity wait can only tell the phase in progress from the one just completed: a
 waiter two phases behind waits forever, and a waiter one phase ahead passes early. The model
@@ -13,7 +13,8 @@ finishes (no deadlock). The agents follow the kernel's protocol:
   * the softmax waits for S, frees its buffer, then waits for the previous P.V before writing P.
 The kernel's variant is one producer per slot and a 3-block ring holding K and V in op order.
 The model also covers the planned split with two producers (one per d-half, the full barrier
-expecting two arrivals).
+expecting two arrivals). Besides the barrier rules it asserts the data hazards the barriers
+exist for: a ring block, an S buffer or P is overwritten only after its last reader finished.
 """
 import random
 
@@ -61,6 +62,9 @@ def run(tiles, rst, producers, rng, mma_latency=3):
     prod = [0] * producers            # next ring position per producer
     mma = {"c": 0, "s": 0, "o": 0}    # next op; S and O ops issued
     soft = {"blk": 0, "step": 0}      # next block; 0: wait S, 1: wait previous P.V, then write P
+    op_done = set()                   # ring positions whose MMA has completed
+    s_read = set()                    # S blocks the softmax has read
+    o_done = set()                    # P.V blocks completed
     nblk = sum(tiles)
     pending = []                      # (time, callback): MMA completions
     t = 0
@@ -72,6 +76,7 @@ def run(tiles, rst, producers, rng, mma_latency=3):
         st = c % rst
         if not empty[st].poll(c // rst - 1, f"producer {p} at {c}"):
             return False
+        assert c < rst or c - rst in op_done, f"ring position {c} refilled before its MMA finished"
         full[st].arrive()
         prod[p] += 1
         return True
@@ -88,13 +93,14 @@ def run(tiles, rst, producers, rng, mma_latency=3):
             k = mma["s"]
             if not sfree[k % 2].poll(k // 2 - 1, f"issuer S{k}"):
                 return False
-            done = [empty[st].arrive, sfull[k % 2].arrive]
+            assert k < 2 or k - 2 in s_read, f"S buffer of block {k} overwritten before it was read"
+            done = [lambda c=c: op_done.add(c), empty[st].arrive, sfull[k % 2].arrive]
             mma["s"] += 1
         else:
             k = mma["o"]
             if not pfull.poll(k, f"issuer O{k}"):
                 return False
-            done = [empty[st].arrive, pvdone.arrive]
+            done = [lambda c=c, k=k: (op_done.add(c), o_done.add(k)), empty[st].arrive, pvdone.arrive]
             mma["o"] += 1
         pending.append((t + rng.randint(1, mma_latency), done))
         mma["c"] += 1
@@ -107,16 +113,19 @@ def run(tiles, rst, producers, rng, mma_latency=3):
         if soft["step"] == 0:
             if not sfull[g % 2].poll(g // 2, f"softmax S{g}"):
                 return False
+            s_read.add(g)
             sfree[g % 2].arrive()
             soft["step"] = 1
             return True
         if g > 0 and not pvdone.poll(g - 1, f"softmax P{g}"):
             return False
+        assert g == 0 or g - 1 in o_done, f"P of block {g} written while P.V of block {g - 1} reads P"
         pfull.arrive()
         soft["blk"], soft["step"] = g + 1, 0
         return True
 
     agents = [lambda p=p: producer(p) for p in range(producers)] + [issuer, softmax]
+    speed = [rng.uniform(0.05, 1.0) for _ in agents]  # skewed speeds expose races
     while mma["c"] < len(ops) or soft["blk"] < nblk or pending:
         t += 1
         due = [x for x in pending if x[0] <= t]
@@ -125,9 +134,9 @@ def run(tiles, rst, producers, rng, mma_latency=3):
             for f in done:
                 f()
         moved = bool(due)
-        for a in rng.sample(agents, len(agents)):
-            if rng.random() < 0.7:
-                moved |= a()
+        for i in rng.sample(range(len(agents)), len(agents)):
+            if rng.random() < speed[i]:
+                moved |= agents[i]()
         assert moved or pending or t < 10_000_000, "deadlock"
         if not moved and not pending and not any(a() for a in agents):
             raise AssertionError(f"deadlock at op {mma['c']} of {len(ops)}, softmax block {soft['blk']}")
@@ -135,7 +144,7 @@ def run(tiles, rst, producers, rng, mma_latency=3):
 
 
 @pytest.mark.parametrize("producers", [1, 2], ids=["kernel", "two_producers"])
-@pytest.mark.parametrize("seed", range(30))
+@pytest.mark.parametrize("seed", range(60))
 def test_ring_protocol_parity_and_progress(producers, seed):
     rng = random.Random(seed)
     tiles = [rng.choice([1, 1, 2, 3, 4, 5, 7, 32]) for _ in range(rng.randint(1, 6))]
@@ -145,3 +154,142 @@ def test_ring_protocol_parity_and_progress(producers, seed):
 def test_op_order_matches_the_kernel_stream():
     assert ops_of([3]) == [("S", 0), ("S", 1), ("O", 0), ("S", 2), ("O", 1), ("O", 2)]
     assert ops_of([1, 2]) == [("S", 0), ("O", 0), ("S", 0), ("S", 1), ("O", 0), ("O", 1)]
+
+
+def run_dkdv(items, rng, rst=6, mma_latency=3):
+    """The dK/dV kernel's protocol: per KV tile (item) of n selecting query tiles, op t loads the
+    tile's Q / dO stage (producer of the position's parity), the first issuer runs S^T / dP^T
+    into the single S buffer, the softmax reads it and writes P / dS into buffer t % 2, the
+    second issuer runs dV / dK from that buffer and releases the stage; after the item's last op
+    the epilogue waits for every MMA, then the next item's K / V rows go to tensor memory. A KV
+    tile that no query tile selected touches no barrier; the per-item phases count non-empty
+    items only, as the kernel's do. Data hazards asserted: a stage is refilled only after both
+    MMAs and the softmax have read it; S only after the softmax read it; a P / dS buffer only
+    after the second MMA two ops back; the K / V rows only after the previous item's MMAs; the
+    accumulators are restarted only after the previous item's epilogue."""
+    total = sum(items)
+    full = [Barrier(1) for _ in range(rst)]
+    empty = [Barrier(1) for _ in range(rst)]
+    spfull, spfree = Barrier(1), Barrier(1)
+    pdsfull, pdsfree = [Barrier(1), Barrier(1)], [Barrier(1), Barrier(1)]
+    itemdone, kvready = Barrier(1), Barrier(1)
+    last_of_item = set()
+    n = 0
+    for k in items:
+        n += k
+        last_of_item.add(n - 1)
+    nonempty = [i for i, k in enumerate(items) if k]
+    item_of = [j for j, i in enumerate(nonempty) for _ in range(items[i])]  # non-empty index per op
+    prod = [0, 1]                   # producer p fills positions p, p + 2, ...
+    a = {"n": 0}
+    b = {"n": 0}
+    soft = {"item": 0, "it": 0, "n": 0, "step": "kv"}  # item, non-empty items done, op, stage
+    a_done, b_done, s_read = set(), set(), set()  # completed first / second MMAs, S blocks read
+    epi_done = set()                              # non-empty items whose epilogue has run
+    first_op = {sum(items[i] for i in nonempty[:j]): j for j in range(len(nonempty))}
+    pending = []
+    t = 0
+
+    def producer(p):
+        pos = prod[p]
+        if pos >= total:
+            return False
+        st = pos % rst
+        if not empty[st].poll(pos // rst - 1, f"producer {p} at {pos}"):
+            return False
+        old = pos - rst
+        assert old < 0 or (old in a_done and old in b_done and old in s_read), f"stage refilled at {pos}"
+        full[st].arrive()
+        prod[p] += 2
+        return True
+
+    def issuer_a():
+        c = a["n"]
+        if c >= total:
+            return False
+        first_of_item = c == 0 or (c - 1) in last_of_item
+        if first_of_item and not kvready.poll(item_of[c], f"issuer A kv {c}"):
+            return False
+        if c > 0 and not spfree.poll(c - 1, f"issuer A S {c}"):
+            return False
+        if not full[c % rst].poll(c // rst, f"issuer A stage {c}"):
+            return False
+        assert c == 0 or c - 1 in s_read, f"S of op {c} overwrites S of op {c - 1} before it was read"
+        pending.append((t + rng.randint(1, mma_latency), [lambda c=c: a_done.add(c), spfull.arrive]))
+        a["n"] += 1
+        return True
+
+    def issuer_b():
+        c = b["n"]
+        if c >= total:
+            return False
+        if not pdsfull[c & 1].poll(c >> 1, f"issuer B {c}"):
+            return False
+        if c in first_op and first_op[c] > 0:
+            assert first_op[c] - 1 in epi_done, f"accumulators restarted at op {c} before the epilogue read them"
+        done = [lambda c=c: b_done.add(c), empty[c % rst].arrive, pdsfree[c & 1].arrive]
+        if c in last_of_item:
+            done.append(itemdone.arrive)
+        pending.append((t + rng.randint(1, mma_latency), done))
+        b["n"] += 1
+        return True
+
+    def softmax():
+        if soft["item"] >= len(items):
+            return False
+        c = soft["n"]
+        if soft["step"] == "kv":  # K / V rows of the item into tensor memory
+            if items[soft["item"]] == 0:  # zero gradients, no barrier
+                soft["item"] += 1
+                return True
+            prev = [c2 for c2 in range(c) if item_of[c2] == soft["it"] - 1]
+            assert all(c2 in a_done for c2 in prev), "K / V rows overwritten under the previous item's MMAs"
+            kvready.arrive()
+            soft["step"] = "s"
+            return True
+        if soft["step"] == "s":
+            if not spfull.poll(c, f"softmax S {c}") or not full[c % rst].poll(c // rst, f"softmax stage {c}"):
+                return False
+            s_read.add(c)
+            spfree.arrive()
+            soft["step"] = "p"
+            return True
+        if soft["step"] == "p":
+            if c >= 2 and not pdsfree[c & 1].poll((c >> 1) - 1, f"softmax P {c}"):
+                return False
+            assert c < 2 or c - 2 in b_done, f"P / dS buffer of op {c} written under the MMA of op {c - 2}"
+            pdsfull[c & 1].arrive()
+            soft["n"] += 1
+            soft["step"] = "epi" if c in last_of_item else "s"
+            return True
+        if not itemdone.poll(soft["it"], f"epilogue {soft['item']}"):
+            return False
+        epi_done.add(soft["it"])
+        soft["item"] += 1
+        soft["it"] += 1
+        soft["step"] = "kv"
+        return True
+
+    agents = [lambda: producer(0), lambda: producer(1), issuer_a, issuer_b, softmax]
+    speed = [rng.uniform(0.05, 1.0) for _ in agents]
+    while soft["item"] < len(items) or pending:
+        t += 1
+        due = [x for x in pending if x[0] <= t]
+        pending[:] = [x for x in pending if x[0] > t]
+        for _, done in due:
+            for f in done:
+                f()
+        moved = bool(due)
+        for i in rng.sample(range(len(agents)), len(agents)):
+            if rng.random() < speed[i]:
+                moved |= agents[i]()
+        if not moved and not pending and not any(ag() for ag in agents):
+            raise AssertionError(f"deadlock: issuer A {a['n']}, B {b['n']}, softmax {soft} of {total}")
+    assert b["n"] == total and itemdone.phases == len(nonempty)
+
+
+@pytest.mark.parametrize("seed", range(60))
+def test_dkdv_protocol_parity_and_progress(seed):
+    rng = random.Random(1000 + seed)
+    items = [rng.choice([0, 1, 2, 3, 5, 8, 13, 64]) for _ in range(rng.randint(1, 6))]
+    run_dkdv(items, rng, mma_latency=rng.choice([1, 3, 10]))
