@@ -1,5 +1,5 @@
-"""Models of the forward kernel's per-slot pipeline and of the dK/dV kernel's pipeline, with
-their mbarriers, run under random schedules on the CPU.
+"""Models of the tensor-core kernels' pipelines (forward, dQ and dK/dV) with their mbarriers,
+run under random schedules on the CPU.
 
 An mbarrier parity wait can only tell the phase in progress from the one just completed: a
 waiter two phases behind waits forever, and a waiter one phase ahead passes early. The model
@@ -293,3 +293,134 @@ def test_dkdv_protocol_parity_and_progress(seed):
     rng = random.Random(1000 + seed)
     items = [rng.choice([0, 1, 2, 3, 5, 8, 13, 64]) for _ in range(rng.randint(1, 6))]
     run_dkdv(items, rng, mma_latency=rng.choice([1, 3, 10]))
+
+
+def run_dq(items, rng, unified, mma_latency=3):
+    """The dQ kernel's per-slot protocol: per block n of a query tile, op A(n) runs S = Q K^T
+    and dP = dO V^T from block n's K and V, after B(n-1) has finished reading dS (which
+    overwrote S); the softmax turns S, dP into dS; op B(n) runs dQ += dS K from the same K block
+    and releases it. Op order A0, B0, A1, B1, ... As built, K blocks have a ring of 2 and V
+    blocks a ring of 1, V released by A, K by B. With `unified`, K(n), V(n) share one ring of 3
+    in load order (the change made in the forward kernel), so a stage's releases must still
+    arrive in position order."""
+    nblk = sum(items)
+    nonempty = [k for k in items if k]
+    item_start = set()
+    acc = 0
+    for k in nonempty:
+        item_start.add(acc)
+        acc += k
+    if unified:
+        rings = {"kv": [Barrier(1) for _ in range(3)]}
+        emp = {"kv": [Barrier(1) for _ in range(3)]}
+        slot = lambda kind, n: ("kv", 2 * n + (kind == "V"), 3)
+    else:
+        rings = {"K": [Barrier(1) for _ in range(2)], "V": [Barrier(1)]}
+        emp = {"K": [Barrier(1) for _ in range(2)], "V": [Barrier(1)]}
+        slot = lambda kind, n: (kind, n, 2 if kind == "K" else 1)
+    sfull, dsfull, bdone, qready = Barrier(1), Barrier(1), Barrier(1), Barrier(1)
+    loads = [(kind, n) for n in range(nblk) for kind in ("K", "V")]
+    prod = {"i": 0}
+    iss = {"a": 0, "b": 0}
+    soft = {"n": 0, "it": 0, "step": "q"}
+    a_done, b_done, ds_written, epi_done = set(), set(), set(), set()
+    pending = []
+    t = 0
+
+    def producer():
+        if prod["i"] >= len(loads):
+            return False
+        kind, n = loads[prod["i"]]
+        ring, pos, rst = slot(kind, n)
+        if not emp[ring][pos % rst].poll(pos // rst - 1, f"producer {kind}{n}"):
+            return False
+        # the previous occupant of this stage has been released by its last reader
+        if pos >= rst:
+            prev_pos = pos - rst
+            if unified:
+                pk, pn = ("V" if prev_pos % 2 else "K"), prev_pos // 2
+            else:
+                pk, pn = kind, prev_pos
+            assert (pn in b_done) if pk == "K" else (pn in a_done), f"{kind}{n} loaded over {pk}{pn}"
+        rings[ring][pos % rst].arrive()
+        prod["i"] += 1
+        return True
+
+    def issuer():
+        a, b = iss["a"], iss["b"]
+        if b >= nblk:
+            return False
+        if a == b:  # A(a)
+            if a in item_start and not qready.poll(sorted(item_start).index(a), f"A{a} Q"):
+                return False
+            if a > 0 and not bdone.poll(a - 1, f"A{a} bdone"):
+                return False
+            rk, pk, sk = slot("K", a)
+            rv, pv, sv = slot("V", a)
+            if not rings[rk][pk % sk].poll(pk // sk, f"A{a} K") or not rings[rv][pv % sv].poll(pv // sv, f"A{a} V"):
+                return False
+            assert a == 0 or a - 1 in b_done, f"S/dP of block {a} overwrite dS of block {a - 1} under its MMA"
+            done = [lambda a=a: a_done.add(a), emp[rv][pv % sv].arrive, sfull.arrive]
+            pending.append((t + rng.randint(1, mma_latency), done))
+            iss["a"] += 1
+            return True
+        if not dsfull.poll(b, f"B{b}"):
+            return False
+        assert b in ds_written
+        if b in item_start and sorted(item_start).index(b) > 0:
+            assert sorted(item_start).index(b) - 1 in epi_done, f"dQ restarted at block {b} before the epilogue"
+        rk, pk, sk = slot("K", b)
+        done = [lambda b=b: b_done.add(b), emp[rk][pk % sk].arrive, bdone.arrive]
+        pending.append((t + rng.randint(1, mma_latency), done))
+        iss["b"] += 1
+        return True
+
+    def softmax():
+        if soft["it"] >= len(nonempty):
+            return False
+        n = soft["n"]
+        if soft["step"] == "q":  # Q and dO rows of the item into tensor memory
+            assert all(m in a_done for m in range(n)), "Q / dO overwritten under the previous item's MMAs"
+            qready.arrive()
+            soft["step"] = "s"
+            return True
+        if soft["step"] == "s":
+            if not sfull.poll(n, f"softmax S{n}"):
+                return False
+            ds_written.add(n)
+            dsfull.arrive()
+            soft["n"] += 1
+            end = soft["n"] == sum(nonempty[:soft["it"] + 1])
+            soft["step"] = "epi" if end else "s"
+            return True
+        if not bdone.poll(n - 1, f"epilogue {soft['it']}"):
+            return False
+        epi_done.add(soft["it"])
+        soft["it"] += 1
+        soft["step"] = "q"
+        return True
+
+    agents = [producer, issuer, softmax]
+    speed = [rng.uniform(0.05, 1.0) for _ in agents]
+    while soft["it"] < len(nonempty) or pending:
+        t += 1
+        due = [x for x in pending if x[0] <= t]
+        pending[:] = [x for x in pending if x[0] > t]
+        for _, done in due:
+            for f in done:
+                f()
+        moved = bool(due)
+        for i in rng.sample(range(len(agents)), len(agents)):
+            if rng.random() < speed[i]:
+                moved |= agents[i]()
+        if not moved and not pending and not any(ag() for ag in agents):
+            raise AssertionError(f"deadlock: A {iss['a']}, B {iss['b']}, softmax {soft} of {nblk}")
+    assert len(b_done) == nblk
+
+
+@pytest.mark.parametrize("unified", [False, True], ids=["kernel", "one_ring"])
+@pytest.mark.parametrize("seed", range(60))
+def test_dq_protocol_parity_and_progress(unified, seed):
+    rng = random.Random(2000 + seed)
+    items = [rng.choice([0, 1, 2, 3, 5, 8, 32]) for _ in range(rng.randint(1, 6))]
+    run_dq(items, rng, unified, mma_latency=rng.choice([1, 3, 10]))
