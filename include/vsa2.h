@@ -110,6 +110,17 @@ vsa2_status vsa2_topk_select(const vsa2_problem* p, const float* scores, int32_t
                              void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Per-query-tile TopK: the selection of VSA that §2.2 contrasts with Eq. 8-9 (§2.1
+ * Background, TopK(Q_c K_c^T) row by row). Every query tile keeps its own topk largest scores,
+ * so each row holds exactly topk KV tiles; equal scores within a row go to the lower KV tile.
+ * Arguments, output format and errors as for vsa2_topk_select (kv_off[.,.,i] = i*topk). The
+ * CSR feeds vsa2_sparse_attn_fwd / _bwd unchanged.
+ */
+vsa2_status vsa2_topk_select_per_row(const vsa2_problem* p, const float* scores, int32_t topk,
+                                     int32_t* kv_off, int32_t* kv_idx, int32_t* q_off, int32_t* q_idx,
+                                     void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Block-sparse attention forward, Eq. 12 with the §2.1 definition. For every query token t
  * of tile i: o_t = sum_u softmax_u(q_t . k_u / sqrt(D)) v_u over the tokens u of the KV tiles
  * listed for tile i; lse_t = ln sum_u exp(q_t . k_u / sqrt(D)). A tile with an empty list

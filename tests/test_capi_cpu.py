@@ -72,6 +72,9 @@ def test_argument_errors_are_synchronous():
     assert lib.vsa2_topk_select(bp, fake, 33, fake, fake, None, None, ws, n, None) == 2
     # CSC pointers must come as a pair
     assert lib.vsa2_topk_select(bp, fake, 8, fake, fake, fake, None, ws, n, None) == 1
+    assert lib.vsa2_topk_select_per_row(bp, fake, 8, fake, fake, fake, None, ws, n, None) == 1
+    assert lib.vsa2_topk_select_per_row(bp, fake, 0, fake, fake, None, None, ws, n, None) == 2
+    assert lib.vsa2_topk_select_per_row(bp, fake, 8, fake, fake, None, None, ws, n - 256, None) == 1
     assert lib.vsa2_sparse_attn_fwd(bp, fake, fake, fake, 8, fake, None, fake, fake, ws, n, None) == 1
     assert lib.vsa2_sparse_attn_bwd(bp, fake, fake, fake, fake, fake, fake, 8, fake, fake, None, fake, fake, fake,
                                     fake, ws, n, None) == 1

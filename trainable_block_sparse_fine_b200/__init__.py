@@ -15,7 +15,7 @@ from ._capi import (VSA2_FLAG_VALIDATE, Problem, Vsa2Error, lib, make_problem, v
                     vsa2_coarse_attn_bwd, vsa2_forward_host, vsa2_forward_host_workspace_size, vsa2_gated_merge,
                     vsa2_gated_merge_bwd, vsa2_get_device_error, vsa2_permute_tokens, vsa2_router_scores,
                     vsa2_selftest_wait_timeout, vsa2_sparse_attn_bwd, vsa2_sparse_attn_fwd, vsa2_status_string,
-                    vsa2_topk_select, vsa2_version, vsa2_workspace_init, vsa2_workspace_size)
+                    vsa2_topk_select, vsa2_topk_select_per_row, vsa2_version, vsa2_workspace_init, vsa2_workspace_size)
 
 from .ulysses import heads_to_seq, seq_to_heads, ulysses_attention
 
@@ -63,6 +63,18 @@ class VSA2:
         q_off = torch.empty(*bh, self.N + 1, **i32) if csc else None
         q_idx = torch.empty(*bh, self.N * topk, **i32) if csc else None
         vsa2_topk_select(self.p, scores, topk, kv_off, kv_idx, q_off, q_idx, self.ws)
+        return kv_off, kv_idx, q_off, q_idx
+
+    def topk_select_per_row(self, scores, topk=None, csc=True):
+        """VSA's per-query-tile TopK: every query tile keeps its own `topk` best KV tiles."""
+        topk = self.topk if topk is None else topk
+        bh = (self.batch, self.heads)
+        i32 = dict(dtype=torch.int32, device=self.device)
+        kv_off = torch.empty(*bh, self.N + 1, **i32)
+        kv_idx = torch.empty(*bh, self.N * topk, **i32)
+        q_off = torch.empty(*bh, self.N + 1, **i32) if csc else None
+        q_idx = torch.empty(*bh, self.N * topk, **i32) if csc else None
+        vsa2_topk_select_per_row(self.p, scores, topk, kv_off, kv_idx, q_off, q_idx, self.ws)
         return kv_off, kv_idx, q_off, q_idx
 
     def attn_fwd(self, q, k, v, kv_off, kv_idx, topk=None, o=None, lse=None):

@@ -22,7 +22,7 @@ EXPORTS = ("vsa2_workspace_size", "vsa2_workspace_init", "vsa2_router_scores", "
            "vsa2_selftest_wait_timeout", "vsa2_status_string", "vsa2_version", "vsa2_last_cuda_error",
            "vsa2_topk_select_noalloc", "vsa2_forward_host", "vsa2_forward_host_workspace_size",
            "vsa2_coarse_attn", "vsa2_gated_merge", "vsa2_gated_merge_bwd", "vsa2_coarse_attn_bwd",
-           "vsa2_permute_tokens")
+           "vsa2_permute_tokens", "vsa2_topk_select_per_row")
 
 
 class Vsa2Error(RuntimeError):
@@ -60,6 +60,7 @@ def lib() -> ctypes.CDLL:
         L.vsa2_sparse_attn_fwd.argtypes = [P, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]
         L.vsa2_sparse_attn_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.vsa2_topk_select_noalloc.argtypes = [P, vp, i32, vp, vp, vp]
+        L.vsa2_topk_select_per_row.argtypes = [P, vp, i32, vp, vp, vp, vp, vp, sz, vp]
         L.vsa2_forward_host_workspace_size.argtypes = [P, i32, i32]
         L.vsa2_forward_host_workspace_size.restype = sz
         L.vsa2_forward_host.argtypes = [P, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
@@ -75,6 +76,7 @@ def lib() -> ctypes.CDLL:
         L.vsa2_version.restype = i32
         L.vsa2_last_cuda_error.restype = ctypes.c_char_p
         for name in ("vsa2_workspace_init", "vsa2_router_scores", "vsa2_topk_select", "vsa2_topk_select_noalloc",
+                     "vsa2_topk_select_per_row",
                      "vsa2_sparse_attn_fwd", "vsa2_forward_host", "vsa2_coarse_attn", "vsa2_gated_merge",
                      "vsa2_gated_merge_bwd", "vsa2_coarse_attn_bwd", "vsa2_permute_tokens",
                      "vsa2_sparse_attn_bwd", "vsa2_get_device_error", "vsa2_selftest_wait_timeout"):
@@ -131,6 +133,12 @@ def vsa2_topk_select(p: Problem, scores, topk, kv_off, kv_idx, q_off, q_idx, ws,
     _check(lib().vsa2_topk_select(ctypes.byref(p), _ptr(scores), topk, _ptr(kv_off), _ptr(kv_idx), _ptr(q_off),
                                   _ptr(q_idx), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "vsa2_topk_select")
+
+
+def vsa2_topk_select_per_row(p: Problem, scores, topk, kv_off, kv_idx, q_off, q_idx, ws, stream=None) -> None:
+    _check(lib().vsa2_topk_select_per_row(ctypes.byref(p), _ptr(scores), topk, _ptr(kv_off), _ptr(kv_idx),
+                                          _ptr(q_off), _ptr(q_idx), _ptr(ws), ws.numel() * ws.element_size(),
+                                          _stream(stream)), "vsa2_topk_select_per_row")
 
 
 def vsa2_topk_select_noalloc(p: Problem, scores, topk, kv_off, kv_idx, stream=None) -> None:

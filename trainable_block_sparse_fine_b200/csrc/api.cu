@@ -93,6 +93,32 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
+// Unique id of the CUDA context current on this thread (cuCtxGetId), so that state a library
+// call keeps per device (a device address, streams, events) can tell a context that replaced
+// an earlier one on the same device, for example after cudaDeviceReset.
+bool current_context_id(unsigned long long* id) {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess && cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) ==
+                                                 cudaSuccess &&
+        qb == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<GetCurrent>(a);
+      get_id = reinterpret_cast<GetId>(b);
+    }
+  });
+  CUcontext c = nullptr;
+  if (!get_current || !get_id || get_current(&c) != CUDA_SUCCESS || !c) return false;
+  return get_id(c, id) == CUDA_SUCCESS;
+}
+
 static thread_local int g_encode_result = 0;
 
 // The encoder is a driver call: make the current device's primary context current on this
@@ -208,6 +234,19 @@ vsa2_status vsa2_topk_select(const vsa2_problem* p, const float* scores, int32_t
   if (!aligned16(scores)) return VSA2_ERR_INVALID_ARG;
   if ((st = check_ws(d, ws, ws_bytes)) != VSA2_OK) return st;
   return launch_topk(d, scores, topk, kv_off, kv_idx, q_off, q_idx, (char*)ws, (cudaStream_t)stream);
+}
+
+vsa2_status vsa2_topk_select_per_row(const vsa2_problem* p, const float* scores, int32_t topk, int32_t* kv_off,
+                                     int32_t* kv_idx, int32_t* q_off, int32_t* q_idx, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  Dims d;
+  vsa2_status st = make_dims(p, &d);
+  if (st != VSA2_OK) return st;
+  if (!scores || !kv_off || !kv_idx) return VSA2_ERR_INVALID_ARG;
+  if ((q_off == nullptr) != (q_idx == nullptr)) return VSA2_ERR_INVALID_ARG;
+  if (topk < 1 || topk > d.N) return VSA2_ERR_UNSUPPORTED;
+  if ((st = check_ws(d, ws, ws_bytes)) != VSA2_OK) return st;
+  return launch_topk_per_row(d, scores, topk, kv_off, kv_idx, q_off, q_idx, (char*)ws, (cudaStream_t)stream);
 }
 
 vsa2_status vsa2_sparse_attn_fwd(const vsa2_problem* p, const void* q, const void* k, const void* v, int32_t topk,

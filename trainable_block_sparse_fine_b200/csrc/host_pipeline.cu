@@ -25,6 +25,7 @@ constexpr int64_t kAutoChunkTokens = 65536;  // automatic group size: at least t
 
 struct Pipe {
   bool ready = false;
+  unsigned long long ctx_id = 0;  // context the streams and events were created in
   cudaStream_t in = nullptr, out = nullptr;
   cudaEvent_t fork = nullptr, join_in = nullptr, join_out = nullptr;
   cudaEvent_t in_ready[kSlots] = {}, comp_done[kSlots] = {}, out_done[kSlots] = {};
@@ -33,11 +34,15 @@ struct Pipe {
 std::mutex g_pipe_mu;
 Pipe g_pipes[kMaxDevices];
 
-// Streams and events of the current device, created on first use and kept for the process.
+// Streams and events of the current device, created on first use and kept for the process;
+// created again if the device's context has been replaced since (the old handles died with it).
 vsa2_status get_pipe(Pipe** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cuda_fail("cudaGetDevice");
-  Pipe& p = g_pipes[dev];
+  if (cudaSetDevice(dev) != cudaSuccess) return cuda_fail("cudaSetDevice");
+  Pipe& p = g_pipes[dev];  // the caller holds g_pipe_mu
+  unsigned long long id = 0;
+  if (current_context_id(&id) && p.ready && p.ctx_id != id) p = Pipe{};
   if (!p.ready) {
     const unsigned ef = cudaEventDisableTiming;
     bool ok = cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking) == cudaSuccess &&
@@ -51,6 +56,7 @@ vsa2_status get_pipe(Pipe** out) {
            cudaEventCreateWithFlags(&p.out_done[s], ef) == cudaSuccess;
     if (!ok) return cuda_fail("creating the copy streams and events of vsa2_forward_host");
     p.ready = true;
+    p.ctx_id = id;
   }
   *out = &p;
   return VSA2_OK;

@@ -61,6 +61,8 @@ bool make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64
 vsa2_status launch_router(const Dims& d, const void* q, const void* k, float* scores, char* ws, cudaStream_t s);
 vsa2_status launch_topk(const Dims& d, const float* scores, int topk, int32_t* kv_off, int32_t* kv_idx,
                         int32_t* q_off, int32_t* q_idx, char* ws, cudaStream_t s);
+vsa2_status launch_topk_per_row(const Dims& d, const float* scores, int topk, int32_t* kv_off, int32_t* kv_idx,
+                                int32_t* q_off, int32_t* q_idx, char* ws, cudaStream_t s);
 vsa2_status launch_attn_fwd(const Dims& d, const void* q, const void* k, const void* v, int topk,
                             const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
                             cudaStream_t s);
@@ -110,6 +112,10 @@ vsa2_status launch_topk_noalloc(const Dims& d, const float* scores, int topk, in
                                 cudaStream_t s);
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Unique id of the CUDA context current on this thread; false if it cannot be read. Call after
+// a runtime call that binds the device's primary context (cudaGetDevice + cudaSetDevice).
+bool current_context_id(unsigned long long* id);
 
 // Records the message of a failed CUDA call (see vsa2_last_cuda_error) and returns VSA2_ERR_CUDA.
 vsa2_status cuda_fail(const char* what);

@@ -334,7 +334,130 @@ __global__ void __launch_bounds__(256) topk_csc_emit_kernel(int N, int topk, con
   }
 }
 
+// Exclusive scan over a 256-thread block; returns this thread's exclusive prefix, *total the sum.
+__device__ __forceinline__ uint32_t block_scan_excl_256(uint32_t v, uint32_t* sh8, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh8[warp] = x;
+  __syncthreads();
+  uint32_t base = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    const uint32_t c = sh8[w];
+    base += w < warp ? c : 0u;
+    tot += c;
+  }
+  __syncthreads();
+  *total = tot;
+  return base + x - v;
+}
+
+// Per-query-tile TopK (VSA's selection, the variant that Eq. 8-9 replace): one 256-thread CTA
+// per row keeps the row's `topk` largest scores. Exact radix select over the row's fp32 bit
+// patterns in three passes (11/11/10 bits); equal scores go to the lower KV tile. The row is
+// read from global memory on every pass (it stays in L1: N*4 bytes). Writes the row's CSR
+// entries in ascending j and, with col_cnt, marks the CSC bitmap like topk_emit_kernel.
+__global__ void __launch_bounds__(256) topk_row_select_kernel(const float* __restrict__ scores, int N, int topk,
+                                                              int32_t* __restrict__ kv_off,
+                                                              int32_t* __restrict__ kv_idx,
+                                                              int32_t* __restrict__ col_cnt,
+                                                              uint32_t* __restrict__ col_bits, int words) {
+  __shared__ uint32_t h[2048];
+  __shared__ uint32_t sh8[8];
+  __shared__ uint32_t s_prefix, s_remain;
+  const int bh = blockIdx.y, row = blockIdx.x, t = threadIdx.x;
+  const float* s = scores + ((size_t)bh * N + row) * N;
+  uint32_t prefix = 0, remain = (uint32_t)topk;
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    for (int b = t; b < 2048; b += 256) h[b] = 0;
+    __syncthreads();
+    for (int j = t; j < N; j += 256) {
+      const uint32_t key = score_key(__ldg(s + j));
+      if (pass == 0) atomicAdd(&h[key >> 21], 1u);
+      else if (pass == 1) {
+        if ((key >> 21) == prefix) atomicAdd(&h[(key >> 10) & 2047u], 1u);
+      } else if ((key >> 10) == prefix) {
+        atomicAdd(&h[key & 1023u], 1u);
+      }
+    }
+    __syncthreads();
+    // descending bins: thread t owns bins NB-1-PER*t-e, e < PER
+    const int NB = pass == 2 ? 1024 : 2048, PER = NB / 256, BITS = pass == 2 ? 10 : 11;
+    uint32_t c[8], mine = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      c[e] = e < PER ? h[NB - 1 - (PER * t + e)] : 0u;
+      mine += c[e];
+    }
+    uint32_t tot;
+    uint32_t above = block_scan_excl_256(mine, sh8, &tot);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (e < PER && above < remain && above + c[e] >= remain) {
+        s_prefix = (prefix << BITS) | (uint32_t)(NB - 1 - (PER * t + e));
+        s_remain = remain - above;
+      }
+      above += c[e];
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    remain = s_remain;
+    __syncthreads();
+  }
+  const uint32_t T = prefix, ties = remain;  // threshold key; entries equal to it still taken
+  int32_t* out = kv_idx + (size_t)bh * N * topk + (size_t)row * topk;
+  uint32_t written = 0, ties_seen = 0;
+  for (int j0 = 0; j0 < N; j0 += 256) {
+    const int j = j0 + t;
+    const uint32_t key = j < N ? score_key(__ldg(s + j)) : 0u;
+    const bool is_eq = j < N && key == T;
+    uint32_t eq_tot, sel_tot;
+    const uint32_t rank = ties_seen + block_scan_excl_256(is_eq, sh8, &eq_tot);
+    const bool sel = j < N && (key > T || (is_eq && rank < ties));
+    const uint32_t pos = written + block_scan_excl_256(sel, sh8, &sel_tot);
+    if (sel) {
+      if (pos < (uint32_t)topk) out[pos] = j;
+      if (col_cnt) {
+        atomicAdd(&col_cnt[(size_t)bh * N + j], 1);
+        atomicOr(&col_bits[((size_t)bh * N + j) * words + (row >> 5)], 1u << (row & 31));
+      }
+    }
+    written += sel_tot;
+    ties_seen += eq_tot;
+  }
+  if (t == 0) {
+    kv_off[(size_t)bh * (N + 1) + row] = row * topk;
+    if (row == N - 1) kv_off[(size_t)bh * (N + 1) + N] = N * topk;
+  }
+}
+
 }  // namespace
+
+vsa2_status launch_topk_per_row(const Dims& d, const float* scores, int topk, int32_t* kv_off, int32_t* kv_idx,
+                                int32_t* q_off, int32_t* q_idx, char* ws, cudaStream_t s) {
+  const WsLayout w = ws_layout(d);
+  int32_t* col_cnt = reinterpret_cast<int32_t*>(ws + w.col_cnt);
+  uint32_t* col_bits = reinterpret_cast<uint32_t*>(ws + w.col_bits);
+  const bool csc = q_off != nullptr;
+  if (csc) {
+    if (cudaMemsetAsync(col_cnt, 0, (size_t)d.BH * d.N * 4, s) != cudaSuccess) return VSA2_ERR_CUDA;
+    if (cudaMemsetAsync(col_bits, 0, (size_t)d.BH * d.N * w.words * 4, s) != cudaSuccess) return VSA2_ERR_CUDA;
+  }
+  topk_row_select_kernel<<<dim3(d.N, d.BH), 256, 0, s>>>(scores, d.N, topk, kv_off, kv_idx, csc ? col_cnt : nullptr,
+                                                         col_bits, w.words);
+  if (csc) {
+    dim3 rgrid((d.N + 7) / 8, d.BH);
+    topk_csc_offsets_kernel<<<d.BH, 1024, 0, s>>>(d.N, col_cnt, q_off);
+    topk_csc_emit_kernel<<<rgrid, 256, 0, s>>>(d.N, topk, col_bits, w.words, q_off, q_idx);
+  }
+  return check_launch(__func__);
+}
 
 vsa2_status launch_topk(const Dims& d, const float* scores, int topk, int32_t* kv_off, int32_t* kv_idx,
                         int32_t* q_off, int32_t* q_idx, char* ws, cudaStream_t s) {
@@ -410,22 +533,34 @@ NoAllocLayout noalloc_layout(const Dims& d) {
 }
 
 std::mutex g_scratch_mu;
-void* g_scratch_ptr[64] = {};  // device address of g_topk_scratch, per device ordinal
+struct ScratchSlot {
+  unsigned long long ctx_id;  // context the address belongs to (0: unknown)
+  void* ptr;                  // device address of g_topk_scratch in that context
+};
+ScratchSlot g_scratch[64] = {};  // per device ordinal
 
-// Device address of the scratch array for the current device, looked up once per device
-// (cudaGetSymbolAddress with that device current; the host-side symbol is not a device address).
+// Device address of the scratch array for the current device, looked up with that device
+// current (cudaGetSymbolAddress; the host-side symbol is not a device address). The address is
+// kept per device and per context: a context that replaced the one it was taken in (after
+// cudaDeviceReset, say) gets a fresh lookup. If the context id cannot be read, every call looks
+// the address up again.
 vsa2_status noalloc_scratch(char** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice failed");
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess)
+    return cuda_fail("cudaGetDevice failed");
   if (dev < 0 || dev >= 64) return cuda_fail("device ordinal out of range for the TopK scratch table");
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id);
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  ScratchSlot& slot = g_scratch[dev];
+  if (!have_id || !slot.ptr || slot.ctx_id != id) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_topk_scratch) != cudaSuccess || !ptr)
       return cuda_fail("cudaGetSymbolAddress of the TopK scratch array failed");
-    g_scratch_ptr[dev] = ptr;
+    slot.ptr = ptr;
+    slot.ctx_id = have_id ? id : 0;
   }
-  *out = static_cast<char*>(g_scratch_ptr[dev]);
+  *out = static_cast<char*>(slot.ptr);
   return VSA2_OK;
 }
 }  // namespace
