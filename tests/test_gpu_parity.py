@@ -229,6 +229,50 @@ def test_topk_odd_tile_count():
     _topk_case(wl, rng.random((1, 3, 45, 45)).astype(np.float32))
 
 
+def _topk_per_row_case(wl, scores32, topk):
+    e = engine(wl)
+    got = e.topk_select_per_row(torch.from_numpy(scores32).cuda(), topk, csc=True)
+    assert e.device_error() == 0
+    for b in range(wl.batch):
+        for h in range(wl.heads):
+            want = O.topk_select_per_row(scores32[b, h], topk)
+            for name, g in zip(("kv_off", "kv_idx", "q_off", "q_idx"), got):
+                assert np.array_equal(g[b, h].cpu().numpy(), want[name]), (name, b, h)
+
+
+@pytest.mark.parametrize("wl", [TINY, SMALL, C480], ids=["tiny", "small", "480p"])
+def test_topk_per_row_bit_exact_on_oracle_scores(wl):
+    """VSA's per-query-tile TopK on the oracle's fp32 router scores: CSR and CSC bit-exact."""
+    x = inputs(wl, ("q", "k"))
+    heads = None if wl is not C480 else [0, 5, 19]
+    sc = oracle_scores(wl, x, heads)
+    s32 = np.random.default_rng(9).random((wl.batch, wl.heads, wl.num_tiles, wl.num_tiles), dtype=np.float32)
+    for (b, h), v in sc.items():
+        s32[b, h] = v.astype(np.float32)
+    _topk_per_row_case(wl, s32, wl.topk)
+
+
+@pytest.mark.parametrize("topk", [1, 7, 45])
+def test_topk_per_row_ties_and_extremes(topk):
+    """Heavy ties (equal scores go to the lower KV tile), topk 1 and topk = N, N = 45 (not a
+    multiple of the 256-column chunk or of 4)."""
+    wl = S.Workload("odd", 1, 3, 64, (12, 12, 20), topk, "bf16")  # N = 45
+    rng = np.random.default_rng(topk)
+    s = (rng.integers(0, 5, (1, 3, 45, 45)) / 8.0).astype(np.float32)
+    s[0, 2] = 0.5  # a head of equal scores: every row keeps its first topk columns
+    _topk_per_row_case(wl, s, topk)
+
+
+def test_fwd_on_per_row_selection():
+    """The forward takes VSA's per-query-tile CSR unchanged."""
+    wl = SMALL
+    x = inputs(wl)
+    e = engine(wl)
+    sc = e.router_scores(dev(x["q"], "bf16"), dev(x["k"], "bf16"))
+    kv_off, kv_idx, _, _ = e.topk_select_per_row(sc, wl.topk, csc=False)
+    _fwd_case(wl, x, kv_off.cpu().numpy(), kv_idx.cpu().numpy())
+
+
 def test_topk_on_gpu_scores_is_valid_within_score_error():
     wl = C480
     x = inputs(wl, ("q", "k"))
@@ -347,6 +391,14 @@ def test_fwd_480p_sampled_heads():
     _fwd_case(wl, inputs(wl), kv_off, kv_idx, heads=heads, tiles=[0, 1, 100, 363, 364, 727])
 
 
+def test_fwd_480p_full_head():
+    """480p top64 in the benchmark's launch configuration (20 heads): head 0 runs on the oracle's
+    selection and every one of its 728 query tiles is compared."""
+    wl = C480
+    kv_off, kv_idx, _, _ = lists_from_masks(c480_lists([0]), wl.topk)
+    _fwd_case(wl, inputs(wl), kv_off, kv_idx, heads=[0])
+
+
 def test_480p_top128_topk_bit_exact_and_forward_sampled():
     """480p with top128 (93,184 selected pairs per head): TopK on the oracle's fp32 scores of all
     20 heads is bit-exact, CSR and CSC, and the forward on that selection matches the oracle on
@@ -432,6 +484,27 @@ def test_bwd_480p_sampled():
     lists = lists_from_masks(c480_lists(heads), wl.topk)
     _bwd_case(wl, inputs(wl, ("q", "k", "v", "do")), lists, heads=heads, q_tiles=[0, 363, 727],
               kv_tiles=[0, 364, 727])
+
+
+def test_bwd_480p_full_head_from_own_forward():
+    """The 480p top64 training step as it runs: the backward takes the forward output (bf16) and
+    LSE that the GPU forward stored, and every row of dQ, dK and dV of head 0 (oracle selection)
+    is compared with the oracle's exact gradient, which recomputes O in fp64 (no stored O)."""
+    wl = C480
+    x = inputs(wl, ("q", "k", "v", "do"))
+    kv_off, kv_idx, q_off, q_idx = lists_from_masks(c480_lists([0]), wl.topk)
+    e = engine(wl)
+    q, k, v, do = (dev(x[n], wl.dtype) for n in ("q", "k", "v", "do"))
+    t = lambda a: torch.from_numpy(a).cuda()
+    o, lse = e.attn_fwd(q, k, v, t(kv_off), t(kv_idx))
+    dq, dk, dv = e.attn_bwd(q, k, v, o, lse, do, t(kv_off), t(kv_idx), t(q_off), t(q_idx))
+    assert e.device_error() == 0
+    want = O.sparse_attn_bwd(x["q"][0, 0], x["k"][0, 0], x["v"][0, 0], x["do"][0, 0], kv_off[0, 0], kv_idx[0, 0])
+    for name, g, w in zip(("dq", "dk", "dv"), (dq, dk, dv), want):
+        g = g[0, 0].cpu().numpy().astype(np.float64)
+        rel = np.linalg.norm(g - w) / np.linalg.norm(w)
+        print(f"480p head 0 {name}: max abs {np.abs(g - w).max():.3e}, rel L2 {rel:.3e}")
+        assert_attn_close(g, w, f"{name}[0,0]")
 
 
 def test_autograd_function_matches_explicit_calls():
