@@ -130,8 +130,7 @@ __device__ __forceinline__ int next_op(SlotSeq& q, int* blk, const int32_t* kv_o
 template <bool kPad>
 __global__ void __launch_bounds__(FT, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                       const __nv_bfloat16* __restrict__ qg, const __nv_bfloat16* __restrict__ kg,
-                       const __nv_bfloat16* __restrict__ vg, const int32_t* __restrict__ kv_off,
+                       const __nv_bfloat16* __restrict__ qg, const int32_t* __restrict__ kv_off,
                        const int32_t* __restrict__ kv_idx, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
                        int N, int L, int topk, int items, float c2, int kv_valid, DevCtx ctx) {
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
@@ -295,24 +294,6 @@ __global__ void __launch_bounds__(FT, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&B.qready[s]);
       }
-      {
-        // Ask L2 for the K and V tiles and the Q tile of this slot's next item now, one item
-        // ahead of its TMA loads: a head's K and V do not stay in L2 whole at large L, and the
-        // ring alone cannot cover a DRAM miss.
-        const int nitem = item + step;
-        if (nitem < items) {
-          const int nbh = nitem / N, nqt = nitem - nbh * N;
-          const Row nr = load_row(kv_off, nbh, nqt, N, cap, ctx, false);
-          const int t = 32 * w + lane;
-          const size_t head = (size_t)nbh * L;
-          if (t == 0) bulk_prefetch_l2(qg + (head + (size_t)nqt * 64) * 128, TILE_B * 2);
-          for (int e = t; e < nr.len; e += 128) {
-            const int j = min(max(__ldg(kv_idx + (size_t)nbh * cap + nr.beg + e), 0), N - 1);
-            bulk_prefetch_l2(kg + (head + (size_t)j * 64) * 128, TILE_B * 2);
-            bulk_prefetch_l2(vg + (head + (size_t)j * 64) * 128, TILE_B * 2);
-          }
-        }
-      }
       float m = -INFINITY, l = 0.f;
       for (int n = 0; n < nblk; ++n, ++g) {
         const bool half = (2 * n + 1 == rw.len);
@@ -444,8 +425,7 @@ vsa2_status launch_fwd_tc(const Dims& d, const void* q, const void* k, const voi
   const int grid = std::max(1, std::min(sms, (items + 1) / 2));
   const float c2 = 1.4426950408889634f / sqrtf(128.f);
   cudaFuncSetAttribute(attn_fwd_tc_kernel<kPad>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
-  attn_fwd_tc_kernel<kPad><<<grid, FT, SMEM_DYN, s>>>(tk, tv, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                                                      (const __nv_bfloat16*)v, kv_off, kv_idx,
+  attn_fwd_tc_kernel<kPad><<<grid, FT, SMEM_DYN, s>>>(tk, tv, (const __nv_bfloat16*)q, kv_off, kv_idx,
                                                       (__nv_bfloat16*)o, lse, d.N, (int)d.L, topk, items, c2,
                                                       kv_valid, ctx);
   return check_launch("attn_fwd_tc");
