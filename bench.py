@@ -1,15 +1,19 @@
 """Benchmark of the VSA2 hot path on B200: router -> per-sequence TopK -> block-sparse attention.
 
-One step = one pass of the whole path over one batch of synthetic input of the 720p workload
-(B=1, H=20, D=128, grid 56x48x80 = 215,040 tokens, 3360 tiles, top64, bf16): router pooling,
-router scores, TopK, attention forward. With --workload 480p_train_top64 the step also runs the
-backward pass (training step of the fine branch; the router gets no gradient).
+One step = one pass of the whole path over one batch of synthetic input: router pooling, router
+scores, TopK, attention forward, and for the training workload the backward pass too (the
+router gets no gradient). The configurations, each printed as one JSON line by rank 0:
+  tiny              B=1, H=2, D=64, grid 8x16x16, top8, fp32 (forward)
+  480p_top64        B=1, H=20, D=128, grid 28x32x52, top64, bf16 (forward)
+  480p_top128       the same tensors, top128
+  480p_train_top64  the same tensors, top64, forward + backward
+  720p_top64        B=1, H=20, D=128, grid 56x48x80 (215,040 tokens, 3360 tiles), top64, bf16
+                    (forward): the headline, printed last, with a digest of all lines.
+`value` is the effective TFLOPS of the whole step: FLOPs of the selected tile pairs only
+(4*64*64*D per pair forward, 2.5x that backward) over the step time, summed over ranks, divided
+by the max step time over ranks. `roofline.frac` is against the measured burst bf16 peak.
 
-Prints one JSON line (rank 0). `value` is the effective TFLOPS of the whole step: FLOPs of the
-selected tile pairs only (4*64*64*D per pair forward, 2.5x that backward) over the step time,
-summed over ranks, divided by the max step time over ranks.
-
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME|all]
 """
 from __future__ import annotations
 
@@ -32,9 +36,19 @@ sys.path.insert(0, ROOT)
 import synthetic as S  # noqa: E402
 
 METRIC = "VSA2 attn fwd ms & effective TFLOPS, 215K tok H20 D128 top64"
-DEFAULT_WORKLOAD = "720p_top64"
+HEADLINE = "720p_top64"
+# every configuration of the benchmark, in the order they run; the headline prints last
+ALL_WORKLOADS = ["tiny", "480p_top64", "480p_top128", "480p_train_top64", HEADLINE]
 # kernels of ours launched per call (memsets are not counted)
 LAUNCHES = {"router": 2, "topk": 9, "topk_csc": 11, "fwd": 1, "bwd": 2}
+
+
+def load_sm_max_mhz():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f).get("sm_max_mhz", 1965.0))
+    except Exception:
+        return 1965.0
 
 
 def load_peaks():
@@ -54,15 +68,15 @@ TRAFFIC_PROFILES = {
 }
 
 
-def profiled_traffic(kind, wl, pairs):
+def profiled_traffic(kind, wl, pairs, root=ROOT):
     """DRAM bytes of one launch from the committed ncu summary, scaled by selected pairs; None
     when the kernel source changed since the counters were taken or for other workloads."""
     name, kernel_src, grid = TRAFFIC_PROFILES[kind]
     if wl.grid != grid or wl.head_dim != 128 or wl.topk != 64:
         return None
     try:
-        txt = open(os.path.join(ROOT, "profiles", name)).read()
-        src = open(os.path.join(ROOT, "trainable_block_sparse_fine_b200", "csrc", kernel_src), "rb").read()
+        txt = open(os.path.join(root, "profiles", name)).read()
+        src = open(os.path.join(root, "trainable_block_sparse_fine_b200", "csrc", kernel_src), "rb").read()
     except OSError:
         return None
     per = re.search(r"dram_bytes_per_pair:\s*(\d+)", txt)
@@ -182,22 +196,25 @@ class Clocks:
 # ----------------------------------------------------------------------------------------------
 def oracle_sample(wl, budget_s=20.0, tiles=None):
     """Time the oracle's hot path on head 0 of batch 0: router + TopK on the whole head, the
-    forward (and backward) on a sample of query tiles; extrapolate to all tiles and heads."""
+    forward (and backward) on a sample of query tiles; extrapolate to all tiles and heads.
+    Returns the extrapolated step time and the seconds the sample actually took."""
     from oracle import vsa2_oracle as O
 
     q, k, v = (S.make_slice(wl, n, 0, 0) for n in ("q", "k", "v"))
+    do = S.make_slice(wl, "do", 0, 0) if wl.backward else None
     t0 = time.perf_counter()
     sc = O.router_scores(q, k).astype(np.float32)
     t1 = time.perf_counter()
     sel = O.topk_select(sc, wl.topk)
     t2 = time.perf_counter()
     N = wl.num_tiles
-    rng = np.random.default_rng(0)
-    order = rng.permutation(N)
+    order = np.random.default_rng(0).permutation(N)
     done, t_att = 0, 0.0
     for i in order:
         ts = time.perf_counter()
         O.sparse_attn_fwd(q, k, v, sel["kv_off"], sel["kv_idx"], query_tiles=[int(i)])
+        if wl.backward:
+            O.sparse_attn_bwd(q, k, v, do, sel["kv_off"], sel["kv_idx"], query_tiles=[int(i)])
         t_att += time.perf_counter() - ts
         done += 1
         if tiles is not None and done >= tiles:
@@ -205,15 +222,14 @@ def oracle_sample(wl, budget_s=20.0, tiles=None):
         if tiles is None and (t2 - t0) + t_att > budget_s:
             break
     per_head = (t1 - t0) + (t2 - t1) + t_att * N / done
-    if wl.backward:
-        per_head += 2.5 * t_att * N / done  # backward restated as 2.5x the forward GEMM work
     total_s = per_head * wl.heads * wl.batch
     pairs = wl.batch * wl.heads * N * wl.topk
     flops = pair_flops(wl, pairs, wl.backward)
+    what = "forward and backward" if wl.backward else "forward"
     return {"seconds_per_step": total_s, "tflops": flops / total_s / 1e12, "router_s": t1 - t0, "topk_s": t2 - t1,
-            "fwd_tiles_sampled": done, "tiles": N,
-            "sample": f"head 0 of {wl.heads}: router+TopK whole head, forward on {done}/{N} query tiles; "
-                      f"extrapolated to {wl.heads} heads"}
+            "sample_s": (t2 - t0) + t_att, "fwd_tiles_sampled": done, "tiles": N,
+            "sample": f"head 0 of {wl.heads}: router+TopK whole head, {what} on {done}/{N} query tiles; "
+                      f"step time extrapolated to all tiles and {wl.heads} heads"}
 
 
 def cores():
@@ -221,6 +237,10 @@ def cores():
 
 
 def run_reference(args, wl):
+    """The reference arm: the fp64 oracle, as it stands, on this host's cores. Each step is a
+    bounded sample (router and TopK of one head, the attention of 8 of its query tiles);
+    `ms_per_step` is the time that sample took, `value` the whole step's effective TFLOPS
+    extrapolated from it."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -230,13 +250,15 @@ def run_reference(args, wl):
     for _ in range(args.steps):
         steps.append(oracle_sample(wl, tiles=8))
     sec = statistics.mean(s["seconds_per_step"] for s in steps)
+    sample_ms = statistics.mean(s["sample_s"] for s in steps) * 1e3
     pairs = wl.batch * wl.heads * wl.num_tiles * wl.topk
     val = pair_flops(wl, pairs, wl.backward) / sec / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOPS", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sample_ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": wl.name, "batch": wl.batch, "heads": wl.heads, "head_dim": wl.head_dim,
                        "grid": list(wl.grid), "tokens": wl.tokens, "topk": wl.topk},
+            "extrapolated_ms_per_full_step": sec * 1e3,
             "cpu_baseline": {"value": val, "unit": "TFLOPS", "cores": cores(), "kind": "oracle",
                              "sample": steps[-1]["sample"]},
             "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -330,7 +352,7 @@ def time_next_rows(e, x, wl, steps, stream, l2_flush, ev, hbm, tc_peak):
     m_bytes = 2 * B * H * L * D * esize + B * H * L * 4 + B * H * N * D * esize
     return {
         "coarse_attn": {"ms": c_ms, "effective_tflops": c_flops / (c_ms * 1e-3) / 1e12,
-                        "frac_of_sustained_bf16": c_flops / (c_ms * 1e-3) / 1e12 / tc_peak,
+                        "frac_of_burst_bf16": c_flops / (c_ms * 1e-3) / 1e12 / tc_peak,
                         "pool_bytes": pool_bytes, "pool_floor_ms": pool_bytes / (hbm * 1e9) * 1e3,
                         "kernels": "coarse_pool_kernel + coarse_csr_kernel + attn_fwd_tc_kernel<true>"},
         "gated_merge": {"ms": m_ms, "algorithmic_bytes": m_bytes, "gbs": m_bytes / (m_ms * 1e-3) / 1e9,
@@ -339,34 +361,94 @@ def time_next_rows(e, x, wl, steps, stream, l2_flush, ev, hbm, tc_peak):
     }
 
 
-def run_ours(args, wl):
+def time_dense(x, wl, stream, l2_flush, ev, iters=2):
+    """Dense softmax attention over the same Q, K, V (every tile pair), the comparison the pages
+    make for their attention speed-up (paper §4, Fig. 8, against FlashAttention-3 on H800). Timed
+    with torch's scaled_dot_product_attention on each backend it offers for these tensors; the
+    fastest is reported. A library kernel, timed for context only: it is not part of the path."""
     import torch
-    import torch.distributed as dist
+    from torch.nn.attention import SDPBackend, sdpa_kernel
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    B, H, L, D = wl.batch, wl.heads, wl.tokens, wl.head_dim
+    flops = 4.0 * L * L * D * B * H
+    out = {}
+    for name, be in (("cudnn", SDPBackend.CUDNN_ATTENTION), ("flash", SDPBackend.FLASH_ATTENTION)):
+        try:
+            with sdpa_kernel([be]):
+                torch.nn.functional.scaled_dot_product_attention(x["q"], x["k"], x["v"])
+                torch.cuda.synchronize()
+                ts = []
+                for _ in range(iters):
+                    l2_flush.zero_()
+                    a, b = ev(), ev()
+                    a.record(stream)
+                    torch.nn.functional.scaled_dot_product_attention(x["q"], x["k"], x["v"])
+                    b.record(stream)
+                    torch.cuda.synchronize()
+                    ts.append(a.elapsed_time(b))
+            out[name] = statistics.mean(ts)
+        except Exception as exc:  # a backend that does not take these shapes on this build
+            out[name] = f"unavailable: {type(exc).__name__}"
+    times = {k: v for k, v in out.items() if isinstance(v, float)}
+    if not times:
+        return {"backends": out}
+    best = min(times, key=times.get)
+    return {"ms": times[best], "backend": f"torch sdpa ({best})", "backends": out,
+            "effective_tflops": flops / (times[best] * 1e-3) / 1e12, "flops": flops}
+
+
+_inputs_cache = {}
+
+
+def device_inputs(wl, names, rank, world, dev):
+    """Pinned host copies (the end-to-end leg copies them every step) and device copies of the
+    workload's tensors; workloads on the same grid and seed share them (480p top64, top128 and
+    the training step use the same Q, K, V)."""
+    import torch
+
+    key = (wl.grid, wl.dtype, wl.head_dim, wl.batch, wl.heads, wl.seed + rank)
+    have = _inputs_cache.get(key)
+    if have is None:
+        _inputs_cache.clear()
+        torch.cuda.empty_cache()
+        have = _inputs_cache[key] = ({}, {})
+    pinned, x = have
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    # each fp32 array is dropped once converted; the generator's worker pool is shared by the
+    # ranks of a node
+    workers = max(1, min(16, len(os.sched_getaffinity(0)) // max(1, int(os.environ.get("LOCAL_WORLD_SIZE", world)))))
+    wl_r = wl.with_(seed=wl.seed + rank)  # weak scaling: every rank its own batch element
+    for n in names:
+        if n not in pinned:
+            a32 = S.make_tensor(wl_r, n, workers=workers)
+            pinned[n] = torch.from_numpy(a32).to(dt).pin_memory()
+            del a32
+            x[n] = pinned[n].to(dev)
+    return pinned, x
+
+
+def fp32_fma_peak_tflops(sm_max_mhz):
+    """CUDA-core fp32 peak: 148 SMs x 128 FP32 lanes x 2 FLOP per FMA x the maximum SM clock."""
+    return 148 * 128 * 2 * sm_max_mhz * 1e6 / 1e12
+
+
+def mufu_peak(sm_max_mhz):
+    """ex2 rate of the SFU (MUFU) pipes: 16 per clock per SM (a probe measured this on B200) x 148
+    SMs x the maximum SM clock, in exponentials per second."""
+    return 16 * 148 * sm_max_mhz * 1e6
+
+
+def measure(args, wl, dev, rank, world):
+    """One workload: warm-up, K timed steps, the end-to-end leg, the next rows; returns the JSON
+    line (rank 0) or None."""
+    import torch
     import trainable_block_sparse_fine_b200 as V
     from trainable_block_sparse_fine_b200.sharding import max_over_ranks
+    import torch.distributed as dist
 
-    dev = torch.device("cuda", local)
-    # weak scaling: every rank runs the full workload on its own batch element (seed offset)
-    wl_r = wl.with_(seed=wl.seed + rank)
     names = ("q", "k", "v", "do") if wl.backward else ("q", "k", "v")
     dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
-    # inputs in pinned host memory (the end-to-end leg copies them every step); each fp32 array
-    # is dropped once converted, and the generator's worker pool is shared by the ranks of a node
-    workers = max(1, min(16, len(os.sched_getaffinity(0)) // max(1, int(os.environ.get("LOCAL_WORLD_SIZE", world)))))
-    pinned = {}
-    for n in names:
-        a32 = S.make_tensor(wl_r, n, workers=workers)
-        pinned[n] = torch.from_numpy(a32).to(dt).pin_memory()
-        del a32
-    x = {n: pinned[n].to(dev) for n in names}
+    pinned, x = device_inputs(wl, names, rank, world, dev)
     e = V.VSA2(wl.batch, wl.heads, wl.head_dim, wl.grid, wl.dtype, wl.topk)
     stream = torch.cuda.current_stream()
     l2_flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -401,7 +483,7 @@ def run_ours(args, wl):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with Clocks(local) as clk:
+    with Clocks(dev.index) as clk:
         for _ in range(args.steps):
             l2_flush.zero_()  # L2 flush between timed steps (outside the timed events)
             timers = {k: ev() for k in keys}
@@ -448,56 +530,116 @@ def run_ours(args, wl):
     e2e = max_over_ranks(statistics.mean(e2e_ms) if e2e_ms else float("nan"), dev)
 
     hbm, bf16_burst, bf16_sus, peak_kind = load_peaks()
+    sm_max = load_sm_max_mhz()
     next_rows = None
-    if not args.no_next:
-        next_rows = time_next_rows(e, x, wl, args.steps, stream, l2_flush, ev, hbm, bf16_sus)
+    if not args.no_next and wl.dtype == "bf16":
+        next_rows = time_next_rows(e, x, wl, args.steps, stream, l2_flush, ev, hbm, bf16_burst)
+        if wl.name == HEADLINE and not wl.backward:
+            dense = time_dense(x, wl, stream, l2_flush, ev)
+            if "ms" in dense:
+                # the pages' ratio covers every op of Fig. 2 but the QKV projections: coarse branch,
+                # router, TopK, fine branch and gated merge
+                vsa2_ms = statistics.mean(per["step"]) + next_rows["coarse_attn"]["ms"] + next_rows["gated_merge"]["ms"]
+                dense["vsa2_all_ops_ms"] = vsa2_ms
+                dense["speedup_all_ops"] = dense["ms"] / vsa2_ms
+                dense["speedup_fine_branch_step"] = dense["ms"] / statistics.mean(per["step"])
+            next_rows["dense_attention"] = dense
     fwd_ms = statistics.mean(per["fwd"])
     fwd_tflops = pair_flops(wl, pairs, False) / (fwd_ms * 1e-3) / 1e12
+    tc = wl.dtype == "bf16" and wl.head_dim == 128
     if wl.backward:  # the backward pass (dQ kernel + dK/dV kernel) dominates a training step
         bwd_ms = statistics.mean(per["bwd"])
         bwd_tflops = 2.5 * pair_flops(wl, pairs, False) / (bwd_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "kernel": "attn_bwd_dq_tc_kernel + attn_bwd_dkdv_tc_kernel (one call)",
                 "achieved": bwd_tflops, "traffic": profiled_traffic("bwd", wl, pairs)}
-    else:
+    elif tc:
         roof = {"bound": "tensor", "kernel": "attn_fwd_tc_kernel", "achieved": fwd_tflops,
                 "traffic": profiled_traffic("fwd", wl, pairs)}
+    else:  # fp32 / D=64: the CUDA-core forward
+        roof = {"bound": "alu", "kernel": "attn_fwd_simt_kernel", "achieved": fwd_tflops, "traffic": None}
+    if roof["bound"] == "tensor":
+        peak, kind = bf16_burst, f"{peak_kind} burst bf16 (dense, cuBLAS 8192^3)"
+        extra_peak = {"frac_of_sustained": roof["achieved"] / bf16_sus, "sustained_peak": bf16_sus}
+    else:
+        peak, kind = fp32_fma_peak_tflops(sm_max), f"derived fp32 FMA: 148 SMs x 128 lanes x 2 x {sm_max:.0f} MHz"
+        extra_peak = {"note": "launch-bound at this size"}
     router_ms = statistics.mean(per["router"])
-    router_bytes = 2 * wl.batch * wl.heads * wl.tokens * wl.head_dim * (2 if wl.dtype == "bf16" else 4) \
-        + wl.batch * wl.heads * wl.num_tiles ** 2 * 4
+    esize = 2 if wl.dtype == "bf16" else 4
+    router_bytes = 2 * wl.batch * wl.heads * wl.tokens * wl.head_dim * esize + wl.batch * wl.heads * wl.num_tiles ** 2 * 4
+    router_ex2 = 2.0 * wl.batch * wl.heads * (wl.tokens // 16) ** 2
     launches = LAUNCHES["router"] + (LAUNCHES["topk_csc"] if wl.backward else LAUNCHES["topk"]) + LAUNCHES["fwd"] \
         + (LAUNCHES["bwd"] if wl.backward else 0)
-    if rank == 0:
-        cpu = None
-        if world == 1 and not args.no_cpu_baseline:
-            c = oracle_sample(wl, budget_s=20.0)
-            cpu = {"value": c["tflops"], "unit": "TFLOPS", "cores": cores(), "kind": "oracle", "sample": c["sample"],
-                   "seconds_per_step": c["seconds_per_step"]}
-        line = {
-            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
-            "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "fp32", "data": "synthetic",
-            "config": {"workload": wl.name, "batch": wl.batch, "heads": wl.heads, "head_dim": wl.head_dim,
-                       "grid": list(wl.grid), "tokens": wl.tokens, "tiles": wl.num_tiles, "topk": wl.topk,
-                       "selected_pairs_per_rank": pairs, "backward": wl.backward,
-                       "l2": "256 MB buffer written between timed steps; inputs also exceed L2"},
-            "stages_ms": {"router": router_ms, "topk": statistics.mean(per["topk"]), "fwd": fwd_ms,
-                          **({"bwd": statistics.mean(per["bwd"])} if wl.backward else {})},
-            "fwd_kernel": {"ms": fwd_ms, "effective_tflops": fwd_tflops},
-            "router": {"ms": router_ms, "algorithmic_bytes": router_bytes,
-                       "gbs": router_bytes / (router_ms * 1e-3) / 1e9, "hbm_frac": router_bytes / (router_ms * 1e-3) / 1e9 / hbm},
-            **({"bwd_pass": {"ms": bwd_ms, "effective_tflops": bwd_tflops}} if wl.backward else {}),
-            "roofline": {"bound": roof["bound"], "kernel": roof["kernel"], "achieved": roof["achieved"],
-                         "peak": bf16_sus, "unit": "TFLOP/s", "frac": roof["achieved"] / bf16_sus,
-                         "peak_kind": f"{peak_kind} sustained bf16", "traffic": roof["traffic"]},
-            "cpu_baseline": cpu,
-            "e2e": {"value": flops_rank * world / (e2e * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "api": "VSA2.forward + attn_bwd after H2D copies" if wl.backward else "vsa2_forward_host"},
-            "gpu_launches": launches * args.steps,
-            "clocks": clk.summary(),
-            **({"next_rows": next_rows} if next_rows else {}),
-        }
-        print(json.dumps(line), flush=True)
+    if rank != 0:
+        return None
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        c = oracle_sample(wl, budget_s=args.cpu_budget if wl.name == HEADLINE else min(args.cpu_budget, 6.0))
+        cpu = {"value": c["tflops"], "unit": "TFLOPS", "cores": cores(), "kind": "oracle", "sample": c["sample"],
+               "seconds_per_step": c["seconds_per_step"]}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "fp32", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "heads": wl.heads, "head_dim": wl.head_dim,
+                   "grid": list(wl.grid), "tokens": wl.tokens, "tiles": wl.num_tiles, "topk": wl.topk,
+                   "selected_pairs_per_rank": pairs, "backward": wl.backward,
+                   "l2": "256 MB buffer written between timed steps"},
+        "stages_ms": {"router": router_ms, "topk": statistics.mean(per["topk"]), "fwd": fwd_ms,
+                      **({"bwd": statistics.mean(per["bwd"])} if wl.backward else {})},
+        "fwd_kernel": {"ms": fwd_ms, "effective_tflops": fwd_tflops,
+                       **({"frac_of_burst": fwd_tflops / bf16_burst} if tc else {})},
+        "router": {"ms": router_ms, "algorithmic_bytes": router_bytes,
+                   "gbs": router_bytes / (router_ms * 1e-3) / 1e9,
+                   "hbm_frac": router_bytes / (router_ms * 1e-3) / 1e9 / hbm,
+                   "roofline": {"bound": "mufu", "achieved": router_ex2 / (router_ms * 1e-3),
+                                "peak": mufu_peak(sm_max), "unit": "ex2/s",
+                                "frac": router_ex2 / (router_ms * 1e-3) / mufu_peak(sm_max),
+                                "exponentials": router_ex2}},
+        **({"bwd_pass": {"ms": bwd_ms, "effective_tflops": bwd_tflops, "frac_of_burst": bwd_tflops / bf16_burst}}
+           if wl.backward else {}),
+        "roofline": {"bound": roof["bound"], "kernel": roof["kernel"], "achieved": roof["achieved"],
+                     "peak": peak, "unit": "TFLOP/s", "frac": roof["achieved"] / peak, "peak_kind": kind,
+                     **extra_peak, "traffic": roof["traffic"]},
+        "cpu_baseline": cpu,
+        "e2e": {"value": flops_rank * world / (e2e * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "api": "VSA2.forward + attn_bwd after H2D copies" if wl.backward else "vsa2_forward_host"},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk.summary(),
+        **({"next_rows": next_rows} if next_rows else {}),
+    }
+    return line
+
+
+def run_ours(args, wls):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    lines = []
+    for wl in wls:
+        line = measure(args, wl, dev, rank, world)
+        if line is not None:
+            lines.append(line)
+            if wl.name != HEADLINE:
+                print(json.dumps(line), flush=True)
+    if rank == 0 and lines:
+        head = next((l for l in lines if l["config"]["workload"] == HEADLINE), lines[-1])
+        if len(lines) > 1:  # one-line digest of every config, at the end of the headline line
+            head["configs"] = {l["config"]["workload"]: {
+                "ms_per_step": round(l["ms_per_step"], 4), "value": round(l["value"], 2),
+                "roofline_frac": round(l["roofline"]["frac"], 4), "bound": l["roofline"]["bound"],
+                "fwd_ms": round(l["fwd_kernel"]["ms"], 4), "router_ms": round(l["router"]["ms"], 4),
+                "topk_ms": round(l["stages_ms"]["topk"], 4),
+                **({"bwd_ms": round(l["bwd_pass"]["ms"], 4)} if "bwd_pass" in l else {})} for l in lines}
+        print(json.dumps(head), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -509,19 +651,22 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(S.WORKLOADS))
+    ap.add_argument("--workload", default="all", choices=["all"] + list(S.WORKLOADS),
+                    help="all (default): every configuration, one JSON line each, the headline last")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--heads", type=int, default=None, help="override the head count (profiling runs)")
     ap.add_argument("--no-next", action="store_true", help="skip timing the coarse branch and the gated merge")
     args = ap.parse_args()
-    wl = S.WORKLOADS[args.workload]
+    names = ALL_WORKLOADS if args.workload == "all" else [args.workload]
+    wls = [S.WORKLOADS[n] for n in names]
     if args.heads:
-        wl = wl.with_(heads=args.heads)
+        wls = [wl.with_(heads=args.heads) for wl in wls]
     if args.impl == "reference":
-        run_reference(args, wl)
+        run_reference(args, S.WORKLOADS[HEADLINE] if args.workload == "all" else wls[0])
     else:
-        run_ours(args, wl)
+        run_ours(args, wls)
 
 
 if __name__ == "__main__":

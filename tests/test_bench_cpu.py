@@ -1,9 +1,11 @@
 """Host-side checks of bench.py that need no GPU: the reference arm prints one JSON line with
 the keys of the benchmark contract, and the DRAM-traffic figure is taken from a committed ncu
 summary only while that summary's kernel source is the one in the tree."""
+import hashlib
 import importlib.util
 import json
 import os
+import re
 import subprocess
 import sys
 
@@ -35,16 +37,36 @@ def test_reference_arm_prints_the_contract_line():
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
 
 
-def test_profiled_traffic_follows_the_kernel_source():
+def _fake_tree(tmp_path, kind, kernel_text, per_pair, recorded_text):
     b = _bench_module()
+    name, src_name, _ = b.TRAFFIC_PROFILES[kind]
+    (tmp_path / "profiles").mkdir(exist_ok=True)
+    csrc = tmp_path / "trainable_block_sparse_fine_b200" / "csrc"
+    csrc.mkdir(parents=True, exist_ok=True)
+    (csrc / src_name).write_bytes(kernel_text)
+    sha = hashlib.sha1(recorded_text).hexdigest()
+    (tmp_path / "profiles" / name).write_text(f"dram_bytes_per_pair: {per_pair}\nsource_sha1: {sha}\n")
+    return b
+
+
+def test_profiled_traffic_follows_the_kernel_source(tmp_path):
     fwd = S.WORKLOADS["720p_top64"]
     pairs = fwd.batch * fwd.heads * fwd.num_tiles * fwd.topk
-    got = b.profiled_traffic("fwd", fwd, pairs)
-    assert got is not None and got > 32768 * pairs * 0.1  # the committed summary matches the tree
+    b = _fake_tree(tmp_path, "fwd", b"kernel v1", 1234, b"kernel v1")
+    assert b.profiled_traffic("fwd", fwd, pairs, root=str(tmp_path)) == 1234 * pairs
+    # another workload shape: no figure
+    assert b.profiled_traffic("fwd", S.WORKLOADS["480p_top64"], pairs, root=str(tmp_path)) is None
+    # the kernel source changed since the counters were taken: no figure
+    b = _fake_tree(tmp_path, "fwd", b"kernel v2", 1234, b"kernel v1")
+    assert b.profiled_traffic("fwd", fwd, pairs, root=str(tmp_path)) is None
     train = S.WORKLOADS["480p_train_top64"]
-    assert b.profiled_traffic("bwd", train, train.batch * train.heads * train.num_tiles * train.topk) is not None
-    # another workload shape, or a summary whose recorded source is not this kernel's: no figure
-    assert b.profiled_traffic("fwd", S.WORKLOADS["480p_top64"], pairs) is None
-    name, _, grid = b.TRAFFIC_PROFILES["fwd"]
-    b.TRAFFIC_PROFILES["fwd"] = (name, "router.cu", grid)
-    assert b.profiled_traffic("fwd", fwd, pairs) is None
+    b = _fake_tree(tmp_path, "bwd", b"bwd", 99, b"bwd")
+    assert b.profiled_traffic("bwd", train, 10, root=str(tmp_path)) == 990
+
+
+def test_committed_summaries_name_a_source_and_a_figure():
+    b = _bench_module()
+    for name, src, _ in b.TRAFFIC_PROFILES.values():
+        txt = open(os.path.join(ROOT, "profiles", name)).read()
+        assert re.search(r"dram_bytes_per_pair:\s*\d+", txt) and re.search(r"source_sha1:\s*[0-9a-f]{40}", txt)
+        assert os.path.exists(os.path.join(ROOT, "trainable_block_sparse_fine_b200", "csrc", src))
