@@ -384,6 +384,50 @@ def test_fwd_720p_sampled_head0():
     assert np.abs(lg - wlse[r]).max() <= 2e-3 * max(1.0, np.abs(wlse[r]).max())
 
 
+def test_fwd_720p_edge_rows():
+    """720p-length sequences (3360 tiles) on a 2-head problem with hand-made rows: an empty
+    row, rows wholly in the lower or the upper half of the tile range, a single tile, odd
+    lengths, a descending (unsorted) row, two adjacent tiles, and random rows elsewhere."""
+    wl = C720.with_(heads=2)
+    N, L, D = wl.num_tiles, wl.tokens, wl.head_dim
+    rng = np.random.default_rng(72)
+    g = torch.Generator(device="cuda").manual_seed(721)
+    x = {n: (torch.randn((1, 2, L, D), generator=g, device="cuda") * 1.1).to(torch.bfloat16) for n in "qkv"}
+    rows = [np.sort(rng.choice(N, 64, replace=False)) for _ in range(N)]
+    half = N // 2
+    special = {0: np.array([], np.int64),
+               1: np.sort(rng.choice(half, 40, replace=False)),
+               2: np.sort(half + rng.choice(N - half, 33, replace=False)),
+               3: np.array([half]),
+               4: np.sort(np.concatenate([rng.choice(half, 7, replace=False), half + rng.choice(half, 8, replace=False)])),
+               5: np.sort(rng.choice(N, 50, replace=False))[::-1].copy(),
+               6: np.array([half - 1, half])}
+    for i, r in special.items():
+        rows[i] = r
+    kv_off = np.zeros((1, 2, N + 1), np.int32)
+    kv_idx = np.zeros((1, 2, N * wl.topk), np.int32)
+    for h in range(2):
+        lens = np.array([len(r) for r in rows])
+        kv_off[0, h, 1:] = np.cumsum(lens)
+        flat = np.concatenate(rows)
+        kv_idx[0, h, :flat.size] = flat
+    e = engine(wl)
+    o, lse = e.attn_fwd(x["q"], x["k"], x["v"], torch.from_numpy(kv_off).cuda(), torch.from_numpy(kv_idx).cuda())
+    assert e.device_error() == 0
+    tiles = sorted(set(special) | {100, N // 2, N - 1})
+    r = np.concatenate([np.arange(64 * i, 64 * i + 64) for i in tiles])
+    for h in range(2):
+        xh = {n: x[n][0, h].float().cpu().numpy() for n in "qkv"}
+        wo, wlse = O.sparse_attn_fwd(xh["q"], xh["k"], xh["v"], kv_off[0, h], kv_idx[0, h], query_tiles=tiles)
+        got = o[0, h].float().cpu().numpy()[r]
+        assert_attn_close(got, wo[r], f"o[0,{h}]")
+        lg, lw = lse[0, h].cpu().numpy()[r], wlse[r]
+        fin = np.isfinite(lw)
+        assert np.array_equal(fin, np.isfinite(lg))
+        assert np.abs(lg[fin] - lw[fin]).max() <= 2e-3 * max(1.0, np.abs(lw[fin]).max())
+        assert np.all(got[~fin] == 0)
+
+
 def test_fwd_480p_sampled_heads():
     wl = C480
     heads = [0, 19]
