@@ -50,8 +50,15 @@ def test_workspace_size_for_every_workload(name):
 
 def test_unsupported_shapes_give_zero_workspace():
     assert C.vsa2_workspace_size(C.make_problem(1, 2, 96, (8, 16, 16)), 8) == 0  # head_dim
-    assert C.vsa2_workspace_size(C.make_problem(1, 2, 64, (6, 16, 16)), 8) == 0  # grid % tile
     assert C.vsa2_workspace_size(C.make_problem(1, 2, 64, (8, 16, 16), pool=(2, 2, 2)), 8) == 0  # R != 16
+    assert C.vsa2_workspace_size(C.make_problem(1, 2, 64, (8, 16, 16), tile=(4, 4, 4), pool=(3, 2, 4)), 8) == 0
+
+
+def test_grid_the_tile_does_not_divide_is_padded():
+    """6x7x10 pads to 8x8x12 (24 tiles): the workspace is the padded problem's, as for 8x8x12."""
+    padded = C.vsa2_workspace_size(C.make_problem(1, 2, 64, (6, 7, 10)), 3)
+    whole = C.vsa2_workspace_size(C.make_problem(1, 2, 64, (8, 8, 12)), 3)
+    assert padded > 0 and padded == whole
 
 
 def test_argument_errors_are_synchronous():

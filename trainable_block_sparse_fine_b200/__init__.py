@@ -37,7 +37,12 @@ class VSA2:
         lib()  # fail loudly if the native library is missing
         self.p = make_problem(batch, heads, head_dim, grid, dtype, flags=flags, wait_timeout_ms=wait_timeout_ms)
         self.batch, self.heads, self.head_dim, self.grid, self.topk = batch, heads, head_dim, tuple(grid), topk
-        self.L = grid[0] * grid[1] * grid[2]
+        # a grid the 4x4x4 tile does not divide is padded to whole tiles (§2.2 "Kernel
+        # Implementation"): every [B, H, L, D] tensor of the path holds the padded grid in
+        # cube-major order; to_cube_major / to_raster pad and crop
+        self.L_real = grid[0] * grid[1] * grid[2]
+        self.grid_padded = tuple(-(-g // 4) * 4 for g in grid)
+        self.L = self.grid_padded[0] * self.grid_padded[1] * self.grid_padded[2]
         self.N = self.L // 64
         self.dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
         self.device = torch.device(device)
@@ -100,15 +105,18 @@ class VSA2:
         return o, lse, sel
 
     def to_cube_major(self, x, out=None):
-        """[B, H, L, D] (or [B, H, T, H, W, D]) in raster token order -> [B, H, L, D] cube-major."""
+        """[B, H, T*H*W, D] (or [B, H, T, H, W, D]) in raster token order -> [B, H, L, D] cube-major
+        (padding tokens of a grid the tile does not divide are written as zeros)."""
         out = out if out is not None else torch.empty(self.batch, self.heads, self.L, self.head_dim, dtype=x.dtype,
                                                       device=self.device)
         vsa2_permute_tokens(self.p, x, out, True)
         return out
 
     def to_raster(self, x, out=None):
-        """[B, H, L, D] cube-major -> [B, H, L, D] in raster token order (t, h, w)."""
-        out = out if out is not None else torch.empty_like(x)
+        """[B, H, L, D] cube-major -> [B, H, T*H*W, D] in raster token order (t, h, w), padding
+        tokens dropped."""
+        out = out if out is not None else torch.empty(self.batch, self.heads, self.L_real, self.head_dim,
+                                                      dtype=x.dtype, device=self.device)
         vsa2_permute_tokens(self.p, x, out, False)
         return out
 

@@ -21,9 +21,14 @@ vsa2_status make_dims(const vsa2_problem* p, Dims* d) {
   if (p->head_dim != 64 && p->head_dim != 128) return VSA2_ERR_UNSUPPORTED;
   if (p->tile_t * p->tile_h * p->tile_w != kTile) return VSA2_ERR_UNSUPPORTED;
   if (p->pool_t * p->pool_h * p->pool_w != kPool) return VSA2_ERR_UNSUPPORTED;
-  if (p->grid_t % p->tile_t || p->grid_h % p->tile_h || p->grid_w % p->tile_w) return VSA2_ERR_UNSUPPORTED;
   if (p->tile_t % p->pool_t || p->tile_h % p->pool_h || p->tile_w % p->pool_w) return VSA2_ERR_UNSUPPORTED;
-  const int64_t L = p->grid_t * p->grid_h * p->grid_w;
+  // a grid the tile does not divide is padded to whole tiles (§2.2 "Kernel Implementation")
+  const bool padded = p->grid_t % p->tile_t || p->grid_h % p->tile_h || p->grid_w % p->tile_w;
+  const int64_t pt = (p->grid_t + p->tile_t - 1) / p->tile_t * p->tile_t;
+  const int64_t ph = (p->grid_h + p->tile_h - 1) / p->tile_h * p->tile_h;
+  const int64_t pw = (p->grid_w + p->tile_w - 1) / p->tile_w * p->tile_w;
+  if (pt > (1 << 20) || ph > (1 << 20) || pw > (1 << 20)) return VSA2_ERR_UNSUPPORTED;
+  const int64_t L = pt * ph * pw;
   const int64_t N = L / kTile;
   const int64_t BH = p->batch * p->heads;
   // index arithmetic below uses 32-bit tile and row counts
@@ -39,6 +44,10 @@ vsa2_status make_dims(const vsa2_problem* p, Dims* d) {
   d->esize = p->dtype == VSA2_BF16 ? 2 : 4;
   d->flags = p->flags;
   d->timeout_ns = (uint64_t)(p->wait_timeout_ms ? p->wait_timeout_ms : 2000u) * 1000000ull;
+  d->gt = (int)p->grid_t, d->gh = (int)p->grid_h, d->gw = (int)p->grid_w;
+  d->tt = p->tile_t, d->th = p->tile_h, d->tw = p->tile_w;
+  d->rt = p->pool_t, d->rh = p->pool_h, d->rw = p->pool_w;
+  d->padded = padded;
   return VSA2_OK;
 }
 
@@ -76,6 +85,7 @@ WsLayout ws_layout(const Dims& d) {
   w.dqc = take((size_t)d.BH * lc * d.D * 4);
   w.dkc = take((size_t)d.BH * lc * d.D * 4);
   w.dvc = take((size_t)d.BH * lc * d.D * 4);
+  w.tmask = take((size_t)d.N * 8);
   w.total = off;
   return w;
 }
@@ -271,6 +281,7 @@ vsa2_status vsa2_sparse_attn_bwd(const vsa2_problem* p, const void* q, const voi
   Dims d;
   vsa2_status st = make_dims(p, &d);
   if (st != VSA2_OK) return st;
+  if (d.padded) return VSA2_ERR_UNSUPPORTED;  // the backward takes whole-tile grids only
   if (!q || !k || !v || !o || !lse || !dout || !kv_off || !kv_idx || !q_off || !q_idx || !dq || !dk || !dv)
     return VSA2_ERR_INVALID_ARG;
   if (topk < 1 || topk > d.N) return VSA2_ERR_UNSUPPORTED;
@@ -321,6 +332,7 @@ vsa2_status vsa2_coarse_attn_bwd(const vsa2_problem* p, const void* q, const voi
   Dims d;
   vsa2_status st = make_dims(p, &d);
   if (st != VSA2_OK) return st;
+  if (d.padded) return VSA2_ERR_UNSUPPORTED;  // the backward takes whole-tile grids only
   if (!q || !k || !v || !oc || !lse_c || !d_oc || !dq || !dk || !dv) return VSA2_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(oc) || !aligned16(lse_c) || !aligned16(d_oc) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))

@@ -22,9 +22,12 @@
 // max is raised (with an O rescale in TMEM) only when a row's new maximum exceeds it by more
 // than 2^8.
 //
-// kPad = true masks keys at or beyond `kv_valid` tokens of a head (a sequence whose last tile is
-// partly padding, such as the coarse branch's N pooled rows, Eq. 1-3). Every listed tile must
-// hold at least one valid key. kPad = false is the fine branch (Eq. 12), with no key mask.
+// kMode selects the key mask: 0 = none (the fine branch, Eq. 12); 1 = keys at or beyond
+// `kv_valid` tokens of a head are padding (a sequence whose last tile is partly padding, such as
+// the coarse branch's N pooled rows, Eq. 1-3); 2 = a grid the tile does not divide, with the
+// real tokens of every tile in `tmask` (§2.2 "Kernel Implementation"): padding keys are masked
+// and padding query rows are written as o = 0, lse = -inf. Every listed tile must hold at least
+// one valid key.
 #include <algorithm>
 
 #include "common.cuh"
@@ -127,12 +130,13 @@ __device__ __forceinline__ int next_op(SlotSeq& q, int* blk, const int32_t* kv_o
   return 0;
 }
 
-template <bool kPad>
+template <int kMode>
 __global__ void __launch_bounds__(FT, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const __nv_bfloat16* __restrict__ qg, const int32_t* __restrict__ kv_off,
                        const int32_t* __restrict__ kv_idx, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
-                       int N, int L, int topk, int items, float c2, int kv_valid, DevCtx ctx) {
+                       int N, int L, int topk, int items, float c2, int kv_valid,
+                       const uint64_t* __restrict__ tmask, DevCtx ctx) {
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
   uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   Bars& B = *reinterpret_cast<Bars*>(dsm + OFF_BAR);
@@ -305,7 +309,7 @@ __global__ void __launch_bounds__(FT, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&B.sfree[s][g & 1]);
-        if constexpr (kPad) {
+        if constexpr (kMode == 1) {
           // keys of the block's two tiles at or beyond kv_valid get a score of -inf
           const int32_t* ix = kv_idx + (size_t)bh * cap + rw.beg + 2 * n;
           const int v1 = kv_valid - 64 * __ldg(ix);
@@ -314,6 +318,16 @@ __global__ void __launch_bounds__(FT, 1)
 #pragma unroll
             for (int i = 0; i < 64; ++i)
               if (((2 * i + par_c) & 63) >= (i < 32 ? v1 : v2)) x[i] = __float_as_uint(-INFINITY);
+          }
+        } else if constexpr (kMode == 2) {
+          // padding tokens of the block's two tiles get a score of -inf
+          const int32_t* ix = kv_idx + (size_t)bh * cap + rw.beg + 2 * n;
+          const uint64_t m1 = __ldg(tmask + min(max(__ldg(ix), 0), N - 1));
+          const uint64_t m2 = half ? ~0ull : __ldg(tmask + min(max(__ldg(ix + 1), 0), N - 1));
+          if ((m1 & m2) != ~0ull) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+              if (!(((i < 32 ? m1 : m2) >> ((2 * i + par_c) & 63)) & 1ull)) x[i] = __float_as_uint(-INFINITY);
           }
         }
         // columns 2i + par_c; in a half block only the first 64 columns are real
@@ -377,11 +391,20 @@ __global__ void __launch_bounds__(FT, 1)
       mbar_wait(&B.pvdone[s], (g - 1) & 1, abort, ctx);
       tc_fence_after();
       l += __shfl_xor_sync(0xffffffffu, l, 2);
-      const float inv = 1.f / l;
-      if (par_c == 0) lse[tok] = (m + __log2f(l)) * 0.6931471805599453f;
+      float inv = 1.f / l;
+      float lse_row = (m + __log2f(l)) * 0.6931471805599453f;
       uint32_t o[64];
       tmem_ld16x64b_x64(tl + TM_O, o);
       tmem_ld_wait();
+      if constexpr (kMode == 2) {
+        if (!((__ldg(tmask + qt) >> row) & 1ull)) {  // a padding query row: o = 0, lse = -inf
+#pragma unroll
+          for (int i = 0; i < 64; ++i) o[i] = 0u;
+          inv = 0.f;
+          lse_row = -INFINITY;
+        }
+      }
+      if (par_c == 0) lse[tok] = lse_row;
       // o[i] = O[row][2i + par_c]; swap so each thread holds adjacent pairs, then 4-byte stores
       uint32_t* dst = reinterpret_cast<uint32_t*>(out + tok * 128);
 #pragma unroll
@@ -409,10 +432,10 @@ bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64
                        uint32_t box_rows);
 
 namespace {
-template <bool kPad>
+template <int kMode>
 vsa2_status launch_fwd_tc(const Dims& d, const void* q, const void* k, const void* v, int topk,
                           const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws, int kv_valid,
-                          cudaStream_t s) {
+                          const uint64_t* tmask, cudaStream_t s) {
   CUtensorMap tk, tv;
   const uint64_t rows = (uint64_t)d.BH * d.L;
   if (!make_tmap_2d_bf16(&tk, k, 128, rows, 64, 64) || !make_tmap_2d_bf16(&tv, v, 128, rows, 64, 64))
@@ -424,23 +447,28 @@ vsa2_status launch_fwd_tc(const Dims& d, const void* q, const void* k, const voi
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::max(1, std::min(sms, (items + 1) / 2));
   const float c2 = 1.4426950408889634f / sqrtf(128.f);
-  cudaFuncSetAttribute(attn_fwd_tc_kernel<kPad>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
-  attn_fwd_tc_kernel<kPad><<<grid, FT, SMEM_DYN, s>>>(tk, tv, (const __nv_bfloat16*)q, kv_off, kv_idx,
-                                                      (__nv_bfloat16*)o, lse, d.N, (int)d.L, topk, items, c2,
-                                                      kv_valid, ctx);
+  cudaFuncSetAttribute(attn_fwd_tc_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
+  attn_fwd_tc_kernel<kMode><<<grid, FT, SMEM_DYN, s>>>(tk, tv, (const __nv_bfloat16*)q, kv_off, kv_idx,
+                                                       (__nv_bfloat16*)o, lse, d.N, (int)d.L, topk, items, c2,
+                                                       kv_valid, tmask, ctx);
   return check_launch("attn_fwd_tc");
 }
 }  // namespace
 
 vsa2_status attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v, int topk, const int32_t* kv_off,
                         const int32_t* kv_idx, void* o, float* lse, char* ws, cudaStream_t s) {
-  return launch_fwd_tc<false>(d, q, k, v, topk, kv_off, kv_idx, o, lse, ws, (int)d.L, s);
+  if (d.padded) {
+    uint64_t* tmask = reinterpret_cast<uint64_t*>(ws + ws_layout(d).tmask);
+    if (launch_tile_masks(d, tmask, s) != VSA2_OK) return VSA2_ERR_CUDA;
+    return launch_fwd_tc<2>(d, q, k, v, topk, kv_off, kv_idx, o, lse, ws, (int)d.L, tmask, s);
+  }
+  return launch_fwd_tc<0>(d, q, k, v, topk, kv_off, kv_idx, o, lse, ws, (int)d.L, nullptr, s);
 }
 
 vsa2_status attn_fwd_tc_masked(const Dims& d, const void* q, const void* k, const void* v, int topk,
                                const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
                                int kv_valid, cudaStream_t s) {
-  return launch_fwd_tc<true>(d, q, k, v, topk, kv_off, kv_idx, o, lse, ws, kv_valid, s);
+  return launch_fwd_tc<1>(d, q, k, v, topk, kv_off, kv_idx, o, lse, ws, kv_valid, nullptr, s);
 }
 
 }  // namespace vsa2

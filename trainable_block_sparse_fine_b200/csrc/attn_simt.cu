@@ -49,7 +49,8 @@ __global__ void __launch_bounds__(64) attn_fwd_simt_kernel(const T* __restrict__
                                                            const T* __restrict__ v, const int32_t* __restrict__ kv_off,
                                                            const int32_t* __restrict__ kv_idx, T* __restrict__ o,
                                                            float* __restrict__ lse, int N, int64_t L, int topk,
-                                                           int64_t kv_valid, DevCtx ctx) {
+                                                           int64_t kv_valid, const uint64_t* __restrict__ tmask,
+                                                           DevCtx ctx) {
   extern __shared__ float sm[];
   float* qT = sm;              // [D][64]
   float* ks = qT + D * 64;     // [64][D]
@@ -72,6 +73,7 @@ __global__ void __launch_bounds__(64) attn_fwd_simt_kernel(const T* __restrict__
     const int j = idx[p];
     if (!idx_ok(j, N, ctx)) break;
     const size_t kt0 = (size_t)bh * L + (size_t)j * kTile;
+    const uint64_t km = tmask ? tmask[j] : ~0ull;  // real tokens of a padded grid's tile
     __syncthreads();
     for (int e = t; e < 64 * D; e += 64) {
       ks[e] = ldf(k + kt0 * D + e);
@@ -84,7 +86,8 @@ __global__ void __launch_bounds__(64) attn_fwd_simt_kernel(const T* __restrict__
     for (int u = 0; u < 64; ++u) {
       float acc = 0.f;
       for (int d = 0; d < D; ++d) acc += qT[d * 64 + t] * ks[u * D + d];
-      s[u] = (int64_t)j * kTile + u < kv_valid ? acc * scale : -INFINITY;  // keys past kv_valid are padding
+      // keys past kv_valid, and padding tokens of a padded grid, are masked
+      s[u] = ((int64_t)j * kTile + u < kv_valid && ((km >> u) & 1ull)) ? acc * scale : -INFINITY;
       mx = fmaxf(mx, s[u]);
     }
     const float mn = fmaxf(m, mx);
@@ -104,9 +107,10 @@ __global__ void __launch_bounds__(64) attn_fwd_simt_kernel(const T* __restrict__
       oT[d * 64 + t] = acc;
     }
   }
-  const float inv = l > 0.f ? 1.f / l : 0.f;
-  for (int d = 0; d < D; ++d) stf(o + (tok0 + t) * D + d, oT[d * 64 + t] * inv);
-  lse[tok0 + t] = l > 0.f ? m + __logf(l) : -INFINITY;
+  const bool q_real = !tmask || ((tmask[i] >> t) & 1ull);  // a padding query row gets o = 0, lse = -inf
+  const float inv = (l > 0.f && q_real) ? 1.f / l : 0.f;
+  for (int d = 0; d < D; ++d) stf(o + (tok0 + t) * D + d, inv != 0.f ? oT[d * 64 + t] * inv : 0.f);
+  lse[tok0 + t] = (l > 0.f && q_real) ? m + __logf(l) : -INFINITY;
 }
 
 // delta = rowsum(dO * O), warp per row.
@@ -264,12 +268,12 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_simt_kernel(const T* __rest
 template <typename T, int D>
 vsa2_status fwd_simt(const Dims& d, const void* q, const void* k, const void* v, const int32_t* kv_off,
                      const int32_t* kv_idx, void* o, float* lse, const DevCtx& ctx, int topk, int64_t kv_valid,
-                     cudaStream_t s) {
+                     const uint64_t* tmask, cudaStream_t s) {
   const size_t smem = (size_t)4 * 64 * D * sizeof(float);
   auto kern = attn_fwd_simt_kernel<T, D>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   kern<<<dim3(d.N, d.BH), 64, smem, s>>>((const T*)q, (const T*)k, (const T*)v, kv_off, kv_idx, (T*)o, lse, d.N,
-                                         d.L, topk, kv_valid, ctx);
+                                         d.L, topk, kv_valid, tmask, ctx);
   return check_launch(__func__);
 }
 
@@ -297,14 +301,15 @@ vsa2_status bwd_simt(const Dims& d, const void* q, const void* k, const void* v,
 
 vsa2_status attn_fwd_simt(const Dims& d, const void* q, const void* k, const void* v, int topk,
                           const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
-                          int64_t kv_valid, cudaStream_t s) {
+                          int64_t kv_valid, const uint64_t* tmask, cudaStream_t s) {
   DevCtx ctx{reinterpret_cast<int*>(ws), d.timeout_ns, d.flags};
   if (d.dtype == VSA2_BF16) {
-    if (d.D == 128) return fwd_simt<__nv_bfloat16, 128>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, s);
-    return fwd_simt<__nv_bfloat16, 64>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, s);
+    if (d.D == 128)
+      return fwd_simt<__nv_bfloat16, 128>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, tmask, s);
+    return fwd_simt<__nv_bfloat16, 64>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, tmask, s);
   }
-  if (d.D == 128) return fwd_simt<float, 128>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, s);
-  return fwd_simt<float, 64>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, s);
+  if (d.D == 128) return fwd_simt<float, 128>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, tmask, s);
+  return fwd_simt<float, 64>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, tmask, s);
 }
 
 vsa2_status attn_bwd_simt(const Dims& d, const void* q, const void* k, const void* v, const void* o, const float* lse,

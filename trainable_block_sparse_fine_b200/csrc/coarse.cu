@@ -60,12 +60,13 @@ __device__ __forceinline__ void store_vec(T* p, const float* f) {
 }
 
 // Eq. 1: warp per pooled row r of head bh; lane owns D/32 consecutive channels. Rows r >= N
-// (padding of the last tile) are written as zeros.
+// (padding of the last tile) are written as zeros. With tmask (a padded grid) each mean runs
+// over the tile's real tokens only.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) coarse_pool_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                           const T* __restrict__ v, T* __restrict__ qc,
                                                           T* __restrict__ kc, T* __restrict__ vc, int N, int Lc,
-                                                          int64_t L) {
+                                                          int64_t L, const uint64_t* __restrict__ tmask) {
   constexpr int V = D / 32;
   const int bh = blockIdx.y;
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -81,15 +82,18 @@ __global__ void __launch_bounds__(256) coarse_pool_kernel(const T* __restrict__ 
     for (int e = 0; e < V; ++e) acc[e] = 0.f;
     if (r < N) {
       const T* p = src[x] + ((size_t)bh * L + (size_t)r * kTile) * D + lane * V;
+      const uint64_t real = tmask ? __ldg(tmask + r) : ~0ull;
 #pragma unroll 8
       for (int t = 0; t < kTile; ++t) {
+        if (!((real >> t) & 1ull)) continue;
         float f[V];
         load_vec<T, V>(p + (size_t)t * D, f);
 #pragma unroll
         for (int e = 0; e < V; ++e) acc[e] += f[e];
       }
+      const float inv = 1.f / __popcll(real);  // every tile holds a real token
 #pragma unroll
-      for (int e = 0; e < V; ++e) acc[e] *= 1.f / kTile;
+      for (int e = 0; e < V; ++e) acc[e] *= inv;
     }
     store_vec<T, V>(out[x] + dst, acc);
   }
@@ -237,10 +241,10 @@ __global__ void __launch_bounds__(256) coarse_pool_bwd_kernel(const float* __res
 
 template <typename T, int D>
 void launch_pool(const Dims& d, const void* q, const void* k, const void* v, char* ws, const WsLayout& w,
-                 cudaStream_t s) {
+                 const uint64_t* tmask, cudaStream_t s) {
   const int Lc = kTile * w.Nc_tiles;
   coarse_pool_kernel<T, D><<<dim3((Lc + 7) / 8, d.BH), 256, 0, s>>>(
-      (const T*)q, (const T*)k, (const T*)v, (T*)(ws + w.qc), (T*)(ws + w.kc), (T*)(ws + w.vc), d.N, Lc, d.L);
+      (const T*)q, (const T*)k, (const T*)v, (T*)(ws + w.qc), (T*)(ws + w.kc), (T*)(ws + w.vc), d.N, Lc, d.L, tmask);
 }
 
 int grid_for(int64_t work, int per_block) {
@@ -256,15 +260,20 @@ vsa2_status launch_coarse_attn(const Dims& d, const void* q, const void* k, cons
   const WsLayout w = ws_layout(d);
   const int Nc = w.Nc_tiles;
   const int Lc = kTile * Nc;
-  // Eq. 1: pooled rows, padded with zeros to whole tiles
+  // Eq. 1: pooled rows (over the real tokens of a padded grid), padded with zeros to whole tiles
+  uint64_t* tmask = nullptr;
+  if (d.padded) {
+    tmask = reinterpret_cast<uint64_t*>(ws + w.tmask);
+    if (launch_tile_masks(d, tmask, s) != VSA2_OK) return VSA2_ERR_CUDA;
+  }
   if (d.dtype == VSA2_BF16 && d.D == 128)
-    launch_pool<__nv_bfloat16, 128>(d, q, k, v, ws, w, s);
+    launch_pool<__nv_bfloat16, 128>(d, q, k, v, ws, w, tmask, s);
   else if (d.dtype == VSA2_BF16)
-    launch_pool<__nv_bfloat16, 64>(d, q, k, v, ws, w, s);
+    launch_pool<__nv_bfloat16, 64>(d, q, k, v, ws, w, tmask, s);
   else if (d.D == 128)
-    launch_pool<float, 128>(d, q, k, v, ws, w, s);
+    launch_pool<float, 128>(d, q, k, v, ws, w, tmask, s);
   else
-    launch_pool<float, 64>(d, q, k, v, ws, w, s);
+    launch_pool<float, 64>(d, q, k, v, ws, w, tmask, s);
   int32_t* c_off = reinterpret_cast<int32_t*>(ws + w.c_off);
   int32_t* c_idx = reinterpret_cast<int32_t*>(ws + w.c_idx);
   coarse_csr_kernel<<<d.BH, 256, 0, s>>>(Nc, c_off, c_idx);
@@ -275,11 +284,12 @@ vsa2_status launch_coarse_attn(const Dims& d, const void* q, const void* k, cons
   dc.L = Lc;
   dc.N = Nc;
   dc.Lr = Lc / kPool;
+  dc.padded = false;  // the pooled sequence's own padding is the kv_valid bound below
   void* oc_pad = ws + w.oc;
   float* lse_pad = reinterpret_cast<float*>(ws + w.lse_c);
   st = (d.dtype == VSA2_BF16 && d.D == 128)
            ? attn_fwd_tc_masked(dc, ws + w.qc, ws + w.kc, ws + w.vc, Nc, c_off, c_idx, oc_pad, lse_pad, ws, d.N, s)
-           : attn_fwd_simt(dc, ws + w.qc, ws + w.kc, ws + w.vc, Nc, c_off, c_idx, oc_pad, lse_pad, ws, d.N, s);
+           : attn_fwd_simt(dc, ws + w.qc, ws + w.kc, ws + w.vc, Nc, c_off, c_idx, oc_pad, lse_pad, ws, d.N, nullptr, s);
   if (st != VSA2_OK) return st;
   // the first N rows of every head, packed
   const size_t row_b = (size_t)d.D * d.esize;
@@ -335,16 +345,16 @@ vsa2_status launch_coarse_attn_bwd(const Dims& d, const void* q, const void* k, 
   if (ws_layout(dc).nlse2 + align256((size_t)dc.BH * Lc * 4) > w.qc) return VSA2_ERR_UNSUPPORTED;
   // pooled operands (Eq. 1) again, the padded O_c_hat, LSE and dO_c_hat, and the dense CSR / CSC
   if (d.dtype == VSA2_BF16 && d.D == 128) {
-    launch_pool<__nv_bfloat16, 128>(d, q, k, v, ws, w, s);
+    launch_pool<__nv_bfloat16, 128>(d, q, k, v, ws, w, nullptr, s);  // whole-tile grids only
     launch_pad_bwd<__nv_bfloat16, 128>(d, oc, lse_c, d_oc, ws, w, s);
   } else if (d.dtype == VSA2_BF16) {
-    launch_pool<__nv_bfloat16, 64>(d, q, k, v, ws, w, s);
+    launch_pool<__nv_bfloat16, 64>(d, q, k, v, ws, w, nullptr, s);  // whole-tile grids only
     launch_pad_bwd<__nv_bfloat16, 64>(d, oc, lse_c, d_oc, ws, w, s);
   } else if (d.D == 128) {
-    launch_pool<float, 128>(d, q, k, v, ws, w, s);
+    launch_pool<float, 128>(d, q, k, v, ws, w, nullptr, s);  // whole-tile grids only
     launch_pad_bwd<float, 128>(d, oc, lse_c, d_oc, ws, w, s);
   } else {
-    launch_pool<float, 64>(d, q, k, v, ws, w, s);
+    launch_pool<float, 64>(d, q, k, v, ws, w, nullptr, s);  // whole-tile grids only
     launch_pad_bwd<float, 64>(d, oc, lse_c, d_oc, ws, w, s);
   }
   int32_t* c_off = reinterpret_cast<int32_t*>(ws + w.c_off);

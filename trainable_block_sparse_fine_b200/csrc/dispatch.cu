@@ -28,7 +28,12 @@ vsa2_status launch_attn_fwd(const Dims& d, const void* q, const void* k, const v
                             const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
                             cudaStream_t s) {
   if (d.dtype == VSA2_BF16 && d.D == 128) return attn_fwd_tc(d, q, k, v, topk, kv_off, kv_idx, o, lse, ws, s);
-  return attn_fwd_simt(d, q, k, v, topk, kv_off, kv_idx, o, lse, ws, d.L, s);
+  uint64_t* tmask = nullptr;
+  if (d.padded) {
+    tmask = reinterpret_cast<uint64_t*>(ws + ws_layout(d).tmask);
+    if (launch_tile_masks(d, tmask, s) != VSA2_OK) return VSA2_ERR_CUDA;
+  }
+  return attn_fwd_simt(d, q, k, v, topk, kv_off, kv_idx, o, lse, ws, d.L, tmask, s);
 }
 
 vsa2_status launch_attn_bwd(const Dims& d, const void* q, const void* k, const void* v, const void* o,

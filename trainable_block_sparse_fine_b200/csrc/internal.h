@@ -16,14 +16,22 @@ constexpr int kG = kTile / kPool;
 
 struct Dims {
   int B, H, D, BH;
-  int64_t L;   // tokens per (b, h)
+  int64_t L;   // tokens per (b, h), of the padded grid when the tile does not divide the grid
   int N;       // tiles per (b, h)
   int Lr;      // pooled rows per (b, h)
   int dtype;   // vsa2_dtype
   int esize;   // bytes per element of Q/K/V/O/dO
   uint32_t flags;
   uint64_t timeout_ns;
+  int gt, gh, gw;  // real token grid
+  int tt, th, tw;  // tile
+  int rt, rh, rw;  // router sub-cube
+  bool padded;     // the tile does not divide the grid: every extent is rounded up to whole tiles
 };
+
+// Real-token mask of every tile of a padded grid (bit u = cube-major token u of the tile is a
+// token of the real grid); the same for every (b, h). Enqueued on `s`, written to `mask` [N].
+vsa2_status launch_tile_masks(const Dims& d, uint64_t* mask, cudaStream_t s);
 
 // Validate a problem description; fills `d` on success.
 vsa2_status make_dims(const vsa2_problem* p, Dims* d);
@@ -48,6 +56,7 @@ struct WsLayout {
   size_t c_off, c_idx;   // coarse branch: CSR listing every tile, [BH, Nc_tiles + 1], [BH, Nc_tiles^2] i32
   size_t doc;            // coarse backward: padded gradient of O_c_hat, [BH, 64 * Nc_tiles, D] dtype
   size_t dqc, dkc, dvc;  // coarse backward: gradients of the pooled rows, [BH, 64 * Nc_tiles, D] fp32
+  size_t tmask;          // padded grids: real-token mask per tile, [N] u64
   size_t total;
 };
 WsLayout ws_layout(const Dims& d);
@@ -71,10 +80,11 @@ vsa2_status launch_attn_bwd(const Dims& d, const void* q, const void* k, const v
                             const int32_t* kv_idx, const int32_t* q_off, const int32_t* q_idx, float* dq, float* dk,
                             float* dv, char* ws, cudaStream_t s);
 // CUDA-core paths (fp32 inputs, head_dim 64, and the backward pass). The forward masks keys at
-// or beyond kv_valid tokens of each head (d.L for the fine branch: no mask).
+// or beyond kv_valid tokens of each head (d.L for the fine branch: no mask) and, with tmask (a
+// padded grid's real-token masks), the padding tokens of every tile.
 vsa2_status attn_fwd_simt(const Dims& d, const void* q, const void* k, const void* v, int topk,
                           const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
-                          int64_t kv_valid, cudaStream_t s);
+                          int64_t kv_valid, const uint64_t* tmask, cudaStream_t s);
 vsa2_status attn_bwd_simt(const Dims& d, const void* q, const void* k, const void* v, const void* o,
                           const float* lse, const void* dout, const int32_t* kv_off, const int32_t* kv_idx,
                           const int32_t* q_off, const int32_t* q_idx, float* dq, float* dk, float* dv, int topk,

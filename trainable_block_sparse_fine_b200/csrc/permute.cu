@@ -5,6 +5,10 @@
 // every row is read once and written once, 16 bytes per thread and iteration, so each group
 // of D*esize/16 threads moves one whole row.
 //
+// A grid the tile does not divide is padded to whole tiles (§2.2 "Kernel Implementation"): the
+// cube-major side then holds the padded grid, raster -> cube-major writes zeros in the padding
+// rows, and cube-major -> raster drops them.
+//
 // The row index arithmetic divides by runtime constants (grid, tile and pool extents) eight
 // times per row. To keep it off the critical path it uses division by invariant integers with
 // a multiply-high and a shift (Granlund and Montgomery, "Division by Invariant Integers using
@@ -37,10 +41,12 @@ struct Geom {
   FastDiv tiles_hw, tiles_w; // tile grid: tiles per t-slab, per h-row
   FastDiv subs_hw, subs_w;   // sub-cubes of a tile: per t-slab, per h-row
   FastDiv pool_hw, pool_w;   // tokens of a sub-cube: per t-slab, per h-row
-  uint32_t bt, bh, bw, rt, rh, rw, gh, gw;
+  uint32_t bt, bh, bw, rt, rh, rw, gt, gh, gw;  // tile, sub-cube, real grid
+  uint32_t Lr;                                    // real tokens per (b, h)
 };
 
-// raster index (t*H + h)*W + w of the token at cube-major index l of a head
+// raster index (t*H + h)*W + w (in the real grid) of the token at cube-major index l of a head,
+// or UINT32_MAX for a padding token
 __device__ __forceinline__ uint32_t raster_of(uint32_t l, const Geom& g) {
   const uint32_t i = fdiv(l, g.tile), in_tile = l - i * g.tile.d;
   const uint32_t sidx = fdiv(in_tile, g.pool), r = in_tile - sidx * g.pool.d;
@@ -53,6 +59,7 @@ __device__ __forceinline__ uint32_t raster_of(uint32_t l, const Geom& g) {
   const uint32_t t = a * g.bt + st * g.rt + dt;
   const uint32_t h = b * g.bh + sh * g.rh + dh;
   const uint32_t w = c * g.bw + sw * g.rw + dw;
+  if (t >= g.gt || h >= g.gh || w >= g.gw) return 0xffffffffu;
   return (t * g.gh + h) * g.gw + w;
 }
 
@@ -63,7 +70,12 @@ __global__ void __launch_bounds__(256) permute_kernel(const uint4* __restrict__ 
   for (uint64_t c = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; c < total; c += (uint64_t)gridDim.x * blockDim.x) {
     const uint32_t row = (uint32_t)(c >> ch_shift), part = (uint32_t)c & ch_mask;
     const uint32_t bh = fdiv(row, g.L), l = row - bh * g.L.d;
-    const uint64_t raster_row = (uint64_t)bh * g.L.d + raster_of(l, g);
+    const uint32_t r = raster_of(l, g);
+    if (r == 0xffffffffu) {  // a padding token: zeros on the cube-major side, nothing in raster order
+      if (to_cube) dst[((uint64_t)row << ch_shift) + part] = make_uint4(0, 0, 0, 0);
+      continue;
+    }
+    const uint64_t raster_row = (uint64_t)bh * g.Lr + r;
     const uint64_t from = ((to_cube ? raster_row : (uint64_t)row) << ch_shift) + part;
     const uint64_t to = ((to_cube ? (uint64_t)row : raster_row) << ch_shift) + part;
     dst[to] = __ldg(src + from);
@@ -81,7 +93,8 @@ vsa2_status launch_permute(const Dims& d, const vsa2_problem* p, const void* src
   g.L = make_fastdiv((uint32_t)d.L);
   g.tile = make_fastdiv((uint32_t)(p->tile_t * p->tile_h * p->tile_w));
   g.pool = make_fastdiv((uint32_t)(p->pool_t * p->pool_h * p->pool_w));
-  const uint32_t nh = (uint32_t)(p->grid_h / p->tile_h), nw = (uint32_t)(p->grid_w / p->tile_w);
+  const uint32_t nh = (uint32_t)((p->grid_h + p->tile_h - 1) / p->tile_h);  // tiles of the padded grid
+  const uint32_t nw = (uint32_t)((p->grid_w + p->tile_w - 1) / p->tile_w);
   g.tiles_hw = make_fastdiv(nh * nw);
   g.tiles_w = make_fastdiv(nw);
   const uint32_t sh_n = (uint32_t)(p->tile_h / p->pool_h), sw_n = (uint32_t)(p->tile_w / p->pool_w);
@@ -91,7 +104,8 @@ vsa2_status launch_permute(const Dims& d, const vsa2_problem* p, const void* src
   g.pool_w = make_fastdiv((uint32_t)p->pool_w);
   g.bt = p->tile_t, g.bh = p->tile_h, g.bw = p->tile_w;
   g.rt = p->pool_t, g.rh = p->pool_h, g.rw = p->pool_w;
-  g.gh = (uint32_t)p->grid_h, g.gw = (uint32_t)p->grid_w;
+  g.gt = (uint32_t)p->grid_t, g.gh = (uint32_t)p->grid_h, g.gw = (uint32_t)p->grid_w;
+  g.Lr = (uint32_t)(p->grid_t * p->grid_h * p->grid_w);
   const uint32_t rows = (uint32_t)((int64_t)d.BH * d.L);
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -13,10 +13,13 @@ namespace {
 // MeanPool_R (Eq. 5): each pooled row is the mean of R = 16 consecutive cube-major rows.
 // One thread per (pooled row, 16-byte column chunk); 16 independent 16-byte loads per thread.
 // ------------------------------------------------------------------------------------------
-template <typename T>
+// With kMask (a padded grid), each mean runs over the sub-cube's real tokens only (tmask, the
+// per-tile real-token masks); a sub-cube without one is written as zeros.
+template <typename T, bool kMask>
 __global__ void __launch_bounds__(256) router_pool_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                           T* __restrict__ qr, T* __restrict__ kr,
-                                                          int64_t pooled_rows, int chunks_per_row) {
+                                                          int64_t pooled_rows, int chunks_per_row,
+                                                          const uint64_t* __restrict__ tmask, int Lr) {
   constexpr int EPC = 16 / sizeof(T);  // elements per 16-byte chunk
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t per_tensor = pooled_rows * chunks_per_row;
@@ -30,11 +33,19 @@ __global__ void __launch_bounds__(256) router_pool_kernel(const T* __restrict__ 
   float acc[EPC];
 #pragma unroll
   for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+  uint32_t valid = 0xffffu;
+  float inv = 1.f / kPool;
+  if constexpr (kMask) {
+    const int a = (int)(prow % Lr);
+    valid = (uint32_t)(__ldg(tmask + (a >> 2)) >> (16 * (a & 3))) & 0xffffu;
+    inv = valid ? 1.f / __popc(valid) : 0.f;
+  }
   uint4 buf[kPool];
 #pragma unroll
   for (int r = 0; r < kPool; ++r) buf[r] = __ldg(reinterpret_cast<const uint4*>(src + r * stride));
 #pragma unroll
   for (int r = 0; r < kPool; ++r) {
+    if (kMask && !((valid >> r) & 1u)) continue;
     if constexpr (sizeof(T) == 2) {
       const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&buf[r]);
 #pragma unroll
@@ -54,11 +65,11 @@ __global__ void __launch_bounds__(256) router_pool_kernel(const T* __restrict__ 
   if constexpr (sizeof(T) == 2) {
     uint32_t* o = reinterpret_cast<uint32_t*>(&out);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) o[e] = pack_bf16(acc[2 * e] * (1.f / kPool), acc[2 * e + 1] * (1.f / kPool));
+    for (int e = 0; e < 4; ++e) o[e] = pack_bf16(acc[2 * e] * inv, acc[2 * e + 1] * inv);
   } else {
     float* o = reinterpret_cast<float*>(&out);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) o[e] = acc[e] * (1.f / kPool);
+    for (int e = 0; e < 4; ++e) o[e] = acc[e] * inv;
   }
   *reinterpret_cast<uint4*>(dst) = out;
 }
@@ -87,10 +98,25 @@ struct RouterSmem {
   static constexpr uint32_t kDyn = (kTotal + 1024 > 119808u) ? kTotal + 1024 : 119808u;
 };
 
-template <int ND>
+// Pooled key b is valid unless it lies past Lr or (kMask) its sub-cube holds no real token.
+// Returns the validity of keys key0 .. key0+31 as a bit mask (the same in every lane).
+template <bool kMask>
+__device__ __forceinline__ uint32_t piece_keys(int key0, int Lr, const uint64_t* tmask) {
+  const int lane = threadIdx.x & 31;
+  const int b = key0 + lane;
+  bool ok = b < Lr;
+  if (kMask && ok) ok = ((__ldg(tmask + (b >> 2)) >> (16 * (b & 3))) & 0xffffu) != 0;
+  return __ballot_sync(0xffffffffu, ok);
+}
+
+// kMask (a padded grid): pooled keys without a real token are masked in the softmax of Eq. 6,
+// pooled query rows without one add nothing, and Eq. 7 averages over the tile's real query
+// sub-cubes (rows still sum to 1).
+template <int ND, bool kMask>
 __global__ void __launch_bounds__(RS_THREADS, 1)
     router_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                            float* __restrict__ scores, int Lr, int N, float c2, DevCtx ctx) {
+                            float* __restrict__ scores, int Lr, int N, float c2, const uint64_t* __restrict__ tmask,
+                            DevCtx ctx) {
   using SL = RouterSmem<ND>;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
@@ -190,7 +216,8 @@ __global__ void __launch_bounds__(RS_THREADS, 1)
         tmem_ld32(tmem + lane_off + st * RS_N + col0, r);
         tmem_ld_wait();
         const int key0 = it * RS_N + col0;
-        if (key0 + 32 <= Lr) {
+        const uint32_t kv = kMask ? piece_keys<true>(key0, Lr, tmask) : (key0 + 32 <= Lr ? 0xffffffffu : 0u);
+        if (kv == 0xffffffffu) {
           // full piece: max on the raw scores (c2 > 0), then one packed FMA per column pair
           float pm = __uint_as_float(r[0]);
 #pragma unroll
@@ -212,7 +239,8 @@ __global__ void __launch_bounds__(RS_THREADS, 1)
         float pm = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          x[j] = (key0 + j < Lr) ? __uint_as_float(r[j]) * c2 : -INFINITY;
+          const bool ok = kMask ? ((kv >> j) & 1u) : key0 + j < Lr;
+          x[j] = ok ? __uint_as_float(r[j]) * c2 : -INFINITY;
           pm = fmaxf(pm, x[j]);
         }
         const float mn = fmaxf(m, pm);
@@ -240,6 +268,16 @@ __global__ void __launch_bounds__(RS_THREADS, 1)
     const float lse2 = lse_sh[row];
     const int qtile = (m0 + row) >> 2;  // G = 4 pooled rows per tile
     const bool row_ok = qtile < N;
+    // kMask: this pooled query row counts only if its sub-cube holds a real token; the tile's
+    // score row is the mean over its real query sub-cubes (lanes 4g .. 4g+3 are tile g's rows)
+    float qw = 1.f, tile_inv = 1.f / kG;
+    if constexpr (kMask) {
+      const int a = m0 + row;
+      qw = (a < Lr && ((__ldg(tmask + (a >> 2)) >> (16 * (a & 3))) & 0xffffu)) ? 1.f : 0.f;
+      float gsum = qw + __shfl_xor_sync(0xffffffffu, qw, 1);
+      gsum += __shfl_xor_sync(0xffffffffu, gsum, 2);
+      tile_inv = gsum > 0.f ? 1.f / gsum : 0.f;
+    }
     float* out_row = scores + ((size_t)bh * N + (row_ok ? qtile : 0)) * N;
     for (int it = nchunk; it < 2 * nchunk; ++it) {
       const int st = it & 1, c = it - nchunk;
@@ -253,7 +291,8 @@ __global__ void __launch_bounds__(RS_THREADS, 1)
         tmem_ld32(tmem + lane_off + st * RS_N + col0, r);
         tmem_ld_wait();
         const int key0 = c * RS_N + col0;
-        if (key0 + 32 <= Lr) {
+        const uint32_t kv = kMask ? piece_keys<true>(key0, Lr, tmask) : (key0 + 32 <= Lr ? 0xffffffffu : 0u);
+        if (kv == 0xffffffffu) {
           // full piece: packed FMA for the exponent arguments and packed sums per key sub-cube
           const float2 cc = make_float2(c2, c2), nl = make_float2(-lse2, -lse2);
 #pragma unroll
@@ -273,7 +312,8 @@ __global__ void __launch_bounds__(RS_THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int j = 4 * jj + e;
-            acc += (key0 + j < Lr) ? ex2(__uint_as_float(r[j]) * c2 - lse2) : 0.f;
+            const bool ok = kMask ? ((kv >> j) & 1u) : key0 + j < Lr;
+            acc += ok ? ex2(__uint_as_float(r[j]) * c2 - lse2) : 0.f;
           }
           t[piece * 8 + jj] = acc;
         }
@@ -282,6 +322,10 @@ __global__ void __launch_bounds__(RS_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_sfree[st]);
       // sum over the G = 4 query sub-rows (lanes 4g..4g+3), reduce-scatter: lane keeps 8 tiles
+      if constexpr (kMask) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) t[j] *= qw;
+      }
       float u[16];
       const bool hi2 = lane & 2;
 #pragma unroll
@@ -296,7 +340,7 @@ __global__ void __launch_bounds__(RS_THREADS, 1)
       for (int j = 0; j < 8; ++j) {
         const float send = hi1 ? u[j] : u[8 + j];
         const float keep = hi1 ? u[8 + j] : u[j];
-        w[j] = (keep + __shfl_xor_sync(0xffffffffu, send, 1)) * (1.f / kG);
+        w[j] = (keep + __shfl_xor_sync(0xffffffffu, send, 1)) * tile_inv;
       }
       const int j0 = (c * RS_N + half * 128) / 4 + (hi2 ? 16 : 0) + (hi1 ? 8 : 0);
       if (row_ok) {
@@ -330,9 +374,12 @@ __global__ void __launch_bounds__(RS_THREADS, 1)
 // (b, h). Step 1: LSE of its G pooled query rows over all pooled keys. Step 2: one thread per
 // key tile sums exp(s - lse) over the G x G pooled pairs.
 // ------------------------------------------------------------------------------------------
+// tmask != nullptr (a padded grid): keys and query rows of sub-cubes without a real token are
+// left out, and the tile's score row is the mean over its real query sub-cubes.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) router_scores_simt_kernel(const T* __restrict__ qr, const T* __restrict__ kr,
-                                                                 float* __restrict__ scores, int Lr, int N) {
+                                                                 float* __restrict__ scores, int Lr, int N,
+                                                                 const uint64_t* __restrict__ tmask) {
   __shared__ float qs[kG][D];
   __shared__ float red_m[kG][128], red_l[kG][128];
   __shared__ float lse_s[kG];
@@ -345,7 +392,9 @@ __global__ void __launch_bounds__(128) router_scores_simt_kernel(const T* __rest
   float m[kG], l[kG];
 #pragma unroll
   for (int a = 0; a < kG; ++a) m[a] = -INFINITY, l[a] = 0.f;
+  auto key_ok = [&](int b) { return !tmask || ((tmask[b >> 2] >> (16 * (b & 3))) & 0xffffu) != 0; };
   for (int b = t; b < Lr; b += 128) {
+    if (!key_ok(b)) continue;
     float s[kG] = {};
     for (int d = 0; d < D; ++d) {
       const float kv = (float)kb[(size_t)b * D + d];
@@ -372,9 +421,17 @@ __global__ void __launch_bounds__(128) router_scores_simt_kernel(const T* __rest
     lse_s[t] = mm + __logf(ll);
   }
   __syncthreads();
+  const uint64_t qm = tmask ? tmask[i] : ~0ull;
+  float qw[kG], g = 0.f;
+#pragma unroll
+  for (int a = 0; a < kG; ++a) {
+    qw[a] = ((qm >> (16 * a)) & 0xffffu) ? 1.f : 0.f;
+    g += qw[a];
+  }
   for (int j = t; j < N; j += 128) {
     float acc = 0.f;
     for (int b = kG * j; b < kG * j + kG; ++b) {
+      if (!key_ok(b)) continue;
       float s[kG] = {};
       for (int d = 0; d < D; ++d) {
         const float kv = (float)kb[(size_t)b * D + d];
@@ -382,9 +439,9 @@ __global__ void __launch_bounds__(128) router_scores_simt_kernel(const T* __rest
         for (int a = 0; a < kG; ++a) s[a] += qs[a][d] * kv;
       }
 #pragma unroll
-      for (int a = 0; a < kG; ++a) acc += __expf(s[a] * scale - lse_s[a]);
+      for (int a = 0; a < kG; ++a) acc += qw[a] * __expf(s[a] * scale - lse_s[a]);
     }
-    scores[((size_t)bh * N + i) * N + j] = acc * (1.f / kG);
+    scores[((size_t)bh * N + i) * N + j] = acc / g;
   }
 }
 
@@ -399,12 +456,18 @@ vsa2_status launch_router(const Dims& d, const void* q, const void* k, float* sc
   const int cpr = d.D * d.esize / 16;
   const int64_t threads = 2 * pooled * cpr;
   const unsigned blocks = (unsigned)((threads + 255) / 256);
+  const uint64_t* tmask = nullptr;
+  if (d.padded) {
+    tmask = reinterpret_cast<const uint64_t*>(ws + w.tmask);
+    if (launch_tile_masks(d, reinterpret_cast<uint64_t*>(ws + w.tmask), s) != VSA2_OK) return VSA2_ERR_CUDA;
+  }
   if (d.dtype == VSA2_BF16) {
-    router_pool_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                                                             (__nv_bfloat16*)qr, (__nv_bfloat16*)kr, pooled, cpr);
+    auto kern = d.padded ? router_pool_kernel<__nv_bfloat16, true> : router_pool_kernel<__nv_bfloat16, false>;
+    kern<<<blocks, 256, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)qr,
+                                (__nv_bfloat16*)kr, pooled, cpr, tmask, d.Lr);
   } else {
-    router_pool_kernel<float><<<blocks, 256, 0, s>>>((const float*)q, (const float*)k, (float*)qr, (float*)kr,
-                                                     pooled, cpr);
+    auto kern = d.padded ? router_pool_kernel<float, true> : router_pool_kernel<float, false>;
+    kern<<<blocks, 256, 0, s>>>((const float*)q, (const float*)k, (float*)qr, (float*)kr, pooled, cpr, tmask, d.Lr);
   }
   if (check_launch(__func__) != VSA2_OK) return VSA2_ERR_CUDA;
 
@@ -415,20 +478,22 @@ vsa2_status launch_router(const Dims& d, const void* q, const void* k, float* sc
     const float c2 = 1.4426950408889634f / sqrtf((float)d.D);
     dim3 grid((d.Lr + RS_M - 1) / RS_M, d.BH);
     if (d.D == 128) {
-      auto kern = router_scores_tc_kernel<2>;
+      auto kern = d.padded ? router_scores_tc_kernel<2, true> : router_scores_tc_kernel<2, false>;
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, RouterSmem<2>::kDyn);
-      kern<<<grid, RS_THREADS, RouterSmem<2>::kDyn, s>>>(tq, tk, scores, d.Lr, d.N, c2, ctx);
+      kern<<<grid, RS_THREADS, RouterSmem<2>::kDyn, s>>>(tq, tk, scores, d.Lr, d.N, c2, tmask, ctx);
     } else {
-      auto kern = router_scores_tc_kernel<1>;
+      auto kern = d.padded ? router_scores_tc_kernel<1, true> : router_scores_tc_kernel<1, false>;
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, RouterSmem<1>::kDyn);
-      kern<<<grid, RS_THREADS, RouterSmem<1>::kDyn, s>>>(tq, tk, scores, d.Lr, d.N, c2, ctx);
+      kern<<<grid, RS_THREADS, RouterSmem<1>::kDyn, s>>>(tq, tk, scores, d.Lr, d.N, c2, tmask, ctx);
     }
   } else {
     dim3 grid(d.N, d.BH);
     if (d.D == 128)
-      router_scores_simt_kernel<float, 128><<<grid, 128, 0, s>>>((const float*)qr, (const float*)kr, scores, d.Lr, d.N);
+      router_scores_simt_kernel<float, 128><<<grid, 128, 0, s>>>((const float*)qr, (const float*)kr, scores, d.Lr, d.N,
+                                                                 tmask);
     else
-      router_scores_simt_kernel<float, 64><<<grid, 128, 0, s>>>((const float*)qr, (const float*)kr, scores, d.Lr, d.N);
+      router_scores_simt_kernel<float, 64><<<grid, 128, 0, s>>>((const float*)qr, (const float*)kr, scores, d.Lr, d.N,
+                                                                tmask);
   }
   if (check_launch(__func__) != VSA2_OK) return VSA2_ERR_CUDA;
   return VSA2_OK;
