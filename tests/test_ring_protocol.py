@@ -5,8 +5,9 @@ An mbarrier parity wait can only tell the phase in progress from the one just co
 waiter two phases behind waits forever, and a waiter one phase ahead passes early. The model
 checks, at every poll, that the awaited phase is one of those two, and that every schedule
 finishes (no deadlock). The agents follow the kernel's protocol:
-  * the producer walks the slot's ops (S0, S1, O0, S2, O1, ... per query tile) and loads K for an
-    S op and V for an O op into ring position c % RST, after the release of position c - RST;
+  * the producer walks the slot's ops (S0, S1, S2, O0, S3, O1, ... per query tile: S runs two
+    blocks ahead of O) and loads K for an S op and V for an O op into ring position c % RST,
+    after the release of position c - RST;
   * the MMA issuer waits for the block in the ring, and for an S op also for the S buffer
     (two buffers, freed by the softmax), for an O op also for P (written by the softmax); the
     MMA's completion releases the ring position and signals S (sfull) or P.V done (pvdone);
@@ -38,13 +39,14 @@ class Barrier:
         return self.phases >= phase + 1
 
 
-def ops_of(tiles):
-    """The slot's op stream: for a tile of n blocks, S0, S1, O0, S2, O1, ..., O(n-1)."""
+def ops_of(tiles, lead=2):
+    """The slot's op stream: for a tile of n blocks, S(k) goes before O(k - lead); the kernel's
+    lead is 2 (S0, S1, S2, O0, S3, O1, ..., O(n-1)), lead 1 was its earlier order."""
     out = []
     for n in tiles:
         s = o = 0
         while o < n:
-            if s < n and s <= o + 1:
+            if s < n and s <= o + lead:
                 out.append(("S", s))
                 s += 1
             else:
@@ -53,8 +55,8 @@ def ops_of(tiles):
     return out
 
 
-def run(tiles, rst, producers, rng, mma_latency=3):
-    ops = ops_of(tiles)
+def run(tiles, rst, producers, rng, mma_latency=3, lead=2):
+    ops = ops_of(tiles, lead)
     full = [Barrier(producers) for _ in range(rst)]
     empty = [Barrier(1) for _ in range(rst)]
     sfull, sfree = [Barrier(1), Barrier(1)], [Barrier(1), Barrier(1)]
@@ -143,17 +145,20 @@ def run(tiles, rst, producers, rng, mma_latency=3):
     assert pvdone.phases == sum(tiles) and all(p == len(ops) for p in prod)
 
 
-@pytest.mark.parametrize("producers", [1, 2], ids=["kernel", "two_producers"])
+@pytest.mark.parametrize("lead", [2, 1], ids=["kernel", "lead1"])
+@pytest.mark.parametrize("producers", [1, 2], ids=["one_producer", "two_producers"])
 @pytest.mark.parametrize("seed", range(60))
-def test_ring_protocol_parity_and_progress(producers, seed):
+def test_ring_protocol_parity_and_progress(lead, producers, seed):
     rng = random.Random(seed)
     tiles = [rng.choice([1, 1, 2, 3, 4, 5, 7, 32]) for _ in range(rng.randint(1, 6))]
-    run(tiles, rst=3, producers=producers, rng=rng, mma_latency=rng.choice([1, 3, 10]))
+    run(tiles, rst=3, producers=producers, rng=rng, mma_latency=rng.choice([1, 3, 10]), lead=lead)
 
 
 def test_op_order_matches_the_kernel_stream():
-    assert ops_of([3]) == [("S", 0), ("S", 1), ("O", 0), ("S", 2), ("O", 1), ("O", 2)]
+    assert ops_of([4]) == [("S", 0), ("S", 1), ("S", 2), ("O", 0), ("S", 3), ("O", 1), ("O", 2), ("O", 3)]
     assert ops_of([1, 2]) == [("S", 0), ("O", 0), ("S", 0), ("S", 1), ("O", 0), ("O", 1)]
+    assert ops_of([3], lead=1) == [("S", 0), ("S", 1), ("O", 0), ("S", 2), ("O", 1), ("O", 2)]
+
 
 
 def run_dkdv(items, rng, rst=6, mma_latency=3):
