@@ -146,6 +146,185 @@ def run(tiles, rst, producers, rng, mma_latency=3, lead=1):
     assert pvdone.phases == sum(tiles) and all(p == len(ops) for p in prod)
 
 
+def run_aliased(tiles, rst, rng, mma_latency=3, rescale_p=0.2, lead=1):
+    """The forward kernel's protocol with P written over the S buffer it came from: per slot two
+    S/P buffers, pfull and pvdone per block parity, no wait for the previous P.V before writing P;
+    the softmax waits for the previous P.V only to rescale O (at random here) and at a tile's end.
+    The tensor pipe completes MMAs in issue order. Asserts, besides the parity rule, that S(k)
+    overwrites a buffer only after O(k-2) read its P, that P(g) is written only after O(g-2)
+    read the previous P of the buffer, and that O is read only after every P.V issued before."""
+    ops = ops_of(tiles, lead=lead)
+    full = [Barrier(1) for _ in range(rst)]
+    empty = [Barrier(1) for _ in range(rst)]
+    sfull, sfree = [Barrier(1), Barrier(1)], [Barrier(1), Barrier(1)]
+    pfull, pvdone = [Barrier(4), Barrier(4)], [Barrier(1), Barrier(1)]
+    for b in pfull:
+        b.count = 1  # one arrival stands for the four softmax warps
+    prod = {"c": 0}
+    mma = {"c": 0, "s": 0, "o": 0}
+    soft = {"blk": 0, "step": 0, "tile": 0, "in_tile": 0}
+    done = {"op": set(), "s": set(), "o": set()}
+    p_written = set()
+    ends = []                      # block index that ends each tile
+    acc = 0
+    for n in tiles:
+        acc += n
+        ends.append(acc - 1)
+    nblk = acc
+    pipe = {"last": 0}
+    pending = []
+    t = 0
+
+    def producer():
+        c = prod["c"]
+        if c >= len(ops):
+            return False
+        st = c % rst
+        if not empty[st].poll(c // rst - 1, f"producer at {c}"):
+            return False
+        assert c < rst or c - rst in done["op"], f"ring position {c} refilled before its MMA finished"
+        full[st].arrive()
+        prod["c"] += 1
+        return True
+
+    def issuer():
+        c = mma["c"]
+        if c >= len(ops):
+            return False
+        st = c % rst
+        if not full[st].poll(c // rst, f"issuer at {c}"):
+            return False
+        kind, _ = ops[c]
+        if kind == "S":
+            k = mma["s"]
+            if not sfree[k % 2].poll(k // 2 - 1, f"issuer S{k}"):
+                return False
+
+            def fin(c=c, k=k, st=st):
+                assert k < 2 or k - 2 in done["o"], f"S{k} overwrote P{k - 2} before O{k - 2} read it"
+                done["op"].add(c)
+                done["s"].add(k)
+                empty[st].arrive()
+                sfull[k % 2].arrive()
+            mma["s"] += 1
+        else:
+            k = mma["o"]
+            if not pfull[k % 2].poll(k // 2, f"issuer O{k}"):
+                return False
+            assert k in p_written
+
+            def fin(c=c, k=k, st=st):
+                done["op"].add(c)
+                done["o"].add(k)
+                empty[st].arrive()
+                pvdone[k % 2].arrive()
+            mma["o"] += 1
+        pipe["last"] = max(pipe["last"], t) + rng.randint(1, mma_latency)  # in order
+        pending.append((pipe["last"], fin))
+        mma["c"] += 1
+        return True
+
+    def wait_pv(g, who):
+        return pvdone[g % 2].poll(g // 2, who)
+
+    def softmax():
+        g = soft["blk"]
+        if g >= nblk:
+            return False
+        st = soft["step"]
+        if st == 0:                       # wait S, read it, free the buffer
+            if not sfull[g % 2].poll(g // 2, f"softmax S{g}"):
+                return False
+            assert g in done["s"]
+            sfree[g % 2].arrive()
+            first = g == 0 or (g - 1) in ends
+            soft["step"] = 1 if (not first and rng.random() < rescale_p) else 2
+            return True
+        if st == 1:                       # rescale O: the previous P.V must be done
+            if not wait_pv(g - 1, f"softmax rescale at {g}"):
+                return False
+            assert all(x in done["o"] for x in range(g)), f"O read at block {g} with a P.V pending"
+            soft["step"] = 2
+            return True
+        if st == 2:                       # write P over the S buffer
+            assert g < 2 or g - 2 in done["o"], f"P{g} written before O{g - 2} read P{g - 2}"
+            p_written.add(g)
+            pfull[g % 2].arrive()
+            soft["step"] = 3 if g in ends else 0
+            if g not in ends:
+                soft["blk"] = g + 1
+            return True
+        if not wait_pv(g, f"softmax epilogue at {g}"):  # st == 3: tile's last P.V, then O
+            return False
+        assert all(x in done["o"] for x in range(g + 1)), f"epilogue at {g} with a P.V pending"
+        soft["blk"], soft["step"] = g + 1, 0
+        return True
+
+    agents = [producer, issuer, softmax]
+    speed = [rng.uniform(0.05, 1.0) for _ in agents]
+    while mma["c"] < len(ops) or soft["blk"] < nblk or pending:
+        t += 1
+        due = [x for x in pending if x[0] <= t]
+        pending[:] = [x for x in pending if x[0] > t]
+        for _, f in sorted(due, key=lambda x: x[0]):
+            f()
+        moved = bool(due)
+        for i in rng.sample(range(len(agents)), len(agents)):
+            if rng.random() < speed[i]:
+                moved |= agents[i]()
+        if not moved and not pending and not any(a() for a in agents):
+            raise AssertionError(f"deadlock at op {mma['c']} of {len(ops)}, softmax block {soft['blk']}")
+    assert len(done["o"]) == nblk
+
+
+@pytest.mark.parametrize("seed", range(80))
+def test_forward_protocol_with_p_over_s(seed):
+    rng = random.Random(seed)
+    tiles = [rng.choice([1, 1, 2, 3, 4, 5, 7, 32]) for _ in range(rng.randint(1, 6))]
+    run_aliased(tiles, rst=3, rng=rng, mma_latency=rng.choice([1, 3, 10, 30]))
+
+
+def test_forward_protocol_flags_a_single_pfull_barrier():
+    """With one pfull barrier instead of one per block parity, the softmax can complete the
+    phase of block n+1 before the issuer waited for block n's: the parity rule flags it."""
+    with pytest.raises(AssertionError):
+        for seed in range(200):
+            _run_single_pfull([32, 32, 5], random.Random(seed))
+
+
+def test_forward_protocol_flags_lead_two_with_p_over_s():
+    """S two blocks ahead would overwrite P(k-2) before O(k-2) read it: the model flags it."""
+    with pytest.raises(AssertionError):
+        for seed in range(50):
+            run_aliased([32, 7], rst=3, rng=random.Random(seed), mma_latency=10, lead=2)
+
+
+def _run_single_pfull(tiles, rng):
+    """The kernel's earlier single pfull barrier (count: one per block), with P over S and no
+    wait for the previous P.V before writing P."""
+    ops = ops_of(tiles, lead=1)
+    pf = Barrier(1)
+    s_done = set()
+    mma_o = 0
+    soft_g = 0
+    nblk = sum(tiles)
+    issued_s = 0
+    t = 0
+    # a minimal schedule: S ops complete at once; the issuer is slow, the softmax fast
+    while soft_g < nblk:
+        t += 1
+        if issued_s < nblk and issued_s <= mma_o + 1:
+            s_done.add(issued_s)
+            issued_s += 1
+        if soft_g in s_done and rng.random() < 0.9:
+            pf.arrive()
+            soft_g += 1
+        if rng.random() < 0.05 and mma_o < soft_g:
+            if pf.poll(mma_o, f"issuer O{mma_o}"):
+                mma_o += 1
+    return True
+
+
 @pytest.mark.parametrize("lead", [1, 2], ids=["kernel", "lead2"])
 @pytest.mark.parametrize("producers", [1, 2], ids=["one_producer", "two_producers"])
 @pytest.mark.parametrize("seed", range(60))

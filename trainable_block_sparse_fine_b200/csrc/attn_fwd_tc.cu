@@ -40,28 +40,35 @@ constexpr int FT = 384;            // 12 warps
 constexpr uint32_t TILE_B = 8192;  // one 64x64 bf16 box (64 rows x 128 B)
 constexpr uint32_t BLK_B = 32768;  // K or V block: [half0: tile A, tile B][half1: tile A, tile B]
 constexpr int RST = 3;             // ring stages per slot (K and V blocks in op order)
+constexpr int kLead = 1;           // S(k) is issued before O(k - 1) and after O(k - 2), which reads
+                                   // the P that S(k) overwrites: the lead must stay 1
 
 // Each slot has its own ring (one producer, one consumer, both in the slot's op order), so
 // every barrier wait is for the phase in progress or the one just completed.
 constexpr uint32_t OFF_RING = 0;                           // [slot][RST] blocks
-constexpr uint32_t OFF_BAR = OFF_RING + 2 * RST * BLK_B;
+constexpr int IDXCAP = 256;                                // KV indices of a row kept in shared memory
+constexpr uint32_t OFF_IDX = OFF_RING + 2 * RST * BLK_B;   // [slot][2 rows][IDXCAP] int32
+constexpr uint32_t OFF_BAR = OFF_IDX + 2 * 2 * IDXCAP * 4;
 constexpr uint32_t OFF_FLAG = OFF_BAR + 512;
 constexpr uint32_t SMEM_USED = OFF_FLAG + 64;
 constexpr uint32_t SMEM_DYN = SMEM_USED + 1024;
 static_assert(SMEM_DYN <= 232448, "shared memory budget");
 
-// TMEM columns (each region used by both slots through the lane halves)
-constexpr uint32_t TM_S = 0;      // two S buffers of 128 fp32 columns
-constexpr uint32_t TM_P = 256;    // P: 128 bf16 = 64 columns
-constexpr uint32_t TM_Q = 320;    // Q: 128 bf16 = 64 columns
-constexpr uint32_t TM_O = 384;    // O: 128 fp32 columns
+// TMEM columns (each region used by both slots through the lane halves). The softmax writes
+// P(n) as bf16 over the first 64 columns of the S buffer it read S(n) from, so P is double
+// buffered with S: the softmax of block n+1 never waits for the P.V MMA of block n. S(n+2)
+// overwrites that buffer only after O(n) has read P(n): the MMA issuer issues S(n+2) after O(n),
+// and the tensor pipe runs one thread's MMAs in order.
+constexpr uint32_t TM_S = 0;      // two S / P buffers of 128 fp32 columns
+constexpr uint32_t TM_Q = 256;    // Q: 128 bf16 = 64 columns
+constexpr uint32_t TM_O = 320;    // O: 128 fp32 columns
 constexpr uint32_t TM_COLS = 512;
 constexpr float kThresh = 8.0f;   // log2 headroom before the running max must move
 
 struct Bars {
   uint64_t full[2][RST], empty[2][RST];                                    // [slot][stage]
   uint64_t sfull[2][2], sfree[2][2];                                       // [slot][buffer]
-  uint64_t pfull[2], pvdone[2], qready[2];
+  uint64_t pfull[2][2], pvdone[2][2], qready[2];  // pfull, pvdone: [slot][block parity]
   uint64_t done[2];
 };
 static_assert(sizeof(Bars) <= 512, "barrier area");
@@ -105,7 +112,7 @@ struct SlotSeq {
 __device__ __forceinline__ int next_op(SlotSeq& q, int* blk, const int32_t* kv_off, int N, int cap,
                                        const DevCtx& ctx) {
   while (q.active) {
-    if (q.s_next < q.nblk && q.s_next <= q.o_next + 1) {
+    if (q.s_next < q.nblk && q.s_next <= q.o_next + kLead) {
       *blk = q.s_next++;
       return 1;
     }
@@ -152,8 +159,10 @@ __global__ void __launch_bounds__(FT, 1)
     for (int s = 0; s < 2; ++s) {
       for (int i = 0; i < RST; ++i) mbar_init(&B.full[s][i], 1), mbar_init(&B.empty[s][i], 1);
       for (int b = 0; b < 2; ++b) mbar_init(&B.sfull[s][b], 1), mbar_init(&B.sfree[s][b], 4);
-      mbar_init(&B.pfull[s], 4);
-      mbar_init(&B.pvdone[s], 1);
+      mbar_init(&B.pfull[s][0], 4);
+      mbar_init(&B.pfull[s][1], 4);
+      mbar_init(&B.pvdone[s][0], 1);
+      mbar_init(&B.pvdone[s][1], 1);
       mbar_init(&B.qready[s], 4);
     }
     mbar_init(&B.done[0], 1);
@@ -171,45 +180,85 @@ __global__ void __launch_bounds__(FT, 1)
 
   if (warp == 8 || warp == 10) {
     // ------------------------------------------------------------------ TMA producer of slot (warp - 8) / 2
-    // K blocks for the slot's S ops and V blocks for its O ops, in the slot's op order, one thread
+    // K blocks for the slot's S ops and V blocks for its O ops, in the slot's op order. The whole
+    // warp copies each item's KV indices into shared memory (cp.async) one item ahead, and its
+    // row offsets two items ahead, so that lane 0, which issues the copies, never waits for a
+    // global load on its way from one op to the next.
+    const int s = (warp - 8) >> 1;
+    int32_t* ibuf = reinterpret_cast<int32_t*>(dsm + OFF_IDX) + s * 2 * IDXCAP;
     if (lane == 0) {
-      const int s = (warp - 8) >> 1;
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      SlotSeq sq;
-      sq.init(2 * blockIdx.x + s, step, items);
-      int c = 0;  // ring position: blocks requested so far
-      bool ok = true;
-      while (ok && sq.active) {
-        int blk;
-        const int op = next_op(sq, &blk, kv_off, N, cap, ctx);
-        if (op == 0) continue;
-        const bool k_op = op == 1;
-        const int ntile = min(2, sq.len - 2 * blk);
-        int j[2] = {0, 0};
-        for (int tt = 0; tt < ntile; ++tt) {
-          int v = kv_idx[(size_t)sq.bh * cap + sq.beg + 2 * blk + tt];
-          if (v < 0 || v >= N) {
-            if (ctx.flags & VSA2_FLAG_VALIDATE) set_error(ctx.err, VSA2_ERR_BAD_INDEX);
-            v = min(max(v, 0), N - 1);
+    }
+    auto row_of = [&](int it) { return it < items ? load_row(kv_off, it / N, it % N, N, cap, ctx, false) : Row{0, 0}; };
+    auto copy_row = [&](int it, const Row& r, int b) {  // whole warp
+      const int32_t* src = kv_idx + (size_t)(it / N) * cap + r.beg;
+      const int n = min(r.len, IDXCAP);
+      for (int e = lane; e < n; e += 32)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(ibuf + b * IDXCAP + e)), "l"(src + e)
+                     : "memory");
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    int item = 2 * blockIdx.x + s;
+    Row cur = row_of(item);
+    if (item < items) copy_row(item, cur, 0);
+    Row nxt = row_of(item + step);
+    int c = 0;  // ring position: blocks requested so far
+    bool ok = true;
+    for (int b = 0; ok && item < items; item += step, b ^= 1) {
+      asm volatile("cp.async.wait_all;" ::: "memory");  // this item's indices (copied an item ago)
+      __syncwarp();
+      if (item + step < items && nxt.len > 0) copy_row(item + step, nxt, b ^ 1);
+      const Row nn = row_of(item + 2 * step);  // used when the next item starts
+      if (lane == 0) {
+        const int bh = item / N;
+        const int32_t* gidx = kv_idx + (size_t)bh * cap + cur.beg;
+        const int32_t* sidx = ibuf + b * IDXCAP;
+        const int nblk = (cur.len + 1) >> 1;
+        int s_next = 0, o_next = 0;
+        while (o_next < nblk) {
+          int blk;
+          bool k_op;
+          if (s_next < nblk && s_next <= o_next + kLead) {
+            blk = s_next++;
+            k_op = true;
+          } else {
+            blk = o_next++;
+            k_op = false;
           }
-          j[tt] = v;
+          const int ntile = min(2, cur.len - 2 * blk);
+          int j[2] = {0, 0};
+#pragma unroll
+          for (int tt = 0; tt < 2; ++tt) {
+            if (tt >= ntile) break;
+            const int e = 2 * blk + tt;
+            int v = e < IDXCAP ? sidx[e] : gidx[e];
+            if (v < 0 || v >= N) {
+              if (ctx.flags & VSA2_FLAG_VALIDATE) set_error(ctx.err, VSA2_ERR_BAD_INDEX);
+              v = min(max(v, 0), N - 1);
+            }
+            j[tt] = v;
+          }
+          const int st = c % RST;
+          uint64_t* full = &B.full[s][st];
+          uint8_t* dst = dsm + OFF_RING + (s * RST + st) * BLK_B;
+          if (!(ok = mbar_wait(&B.empty[s][st], ((c / RST) & 1) ^ 1, abort, ctx))) break;
+          mbar_arrive_expect_tx(full, ntile * 2 * TILE_B);
+          for (int tt = 0; tt < ntile; ++tt)
+            for (int h = 0; h < 2; ++h)
+              tma_load_2d(dst + h * 2 * TILE_B + tt * TILE_B, k_op ? &tm_k : &tm_v, h * 64, bh * L + j[tt] * 64,
+                          full);
+          ++c;
         }
-        const int st = c % RST;
-        uint64_t* full = &B.full[s][st];
-        uint8_t* dst = dsm + OFF_RING + (s * RST + st) * BLK_B;
-        if (!(ok = mbar_wait(&B.empty[s][st], ((c / RST) & 1) ^ 1, abort, ctx))) break;
-        mbar_arrive_expect_tx(full, ntile * 2 * TILE_B);
-        for (int tt = 0; tt < ntile; ++tt)
-          for (int h = 0; h < 2; ++h)
-            tma_load_2d(dst + h * 2 * TILE_B + tt * TILE_B, k_op ? &tm_k : &tm_v, h * 64, sq.bh * L + j[tt] * 64,
-                        full);
-        ++c;
       }
-      if (*abort) {  // let copies still in flight land before the CTA exits
-        for (int cc = max(0, c - RST); cc < c; ++cc)
-          mbar_wait_drain(&B.full[s][cc % RST], (cc / RST) & 1, ctx.timeout_ns);
-      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      cur = nxt;
+      nxt = nn;
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // no copy outlives the CTA
+    if (lane == 0 && *abort) {  // let copies still in flight land before the CTA exits
+      for (int cc = max(0, c - RST); cc < c; ++cc)
+        mbar_wait_drain(&B.full[s][cc % RST], (cc / RST) & 1, ctx.timeout_ns);
     }
   } else if (warp == 9 || warp == 11) {
     // ------------------------------------------------------------------ MMA issuer of slot (warp - 9) / 2
@@ -244,15 +293,15 @@ __global__ void __launch_bounds__(FT, 1)
         } else if (op == 2) {
           const int st = c % RST;
           if (!(ok = mbar_wait(&B.full[s][st], (c / RST) & 1, abort, ctx))) break;
-          if (!(ok = mbar_wait(&B.pfull[s], vc & 1, abort, ctx))) break;
+          if (!(ok = mbar_wait(&B.pfull[s][vc & 1], (vc >> 1) & 1, abort, ctx))) break;
           tc_fence_after();
           const uint32_t va = smem_u32(dsm + OFF_RING + (s * RST + st) * BLK_B);
           const int ksteps = (2 * blk + 1 == sq.len) ? 4 : 8;
           for (int kk = 0; kk < ksteps; ++kk)
-            mma_bf16_ts(tmem + lanes + TM_O, tmem + lanes + TM_P + 8 * kk,
+            mma_bf16_ts(tmem + lanes + TM_O, tmem + lanes + TM_S + (vc & 1) * 128 + 8 * kk,
                         sdesc_sw128(va + kk * 2048, 2 * TILE_B, 1024), id_o, (blk > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&B.empty[s][st]);
-          mma_commit(&B.pvdone[s]);
+          mma_commit(&B.pvdone[s][vc & 1]);
           ++vc;
           ++c;
         }
@@ -351,7 +400,7 @@ __global__ void __launch_bounds__(FT, 1)
         }
         if (__any_sync(0xffffffffu, raise && n > 0)) {
           // O holds blocks 0..n-1 of this tile: scale the raised rows once the last O MMA is done
-          mbar_wait(&B.pvdone[s], (g - 1) & 1, abort, ctx);
+          mbar_wait(&B.pvdone[s][(g - 1) & 1], ((g - 1) >> 1) & 1, abort, ctx);
           tc_fence_after();
           uint32_t o[64];
           tmem_ld16x64b_x64(tl + TM_O, o);
@@ -379,16 +428,15 @@ __global__ void __launch_bounds__(FT, 1)
           pk[i2] = pair_pack_bf16(pa, pb, perm);
         }
         l += ls.x + ls.y;
-        // P region is free once the O MMA of the previous block has finished
-        if (n > 0) mbar_wait(&B.pvdone[s], (g - 1) & 1, abort, ctx);
-        tmem_st16x64b_x32(tl + TM_P, pk);
+        // P over the S buffer just read (its S values are in registers)
+        tmem_st16x64b_x32(tl + TM_S + (g & 1) * 128, pk);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&B.pfull[s]);
+        if (lane == 0) mbar_arrive(&B.pfull[s][g & 1]);
       }
       // ---- epilogue: last O block done -> normalise and store
-      mbar_wait(&B.pvdone[s], (g - 1) & 1, abort, ctx);
+      mbar_wait(&B.pvdone[s][(g - 1) & 1], ((g - 1) >> 1) & 1, abort, ctx);
       tc_fence_after();
       l += __shfl_xor_sync(0xffffffffu, l, 2);
       float inv = 1.f / l;
