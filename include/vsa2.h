@@ -137,6 +137,24 @@ vsa2_status vsa2_sparse_attn_fwd(const vsa2_problem* p, const void* q, const voi
                                  void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * The fine branch of Eq. 12 with the gated merge of Eq. 13-14 in the same pass (§2.2 "Gated
+ * Merge"): o = tanh(gate_logits) * Repeat_B(oc) + O_f, where O_f is what vsa2_sparse_attn_fwd
+ * computes, without writing O_f and reading it back.
+ *   q, k, v, topk, kv_off, kv_idx, lse : as for vsa2_sparse_attn_fwd (lse is the fine branch's)
+ *   gate_logits : [batch, heads, L] fp32, the per-token logits X W_g of Eq. 13 (read only)
+ *   oc          : [batch, heads, N, D] of dtype, the coarse output from vsa2_coarse_attn (read only)
+ *   o           : [batch, heads, L, D] of dtype (written); must not alias q, k, v or o_f
+ *   o_f         : NULL, or [batch, heads, L, D] of dtype receiving O_f (the backward forms
+ *                 rowsum(dO * O_f) from it)
+ * The merge is applied to O_f before its rounding to dtype. A tile with an empty list gets
+ * o = tanh(g) * oc[tile], O_f = 0 and lse = -inf.
+ */
+vsa2_status vsa2_sparse_attn_fwd_gated(const vsa2_problem* p, const void* q, const void* k, const void* v,
+                                       int32_t topk, const int32_t* kv_off, const int32_t* kv_idx,
+                                       const float* gate_logits, const void* oc, void* o, float* lse, void* o_f,
+                                       void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Block-sparse attention backward (gradients of Eq. 12; the router receives none, §2.1).
  *   q, k, v, o, dout : [batch, heads, L, D] of dtype (read only); o and lse from the forward
  *   lse              : [batch, heads, L] fp32 (read only)

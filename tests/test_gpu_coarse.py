@@ -152,6 +152,49 @@ def test_attention_output_is_the_gated_sum_of_both_branches():
             _close(o[b, h], O.gated_merge(o_f, oc, logits[b, h]), f"o[{b},{h}]")
 
 
+@pytest.mark.parametrize("case", ["ragged_tail", "one_padded_tile", "d64_bf16", "fp32_d128_ragged"])
+def test_fine_forward_with_fused_gate(case):
+    """vsa2_sparse_attn_fwd_gated: O_f equals the plain forward bit for bit, LSE too, and the
+    gated output equals the oracle's Eq. 14 (fine branch on the same selection, merge with the
+    GPU's coarse output and logits) within the attention tolerance. Rows with an empty list get
+    the coarse term alone. The tensor-core path merges in the epilogue; the CUDA-core shapes (fp32,
+    head_dim 64) run the forward and then the merge kernel."""
+    wl = CASES[case]
+    x = {n: S.make_tensor(wl, n) for n in "qkv"}
+    rng = np.random.default_rng(46)
+    logits = (rng.standard_normal((wl.batch, wl.heads, wl.tokens)) * 1.5).astype(np.float32)
+    e = _engine(wl)
+    xd = {n: _dev(x[n], wl.dtype) for n in "qkv"}
+    kv_off, kv_idx, _, _ = e.topk_select(e.router_scores(xd["q"], xd["k"]), wl.topk, csc=False)
+    off, idx = kv_off.cpu().numpy(), kv_idx.cpu().numpy()
+    # query tile 1 of head (0, 0) loses its list: an empty row
+    N = wl.num_tiles
+    rows = [idx[0, 0, off[0, 0, i]:off[0, 0, i + 1]] for i in range(N)]
+    rows[1] = rows[1][:0]
+    kv_off_np, kv_idx_np = off.copy(), idx.copy()
+    kv_off_np[0, 0, 1:] = np.cumsum([len(r) for r in rows])
+    flat = np.concatenate(rows)
+    kv_idx_np[0, 0, :] = 0
+    kv_idx_np[0, 0, :flat.size] = flat
+    kv_off_d, kv_idx_d = torch.from_numpy(kv_off_np).cuda(), torch.from_numpy(kv_idx_np).cuda()
+    oc, _ = e.coarse_attn(xd["q"], xd["k"], xd["v"])
+    o_plain, lse_plain = e.attn_fwd(xd["q"], xd["k"], xd["v"], kv_off_d, kv_idx_d)
+    o, lse, o_f = e.attn_fwd_gated(xd["q"], xd["k"], xd["v"], kv_off_d, kv_idx_d, torch.from_numpy(logits).cuda(),
+                                   oc, want_fine=True)
+    assert e.device_error() == 0
+    assert torch.equal(o_f, o_plain) and torch.equal(lse, lse_plain)
+    got = o.float().cpu().numpy()
+    oc_np = oc.float().cpu().numpy()
+    for b in range(wl.batch):
+        for h in range(wl.heads):
+            fine, _ = O.sparse_attn_fwd(x["q"][b, h], x["k"][b, h], x["v"][b, h], kv_off_np[b, h], kv_idx_np[b, h])
+            want = O.gated_merge(fine, oc_np[b, h], logits[b, h])
+            _close(got[b, h], want, f"{case} gated o[{b},{h}]")
+    # query tile 1 of head 0 has no KV tile: its rows are tanh(g) * oc[1]
+    np.testing.assert_allclose(got[0, 0, 64:128], np.tanh(logits[0, 0, 64:128])[:, None] * oc_np[0, 0, 1][None, :],
+                               atol=1e-2, rtol=1e-2)
+
+
 # ------------------------------------------------------------------------------------------
 # gradients
 # ------------------------------------------------------------------------------------------

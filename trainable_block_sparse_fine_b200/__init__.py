@@ -14,7 +14,8 @@ import torch
 from ._capi import (VSA2_FLAG_VALIDATE, Problem, Vsa2Error, lib, make_problem, vsa2_coarse_attn,
                     vsa2_coarse_attn_bwd, vsa2_forward_host, vsa2_forward_host_workspace_size, vsa2_gated_merge,
                     vsa2_gated_merge_bwd, vsa2_get_device_error, vsa2_permute_tokens, vsa2_router_scores,
-                    vsa2_selftest_wait_timeout, vsa2_sparse_attn_bwd, vsa2_sparse_attn_fwd, vsa2_status_string,
+                    vsa2_selftest_wait_timeout, vsa2_sparse_attn_bwd, vsa2_sparse_attn_fwd,
+                    vsa2_sparse_attn_fwd_gated, vsa2_status_string,
                     vsa2_topk_select, vsa2_topk_select_per_row, vsa2_version, vsa2_workspace_init, vsa2_workspace_size)
 
 from .ulysses import heads_to_seq, seq_to_heads, ulysses_attention
@@ -31,19 +32,23 @@ class VSA2:
     """One problem shape with its workspace; methods enqueue on the current CUDA stream."""
 
     def __init__(self, batch, heads, head_dim, grid, dtype="bf16", topk=64, device="cuda", flags=0,
-                 wait_timeout_ms=0):
+                 wait_timeout_ms=0, tile=(4, 4, 4), pool=(2, 2, 4)):
+        """tile / pool: the token cube of a tile and of a router sub-cube, 64 / 16 tokens (the
+        pages' shapes, default) or 128 / 8 tokens (e.g. (4, 4, 8) / (2, 2, 2))."""
         if not torch.cuda.is_available():
             raise RuntimeError("VSA2 needs a CUDA device")
         lib()  # fail loudly if the native library is missing
-        self.p = make_problem(batch, heads, head_dim, grid, dtype, flags=flags, wait_timeout_ms=wait_timeout_ms)
+        self.p = make_problem(batch, heads, head_dim, grid, dtype, tile=tuple(tile), pool=tuple(pool), flags=flags,
+                              wait_timeout_ms=wait_timeout_ms)
+        self.tile, self.pool = tuple(tile), tuple(pool)
         self.batch, self.heads, self.head_dim, self.grid, self.topk = batch, heads, head_dim, tuple(grid), topk
         # a grid the 4x4x4 tile does not divide is padded to whole tiles (§2.2 "Kernel
         # Implementation"): every [B, H, L, D] tensor of the path holds the padded grid in
         # cube-major order; to_cube_major / to_raster pad and crop
         self.L_real = grid[0] * grid[1] * grid[2]
-        self.grid_padded = tuple(-(-g // 4) * 4 for g in grid)
+        self.grid_padded = tuple(-(-g // b) * b for g, b in zip(grid, self.tile))
         self.L = self.grid_padded[0] * self.grid_padded[1] * self.grid_padded[2]
-        self.N = self.L // 64
+        self.N = self.L // (self.tile[0] * self.tile[1] * self.tile[2])
         self.dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
         self.device = torch.device(device)
         n = vsa2_workspace_size(self.p, topk)
@@ -89,6 +94,16 @@ class VSA2:
                                                       device=self.device)
         vsa2_sparse_attn_fwd(self.p, q, k, v, topk, kv_off, kv_idx, o, lse, self.ws)
         return o, lse
+
+    def attn_fwd_gated(self, q, k, v, kv_off, kv_idx, gate_logits, oc, topk=None, want_fine=False):
+        """Eq. 12 with the gated merge of Eq. 13-14 in the same pass: returns (o, lse, o_f), o_f the
+        fine output alone when want_fine (the backward needs it), else None."""
+        topk = self.topk if topk is None else topk
+        o = torch.empty_like(q)
+        lse = torch.empty(self.batch, self.heads, self.L, dtype=torch.float32, device=self.device)
+        o_f = torch.empty_like(q) if want_fine else None
+        vsa2_sparse_attn_fwd_gated(self.p, q, k, v, topk, kv_off, kv_idx, gate_logits, oc, o, lse, o_f, self.ws)
+        return o, lse, o_f
 
     def attn_bwd(self, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, topk=None):
         topk = self.topk if topk is None else topk
@@ -150,9 +165,10 @@ class VSA2:
     def attention(self, q, k, v, gate_logits, topk=None):
         """The whole VSA2 attention output, Eq. 14: fine branch (router, TopK, Eq. 12) plus the
         gated coarse branch. Returns o."""
-        o_f, _, _ = self.forward(q, k, v, topk)
+        scores = self.router_scores(q, k)
+        kv_off, kv_idx, _, _ = self.topk_select(scores, topk, csc=False)
         oc, _ = self.coarse_attn(q, k, v)
-        return self.gated_merge(o_f, gate_logits, oc, out=o_f)
+        return self.attn_fwd_gated(q, k, v, kv_off, kv_idx, gate_logits, oc, topk)[0]
 
     def forward_host(self, q, k, v, topk=None, o=None, lse=None, heads_per_group=0, want_lse=False):
         """Router -> TopK -> forward on HOST tensors, copies overlapped with the kernels per group of
@@ -206,9 +222,9 @@ class _Vsa2Attention(torch.autograd.Function):
         with torch.no_grad():  # the router receives no gradient (§2.1)
             scores = engine.router_scores(q, k)
             kv_off, kv_idx, q_off, q_idx = engine.topk_select(scores, topk, csc=True)
-        o_f, lse = engine.attn_fwd(q, k, v, kv_off, kv_idx, topk)
         oc, lse_c = engine.coarse_attn(q, k, v)
-        o = engine.gated_merge(o_f, gate_logits, oc)
+        o, lse, o_f = engine.attn_fwd_gated(q, k, v, kv_off, kv_idx, gate_logits.contiguous(), oc, topk,
+                                            want_fine=True)
         ctx.save_for_backward(q, k, v, o_f, lse, kv_off, kv_idx, q_off, q_idx, oc, lse_c, gate_logits)
         ctx.engine, ctx.topk = engine, topk
         return o

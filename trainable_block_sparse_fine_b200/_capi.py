@@ -22,7 +22,7 @@ EXPORTS = ("vsa2_workspace_size", "vsa2_workspace_init", "vsa2_router_scores", "
            "vsa2_selftest_wait_timeout", "vsa2_status_string", "vsa2_version", "vsa2_last_cuda_error",
            "vsa2_topk_select_noalloc", "vsa2_forward_host", "vsa2_forward_host_workspace_size",
            "vsa2_coarse_attn", "vsa2_gated_merge", "vsa2_gated_merge_bwd", "vsa2_coarse_attn_bwd",
-           "vsa2_permute_tokens", "vsa2_topk_select_per_row")
+           "vsa2_permute_tokens", "vsa2_topk_select_per_row", "vsa2_sparse_attn_fwd_gated")
 
 
 class Vsa2Error(RuntimeError):
@@ -61,6 +61,7 @@ def lib() -> ctypes.CDLL:
         L.vsa2_sparse_attn_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.vsa2_topk_select_noalloc.argtypes = [P, vp, i32, vp, vp, vp]
         L.vsa2_topk_select_per_row.argtypes = [P, vp, i32, vp, vp, vp, vp, vp, sz, vp]
+        L.vsa2_sparse_attn_fwd_gated.argtypes = [P, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.vsa2_forward_host_workspace_size.argtypes = [P, i32, i32]
         L.vsa2_forward_host_workspace_size.restype = sz
         L.vsa2_forward_host.argtypes = [P, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
@@ -76,7 +77,7 @@ def lib() -> ctypes.CDLL:
         L.vsa2_version.restype = i32
         L.vsa2_last_cuda_error.restype = ctypes.c_char_p
         for name in ("vsa2_workspace_init", "vsa2_router_scores", "vsa2_topk_select", "vsa2_topk_select_noalloc",
-                     "vsa2_topk_select_per_row",
+                     "vsa2_topk_select_per_row", "vsa2_sparse_attn_fwd_gated",
                      "vsa2_sparse_attn_fwd", "vsa2_forward_host", "vsa2_coarse_attn", "vsa2_gated_merge",
                      "vsa2_gated_merge_bwd", "vsa2_coarse_attn_bwd", "vsa2_permute_tokens",
                      "vsa2_sparse_attn_bwd", "vsa2_get_device_error", "vsa2_selftest_wait_timeout"):
@@ -151,6 +152,14 @@ def vsa2_sparse_attn_fwd(p: Problem, q, k, v, topk, kv_off, kv_idx, o, lse, ws, 
     _check(lib().vsa2_sparse_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), topk, _ptr(kv_off), _ptr(kv_idx),
                                       _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "vsa2_sparse_attn_fwd")
+
+
+def vsa2_sparse_attn_fwd_gated(p: Problem, q, k, v, topk, kv_off, kv_idx, gate_logits, oc, o, lse, o_f, ws,
+                               stream=None) -> None:
+    _check(lib().vsa2_sparse_attn_fwd_gated(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), topk, _ptr(kv_off),
+                                            _ptr(kv_idx), _ptr(gate_logits), _ptr(oc), _ptr(o), _ptr(lse), _ptr(o_f),
+                                            _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "vsa2_sparse_attn_fwd_gated")
 
 
 def vsa2_sparse_attn_bwd(p: Problem, q, k, v, o, lse, dout, topk, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, ws,

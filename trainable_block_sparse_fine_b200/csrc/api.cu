@@ -1,6 +1,7 @@
 // C ABI of libvsa2: argument validation, workspace layout and dispatch to the kernels.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdio>
 #include <cstring>
@@ -19,17 +20,20 @@ vsa2_status make_dims(const vsa2_problem* p, Dims* d) {
     return VSA2_ERR_INVALID_ARG;
   if (p->dtype != VSA2_BF16 && p->dtype != VSA2_FP32) return VSA2_ERR_UNSUPPORTED;
   if (p->head_dim != 64 && p->head_dim != 128) return VSA2_ERR_UNSUPPORTED;
-  if (p->tile_t * p->tile_h * p->tile_w != kTile) return VSA2_ERR_UNSUPPORTED;
-  if (p->pool_t * p->pool_h * p->pool_w != kPool) return VSA2_ERR_UNSUPPORTED;
+  // 64-token tiles with 16-token sub-cubes (the pages' shapes), or 128-token tiles with 8-token
+  // sub-cubes (the B = 128, R = 8 reading of the deep-read blog)
+  const int Bt = p->tile_t * p->tile_h * p->tile_w, R = p->pool_t * p->pool_h * p->pool_w;
+  if (!((Bt == 64 && R == 16) || (Bt == 128 && R == 8))) return VSA2_ERR_UNSUPPORTED;
   if (p->tile_t % p->pool_t || p->tile_h % p->pool_h || p->tile_w % p->pool_w) return VSA2_ERR_UNSUPPORTED;
   // a grid the tile does not divide is padded to whole tiles (§2.2 "Kernel Implementation")
   const bool padded = p->grid_t % p->tile_t || p->grid_h % p->tile_h || p->grid_w % p->tile_w;
+  if (padded && Bt != 64) return VSA2_ERR_UNSUPPORTED;  // padding is built for 64-token tiles
   const int64_t pt = (p->grid_t + p->tile_t - 1) / p->tile_t * p->tile_t;
   const int64_t ph = (p->grid_h + p->tile_h - 1) / p->tile_h * p->tile_h;
   const int64_t pw = (p->grid_w + p->tile_w - 1) / p->tile_w * p->tile_w;
   if (pt > (1 << 20) || ph > (1 << 20) || pw > (1 << 20)) return VSA2_ERR_UNSUPPORTED;
   const int64_t L = pt * ph * pw;
-  const int64_t N = L / kTile;
+  const int64_t N = L / Bt;
   const int64_t BH = p->batch * p->heads;
   // index arithmetic below uses 32-bit tile and row counts
   if (N > 32768 || BH > 65535 || BH * L > (int64_t(1) << 31)) return VSA2_ERR_UNSUPPORTED;
@@ -39,7 +43,7 @@ vsa2_status make_dims(const vsa2_problem* p, Dims* d) {
   d->BH = (int)BH;
   d->L = L;
   d->N = (int)N;
-  d->Lr = (int)(L / kPool);
+  d->Lr = (int)(L / R);
   d->dtype = p->dtype;
   d->esize = p->dtype == VSA2_BF16 ? 2 : 4;
   d->flags = p->flags;
@@ -48,6 +52,9 @@ vsa2_status make_dims(const vsa2_problem* p, Dims* d) {
   d->tt = p->tile_t, d->th = p->tile_h, d->tw = p->tile_w;
   d->rt = p->pool_t, d->rh = p->pool_h, d->rw = p->pool_w;
   d->padded = padded;
+  d->Bt = Bt;
+  d->R = R;
+  d->G = Bt / R;
   return VSA2_OK;
 }
 
@@ -89,6 +96,27 @@ WsLayout ws_layout(const Dims& d) {
   w.total = off;
   return w;
 }
+
+ExpLayout exp_layout(const Dims& d, int topk) {
+  ExpLayout e{};
+  size_t base = ws_layout(d).total;
+  if (d.Bt != kTile) base = std::max(base, ws_layout(dims64(d)).total);
+  e.total = base;
+  if (d.Bt == kTile || topk <= 0) return e;
+  auto take = [&](size_t bytes) {
+    const size_t at = e.total;
+    e.total += align256(bytes);
+    return at;
+  };
+  const size_t n64 = (size_t)2 * d.N;
+  e.off = take((size_t)d.BH * (n64 + 1) * 4);
+  e.idx = take((size_t)d.BH * 4 * (size_t)d.N * topk * 4);
+  e.qoff = take((size_t)d.BH * (n64 + 1) * 4);
+  e.qidx = take((size_t)d.BH * 4 * (size_t)d.N * topk * 4);
+  return e;
+}
+
+size_t ws_required(const Dims& d, int topk) { return exp_layout(d, topk).total; }
 
 static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -196,9 +224,9 @@ vsa2_status check_launch(const char* what) {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-static vsa2_status check_ws(const Dims& d, void* ws, size_t ws_bytes) {
+static vsa2_status check_ws(const Dims& d, void* ws, size_t ws_bytes, int topk = 0) {
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return VSA2_ERR_INVALID_ARG;
-  if (ws_bytes < ws_layout(d).total) return VSA2_ERR_INVALID_ARG;
+  if (ws_bytes < ws_required(d, topk)) return VSA2_ERR_INVALID_ARG;
   return VSA2_OK;
 }
 
@@ -209,10 +237,9 @@ using namespace vsa2;
 extern "C" {
 
 size_t vsa2_workspace_size(const vsa2_problem* p, int32_t topk) {
-  (void)topk;
   Dims d;
   if (make_dims(p, &d) != VSA2_OK) return 0;
-  return ws_layout(d).total;
+  return ws_required(d, topk);
 }
 
 vsa2_status vsa2_workspace_init(void* ws, size_t ws_bytes, void* stream) {
@@ -269,8 +296,43 @@ vsa2_status vsa2_sparse_attn_fwd(const vsa2_problem* p, const void* q, const voi
   if (topk < 1 || topk > d.N) return VSA2_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return VSA2_ERR_INVALID_ARG;
-  if ((st = check_ws(d, ws, ws_bytes)) != VSA2_OK) return st;
+  if ((st = check_ws(d, ws, ws_bytes, topk)) != VSA2_OK) return st;
+  if (d.Bt != kTile) {  // 128-token tiles: expand the selection, run on 64-token tiles
+    const ExpLayout e = exp_layout(d, topk);
+    char* w = (char*)ws;
+    int32_t* off64 = reinterpret_cast<int32_t*>(w + e.off);
+    int32_t* idx64 = reinterpret_cast<int32_t*>(w + e.idx);
+    if ((st = launch_expand_lists(d, topk, kv_off, kv_idx, off64, idx64, (cudaStream_t)stream)) != VSA2_OK) return st;
+    return launch_attn_fwd(dims64(d), q, k, v, 2 * topk, off64, idx64, o, lse, w, (cudaStream_t)stream);
+  }
   return launch_attn_fwd(d, q, k, v, topk, kv_off, kv_idx, o, lse, (char*)ws, (cudaStream_t)stream);
+}
+
+vsa2_status vsa2_sparse_attn_fwd_gated(const vsa2_problem* p, const void* q, const void* k, const void* v,
+                                       int32_t topk, const int32_t* kv_off, const int32_t* kv_idx,
+                                       const float* gate_logits, const void* oc, void* o, float* lse, void* o_f,
+                                       void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  vsa2_status st = make_dims(p, &d);
+  if (st != VSA2_OK) return st;
+  if (!q || !k || !v || !kv_off || !kv_idx || !gate_logits || !oc || !o || !lse) return VSA2_ERR_INVALID_ARG;
+  if (topk < 1 || topk > d.N) return VSA2_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(oc) ||
+      !aligned16(gate_logits) || (o_f && !aligned16(o_f)))
+    return VSA2_ERR_INVALID_ARG;
+  if (o == o_f || o == q || o == k || o == v) return VSA2_ERR_INVALID_ARG;
+  if (d.Bt != kTile) return VSA2_ERR_UNSUPPORTED;  // the merge repeats 64-token tiles
+  if ((st = check_ws(d, ws, ws_bytes, topk)) != VSA2_OK) return st;
+  const cudaStream_t s = (cudaStream_t)stream;
+  if (d.dtype == VSA2_BF16 && d.D == 128)
+    return attn_fwd_tc_gated(d, q, k, v, topk, kv_off, kv_idx, gate_logits, oc, o, lse, o_f, (char*)ws, s);
+  // CUDA-core shapes (fp32, head_dim 64): the same merge in the CUDA-core forward's epilogue
+  uint64_t* tmask = nullptr;
+  if (d.padded) {
+    tmask = reinterpret_cast<uint64_t*>((char*)ws + ws_layout(d).tmask);
+    if ((st = launch_tile_masks(d, tmask, s)) != VSA2_OK) return st;
+  }
+  return attn_fwd_simt(d, q, k, v, topk, kv_off, kv_idx, o, lse, (char*)ws, d.L, tmask, s, gate_logits, oc, o_f);
 }
 
 vsa2_status vsa2_sparse_attn_bwd(const vsa2_problem* p, const void* q, const void* k, const void* v, const void* o,
@@ -288,7 +350,19 @@ vsa2_status vsa2_sparse_attn_bwd(const vsa2_problem* p, const void* q, const voi
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
       !aligned16(dk) || !aligned16(dv) || !aligned16(lse))
     return VSA2_ERR_INVALID_ARG;
-  if ((st = check_ws(d, ws, ws_bytes)) != VSA2_OK) return st;
+  if ((st = check_ws(d, ws, ws_bytes, topk)) != VSA2_OK) return st;
+  if (d.Bt != kTile) {  // 128-token tiles: expand the CSR and the CSC, run on 64-token tiles
+    const ExpLayout e = exp_layout(d, topk);
+    char* w = (char*)ws;
+    const cudaStream_t s = (cudaStream_t)stream;
+    int32_t* off64 = reinterpret_cast<int32_t*>(w + e.off);
+    int32_t* idx64 = reinterpret_cast<int32_t*>(w + e.idx);
+    int32_t* qoff64 = reinterpret_cast<int32_t*>(w + e.qoff);
+    int32_t* qidx64 = reinterpret_cast<int32_t*>(w + e.qidx);
+    if ((st = launch_expand_lists(d, topk, kv_off, kv_idx, off64, idx64, s)) != VSA2_OK) return st;
+    if ((st = launch_expand_lists(d, topk, q_off, q_idx, qoff64, qidx64, s)) != VSA2_OK) return st;
+    return launch_attn_bwd(dims64(d), q, k, v, o, lse, dout, 2 * topk, off64, idx64, qoff64, qidx64, dq, dk, dv, w, s);
+  }
   return launch_attn_bwd(d, q, k, v, o, lse, dout, topk, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, (char*)ws,
                          (cudaStream_t)stream);
 }
@@ -298,6 +372,7 @@ vsa2_status vsa2_coarse_attn(const vsa2_problem* p, const void* q, const void* k
   Dims d;
   vsa2_status st = make_dims(p, &d);
   if (st != VSA2_OK) return st;
+  if (d.Bt != kTile) return VSA2_ERR_UNSUPPORTED;  // the coarse branch and the merge take 64-token tiles
   if (!q || !k || !v || !oc) return VSA2_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(oc) || (lse_c && !aligned16(lse_c)))
     return VSA2_ERR_INVALID_ARG;
@@ -310,6 +385,7 @@ vsa2_status vsa2_gated_merge(const vsa2_problem* p, const void* o_f, const float
   Dims d;
   vsa2_status st = make_dims(p, &d);
   if (st != VSA2_OK) return st;
+  if (d.Bt != kTile) return VSA2_ERR_UNSUPPORTED;  // the coarse branch and the merge take 64-token tiles
   if (!o_f || !gate_logits || !oc || !o) return VSA2_ERR_INVALID_ARG;
   if (!aligned16(o_f) || !aligned16(gate_logits) || !aligned16(oc) || !aligned16(o)) return VSA2_ERR_INVALID_ARG;
   return launch_gated_merge(d, o_f, gate_logits, oc, o, (cudaStream_t)stream);
@@ -320,6 +396,7 @@ vsa2_status vsa2_gated_merge_bwd(const vsa2_problem* p, const void* dout, const 
   Dims d;
   vsa2_status st = make_dims(p, &d);
   if (st != VSA2_OK) return st;
+  if (d.Bt != kTile) return VSA2_ERR_UNSUPPORTED;  // the coarse branch and the merge take 64-token tiles
   if (!dout || !gate_logits || !oc || !d_logits || !d_oc) return VSA2_ERR_INVALID_ARG;
   if (!aligned16(dout) || !aligned16(gate_logits) || !aligned16(oc) || !aligned16(d_logits) || !aligned16(d_oc))
     return VSA2_ERR_INVALID_ARG;
@@ -332,6 +409,7 @@ vsa2_status vsa2_coarse_attn_bwd(const vsa2_problem* p, const void* q, const voi
   Dims d;
   vsa2_status st = make_dims(p, &d);
   if (st != VSA2_OK) return st;
+  if (d.Bt != kTile) return VSA2_ERR_UNSUPPORTED;  // the coarse branch and the merge take 64-token tiles
   if (d.padded) return VSA2_ERR_UNSUPPORTED;  // the backward takes whole-tile grids only
   if (!q || !k || !v || !oc || !lse_c || !d_oc || !dq || !dk || !dv) return VSA2_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(oc) || !aligned16(lse_c) || !aligned16(d_oc) ||

@@ -137,13 +137,22 @@ __device__ __forceinline__ int next_op(SlotSeq& q, int* blk, const int32_t* kv_o
   return 0;
 }
 
-template <int kMode>
+// The gated merge of Eq. 13-14 fused into the epilogue (kGate): O = tanh(g) * O_c_hat[tile] + O_f
+// with the gate logit g = (X W_g) of the row and the coarse output row of the query tile; the
+// fine output O_f can be written too (the backward forms Delta from it).
+struct GateArgs {
+  const float* logits;           // [b*h, L] fp32
+  const __nv_bfloat16* oc;       // [b*h, N, 128], the coarse branch's output
+  __nv_bfloat16* of;             // [b*h, L, 128] or nullptr
+};
+
+template <int kMode, bool kGate>
 __global__ void __launch_bounds__(FT, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const __nv_bfloat16* __restrict__ qg, const int32_t* __restrict__ kv_off,
                        const int32_t* __restrict__ kv_idx, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
                        int N, int L, int topk, int items, float c2, int kv_valid,
-                       const uint64_t* __restrict__ tmask, DevCtx ctx) {
+                       const uint64_t* __restrict__ tmask, GateArgs gate, DevCtx ctx) {
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
   uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   Bars& B = *reinterpret_cast<Bars*>(dsm + OFF_BAR);
@@ -325,10 +334,31 @@ __global__ void __launch_bounds__(FT, 1)
       const int nblk = (rw.len + 1) >> 1;
       const size_t tok = (size_t)bh * L + (size_t)qt * 64 + row;
       if (nblk == 0) {
-        // empty selection: o = 0, lse = -inf (each thread of a pair writes half the row)
+        // empty selection: o = 0, lse = -inf (each thread of a pair writes half the row); with the
+        // gate the output is the coarse term alone
         uint4* o4 = reinterpret_cast<uint4*>(out + tok * 128 + par_c * 64);
+        if constexpr (kGate) {
+          const float gt = tanhf(__ldg(gate.logits + tok));
+          const uint4* c4 = reinterpret_cast<const uint4*>(gate.oc + ((size_t)bh * N + qt) * 128 + par_c * 64);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o4[e] = make_uint4(0, 0, 0, 0);
+          for (int e = 0; e < 8; ++e) {
+            const uint4 c = __ldg(c4 + e);
+            const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+            uint32_t r[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              r[u] = pack_bf16(gt * __uint_as_float(cw[u] << 16), gt * __uint_as_float(cw[u] & 0xffff0000u));
+            o4[e] = make_uint4(r[0], r[1], r[2], r[3]);
+          }
+          if (gate.of) {
+            uint4* f4 = reinterpret_cast<uint4*>(gate.of + tok * 128 + par_c * 64);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f4[e] = make_uint4(0, 0, 0, 0);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o4[e] = make_uint4(0, 0, 0, 0);
+        }
         if (par_c == 0) lse[tok] = -INFINITY;
         continue;
       }
@@ -455,12 +485,30 @@ __global__ void __launch_bounds__(FT, 1)
       if (par_c == 0) lse[tok] = lse_row;
       // o[i] = O[row][2i + par_c]; swap so each thread holds adjacent pairs, then 4-byte stores
       uint32_t* dst = reinterpret_cast<uint32_t*>(out + tok * 128);
+      if constexpr (kGate) {
+        // word w = 2*i2 + par_c holds columns 2w, 2w+1: O_f there in fp32, then the gated sum
+        const float gt = tanhf(__ldg(gate.logits + tok));
+        const uint32_t* ocw = reinterpret_cast<const uint32_t*>(gate.oc + ((size_t)bh * N + qt) * 128);
+        uint32_t* fdst = gate.of ? reinterpret_cast<uint32_t*>(gate.of + tok * 128) : nullptr;
 #pragma unroll
-      for (int i2 = 0; i2 < 32; ++i2) {
-        const float a = __uint_as_float(o[2 * i2]) * inv, b = __uint_as_float(o[2 * i2 + 1]) * inv;
-        const float send = par_c ? a : b;
-        const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
-        dst[2 * i2 + par_c] = par_c ? pack_bf16(recv, b) : pack_bf16(a, recv);
+        for (int i2 = 0; i2 < 32; ++i2) {
+          const float a = __uint_as_float(o[2 * i2]) * inv, b = __uint_as_float(o[2 * i2 + 1]) * inv;
+          const float send = par_c ? a : b;
+          const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
+          const float lo = par_c ? recv : a, hi = par_c ? b : recv;
+          const int wd = 2 * i2 + par_c;
+          const uint32_t c = __ldg(ocw + wd);
+          dst[wd] = pack_bf16(fmaf(gt, __uint_as_float(c << 16), lo), fmaf(gt, __uint_as_float(c & 0xffff0000u), hi));
+          if (fdst) fdst[wd] = pack_bf16(lo, hi);
+        }
+      } else {
+#pragma unroll
+        for (int i2 = 0; i2 < 32; ++i2) {
+          const float a = __uint_as_float(o[2 * i2]) * inv, b = __uint_as_float(o[2 * i2 + 1]) * inv;
+          const float send = par_c ? a : b;
+          const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
+          dst[2 * i2 + par_c] = par_c ? pack_bf16(recv, b) : pack_bf16(a, recv);
+        }
       }
       // leave together if any wait of this CTA has expired
       if (named_bar_or(bar_id, 128, *abort != 0)) break;
@@ -480,10 +528,10 @@ bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64
                        uint32_t box_rows);
 
 namespace {
-template <int kMode>
+template <int kMode, bool kGate = false>
 vsa2_status launch_fwd_tc(const Dims& d, const void* q, const void* k, const void* v, int topk,
                           const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws, int kv_valid,
-                          const uint64_t* tmask, cudaStream_t s) {
+                          const uint64_t* tmask, cudaStream_t s, GateArgs gate = GateArgs{nullptr, nullptr, nullptr}) {
   CUtensorMap tk, tv;
   const uint64_t rows = (uint64_t)d.BH * d.L;
   if (!make_tmap_2d_bf16(&tk, k, 128, rows, 64, 64) || !make_tmap_2d_bf16(&tv, v, 128, rows, 64, 64))
@@ -495,10 +543,10 @@ vsa2_status launch_fwd_tc(const Dims& d, const void* q, const void* k, const voi
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::max(1, std::min(sms, (items + 1) / 2));
   const float c2 = 1.4426950408889634f / sqrtf(128.f);
-  cudaFuncSetAttribute(attn_fwd_tc_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
-  attn_fwd_tc_kernel<kMode><<<grid, FT, SMEM_DYN, s>>>(tk, tv, (const __nv_bfloat16*)q, kv_off, kv_idx,
-                                                       (__nv_bfloat16*)o, lse, d.N, (int)d.L, topk, items, c2,
-                                                       kv_valid, tmask, ctx);
+  auto kern = attn_fwd_tc_kernel<kMode, kGate>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
+  kern<<<grid, FT, SMEM_DYN, s>>>(tk, tv, (const __nv_bfloat16*)q, kv_off, kv_idx, (__nv_bfloat16*)o, lse, d.N,
+                                  (int)d.L, topk, items, c2, kv_valid, tmask, gate, ctx);
   return check_launch("attn_fwd_tc");
 }
 }  // namespace
@@ -511,6 +559,18 @@ vsa2_status attn_fwd_tc(const Dims& d, const void* q, const void* k, const void*
     return launch_fwd_tc<2>(d, q, k, v, topk, kv_off, kv_idx, o, lse, ws, (int)d.L, tmask, s);
   }
   return launch_fwd_tc<0>(d, q, k, v, topk, kv_off, kv_idx, o, lse, ws, (int)d.L, nullptr, s);
+}
+
+vsa2_status attn_fwd_tc_gated(const Dims& d, const void* q, const void* k, const void* v, int topk,
+                              const int32_t* kv_off, const int32_t* kv_idx, const float* gate_logits, const void* oc,
+                              void* o, float* lse, void* o_f, char* ws, cudaStream_t s) {
+  const GateArgs g{gate_logits, (const __nv_bfloat16*)oc, (__nv_bfloat16*)o_f};
+  if (d.padded) {
+    uint64_t* tmask = reinterpret_cast<uint64_t*>(ws + ws_layout(d).tmask);
+    if (launch_tile_masks(d, tmask, s) != VSA2_OK) return VSA2_ERR_CUDA;
+    return launch_fwd_tc<2, true>(d, q, k, v, topk, kv_off, kv_idx, o, lse, ws, (int)d.L, tmask, s, g);
+  }
+  return launch_fwd_tc<0, true>(d, q, k, v, topk, kv_off, kv_idx, o, lse, ws, (int)d.L, nullptr, s, g);
 }
 
 vsa2_status attn_fwd_tc_masked(const Dims& d, const void* q, const void* k, const void* v, int topk,

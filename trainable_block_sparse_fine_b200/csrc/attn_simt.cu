@@ -50,7 +50,8 @@ __global__ void __launch_bounds__(64) attn_fwd_simt_kernel(const T* __restrict__
                                                            const int32_t* __restrict__ kv_idx, T* __restrict__ o,
                                                            float* __restrict__ lse, int N, int64_t L, int topk,
                                                            int64_t kv_valid, const uint64_t* __restrict__ tmask,
-                                                           DevCtx ctx) {
+                                                           const float* __restrict__ gate, const T* __restrict__ oc,
+                                                           T* __restrict__ of, DevCtx ctx) {
   extern __shared__ float sm[];
   float* qT = sm;              // [D][64]
   float* ks = qT + D * 64;     // [64][D]
@@ -109,7 +110,17 @@ __global__ void __launch_bounds__(64) attn_fwd_simt_kernel(const T* __restrict__
   }
   const bool q_real = !tmask || ((tmask[i] >> t) & 1ull);  // a padding query row gets o = 0, lse = -inf
   const float inv = (l > 0.f && q_real) ? 1.f / l : 0.f;
-  for (int d = 0; d < D; ++d) stf(o + (tok0 + t) * D + d, inv != 0.f ? oT[d * 64 + t] * inv : 0.f);
+  if (gate) {  // Eq. 13-14 on the fp32 fine output: o = tanh(g) * oc[tile] + O_f
+    const float gt = tanhf(gate[tok0 + t]);
+    const T* crow = oc + ((size_t)bh * N + i) * D;
+    for (int d = 0; d < D; ++d) {
+      const float f = inv != 0.f ? oT[d * 64 + t] * inv : 0.f;
+      stf(o + (tok0 + t) * D + d, fmaf(gt, ldf(crow + d), f));
+      if (of) stf(of + (tok0 + t) * D + d, f);
+    }
+  } else {
+    for (int d = 0; d < D; ++d) stf(o + (tok0 + t) * D + d, inv != 0.f ? oT[d * 64 + t] * inv : 0.f);
+  }
   lse[tok0 + t] = (l > 0.f && q_real) ? m + __logf(l) : -INFINITY;
 }
 
@@ -268,12 +279,12 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_simt_kernel(const T* __rest
 template <typename T, int D>
 vsa2_status fwd_simt(const Dims& d, const void* q, const void* k, const void* v, const int32_t* kv_off,
                      const int32_t* kv_idx, void* o, float* lse, const DevCtx& ctx, int topk, int64_t kv_valid,
-                     const uint64_t* tmask, cudaStream_t s) {
+                     const uint64_t* tmask, const float* gate, const void* oc, void* of, cudaStream_t s) {
   const size_t smem = (size_t)4 * 64 * D * sizeof(float);
   auto kern = attn_fwd_simt_kernel<T, D>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   kern<<<dim3(d.N, d.BH), 64, smem, s>>>((const T*)q, (const T*)k, (const T*)v, kv_off, kv_idx, (T*)o, lse, d.N,
-                                         d.L, topk, kv_valid, tmask, ctx);
+                                         d.L, topk, kv_valid, tmask, gate, (const T*)oc, (T*)of, ctx);
   return check_launch(__func__);
 }
 
@@ -301,15 +312,19 @@ vsa2_status bwd_simt(const Dims& d, const void* q, const void* k, const void* v,
 
 vsa2_status attn_fwd_simt(const Dims& d, const void* q, const void* k, const void* v, int topk,
                           const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
-                          int64_t kv_valid, const uint64_t* tmask, cudaStream_t s) {
+                          int64_t kv_valid, const uint64_t* tmask, cudaStream_t s, const float* gate,
+                          const void* oc, void* of) {
   DevCtx ctx{reinterpret_cast<int*>(ws), d.timeout_ns, d.flags};
   if (d.dtype == VSA2_BF16) {
     if (d.D == 128)
-      return fwd_simt<__nv_bfloat16, 128>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, tmask, s);
-    return fwd_simt<__nv_bfloat16, 64>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, tmask, s);
+      return fwd_simt<__nv_bfloat16, 128>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, tmask, gate, oc,
+                                          of, s);
+    return fwd_simt<__nv_bfloat16, 64>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, tmask, gate, oc, of,
+                                       s);
   }
-  if (d.D == 128) return fwd_simt<float, 128>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, tmask, s);
-  return fwd_simt<float, 64>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, tmask, s);
+  if (d.D == 128)
+    return fwd_simt<float, 128>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, tmask, gate, oc, of, s);
+  return fwd_simt<float, 64>(d, q, k, v, kv_off, kv_idx, o, lse, ctx, topk, kv_valid, tmask, gate, oc, of, s);
 }
 
 vsa2_status attn_bwd_simt(const Dims& d, const void* q, const void* k, const void* v, const void* o, const float* lse,

@@ -10,8 +10,12 @@
 
 namespace vsa2 {
 
-constexpr int kTile = 64;  // tokens per tile (4 x 4 x 4 cube)
-constexpr int kPool = 16;  // tokens per router sub-cube (2 x 2 x 4)
+// The attention kernels work on 64-token tiles. The router and the TopK work on the problem's
+// tiles: 64 tokens with 16-token sub-cubes (G = 4), or 128 tokens with 8-token sub-cubes
+// (G = 16); a 128-token tile is two consecutive 64-token tiles of the cube-major order, so its
+// selection is expanded to 64-token tiles before the attention kernels run.
+constexpr int kTile = 64;  // tokens per attention tile (4 x 4 x 4 cube)
+constexpr int kPool = 16;  // tokens per router sub-cube of a 64-token tile (2 x 2 x 4)
 constexpr int kG = kTile / kPool;
 
 struct Dims {
@@ -27,7 +31,20 @@ struct Dims {
   int tt, th, tw;  // tile
   int rt, rh, rw;  // router sub-cube
   bool padded;     // the tile does not divide the grid: every extent is rounded up to whole tiles
+  int Bt, R, G;    // tokens per tile (64 or 128), per sub-cube (16 or 8), sub-cubes per tile
 };
+
+// The same problem seen in 64-token tiles (what the attention kernels take): d itself for
+// 64-token tiles; for 128-token tiles N doubles.
+inline Dims dims64(const Dims& d) {
+  Dims e = d;
+  e.N = (int)(d.L / kTile);
+  e.Bt = kTile;
+  e.R = kPool;
+  e.G = kG;
+  e.Lr = (int)(d.L / kPool);
+  return e;
+}
 
 // Real-token mask of every tile of a padded grid (bit u = cube-major token u of the tile is a
 // token of the real grid); the same for every (b, h). Enqueued on `s`, written to `mask` [N].
@@ -61,6 +78,19 @@ struct WsLayout {
 };
 WsLayout ws_layout(const Dims& d);
 
+// 128-token tiles: the selection expanded to 64-token tiles (CSR, and CSC for the backward),
+// after every region the kernels of d and of dims64(d) use. topk is the problem's budget.
+struct ExpLayout {
+  size_t off, idx, qoff, qidx, total;
+};
+ExpLayout exp_layout(const Dims& d, int topk);
+// Workspace bytes a call with budget topk (0: calls without a selection) needs.
+size_t ws_required(const Dims& d, int topk);
+// Expand a tile-granularity list (CSR or CSC) of 128-token tiles into 64-token tiles: 64-tile u
+// of head bh gets 2J, 2J+1 for every J in list u / 2. Enqueued on s.
+vsa2_status launch_expand_lists(const Dims& d, int topk, const int32_t* off, const int32_t* idx, int32_t* off64,
+                                int32_t* idx64, cudaStream_t s);
+
 // Tensor map for a row-major [outer, rows, cols] bf16 tensor, box (box_cols x box_rows x 1),
 // 128-byte swizzle. Returns false if the driver entry point is unavailable or encoding failed.
 bool make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t outer,
@@ -84,7 +114,8 @@ vsa2_status launch_attn_bwd(const Dims& d, const void* q, const void* k, const v
 // padded grid's real-token masks), the padding tokens of every tile.
 vsa2_status attn_fwd_simt(const Dims& d, const void* q, const void* k, const void* v, int topk,
                           const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
-                          int64_t kv_valid, const uint64_t* tmask, cudaStream_t s);
+                          int64_t kv_valid, const uint64_t* tmask, cudaStream_t s, const float* gate = nullptr,
+                          const void* oc = nullptr, void* of = nullptr);
 vsa2_status attn_bwd_simt(const Dims& d, const void* q, const void* k, const void* v, const void* o,
                           const float* lse, const void* dout, const int32_t* kv_off, const int32_t* kv_idx,
                           const int32_t* q_off, const int32_t* q_idx, float* dq, float* dk, float* dv, int topk,
@@ -94,6 +125,11 @@ vsa2_status attn_bwd_simt(const Dims& d, const void* q, const void* k, const voi
 vsa2_status attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v, int topk,
                         const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
                         cudaStream_t s);
+// the fine forward with the gated merge of Eq. 13-14 in its epilogue (bf16, head_dim 128):
+// o = tanh(gate_logits) * oc[tile] + O_f; O_f also written to o_f when it is not null
+vsa2_status attn_fwd_tc_gated(const Dims& d, const void* q, const void* k, const void* v, int topk,
+                              const int32_t* kv_off, const int32_t* kv_idx, const float* gate_logits, const void* oc,
+                              void* o, float* lse, void* o_f, char* ws, cudaStream_t s);
 vsa2_status attn_fwd_tc_masked(const Dims& d, const void* q, const void* k, const void* v, int topk,
                                const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
                                int kv_valid, cudaStream_t s);
