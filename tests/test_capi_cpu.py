@@ -54,6 +54,17 @@ def test_unsupported_shapes_give_zero_workspace():
     assert C.vsa2_workspace_size(C.make_problem(1, 2, 64, (8, 16, 16), tile=(4, 4, 4), pool=(3, 2, 4)), 8) == 0
 
 
+def test_128_token_tiles_take_a_budget_dependent_workspace():
+    """B = 128, R = 8: the workspace holds the selection expanded to 64-token tiles, so it grows
+    with the budget; grids the 128-token tile does not divide are not taken."""
+    p = C.make_problem(1, 2, 128, (8, 16, 32), tile=(4, 4, 8), pool=(2, 2, 2))
+    a, b = C.vsa2_workspace_size(p, 2), C.vsa2_workspace_size(p, 8)
+    assert 0 < a < b
+    assert C.vsa2_workspace_size(p, 0) > 0  # the router and the TopK need no expansion
+    assert C.vsa2_workspace_size(C.make_problem(1, 2, 128, (8, 16, 30), tile=(4, 4, 8), pool=(2, 2, 2)), 2) == 0
+    assert C.vsa2_workspace_size(C.make_problem(1, 2, 128, (8, 16, 32), tile=(4, 4, 8), pool=(2, 2, 4)), 2) == 0
+
+
 def test_grid_the_tile_does_not_divide_is_padded():
     """6x7x10 pads to 8x8x12 (24 tiles): the workspace is the padded problem's, as for 8x8x12."""
     padded = C.vsa2_workspace_size(C.make_problem(1, 2, 64, (6, 7, 10)), 3)

@@ -115,7 +115,7 @@ extern "C" {
 size_t vsa2_forward_host_workspace_size(const vsa2_problem* p, int32_t topk, int32_t heads_per_group) {
   Dims d;
   HostLayout h;
-  if (make_dims(p, &d) != VSA2_OK || topk < 1 || topk > d.N || heads_per_group < 0) return 0;
+  if (make_dims(p, &d) != VSA2_OK || topk < 1 || topk > d.N || heads_per_group < 0 || d.Bt != kTile) return 0;
   if (!host_layout(d, p, topk, heads_per_group, &h)) return 0;
   return h.total;
 }
@@ -129,6 +129,7 @@ vsa2_status vsa2_forward_host(const vsa2_problem* p, const void* q, const void* 
   if (!q || !k || !v || !o) return VSA2_ERR_INVALID_ARG;
   if (topk < 1 || topk > d.N) return VSA2_ERR_UNSUPPORTED;
   if (heads_per_group < 0) return VSA2_ERR_INVALID_ARG;
+  if (d.Bt != kTile) return VSA2_ERR_UNSUPPORTED;  // 64-token tiles
   HostLayout h;
   if (!host_layout(d, p, topk, heads_per_group, &h)) return VSA2_ERR_UNSUPPORTED;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < h.total) return VSA2_ERR_INVALID_ARG;

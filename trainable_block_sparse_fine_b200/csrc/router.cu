@@ -10,12 +10,13 @@ namespace vsa2 {
 namespace {
 
 // ------------------------------------------------------------------------------------------
-// MeanPool_R (Eq. 5): each pooled row is the mean of R = 16 consecutive cube-major rows.
+// MeanPool_R (Eq. 5): each pooled row is the mean of R consecutive cube-major rows (R = 16, or 8
+// with 128-token tiles).
 // One thread per (pooled row, 16-byte column chunk); 16 independent 16-byte loads per thread.
 // ------------------------------------------------------------------------------------------
 // With kMask (a padded grid), each mean runs over the sub-cube's real tokens only (tmask, the
 // per-tile real-token masks); a sub-cube without one is written as zeros.
-template <typename T, bool kMask>
+template <typename T, bool kMask, int R>
 __global__ void __launch_bounds__(256) router_pool_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                           T* __restrict__ qr, T* __restrict__ kr,
                                                           int64_t pooled_rows, int chunks_per_row,
@@ -28,23 +29,23 @@ __global__ void __launch_bounds__(256) router_pool_kernel(const T* __restrict__ 
   const int64_t t = is_k ? tid - per_tensor : tid;
   const int64_t prow = t / chunks_per_row;
   const int chunk = (int)(t % chunks_per_row);
-  const T* src = (is_k ? k : q) + (prow * kPool) * (int64_t)chunks_per_row * EPC + chunk * EPC;
+  const T* src = (is_k ? k : q) + (prow * R) * (int64_t)chunks_per_row * EPC + chunk * EPC;
   const int64_t stride = (int64_t)chunks_per_row * EPC;
   float acc[EPC];
 #pragma unroll
   for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
   uint32_t valid = 0xffffu;
-  float inv = 1.f / kPool;
+  float inv = 1.f / R;
   if constexpr (kMask) {
     const int a = (int)(prow % Lr);
     valid = (uint32_t)(__ldg(tmask + (a >> 2)) >> (16 * (a & 3))) & 0xffffu;
     inv = valid ? 1.f / __popc(valid) : 0.f;
   }
-  uint4 buf[kPool];
+  uint4 buf[R];
 #pragma unroll
-  for (int r = 0; r < kPool; ++r) buf[r] = __ldg(reinterpret_cast<const uint4*>(src + r * stride));
+  for (int r = 0; r < R; ++r) buf[r] = __ldg(reinterpret_cast<const uint4*>(src + r * stride));
 #pragma unroll
-  for (int r = 0; r < kPool; ++r) {
+  for (int r = 0; r < R; ++r) {
     if (kMask && !((valid >> r) & 1u)) continue;
     if constexpr (sizeof(T) == 2) {
       const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&buf[r]);
@@ -112,7 +113,9 @@ __device__ __forceinline__ uint32_t piece_keys(int key0, int Lr, const uint64_t*
 // kMask (a padded grid): pooled keys without a real token are masked in the softmax of Eq. 6,
 // pooled query rows without one add nothing, and Eq. 7 averages over the tile's real query
 // sub-cubes (rows still sum to 1).
-template <int ND, bool kMask>
+// G is the number of sub-cubes per tile: 4 (64-token tiles, 16-token sub-cubes) or 16 (128-token
+// tiles, 8-token sub-cubes, no padded grids).
+template <int ND, bool kMask, int G>
 __global__ void __launch_bounds__(RS_THREADS, 1)
     router_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             float* __restrict__ scores, int Lr, int N, float c2, const uint64_t* __restrict__ tmask,
@@ -266,11 +269,11 @@ __global__ void __launch_bounds__(RS_THREADS, 1)
     }
     named_bar_sync(1, 256);
     const float lse2 = lse_sh[row];
-    const int qtile = (m0 + row) >> 2;  // G = 4 pooled rows per tile
+    const int qtile = (m0 + row) / G;  // G pooled rows per tile
     const bool row_ok = qtile < N;
     // kMask: this pooled query row counts only if its sub-cube holds a real token; the tile's
     // score row is the mean over its real query sub-cubes (lanes 4g .. 4g+3 are tile g's rows)
-    float qw = 1.f, tile_inv = 1.f / kG;
+    float qw = 1.f, tile_inv = 1.f / G;
     if constexpr (kMask) {
       const int a = m0 + row;
       qw = (a < Lr && ((__ldg(tmask + (a >> 2)) >> (16 * (a & 3))) & 0xffffu)) ? 1.f : 0.f;
@@ -292,30 +295,33 @@ __global__ void __launch_bounds__(RS_THREADS, 1)
         tmem_ld_wait();
         const int key0 = c * RS_N + col0;
         const uint32_t kv = kMask ? piece_keys<true>(key0, Lr, tmask) : (key0 + 32 <= Lr ? 0xffffffffu : 0u);
+        constexpr int TPP = 32 / G;  // key tiles per 32-key piece
         if (kv == 0xffffffffu) {
-          // full piece: packed FMA for the exponent arguments and packed sums per key sub-cube
+          // full piece: packed FMA for the exponent arguments and packed sums per key tile
           const float2 cc = make_float2(c2, c2), nl = make_float2(-lse2, -lse2);
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            const float2 a0 =
-                __ffma2_rn(make_float2(__uint_as_float(r[4 * jj]), __uint_as_float(r[4 * jj + 1])), cc, nl);
-            const float2 a1 =
-                __ffma2_rn(make_float2(__uint_as_float(r[4 * jj + 2]), __uint_as_float(r[4 * jj + 3])), cc, nl);
-            const float2 sum = __fadd2_rn(make_float2(ex2(a0.x), ex2(a0.y)), make_float2(ex2(a1.x), ex2(a1.y)));
-            t[piece * 8 + jj] = sum.x + sum.y;
+          for (int jj = 0; jj < TPP; ++jj) {
+            float2 sum = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int e = 0; e < G; e += 2) {
+              const float2 a = __ffma2_rn(
+                  make_float2(__uint_as_float(r[G * jj + e]), __uint_as_float(r[G * jj + e + 1])), cc, nl);
+              sum = __fadd2_rn(sum, make_float2(ex2(a.x), ex2(a.y)));
+            }
+            t[piece * TPP + jj] = sum.x + sum.y;
           }
           continue;
         }
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
+        for (int jj = 0; jj < TPP; ++jj) {
           float acc = 0.f;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = 4 * jj + e;
+          for (int e = 0; e < G; ++e) {
+            const int j = G * jj + e;
             const bool ok = kMask ? ((kv >> j) & 1u) : key0 + j < Lr;
             acc += ok ? ex2(__uint_as_float(r[j]) * c2 - lse2) : 0.f;
           }
-          t[piece * 8 + jj] = acc;
+          t[piece * TPP + jj] = acc;
         }
       }
       tc_fence_before();
@@ -325,6 +331,23 @@ __global__ void __launch_bounds__(RS_THREADS, 1)
       if constexpr (kMask) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) t[j] *= qw;
+      }
+      if constexpr (G == 16) {
+        // t[0..7]: this pooled query row's sums over the 8 key tiles of the chunk half. Sum the
+        // 16 query rows of the tile (lanes 16g .. 16g+15); lane 16g writes the 8 tile scores.
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+#pragma unroll
+          for (int o = 1; o < 16; o <<= 1) t[j] += __shfl_xor_sync(0xffffffffu, t[j], o);
+          t[j] *= tile_inv;
+        }
+        const int j0 = (c * RS_N + half * 128) / G;
+        if (row_ok && (lane & 15) == 0) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (j0 + j < N) out_row[j0 + j] = t[j];
+        }
+        continue;
       }
       float u[16];
       const bool hi2 = lane & 2;
@@ -376,7 +399,7 @@ __global__ void __launch_bounds__(RS_THREADS, 1)
 // ------------------------------------------------------------------------------------------
 // tmask != nullptr (a padded grid): keys and query rows of sub-cubes without a real token are
 // left out, and the tile's score row is the mean over its real query sub-cubes.
-template <typename T, int D>
+template <typename T, int D, int kG>
 __global__ void __launch_bounds__(128) router_scores_simt_kernel(const T* __restrict__ qr, const T* __restrict__ kr,
                                                                  float* __restrict__ scores, int Lr, int N,
                                                                  const uint64_t* __restrict__ tmask) {
@@ -392,7 +415,7 @@ __global__ void __launch_bounds__(128) router_scores_simt_kernel(const T* __rest
   float m[kG], l[kG];
 #pragma unroll
   for (int a = 0; a < kG; ++a) m[a] = -INFINITY, l[a] = 0.f;
-  auto key_ok = [&](int b) { return !tmask || ((tmask[b >> 2] >> (16 * (b & 3))) & 0xffffu) != 0; };
+  auto key_ok = [&](int b) { return !tmask || ((tmask[b / kG] >> (16 * (b % kG))) & 0xffffu) != 0; };
   for (int b = t; b < Lr; b += 128) {
     if (!key_ok(b)) continue;
     float s[kG] = {};
@@ -425,7 +448,7 @@ __global__ void __launch_bounds__(128) router_scores_simt_kernel(const T* __rest
   float qw[kG], g = 0.f;
 #pragma unroll
   for (int a = 0; a < kG; ++a) {
-    qw[a] = ((qm >> (16 * a)) & 0xffffu) ? 1.f : 0.f;
+    qw[a] = (!tmask || ((qm >> (16 * a)) & 0xffffu)) ? 1.f : 0.f;
     g += qw[a];
   }
   for (int j = t; j < N; j += 128) {
@@ -462,11 +485,14 @@ vsa2_status launch_router(const Dims& d, const void* q, const void* k, float* sc
     if (launch_tile_masks(d, reinterpret_cast<uint64_t*>(ws + w.tmask), s) != VSA2_OK) return VSA2_ERR_CUDA;
   }
   if (d.dtype == VSA2_BF16) {
-    auto kern = d.padded ? router_pool_kernel<__nv_bfloat16, true> : router_pool_kernel<__nv_bfloat16, false>;
+    auto kern = d.R == 8 ? router_pool_kernel<__nv_bfloat16, false, 8>
+                         : (d.padded ? router_pool_kernel<__nv_bfloat16, true, 16>
+                                     : router_pool_kernel<__nv_bfloat16, false, 16>);
     kern<<<blocks, 256, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)qr,
                                 (__nv_bfloat16*)kr, pooled, cpr, tmask, d.Lr);
   } else {
-    auto kern = d.padded ? router_pool_kernel<float, true> : router_pool_kernel<float, false>;
+    auto kern = d.R == 8 ? router_pool_kernel<float, false, 8>
+                         : (d.padded ? router_pool_kernel<float, true, 16> : router_pool_kernel<float, false, 16>);
     kern<<<blocks, 256, 0, s>>>((const float*)q, (const float*)k, (float*)qr, (float*)kr, pooled, cpr, tmask, d.Lr);
   }
   if (check_launch(__func__) != VSA2_OK) return VSA2_ERR_CUDA;
@@ -478,22 +504,30 @@ vsa2_status launch_router(const Dims& d, const void* q, const void* k, float* sc
     const float c2 = 1.4426950408889634f / sqrtf((float)d.D);
     dim3 grid((d.Lr + RS_M - 1) / RS_M, d.BH);
     if (d.D == 128) {
-      auto kern = d.padded ? router_scores_tc_kernel<2, true> : router_scores_tc_kernel<2, false>;
+      auto kern = d.G == 16 ? router_scores_tc_kernel<2, false, 16>
+                            : (d.padded ? router_scores_tc_kernel<2, true, 4> : router_scores_tc_kernel<2, false, 4>);
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, RouterSmem<2>::kDyn);
       kern<<<grid, RS_THREADS, RouterSmem<2>::kDyn, s>>>(tq, tk, scores, d.Lr, d.N, c2, tmask, ctx);
     } else {
-      auto kern = d.padded ? router_scores_tc_kernel<1, true> : router_scores_tc_kernel<1, false>;
+      auto kern = d.G == 16 ? router_scores_tc_kernel<1, false, 16>
+                            : (d.padded ? router_scores_tc_kernel<1, true, 4> : router_scores_tc_kernel<1, false, 4>);
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, RouterSmem<1>::kDyn);
       kern<<<grid, RS_THREADS, RouterSmem<1>::kDyn, s>>>(tq, tk, scores, d.Lr, d.N, c2, tmask, ctx);
     }
   } else {
     dim3 grid(d.N, d.BH);
-    if (d.D == 128)
-      router_scores_simt_kernel<float, 128><<<grid, 128, 0, s>>>((const float*)qr, (const float*)kr, scores, d.Lr, d.N,
-                                                                 tmask);
-    else
-      router_scores_simt_kernel<float, 64><<<grid, 128, 0, s>>>((const float*)qr, (const float*)kr, scores, d.Lr, d.N,
-                                                                tmask);
+    const float* fq = (const float*)qr;
+    const float* fk = (const float*)kr;
+    if (d.G == 16) {
+      if (d.D == 128)
+        router_scores_simt_kernel<float, 128, 16><<<grid, 128, 0, s>>>(fq, fk, scores, d.Lr, d.N, tmask);
+      else
+        router_scores_simt_kernel<float, 64, 16><<<grid, 128, 0, s>>>(fq, fk, scores, d.Lr, d.N, tmask);
+    } else if (d.D == 128) {
+      router_scores_simt_kernel<float, 128, 4><<<grid, 128, 0, s>>>(fq, fk, scores, d.Lr, d.N, tmask);
+    } else {
+      router_scores_simt_kernel<float, 64, 4><<<grid, 128, 0, s>>>(fq, fk, scores, d.Lr, d.N, tmask);
+    }
   }
   if (check_launch(__func__) != VSA2_OK) return VSA2_ERR_CUDA;
   return VSA2_OK;
