@@ -268,7 +268,7 @@ def run_reference(args, wl):
 # ----------------------------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------------------------
-def time_next_rows(e, x, wl, steps, stream, l2_flush, ev, hbm, tc_peak):
+def time_next_rows(e, x, wl, steps, stream, l2_flush, ev, hbm, tc_peak, sel=None):
     """The coarse branch (Eq. 1-3) and the gated merge (Eq. 4, 13-14), and for training
     workloads their gradients, each timed on its own after the step, with L2 flushed before every
     launch. They are not part of the fine-branch step that the headline metric times."""
@@ -328,6 +328,27 @@ def time_next_rows(e, x, wl, steps, stream, l2_flush, ev, hbm, tc_peak):
                                 "kernels": "pool + pad + attn_bwd_dq_tc_kernel + attn_bwd_dkdv_tc_kernel + "
                                            "coarse_pool_bwd_kernel"},
         }
+    if sel is not None:
+        # the fine forward with the gated merge in its epilogue (Eq. 12-14 in one pass), against the
+        # forward followed by the merge kernel; both on the step's selection
+        tf, ts = [], []
+        for it in range(3 + steps):
+            t = [ev() for _ in range(4)]
+            l2_flush.zero_()
+            t[0].record(stream)
+            e.attn_fwd_gated(x["q"], x["k"], x["v"], sel[0], sel[1], logits, oc)
+            t[1].record(stream)
+            l2_flush.zero_()
+            t[2].record(stream)
+            o_f, _ = e.attn_fwd(x["q"], x["k"], x["v"], sel[0], sel[1])
+            e.gated_merge(o_f, logits, oc, out=o_f)
+            t[3].record(stream)
+            torch.cuda.synchronize()
+            if it >= 3:
+                tf.append(t[0].elapsed_time(t[1]))
+                ts.append(t[2].elapsed_time(t[3]))
+        extra["fine_fwd_gated"] = {"ms": statistics.mean(tf), "fwd_then_merge_ms": statistics.mean(ts),
+                                   "kernel": "attn_fwd_tc_kernel<0, true> (merge in the epilogue)"}
     # the token permutation (§2.2): Q from raster to cube-major order, one read and one write
     tp = []
     for it in range(3 + steps):
@@ -456,12 +477,15 @@ def measure(args, wl, dev, rank, world):
     scores = torch.empty(wl.batch, wl.heads, wl.num_tiles, wl.num_tiles, dtype=torch.float32, device=dev)
     ev = lambda: torch.cuda.Event(enable_timing=True)
 
+    last_sel = {}
+
     def step(timers=None):
         t = timers or {}
         if t: t["r0"].record(stream)
         e.router_scores(x["q"], x["k"], out=scores)
         if t: t["r1"].record(stream)
         sel = e.topk_select(scores, wl.topk, csc=wl.backward)
+        last_sel["sel"] = sel
         if t: t["t1"].record(stream)
         o, lse = e.attn_fwd(x["q"], x["k"], x["v"], sel[0], sel[1])
         if t: t["f1"].record(stream)
@@ -533,13 +557,18 @@ def measure(args, wl, dev, rank, world):
     sm_max = load_sm_max_mhz()
     next_rows = None
     if not args.no_next and wl.dtype == "bf16":
-        next_rows = time_next_rows(e, x, wl, args.steps, stream, l2_flush, ev, hbm, bf16_burst)
+        next_rows = time_next_rows(e, x, wl, args.steps, stream, l2_flush, ev, hbm, bf16_burst,
+                                   sel=last_sel.get("sel") if wl.head_dim == 128 else None)
         if wl.name == HEADLINE and not wl.backward:
             dense = time_dense(x, wl, stream, l2_flush, ev)
             if "ms" in dense:
                 # the pages' ratio covers every op of Fig. 2 but the QKV projections: coarse branch,
-                # router, TopK, fine branch and gated merge
-                vsa2_ms = statistics.mean(per["step"]) + next_rows["coarse_attn"]["ms"] + next_rows["gated_merge"]["ms"]
+                # router, TopK, fine branch and gated merge (here the fine forward with the merge
+                # in its epilogue)
+                fused = next_rows.get("fine_fwd_gated", {}).get("ms")
+                vsa2_ms = statistics.mean(per["router"]) + statistics.mean(per["topk"]) + \
+                    next_rows["coarse_attn"]["ms"] + (fused if fused is not None else
+                                                      statistics.mean(per["fwd"]) + next_rows["gated_merge"]["ms"])
                 dense["vsa2_all_ops_ms"] = vsa2_ms
                 dense["speedup_all_ops"] = dense["ms"] / vsa2_ms
                 dense["speedup_fine_branch_step"] = dense["ms"] / statistics.mean(per["step"])
@@ -611,6 +640,110 @@ def measure(args, wl, dev, rank, world):
     return line
 
 
+def measure_sharded(args, wl, dev, rank, world):
+    """Strong scaling of one workload over the ranks (§8(e) of the design: the path shards by
+    (b, h)). --shard heads: rank r runs the router, TopK and forward of its heads (sharding
+    .shard_units) and nothing crosses ranks. --shard ulysses: rank r holds a contiguous 1/P of
+    the cube-major tokens of every head (a sequence-sharded model); one all-to-all per tensor
+    gathers whole sequences of H/P heads (App. E), the same path runs on them, and one
+    all-to-all returns the output shard; the two exchanges are timed beside the path. One step
+    = the whole workload over all ranks; the time is the max over ranks."""
+    import torch
+    import torch.distributed as dist
+    import trainable_block_sparse_fine_b200 as V
+    from trainable_block_sparse_fine_b200.sharding import max_over_ranks, shard_units
+    from trainable_block_sparse_fine_b200.ulysses import heads_to_seq, seq_to_heads
+
+    if wl.batch != 1 or wl.backward:
+        raise SystemExit("--shard takes the forward workloads with batch 1")
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    workers = max(1, min(16, len(os.sched_getaffinity(0)) // max(1, int(os.environ.get("LOCAL_WORLD_SIZE", world)))))
+    if args.shard == "heads":
+        heads = [h for _, h in shard_units(wl.batch, wl.heads, rank, world)]
+        x = {n: torch.from_numpy(S.make_tensor(wl, n, heads=heads, workers=workers)).to(dt).to(dev)
+             for n in ("q", "k", "v")}
+        hr = len(heads)
+    else:
+        if wl.heads % world or wl.tokens % world:
+            raise SystemExit("--shard ulysses needs heads and tokens divisible by the rank count")
+        if not dist.is_initialized():
+            import socket
+            with socket.socket() as sk:
+                sk.bind(("127.0.0.1", 0))
+                port = sk.getsockname()[1]
+            dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                    device_id=dev)
+        ls = wl.tokens // world
+        x = {}
+        for n in ("q", "k", "v"):
+            full = S.make_tensor(wl, n, workers=workers)
+            x[n] = torch.from_numpy(full[:, :, rank * ls:(rank + 1) * ls]).to(dt).to(dev).contiguous()
+            del full
+        hr = wl.heads // world
+    e = V.VSA2(wl.batch, hr, wl.head_dim, wl.grid, wl.dtype, wl.topk)
+    stream = torch.cuda.current_stream()
+    l2_flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def step(t=None):
+        if args.shard == "ulysses":
+            if t: t[0].record(stream)
+            xs = {n: seq_to_heads(x[n]) for n in ("q", "k", "v")}
+            if t: t[1].record(stream)
+        else:
+            xs = x
+        o, _, _ = e.forward(xs["q"], xs["k"], xs["v"])
+        if args.shard == "ulysses":
+            if t: t[2].record(stream)
+            o = heads_to_seq(o)
+            if t: t[3].record(stream)
+        return o
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    parts = {"a2a_in": [], "path": [], "a2a_out": [], "step": []}
+    if world > 1:
+        dist.barrier()
+    with Clocks(dev.index) as clk:
+        for _ in range(args.steps):
+            l2_flush.zero_()
+            t = [ev() for _ in range(4)]
+            if args.shard == "heads":
+                t[0].record(stream)
+                step()
+                t[3].record(stream)
+            else:
+                step(t)
+            torch.cuda.synchronize()
+            parts["step"].append(t[0].elapsed_time(t[3]))
+            if args.shard == "ulysses":
+                parts["a2a_in"].append(t[0].elapsed_time(t[1]))
+                parts["path"].append(t[1].elapsed_time(t[2]))
+                parts["a2a_out"].append(t[2].elapsed_time(t[3]))
+    if world > 1:
+        dist.barrier()
+    if e.device_error() != 0:
+        raise RuntimeError("device error in the sharded run")
+    ms = max_over_ranks(statistics.mean(parts["step"]), dev)
+    pairs = wl.batch * wl.heads * wl.num_tiles * wl.topk
+    value = pair_flops(wl, pairs, False) / (ms * 1e-3) / 1e12
+    if rank != 0:
+        return None
+    line = {"metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "fp32", "data": "synthetic",
+            "config": {"workload": wl.name, "shard": args.shard, "heads_per_rank": hr, "tokens": wl.tokens,
+                       "topk": wl.topk, "l2": "256 MB buffer written between timed steps"},
+            "clocks": clk.summary()}
+    if args.shard == "ulysses":
+        line["ulysses_ms"] = {k: statistics.mean(v) for k, v in parts.items() if k != "step"}
+        line["ulysses_bytes_per_rank"] = {
+            "a2a_in": 3 * wl.heads * (wl.tokens // world) * wl.head_dim * (2 if wl.dtype == "bf16" else 4),
+            "a2a_out": wl.heads * (wl.tokens // world) * wl.head_dim * (2 if wl.dtype == "bf16" else 4)}
+    return line
+
+
 def run_ours(args, wls):
     import torch
     import torch.distributed as dist
@@ -624,6 +757,17 @@ def run_ours(args, wls):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     dev = torch.device("cuda", local)
     lines = []
+    if args.shard != "batch":
+        for wl in wls:
+            if wl.backward:
+                continue  # the sharded modes time the forward path
+            line = measure_sharded(args, wl, dev, rank, world)
+            if line is not None:
+                print(json.dumps(line), flush=True)
+        if dist.is_initialized():
+            dist.barrier()
+            dist.destroy_process_group()
+        return
     for wl in wls:
         line = measure(args, wl, dev, rank, world)
         if line is not None:
@@ -658,6 +802,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--heads", type=int, default=None, help="override the head count (profiling runs)")
     ap.add_argument("--no-next", action="store_true", help="skip timing the coarse branch and the gated merge")
+    ap.add_argument("--shard", default="batch", choices=["batch", "heads", "ulysses"],
+                    help="batch (default): weak scaling, every rank its own batch element; heads / ulysses: "
+                         "strong scaling of one forward workload (a single --workload) split by heads, or "
+                         "held sequence-sharded with Ulysses all-to-alls around the per-head path")
     args = ap.parse_args()
     names = ALL_WORKLOADS if args.workload == "all" else [args.workload]
     wls = [S.WORKLOADS[n] for n in names]
