@@ -58,7 +58,14 @@ typedef enum {
 typedef enum { VSA2_BF16 = 0, VSA2_FP32 = 1 } vsa2_dtype;
 
 enum {
-  VSA2_FLAG_VALIDATE = 1u << 0 /* kernels bounds-check every offset and index they read */
+  VSA2_FLAG_VALIDATE = 1u << 0, /* kernels bounds-check every offset and index they read */
+  /* Eq. 1's pooled Q and K (the coarse branch's 64-token means) from the router's read of Q and
+   * K: with this flag, vsa2_router_scores also writes them into the workspace, and
+   * vsa2_coarse_attn reads them from there and pools only V. The caller must call
+   * vsa2_router_scores with the flag on the same q, k and workspace before vsa2_coarse_attn
+   * with the flag. Takes effect for bf16, D = 128, 64-token tiles with 16-token sub-cubes; the
+   * two calls ignore it otherwise (vsa2_coarse_attn then pools Q and K itself). */
+  VSA2_FLAG_COARSE_POOL_IN_ROUTER = 1u << 1
 };
 
 typedef struct vsa2_problem {
@@ -88,7 +95,8 @@ vsa2_status vsa2_workspace_init(void* ws, size_t ws_bytes, void* stream);
  *             L/R pooled keys of (b, h) (Eq. 6), pooled G x G (Eq. 7) and scaled by G so each
  *             row sums to 1 (the pages' MeanPool_{GxG} divided by G; TopK is unaffected).
  * The pooled Qr, Kr and per-row LSE live in the workspace; the L/R x L/R matrix is never
- * written to memory.
+ * written to memory. With VSA2_FLAG_COARSE_POOL_IN_ROUTER the pooling pass also writes the
+ * coarse branch's Qc, Kc (Eq. 1) into the workspace for a following vsa2_coarse_attn.
  */
 vsa2_status vsa2_router_scores(const vsa2_problem* p, const void* q, const void* k, float* scores,
                                void* ws, size_t ws_bytes, void* stream);
@@ -181,6 +189,8 @@ vsa2_status vsa2_sparse_attn_bwd(const vsa2_problem* p, const void* q, const voi
  *   lse_c   : [batch, heads, N] fp32 (written), or NULL
  * The pooled rows are rounded to dtype before the attention (as the inputs of the fine branch
  * are); the softmax and accumulation are fp32. Uses the workspace of vsa2_workspace_size().
+ * With VSA2_FLAG_COARSE_POOL_IN_ROUTER (see the flag) Qc and Kc are the ones the preceding
+ * vsa2_router_scores call left in the workspace, and only V is read here.
  */
 vsa2_status vsa2_coarse_attn(const vsa2_problem* p, const void* q, const void* k, const void* v, void* oc,
                              float* lse_c, void* ws, size_t ws_bytes, void* stream);

@@ -32,6 +32,13 @@ def test_problem_struct_layout():
     assert C.Problem.dtype.offset == 72
 
 
+def test_flag_values_match_the_header():
+    text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "vsa2.h")).read(), flags=re.S)
+    flags = {name: 1 << int(bit) for name, bit in re.findall(r"\b(VSA2_FLAG_[A-Z_]+)\s*=\s*1u\s*<<\s*(\d+)", text)}
+    assert flags == {"VSA2_FLAG_VALIDATE": C.VSA2_FLAG_VALIDATE,
+                     "VSA2_FLAG_COARSE_POOL_IN_ROUTER": C.VSA2_FLAG_COARSE_POOL_IN_ROUTER}
+
+
 def test_status_strings_and_version():
     for code, name in C.STATUS_NAMES.items():
         assert C.vsa2_status_string(code) == name

@@ -72,6 +72,26 @@ def test_coarse_attn_matches_oracle(case):
             _close(oc[b, h], want, f"{case} oc[{b},{h}]", lse_c[b, h], want_lse)
 
 
+@pytest.mark.parametrize("case", list(CASES))
+def test_coarse_attn_with_pooling_in_the_router(case):
+    """VSA2_FLAG_COARSE_POOL_IN_ROUTER: Qc and Kc (Eq. 1) come from the router's pass over Q and
+    K and the coarse call reads only V (bf16, D = 128). The other cases ignore the flag in both
+    calls and pool Q and K in the coarse call. The workspace is fresh, so Qc and Kc are read from
+    what the router call wrote."""
+    wl = CASES[case]
+    x = {n: S.make_tensor(wl, n) for n in "qkv"}
+    e = _engine(wl)
+    xd = {n: _dev(x[n], wl.dtype) for n in "qkv"}
+    e.router_scores(xd["q"], xd["k"], coarse_pool=True)
+    oc, lse_c = e.coarse_attn(xd["q"], xd["k"], xd["v"], pooled_qk=True)
+    assert e.device_error() == 0
+    oc, lse_c = oc.float().cpu().numpy(), lse_c.cpu().numpy()
+    for b in range(wl.batch):
+        for h in range(wl.heads):
+            want, want_lse = O.coarse_attn(x["q"][b, h], x["k"][b, h], x["v"][b, h])
+            _close(oc[b, h], want, f"{case} oc[{b},{h}]", lse_c[b, h], want_lse)
+
+
 def test_coarse_attn_480p_two_heads():
     """480p: 728 pooled rows per head, 12 tiles of which the last holds 24 rows."""
     wl480 = S.WORKLOADS["480p_top64"]

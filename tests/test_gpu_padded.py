@@ -68,8 +68,10 @@ def test_padded_grid_path_matches_oracle(case):
     xd = {n: e.to_cube_major(_dev(x[n], dtype)) for n in "qkv"}
     assert xd["q"].shape[2] == e.L and e.L % 64 == 0 and e.L > e.L_real
     N = e.N
-    scores = e.router_scores(xd["q"], xd["k"]).cpu().numpy()
+    # the router's pooling pass also leaves the coarse branch's Qc, Kc (Eq. 1, over real tokens)
+    scores = e.router_scores(xd["q"], xd["k"], coarse_pool=True).cpu().numpy()
     o_sc = np.zeros((1, heads, N, N), np.float32)
+    oc_fold = e.coarse_attn(xd["q"], xd["k"], xd["v"], pooled_qk=True)[0].float().cpu().numpy()
     oc_all = e.coarse_attn(xd["q"], xd["k"], xd["v"])[0].float().cpu().numpy()
     sels = []
     for h in range(heads):
@@ -84,7 +86,9 @@ def test_padded_grid_path_matches_oracle(case):
         assert rel <= 5e-3 and np.abs(g - want).max() <= 1e-2 * want.max(), (h, rel)
         np.testing.assert_allclose(g.sum(1), 1.0, atol=5e-3)
         o_sc[0, h] = want.astype(np.float32)
-        _close(oc_all[0, h], O.coarse_attn_padded(qc, kc, vc, vm), f"coarse h{h}")
+        want_c = O.coarse_attn_padded(qc, kc, vc, vm)
+        _close(oc_all[0, h], want_c, f"coarse h{h}")
+        _close(oc_fold[0, h], want_c, f"coarse, Qc and Kc from the router, h{h}")
         sels.append((qc, kc, vc, vm))
     # TopK over the padded grid's tiles, bit-exact on the oracle's fp32 scores
     kv_off, kv_idx, q_off, q_idx = e.topk_select(torch.from_numpy(o_sc).cuda(), topk, csc=True)

@@ -11,7 +11,7 @@ from __future__ import annotations
 
 import torch
 
-from ._capi import (VSA2_FLAG_VALIDATE, Problem, Vsa2Error, lib, make_problem, vsa2_coarse_attn,
+from ._capi import (VSA2_FLAG_COARSE_POOL_IN_ROUTER, VSA2_FLAG_VALIDATE, Problem, Vsa2Error, lib, make_problem, vsa2_coarse_attn,
                     vsa2_coarse_attn_bwd, vsa2_forward_host, vsa2_forward_host_workspace_size, vsa2_gated_merge,
                     vsa2_gated_merge_bwd, vsa2_get_device_error, vsa2_permute_tokens, vsa2_router_scores,
                     vsa2_selftest_wait_timeout, vsa2_sparse_attn_bwd, vsa2_sparse_attn_fwd,
@@ -20,7 +20,7 @@ from ._capi import (VSA2_FLAG_VALIDATE, Problem, Vsa2Error, lib, make_problem, v
 
 from .ulysses import heads_to_seq, seq_to_heads, ulysses_attention
 
-__all__ = ["VSA2", "ulysses_attention", "seq_to_heads", "heads_to_seq", "Vsa2Error", "Problem", "make_problem", "block_sparse_attention", "lib", "VSA2_FLAG_VALIDATE",
+__all__ = ["VSA2", "ulysses_attention", "seq_to_heads", "heads_to_seq", "Vsa2Error", "Problem", "make_problem", "block_sparse_attention", "lib", "VSA2_FLAG_VALIDATE", "VSA2_FLAG_COARSE_POOL_IN_ROUTER",
            "vsa2_router_scores", "vsa2_topk_select", "vsa2_sparse_attn_fwd", "vsa2_sparse_attn_bwd",
            "vsa2_workspace_size", "vsa2_workspace_init", "vsa2_get_device_error", "vsa2_selftest_wait_timeout",
            "vsa2_status_string", "vsa2_version", "vsa2_forward_host", "vsa2_forward_host_workspace_size",
@@ -40,6 +40,10 @@ class VSA2:
         lib()  # fail loudly if the native library is missing
         self.p = make_problem(batch, heads, head_dim, grid, dtype, tile=tuple(tile), pool=tuple(pool), flags=flags,
                               wait_timeout_ms=wait_timeout_ms)
+        # the same problem for the whole-attention calls: the router's pass over Q and K also
+        # writes the coarse branch's pooled Qc, Kc (Eq. 1), and the coarse call then reads only V
+        self.p_fold = make_problem(batch, heads, head_dim, grid, dtype, tile=tuple(tile), pool=tuple(pool),
+                                   flags=flags | VSA2_FLAG_COARSE_POOL_IN_ROUTER, wait_timeout_ms=wait_timeout_ms)
         self.tile, self.pool = tuple(tile), tuple(pool)
         self.batch, self.heads, self.head_dim, self.grid, self.topk = batch, heads, head_dim, tuple(grid), topk
         # a grid the 4x4x4 tile does not divide is padded to whole tiles (§2.2 "Kernel
@@ -58,10 +62,12 @@ class VSA2:
         vsa2_workspace_init(self.ws)
 
     # -- the calls of the hot path -----------------------------------------------------------
-    def router_scores(self, q, k, out=None):
+    def router_scores(self, q, k, out=None, coarse_pool=False):
+        """Eq. 5-7 scores [B, H, N, N]. coarse_pool: also leave the coarse branch's pooled Q and K
+        in the workspace for a following coarse_attn(..., pooled_qk=True)."""
         out = out if out is not None else torch.empty(self.batch, self.heads, self.N, self.N, dtype=torch.float32,
                                                       device=self.device)
-        vsa2_router_scores(self.p, q, k, out, self.ws)
+        vsa2_router_scores(self.p_fold if coarse_pool else self.p, q, k, out, self.ws)
         return out
 
     def topk_select(self, scores, topk=None, csc=True):
@@ -135,13 +141,14 @@ class VSA2:
         vsa2_permute_tokens(self.p, x, out, False)
         return out
 
-    def coarse_attn(self, q, k, v, oc=None, lse_c=None):
-        """Coarse branch, Eq. 1-3: O_c_hat [B, H, N, D] (input dtype) and its LSE [B, H, N]."""
+    def coarse_attn(self, q, k, v, oc=None, lse_c=None, pooled_qk=False):
+        """Coarse branch, Eq. 1-3: O_c_hat [B, H, N, D] (input dtype) and its LSE [B, H, N].
+        pooled_qk: take Qc, Kc from the preceding router_scores(q, k, coarse_pool=True) call."""
         oc = oc if oc is not None else torch.empty(self.batch, self.heads, self.N, self.head_dim, dtype=q.dtype,
                                                    device=self.device)
         lse_c = lse_c if lse_c is not None else torch.empty(self.batch, self.heads, self.N, dtype=torch.float32,
                                                             device=self.device)
-        vsa2_coarse_attn(self.p, q, k, v, oc, lse_c, self.ws)
+        vsa2_coarse_attn(self.p_fold if pooled_qk else self.p, q, k, v, oc, lse_c, self.ws)
         return oc, lse_c
 
     def gated_merge(self, o_f, gate_logits, oc, out=None):
@@ -165,9 +172,9 @@ class VSA2:
     def attention(self, q, k, v, gate_logits, topk=None):
         """The whole VSA2 attention output, Eq. 14: fine branch (router, TopK, Eq. 12) plus the
         gated coarse branch. Returns o."""
-        scores = self.router_scores(q, k)
+        scores = self.router_scores(q, k, coarse_pool=True)
         kv_off, kv_idx, _, _ = self.topk_select(scores, topk, csc=False)
-        oc, _ = self.coarse_attn(q, k, v)
+        oc, _ = self.coarse_attn(q, k, v, pooled_qk=True)
         return self.attn_fwd_gated(q, k, v, kv_off, kv_idx, gate_logits, oc, topk)[0]
 
     def forward_host(self, q, k, v, topk=None, o=None, lse=None, heads_per_group=0, want_lse=False):
@@ -220,9 +227,9 @@ class _Vsa2Attention(torch.autograd.Function):
     @staticmethod
     def forward(ctx, q, k, v, gate_logits, engine: VSA2, topk):
         with torch.no_grad():  # the router receives no gradient (§2.1)
-            scores = engine.router_scores(q, k)
+            scores = engine.router_scores(q, k, coarse_pool=True)
             kv_off, kv_idx, q_off, q_idx = engine.topk_select(scores, topk, csc=True)
-        oc, lse_c = engine.coarse_attn(q, k, v)
+        oc, lse_c = engine.coarse_attn(q, k, v, pooled_qk=True)
         o, lse, o_f = engine.attn_fwd_gated(q, k, v, kv_off, kv_idx, gate_logits.contiguous(), oc, topk,
                                             want_fine=True)
         ctx.save_for_backward(q, k, v, o_f, lse, kv_off, kv_idx, q_off, q_idx, oc, lse_c, gate_logits)

@@ -15,6 +15,7 @@ STATUS_NAMES = {0: "VSA2_OK", 1: "VSA2_ERR_INVALID_ARG", 2: "VSA2_ERR_UNSUPPORTE
                 4: "VSA2_ERR_TIMEOUT", 5: "VSA2_ERR_BAD_INDEX"}
 VSA2_BF16, VSA2_FP32 = 0, 1
 VSA2_FLAG_VALIDATE = 1
+VSA2_FLAG_COARSE_POOL_IN_ROUTER = 2
 
 # every symbol the header declares
 EXPORTS = ("vsa2_workspace_size", "vsa2_workspace_init", "vsa2_router_scores", "vsa2_topk_select",

@@ -61,12 +61,14 @@ __device__ __forceinline__ void store_vec(T* p, const float* f) {
 
 // Eq. 1: warp per pooled row r of head bh; lane owns D/32 consecutive channels. Rows r >= N
 // (padding of the last tile) are written as zeros. With tmask (a padded grid) each mean runs
-// over the tile's real tokens only.
+// over the tile's real tokens only. With v_only the rows r < N of Qc and Kc are left as they are
+// (the router's pooling pass wrote them) and only V is read.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) coarse_pool_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                           const T* __restrict__ v, T* __restrict__ qc,
                                                           T* __restrict__ kc, T* __restrict__ vc, int N, int Lc,
-                                                          int64_t L, const uint64_t* __restrict__ tmask) {
+                                                          int64_t L, const uint64_t* __restrict__ tmask,
+                                                          bool v_only) {
   constexpr int V = D / 32;
   const int bh = blockIdx.y;
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -77,6 +79,7 @@ __global__ void __launch_bounds__(256) coarse_pool_kernel(const T* __restrict__ 
   T* out[3] = {qc, kc, vc};
 #pragma unroll
   for (int x = 0; x < 3; ++x) {
+    if (v_only && x < 2 && r < N) continue;
     float acc[V];
 #pragma unroll
     for (int e = 0; e < V; ++e) acc[e] = 0.f;
@@ -241,10 +244,11 @@ __global__ void __launch_bounds__(256) coarse_pool_bwd_kernel(const float* __res
 
 template <typename T, int D>
 void launch_pool(const Dims& d, const void* q, const void* k, const void* v, char* ws, const WsLayout& w,
-                 const uint64_t* tmask, cudaStream_t s) {
+                 const uint64_t* tmask, cudaStream_t s, bool v_only = false) {
   const int Lc = kTile * w.Nc_tiles;
   coarse_pool_kernel<T, D><<<dim3((Lc + 7) / 8, d.BH), 256, 0, s>>>(
-      (const T*)q, (const T*)k, (const T*)v, (T*)(ws + w.qc), (T*)(ws + w.kc), (T*)(ws + w.vc), d.N, Lc, d.L, tmask);
+      (const T*)q, (const T*)k, (const T*)v, (T*)(ws + w.qc), (T*)(ws + w.kc), (T*)(ws + w.vc), d.N, Lc, d.L, tmask,
+      v_only);
 }
 
 int grid_for(int64_t work, int per_block) {
@@ -267,7 +271,7 @@ vsa2_status launch_coarse_attn(const Dims& d, const void* q, const void* k, cons
     if (launch_tile_masks(d, tmask, s) != VSA2_OK) return VSA2_ERR_CUDA;
   }
   if (d.dtype == VSA2_BF16 && d.D == 128)
-    launch_pool<__nv_bfloat16, 128>(d, q, k, v, ws, w, tmask, s);
+    launch_pool<__nv_bfloat16, 128>(d, q, k, v, ws, w, tmask, s, coarse_pool_in_router(d));
   else if (d.dtype == VSA2_BF16)
     launch_pool<__nv_bfloat16, 64>(d, q, k, v, ws, w, tmask, s);
   else if (d.D == 128)

@@ -46,6 +46,13 @@ inline Dims dims64(const Dims& d) {
   return e;
 }
 
+// VSA2_FLAG_COARSE_POOL_IN_ROUTER in effect: the router's pooling pass writes the coarse branch's
+// Qc, Kc and the coarse branch pools only V (bf16, D = 128, 64-token tiles of 16-token sub-cubes).
+inline bool coarse_pool_in_router(const Dims& d) {
+  return (d.flags & VSA2_FLAG_COARSE_POOL_IN_ROUTER) && d.dtype == VSA2_BF16 && d.D == 128 && d.Bt == kTile &&
+         d.R == kPool;
+}
+
 // Real-token mask of every tile of a padded grid (bit u = cube-major token u of the tile is a
 // token of the real grid); the same for every (b, h). Enqueued on `s`, written to `mask` [N].
 vsa2_status launch_tile_masks(const Dims& d, uint64_t* mask, cudaStream_t s);

@@ -16,11 +16,16 @@ namespace {
 // ------------------------------------------------------------------------------------------
 // With kMask (a padded grid), each mean runs over the sub-cube's real tokens only (tmask, the
 // per-tile real-token masks); a sub-cube without one is written as zeros.
-template <typename T, bool kMask, int R>
+// With kCoarse (bf16, D = 128, R = 16: a tile's four sub-cubes are the 64 consecutive threads of
+// a warp pair) the same read also gives the coarse branch's tile means (Eq. 1) over the tile's
+// real tokens, written as row (b*h) * Lc + tile of qc / kc.
+template <typename T, bool kMask, int R, bool kCoarse = false>
 __global__ void __launch_bounds__(256) router_pool_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                           T* __restrict__ qr, T* __restrict__ kr,
                                                           int64_t pooled_rows, int chunks_per_row,
-                                                          const uint64_t* __restrict__ tmask, int Lr) {
+                                                          const uint64_t* __restrict__ tmask, int Lr,
+                                                          T* __restrict__ qc, T* __restrict__ kc, int Lc) {
+  static_assert(!kCoarse || (sizeof(T) == 2 && R == 16), "tile means need 16 chunks per row and 4 sub-cubes");
   constexpr int EPC = 16 / sizeof(T);  // elements per 16-byte chunk
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t per_tensor = pooled_rows * chunks_per_row;
@@ -73,6 +78,39 @@ __global__ void __launch_bounds__(256) router_pool_kernel(const T* __restrict__ 
     for (int e = 0; e < 4; ++e) o[e] = acc[e] * inv;
   }
   *reinterpret_cast<uint4*>(dst) = out;
+  if constexpr (kCoarse) {
+    // rows 4T .. 4T+3 of tile T are threads 64T + 16g + chunk (g < 4): lanes 0-15 / 16-31 of the
+    // pair's two warps. (Each 64-thread group is active or inactive as a whole: pooled_rows is a
+    // multiple of 4 and the block holds 256 threads.)
+    __shared__ float part[4][16][EPC + 1];
+    float cnt = kMask ? (float)__popc(valid) : (float)R;
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, 16);
+    const int pair = threadIdx.x >> 6;
+    const bool upper = threadIdx.x & 32;
+    const int lane = threadIdx.x & 31;
+    if (upper && lane < 16) {
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) part[pair][lane][e] = acc[e];
+      part[pair][lane][EPC] = cnt;
+    }
+    named_bar_sync(1 + pair, 64);
+    if (!upper && lane < 16) {
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) acc[e] += part[pair][lane][e];
+      cnt += part[pair][lane][EPC];
+      const float ti = cnt > 0.f ? 1.f / cnt : 0.f;
+      const int64_t bh = prow / Lr;
+      const int tile = (int)(prow % Lr) >> 2;
+      T* cdst = (is_k ? kc : qc) + ((bh * Lc + tile) * chunks_per_row + chunk) * EPC;
+      uint4 co;
+      uint32_t* o = reinterpret_cast<uint32_t*>(&co);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[e] = pack_bf16(acc[2 * e] * ti, acc[2 * e + 1] * ti);
+      *reinterpret_cast<uint4*>(cdst) = co;
+    }
+  }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -485,15 +523,19 @@ vsa2_status launch_router(const Dims& d, const void* q, const void* k, float* sc
     if (launch_tile_masks(d, reinterpret_cast<uint64_t*>(ws + w.tmask), s) != VSA2_OK) return VSA2_ERR_CUDA;
   }
   if (d.dtype == VSA2_BF16) {
-    auto kern = d.R == 8 ? router_pool_kernel<__nv_bfloat16, false, 8>
-                         : (d.padded ? router_pool_kernel<__nv_bfloat16, true, 16>
-                                     : router_pool_kernel<__nv_bfloat16, false, 16>);
-    kern<<<blocks, 256, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)qr,
-                                (__nv_bfloat16*)kr, pooled, cpr, tmask, d.Lr);
+    using bf = __nv_bfloat16;
+    const bool fold = coarse_pool_in_router(d);
+    auto kern = d.R == 8 ? router_pool_kernel<bf, false, 8>
+                         : (d.padded ? (fold ? router_pool_kernel<bf, true, 16, true> : router_pool_kernel<bf, true, 16>)
+                                     : (fold ? router_pool_kernel<bf, false, 16, true> : router_pool_kernel<bf, false, 16>));
+    kern<<<blocks, 256, 0, s>>>((const bf*)q, (const bf*)k, (bf*)qr, (bf*)kr, pooled, cpr, tmask, d.Lr,
+                                fold ? (bf*)(ws + w.qc) : nullptr, fold ? (bf*)(ws + w.kc) : nullptr,
+                                kTile * w.Nc_tiles);
   } else {
     auto kern = d.R == 8 ? router_pool_kernel<float, false, 8>
                          : (d.padded ? router_pool_kernel<float, true, 16> : router_pool_kernel<float, false, 16>);
-    kern<<<blocks, 256, 0, s>>>((const float*)q, (const float*)k, (float*)qr, (float*)kr, pooled, cpr, tmask, d.Lr);
+    kern<<<blocks, 256, 0, s>>>((const float*)q, (const float*)k, (float*)qr, (float*)kr, pooled, cpr, tmask, d.Lr,
+                                nullptr, nullptr, 0);
   }
   if (check_launch(__func__) != VSA2_OK) return VSA2_ERR_CUDA;
 
