@@ -146,26 +146,37 @@ def run(tiles, rst, producers, rng, mma_latency=3, lead=1):
     assert pvdone.phases == sum(tiles) and all(p == len(ops) for p in prod)
 
 
-def run_aliased(tiles, rst, rng, mma_latency=3, rescale_p=0.2, lead=1):
+def run_aliased(tiles, rst, rng, mma_latency=3, rescale_p=0.2, lead=1, halves=1, xch_bufs=2, sfree_count=None):
     """The forward kernel's protocol with P written over the S buffer it came from: per slot two
     S/P buffers, pfull and pvdone per block parity, no wait for the previous P.V before writing P;
     the softmax waits for the previous P.V only to rescale O (at random here) and at a tile's end.
     The tensor pipe completes MMAs in issue order. Asserts, besides the parity rule, that S(k)
     overwrites a buffer only after O(k-2) read its P, that P(g) is written only after O(g-2)
-    read the previous P of the buffer, and that O is read only after every P.V issued before."""
+    read the previous P of the buffer, and that O is read only after every P.V issued before.
+
+    `halves` = 2 models the softmax split over two warps per lane quarter, each owning one KV tile
+    of the block: each half reads its S columns and writes its P inside them, the halves meet at a
+    pair barrier once per block to combine the row max through a shared-memory slot chosen by
+    block parity (`xch_bufs` slots), and once at a tile's end to combine the row sums. sfree and
+    pfull then expect one arrival per half. The model asserts that an exchange slot is rewritten
+    only after the other half read it, and that S(k) overwrites a buffer only after every half
+    read S(k-2)."""
     ops = ops_of(tiles, lead=lead)
     full = [Barrier(1) for _ in range(rst)]
     empty = [Barrier(1) for _ in range(rst)]
-    sfull, sfree = [Barrier(1), Barrier(1)], [Barrier(1), Barrier(1)]
-    pfull, pvdone = [Barrier(4), Barrier(4)], [Barrier(1), Barrier(1)]
-    for b in pfull:
-        b.count = 1  # one arrival stands for the four softmax warps
+    sfc = halves if sfree_count is None else sfree_count
+    sfull, sfree = [Barrier(1), Barrier(1)], [Barrier(sfc), Barrier(sfc)]
+    pfull, pvdone = [Barrier(halves), Barrier(halves)], [Barrier(1), Barrier(1)]
     prod = {"c": 0}
     mma = {"c": 0, "s": 0, "o": 0}
-    soft = {"blk": 0, "step": 0, "tile": 0, "in_tile": 0}
+    soft = [{"blk": 0, "step": 0} for _ in range(halves)]
     done = {"op": set(), "s": set(), "o": set()}
-    p_written = set()
-    ends = []                      # block index that ends each tile
+    p_written = [set() for _ in range(halves)]
+    s_read = [set() for _ in range(halves)]
+    gen = [0] * halves               # pair-barrier arrivals per half
+    xslot = {}                       # (kind, slot, half) -> [value, halves that have read it]
+    rescale = {}                     # block -> rescale decision, the same for every half
+    ends = []                        # block index that ends each tile
     acc = 0
     for n in tiles:
         acc += n
@@ -202,6 +213,7 @@ def run_aliased(tiles, rst, rng, mma_latency=3, rescale_p=0.2, lead=1):
 
             def fin(c=c, k=k, st=st):
                 assert k < 2 or k - 2 in done["o"], f"S{k} overwrote P{k - 2} before O{k - 2} read it"
+                assert k < 2 or all(k - 2 in r for r in s_read), f"S{k} overwrote S{k - 2} before every half read it"
                 done["op"].add(c)
                 done["s"].add(k)
                 empty[st].arrive()
@@ -211,7 +223,7 @@ def run_aliased(tiles, rst, rng, mma_latency=3, rescale_p=0.2, lead=1):
             k = mma["o"]
             if not pfull[k % 2].poll(k // 2, f"issuer O{k}"):
                 return False
-            assert k in p_written
+            assert all(k in w for w in p_written), f"O{k} issued before every half wrote P{k}"
 
             def fin(c=c, k=k, st=st):
                 done["op"].add(c)
@@ -227,42 +239,77 @@ def run_aliased(tiles, rst, rng, mma_latency=3, rescale_p=0.2, lead=1):
     def wait_pv(g, who):
         return pvdone[g % 2].poll(g // 2, who)
 
-    def softmax():
-        g = soft["blk"]
+    def put(kind, slot, h, value):
+        old = xslot.get((kind, slot, h))
+        assert old is None or len(old[1]) == halves - 1, f"{kind} slot {slot} of half {h} rewritten before it was read"
+        xslot[(kind, slot, h)] = [value, set()]
+        gen[h] += 1
+
+    def take(kind, slot, h, value):
+        if any(gen[j] < gen[h] for j in range(halves)):
+            return False  # the pair barrier: every half has arrived
+        for j in range(halves):
+            if j != h:
+                v = xslot[(kind, slot, j)]
+                assert v[0] == value, f"half {h} read {kind} {v[0]} for {value}"
+                v[1].add(h)
+        return True
+
+    def softmax(h):
+        sm = soft[h]
+        g = sm["blk"]
         if g >= nblk:
             return False
-        st = soft["step"]
-        if st == 0:                       # wait S, read it, free the buffer
+        st = sm["step"]
+        if st == 0:                       # wait S, read this half's columns, free the buffer
             if not sfull[g % 2].poll(g // 2, f"softmax S{g}"):
                 return False
             assert g in done["s"]
+            s_read[h].add(g)
             sfree[g % 2].arrive()
-            first = g == 0 or (g - 1) in ends
-            soft["step"] = 1 if (not first and rng.random() < rescale_p) else 2
+            sm["step"] = 1
             return True
-        if st == 1:                       # rescale O: the previous P.V must be done
+        if st == 1:                       # row max of this half into the exchange slot
+            put("max", g % xch_bufs, h, g)
+            sm["step"] = 2
+            return True
+        if st == 2:                       # pair barrier, then the other halves' max
+            if not take("max", g % xch_bufs, h, g):
+                return False
+            first = g == 0 or (g - 1) in ends
+            r = rescale.setdefault(g, (not first) and rng.random() < rescale_p)
+            sm["step"] = 3 if r else 4
+            return True
+        if st == 3:                       # rescale O: the previous P.V must be done
             if not wait_pv(g - 1, f"softmax rescale at {g}"):
                 return False
             assert all(x in done["o"] for x in range(g)), f"O read at block {g} with a P.V pending"
-            soft["step"] = 2
+            sm["step"] = 4
             return True
-        if st == 2:                       # write P over the S buffer
+        if st == 4:                       # write P over this half's S columns
             assert g < 2 or g - 2 in done["o"], f"P{g} written before O{g - 2} read P{g - 2}"
-            p_written.add(g)
+            p_written[h].add(g)
             pfull[g % 2].arrive()
-            soft["step"] = 3 if g in ends else 0
-            if g not in ends:
-                soft["blk"] = g + 1
+            if g in ends:
+                sm["step"] = 5
+            else:
+                sm["blk"], sm["step"] = g + 1, 0
             return True
-        if not wait_pv(g, f"softmax epilogue at {g}"):  # st == 3: tile's last P.V, then O
+        if st == 5:                       # tile's last P.V, then this half's row sum
+            if not wait_pv(g, f"softmax epilogue at {g}"):
+                return False
+            assert all(x in done["o"] for x in range(g + 1)), f"epilogue at {g} with a P.V pending"
+            put("sum", 0, h, g)
+            sm["step"] = 6
+            return True
+        if not take("sum", 0, h, g):      # st == 6: pair barrier, the other halves' sums
             return False
-        assert all(x in done["o"] for x in range(g + 1)), f"epilogue at {g} with a P.V pending"
-        soft["blk"], soft["step"] = g + 1, 0
+        sm["blk"], sm["step"] = g + 1, 0
         return True
 
-    agents = [producer, issuer, softmax]
+    agents = [producer, issuer] + [lambda h=h: softmax(h) for h in range(halves)]
     speed = [rng.uniform(0.05, 1.0) for _ in agents]
-    while mma["c"] < len(ops) or soft["blk"] < nblk or pending:
+    while mma["c"] < len(ops) or any(sm["blk"] < nblk for sm in soft) or pending:
         t += 1
         due = [x for x in pending if x[0] <= t]
         pending[:] = [x for x in pending if x[0] > t]
@@ -273,7 +320,7 @@ def run_aliased(tiles, rst, rng, mma_latency=3, rescale_p=0.2, lead=1):
             if rng.random() < speed[i]:
                 moved |= agents[i]()
         if not moved and not pending and not any(a() for a in agents):
-            raise AssertionError(f"deadlock at op {mma['c']} of {len(ops)}, softmax block {soft['blk']}")
+            raise AssertionError(f"deadlock at op {mma['c']} of {len(ops)}, softmax blocks {[sm['blk'] for sm in soft]}")
     assert len(done["o"]) == nblk
 
 
@@ -282,6 +329,30 @@ def test_forward_protocol_with_p_over_s(seed):
     rng = random.Random(seed)
     tiles = [rng.choice([1, 1, 2, 3, 4, 5, 7, 32]) for _ in range(rng.randint(1, 6))]
     run_aliased(tiles, rst=3, rng=rng, mma_latency=rng.choice([1, 3, 10, 30]))
+
+
+@pytest.mark.parametrize("seed", range(80))
+def test_forward_protocol_split_softmax(seed):
+    """Two softmax warps per lane quarter (one per KV tile of a block), as the kernel runs it."""
+    rng = random.Random(seed)
+    tiles = [rng.choice([1, 1, 2, 3, 4, 5, 7, 32]) for _ in range(rng.randint(1, 6))]
+    run_aliased(tiles, rst=3, rng=rng, mma_latency=rng.choice([1, 3, 10, 30]), halves=2)
+
+
+def test_forward_protocol_split_flags_a_single_exchange_slot():
+    """One row-max slot per half instead of one per block parity: a fast half rewrites it for the
+    next block before the other half has read it."""
+    with pytest.raises(AssertionError):
+        for seed in range(200):
+            run_aliased([32, 5], rst=3, rng=random.Random(seed), mma_latency=3, halves=2, xch_bufs=1)
+
+
+def test_forward_protocol_split_flags_one_sfree_arrival():
+    """With sfree released by one arrival, S(k+2) can overwrite a buffer the other half has not
+    read yet."""
+    with pytest.raises(AssertionError):
+        for seed in range(200):
+            run_aliased([32, 5], rst=3, rng=random.Random(seed), mma_latency=1, halves=2, sfree_count=1)
 
 
 def test_forward_protocol_flags_a_single_pfull_barrier():
@@ -480,14 +551,19 @@ def test_dkdv_protocol_parity_and_progress(seed):
     run_dkdv(items, rng, mma_latency=rng.choice([1, 3, 10]))
 
 
-def run_dq(items, rng, unified, mma_latency=3):
+def run_dq(items, rng, unified, mma_latency=3, ds_smem=True, ds_wait=True):
     """The dQ kernel's per-slot protocol: per block n of a query tile, op A(n) runs S = Q K^T
-    and dP = dO V^T from block n's K and V, after B(n-1) has finished reading dS (which
-    overwrote S); the softmax turns S, dP into dS; op B(n) runs dQ += dS K from the same K block
-    and releases it. Op order A0, B0, A1, B1, ... As built, K blocks have a ring of 2 and V
-    blocks a ring of 1, V released by A, K by B. With `unified`, K(n), V(n) share one ring of 3
-    in load order (the change made in the forward kernel), so a stage's releases must still
-    arrive in position order."""
+    and dP = dO V^T from block n's K and V; the softmax turns S, dP into dS; op B(n) runs
+    dQ += dS K from the same K block and releases it. K blocks have a ring of 2 and V blocks a
+    ring of 1, V released by A, K by B. With `unified`, K(n), V(n) share one ring of 3 in load
+    order, so a stage's releases must still arrive in position order.
+
+    As built (`ds_smem`), the softmax writes dS to shared memory: it frees S/dP (sfree) as soon as
+    both are in registers, and waits for B(n-1) before writing dS(n) over the buffer B(n-1) reads.
+    The issuer then runs A(n+1) before B(n) (order A0, A1, B0, A2, B1, ...), and the tensor pipe
+    completes MMAs in issue order. The earlier layout (dS written over S in tensor memory, order
+    A0, B0, A1, B1, ..., A(n) after B(n-1) done) is kept as `ds_smem=False`. `ds_wait=False`
+    drops the softmax's wait for B(n-1) (a seeded mistake)."""
     nblk = sum(items)
     nonempty = [k for k in items if k]
     item_start = set()
@@ -495,6 +571,7 @@ def run_dq(items, rng, unified, mma_latency=3):
     for k in nonempty:
         item_start.add(acc)
         acc += k
+    item_end = {st + k - 1 for st, k in zip(sorted(item_start), nonempty)}
     if unified:
         rings = {"kv": [Barrier(1) for _ in range(3)]}
         emp = {"kv": [Barrier(1) for _ in range(3)]}
@@ -503,13 +580,26 @@ def run_dq(items, rng, unified, mma_latency=3):
         rings = {"K": [Barrier(1) for _ in range(2)], "V": [Barrier(1)]}
         emp = {"K": [Barrier(1) for _ in range(2)], "V": [Barrier(1)]}
         slot = lambda kind, n: (kind, n, 2 if kind == "K" else 1)
-    sfull, dsfull, bdone, qready = Barrier(1), Barrier(1), Barrier(1), Barrier(1)
+    sfull, sfree, dsfull, bdone, qready = Barrier(1), Barrier(1), Barrier(1), Barrier(1), Barrier(1)
     loads = [(kind, n) for n in range(nblk) for kind in ("K", "V")]
+    # the issuer's op stream
+    ops = []
+    for st, k in zip(sorted(item_start), nonempty):
+        an = bn = 0
+        while bn < k:
+            if an < k and an <= bn + (1 if ds_smem else 0):
+                ops.append(("A", st + an))
+                an += 1
+            else:
+                ops.append(("B", st + bn))
+                bn += 1
     prod = {"i": 0}
-    iss = {"a": 0, "b": 0}
+    iss = {"c": 0}
     soft = {"n": 0, "it": 0, "step": "q"}
-    a_done, b_done, ds_written, epi_done = set(), set(), set(), set()
+    a_done, b_done, s_read, ds_written, epi_done = set(), set(), set(), set(), set()
+    ds_buf = {"block": None}  # which block's dS the shared buffer holds
     pending = []
+    pipe = {"last": 0}
     t = 0
 
     def producer():
@@ -531,33 +621,47 @@ def run_dq(items, rng, unified, mma_latency=3):
         prod["i"] += 1
         return True
 
-    def issuer():
-        a, b = iss["a"], iss["b"]
-        if b >= nblk:
-            return False
-        if a == b:  # A(a)
-            if a in item_start and not qready.poll(sorted(item_start).index(a), f"A{a} Q"):
-                return False
-            if a > 0 and not bdone.poll(a - 1, f"A{a} bdone"):
-                return False
-            rk, pk, sk = slot("K", a)
-            rv, pv, sv = slot("V", a)
-            if not rings[rk][pk % sk].poll(pk // sk, f"A{a} K") or not rings[rv][pv % sv].poll(pv // sv, f"A{a} V"):
-                return False
-            assert a == 0 or a - 1 in b_done, f"S/dP of block {a} overwrite dS of block {a - 1} under its MMA"
-            done = [lambda a=a: a_done.add(a), emp[rv][pv % sv].arrive, sfull.arrive]
+    def run_mma(done):
+        if ds_smem:  # in issue order
+            pipe["last"] = max(pipe["last"], t) + rng.randint(1, mma_latency)
+            pending.append((pipe["last"], done))
+        else:
             pending.append((t + rng.randint(1, mma_latency), done))
-            iss["a"] += 1
-            return True
-        if not dsfull.poll(b, f"B{b}"):
+
+    def issuer():
+        if iss["c"] >= len(ops):
             return False
-        assert b in ds_written
-        if b in item_start and sorted(item_start).index(b) > 0:
-            assert sorted(item_start).index(b) - 1 in epi_done, f"dQ restarted at block {b} before the epilogue"
-        rk, pk, sk = slot("K", b)
-        done = [lambda b=b: b_done.add(b), emp[rk][pk % sk].arrive, bdone.arrive]
-        pending.append((t + rng.randint(1, mma_latency), done))
-        iss["b"] += 1
+        kind, n = ops[iss["c"]]
+        if kind == "A":
+            if n in item_start and not qready.poll(sorted(item_start).index(n), f"A{n} Q"):
+                return False
+            if ds_smem:
+                if n > 0 and not sfree.poll(n - 1, f"A{n} sfree"):
+                    return False
+            elif n > 0 and not bdone.poll(n - 1, f"A{n} bdone"):
+                return False
+            rk, pk, sk = slot("K", n)
+            rv, pv, sv = slot("V", n)
+            if not rings[rk][pk % sk].poll(pk // sk, f"A{n} K") or not rings[rv][pv % sv].poll(pv // sv, f"A{n} V"):
+                return False
+            if ds_smem:
+                assert n == 0 or n - 1 in s_read, f"S/dP of block {n} overwrite block {n - 1} before the softmax read it"
+            else:
+                assert n == 0 or n - 1 in b_done, f"S/dP of block {n} overwrite dS of block {n - 1} under its MMA"
+            run_mma([lambda n=n: a_done.add(n), emp[rv][pv % sv].arrive, sfull.arrive])
+        else:
+            if not dsfull.poll(n, f"B{n}"):
+                return False
+            assert n in ds_written
+            if n in item_start and sorted(item_start).index(n) > 0:
+                assert sorted(item_start).index(n) - 1 in epi_done, f"dQ restarted at block {n} before the epilogue"
+            rk, pk, sk = slot("K", n)
+
+            def fin(n=n):
+                assert not ds_smem or ds_buf["block"] == n, f"B{n} read dS of block {ds_buf['block']}"
+                b_done.add(n)
+            run_mma([fin, emp[rk][pk % sk].arrive, bdone.arrive])
+        iss["c"] += 1
         return True
 
     def softmax():
@@ -572,17 +676,33 @@ def run_dq(items, rng, unified, mma_latency=3):
         if soft["step"] == "s":
             if not sfull.poll(n, f"softmax S{n}"):
                 return False
+            assert n in a_done
+            s_read.add(n)
+            if ds_smem:
+                sfree.arrive()
+                soft["step"] = "w"
+                return True
             ds_written.add(n)
             dsfull.arrive()
-            soft["n"] += 1
-            end = soft["n"] == sum(nonempty[:soft["it"] + 1])
-            soft["step"] = "epi" if end else "s"
-            return True
+            return advance(n)
+        if soft["step"] == "w":  # dS into shared memory once B(n-1) has read the previous dS
+            if ds_wait and n > 0 and not bdone.poll(n - 1, f"softmax dS{n}"):
+                return False
+            assert n == 0 or (n - 1) in b_done or (n - 1) not in ds_written, f"dS{n} written under B{n - 1}"
+            ds_buf["block"] = n
+            ds_written.add(n)
+            dsfull.arrive()
+            return advance(n)
         if not bdone.poll(n - 1, f"epilogue {soft['it']}"):
             return False
         epi_done.add(soft["it"])
         soft["it"] += 1
         soft["step"] = "q"
+        return True
+
+    def advance(n):
+        soft["n"] += 1
+        soft["step"] = "epi" if n in item_end else "s"
         return True
 
     agents = [producer, issuer, softmax]
@@ -591,7 +711,7 @@ def run_dq(items, rng, unified, mma_latency=3):
         t += 1
         due = [x for x in pending if x[0] <= t]
         pending[:] = [x for x in pending if x[0] > t]
-        for _, done in due:
+        for _, done in sorted(due, key=lambda x: x[0]):
             for f in done:
                 f()
         moved = bool(due)
@@ -599,13 +719,119 @@ def run_dq(items, rng, unified, mma_latency=3):
             if rng.random() < speed[i]:
                 moved |= agents[i]()
         if not moved and not pending and not any(ag() for ag in agents):
-            raise AssertionError(f"deadlock: A {iss['a']}, B {iss['b']}, softmax {soft} of {nblk}")
+            raise AssertionError(f"deadlock: op {iss['c']} of {len(ops)}, softmax {soft} of {nblk}")
     assert len(b_done) == nblk
 
 
-@pytest.mark.parametrize("unified", [False, True], ids=["kernel", "one_ring"])
+@pytest.mark.parametrize("layout", ["kernel", "tmem_ds", "tmem_ds_one_ring"])
 @pytest.mark.parametrize("seed", range(60))
-def test_dq_protocol_parity_and_progress(unified, seed):
+def test_dq_protocol_parity_and_progress(layout, seed):
     rng = random.Random(2000 + seed)
     items = [rng.choice([0, 1, 2, 3, 5, 8, 32]) for _ in range(rng.randint(1, 6))]
-    run_dq(items, rng, unified, mma_latency=rng.choice([1, 3, 10]))
+    run_dq(items, rng, unified=layout.endswith("one_ring"), mma_latency=rng.choice([1, 3, 10]),
+           ds_smem=layout == "kernel")
+
+
+def test_dq_protocol_flags_a_missing_ds_wait():
+    """Without the softmax's wait for B(n-1), dS(n) can land in shared memory while the previous
+    dQ MMA still reads it."""
+    with pytest.raises(AssertionError):
+        for seed in range(200):
+            run_dq([32, 5], random.Random(seed), unified=False, mma_latency=10, ds_wait=False)
+
+
+def test_dq_protocol_one_ring_deadlocks_with_a_ahead():
+    """A single K/V ring in load order cannot serve A(n+1) before B(n): V(n+1) would wait for the
+    release of K(n) by B(n), which the in-order issuer holds behind A(n+1)."""
+    with pytest.raises(AssertionError, match="deadlock"):
+        run_dq([8], random.Random(0), unified=True, mma_latency=3, ds_smem=True)
+
+
+def run_item_queue(n_items, qd, rng, empty_count=2, ahead=2):
+    """The forward kernel's per-slot item queue: the producer warp takes items from a global
+    counter and writes each into entry k % qd (after the entry's release, iqempty), `ahead`
+    items before it loads the item's blocks, then -1 at the end. The MMA issuer and the
+    softmax's first warp each read every entry in order (after iqfull) and release it; a
+    consumer can finish item k only once the producer has reached item k's loads. Asserts the
+    parity rule, that no entry is rewritten before both consumers read it, that both read the
+    producer's sequence exactly, and progress."""
+    ids = list(range(n_items)) + [-1]
+    full = [Barrier(1) for _ in range(qd)]
+    empty = [Barrier(empty_count) for _ in range(qd)]
+    slots = [None] * qd
+    readers = [set() for _ in range(qd)]
+    prod = {"k": 0}
+    cons = [{"k": 0, "got": [], "working": None} for _ in range(2)]
+
+    def loads_reached():  # items whose blocks the producer has issued
+        return max(0, prod["k"] - ahead)
+
+    def producer():
+        k = prod["k"]
+        if k >= len(ids):
+            return False
+        e = k % qd
+        if not empty[e].poll(k // qd - 1, f"producer entry {k}"):
+            return False
+        assert slots[e] is None or readers[e] == {0, 1}, f"entry {k} written before both consumers read {k - qd}"
+        slots[e] = ids[k]
+        readers[e] = set()
+        full[e].arrive()
+        prod["k"] += 1
+        return True
+
+    def consumer(c):
+        st = cons[c]
+        if st["working"] is not None:  # finish the current item once its loads were issued
+            if st["working"] < loads_reached() or prod["k"] == len(ids):
+                st["working"] = None
+                return True
+            return False
+        k = st["k"]
+        if st["got"] and st["got"][-1] == -1:
+            return False
+        e = k % qd
+        if not full[e].poll(k // qd, f"consumer {c} entry {k}"):
+            return False
+        v = slots[e]
+        readers[e].add(c)
+        empty[e].arrive()
+        st["got"].append(v)
+        st["k"] += 1
+        if v >= 0:
+            st["working"] = v
+        return True
+
+    agents = [producer, lambda: consumer(0), lambda: consumer(1)]
+    speed = [rng.uniform(0.05, 1.0) for _ in agents]
+    while not all(st["got"] and st["got"][-1] == -1 for st in cons):
+        moved = False
+        for i in rng.sample(range(len(agents)), len(agents)):
+            if rng.random() < speed[i]:
+                moved |= agents[i]()
+        if not moved and not any(a() for a in agents):
+            raise AssertionError(f"deadlock: producer at {prod['k']}, consumers at {[st['k'] for st in cons]}")
+    for st in cons:
+        assert st["got"] == ids
+
+
+@pytest.mark.parametrize("seed", range(60))
+def test_item_queue_parity_and_progress(seed):
+    rng = random.Random(seed)
+    run_item_queue(rng.randint(0, 40), qd=4, rng=rng)
+
+
+def test_item_queue_flags_a_single_release():
+    """iqempty completing on one consumer's release lets the producer rewrite an entry the other
+    consumer has not read."""
+    with pytest.raises(AssertionError):
+        for seed in range(200):
+            run_item_queue(30, qd=4, rng=random.Random(seed), empty_count=1)
+
+
+def test_item_queue_needs_as_many_entries_as_the_lookahead():
+    """With qd < ahead the producer waits for a release that needs its own loads: deadlock (the
+    kernel has qd = 4, ahead = 2)."""
+    run_item_queue(10, qd=2, rng=random.Random(0), ahead=2)
+    with pytest.raises(AssertionError, match="deadlock"):
+        run_item_queue(10, qd=1, rng=random.Random(0), ahead=2)
