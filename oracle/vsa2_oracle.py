@@ -46,6 +46,9 @@ __all__ = [
     "sparse_attn_fwd_padded",
     "coarse_attn_padded",
     "vsa2_forward_padded",
+    "sparse_attn_bwd_padded",
+    "coarse_attn_bwd_padded",
+    "gated_merge_bwd_padded",
 ]
 
 
@@ -466,3 +469,71 @@ def vsa2_forward_padded(q, k, v, gate_logits, topk, tile=(4, 4, 4), pool=(2, 2, 
     o_c = coarse_attn_padded(qc, kc, vc, vm, tile_tokens)
     o = gated_merge(o_f, o_c, gc[:, 0], tile_tokens)
     return permute_to_raster(o, grid_p, tile, pool)[:T, :H, :W], sel
+
+
+def sparse_attn_bwd_padded(q, k, v, do, kv_off, kv_idx, valid, tile_tokens: int = 64, o=None):
+    """Gradients (dQ, dK, dV) of `sparse_attn_fwd_padded` for one (b, h), given dO.
+
+    The output of a padding query row is the constant 0 (it is dropped with the padding), so its
+    dO reaches no input and its dQ is 0; padding keys take no part in any softmax, so the dK and
+    dV of padding tokens are 0. On the real rows of query tile i, with the real tokens of its
+    selected tiles as the keys, the textbook backward of `sparse_attn_bwd`:
+    dV += P^T dO, dS = P * (dO V^T - rowsum(dO * O)), dQ = dS K / sqrt(D), dK += dS^T Q / sqrt(D).
+    `o`, when given, is the stored forward output the rowsum is formed from."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    valid = np.asarray(valid, dtype=bool)
+    L, D = q.shape
+    N = L // tile_tokens
+    scale = 1.0 / np.sqrt(D)
+    dq, dk, dv = np.zeros((L, D)), np.zeros((L, D)), np.zeros((L, D))
+    for i in range(N):
+        sel = np.asarray(kv_idx[kv_off[i]:kv_off[i + 1]])
+        rows = np.arange(i * tile_tokens, (i + 1) * tile_tokens)
+        rows = rows[valid[rows]]
+        if sel.size == 0 or rows.size == 0:
+            continue
+        keys = np.concatenate([np.arange(j * tile_tokens, (j + 1) * tile_tokens) for j in sel])
+        keys = keys[valid[keys]]  # distinct tokens: the selected tiles are distinct
+        s = (q[rows] @ k[keys].T) * scale
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        oi = p @ v[keys] if o is None else np.asarray(o, dtype=np.float64)[rows]
+        delta = np.sum(do[rows] * oi, axis=1, keepdims=True)
+        dv[keys] += p.T @ do[rows]
+        ds = p * (do[rows] @ v[keys].T - delta)
+        dq[rows] = (ds @ k[keys]) * scale
+        dk[keys] += (ds.T @ q[rows]) * scale
+    return dq, dk, dv
+
+
+def coarse_attn_bwd_padded(q, k, v, d_oc, valid, tile_tokens: int = 64, o_c_hat=None):
+    """Gradients of `coarse_attn_padded` for one (b, h), given d_oc = dLoss/dO_c_hat (N, D):
+    the pooled-level backward of Eq. 2-3 as in `coarse_attn_bwd`, then the adjoint of the mean
+    over a tile's real tokens: each of the n_i real tokens of tile i gets dQc[i] / n_i (same for
+    K, V); padding tokens get 0."""
+    valid = np.asarray(valid, dtype=bool)
+    qc, cnt = _masked_mean_pool(q, valid, tile_tokens)
+    kc, _ = _masked_mean_pool(k, valid, tile_tokens)
+    vc, _ = _masked_mean_pool(v, valid, tile_tokens)
+    d_oc = np.asarray(d_oc, dtype=np.float64)
+    D = qc.shape[1]
+    s = (qc @ kc.T) / np.sqrt(D)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    o = p @ vc if o_c_hat is None else np.asarray(o_c_hat, dtype=np.float64)
+    ds = p * (d_oc @ vc.T - (d_oc * o).sum(axis=1, keepdims=True))
+    pooled = (ds @ kc / np.sqrt(D), ds.T @ qc / np.sqrt(D), p.T @ d_oc)
+    w = valid[:, None] / np.repeat(np.maximum(cnt, 1), tile_tokens)[:, None]
+    return tuple(np.repeat(x, tile_tokens, axis=0) * w for x in pooled)
+
+
+def gated_merge_bwd_padded(dout, o_c_hat, gate_logits, valid, tile_tokens: int = 64):
+    """Gradients of Eq. 4, 13-14 on a padded sequence: the outputs of padding rows are dropped,
+    so their dout reaches nothing: `gated_merge_bwd` with dout set to 0 on padding rows (dO_f,
+    d gate_logits 0 there; dO_c_hat sums the real tokens of each tile)."""
+    valid = np.asarray(valid, dtype=bool)
+    dout = np.where(valid[:, None], np.asarray(dout, dtype=np.float64), 0.0)
+    return gated_merge_bwd(dout, o_c_hat, gate_logits, tile_tokens)

@@ -678,6 +678,89 @@ def test_padded_full_budget_fine_branch_is_dense_attention_over_real_tokens():
     np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
 
 
+def _padded_case(grid=(5, 6, 7), d=8, seed=90):
+    """Padded cube-major q, k, v, dO (real rows smooth fields, padding rows large noise, which
+    must not matter) and the real-token mask."""
+    rng = np.random.default_rng(seed)
+    cm = [_padded_cube_major(_raster_inputs(grid, d, seed + i, smooth=False)) for i in range(4)]
+    vm = cm[0][1]
+    q, k, v, do = (np.where(vm[:, None], c[0], 30.0 * rng.standard_normal(c[0].shape)) for c in cm)
+    return q, k, v, do, vm
+
+
+def test_padded_backward_equals_the_unpadded_one_on_divisible_grids():
+    rng = np.random.default_rng(91)
+    L, D = 3 * 64, 8
+    q, k, v, do = (rng.standard_normal((L, D)) for _ in range(4))
+    valid = np.ones(L, bool)
+    off, idx = _csr(np.array([[1, 0, 1], [0, 0, 0], [1, 1, 0]], bool))
+    for got, want in zip(O.sparse_attn_bwd_padded(q, k, v, do, off, idx, valid), O.sparse_attn_bwd(q, k, v, do, off, idx)):
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-14)
+    d_oc = rng.standard_normal((3, D))
+    for got, want in zip(O.coarse_attn_bwd_padded(q, k, v, d_oc, valid), O.coarse_attn_bwd(q, k, v, d_oc)):
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-14)
+    oc, g = rng.standard_normal((3, D)), rng.standard_normal(L)
+    for got, want in zip(O.gated_merge_bwd_padded(do, oc, g, valid), O.gated_merge_bwd(do, oc, g)):
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-14)
+
+
+def _fd_check(loss, args, grads, rng, eps=1e-6):
+    """Central differences of `loss` along a random direction of every argument (padding rows
+    included) against the analytic directional derivative."""
+    for name in grads:
+        dirn = rng.standard_normal(args[name].shape)
+        plus = dict(args, **{name: args[name] + eps * dirn})
+        minus = dict(args, **{name: args[name] - eps * dirn})
+        fd = (loss(**plus) - loss(**minus)) / (2 * eps)
+        an = float(np.sum(grads[name] * dirn))
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+
+
+def test_padded_fine_backward_central_finite_differences():
+    """The loss sums dO * O over real rows only (padding rows are dropped); padding tokens of
+    q, k, v are perturbed too and must have zero gradient."""
+    q, k, v, do, vm = _padded_case()
+    N = q.shape[0] // 64
+    rng = np.random.default_rng(92)
+    mask = rng.random((N, N)) < 0.4
+    mask[1] = False  # an empty row
+    mask[2, 3] = True
+    off, idx = _csr(mask)
+
+    def loss(q, k, v):
+        o = O.sparse_attn_fwd_padded(q, k, v, off, idx, vm)
+        return float(np.sum((o * do)[vm]))
+
+    dq, dk, dv = O.sparse_attn_bwd_padded(q, k, v, do, off, idx, vm)
+    for g in (dq, dk, dv):
+        assert np.all(g[~vm] == 0)
+    assert np.all(dq[64:128] == 0)
+    _fd_check(loss, {"q": q, "k": k, "v": v}, {"q": dq, "k": dk, "v": dv}, rng)
+
+
+def test_padded_coarse_and_merge_backward_central_finite_differences():
+    q, k, v, do, vm = _padded_case(seed=93)
+    N, D = q.shape[0] // 64, q.shape[1]
+    rng = np.random.default_rng(94)
+    d_oc = rng.standard_normal((N, D))
+
+    def loss_c(q, k, v):
+        return float(np.sum(O.coarse_attn_padded(q, k, v, vm) * d_oc))
+
+    dq, dk, dv = O.coarse_attn_bwd_padded(q, k, v, d_oc, vm)
+    for g in (dq, dk, dv):
+        assert np.all(g[~vm] == 0)
+    _fd_check(loss_c, {"q": q, "k": k, "v": v}, {"q": dq, "k": dk, "v": dv}, rng)
+    o_f, oc, g = rng.standard_normal((q.shape[0], D)), rng.standard_normal((N, D)), rng.standard_normal(q.shape[0])
+
+    def loss_m(o_f, oc, g):
+        return float(np.sum((O.gated_merge(o_f, oc, g) * do)[vm]))
+
+    d_of, d_oc2, d_g = O.gated_merge_bwd_padded(do, oc, g, vm)
+    assert np.all(d_of[~vm] == 0) and np.all(d_g[~vm] == 0)
+    _fd_check(loss_m, {"o_f": o_f, "oc": oc, "g": g}, {"o_f": d_of, "oc": d_oc2, "g": d_g}, rng)
+
+
 def _router_padded_bruteforce(xq, xk, grid):
     """Eq. 5-7 with padding on the raster grid, explicit loops: pad to whole 4x4x4 tiles; each
     2x2x4 sub-cube's pooled vectors average its real tokens; sub-cubes without one are skipped
