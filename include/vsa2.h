@@ -22,9 +22,12 @@
  *    tile, the router sub-cubes of pool_t x pool_h x pool_w tokens in raster order; inside a
  *    sub-cube, tokens in raster order. So tile i is rows [i*Bt, (i+1)*Bt) and its G = Bt/R
  *    sub-cubes are consecutive groups of R rows.
- *  - Sizes: Bt = tile_t*tile_h*tile_w must be 64; R = pool_t*pool_h*pool_w must be 16
- *    (G = 4); the grid must be divisible by the tile and the tile by the pool; head_dim is
- *    64 or 128; N = L/64 tiles; 1 <= topk <= N. Other shapes return VSA2_ERR_UNSUPPORTED.
+ *  - Sizes: Bt = tile_t*tile_h*tile_w is 64 with R = pool_t*pool_h*pool_w = 16 (G = 4), or
+ *    128 with R = 8 (G = 16); the tile must be divisible by the pool; head_dim is 64 or 128;
+ *    N = L/Bt tiles; 1 <= topk <= N. A grid the 64-token tile does not divide is padded to
+ *    whole tiles (§2.2 "Kernel Implementation"): L then counts the padded grid, and padding
+ *    tokens are masked everywhere (see vsa2_permute_tokens, which fills them). The coarse
+ *    branch and the merge take 64-token tiles only. Other shapes return VSA2_ERR_UNSUPPORTED.
  *  - dtype covers Q, K, V, O and dO. Router scores, LSE and gradients are fp32; index lists
  *    are int32. Pointers must be 16-byte aligned.
  *  - Softmax scale is 1/sqrt(head_dim) everywhere (§2.1).
@@ -171,6 +174,8 @@ vsa2_status vsa2_sparse_attn_fwd_gated(const vsa2_problem* p, const void* q, con
  *   dq, dk, dv       : [batch, heads, L, D] fp32 (written; fully overwritten)
  * With P = exp(S - lse), dV = P^T dO, dS = P * (dO V^T - rowsum(dO * O)),
  * dQ = dS K / sqrt(D), dK = dS^T Q / sqrt(D), each restricted to the selected tile pairs.
+ * On a padded grid the padding keys take no part and the outputs of padding query rows are
+ * dropped, so dout there reaches nothing: dQ, dK, dV of padding tokens are 0.
  */
 vsa2_status vsa2_sparse_attn_bwd(const vsa2_problem* p, const void* q, const void* k, const void* v,
                                  const void* o, const float* lse, const void* dout, int32_t topk,
@@ -217,7 +222,8 @@ vsa2_status vsa2_gated_merge(const vsa2_problem* p, const void* o_f, const float
  *   dout        : [batch, heads, L, D] of dtype (read only), the gradient of o
  *   gate_logits : [batch, heads, L] fp32 (read only); oc : [batch, heads, N, D] of dtype
  *   d_logits    : [batch, heads, L] fp32 (written); d_oc : [batch, heads, N, D] fp32 (written)
- * Takes no workspace.
+ * On a padded grid the outputs of padding rows are dropped: d_logits is 0 there and d_oc sums
+ * the real tokens of each tile. Takes no workspace.
  */
 vsa2_status vsa2_gated_merge_bwd(const vsa2_problem* p, const void* dout, const float* gate_logits, const void* oc,
                                  float* d_logits, float* d_oc, void* stream);
@@ -226,7 +232,8 @@ vsa2_status vsa2_gated_merge_bwd(const vsa2_problem* p, const void* dout, const 
  * Gradients of the coarse branch, Eq. 1-3, ADDED to dq, dk, dv. With P_c and O_c_hat = oc:
  *   dS = P_c * (d_oc Vc^T - rowsum(d_oc * oc)),  dQc = dS Kc / sqrt(D),  dKc = dS^T Qc / sqrt(D),
  *   dVc = P_c^T d_oc, and MeanPool_B's adjoint spreads them: dq[t] += dQc[t/64] / 64 (same for
- *   dk, dv). Call it after vsa2_sparse_attn_bwd (which overwrites dq, dk, dv) to obtain the
+ *   dk, dv); on a padded grid the n real tokens of a tile get dQc / n and padding tokens
+ *   nothing. Call it after vsa2_sparse_attn_bwd (which overwrites dq, dk, dv) to obtain the
  *   gradients of the whole Eq. 14 output.
  *   q, k, v : [batch, heads, L, D] of dtype (read only)
  *   oc      : [batch, heads, N, D] of dtype and lse_c : [batch, heads, N] fp32, from

@@ -150,11 +150,68 @@ def test_padded_grid_whole_output_matches_oracle(case):
         _close(out[0, h], want_c, f"merge and crop h{h}")
 
 
-def test_padded_grid_backward_is_refused():
-    e = V.VSA2(1, 1, 128, (6, 7, 10), "bf16", 3)
-    z = torch.zeros(1, 1, e.L, 128, dtype=torch.bfloat16, device="cuda")
-    off = torch.zeros(1, 1, e.N + 1, dtype=torch.int32, device="cuda")
-    idx = torch.zeros(1, 1, e.N * 3, dtype=torch.int32, device="cuda")
-    with pytest.raises(V.Vsa2Error) as ex:
-        e.attn_bwd(z, z, z, z, torch.zeros(1, 1, e.L, device="cuda"), z, off, idx, off, idx)
-    assert ex.value.status == 2
+@pytest.mark.parametrize("case", list(CASES))
+def test_padded_grid_backward_matches_oracle(case):
+    """Gradients on a grid the tile does not divide, from the GPU's own forward (stored O in the
+    dtype and LSE), against the oracle's exact padded backward: padding keys take no part, the
+    outputs of padding rows are dropped (dout there is noise and must not matter), and the
+    gradients of padding tokens are exactly 0. The selection is the GPU's own (router, TopK)."""
+    grid, d, dtype, topk, heads = CASES[case]
+    x = {n: _raster(grid, d, heads, dtype, 20 + i) for i, n in enumerate("qkv")}
+    e = V.VSA2(1, heads, d, grid, dtype, topk)
+    xd = {n: e.to_cube_major(_dev(x[n], dtype)) for n in "qkv"}
+    rng = np.random.default_rng(7)
+    sels = [(_padded_oracle_inputs(x[n][0, h], grid, d) for n in "qkv") for h in range(heads)]
+    sels = [tuple(sel) for sel in sels]
+    vm = sels[0][0][1]
+    do_np = rng.standard_normal((1, heads, e.L, d)).astype(np.float32)
+    do_np[:, :, ~vm] = 50.0 * rng.standard_normal((1, heads, int((~vm).sum()), d))  # must not matter
+    do_np = S.round_to_dtype(do_np, dtype)
+    do = _dev(do_np, dtype)
+    o, lse, sel = e.forward(xd["q"], xd["k"], xd["v"], csc=True)
+    dq, dk, dv = e.attn_bwd(xd["q"], xd["k"], xd["v"], o, lse, do, *sel)
+    assert e.device_error() == 0
+    kv_off, kv_idx = sel[0].cpu().numpy(), sel[1].cpu().numpy()
+    got = [g.cpu().numpy() for g in (dq, dk, dv)]
+    for h in range(heads):
+        (qc, vmh), (kc, _), (vc, _) = sels[h]
+        want = O.sparse_attn_bwd_padded(qc, kc, vc, do_np[0, h], kv_off[0, h], kv_idx[0, h], vmh)
+        for name, g, w in zip(("dq", "dk", "dv"), got, want):
+            assert np.all(g[0, h][~vmh] == 0), f"{name} h{h}: padding tokens"
+            _close(g[0, h][vmh], w[vmh], f"{name} h{h}")
+
+
+@pytest.mark.parametrize("case", ["6x7x10_bf16", "6x7x10_fp32_d64", "480p_ragged_27x30x50"])
+def test_padded_grid_coarse_and_merge_backward_match_oracle(case):
+    """Gradients of the coarse branch (Eq. 1-3, means over real tokens) and of the gated merge on
+    a padded grid against the oracle's padded backward; d_oc comes from the merge backward, whose
+    dout is noise on padding rows."""
+    grid, d, dtype, topk, heads = CASES[case]
+    x = {n: _raster(grid, d, heads, dtype, 30 + i) for i, n in enumerate("qkv")}
+    e = V.VSA2(1, heads, d, grid, dtype, topk)
+    xd = {n: e.to_cube_major(_dev(x[n], dtype)) for n in "qkv"}
+    rng = np.random.default_rng(8)
+    vm = _padded_oracle_inputs(x["q"][0, 0], grid, d)[1]
+    do_np = rng.standard_normal((1, heads, e.L, d)).astype(np.float32)
+    do_np[:, :, ~vm] = 50.0 * rng.standard_normal((1, heads, int((~vm).sum()), d))
+    do_np = S.round_to_dtype(do_np, dtype)
+    logits = rng.standard_normal((1, heads, e.L)).astype(np.float32)
+    oc, lse_c = e.coarse_attn(xd["q"], xd["k"], xd["v"])
+    d_logits, d_oc = e.gated_merge_bwd(_dev(do_np, dtype), torch.from_numpy(logits).cuda(), oc)
+    grads = [torch.zeros(1, heads, e.L, d, dtype=torch.float32, device="cuda") for _ in range(3)]
+    e.coarse_attn_bwd(xd["q"], xd["k"], xd["v"], oc, lse_c, d_oc, *grads)
+    assert e.device_error() == 0
+    oc_np, d_logits, d_oc_np = oc.float().cpu().numpy(), d_logits.cpu().numpy(), d_oc.cpu().numpy()
+    got = [g.cpu().numpy() for g in grads]
+    for h in range(heads):
+        qc, _ = _padded_oracle_inputs(x["q"][0, h], grid, d)
+        kc, _ = _padded_oracle_inputs(x["k"][0, h], grid, d)
+        vc, _ = _padded_oracle_inputs(x["v"][0, h], grid, d)
+        _, w_doc, w_dlog = O.gated_merge_bwd_padded(do_np[0, h], oc_np[0, h], logits[0, h], vm)
+        _close(d_oc_np[0, h], w_doc, f"d_oc h{h}", tol_abs=2e-2 * max(1.0, np.abs(w_doc).max()))
+        assert np.all(d_logits[0, h][~vm] == 0)
+        _close(d_logits[0, h][vm], w_dlog[vm], f"d_logits h{h}")
+        want = O.coarse_attn_bwd_padded(qc, kc, vc, d_oc_np[0, h], vm, o_c_hat=oc_np[0, h])
+        for name, g, w in zip(("dq", "dk", "dv"), got, want):
+            assert np.all(g[0, h][~vm] == 0), f"coarse {name} h{h}: padding tokens"
+            _close(g[0, h][vm], w[vm], f"coarse {name} h{h}")

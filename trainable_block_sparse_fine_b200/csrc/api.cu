@@ -343,7 +343,6 @@ vsa2_status vsa2_sparse_attn_bwd(const vsa2_problem* p, const void* q, const voi
   Dims d;
   vsa2_status st = make_dims(p, &d);
   if (st != VSA2_OK) return st;
-  if (d.padded) return VSA2_ERR_UNSUPPORTED;  // the backward takes whole-tile grids only
   if (!q || !k || !v || !o || !lse || !dout || !kv_off || !kv_idx || !q_off || !q_idx || !dq || !dk || !dv)
     return VSA2_ERR_INVALID_ARG;
   if (topk < 1 || topk > d.N) return VSA2_ERR_UNSUPPORTED;
@@ -410,7 +409,6 @@ vsa2_status vsa2_coarse_attn_bwd(const vsa2_problem* p, const void* q, const voi
   vsa2_status st = make_dims(p, &d);
   if (st != VSA2_OK) return st;
   if (d.Bt != kTile) return VSA2_ERR_UNSUPPORTED;  // the coarse branch and the merge take 64-token tiles
-  if (d.padded) return VSA2_ERR_UNSUPPORTED;  // the backward takes whole-tile grids only
   if (!q || !k || !v || !oc || !lse_c || !d_oc || !dq || !dk || !dv) return VSA2_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(oc) || !aligned16(lse_c) || !aligned16(d_oc) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))

@@ -155,6 +155,14 @@ __device__ __forceinline__ void ds_half(const uint32_t (&sv)[32], const uint32_t
     pk[i2] = pair_pack_bf16(ds.x, ds.y, pair_perm(par_c));
   }
 }
+// Scores of the padding keys of a tile (bit u of `real` clear for padding token u; this thread
+// holds columns 2i + par_c) set to -inf.
+__device__ __forceinline__ void mask_keys(uint32_t (&sv)[32], uint64_t real, int par_c) {
+  if (real == ~0ull) return;
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if (!((real >> (2 * i + par_c)) & 1ull)) sv[i] = __float_as_uint(-INFINITY);
+}
 }  // namespace dqk
 
 __global__ void __launch_bounds__(BT, 1)
@@ -163,7 +171,7 @@ __global__ void __launch_bounds__(BT, 1)
                           const __nv_bfloat16* __restrict__ dog, const float* __restrict__ lse,
                           float* __restrict__ ndelta, float* __restrict__ nlse2, const int32_t* __restrict__ kv_off,
                           const int32_t* __restrict__ kv_idx, float* __restrict__ dq_out, int N, int L, int topk,
-                          int items, float c2, float scale, DevCtx ctx) {
+                          int items, float c2, float scale, const uint64_t* __restrict__ tmask, DevCtx ctx) {
   using namespace dqk;
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
   uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
@@ -336,7 +344,10 @@ __global__ void __launch_bounds__(BT, 1)
         tmem_st16x64b_x32(tl + TM_DO, v);
         dlt = part + __shfl_xor_sync(0xffffffffu, part, 2);
       }
-      const float nl2 = -lse[tok] * kLog2e;
+      // a row with lse = -inf (a padding query row of a padded grid) has P = 0: -lse * log2(e)
+      // is taken as -inf here and in the dK/dV kernel, which reads it from the workspace
+      const float lse_t = lse[tok];
+      const float nl2 = lse_t == -INFINITY ? -INFINITY : -lse_t * kLog2e;
       if (par_c == 0) {  // for the dK/dV kernel
         ndelta[tok] = -dlt;
         nlse2[tok] = nl2;
@@ -350,11 +361,19 @@ __global__ void __launch_bounds__(BT, 1)
         mbar_wait(&B.sfull[s], g & 1, abort, ctx);
         tc_fence_after();
         uint32_t pk[32];
+        // padding keys of a padded grid (tmask): S = -inf, so P = dS = 0
+        uint64_t km[2] = {~0ull, ~0ull};
+        if (tmask) {
+          const int32_t* ix = kv_idx + (size_t)bh * cap + rw.beg + 2 * n;
+          km[0] = __ldg(tmask + min(max(__ldg(ix), 0), N - 1));
+          if (!half) km[1] = __ldg(tmask + min(max(__ldg(ix + 1), 0), N - 1));
+        }
         {
           uint32_t sv[32], dp[32];
           tmem_ld16x64b_x32(tl + TM_S, sv);
           tmem_ld16x64b_x32(tl + TM_DP, dp);
           tmem_ld_wait();
+          mask_keys(sv, km[0], par_c);
           ds_half(sv, dp, c2, nl2, -dlt, par_c, pk);
         }
         if (!half) {
@@ -362,6 +381,7 @@ __global__ void __launch_bounds__(BT, 1)
           tmem_ld16x64b_x32(tl + TM_S + 64, sv);
           tmem_ld16x64b_x32(tl + TM_DP + 64, dp);
           tmem_ld_wait();
+          mask_keys(sv, km[1], par_c);
           ds_half(sv, dp, c2, nl2, -dlt, par_c, pk + 16);
         } else {
 #pragma unroll
@@ -429,7 +449,7 @@ __global__ void __launch_bounds__(dkv::KT, 1)
                             const float* __restrict__ nlse2, const float* __restrict__ ndelta,
                             const int32_t* __restrict__ q_off, const int32_t* __restrict__ q_idx,
                             float* __restrict__ dk_out, float* __restrict__ dv_out, int N, int L, int topk, int items,
-                            float c2, float scale, DevCtx ctx) {
+                            float c2, float scale, const uint64_t* __restrict__ tmask, DevCtx ctx) {
   using namespace dkv;
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
   uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
@@ -564,6 +584,8 @@ __global__ void __launch_bounds__(dkv::KT, 1)
       const Row rw = load_list(q_off, bh, kt, N, cap, ctx, warp == 0 && lane == 0);
       const size_t tok = (size_t)bh * L + (size_t)kt * 64 + j;
       float* gout = (kind ? dk_out : dv_out) + tok * 128 + 64 * c;
+      // a padding key of a padded grid takes no part: S = -inf, so its P, dS, dK and dV are 0
+      const bool key_real = !tmask || ((__ldg(tmask + kt) >> j) & 1ull);
       if (rw.len == 0) {
         float4* z = reinterpret_cast<float4*>(gout);
 #pragma unroll
@@ -599,7 +621,7 @@ __global__ void __launch_bounds__(dkv::KT, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const uint32_t recv = __shfl_xor_sync(0xffffffffu, kind ? da[i] : sa[16 + i], 1);
-          sv[i] = __uint_as_float(kind ? recv : sa[i]);
+          sv[i] = key_real ? __uint_as_float(kind ? recv : sa[i]) : -INFINITY;
           dv[i] = __uint_as_float(kind ? da[16 + i] : recv);
         }
         const float2* nl = reinterpret_cast<const float2*>(dsm + st * STAGE_B + 4 * TILE_B) + 16 * c + 8 * kind;
@@ -666,7 +688,8 @@ bool make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64
 
 vsa2_status attn_bwd_tc(const Dims& d, const void* q, const void* k, const void* v, const void* o, const float* lse,
                         const void* dout, const int32_t* kv_off, const int32_t* kv_idx, const int32_t* q_off,
-                        const int32_t* q_idx, float* dq, float* dk, float* dv, int topk, char* ws, cudaStream_t s) {
+                        const int32_t* q_idx, float* dq, float* dk, float* dv, int topk, char* ws,
+                        const uint64_t* tmask, cudaStream_t s) {
   CUtensorMap tk, tv, tq, tdo;
   const uint64_t rows = (uint64_t)d.BH * d.L;
   if (!make_tmap_2d_bf16(&tk, k, 128, rows, 64, 64) || !make_tmap_2d_bf16(&tv, v, 128, rows, 64, 64) ||
@@ -685,13 +708,13 @@ vsa2_status attn_bwd_tc(const Dims& d, const void* q, const void* k, const void*
   cudaFuncSetAttribute(attn_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dqk::SMEM_DYN);
   attn_bwd_dq_tc_kernel<<<grid, BT, dqk::SMEM_DYN, s>>>(
       tk, tv, (const __nv_bfloat16*)q, (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, lse, ndelta, nlse2, kv_off,
-      kv_idx, dq, d.N, (int)d.L, topk, items, c2, c1, ctx);
+      kv_idx, dq, d.N, (int)d.L, topk, items, c2, c1, tmask, ctx);
   if (check_launch("attn_bwd_dq_tc_kernel") != VSA2_OK) return VSA2_ERR_CUDA;
   cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dkv::SMEM_DYN);
   const int grid_kv = std::max(1, std::min(sms, items));
   attn_bwd_dkdv_tc_kernel<<<grid_kv, dkv::KT, dkv::SMEM_DYN, s>>>(tq, tdo, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
                                                           nlse2, ndelta, q_off, q_idx, dk, dv, d.N, (int)d.L, topk,
-                                                          items, c2, c1, ctx);
+                                                          items, c2, c1, tmask, ctx);
   return check_launch("attn_bwd_dkdv_tc_kernel");
 }
 

@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_simt_kernel(const T* __restri
                                                                const int32_t* __restrict__ kv_off,
                                                                const int32_t* __restrict__ kv_idx,
                                                                float* __restrict__ dq, int N, int64_t L, int topk,
-                                                               DevCtx ctx) {
+                                                               const uint64_t* __restrict__ tmask, DevCtx ctx) {
   extern __shared__ float sm[];
   float* qT = sm;             // [D][64]
   float* doT = qT + D * 64;   // [D][64]
@@ -174,6 +174,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_simt_kernel(const T* __restri
     const int j = idx[p];
     if (!idx_ok(j, N, ctx)) break;
     const size_t kt0 = (size_t)bh * L + (size_t)j * kTile;
+    const uint64_t km = tmask ? tmask[j] : ~0ull;  // padding keys of a padded grid take no part
     __syncthreads();
     for (int e = threadIdx.x; e < 64 * D; e += 128) {
       ks[e] = ldf(k + kt0 * D + e);
@@ -186,7 +187,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_simt_kernel(const T* __restri
         s += qT[d * 64 + t] * ks[u * D + d];
         dp += doT[d * 64 + t] * vs[u * D + d];
       }
-      const float pr = my_lse == -INFINITY ? 0.f : __expf(s * scale - my_lse);
+      // a row with lse = -inf (no selection, or a padding query row) has P = 0
+      const float pr = (my_lse == -INFINITY || !((km >> u) & 1ull)) ? 0.f : __expf(s * scale - my_lse);
       dsT[u * 64 + t] = pr * (dp - my_delta);
     }
     __syncthreads();
@@ -210,7 +212,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_simt_kernel(const T* __rest
                                                                  const int32_t* __restrict__ q_off,
                                                                  const int32_t* __restrict__ q_idx,
                                                                  float* __restrict__ dk, float* __restrict__ dv, int N,
-                                                                 int64_t L, int topk, DevCtx ctx) {
+                                                                 int64_t L, int topk, const uint64_t* __restrict__ tmask,
+                                                                 DevCtx ctx) {
   extern __shared__ float sm[];
   float* kT = sm;             // [D][64]
   float* vT = kT + D * 64;    // [D][64]
@@ -228,6 +231,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_simt_kernel(const T* __rest
     vT[c * 64 + r] = ldf(v + (kt0 + r) * D + c);
   }
   const float scale = rsqrtf((float)D);
+  const bool key_real = !tmask || ((tmask[j] >> u) & 1ull);  // a padding key gets dK = dV = 0
   float adk[D / 2], adv[D / 2];
 #pragma unroll
   for (int d = 0; d < D / 2; ++d) adk[d] = 0.f, adv[d] = 0.f;
@@ -254,7 +258,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_simt_kernel(const T* __rest
         s += qs[t * D + d] * kT[d * 64 + u];
         dp += dos[t * D + d] * vT[d * 64 + u];
       }
-      const float pr = lse_s[t] == -INFINITY ? 0.f : __expf(s * scale - lse_s[t]);
+      const float pr = (lse_s[t] == -INFINITY || !key_real) ? 0.f : __expf(s * scale - lse_s[t]);
       ps[t * 64 + u] = pr;
       dss[t * 64 + u] = pr * (dp - delta_s[t]);
     }
@@ -292,19 +296,19 @@ template <typename T, int D>
 vsa2_status bwd_simt(const Dims& d, const void* q, const void* k, const void* v, const void* o, const float* lse,
                      const void* dout, const int32_t* kv_off, const int32_t* kv_idx, const int32_t* q_off,
                      const int32_t* q_idx, float* dq, float* dk, float* dv, float* delta, int topk,
-                     const DevCtx& ctx, cudaStream_t s) {
+                     const uint64_t* tmask, const DevCtx& ctx, cudaStream_t s) {
   const int64_t rows = (int64_t)d.BH * d.L;
   attn_bwd_delta_kernel<T><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>((const T*)o, (const T*)dout, delta, rows, d.D);
   const size_t smem_dq = ((size_t)4 * 64 * D + 64 * 64) * sizeof(float);
   auto kq = attn_bwd_dq_simt_kernel<T, D>;
   cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dq);
   kq<<<dim3(d.N, d.BH), 128, smem_dq, s>>>((const T*)q, (const T*)k, (const T*)v, (const T*)dout, lse, delta,
-                                           kv_off, kv_idx, dq, d.N, d.L, topk, ctx);
+                                           kv_off, kv_idx, dq, d.N, d.L, topk, tmask, ctx);
   const size_t smem_kv = ((size_t)4 * 64 * D + 2 * 64 * 64) * sizeof(float);
   auto kk = attn_bwd_dkdv_simt_kernel<T, D>;
   cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_kv);
   kk<<<dim3(d.N, d.BH), 128, smem_kv, s>>>((const T*)q, (const T*)k, (const T*)v, (const T*)dout, lse, delta, q_off,
-                                           q_idx, dk, dv, d.N, d.L, topk, ctx);
+                                           q_idx, dk, dv, d.N, d.L, topk, tmask, ctx);
   return check_launch(__func__);
 }
 
@@ -329,20 +333,21 @@ vsa2_status attn_fwd_simt(const Dims& d, const void* q, const void* k, const voi
 
 vsa2_status attn_bwd_simt(const Dims& d, const void* q, const void* k, const void* v, const void* o, const float* lse,
                           const void* dout, const int32_t* kv_off, const int32_t* kv_idx, const int32_t* q_off,
-                          const int32_t* q_idx, float* dq, float* dk, float* dv, int topk, char* ws, cudaStream_t s) {
+                          const int32_t* q_idx, float* dq, float* dk, float* dv, int topk, char* ws,
+                          const uint64_t* tmask, cudaStream_t s) {
   DevCtx ctx{reinterpret_cast<int*>(ws), d.timeout_ns, d.flags};
   float* delta = reinterpret_cast<float*>(ws + ws_layout(d).delta);
   if (d.dtype == VSA2_BF16) {
     if (d.D == 128)
       return bwd_simt<__nv_bfloat16, 128>(d, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, delta,
-                                          topk, ctx, s);
+                                          topk, tmask, ctx, s);
     return bwd_simt<__nv_bfloat16, 64>(d, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, delta,
-                                       topk, ctx, s);
+                                       topk, tmask, ctx, s);
   }
   if (d.D == 128)
-    return bwd_simt<float, 128>(d, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, delta, topk, ctx,
-                                s);
-  return bwd_simt<float, 64>(d, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, delta, topk, ctx, s);
+    return bwd_simt<float, 128>(d, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, delta, topk, tmask,
+                                ctx, s);
+  return bwd_simt<float, 64>(d, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, delta, topk, tmask, ctx, s);
 }
 
 }  // namespace vsa2

@@ -146,16 +146,20 @@ __global__ void __launch_bounds__(256) gated_merge_kernel(const T* o_f, const fl
 
 // Gradients of Eq. 4, 13-14, warp per tile i of head bh (64 tokens t):
 //   d_logits[t] = (1 - G[t]^2) * (dout[t] . oc[i]),   d_oc[i] = sum_t G[t] * dout[t],   G = tanh(logits)
+// On a grid the tile does not divide (padded), the outputs of padding rows are dropped, so their
+// dout reaches nothing: d_logits is 0 there and d_oc sums the real tokens only.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) gated_merge_bwd_kernel(const T* __restrict__ dout,
                                                               const float* __restrict__ gate_logits,
                                                               const T* __restrict__ oc, float* __restrict__ d_logits,
-                                                              float* __restrict__ d_oc, int N, int64_t L) {
+                                                              float* __restrict__ d_oc, int N, int64_t L,
+                                                              GridGeom geom, bool padded) {
   constexpr int V = D / 32;
   const int bh = blockIdx.y;
   const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (i >= N) return;
+  const bool real0 = !padded || token_real(geom, i, lane), real1 = !padded || token_real(geom, i, 32 + lane);
   const size_t row0 = (size_t)bh * L + (size_t)i * kTile;
   float c[V], acc[V];
   load_vec<T, V>(oc + ((size_t)bh * N + i) * D + lane * V, c);
@@ -165,6 +169,7 @@ __global__ void __launch_bounds__(256) gated_merge_bwd_kernel(const T* __restric
   float r0 = 0.f, r1 = 0.f;
 #pragma unroll 4
   for (int t = 0; t < kTile; ++t) {
+    if (!__shfl_sync(0xffffffffu, t < 32 ? real0 : real1, t & 31)) continue;  // warp-uniform
     float x[V];
     load_vec<T, V>(dout + (row0 + t) * D + lane * V, x);
     const float G = __shfl_sync(0xffffffffu, t < 32 ? g0 : g1, t & 31);
@@ -213,19 +218,28 @@ __global__ void __launch_bounds__(256) coarse_pad_bwd_kernel(const T* __restrict
 }
 
 // MeanPool_B's adjoint, accumulated: dx[t] += dxc[tile(t)] / 64 for Q, K and V (fp32), four
-// channels per thread and iteration.
+// channels per thread and iteration. With tmask (a padded grid) the mean ran over the tile's n
+// real tokens: each of them gets dxc / n and the padding tokens nothing.
 __global__ void __launch_bounds__(256) coarse_pool_bwd_kernel(const float* __restrict__ dqc,
                                                               const float* __restrict__ dkc,
                                                               const float* __restrict__ dvc, float* __restrict__ dq,
                                                               float* __restrict__ dk, float* __restrict__ dv,
-                                                              int64_t rows, int64_t L, int Lc, int D) {
+                                                              int64_t rows, int64_t L, int Lc, int D,
+                                                              const uint64_t* __restrict__ tmask) {
   const int cpr = D / 4;
   const int64_t total = rows * cpr;
   for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < total; c += (int64_t)gridDim.x * blockDim.x) {
     const int64_t row = c / cpr;
     const int col = (int)(c - row * cpr) * 4;
     const int64_t bh = row / L;
-    const int64_t src = ((size_t)bh * Lc + (row - bh * L) / kTile) * D + col;
+    const int64_t tile = (row - bh * L) / kTile;
+    const int64_t src = ((size_t)bh * Lc + tile) * D + col;
+    float w = 1.f / kTile;
+    if (tmask) {
+      const uint64_t real = __ldg(tmask + tile);
+      if (!((real >> ((row - bh * L) % kTile)) & 1ull)) continue;
+      w = 1.f / __popcll(real);  // every tile holds a real token
+    }
     const float* in[3] = {dqc, dkc, dvc};
     float* out[3] = {dq, dk, dv};
 #pragma unroll
@@ -233,10 +247,10 @@ __global__ void __launch_bounds__(256) coarse_pool_bwd_kernel(const float* __res
       const float4 a = __ldg(reinterpret_cast<const float4*>(in[x] + src));
       float4* o = reinterpret_cast<float4*>(out[x] + row * D + col);
       float4 b = *o;
-      b.x = fmaf(a.x, 1.f / kTile, b.x);
-      b.y = fmaf(a.y, 1.f / kTile, b.y);
-      b.z = fmaf(a.z, 1.f / kTile, b.z);
-      b.w = fmaf(a.w, 1.f / kTile, b.w);
+      b.x = fmaf(a.x, w, b.x);
+      b.y = fmaf(a.y, w, b.y);
+      b.z = fmaf(a.z, w, b.z);
+      b.w = fmaf(a.w, w, b.w);
       *o = b;
     }
   }
@@ -309,18 +323,19 @@ vsa2_status launch_coarse_attn(const Dims& d, const void* q, const void* k, cons
 vsa2_status launch_gated_merge_bwd(const Dims& d, const void* dout, const float* gate_logits, const void* oc,
                                    float* d_logits, float* d_oc, cudaStream_t s) {
   const dim3 grid((d.N + 7) / 8, d.BH);
+  const GridGeom geom = grid_geom(d);
   if (d.dtype == VSA2_BF16 && d.D == 128)
     gated_merge_bwd_kernel<__nv_bfloat16, 128><<<grid, 256, 0, s>>>((const __nv_bfloat16*)dout, gate_logits,
-                                                                    (const __nv_bfloat16*)oc, d_logits, d_oc, d.N, d.L);
+                                                                    (const __nv_bfloat16*)oc, d_logits, d_oc, d.N, d.L, geom, d.padded);
   else if (d.dtype == VSA2_BF16)
     gated_merge_bwd_kernel<__nv_bfloat16, 64><<<grid, 256, 0, s>>>((const __nv_bfloat16*)dout, gate_logits,
-                                                                   (const __nv_bfloat16*)oc, d_logits, d_oc, d.N, d.L);
+                                                                   (const __nv_bfloat16*)oc, d_logits, d_oc, d.N, d.L, geom, d.padded);
   else if (d.D == 128)
     gated_merge_bwd_kernel<float, 128><<<grid, 256, 0, s>>>((const float*)dout, gate_logits, (const float*)oc,
-                                                            d_logits, d_oc, d.N, d.L);
+                                                            d_logits, d_oc, d.N, d.L, geom, d.padded);
   else
     gated_merge_bwd_kernel<float, 64><<<grid, 256, 0, s>>>((const float*)dout, gate_logits, (const float*)oc,
-                                                           d_logits, d_oc, d.N, d.L);
+                                                           d_logits, d_oc, d.N, d.L, geom, d.padded);
   return check_launch("gated_merge_bwd_kernel");
 }
 
@@ -344,21 +359,28 @@ vsa2_status launch_coarse_attn_bwd(const Dims& d, const void* q, const void* k, 
   dc.L = Lc;
   dc.N = Nc;
   dc.Lr = Lc / kPool;
+  dc.padded = false;  // the pooled sequence is dense (its zero rows past N add nothing)
   // the backward of the pooled sequence keeps its Delta and LSE where ws_layout(dc) puts them;
   // every region of dc is at most the size of d's, so they end before the coarse regions
   if (ws_layout(dc).nlse2 + align256((size_t)dc.BH * Lc * 4) > w.qc) return VSA2_ERR_UNSUPPORTED;
-  // pooled operands (Eq. 1) again, the padded O_c_hat, LSE and dO_c_hat, and the dense CSR / CSC
+  // pooled operands (Eq. 1) again (over the real tokens of a padded grid), the padded O_c_hat,
+  // LSE and dO_c_hat, and the dense CSR / CSC
+  uint64_t* tmask = nullptr;
+  if (d.padded) {
+    tmask = reinterpret_cast<uint64_t*>(ws + w.tmask);
+    if (launch_tile_masks(d, tmask, s) != VSA2_OK) return VSA2_ERR_CUDA;
+  }
   if (d.dtype == VSA2_BF16 && d.D == 128) {
-    launch_pool<__nv_bfloat16, 128>(d, q, k, v, ws, w, nullptr, s);  // whole-tile grids only
+    launch_pool<__nv_bfloat16, 128>(d, q, k, v, ws, w, tmask, s);
     launch_pad_bwd<__nv_bfloat16, 128>(d, oc, lse_c, d_oc, ws, w, s);
   } else if (d.dtype == VSA2_BF16) {
-    launch_pool<__nv_bfloat16, 64>(d, q, k, v, ws, w, nullptr, s);  // whole-tile grids only
+    launch_pool<__nv_bfloat16, 64>(d, q, k, v, ws, w, tmask, s);
     launch_pad_bwd<__nv_bfloat16, 64>(d, oc, lse_c, d_oc, ws, w, s);
   } else if (d.D == 128) {
-    launch_pool<float, 128>(d, q, k, v, ws, w, nullptr, s);  // whole-tile grids only
+    launch_pool<float, 128>(d, q, k, v, ws, w, tmask, s);
     launch_pad_bwd<float, 128>(d, oc, lse_c, d_oc, ws, w, s);
   } else {
-    launch_pool<float, 64>(d, q, k, v, ws, w, nullptr, s);  // whole-tile grids only
+    launch_pool<float, 64>(d, q, k, v, ws, w, tmask, s);
     launch_pad_bwd<float, 64>(d, oc, lse_c, d_oc, ws, w, s);
   }
   int32_t* c_off = reinterpret_cast<int32_t*>(ws + w.c_off);
@@ -377,7 +399,7 @@ vsa2_status launch_coarse_attn_bwd(const Dims& d, const void* q, const void* k, 
   // MeanPool_B's adjoint, added to the caller's gradients
   const int64_t rows = (int64_t)d.BH * d.L;
   coarse_pool_bwd_kernel<<<grid_for(rows * (d.D / 4), 256), 256, 0, s>>>(dqc, dkc, dvc, dq, dk, dv, rows, d.L, Lc,
-                                                                         d.D);
+                                                                         d.D, tmask);
   return check_launch("coarse_pool_bwd_kernel");
 }
 

@@ -40,9 +40,14 @@ vsa2_status launch_attn_bwd(const Dims& d, const void* q, const void* k, const v
                             const float* lse, const void* dout, int topk, const int32_t* kv_off,
                             const int32_t* kv_idx, const int32_t* q_off, const int32_t* q_idx, float* dq, float* dk,
                             float* dv, char* ws, cudaStream_t s) {
+  uint64_t* tmask = nullptr;
+  if (d.padded) {  // padding keys are masked and padding query rows (lse = -inf) add nothing
+    tmask = reinterpret_cast<uint64_t*>(ws + ws_layout(d).tmask);
+    if (launch_tile_masks(d, tmask, s) != VSA2_OK) return VSA2_ERR_CUDA;
+  }
   if (d.dtype == VSA2_BF16 && d.D == 128)
-    return attn_bwd_tc(d, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, topk, ws, s);
-  return attn_bwd_simt(d, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, topk, ws, s);
+    return attn_bwd_tc(d, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, topk, ws, tmask, s);
+  return attn_bwd_simt(d, q, k, v, o, lse, dout, kv_off, kv_idx, q_off, q_idx, dq, dk, dv, topk, ws, tmask, s);
 }
 
 }  // namespace vsa2

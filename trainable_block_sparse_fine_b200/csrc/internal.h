@@ -53,6 +53,35 @@ inline bool coarse_pool_in_router(const Dims& d) {
          d.R == kPool;
 }
 
+// Geometry of a grid the tile does not divide: which cube-major tokens of a tile are real.
+struct GridGeom {
+  int gt, gh, gw;  // real grid
+  int tt, th, tw;  // tile
+  int rt, rh, rw;  // sub-cube
+  int nth, ntw;    // tiles along h and w of the padded grid
+};
+inline GridGeom grid_geom(const Dims& d) {
+  GridGeom g;
+  g.gt = d.gt, g.gh = d.gh, g.gw = d.gw;
+  g.tt = d.tt, g.th = d.th, g.tw = d.tw;
+  g.rt = d.rt, g.rh = d.rh, g.rw = d.rw;
+  g.nth = (d.gh + d.th - 1) / d.th;
+  g.ntw = (d.gw + d.tw - 1) / d.tw;
+  return g;
+}
+// Cube-major token u of tile i (sub-cube u / R in raster order over the tile's sub-cubes, token
+// u % R in raster order inside it) lies inside the real grid.
+__host__ __device__ inline bool token_real(const GridGeom& g, int i, int u) {
+  const int per_t = g.nth * g.ntw;
+  const int it = i / per_t, ih = (i % per_t) / g.ntw, iw = i % g.ntw;
+  const int sh_n = g.th / g.rh, sw_n = g.tw / g.rw, R = g.rt * g.rh * g.rw;
+  const int sub = u / R, r = u % R;
+  const int st = sub / (sh_n * sw_n), s2 = sub % (sh_n * sw_n), sh = s2 / sw_n, sw = s2 % sw_n;
+  const int dt = r / (g.rh * g.rw), r2 = r % (g.rh * g.rw), dh = r2 / g.rw, dw = r2 % g.rw;
+  const int t = it * g.tt + st * g.rt + dt, h = ih * g.th + sh * g.rh + dh, w = iw * g.tw + sw * g.rw + dw;
+  return t < g.gt && h < g.gh && w < g.gw;
+}
+
 // Real-token mask of every tile of a padded grid (bit u = cube-major token u of the tile is a
 // token of the real grid); the same for every (b, h). Enqueued on `s`, written to `mask` [N].
 vsa2_status launch_tile_masks(const Dims& d, uint64_t* mask, cudaStream_t s);
@@ -123,10 +152,12 @@ vsa2_status attn_fwd_simt(const Dims& d, const void* q, const void* k, const voi
                           const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
                           int64_t kv_valid, const uint64_t* tmask, cudaStream_t s, const float* gate = nullptr,
                           const void* oc = nullptr, void* of = nullptr);
+// backward on CUDA cores; tmask (a padded grid's real-token masks, or null): padding keys take
+// no part and get dK = dV = 0, padding query rows (lse = -inf) add nothing
 vsa2_status attn_bwd_simt(const Dims& d, const void* q, const void* k, const void* v, const void* o,
                           const float* lse, const void* dout, const int32_t* kv_off, const int32_t* kv_idx,
                           const int32_t* q_off, const int32_t* q_idx, float* dq, float* dk, float* dv, int topk,
-                          char* ws, cudaStream_t s);
+                          char* ws, const uint64_t* tmask, cudaStream_t s);
 // tensor-core forward (bf16, head_dim 128); the masked variant treats keys at or beyond
 // kv_valid tokens of each head as padding (each listed tile must hold a valid key)
 vsa2_status attn_fwd_tc(const Dims& d, const void* q, const void* k, const void* v, int topk,
@@ -150,10 +181,12 @@ vsa2_status launch_gated_merge_bwd(const Dims& d, const void* dout, const float*
 vsa2_status launch_coarse_attn_bwd(const Dims& d, const void* q, const void* k, const void* v, const void* oc,
                                    const float* lse_c, const float* d_oc, float* dq, float* dk, float* dv, char* ws,
                                    cudaStream_t s);
-// tensor-core backward (bf16, head_dim 128): dQ kernel (also writes Delta), then dK/dV kernel
+// tensor-core backward (bf16, head_dim 128): dQ kernel (also writes Delta), then dK/dV kernel;
+// tmask as for attn_bwd_simt
 vsa2_status attn_bwd_tc(const Dims& d, const void* q, const void* k, const void* v, const void* o, const float* lse,
                         const void* dout, const int32_t* kv_off, const int32_t* kv_idx, const int32_t* q_off,
-                        const int32_t* q_idx, float* dq, float* dk, float* dv, int topk, char* ws, cudaStream_t s);
+                        const int32_t* q_idx, float* dq, float* dk, float* dv, int topk, char* ws,
+                        const uint64_t* tmask, cudaStream_t s);
 // Token permutation raster <-> cube-major (to_cube != 0: raster -> cube-major)
 vsa2_status launch_permute(const Dims& d, const vsa2_problem* p, const void* src, void* dst, int to_cube,
                            cudaStream_t s);
