@@ -161,8 +161,7 @@ def test_padded_grid_backward_matches_oracle(case):
     e = V.VSA2(1, heads, d, grid, dtype, topk)
     xd = {n: e.to_cube_major(_dev(x[n], dtype)) for n in "qkv"}
     rng = np.random.default_rng(7)
-    sels = [(_padded_oracle_inputs(x[n][0, h], grid, d) for n in "qkv") for h in range(heads)]
-    sels = [tuple(sel) for sel in sels]
+    sels = [tuple(_padded_oracle_inputs(x[n][0, h], grid, d) for n in "qkv") for h in range(heads)]
     vm = sels[0][0][1]
     do_np = rng.standard_normal((1, heads, e.L, d)).astype(np.float32)
     do_np[:, :, ~vm] = 50.0 * rng.standard_normal((1, heads, int((~vm).sum()), d))  # must not matter

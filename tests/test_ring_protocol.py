@@ -56,13 +56,16 @@ def ops_of(tiles, lead=1):
     return out
 
 
-def run(tiles, rst, producers, rng, mma_latency=3, lead=1):
+def run(tiles, rst, producers, rng, mma_latency=3, lead=1, parity=False, ordered=False):
+    """`producers` = 2 splits each block between two producers (one per d-half, the full barrier
+    expecting both), or with `parity` gives ring position c to producer c % 2 alone; with
+    `ordered` a producer loads position c only after position c - 1 was loaded (by the other)."""
     ops = ops_of(tiles, lead)
-    full = [Barrier(producers) for _ in range(rst)]
+    full = [Barrier(1 if parity else producers) for _ in range(rst)]
     empty = [Barrier(1) for _ in range(rst)]
     sfull, sfree = [Barrier(1), Barrier(1)], [Barrier(1), Barrier(1)]
     pfull, pvdone = Barrier(1), Barrier(1)
-    prod = [0] * producers            # next ring position per producer
+    prod = [p if parity else 0 for p in range(producers)]  # next ring position per producer
     mma = {"c": 0, "s": 0, "o": 0}    # next op; S and O ops issued
     soft = {"blk": 0, "step": 0}      # next block; 0: wait S, 1: wait previous P.V, then write P
     op_done = set()                   # ring positions whose MMA has completed
@@ -76,12 +79,14 @@ def run(tiles, rst, producers, rng, mma_latency=3, lead=1):
         c = prod[p]
         if c >= len(ops):
             return False
+        if ordered and c > 0 and prod[1 - p] < c:  # position c - 1 not loaded yet
+            return False
         st = c % rst
         if not empty[st].poll(c // rst - 1, f"producer {p} at {c}"):
             return False
         assert c < rst or c - rst in op_done, f"ring position {c} refilled before its MMA finished"
         full[st].arrive()
-        prod[p] += 1
+        prod[p] += producers if parity else 1
         return True
 
     def issuer():
@@ -143,7 +148,7 @@ def run(tiles, rst, producers, rng, mma_latency=3, lead=1):
         assert moved or pending or t < 10_000_000, "deadlock"
         if not moved and not pending and not any(a() for a in agents):
             raise AssertionError(f"deadlock at op {mma['c']} of {len(ops)}, softmax block {soft['blk']}")
-    assert pvdone.phases == sum(tiles) and all(p == len(ops) for p in prod)
+    assert pvdone.phases == sum(tiles) and all(p >= len(ops) for p in prod)
 
 
 def run_aliased(tiles, rst, rng, mma_latency=3, rescale_p=0.2, lead=1, halves=1, xch_bufs=2, sfree_count=None):
@@ -403,6 +408,25 @@ def test_ring_protocol_parity_and_progress(lead, producers, seed):
     rng = random.Random(seed)
     tiles = [rng.choice([1, 1, 2, 3, 4, 5, 7, 32]) for _ in range(rng.randint(1, 6))]
     run(tiles, rst=3, producers=producers, rng=rng, mma_latency=rng.choice([1, 3, 10]), lead=lead)
+
+
+@pytest.mark.parametrize("seed", range(60))
+def test_ring_protocol_parity_split_producers_in_order(seed):
+    """Two producers per slot on ring-position parity with the kernel's three stages: each loads
+    position c only after the other has loaded c - 1, so no stage is waited on two phases ahead."""
+    rng = random.Random(5000 + seed)
+    tiles = [rng.choice([1, 1, 2, 3, 4, 5, 7, 32]) for _ in range(rng.randint(1, 6))]
+    run(tiles, rst=3, producers=2, rng=rng, mma_latency=rng.choice([1, 3, 10]), parity=True, ordered=True)
+
+
+def test_ring_protocol_parity_split_without_order_is_flagged():
+    """Without that order a producer can wait on a stage two phases ahead (three stages shared by
+    two producers): the parity rule flags it."""
+    with pytest.raises(AssertionError):
+        for seed in range(5000, 5100):
+            rng = random.Random(seed)
+            tiles = [rng.choice([1, 1, 2, 3, 4, 5, 7, 32]) for _ in range(rng.randint(1, 6))]
+            run(tiles, rst=3, producers=2, rng=rng, mma_latency=rng.choice([1, 3, 10]), parity=True)
 
 
 def test_op_order_matches_the_kernel_stream():
