@@ -153,9 +153,10 @@ def test_padded_grid_whole_output_matches_oracle(case):
 @pytest.mark.parametrize("case", list(CASES))
 def test_padded_grid_backward_matches_oracle(case):
     """Gradients on a grid the tile does not divide, from the GPU's own forward (stored O in the
-    dtype and LSE), against the oracle's exact padded backward: padding keys take no part, the
-    outputs of padding rows are dropped (dout there is noise and must not matter), and the
-    gradients of padding tokens are exactly 0. The selection is the GPU's own (router, TopK)."""
+    dtype and LSE), against the oracle's padded backward given the same stored O (the backward
+    forms rowsum(dO * O) from the O it receives): padding keys take no part, the outputs of
+    padding rows are dropped (dout there is noise and must not matter), and the gradients of
+    padding tokens are exactly 0. The selection is the GPU's own (router, TopK)."""
     grid, d, dtype, topk, heads = CASES[case]
     x = {n: _raster(grid, d, heads, dtype, 20 + i) for i, n in enumerate("qkv")}
     e = V.VSA2(1, heads, d, grid, dtype, topk)
@@ -172,9 +173,10 @@ def test_padded_grid_backward_matches_oracle(case):
     assert e.device_error() == 0
     kv_off, kv_idx = sel[0].cpu().numpy(), sel[1].cpu().numpy()
     got = [g.cpu().numpy() for g in (dq, dk, dv)]
+    o_np = o.float().cpu().numpy()
     for h in range(heads):
         (qc, vmh), (kc, _), (vc, _) = sels[h]
-        want = O.sparse_attn_bwd_padded(qc, kc, vc, do_np[0, h], kv_off[0, h], kv_idx[0, h], vmh)
+        want = O.sparse_attn_bwd_padded(qc, kc, vc, do_np[0, h], kv_off[0, h], kv_idx[0, h], vmh, o=o_np[0, h])
         for name, g, w in zip(("dq", "dk", "dv"), got, want):
             assert np.all(g[0, h][~vmh] == 0), f"{name} h{h}: padding tokens"
             _close(g[0, h][vmh], w[vmh], f"{name} h{h}")
@@ -184,12 +186,22 @@ def test_padded_grid_backward_matches_oracle(case):
 def test_padded_grid_coarse_and_merge_backward_match_oracle(case):
     """Gradients of the coarse branch (Eq. 1-3, means over real tokens) and of the gated merge on
     a padded grid against the oracle's padded backward; d_oc comes from the merge backward, whose
-    dout is noise on padding rows."""
+    dout is noise on padding rows. Inputs are tile-constant (as in the whole-tile coarse backward
+    tests), so the GPU's pooled operands, rounded to the dtype, equal the oracle's exactly."""
     grid, d, dtype, topk, heads = CASES[case]
-    x = {n: _raster(grid, d, heads, dtype, 30 + i) for i, n in enumerate("qkv")}
+    # tile-constant inputs with dtype-exact tile values: every real token of a tile holds the
+    # tile's vector, so both sides pool to the same (representable) operands
+    T, H, W = grid
+    rng = np.random.default_rng(8)
+    tgrid = tuple(-(-g // 4) for g in grid)
+    t, hh, w = np.meshgrid(np.arange(T) // 4, np.arange(H) // 4, np.arange(W) // 4, indexing="ij")
+    tile_of = ((t * tgrid[1] + hh) * tgrid[2] + w).reshape(-1)
+    x = {}
+    for n in "qkv":
+        vals = S.round_to_dtype(rng.standard_normal((heads, int(np.prod(tgrid)), d)).astype(np.float32), dtype)
+        x[n] = vals[:, tile_of][None].astype(np.float32)
     e = V.VSA2(1, heads, d, grid, dtype, topk)
     xd = {n: e.to_cube_major(_dev(x[n], dtype)) for n in "qkv"}
-    rng = np.random.default_rng(8)
     vm = _padded_oracle_inputs(x["q"][0, 0], grid, d)[1]
     do_np = rng.standard_normal((1, heads, e.L, d)).astype(np.float32)
     do_np[:, :, ~vm] = 50.0 * rng.standard_normal((1, heads, int((~vm).sum()), d))
@@ -210,7 +222,9 @@ def test_padded_grid_coarse_and_merge_backward_match_oracle(case):
         _close(d_oc_np[0, h], w_doc, f"d_oc h{h}", tol_abs=2e-2 * max(1.0, np.abs(w_doc).max()))
         assert np.all(d_logits[0, h][~vm] == 0)
         _close(d_logits[0, h][vm], w_dlog[vm], f"d_logits h{h}")
-        want = O.coarse_attn_bwd_padded(qc, kc, vc, d_oc_np[0, h], vm, o_c_hat=oc_np[0, h])
+        # the coarse backward takes d_oc rounded to the dtype (its tensor-core operand)
+        d_oc_in = S.round_to_dtype(d_oc_np[0, h], dtype)
+        want = O.coarse_attn_bwd_padded(qc, kc, vc, d_oc_in, vm, o_c_hat=oc_np[0, h])
         for name, g, w in zip(("dq", "dk", "dv"), got, want):
             assert np.all(g[0, h][~vm] == 0), f"coarse {name} h{h}: padding tokens"
             _close(g[0, h][vm], w[vm], f"coarse {name} h{h}")

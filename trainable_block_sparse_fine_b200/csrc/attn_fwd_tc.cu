@@ -50,7 +50,9 @@ constexpr int IDXCAP = 256;                                // KV indices of a ro
 constexpr uint32_t OFF_IDX = OFF_RING + 2 * RST * BLK_B;   // [slot][2 rows][IDXCAP] int32
 constexpr uint32_t OFF_BAR = OFF_IDX + 2 * 2 * IDXCAP * 4;
 constexpr uint32_t OFF_FLAG = OFF_BAR + 512;
-constexpr uint32_t SMEM_USED = OFF_FLAG + 64;
+constexpr int QD = 4;                                       // item queue entries per slot
+constexpr uint32_t OFF_IQ = OFF_FLAG + 64;                  // [slot][QD] items, then [slot][2] hand-over
+constexpr uint32_t SMEM_USED = OFF_IQ + (2 * QD + 2 * 2) * 4;
 constexpr uint32_t SMEM_DYN = SMEM_USED + 1024;
 static_assert(SMEM_DYN <= 232448, "shared memory budget");
 
@@ -70,6 +72,7 @@ struct Bars {
   uint64_t sfull[2][2], sfree[2][2];                                       // [slot][buffer]
   uint64_t pfull[2][2], pvdone[2][2], qready[2];  // pfull, pvdone: [slot][block parity]
   uint64_t done[2];
+  uint64_t iqfull[2][QD], iqempty[2][QD];  // [slot][entry]: the slot's item queue
 };
 static_assert(sizeof(Bars) <= 512, "barrier area");
 
@@ -88,19 +91,20 @@ __device__ __forceinline__ Row load_row(const int32_t* kv_off, int bh, int i, in
   return Row{b, e - b};
 }
 
-// Per-slot op stream of a CTA: items (b*h, query tile) in head-major order, slot s of CTA c takes
-// items r*2G + 2c + s. For a tile of n blocks the ops are S0, S1, O0, S2, O1, ..., O(n-1).
-// The MMA issuer and both producers walk the same merged stream (slot 0 op, slot 1 op, ...).
+// Per-slot op stream: items (b*h, query tile) come from a global counter in head-major order, one
+// at a time, to whichever slot's producer asks next (the per-sequence TopK gives rows of unequal
+// length, so a fixed assignment leaves some slots finishing late). The producer passes each item
+// to its slot's MMA issuer and softmax warps through a queue in shared memory. For a tile of n
+// blocks the ops are S0, S1, O0, S2, O1, ..., O(n-1); the producer and the MMA issuer walk them in
+// the same order.
 struct SlotSeq {
-  int item, stride, items;
+  int kq;  // queue entries taken
   int bh, qt, nblk, len, beg;
   int s_next, o_next;
   int tile;  // non-empty tiles started so far
   bool active;
-  __device__ void init(int first, int step, int total) {
-    item = first - step;
-    stride = step;
-    items = total;
+  __device__ void init() {
+    kq = 0;
     nblk = 0;
     s_next = o_next = 0;
     tile = 0;
@@ -108,9 +112,11 @@ struct SlotSeq {
   }
 };
 
-// 0 = none, 1 = S op, 2 = O op; *blk = block index within the tile
+// 0 = none, 1 = S op, 2 = O op; *blk = block index within the tile. The next item comes from the
+// slot's queue (entry kq % QD); -1 ends the stream.
 __device__ __forceinline__ int next_op(SlotSeq& q, int* blk, const int32_t* kv_off, int N, int cap,
-                                       const DevCtx& ctx) {
+                                       const DevCtx& ctx, const volatile int* iq, uint64_t* iqfull,
+                                       uint64_t* iqempty, volatile int* abort) {
   while (q.active) {
     if (q.s_next < q.nblk && q.s_next <= q.o_next + kLead) {
       *blk = q.s_next++;
@@ -120,13 +126,17 @@ __device__ __forceinline__ int next_op(SlotSeq& q, int* blk, const int32_t* kv_o
       *blk = q.o_next++;
       return 2;
     }
-    q.item += q.stride;
-    if (q.item >= q.items) {
+    const int e = q.kq % QD;
+    int item = -1;
+    if (mbar_wait(&iqfull[e], (q.kq / QD) & 1, abort, ctx)) item = iq[e];
+    mbar_arrive(&iqempty[e]);
+    ++q.kq;
+    if (item < 0) {
       q.active = false;
       return 0;
     }
-    q.bh = q.item / N;
-    q.qt = q.item - q.bh * N;
+    q.bh = item / N;
+    q.qt = item - q.bh * N;
     const Row r = load_row(kv_off, q.bh, q.qt, N, cap, ctx, false);
     q.len = r.len;
     q.beg = r.beg;
@@ -152,7 +162,7 @@ __global__ void __launch_bounds__(FT, 1)
                        const __nv_bfloat16* __restrict__ qg, const int32_t* __restrict__ kv_off,
                        const int32_t* __restrict__ kv_idx, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
                        int N, int L, int topk, int items, float c2, int kv_valid,
-                       const uint64_t* __restrict__ tmask, GateArgs gate, DevCtx ctx) {
+                       const uint64_t* __restrict__ tmask, GateArgs gate, int* __restrict__ work_ctr, DevCtx ctx) {
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
   uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   Bars& B = *reinterpret_cast<Bars*>(dsm + OFF_BAR);
@@ -161,7 +171,6 @@ __global__ void __launch_bounds__(FT, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cap = N * topk;
-  const int step = 2 * gridDim.x;
 
   if (threadIdx.x == 0) {
     flag_sh[0] = 0;
@@ -176,6 +185,8 @@ __global__ void __launch_bounds__(FT, 1)
     }
     mbar_init(&B.done[0], 1);
     mbar_init(&B.done[1], 1);
+    for (int s = 0; s < 2; ++s)
+      for (int i = 0; i < QD; ++i) mbar_init(&B.iqfull[s][i], 1), mbar_init(&B.iqempty[s][i], 2);
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -199,7 +210,7 @@ __global__ void __launch_bounds__(FT, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
     }
-    auto row_of = [&](int it) { return it < items ? load_row(kv_off, it / N, it % N, N, cap, ctx, false) : Row{0, 0}; };
+    auto row_of = [&](int it) { return it >= 0 ? load_row(kv_off, it / N, it % N, N, cap, ctx, false) : Row{0, 0}; };
     auto copy_row = [&](int it, const Row& r, int b) {  // whole warp
       const int32_t* src = kv_idx + (size_t)(it / N) * cap + r.beg;
       const int n = min(r.len, IDXCAP);
@@ -208,17 +219,49 @@ __global__ void __launch_bounds__(FT, 1)
                      : "memory");
       asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    int item = 2 * blockIdx.x + s;
-    Row cur = row_of(item);
-    if (item < items) copy_row(item, cur, 0);
-    Row nxt = row_of(item + step);
-    int c = 0;  // ring position: blocks requested so far
+    // Items come from a global counter (dynamic balance across slots). Lane 0 takes one when the
+    // warp needs it, two items ahead of the loads, and passes it to the slot's MMA issuer and
+    // softmax warps through the queue, in load order; -1 marks the end.
+    volatile int* iq = reinterpret_cast<volatile int*>(dsm + OFF_IQ) + s * QD;
+    int kq = 0;  // queue entries written
+    bool ended = false;
     bool ok = true;
-    for (int b = 0; ok && item < items; item += step, b ^= 1) {
+    auto next_id = [&]() -> int {  // whole warp
+      if (ended) return -1;
+      int id = -1, good = 1;
+      if (lane == 0) {
+        id = atomicAdd(work_ctr, 1);
+        if (id >= items) id = -1;
+        const int e = kq % QD;
+        if (mbar_wait(&B.iqempty[s][e], ((kq / QD) & 1) ^ 1, abort, ctx)) {
+          iq[e] = id;
+          mbar_arrive(&B.iqfull[s][e]);
+        } else {
+          good = 0;
+        }
+      }
+      id = __shfl_sync(0xffffffffu, id, 0);
+      good = __shfl_sync(0xffffffffu, good, 0);
+      ++kq;
+      if (!good) ok = false;
+      if (id < 0 || !good) {
+        ended = true;
+        id = -1;
+      }
+      return id;
+    };
+    int item = next_id();
+    Row cur = row_of(item);
+    if (item >= 0) copy_row(item, cur, 0);
+    int nxt_id = next_id();
+    Row nxt = row_of(nxt_id);
+    int c = 0;  // ring position: blocks requested so far
+    for (int b = 0; ok && item >= 0; b ^= 1) {
       asm volatile("cp.async.wait_all;" ::: "memory");  // this item's indices (copied an item ago)
       __syncwarp();
-      if (item + step < items && nxt.len > 0) copy_row(item + step, nxt, b ^ 1);
-      const Row nn = row_of(item + 2 * step);  // used when the next item starts
+      if (nxt_id >= 0 && nxt.len > 0) copy_row(nxt_id, nxt, b ^ 1);
+      const int nn_id = next_id();
+      const Row nn = row_of(nn_id);  // used when the next item starts
       if (lane == 0) {
         const int bh = item / N;
         const int32_t* gidx = kv_idx + (size_t)bh * cap + cur.beg;
@@ -260,8 +303,10 @@ __global__ void __launch_bounds__(FT, 1)
           ++c;
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 && ok;
+      item = nxt_id;
       cur = nxt;
+      nxt_id = nn_id;
       nxt = nn;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");  // no copy outlives the CTA
@@ -277,13 +322,14 @@ __global__ void __launch_bounds__(FT, 1)
       constexpr uint32_t id_o = idesc_bf16_f32(64, 128, false, true);
       const uint32_t lanes = (uint32_t)(16 * s) << 16;
       SlotSeq sq;
-      sq.init(2 * blockIdx.x + s, step, items);
+      sq.init();
+      const volatile int* iq = reinterpret_cast<const volatile int*>(dsm + OFF_IQ) + s * QD;
       int kc = 0, vc = 0;  // S and O blocks issued
       int c = 0;           // ring position
       bool ok = true;
       while (ok && sq.active) {
         int blk;
-        const int op = next_op(sq, &blk, kv_off, N, cap, ctx);
+        const int op = next_op(sq, &blk, kv_off, N, cap, ctx, iq, B.iqfull[s], B.iqempty[s], abort);
         if (op == 1) {
           if (blk == 0 && !(ok = mbar_wait(&B.qready[s], (sq.tile - 1) & 1, abort, ctx))) break;
           const int st = c % RST;
@@ -328,7 +374,22 @@ __global__ void __launch_bounds__(FT, 1)
     const int row = 16 * w + r16;                  // row within the query tile
     const uint32_t tl = tmem + ((uint32_t)(32 * w + 16 * s) << 16);
     int g = 0;  // blocks processed by this slot
-    for (int item = 2 * blockIdx.x + s; item < items; item += step) {
+    const volatile int* iq = reinterpret_cast<const volatile int*>(dsm + OFF_IQ) + s * QD;
+    volatile int* cur_item = reinterpret_cast<volatile int*>(dsm + OFF_IQ) + 2 * QD + 2 * s;  // [kq parity]
+    for (int kq = 0;; ++kq) {
+      // the slot's first warp takes the next queue entry and hands it to the slot's 4 warps; the
+      // hand-over slot alternates with the entry's parity, so it is rewritten only after every
+      // warp passed the next barrier
+      if (w == 0 && lane == 0) {
+        const int e = kq % QD;
+        int id = -1;
+        if (mbar_wait(&B.iqfull[s][e], (kq / QD) & 1, abort, ctx)) id = iq[e];
+        mbar_arrive(&B.iqempty[s][e]);
+        cur_item[kq & 1] = id;
+      }
+      named_bar_sync(bar_id, 128);
+      const int item = cur_item[kq & 1];
+      if (item < 0) break;
       const int bh = item / N, qt = item - bh * N;
       const Row rw = load_row(kv_off, bh, qt, N, cap, ctx, w == 0 && lane == 0);
       const int nblk = (rw.len + 1) >> 1;
@@ -545,8 +606,11 @@ vsa2_status launch_fwd_tc(const Dims& d, const void* q, const void* k, const voi
   const float c2 = 1.4426950408889634f / sqrtf(128.f);
   auto kern = attn_fwd_tc_kernel<kMode, kGate>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
+  // the item counter the CTAs' producers draw from, in the workspace header
+  int* ctr = reinterpret_cast<int*>(ws + kWsWorkCounter);
+  if (cudaMemsetAsync(ctr, 0, sizeof(int), s) != cudaSuccess) return cuda_fail("attn_fwd_tc: item counter reset");
   kern<<<grid, FT, SMEM_DYN, s>>>(tk, tv, (const __nv_bfloat16*)q, kv_off, kv_idx, (__nv_bfloat16*)o, lse, d.N,
-                                  (int)d.L, topk, items, c2, kv_valid, tmask, gate, ctx);
+                                  (int)d.L, topk, items, c2, kv_valid, tmask, gate, ctr, ctx);
   return check_launch("attn_fwd_tc");
 }
 }  // namespace

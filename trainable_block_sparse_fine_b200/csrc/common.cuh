@@ -11,8 +11,10 @@
 
 namespace vsa2 {
 
-// Workspace header: the device error word lives at offset 0; regions start at 256.
+// Workspace header: the device error word lives at offset 0, the attention forward's item
+// counter (reset before each launch) at offset 128; regions start at 256.
 constexpr size_t kWsHeader = 256;
+constexpr size_t kWsWorkCounter = 128;
 
 struct DevCtx {
   int* err;             // device error word (first failure wins)
