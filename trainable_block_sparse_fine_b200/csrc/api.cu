@@ -93,6 +93,8 @@ WsLayout ws_layout(const Dims& d) {
   w.dkc = take((size_t)d.BH * lc * d.D * 4);
   w.dvc = take((size_t)d.BH * lc * d.D * 4);
   w.tmask = take((size_t)d.N * 8);
+  w.cand = take((size_t)d.BH * kCandCap * 4);
+  w.cand_cnt = take((size_t)d.BH * 4);
   w.total = off;
   return w;
 }

@@ -90,6 +90,7 @@ vsa2_status launch_tile_masks(const Dims& d, uint64_t* mask, cudaStream_t s);
 vsa2_status make_dims(const vsa2_problem* p, Dims* d);
 
 // Workspace regions (byte offsets from the workspace base, all 256-byte aligned).
+constexpr int kCandCap = 8192;  // TopK candidate list per (b, h)
 struct WsLayout {
   size_t qr, kr;         // pooled Q, K: [BH, Lr, D] in the input dtype
   size_t lse_r;          // router per-pooled-row LSE (log2 domain), [BH, Lr] fp32
@@ -110,6 +111,8 @@ struct WsLayout {
   size_t doc;            // coarse backward: padded gradient of O_c_hat, [BH, 64 * Nc_tiles, D] dtype
   size_t dqc, dkc, dvc;  // coarse backward: gradients of the pooled rows, [BH, 64 * Nc_tiles, D] fp32
   size_t tmask;          // padded grids: real-token mask per tile, [N] u64
+  size_t cand, cand_cnt; // TopK: entries sharing the 22-bit threshold prefix, [BH, kCandCap] u32
+                         // (row << 10 | low 10 bits), and their count per (b, h)
   size_t total;
 };
 WsLayout ws_layout(const Dims& d);

@@ -2,11 +2,15 @@
 // Sparse Rebasing", §2.2 Eq. 8-9): per (b, h) keep the N*K largest of the N*N tile scores.
 //
 // Exact radix select on the fp32 bit patterns (scores are >= 0, so unsigned order equals
-// float order): three histogram passes over 11/11/10-bit digits find the threshold T and how
-// many entries equal to T still fit the budget. Ties at T go to the lowest flat index i*N+j:
-// a per-row scan assigns the tie quota row by row, then each row is compacted in ascending j
+// float order): three histograms over 11/11/10-bit digits find the threshold T and how many
+// entries equal to T still fit the budget. Ties at T go to the lowest flat index i*N+j: a
+// per-row scan assigns the tie quota row by row, then each row is compacted in ascending j
 // (CSR). The CSC used by the backward pass is built from a per-column bitmap, so both lists
-// are deterministic.
+// are deterministic. The third histogram is formed in the same pass over the scores as the
+// per-row counts: that pass counts, per row, the entries whose top 22 bits exceed the prefix
+// found so far, and lists the few entries that share it (row and low 10 bits) for a small fix-up
+// once T is known; when a head has more of them than the list holds (heavy ties), a full
+// recount against T takes over.
 #include <mutex>
 
 #include "common.cuh"
@@ -131,12 +135,15 @@ __device__ __forceinline__ bool rows_vec4(const float* scores, int N) {
   return (N & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0;
 }
 
+// With cand_cnt, the recount runs only for heads whose candidate list overflowed.
 __global__ void __launch_bounds__(256) topk_row_count_kernel(const float* __restrict__ scores, int N,
                                                              const uint32_t* __restrict__ state,
-                                                             int32_t* __restrict__ row_gt, int32_t* __restrict__ row_eq) {
+                                                             int32_t* __restrict__ row_gt, int32_t* __restrict__ row_eq,
+                                                             const uint32_t* __restrict__ cand_cnt) {
   const int bh = blockIdx.y;
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (row >= N) return;
+  if (cand_cnt && cand_cnt[bh] <= (uint32_t)kCandCap) return;
   const uint32_t T = state[bh * 8 + ST_THRESH];
   const float* s = scores + ((size_t)bh * N + row) * N;
   int gt = 0, eq = 0;
@@ -164,6 +171,72 @@ __global__ void __launch_bounds__(256) topk_row_count_kernel(const float* __rest
   if (lane == 0) {
     row_gt[(size_t)bh * N + row] = gt;
     row_eq[(size_t)bh * N + row] = eq;
+  }
+}
+
+// Warp per row, after the second digit: entries whose top 22 bits exceed the prefix P22 (row_gt),
+// and the entries equal to it: their low 10 bits go to the third histogram and, with the row, to
+// the head's candidate list (the count goes on past kCandCap to flag an overflow).
+__global__ void __launch_bounds__(256) topk_row_count22_kernel(const float* __restrict__ scores, int N,
+                                                               const uint32_t* __restrict__ state,
+                                                               int32_t* __restrict__ row_gt, int32_t* __restrict__ row_eq,
+                                                               uint32_t* __restrict__ hist, uint32_t* __restrict__ cand,
+                                                               uint32_t* __restrict__ cand_cnt) {
+  const int bh = blockIdx.y;
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= N) return;
+  const uint32_t P = state[bh * 8 + ST_PREFIX];
+  const float* s = scores + ((size_t)bh * N + row) * N;
+  uint32_t* h2 = hist + ((size_t)bh * 3 + 2) * 2048;
+  int gt = 0;
+  auto cand_add = [&](uint32_t key) {
+    atomicAdd(&h2[key & 1023u], 1u);
+    const uint32_t at = atomicAdd(&cand_cnt[bh], 1u);
+    if (at < (uint32_t)kCandCap) cand[(size_t)bh * kCandCap + at] = ((uint32_t)row << 10) | (key & 1023u);
+  };
+  if (rows_vec4(scores, N)) {
+    const float4* s4 = reinterpret_cast<const float4*>(s);
+#pragma unroll 4
+    for (int q = lane; q < (N >> 2); q += 32) {
+      const float4 v = __ldg(s4 + q);
+      const uint32_t k[4] = {score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w)};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t p = k[e] >> 10;
+        gt += p > P;
+        if (p == P) cand_add(k[e]);
+      }
+    }
+  } else {
+    for (int j = lane; j < N; j += 32) {
+      const uint32_t key = score_key(__ldg(s + j));
+      gt += (key >> 10) > P;
+      if ((key >> 10) == P) cand_add(key);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) gt += __shfl_xor_sync(0xffffffffu, gt, o);
+  if (lane == 0) {
+    row_gt[(size_t)bh * N + row] = gt;
+    row_eq[(size_t)bh * N + row] = 0;
+  }
+}
+
+// Per (b, h), once T is known: the listed candidates above T join their row's count, those equal
+// to T its ties. Heads whose list overflowed are recounted in full instead.
+__global__ void __launch_bounds__(256) topk_cand_fix_kernel(const uint32_t* __restrict__ state,
+                                                            const uint32_t* __restrict__ cand,
+                                                            const uint32_t* __restrict__ cand_cnt, int N,
+                                                            int32_t* __restrict__ row_gt, int32_t* __restrict__ row_eq) {
+  const int bh = blockIdx.x;
+  const uint32_t n = cand_cnt[bh];
+  if (n > (uint32_t)kCandCap) return;
+  const uint32_t d = state[bh * 8 + ST_THRESH] & 1023u;
+  for (uint32_t c = threadIdx.x; c < n; c += blockDim.x) {
+    const uint32_t e = cand[(size_t)bh * kCandCap + c];
+    const uint32_t row = e >> 10, low = e & 1023u;
+    if (low > d) atomicAdd(&row_gt[(size_t)bh * N + row], 1);
+    else if (low == d) atomicAdd(&row_eq[(size_t)bh * N + row], 1);
   }
 }
 
@@ -474,7 +547,10 @@ vsa2_status launch_topk(const Dims& d, const float* scores, int topk, int32_t* k
   const int64_t nn = (int64_t)d.N * d.N;
   const uint32_t budget = (uint32_t)d.N * (uint32_t)topk;
 
+  uint32_t* cand = reinterpret_cast<uint32_t*>(ws + w.cand);
+  uint32_t* cand_cnt = reinterpret_cast<uint32_t*>(ws + w.cand_cnt);
   if (cudaMemsetAsync(hist, 0, (size_t)d.BH * 3 * 2048 * 4, s) != cudaSuccess) return VSA2_ERR_CUDA;
+  if (cudaMemsetAsync(cand_cnt, 0, (size_t)d.BH * 4, s) != cudaSuccess) return VSA2_ERR_CUDA;
   if (csc) {
     if (cudaMemsetAsync(col_cnt, 0, (size_t)d.BH * d.N * 4, s) != cudaSuccess) return VSA2_ERR_CUDA;
     if (cudaMemsetAsync(col_bits, 0, (size_t)d.BH * d.N * w.words * 4, s) != cudaSuccess) return VSA2_ERR_CUDA;
@@ -488,10 +564,11 @@ vsa2_status launch_topk(const Dims& d, const float* scores, int topk, int32_t* k
   topk_select_digit_kernel<0><<<d.BH, 1024, 0, s>>>(hist, state, budget);
   topk_hist_kernel<1><<<hgrid, 512, 0, s>>>(scores, nn, state, hist);
   topk_select_digit_kernel<1><<<d.BH, 1024, 0, s>>>(hist, state, budget);
-  topk_hist_kernel<2><<<hgrid, 512, 0, s>>>(scores, nn, state, hist);
-  topk_select_digit_kernel<2><<<d.BH, 1024, 0, s>>>(hist, state, budget);
   dim3 rgrid((d.N + 7) / 8, d.BH);
-  topk_row_count_kernel<<<rgrid, 256, 0, s>>>(scores, d.N, state, row_gt, row_eq);
+  topk_row_count22_kernel<<<rgrid, 256, 0, s>>>(scores, d.N, state, row_gt, row_eq, hist, cand, cand_cnt);
+  topk_select_digit_kernel<2><<<d.BH, 1024, 0, s>>>(hist, state, budget);
+  topk_cand_fix_kernel<<<d.BH, 256, 0, s>>>(state, cand, cand_cnt, d.N, row_gt, row_eq);
+  topk_row_count_kernel<<<rgrid, 256, 0, s>>>(scores, d.N, state, row_gt, row_eq, cand_cnt);  // overflow only
   topk_offsets_kernel<<<d.BH, 1024, 0, s>>>(d.N, state, row_gt, row_eq, row_take, kv_off);
   topk_emit_kernel<<<rgrid, 256, 0, s>>>(scores, d.N, topk, state, row_take, kv_off, kv_idx,
                                          csc ? col_cnt : nullptr, col_bits, w.words, ctx);
@@ -598,7 +675,7 @@ vsa2_status launch_topk_noalloc(const Dims& d, const float* scores, int topk, in
   topk_hist_kernel<2><<<hgrid, 512, 0, s>>>(scores, nn, state, hist);
   topk_select_digit_kernel<2><<<d.BH, 1024, 0, s>>>(hist, state, budget);
   dim3 rgrid((d.N + 7) / 8, d.BH);
-  topk_row_count_kernel<<<rgrid, 256, 0, s>>>(scores, d.N, state, row_gt, row_eq);
+  topk_row_count_kernel<<<rgrid, 256, 0, s>>>(scores, d.N, state, row_gt, row_eq, nullptr);
   topk_offsets_kernel<<<d.BH, 1024, 0, s>>>(d.N, state, row_gt, row_eq, row_take, kv_off);
   topk_emit_kernel<<<rgrid, 256, 0, s>>>(scores, d.N, topk, state, row_take, kv_off, kv_idx, nullptr, nullptr, 0, ctx);
   return check_launch(__func__);
