@@ -43,31 +43,68 @@ __device__ __forceinline__ Row load_list(const int32_t* off, int bh, int i, int 
   return Row{b, e - b};
 }
 
-// Op stream of one slot: items r*2G + 2c + s of CTA c, each item's list cut into blocks of
-// `per_blk` tiles, ops A(0), B(0), A(1), B(1), ... (A = the MMAs that need fresh operands,
-// B = the MMAs that consume the softmax output). The producers and the MMA issuer walk the
-// merged stream slot 0, slot 1, slot 0, ... identically.
+// Items (b*h, tile) come from a global counter, one at a time, to the role that draws them (the
+// rows of the per-sequence TopK have unequal lengths, so a fixed assignment leaves some CTAs
+// finishing late); it passes each item to the other roles that walk the same stream through a
+// queue of QD entries in shared memory (full / empty mbarriers, -1 ends the stream).
+constexpr int QD = 4;
+struct ItemQueue {
+  volatile int* slot;  // [QD]
+  uint64_t* full;      // [QD], one arrival (the drawing role)
+  uint64_t* empty;     // [QD], one arrival per taking role
+};
+// The next item of a stream, as entry k of its queue: drawn from *ctr and written there (draw),
+// or taken from there. -1 at the end of the items, or when a wait expired.
+__device__ __forceinline__ int next_item(const ItemQueue& q, int& k, bool draw, int* ctr, int items,
+                                         volatile int* abort, const DevCtx& ctx) {
+  const int e = k % QD;
+  int item = -1;
+  if (draw) {
+    item = atomicAdd(ctr, 1);
+    if (item >= items) item = -1;
+    if (mbar_wait(&q.empty[e], ((k / QD) & 1) ^ 1, abort, ctx)) {
+      q.slot[e] = item;
+      mbar_arrive(&q.full[e]);
+    } else {
+      item = -1;
+    }
+  } else {
+    if (mbar_wait(&q.full[e], (k / QD) & 1, abort, ctx)) item = q.slot[e];
+    mbar_arrive(&q.empty[e]);
+  }
+  ++k;
+  return item;
+}
+
+// Op stream of one item sequence, each item's list cut into blocks of `per_blk` tiles, ops
+// A(0), B(0), A(1), B(1), ... (A = the MMAs that need fresh operands, B = the MMAs that consume
+// the softmax output). The producers and the MMA issuers walk it identically.
 struct Seq {
-  int item, stride, items;
+  int kq;  // queue entries passed
   int bh, it, nblk, len, beg;
   int a_next, b_next;
   int tile;  // non-empty items started so far
   bool active;
-  __device__ void init(int first, int step, int total) {
-    item = first - step;
-    stride = step;
-    items = total;
+  __device__ void init() {
+    kq = 0;
     nblk = len = beg = bh = it = 0;
     a_next = b_next = 0;
     tile = 0;
     active = true;
   }
 };
+struct SeqSrc {  // where a walker's next item comes from
+  ItemQueue q;
+  bool draw;
+  int* ctr;
+  int items;
+  volatile int* abort;
+};
 
 // 0 = none (slot finished), 1 = A op, 2 = B op; *blk = block index within the item. With
 // ahead = 1 the A op of block n+1 comes before the B op of block n.
 __device__ __forceinline__ int next_op(Seq& q, int* blk, const int32_t* off, int N, int cap, int per_blk,
-                                       const DevCtx& ctx, int ahead = 0) {
+                                       const DevCtx& ctx, const SeqSrc& src, int ahead = 0) {
   while (q.active) {
     if (q.a_next < q.nblk && q.a_next <= q.b_next + ahead) {
       *blk = q.a_next++;
@@ -77,13 +114,13 @@ __device__ __forceinline__ int next_op(Seq& q, int* blk, const int32_t* off, int
       *blk = q.b_next++;
       return 2;
     }
-    q.item += q.stride;
-    if (q.item >= q.items) {
+    const int item = next_item(src.q, q.kq, src.draw, src.ctr, src.items, src.abort, ctx);
+    if (item < 0) {
       q.active = false;
       return 0;
     }
-    q.bh = q.item / N;
-    q.it = q.item - q.bh * N;
+    q.bh = item / N;
+    q.it = item - q.bh * N;
     const Row r = load_list(off, q.bh, q.it, N, cap, ctx, false);
     q.len = r.len;
     q.beg = r.beg;
@@ -130,7 +167,8 @@ constexpr uint32_t OFF_K = 0;                          // [slot][KST] blocks
 constexpr uint32_t OFF_V = OFF_K + 2 * KST * BLK_B;    // [slot][VST] blocks
 constexpr uint32_t OFF_BAR = OFF_V + 2 * VST * BLK_B;
 constexpr uint32_t OFF_FLAG = OFF_BAR + 512;
-constexpr uint32_t SMEM_DYN = OFF_FLAG + 64 + 1024;
+constexpr uint32_t OFF_IQ = OFF_FLAG + 64;  // [slot][QD] item queue, then [slot][2] softmax hand-over
+constexpr uint32_t SMEM_DYN = OFF_IQ + 64 + 1024;
 static_assert(SMEM_DYN <= 232448, "shared memory budget");
 // TMEM columns (both slots, through the lane halves)
 constexpr uint32_t TM_S = 0, TM_DP = 128, TM_Q = 256, TM_DO = 320, TM_DQ = 384;
@@ -138,6 +176,7 @@ struct Bars {
   uint64_t kfull[2][KST], kempty[2][KST], vfull[2][VST], vempty[2][VST];  // [slot][stage]
   uint64_t sfull[2], dsfull[2], bdone[2], qready[2];
   uint64_t done[2];
+  uint64_t iqfull[2][QD], iqempty[2][QD];  // [slot][entry]
 };
 static_assert(sizeof(Bars) <= 512, "barrier area");
 
@@ -171,7 +210,8 @@ __global__ void __launch_bounds__(BT, 1)
                           const __nv_bfloat16* __restrict__ dog, const float* __restrict__ lse,
                           float* __restrict__ ndelta, float* __restrict__ nlse2, const int32_t* __restrict__ kv_off,
                           const int32_t* __restrict__ kv_idx, float* __restrict__ dq_out, int N, int L, int topk,
-                          int items, float c2, float scale, const uint64_t* __restrict__ tmask, DevCtx ctx) {
+                          int items, float c2, float scale, const uint64_t* __restrict__ tmask,
+                          int* __restrict__ work_ctr, DevCtx ctx) {
   using namespace dqk;
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
   uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
@@ -180,7 +220,6 @@ __global__ void __launch_bounds__(BT, 1)
   volatile int* abort = flag_sh;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cap = N * topk;
-  const int step = 2 * gridDim.x;
 
   if (threadIdx.x == 0) {
     flag_sh[0] = 0;
@@ -192,6 +231,7 @@ __global__ void __launch_bounds__(BT, 1)
       mbar_init(&B.bdone[s], 1);
       mbar_init(&B.qready[s], 4);
       mbar_init(&B.done[s], 1);
+      for (int i = 0; i < QD; ++i) mbar_init(&B.iqfull[s][i], 1), mbar_init(&B.iqempty[s][i], 2);
     }
     fence_mbar_init();
   }
@@ -211,13 +251,16 @@ __global__ void __launch_bounds__(BT, 1)
       const int s = (warp - 8) >> 1;
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
+      // the slot's items: drawn here from the counter and passed to its MMA issuer and softmax
+      const SeqSrc src{ItemQueue{reinterpret_cast<volatile int*>(dsm + OFF_IQ) + s * QD, B.iqfull[s], B.iqempty[s]},
+                       true, work_ctr, items, abort};
       Seq sq;
-      sq.init(2 * blockIdx.x + s, step, items);
+      sq.init();
       int c = 0;
       bool ok = true;
       while (ok && sq.active) {
         int blk;
-        if (next_op(sq, &blk, kv_off, N, cap, 2, ctx) != 1) continue;
+        if (next_op(sq, &blk, kv_off, N, cap, 2, ctx, src) != 1) continue;
         const int ntile = min(2, sq.len - 2 * blk);
         int j[2] = {0, 0};
         for (int tt = 0; tt < ntile; ++tt) {
@@ -260,13 +303,15 @@ __global__ void __launch_bounds__(BT, 1)
       constexpr uint32_t id_kmaj = idesc_bf16_f32(64, 128, false, false);  // S, dP: N = 128 keys
       constexpr uint32_t id_mn = idesc_bf16_f32(64, 128, false, true);     // dQ: N = 128 (d)
       const uint32_t lanes = (uint32_t)(16 * s) << 16;
+      const SeqSrc src{ItemQueue{reinterpret_cast<volatile int*>(dsm + OFF_IQ) + s * QD, B.iqfull[s], B.iqempty[s]},
+                       false, work_ctr, items, abort};
       Seq sq;
-      sq.init(2 * blockIdx.x + s, step, items);
+      sq.init();
       int ga = 0, gb = 0;  // A and B ops issued
       bool ok = true;
       while (ok && sq.active) {
         int blk;
-        const int op = next_op(sq, &blk, kv_off, N, cap, 2, ctx);
+        const int op = next_op(sq, &blk, kv_off, N, cap, 2, ctx, src);
         if (op == 1) {
           if (blk == 0 && !(ok = mbar_wait(&B.qready[s], (sq.tile - 1) & 1, abort, ctx))) break;
           // S / dP of this slot are free once the previous dQ MMAs (which read dS) are done
@@ -314,7 +359,18 @@ __global__ void __launch_bounds__(BT, 1)
     const int row = 16 * w + 8 * (lane & 1) + (lane >> 2);
     const uint32_t tl = tmem + ((uint32_t)(32 * w + 16 * s) << 16);
     int g = 0;  // blocks processed by this slot
-    for (int item = 2 * blockIdx.x + s; item < items; item += step) {
+    const ItemQueue iq{reinterpret_cast<volatile int*>(dsm + OFF_IQ) + s * QD, B.iqfull[s], B.iqempty[s]};
+    volatile int* handover = reinterpret_cast<volatile int*>(dsm + OFF_IQ) + 2 * QD + 2 * s;  // [kq parity]
+    for (int kq = 0;;) {
+      // the slot's first warp takes the next item and hands it to the other three (the hand-over
+      // word alternates with the entry's parity, so it is rewritten only after every warp passed
+      // the next barrier)
+      const int par = kq & 1;
+      if (w == 0 && lane == 0) handover[par] = next_item(iq, kq, false, nullptr, items, abort, ctx);
+      else ++kq;
+      named_bar_sync(bar_id, 128);
+      const int item = handover[par];
+      if (item < 0) break;
       const int bh = item / N, qt = item - bh * N;
       const Row rw = load_list(kv_off, bh, qt, N, cap, ctx, w == 0 && lane == 0);
       const int nblk = (rw.len + 1) >> 1;
@@ -427,7 +483,8 @@ constexpr int RST = 6;                // ring stages; warp 8 fills the even ring
 constexpr uint32_t STAGE_B = 33792;   // [d half 0: Q, dO][d half 1: Q, dO], then 64 -lse*log2e, 64 -Delta
 constexpr uint32_t OFF_BAR = RST * STAGE_B;
 constexpr uint32_t OFF_FLAG = OFF_BAR + 512;
-constexpr uint32_t SMEM_DYN = OFF_FLAG + 64 + 1024;
+constexpr uint32_t OFF_IQ = OFF_FLAG + 64;  // [QD] item queue, then [2] softmax hand-over
+constexpr uint32_t SMEM_DYN = OFF_IQ + 64 + 1024;
 static_assert(SMEM_DYN <= 232448, "shared memory budget");
 static_assert(RST % 2 == 0, "each ring stage must have a single producer");
 // TMEM columns (all 128 lanes)
@@ -439,6 +496,7 @@ struct Bars {
   uint64_t full[RST], empty[RST];
   uint64_t spfull, spfree, pdsfull[2], pdsfree[2], itemdone, kvready;
   uint64_t done[2];
+  uint64_t iqfull[QD], iqempty[QD];
 };
 static_assert(sizeof(Bars) <= 512, "barrier area");
 }  // namespace dkv
@@ -449,7 +507,8 @@ __global__ void __launch_bounds__(dkv::KT, 1)
                             const float* __restrict__ nlse2, const float* __restrict__ ndelta,
                             const int32_t* __restrict__ q_off, const int32_t* __restrict__ q_idx,
                             float* __restrict__ dk_out, float* __restrict__ dv_out, int N, int L, int topk, int items,
-                            float c2, float scale, const uint64_t* __restrict__ tmask, DevCtx ctx) {
+                            float c2, float scale, const uint64_t* __restrict__ tmask, int* __restrict__ work_ctr,
+                            DevCtx ctx) {
   using namespace dkv;
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
   uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
@@ -458,7 +517,6 @@ __global__ void __launch_bounds__(dkv::KT, 1)
   volatile int* abort = flag_sh;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cap = N * topk;
-  const int step = gridDim.x;
 
   if (threadIdx.x == 0) {
     flag_sh[0] = 0;
@@ -470,6 +528,9 @@ __global__ void __launch_bounds__(dkv::KT, 1)
     mbar_init(&B.kvready, 8);
     mbar_init(&B.done[0], 1);
     mbar_init(&B.done[1], 1);
+    // the KV tiles: drawn from the counter by warp 8, taken by warp 10, both MMA issuers and
+    // the softmax
+    for (int i = 0; i < QD; ++i) mbar_init(&B.iqfull[i], 1), mbar_init(&B.iqempty[i], 4);
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -480,6 +541,7 @@ __global__ void __launch_bounds__(dkv::KT, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(flag_sh + 4);
+  const ItemQueue iq{reinterpret_cast<volatile int*>(dsm + OFF_IQ), B.iqfull, B.iqempty};
 
   if (warp == 8 || warp == 10) {
     // ------------------------------------------------------------------ producers (lane 0)
@@ -490,13 +552,14 @@ __global__ void __launch_bounds__(dkv::KT, 1)
       const int par = (warp - 8) >> 1;
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
+      const SeqSrc src{iq, par == 0, work_ctr, items, abort};
       Seq sq;
-      sq.init(blockIdx.x, step, items);
+      sq.init();
       int c = 0, last = -1;
       bool ok = true;
       while (ok && sq.active) {
         int blk;
-        if (next_op(sq, &blk, q_off, N, cap, 1, ctx) != 1) continue;
+        if (next_op(sq, &blk, q_off, N, cap, 1, ctx, src) != 1) continue;
         const int pos = c++;
         if ((pos & 1) != par) continue;
         int i = q_idx[(size_t)sq.bh * cap + sq.beg + blk];
@@ -531,13 +594,14 @@ __global__ void __launch_bounds__(dkv::KT, 1)
       const bool first = warp == 9;
       constexpr uint32_t id_a = idesc_bf16_f32(128, 128, false, false);  // [K;V] x [Q;dO]^T
       constexpr uint32_t id_b = idesc_bf16_f32(128, 256, false, true);   // [P;dS] x [Q | dO]
+      const SeqSrc src{iq, false, work_ctr, items, abort};
       Seq sq;
-      sq.init(blockIdx.x, step, items);
+      sq.init();
       int cnt = 0;  // MMAs groups issued by this thread
       bool ok = true;
       while (ok && sq.active) {
         int blk;
-        const int op = next_op(sq, &blk, q_off, N, cap, 1, ctx);
+        const int op = next_op(sq, &blk, q_off, N, cap, 1, ctx, src);
         if (op == 1 && first) {
           if (blk == 0 && !(ok = mbar_wait(&B.kvready, (sq.tile - 1) & 1, abort, ctx))) break;
           // S^T / dP^T of the previous query tile must have been read by the softmax
@@ -579,7 +643,17 @@ __global__ void __launch_bounds__(dkv::KT, 1)
     const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     const float2 cc = make_float2(c2, c2);
     int n = 0, it = 0;  // query tiles processed, non-empty items processed
-    for (int item = blockIdx.x; item < items; item += step) {
+    volatile int* handover = reinterpret_cast<volatile int*>(dsm + OFF_IQ) + QD;  // [kq parity]
+    for (int kq = 0;;) {
+      // warp 0 takes the next KV tile and hands it to the other seven (the hand-over word
+      // alternates with the entry's parity, so it is rewritten only after every warp passed the
+      // next barrier)
+      const int par = kq & 1;
+      if (warp == 0 && lane == 0) handover[par] = next_item(iq, kq, false, nullptr, items, abort, ctx);
+      else ++kq;
+      named_bar_sync(1, 256);
+      const int item = handover[par];
+      if (item < 0) break;
       const int bh = item / N, kt = item - bh * N;
       const Row rw = load_list(q_off, bh, kt, N, cap, ctx, warp == 0 && lane == 0);
       const size_t tok = (size_t)bh * L + (size_t)kt * 64 + j;
@@ -705,16 +779,20 @@ vsa2_status attn_bwd_tc(const Dims& d, const void* q, const void* k, const void*
   const int grid = std::max(1, std::min(sms, (items + 1) / 2));
   const float c1 = 1.f / sqrtf(128.f);
   const float c2 = kLog2e * c1;
+  // the item counter the kernels draw from (workspace header), reset before each of them
+  int* ctr = reinterpret_cast<int*>(ws + kWsWorkCounter);
   cudaFuncSetAttribute(attn_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dqk::SMEM_DYN);
+  if (cudaMemsetAsync(ctr, 0, sizeof(int), s) != cudaSuccess) return cuda_fail("attn_bwd_tc: item counter reset");
   attn_bwd_dq_tc_kernel<<<grid, BT, dqk::SMEM_DYN, s>>>(
       tk, tv, (const __nv_bfloat16*)q, (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, lse, ndelta, nlse2, kv_off,
-      kv_idx, dq, d.N, (int)d.L, topk, items, c2, c1, tmask, ctx);
+      kv_idx, dq, d.N, (int)d.L, topk, items, c2, c1, tmask, ctr, ctx);
   if (check_launch("attn_bwd_dq_tc_kernel") != VSA2_OK) return VSA2_ERR_CUDA;
   cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dkv::SMEM_DYN);
   const int grid_kv = std::max(1, std::min(sms, items));
+  if (cudaMemsetAsync(ctr, 0, sizeof(int), s) != cudaSuccess) return cuda_fail("attn_bwd_tc: item counter reset");
   attn_bwd_dkdv_tc_kernel<<<grid_kv, dkv::KT, dkv::SMEM_DYN, s>>>(tq, tdo, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
                                                           nlse2, ndelta, q_off, q_idx, dk, dv, d.N, (int)d.L, topk,
-                                                          items, c2, c1, tmask, ctx);
+                                                          items, c2, c1, tmask, ctr, ctx);
   return check_launch("attn_bwd_dkdv_tc_kernel");
 }
 
