@@ -771,7 +771,7 @@ def test_dq_protocol_one_ring_deadlocks_with_a_ahead():
         run_dq([8], random.Random(0), unified=True, mma_latency=3, ds_smem=True)
 
 
-def run_item_queue(n_items, qd, rng, empty_count=2, ahead=2):
+def run_item_queue(n_items, qd, rng, empty_count=None, ahead=2, consumers=2):
     """The forward kernel's per-slot item queue: the producer warp takes items from a global
     counter and writes each into entry k % qd (after the entry's release, iqempty), `ahead`
     items before it loads the item's blocks, then -1 at the end. The MMA issuer and the
@@ -781,11 +781,11 @@ def run_item_queue(n_items, qd, rng, empty_count=2, ahead=2):
     producer's sequence exactly, and progress."""
     ids = list(range(n_items)) + [-1]
     full = [Barrier(1) for _ in range(qd)]
-    empty = [Barrier(empty_count) for _ in range(qd)]
+    empty = [Barrier(consumers if empty_count is None else empty_count) for _ in range(qd)]
     slots = [None] * qd
     readers = [set() for _ in range(qd)]
     prod = {"k": 0}
-    cons = [{"k": 0, "got": [], "working": None} for _ in range(2)]
+    cons = [{"k": 0, "got": [], "working": None} for _ in range(consumers)]
 
     def loads_reached():  # items whose blocks the producer has issued
         return max(0, prod["k"] - ahead)
@@ -797,7 +797,7 @@ def run_item_queue(n_items, qd, rng, empty_count=2, ahead=2):
         e = k % qd
         if not empty[e].poll(k // qd - 1, f"producer entry {k}"):
             return False
-        assert slots[e] is None or readers[e] == {0, 1}, f"entry {k} written before both consumers read {k - qd}"
+        assert slots[e] is None or readers[e] == set(range(consumers)), f"entry {k} rewritten before every consumer read it"
         slots[e] = ids[k]
         readers[e] = set()
         full[e].arrive()
@@ -826,7 +826,7 @@ def run_item_queue(n_items, qd, rng, empty_count=2, ahead=2):
             st["working"] = v
         return True
 
-    agents = [producer, lambda: consumer(0), lambda: consumer(1)]
+    agents = [producer] + [lambda c=c: consumer(c) for c in range(consumers)]
     speed = [rng.uniform(0.05, 1.0) for _ in agents]
     while not all(st["got"] and st["got"][-1] == -1 for st in cons):
         moved = False
@@ -843,6 +843,15 @@ def run_item_queue(n_items, qd, rng, empty_count=2, ahead=2):
 def test_item_queue_parity_and_progress(seed):
     rng = random.Random(seed)
     run_item_queue(rng.randint(0, 40), qd=4, rng=rng)
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_item_queue_backward_kernels(seed):
+    """The backward kernels' queues: the drawing producer writes an item when it reaches it (no
+    lookahead); the dQ kernel has two takers per slot, the dK/dV kernel four."""
+    rng = random.Random(300 + seed)
+    run_item_queue(rng.randint(0, 40), qd=4, rng=rng, ahead=0, consumers=2)
+    run_item_queue(rng.randint(0, 40), qd=4, rng=rng, ahead=0, consumers=4)
 
 
 def test_item_queue_flags_a_single_release():
