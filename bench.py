@@ -627,7 +627,7 @@ def measure(args, wl, dev, rank, world):
         extra_peak = {"frac_of_sustained": roof["achieved"] / bf16_sus, "sustained_peak": bf16_sus}
     else:
         peak, kind = fp32_fma_peak_tflops(sm_max), f"derived fp32 FMA: 148 SMs x 128 lanes x 2 x {sm_max:.0f} MHz"
-        extra_peak = {"note": "latency-bound at this size: the longest CSR row runs serially in one 64-thread CTA"}
+        extra_peak = {"note": "latency-bound at this size: the longest CSR row runs serially in one CTA (four threads per query row)"}
     router_ms = statistics.mean(per["router"])
     esize = 2 if wl.dtype == "bf16" else 4
     router_bytes = 2 * wl.batch * wl.heads * wl.tokens * wl.head_dim * esize + wl.batch * wl.heads * wl.num_tiles ** 2 * 4

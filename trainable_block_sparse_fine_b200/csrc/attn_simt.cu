@@ -43,85 +43,111 @@ __device__ __forceinline__ bool idx_ok(int j, int N, const DevCtx& ctx) {
 
 namespace {
 
-// Forward: CTA = one query tile of one (b, h), thread t = query row t.
+// Forward: CTA = one query tile of one (b, h), four threads per query row t (lanes 4t .. 4t+3 of
+// the row's warp). Thread (t, g) scores the keys u = 4k + g and accumulates the output columns
+// d = 4e + g; the row's maximum and sum combine over the four lanes, and its probabilities pass
+// through shared memory inside the warp. K and V rows are stored with a stride of D + 1 floats
+// and the probability rows with 65, so the four threads of a row read different banks.
 template <typename T, int D>
-__global__ void __launch_bounds__(64) attn_fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
-                                                           const T* __restrict__ v, const int32_t* __restrict__ kv_off,
-                                                           const int32_t* __restrict__ kv_idx, T* __restrict__ o,
-                                                           float* __restrict__ lse, int N, int64_t L, int topk,
-                                                           int64_t kv_valid, const uint64_t* __restrict__ tmask,
-                                                           const float* __restrict__ gate, const T* __restrict__ oc,
-                                                           T* __restrict__ of, DevCtx ctx) {
+__global__ void __launch_bounds__(256) attn_fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                            const T* __restrict__ v, const int32_t* __restrict__ kv_off,
+                                                            const int32_t* __restrict__ kv_idx, T* __restrict__ o,
+                                                            float* __restrict__ lse, int N, int64_t L, int topk,
+                                                            int64_t kv_valid, const uint64_t* __restrict__ tmask,
+                                                            const float* __restrict__ gate, const T* __restrict__ oc,
+                                                            T* __restrict__ of, DevCtx ctx) {
+  constexpr int KS = D + 1;    // K / V row stride
+  constexpr int PS = 65;       // probability row stride
+  constexpr int DQ = D / 4;    // output columns per thread
   extern __shared__ float sm[];
   float* qT = sm;              // [D][64]
-  float* ks = qT + D * 64;     // [64][D]
-  float* vs = ks + 64 * D;     // [64][D]
-  float* oT = vs + 64 * D;     // [D][64]
-  const int i = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+  float* ks = qT + D * 64;     // [64][KS]
+  float* vs = ks + 64 * KS;    // [64][KS]
+  float* ps = vs + 64 * KS;    // [64][PS]
+  const int i = blockIdx.x, bh = blockIdx.y;
+  const int t = threadIdx.x >> 2, g = threadIdx.x & 3;
   const size_t tok0 = (size_t)bh * L + (size_t)i * kTile;
-  for (int e = t; e < 64 * D; e += 64) {
+  for (int e = threadIdx.x; e < 64 * D; e += 256) {
     const int r = e / D, c = e % D;
     qT[c * 64 + r] = ldf(q + (tok0 + r) * D + c);
-    oT[c * 64 + r] = 0.f;
   }
   const int beg = kv_off[(size_t)bh * (N + 1) + i], end = kv_off[(size_t)bh * (N + 1) + i + 1];
   const bool ok = row_ok(beg, end, N * topk, ctx);
   const int32_t* idx = kv_idx + (size_t)bh * N * topk;
   const float scale = rsqrtf((float)D);
   float m = -INFINITY, l = 0.f;
-  __syncthreads();
+  float acc[DQ];
+#pragma unroll
+  for (int e = 0; e < DQ; ++e) acc[e] = 0.f;
+  float* prow = ps + t * PS;
   for (int p = beg; ok && p < end; ++p) {
     const int j = idx[p];
     if (!idx_ok(j, N, ctx)) break;
     const size_t kt0 = (size_t)bh * L + (size_t)j * kTile;
     const uint64_t km = tmask ? tmask[j] : ~0ull;  // real tokens of a padded grid's tile
     __syncthreads();
-    for (int e = t; e < 64 * D; e += 64) {
-      ks[e] = ldf(k + kt0 * D + e);
-      vs[e] = ldf(v + kt0 * D + e);
+    for (int e = threadIdx.x; e < 64 * D; e += 256) {
+      const int r = e / D, c = e % D;
+      ks[r * KS + c] = ldf(k + kt0 * D + e);
+      vs[r * KS + c] = ldf(v + kt0 * D + e);
     }
     __syncthreads();
-    float s[64];
+    float s[16];
     float mx = -INFINITY;
-#pragma unroll 4
-    for (int u = 0; u < 64; ++u) {
-      float acc = 0.f;
-      for (int d = 0; d < D; ++d) acc += qT[d * 64 + t] * ks[u * D + d];
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      const int u = 4 * kk + g;
+      float a = 0.f;
+#pragma unroll 8
+      for (int d = 0; d < D; ++d) a = fmaf(qT[d * 64 + t], ks[u * KS + d], a);
       // keys past kv_valid, and padding tokens of a padded grid, are masked
-      s[u] = ((int64_t)j * kTile + u < kv_valid && ((km >> u) & 1ull)) ? acc * scale : -INFINITY;
-      mx = fmaxf(mx, s[u]);
+      s[kk] = ((int64_t)j * kTile + u < kv_valid && ((km >> u) & 1ull)) ? a * scale : -INFINITY;
+      mx = fmaxf(mx, s[kk]);
     }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     const float mn = fmaxf(m, mx);
     const float alpha = __expf(m - mn);
     float sum = 0.f;
 #pragma unroll
-    for (int u = 0; u < 64; ++u) {
-      s[u] = __expf(s[u] - mn);
-      sum += s[u];
+    for (int kk = 0; kk < 16; ++kk) {
+      const float pr = __expf(s[kk] - mn);
+      sum += pr;
+      prow[4 * kk + g] = pr;
     }
+    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
     l = l * alpha + sum;
     m = mn;
-    for (int d = 0; d < D; ++d) {
-      float acc = oT[d * 64 + t] * alpha;
+    __syncwarp();  // the row's 64 probabilities are written by its four lanes
 #pragma unroll
-      for (int u = 0; u < 64; ++u) acc += s[u] * vs[u * D + d];
-      oT[d * 64 + t] = acc;
+    for (int e = 0; e < DQ; ++e) acc[e] *= alpha;
+#pragma unroll 4
+    for (int u = 0; u < 64; ++u) {
+      const float pr = prow[u];
+      const float* vr = vs + u * KS + g;
+#pragma unroll
+      for (int e = 0; e < DQ; ++e) acc[e] = fmaf(pr, vr[4 * e], acc[e]);
     }
+    __syncwarp();  // before the next tile's probabilities overwrite the row
   }
   const bool q_real = !tmask || ((tmask[i] >> t) & 1ull);  // a padding query row gets o = 0, lse = -inf
   const float inv = (l > 0.f && q_real) ? 1.f / l : 0.f;
+  T* orow = o + (tok0 + t) * D + g;
   if (gate) {  // Eq. 13-14 on the fp32 fine output: o = tanh(g) * oc[tile] + O_f
     const float gt = tanhf(gate[tok0 + t]);
-    const T* crow = oc + ((size_t)bh * N + i) * D;
-    for (int d = 0; d < D; ++d) {
-      const float f = inv != 0.f ? oT[d * 64 + t] * inv : 0.f;
-      stf(o + (tok0 + t) * D + d, fmaf(gt, ldf(crow + d), f));
-      if (of) stf(of + (tok0 + t) * D + d, f);
+    const T* crow = oc + ((size_t)bh * N + i) * D + g;
+#pragma unroll
+    for (int e = 0; e < DQ; ++e) {
+      const float f = inv != 0.f ? acc[e] * inv : 0.f;
+      stf(orow + 4 * e, fmaf(gt, ldf(crow + 4 * e), f));
+      if (of) stf(of + (tok0 + t) * D + g + 4 * e, f);
     }
   } else {
-    for (int d = 0; d < D; ++d) stf(o + (tok0 + t) * D + d, inv != 0.f ? oT[d * 64 + t] * inv : 0.f);
+#pragma unroll
+    for (int e = 0; e < DQ; ++e) stf(orow + 4 * e, inv != 0.f ? acc[e] * inv : 0.f);
   }
-  lse[tok0 + t] = (l > 0.f && q_real) ? m + __logf(l) : -INFINITY;
+  if (g == 0) lse[tok0 + t] = (l > 0.f && q_real) ? m + __logf(l) : -INFINITY;
 }
 
 // delta = rowsum(dO * O), warp per row.
@@ -284,10 +310,10 @@ template <typename T, int D>
 vsa2_status fwd_simt(const Dims& d, const void* q, const void* k, const void* v, const int32_t* kv_off,
                      const int32_t* kv_idx, void* o, float* lse, const DevCtx& ctx, int topk, int64_t kv_valid,
                      const uint64_t* tmask, const float* gate, const void* oc, void* of, cudaStream_t s) {
-  const size_t smem = (size_t)4 * 64 * D * sizeof(float);
+  const size_t smem = ((size_t)64 * D + 2 * 64 * (D + 1) + 64 * 65) * sizeof(float);
   auto kern = attn_fwd_simt_kernel<T, D>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  kern<<<dim3(d.N, d.BH), 64, smem, s>>>((const T*)q, (const T*)k, (const T*)v, kv_off, kv_idx, (T*)o, lse, d.N,
+  kern<<<dim3(d.N, d.BH), 256, smem, s>>>((const T*)q, (const T*)k, (const T*)v, kv_off, kv_idx, (T*)o, lse, d.N,
                                          d.L, topk, kv_valid, tmask, gate, (const T*)oc, (T*)of, ctx);
   return check_launch(__func__);
 }
