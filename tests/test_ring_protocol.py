@@ -13,9 +13,15 @@ finishes (no deadlock). The agents follow the kernel's protocol:
     MMA's completion releases the ring position and signals S (sfull) or P.V done (pvdone);
   * the softmax waits for S, frees its buffer, then waits for the previous P.V before writing P.
 The kernel's variant is one producer per slot and a 3-block ring holding K and V in op order.
-The model also covers the planned split with two producers (one per d-half, the full barrier
-expecting two arrivals). Besides the barrier rules it asserts the data hazards the barriers
+The model also covers splits with two producers per slot (one per d-half, the full barrier
+expecting two arrivals; or one per ring-position parity, which with three stages needs the
+positions issued in order). Besides the barrier rules it asserts the data hazards the barriers
 exist for: a ring block, an S buffer or P is overwritten only after its last reader finished.
+
+Further models: P written over its S buffer and the softmax split over two warps per lane
+quarter (`run_aliased`), the dK/dV and dQ kernels (`run_dkdv`, `run_dq`, the latter with dS in
+shared memory), and the item queues through which the kernels hand out the items they draw
+from a global counter (`run_item_queue`).
 """
 import random
 
