@@ -15,7 +15,8 @@
 //      S^T = K Q^T and dP^T = V dO^T (A = K, V in TMEM; B = Q, dO, K-major)
 //      P^T and dS^T written back as bf16
 //      dV += P^T dO and dK += dS^T Q (B = dO, Q read MN-major)
-// Every output row is owned by one CTA: no atomics, deterministic results.
+// Every output row is written by one CTA (items are drawn from a global counter, but each is
+// computed whole by the CTA that drew it): no atomics on the outputs, deterministic results.
 #include <algorithm>
 
 #include "common.cuh"
