@@ -219,7 +219,7 @@ def test_padded_grid_coarse_and_merge_backward_match_oracle(case):
         kc, _ = _padded_oracle_inputs(x["k"][0, h], grid, d)
         vc, _ = _padded_oracle_inputs(x["v"][0, h], grid, d)
         _, w_doc, w_dlog = O.gated_merge_bwd_padded(do_np[0, h], oc_np[0, h], logits[0, h], vm)
-        _close(d_oc_np[0, h], w_doc, f"d_oc h{h}", tol_abs=2e-2 * max(1.0, np.abs(w_doc).max()))
+        _close(d_oc_np[0, h], w_doc, f"d_oc h{h}")
         assert np.all(d_logits[0, h][~vm] == 0)
         _close(d_logits[0, h][vm], w_dlog[vm], f"d_logits h{h}")
         # the coarse backward takes d_oc rounded to the dtype (its tensor-core operand)
