@@ -3,9 +3,10 @@ tile and pooling sizes the deep-read blog infers for VSA2 (its section 07, "fine
 a variant of the pages' 64 / 16 shapes. Tiles are 4x4x8 tokens, sub-cubes 2x2x2.
 
 The router pools 8-token sub-cubes and sums 16 x 16 sub-cube pairs per tile pair (Eq. 5-7); the
-per-sequence TopK ranks N x N tiles (Eq. 8-9); the attention runs on the library's 64-token
-kernels after the selection of every 128-token tile is expanded to its two 64-token halves
-(the result is the same softmax over the same keys). Everything is compared with the oracle at
+per-sequence TopK ranks N x N tiles (Eq. 8-9); the bf16 forward with head_dim 128 runs M=128
+query tiles against whole 128-token KV tiles, and the other paths (fp32, head_dim 64, the
+backward) run on the library's 64-token kernels after the selection of every 128-token tile is
+expanded to its two 64-token halves (the same softmax over the same keys). Everything is compared with the oracle at
 tile_tokens = 128, pool_tokens = 8, with the tolerances of the 64-token tests.
 """
 import numpy as np
@@ -77,6 +78,66 @@ def test_b128_router_topk_forward_backward(case):
                                   sel["kv_idx"], tile_tokens=128)
         for n, got, w in zip(("dq", "dk", "dv"), (dq, dk, dv), grads):
             _close(got[0, h].cpu().numpy(), w, f"{n} h{h}")
+
+
+def _lists(masks):
+    """Boolean tile masks [H, N, N] -> CSR (kv_off, kv_idx) with room for the largest row budget."""
+    H, N, _ = masks.shape
+    topk = max(1, max(int(np.ceil(m.sum() / N)) for m in masks))
+    kv_off = np.zeros((1, H, N + 1), np.int32)
+    kv_idx = np.zeros((1, H, N * topk), np.int32)
+    for h in range(H):
+        kv_off[0, h, 1:] = np.cumsum(masks[h].sum(1))
+        r = np.nonzero(masks[h])[1]
+        kv_idx[0, h, :r.size] = r
+    return kv_off, kv_idx, topk
+
+
+def _edge_masks(pattern, H, N, rng):
+    masks = np.zeros((H, N, N), bool)
+    for h in range(H):
+        m = masks[h]
+        if pattern == "empty_rows":
+            m[:] = rng.random((N, N)) < 6 / N
+            m[::3] = False
+        elif pattern == "single":
+            m[np.arange(N), rng.integers(0, N, N)] = True
+        elif pattern == "odd":
+            for i in range(N):
+                m[i, rng.choice(N, size=min(N, 2 * (i % 5) + 1), replace=False)] = True
+        elif pattern == "dense":
+            m[:] = True
+        else:  # "long": a few rows take every tile (more indices than the kernel keeps on chip)
+            m[:] = rng.random((N, N)) < 4 / N
+            m[rng.choice(N, size=6, replace=False)] = True
+    return masks
+
+
+@pytest.mark.parametrize("case,pattern", [("small_bf16", p) for p in ("empty_rows", "single", "odd", "dense")]
+                         + [("480p_like", "long")])
+def test_b128_fwd_edge_selections(case, pattern):
+    """The forward on 128-token tiles (M=128 query tiles against whole 128-token KV tiles) on
+    selections at its edges: rows with no tile (o = 0, lse = -inf), one tile (a single S and O
+    op), odd lengths, every tile, and rows of all 336 tiles (past the indices kept in shared
+    memory); O and LSE against the oracle."""
+    wl = CASES[case]
+    rng = np.random.default_rng(11)
+    x = {n: S.make_tensor(wl, n) for n in ("q", "k", "v")}
+    xd = {n: _dev(x[n], wl.dtype) for n in x}
+    masks = _edge_masks(pattern, wl.heads, wl.tokens // 128, rng)
+    kv_off, kv_idx, topk = _lists(masks)
+    e = V.VSA2(wl.batch, wl.heads, wl.head_dim, wl.grid, wl.dtype, topk, tile=TILE, pool=POOL)
+    o, lse = e.attn_fwd(xd["q"], xd["k"], xd["v"], torch.from_numpy(kv_off).cuda(), torch.from_numpy(kv_idx).cuda(),
+                        topk)
+    assert e.device_error() == 0
+    o, lse = o.float().cpu().numpy(), lse.cpu().numpy()
+    for h in range(wl.heads):
+        wo, wlse = O.sparse_attn_fwd(x["q"][0, h], x["k"][0, h], x["v"][0, h], kv_off[0, h], kv_idx[0, h],
+                                     tile_tokens=128)
+        _close(o[0, h], wo, f"{pattern} o h{h}")
+        fin = np.isfinite(wlse)
+        assert np.array_equal(np.isfinite(lse[0, h]), fin), f"{pattern} lse -inf rows h{h}"
+        assert np.abs(lse[0, h][fin] - wlse[fin]).max() <= 2e-3 * max(1.0, np.abs(wlse[fin]).max()), pattern
 
 
 def test_b128_refuses_what_it_does_not_take():

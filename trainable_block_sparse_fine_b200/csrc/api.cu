@@ -299,7 +299,9 @@ vsa2_status vsa2_sparse_attn_fwd(const vsa2_problem* p, const void* q, const voi
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return VSA2_ERR_INVALID_ARG;
   if ((st = check_ws(d, ws, ws_bytes, topk)) != VSA2_OK) return st;
-  if (d.Bt != kTile) {  // 128-token tiles: expand the selection, run on 64-token tiles
+  if (d.Bt != kTile && d.dtype == VSA2_BF16 && d.D == 128 && !d.padded)  // M=128 query tiles
+    return attn_fwd_b128_tc(d, q, k, v, topk, kv_off, kv_idx, o, lse, (char*)ws, (cudaStream_t)stream);
+  if (d.Bt != kTile) {  // 128-token tiles otherwise: expand the selection, run on 64-token tiles
     const ExpLayout e = exp_layout(d, topk);
     char* w = (char*)ws;
     int32_t* off64 = reinterpret_cast<int32_t*>(w + e.off);

@@ -174,6 +174,11 @@ vsa2_status attn_fwd_tc_gated(const Dims& d, const void* q, const void* k, const
 vsa2_status attn_fwd_tc_masked(const Dims& d, const void* q, const void* k, const void* v, int topk,
                                const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
                                int kv_valid, cudaStream_t s);
+// tensor-core forward on 128-token tiles (d.Bt = 128, bf16, head_dim 128, grids the tile
+// divides): M=128 query tiles against whole 128-token KV tiles of the selection as given
+vsa2_status attn_fwd_b128_tc(const Dims& d, const void* q, const void* k, const void* v, int topk,
+                             const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
+                             cudaStream_t s);
 // Coarse branch (Eq. 1-3) and gated merge (Eq. 4, 13-14)
 vsa2_status launch_coarse_attn(const Dims& d, const void* q, const void* k, const void* v, void* oc, float* lse_c,
                                char* ws, cudaStream_t s);
