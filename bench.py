@@ -381,6 +381,38 @@ def time_next_rows(e, x, wl, steps, stream, l2_flush, ev, hbm, tc_peak, sel=None
             "v_pool_floor_ms": v_bytes / (hbm * 1e9) * 1e3,
             "kernels": "router_pool_kernel<..., true> writes Qc, Kc; coarse_pool_kernel (V) + coarse_csr_kernel + "
                        "attn_fwd_tc_kernel<1>"}
+    if (wl.dtype == "bf16" and D == 128 and wl.topk % 2 == 0 and not getattr(wl, "padded", False)
+            and wl.grid[0] % 4 == 0 and wl.grid[1] % 4 == 0 and wl.grid[2] % 8 == 0):
+        # 128-token tiles (4x4x8, 8-token router sub-cubes): the same tensors reordered by the
+        # permutation kernels, the same sparsity (top k/2 of tiles twice as large); router + TopK
+        # once, then the forward, which runs M=128 query tiles against whole 128-token KV tiles
+        from trainable_block_sparse_fine_b200 import VSA2
+        k2 = wl.topk // 2
+        e2 = VSA2(B, H, D, wl.grid, "bf16", k2, tile=(4, 4, 8), pool=(2, 2, 2))
+        x2 = {n: e2.to_cube_major(e.to_raster(x[n])) for n in ("q", "k", "v")}
+        sc2 = e2.router_scores(x2["q"], x2["k"])
+        off2, idx2 = e2.topk_select(sc2, k2, csc=False)[:2]
+        del sc2
+        t2 = []
+        for it in range(3 + steps):
+            t = [ev() for _ in range(2)]
+            l2_flush.zero_()
+            t[0].record(stream)
+            e2.attn_fwd(x2["q"], x2["k"], x2["v"], off2, idx2)
+            t[1].record(stream)
+            torch.cuda.synchronize()
+            if it >= 3:
+                t2.append(t[0].elapsed_time(t[1]))
+        if e2.device_error() != 0:
+            raise RuntimeError("device error in the 128-token-tile forward")
+        pairs2 = int(off2[..., -1].sum().item())
+        f2 = 4.0 * 128 * 128 * D * pairs2
+        ms2 = statistics.mean(t2)
+        extra["fwd_128_token_tiles"] = {
+            "ms": ms2, "topk": k2, "tile_pairs": pairs2, "effective_tflops": f2 / (ms2 * 1e-3) / 1e12,
+            "frac_of_burst_bf16": f2 / (ms2 * 1e-3) / 1e12 / tc_peak,
+            "kernel": "attn_fwd_b128_kernel (M=128 query tiles, whole 128-token KV tiles)"}
+        del x2, off2, idx2, e2
     # the token permutation (§2.2): Q from raster to cube-major order, one read and one write
     tp = []
     for it in range(3 + steps):
