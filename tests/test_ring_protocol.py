@@ -20,8 +20,9 @@ exist for: a ring block, an S buffer or P is overwritten only after its last rea
 
 Further models: P written over its S buffer and the softmax split over two warps per lane
 quarter (`run_aliased`), the dK/dV and dQ kernels (`run_dkdv`, `run_dq`, the latter also with
-dS in shared memory), and the item queues through which the kernels hand out the items they
-draw from a global counter (`run_item_queue`).
+dS in shared memory), the item queues through which the kernels hand out the items they
+draw from a global counter (`run_item_queue`), and the forward on 128-token tiles with its
+separate K and V rings, P over S and Q rewritten per query tile (`run_b128`).
 """
 import random
 
@@ -875,3 +876,188 @@ def test_item_queue_needs_as_many_entries_as_the_lookahead():
     run_item_queue(10, qd=2, rng=random.Random(0), ahead=2)
     with pytest.raises(AssertionError, match="deadlock"):
         run_item_queue(10, qd=1, rng=random.Random(0), ahead=2)
+
+
+def run_b128(items, rng, kst=3, vst=3, mma_latency=3, rescale_p=0.2, lead=1, qready_count=True):
+    """The forward on 128-token tiles: a K ring and a V ring, each with its own producer (in the
+    item's block order); one MMA issuer walking S0, S1, O0, S2, O1, ... per item; S(n) and P(n)
+    share TMEM buffer n % 2 (P written over S by the softmax), so S(n + 2) may overwrite it only
+    after O(n) has read P(n), which the in-order tensor pipe gives because S(n + 2) is issued
+    after O(n). Per item the softmax writes Q (after reading the item's last S) and signals
+    qready, which the first S MMA of the item waits for; O(0) of an item starts a fresh
+    accumulation, after the softmax's epilogue of the previous item read O (ordered through
+    pfull). A raise (random here) waits for O(n - 1) before rescaling O. `qready_count=False`
+    lets the first S of an item skip its wait (a seeded mistake)."""
+    tiles = [n for n in items]
+    ops = []  # (kind, item, block, global block index)
+    gb = 0
+    for it, n in enumerate(tiles):
+        for kind, k in ops_of([n], lead):
+            ops.append((kind, it, k, gb + k))
+        gb += n
+    nblk = gb
+    kfull, kempty = [Barrier(1) for _ in range(kst)], [Barrier(1) for _ in range(kst)]
+    vfull, vempty = [Barrier(1) for _ in range(vst)], [Barrier(1) for _ in range(vst)]
+    sfull, pfull, pvdone = [Barrier(1), Barrier(1)], [Barrier(1), Barrier(1)], [Barrier(1), Barrier(1)]
+    qready = Barrier(1)
+    prod = {"k": 0, "v": 0}
+    mma = {"c": 0, "s": 0, "o": 0, "tile": 0}
+    soft = {"item": 0, "blk": 0, "g": 0, "step": 0}
+    s_done, o_done, s_read, p_written, o_issued = set(), set(), set(), set(), set()
+    q_written = set()       # items whose Q is in TMEM
+    epi_done = set()        # items whose epilogue has read O
+    k_read, v_read = set(), set()
+    pipe = {"free": 0}      # the tensor pipe completes in issue order
+    pending = []
+    t = 0
+    nonempty = [i for i, n in enumerate(tiles) if n > 0]
+
+    def producer(kind):
+        c = prod[kind]
+        if c >= nblk:
+            return False
+        nst, empty, full, read = (kst, kempty, kfull, k_read) if kind == "k" else (vst, vempty, vfull, v_read)
+        st = c % nst
+        if not empty[st].poll(c // nst - 1, f"{kind} producer at {c}"):
+            return False
+        assert c < nst or c - nst in read, f"{kind} ring position {c} refilled before its MMA finished"
+        full[st].arrive()
+        prod[kind] += 1
+        return True
+
+    def issue(done):
+        pipe["free"] = max(pipe["free"], t) + rng.randint(1, mma_latency)
+        pending.append((pipe["free"], done))
+
+    def issuer():
+        c = mma["c"]
+        if c >= len(ops):
+            return False
+        kind, it, k, g = ops[c]
+        if kind == "S":
+            if k == 0:
+                tl = nonempty.index(it)
+                if qready_count and not qready.poll(tl, f"issuer Q of item {it}"):
+                    return False
+            if not kfull[g % kst].poll(g // kst, f"issuer S{g}"):
+                return False
+            # the pipe runs one thread's MMAs in order: O(g - 2) issued means it reads P(g - 2) first
+            assert g < 2 or g - 2 in o_issued, f"S{g} issued before O{g - 2}"
+            assert g < 2 or g - 2 in s_read, f"S{g} overwrites S{g - 2} before the softmax read it"
+
+            def done(g=g, it=it):
+                assert it in q_written, f"S{g} read Q of item {it} before it was written"
+                assert (g - 2 < 0) or (g - 2 in o_done) or (g - 2 not in p_written), f"S{g} overwrote P{g - 2}"
+                s_done.add(g)
+                k_read.add(g)
+                kempty[g % kst].arrive()
+                sfull[g % 2].arrive()
+            issue(done)
+            mma["s"] += 1
+        else:
+            if not vfull[g % vst].poll(g // vst, f"issuer O{g} V"):
+                return False
+            if not pfull[g % 2].poll(g // 2, f"issuer O{g} P"):
+                return False
+            if k == 0:
+                assert it == 0 or (it - 1) in epi_done or all(tiles[j] == 0 for j in range(it)), \
+                    f"O(0) of item {it} would reset O before the previous epilogue read it"
+
+            o_issued.add(g)
+
+            def done(g=g):
+                assert g in p_written
+                o_done.add(g)
+                v_read.add(g)
+                vempty[g % vst].arrive()
+                pvdone[g % 2].arrive()
+            issue(done)
+            mma["o"] += 1
+        mma["c"] += 1
+        return True
+
+    def softmax():
+        it = soft["item"]
+        if it >= len(tiles):
+            return False
+        n = tiles[it]
+        if soft["step"] == 0:  # item start: write Q (the previous item's S are all read)
+            if n > 0:
+                assert all(x in s_done for x in range(soft["g"])), "Q rewritten before the last S finished"
+                q_written.discard(it - 1)
+                q_written.add(it)
+                qready.arrive()
+            soft["step"] = 1
+            return True
+        b = soft["blk"]
+        g = soft["g"]
+        if b < n:
+            if soft["step"] == 1:
+                if not sfull[g % 2].poll(g // 2, f"softmax S{g}"):
+                    return False
+                s_read.add(g)
+                soft["step"] = 2 if (b > 0 and rng.random() < rescale_p) else 3
+                return True
+            if soft["step"] == 2:  # raise: rescale O once O(g - 1) is done
+                if not pvdone[(g - 1) % 2].poll((g - 1) // 2, f"softmax rescale at {g}"):
+                    return False
+                assert g - 1 in o_done
+                soft["step"] = 3
+                return True
+            p_written.add(g)  # P over its own S buffer: nothing to wait for
+            pfull[g % 2].arrive()
+            soft["blk"], soft["g"], soft["step"] = b + 1, g + 1, 1
+            return True
+        if n > 0:  # epilogue: O of the item complete
+            if not pvdone[(g - 1) % 2].poll((g - 1) // 2, f"softmax epilogue of item {it}"):
+                return False
+            assert g - 1 in o_done
+        epi_done.add(it)
+        soft["item"], soft["blk"], soft["step"] = it + 1, 0, 0
+        return True
+
+    agents = [lambda: producer("k"), lambda: producer("v"), issuer, softmax]
+    speed = [rng.uniform(0.05, 1.0) for _ in agents]
+    while mma["c"] < len(ops) or soft["item"] < len(tiles) or pending:
+        t += 1
+        due = sorted([x for x in pending if x[0] <= t], key=lambda x: x[0])
+        pending[:] = [x for x in pending if x[0] > t]
+        for _, done in due:
+            done()
+        moved = bool(due)
+        for i in rng.sample(range(len(agents)), len(agents)):
+            if rng.random() < speed[i]:
+                moved |= agents[i]()
+        if not moved and not pending and not any(a() for a in agents):
+            raise AssertionError(f"deadlock at op {mma['c']} of {len(ops)}, softmax item {soft['item']}")
+    assert len(o_done) == nblk and prod["k"] == nblk and prod["v"] == nblk
+
+
+@pytest.mark.parametrize("seed", range(30))
+def test_b128_forward_protocol(seed):
+    rng = random.Random(seed)
+    items = [rng.choice([0, 1, 2, 3, 5, 8]) for _ in range(rng.randint(2, 8))]
+    run_b128(items, rng)
+
+
+def test_b128_forward_protocol_flags_a_skipped_qready_wait():
+    hits = 0
+    for seed in range(60):
+        rng = random.Random(seed)
+        try:
+            run_b128([3, 4, 2, 5], rng, qready_count=False)
+        except AssertionError:
+            hits += 1
+    assert hits > 0
+
+
+def test_b128_forward_protocol_flags_lead_two_with_p_over_s():
+    """With S two blocks ahead (S0, S1, S2, O0, ...), S(n + 2) would be issued before O(n) has
+    read P(n) from the buffer it overwrites."""
+    hits = 0
+    for seed in range(30):
+        try:
+            run_b128([4, 3, 5], random.Random(seed), lead=2)
+        except AssertionError:
+            hits += 1
+    assert hits == 30
