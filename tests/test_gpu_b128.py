@@ -3,10 +3,10 @@ tile and pooling sizes the deep-read blog infers for VSA2 (its section 07, "fine
 a variant of the pages' 64 / 16 shapes. Tiles are 4x4x8 tokens, sub-cubes 2x2x2.
 
 The router pools 8-token sub-cubes and sums 16 x 16 sub-cube pairs per tile pair (Eq. 5-7); the
-per-sequence TopK ranks N x N tiles (Eq. 8-9); the bf16 forward with head_dim 128 runs M=128
-query tiles against whole 128-token KV tiles, and the other paths (fp32, head_dim 64, the
-backward) run on the library's 64-token kernels after the selection of every 128-token tile is
-expanded to its two 64-token halves (the same softmax over the same keys). Everything is compared with the oracle at
+per-sequence TopK ranks N x N tiles (Eq. 8-9); with bf16 and head_dim 128 the forward and the dQ
+kernel run M=128 query tiles against whole 128-token KV tiles, while dK/dV and the other paths
+(fp32, head_dim 64) run on the library's 64-token kernels after the selection of every
+128-token tile is expanded to its two 64-token halves (the same softmax over the same keys). Everything is compared with the oracle at
 tile_tokens = 128, pool_tokens = 8, with the tolerances of the 64-token tests.
 """
 import numpy as np

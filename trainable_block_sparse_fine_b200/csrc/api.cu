@@ -11,7 +11,6 @@
 #include "internal.h"
 
 namespace vsa2 {
-
 vsa2_status make_dims(const vsa2_problem* p, Dims* d) {
   if (!p || !d) return VSA2_ERR_INVALID_ARG;
   if (p->batch <= 0 || p->heads <= 0 || p->head_dim <= 0 || p->grid_t <= 0 || p->grid_h <= 0 || p->grid_w <= 0)
@@ -362,6 +361,17 @@ vsa2_status vsa2_sparse_attn_bwd(const vsa2_problem* p, const void* q, const voi
     int32_t* idx64 = reinterpret_cast<int32_t*>(w + e.idx);
     int32_t* qoff64 = reinterpret_cast<int32_t*>(w + e.qoff);
     int32_t* qidx64 = reinterpret_cast<int32_t*>(w + e.qidx);
+    if (d.dtype == VSA2_BF16 && d.D == 128 && !d.padded) {
+      // dQ on the 128-token CSR (M=128 query tiles); dK, dV on the expanded CSC
+      if ((st = launch_expand_lists(d, topk, q_off, q_idx, qoff64, qidx64, s)) != VSA2_OK) return st;
+      const Dims d64 = dims64(d);
+      float* ndelta = reinterpret_cast<float*>(w + ws_layout(d64).delta);
+      float* nlse2 = reinterpret_cast<float*>(w + ws_layout(d64).nlse2);
+      if ((st = attn_bwd_dq_b128_tc(d, q, k, v, o, lse, dout, kv_off, kv_idx, dq, ndelta, nlse2, topk, w, s)) !=
+          VSA2_OK)
+        return st;
+      return attn_bwd_dkdv_only_tc(d64, q, k, v, dout, qoff64, qidx64, dk, dv, 2 * topk, w, s);
+    }
     if ((st = launch_expand_lists(d, topk, kv_off, kv_idx, off64, idx64, s)) != VSA2_OK) return st;
     if ((st = launch_expand_lists(d, topk, q_off, q_idx, qoff64, qidx64, s)) != VSA2_OK) return st;
     return launch_attn_bwd(dims64(d), q, k, v, o, lse, dout, 2 * topk, off64, idx64, qoff64, qidx64, dq, dk, dv, w, s);

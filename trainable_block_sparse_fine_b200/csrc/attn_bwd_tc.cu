@@ -797,4 +797,31 @@ vsa2_status attn_bwd_tc(const Dims& d, const void* q, const void* k, const void*
   return check_launch("attn_bwd_dkdv_tc_kernel");
 }
 
+// The dK/dV kernel alone, on the CSC of 64-token tiles, with -Delta and -lse * log2(e) already in
+// the workspace (written by a dQ kernel of 128-token tiles).
+vsa2_status attn_bwd_dkdv_only_tc(const Dims& d, const void* q, const void* k, const void* v, const void* dout,
+                                  const int32_t* q_off, const int32_t* q_idx, float* dk, float* dv, int topk, char* ws,
+                                  cudaStream_t s) {
+  CUtensorMap tq, tdo;
+  const uint64_t rows = (uint64_t)d.BH * d.L;
+  if (!make_tmap_2d_bf16(&tq, q, 128, rows, 64, 64) || !make_tmap_2d_bf16(&tdo, dout, 128, rows, 64, 64))
+    return tmap_fail("tensor map encoding for the backward operands failed");
+  DevCtx ctx{reinterpret_cast<int*>(ws), d.timeout_ns, d.flags};
+  const float* ndelta = reinterpret_cast<const float*>(ws + ws_layout(d).delta);
+  const float* nlse2 = reinterpret_cast<const float*>(ws + ws_layout(d).nlse2);
+  const int items = d.BH * d.N;
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const float c1 = 1.f / sqrtf(128.f);
+  int* ctr = reinterpret_cast<int*>(ws + kWsWorkCounter);
+  cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dkv::SMEM_DYN);
+  const int grid_kv = std::max(1, std::min(sms, items));
+  if (cudaMemsetAsync(ctr, 0, sizeof(int), s) != cudaSuccess) return cuda_fail("attn_bwd_dkdv: item counter reset");
+  attn_bwd_dkdv_tc_kernel<<<grid_kv, dkv::KT, dkv::SMEM_DYN, s>>>(tq, tdo, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+                                                          nlse2, ndelta, q_off, q_idx, dk, dv, d.N, (int)d.L, topk,
+                                                          items, kLog2e * c1, c1, nullptr, ctr, ctx);
+  return check_launch("attn_bwd_dkdv_tc_kernel");
+}
+
 }  // namespace vsa2

@@ -179,6 +179,15 @@ vsa2_status attn_fwd_tc_masked(const Dims& d, const void* q, const void* k, cons
 vsa2_status attn_fwd_b128_tc(const Dims& d, const void* q, const void* k, const void* v, int topk,
                              const int32_t* kv_off, const int32_t* kv_idx, void* o, float* lse, char* ws,
                              cudaStream_t s);
+// dQ on 128-token tiles (d.Bt = 128, bf16, head_dim 128, grids the tile divides) from the
+// 128-token CSR, with -Delta and -lse * log2(e) per token written to ndelta / nlse2 for the
+// dK/dV kernel; and that dK/dV kernel alone, on a CSC of 64-token tiles (d in 64-token tiles)
+vsa2_status attn_bwd_dq_b128_tc(const Dims& d, const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dout, const int32_t* kv_off, const int32_t* kv_idx,
+                                float* dq, float* ndelta, float* nlse2, int topk, char* ws, cudaStream_t s);
+vsa2_status attn_bwd_dkdv_only_tc(const Dims& d, const void* q, const void* k, const void* v, const void* dout,
+                                  const int32_t* q_off, const int32_t* q_idx, float* dk, float* dv, int topk, char* ws,
+                                  cudaStream_t s);
 // Coarse branch (Eq. 1-3) and gated merge (Eq. 4, 13-14)
 vsa2_status launch_coarse_attn(const Dims& d, const void* q, const void* k, const void* v, void* oc, float* lse_c,
                                char* ws, cudaStream_t s);
