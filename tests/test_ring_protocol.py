@@ -21,8 +21,9 @@ exist for: a ring block, an S buffer or P is overwritten only after its last rea
 Further models: P written over its S buffer and the softmax split over two warps per lane
 quarter (`run_aliased`), the dK/dV and dQ kernels (`run_dkdv`, `run_dq`, the latter also with
 dS in shared memory), the item queues through which the kernels hand out the items they
-draw from a global counter (`run_item_queue`), and the forward on 128-token tiles with its
-separate K and V rings, P over S and Q rewritten per query tile (`run_b128`).
+draw from a global counter (`run_item_queue`), the forward on 128-token tiles with its
+separate K and V rings, P over S and Q rewritten per query tile (`run_b128`), and the dQ kernel
+on 128-token tiles with dS over S and K held until dQ has read it (`run_dq_b128`).
 """
 import random
 
@@ -1061,3 +1062,149 @@ def test_b128_forward_protocol_flags_lead_two_with_p_over_s():
         except AssertionError:
             hits += 1
     assert hits == 30
+
+
+def run_dq_b128(items, rng, kst=3, vst=2, mma_latency=3, skip_dsfull=False, skip_qready=False):
+    """The dQ kernel on 128-token tiles: a K ring (a tile held until dQ(n) has read it) and a V
+    ring (released after S/dP(n)), each with its own producer; one MMA issuer walking
+    S/dP(0), dQ(0), S/dP(1), dQ(1), ... with one S and one dP buffer, reused for block n once
+    dQ(n - 1) is done (bdone); the softmax reads S and dP of block n, writes dS over S and signals
+    dsfull; per item it writes Q and dO (after the item before has had all its S/dP read) and
+    signals qready, and its epilogue reads dQ after the item's last dQ MMA. The tensor pipe
+    completes one thread's MMAs in issue order. `skip_dsfull` / `skip_qready` drop a wait (seeded
+    mistakes)."""
+    tiles = list(items)
+    nblk = sum(tiles)
+    kfull, kempty = [Barrier(1) for _ in range(kst)], [Barrier(1) for _ in range(kst)]
+    vfull, vempty = [Barrier(1) for _ in range(vst)], [Barrier(1) for _ in range(vst)]
+    sfull, dsfull, bdone, qready = Barrier(1), Barrier(1), Barrier(1), Barrier(1)
+    prod = {"k": 0, "v": 0}
+    mma = {"c": 0, "phase": 0, "item": 0, "blk": 0}  # phase 0: S/dP of block c, 1: dQ of block c
+    soft = {"item": 0, "blk": 0, "g": 0, "step": 0}
+    sp_done, dq_done, sp_read, ds_written = set(), set(), set(), set()
+    k_read, v_read = set(), set()
+    q_items, epi_done = set(), set()
+    pipe = {"free": 0}
+    pending = []
+    t = 0
+    nonempty = [i for i, n in enumerate(tiles) if n > 0]
+    blocks = [(it, b) for it, n in enumerate(tiles) for b in range(n)]  # block c -> (item, index)
+
+    def producer(kind):
+        c = prod[kind]
+        if c >= nblk:
+            return False
+        nst, empty, full, read = (kst, kempty, kfull, k_read) if kind == "k" else (vst, vempty, vfull, v_read)
+        st = c % nst
+        if not empty[st].poll(c // nst - 1, f"{kind} producer at {c}"):
+            return False
+        assert c < nst or c - nst in read, f"{kind} ring position {c} refilled before its last MMA"
+        full[st].arrive()
+        prod[kind] += 1
+        return True
+
+    def issue(done):
+        pipe["free"] = max(pipe["free"], t) + rng.randint(1, mma_latency)
+        pending.append((pipe["free"], done))
+
+    def issuer():
+        c = mma["c"]
+        if c >= nblk:
+            return False
+        it, b = blocks[c]
+        if mma["phase"] == 0:
+            if b == 0 and not skip_qready and not qready.poll(nonempty.index(it), f"issuer Q of item {it}"):
+                return False
+            if c > 0 and not bdone.poll(c - 1, f"issuer S/dP{c}"):
+                return False
+            if not kfull[c % kst].poll(c // kst, f"issuer K{c}") or not vfull[c % vst].poll(c // vst, f"issuer V{c}"):
+                return False
+
+            def done(c=c, it=it):
+                assert it in q_items, f"S/dP{c} read Q/dO of item {it} before they were written"
+                assert c == 0 or (c - 1 in dq_done and c - 1 in sp_read), f"S/dP{c} overwrote block {c - 1}"
+                sp_done.add(c)
+                v_read.add(c)
+                vempty[c % vst].arrive()
+                sfull.arrive()
+            issue(done)
+            mma["phase"] = 1
+            return True
+        if not skip_dsfull and not dsfull.poll(c, f"issuer dQ{c}"):
+            return False
+        if b == 0:
+            assert it == 0 or all(j in epi_done for j in range(it)), f"dQ(0) of item {it} before the epilogue"
+
+        def done(c=c):
+            assert c in ds_written, f"dQ{c} read dS before it was written"
+            dq_done.add(c)
+            k_read.add(c)
+            kempty[c % kst].arrive()
+            bdone.arrive()
+        issue(done)
+        mma["phase"], mma["c"] = 0, c + 1
+        return True
+
+    def softmax():
+        it = soft["item"]
+        if it >= len(tiles):
+            return False
+        n, g = tiles[it], soft["g"]
+        if soft["step"] == 0:  # item start: Q and dO into TMEM
+            if n > 0:
+                assert all(x in sp_done for x in range(g)), "Q/dO rewritten before the last S/dP finished"
+                q_items.add(it)
+                qready.arrive()
+            soft["step"] = 1
+            return True
+        if soft["blk"] < n:
+            if soft["step"] == 1:
+                if not sfull.poll(g, f"softmax S/dP{g}"):
+                    return False
+                sp_read.add(g)
+                soft["step"] = 2
+                return True
+            ds_written.add(g)  # dS over S
+            dsfull.arrive()
+            soft["blk"], soft["g"], soft["step"] = soft["blk"] + 1, g + 1, 1
+            return True
+        if n > 0:
+            if not bdone.poll(g - 1, f"softmax epilogue of item {it}"):
+                return False
+            assert all(x in dq_done for x in range(g - n, g))
+        epi_done.add(it)
+        soft["item"], soft["blk"], soft["step"] = it + 1, 0, 0
+        return True
+
+    agents = [lambda: producer("k"), lambda: producer("v"), issuer, softmax]
+    speed = [rng.uniform(0.05, 1.0) for _ in agents]
+    while mma["c"] < nblk or soft["item"] < len(tiles) or pending:
+        t += 1
+        due = sorted([x for x in pending if x[0] <= t], key=lambda x: x[0])
+        pending[:] = [x for x in pending if x[0] > t]
+        for _, done in due:
+            done()
+        moved = bool(due)
+        for i in rng.sample(range(len(agents)), len(agents)):
+            if rng.random() < speed[i]:
+                moved |= agents[i]()
+        if not moved and not pending and not any(a() for a in agents):
+            raise AssertionError(f"deadlock at block {mma['c']} of {nblk}, softmax item {soft['item']}")
+    assert len(dq_done) == nblk and prod["k"] == nblk and prod["v"] == nblk
+
+
+@pytest.mark.parametrize("seed", range(30))
+def test_dq_b128_protocol(seed):
+    rng = random.Random(seed)
+    run_dq_b128([rng.choice([0, 1, 2, 3, 5, 8]) for _ in range(rng.randint(2, 8))], rng)
+
+
+@pytest.mark.parametrize("mistake", ["skip_dsfull", "skip_qready"])
+def test_dq_b128_protocol_flags_a_skipped_wait(mistake):
+    hits = 0
+    for seed in range(60):
+        try:
+            run_dq_b128([3, 4, 2, 5], random.Random(seed), **{mistake: True})
+        except AssertionError:
+            hits += 1
+    assert hits > 0
